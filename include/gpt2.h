@@ -1,0 +1,199 @@
+/*
+ * gpt2.h -- C ABI of the B200-native GPT-2 pretraining step.
+ *
+ * One handle holds one decoder-only GPT-2 (tied token embedding / LM head,
+ * learned positions, pre-LayerNorm, causal multi-head attention, 4C tanh-GELU
+ * MLP, softmax cross-entropy over a vocabulary padded to a multiple of 64)
+ * and its optimiser state.  The step the calls below make up is the one the
+ * pages describe: forward, backward (accumulated over micro-batches with the
+ * loss divided by the number of micro-batches), global-norm gradient clipping
+ * at 1.0, and AdamW with beta = (0.9, 0.95), eps = 1e-8 and weight decay 0.1
+ * on 2-D parameters only, driven by a warmup-then-cosine LR schedule
+ * ("Let's reproduce GPT-2 (124M)" condensed, sections 1-3; "TinyStories
+ * training", the training excerpt).
+ *
+ * Conventions for every call:
+ *  - Pointers named *_dev are device pointers; *_host are host pointers.
+ *  - All device work is enqueued on the handle's stream (gpt2_set_stream;
+ *    default: the legacy default stream) and is asynchronous, except where a
+ *    host out-pointer is given: then the call synchronises the stream.
+ *  - Every call that can fail returns a gpt2_status: 0 on success, a
+ *    negative GPT2_ERR_* code otherwise; gpt2_last_error() gives the text.
+ *  - Memory: the caller owns the device memory it binds with
+ *    gpt2_bind_memory (e.g. allocated by PyTorch).  If nothing is bound when
+ *    the first call needs memory, the library allocates it with cudaMalloc
+ *    and frees it in gpt2_destroy.
+ *  - Precision (this library build): parameters, gradients and AdamW moments
+ *    are fp32; activations, the GEMM weight copies and the logits are bf16;
+ *    LayerNorm statistics, the attention log-sum-exp and every reduction are
+ *    fp32.  The validation build (libgpt2_fp32.so) keeps everything in fp32
+ *    and uses no tensor cores.
+ *  - Determinism: no call uses floating-point atomics; two runs with the
+ *    same inputs give bit-identical parameters, gradients and losses.
+ */
+#ifndef GPT2_B200_H
+#define GPT2_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct gpt2 gpt2_t;
+typedef int gpt2_status;
+
+#define GPT2_OK 0
+#define GPT2_ERR_ARG (-1)       /* bad shape or argument */
+#define GPT2_ERR_STATE (-2)     /* call out of order or memory not bound */
+#define GPT2_ERR_TOKEN (-3)     /* a token or target outside [0, V) */
+#define GPT2_ERR_NONFINITE (-4) /* loss or gradient norm is not finite */
+#define GPT2_ERR_CUDA (-5)      /* a CUDA runtime error */
+#define GPT2_ERR_TIMEOUT (-6)   /* a kernel's bounded wait expired */
+
+/* Build variant: 1 for the bf16 tensor-core build, 0 for the fp32 validation
+ * build. */
+int gpt2_build_is_bf16(void);
+
+/* Create a model.  L layers, H heads, width C (C % H == 0, C % 8 == 0,
+ * head dim C/H in {32, 64, 128}), vocabulary V padded to Vpad (Vpad >= V,
+ * Vpad % 64 == 0), context Tmax.  Parameters are initialised on the device
+ * at the first gpt2_bind_memory/allocation: N(0, 0.02) for wte (rows < V),
+ * wpe, W_qkv and W_fc; N(0, 0.02/sqrt(2L)) for the residual projections W_o
+ * and W_p (condensed GPT-2 page, section 1); LayerNorm gains 1; biases, LN
+ * betas and the padded wte rows 0.  Normals come from a counter-based
+ * SplitMix64 + Box-Muller generator keyed by (seed, tensor, element).
+ * Errors: GPT2_ERR_ARG on a bad shape. */
+gpt2_status gpt2_create(int L, int H, int C, int V, int Vpad, int Tmax, uint64_t seed,
+                        gpt2_t** out);
+void gpt2_destroy(gpt2_t* h);
+
+/* Number of parameters in the flat buffer (including the Vpad - V padded
+ * wte rows): 12 L C^2 + 13 L C + 2 C + Vpad C + Tmax C. */
+size_t gpt2_num_params(const gpt2_t* h);
+
+/* Device bytes for the persistent state (fp32 params, grads, m, v, the bf16
+ * weight copy and a few scalars). */
+size_t gpt2_state_bytes(const gpt2_t* h);
+
+/* Device bytes of workspace (activations kept for the backward pass, logits,
+ * backward scratch) for micro-batches of B sequences of length T. */
+size_t gpt2_workspace_bytes(const gpt2_t* h, int B, int T);
+
+/* Bind caller-owned device memory: dev_state (>= gpt2_state_bytes) and
+ * dev_work (>= gpt2_workspace_bytes for the largest B,T used later).  Both
+ * must be 256-byte aligned.  Binding new state memory re-initialises the
+ * parameters from the seed and zeroes grads, moments and the step count.
+ * dev_state may be NULL to keep the current state; dev_work may be NULL to
+ * keep the current workspace. */
+gpt2_status gpt2_bind_memory(gpt2_t* h, void* dev_state, size_t state_bytes, void* dev_work,
+                             size_t work_bytes);
+
+/* Stream (a cudaStream_t) on which every later call enqueues its work. */
+gpt2_status gpt2_set_stream(gpt2_t* h, void* cuda_stream);
+
+/* Forward pass over tok_dev [B, T] (int32, row-major, values in [0, V)).
+ * With tgt_dev (int32 [B, T]) it also computes the mean softmax
+ * cross-entropy over the B*T positions (padded logits excluded) and leaves in
+ * the logits buffer the gradient of that mean loss w.r.t. the logits, ready
+ * for gpt2_backward.  loss_host (may be NULL) receives the mean loss and
+ * makes the call synchronous; tokens are then also validated (GPT2_ERR_TOKEN;
+ * out-of-range ids are read as id 0 on the device, never out of bounds).
+ * Without targets the logits [B*T, Vpad] stay in the workspace (see
+ * gpt2_logits).  Errors: GPT2_ERR_ARG (T > Tmax, workspace too small),
+ * GPT2_ERR_STATE (no memory), GPT2_ERR_TOKEN, GPT2_ERR_NONFINITE. */
+gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok_dev, const int32_t* tgt_dev, int B, int T,
+                         float* loss_host);
+
+/* Mean loss of the last forward with targets, read back to the host
+ * (synchronises the stream). */
+gpt2_status gpt2_read_loss(gpt2_t* h, float* loss_host);
+
+/* Zero the gradient buffer. */
+gpt2_status gpt2_zero_grad(gpt2_t* h);
+
+/* Backward pass of the preceding forward (which must have had targets, at
+ * the same B, T): adds d(loss_scale * mean loss)/d(params) into the fp32
+ * gradient buffer.  Use loss_scale = 1/n_micro to accumulate n_micro
+ * micro-batches (condensed GPT-2 page, section 3).  Errors: GPT2_ERR_STATE
+ * (no forward with targets since the last backward). */
+gpt2_status gpt2_backward(gpt2_t* h, float loss_scale);
+
+/* Global L2 norm n of all gradients (fixed-order two-stage reduction); when
+ * n > max_norm every gradient is to be scaled by max_norm / (n + 1e-6).  The
+ * scale is kept on the device and applied inside gpt2_adamw_step.
+ * norm_host (may be NULL) receives n and makes the call synchronous; a
+ * non-finite n then returns GPT2_ERR_NONFINITE (and AdamW skips the update
+ * on the device whatever the caller does). */
+gpt2_status gpt2_grad_norm_clip(gpt2_t* h, float max_norm, float* norm_host);
+
+/* One AdamW step on every parameter (t += 1; bias-corrected moments;
+ * p -= lr (mhat / (sqrt(vhat) + eps) + wd p) with wd applied to the 2-D
+ * tensors wte, wpe, W_qkv, W_o, W_fc, W_p only), using the clip scale of the
+ * last gpt2_grad_norm_clip (1 if none since the last step).  Refreshes the
+ * bf16 weight copy.  Gradients are left as they are. */
+gpt2_status gpt2_adamw_step(gpt2_t* h, float lr, float beta1, float beta2, float eps,
+                            float weight_decay);
+
+/* Host-side schedule: lr = max_lr (step+1)/warmup for step < warmup, then a
+ * cosine from max_lr at step = warmup to min_lr at step = max_steps, and
+ * min_lr after (condensed GPT-2 page, section 3: warmup 715, cosine to 10 %
+ * of 6e-4). Pure function. */
+double gpt2_lr(long step, double max_lr, double min_lr, long warmup, long max_steps);
+
+/* Host copies of the fp32 flat parameter / gradient buffers
+ * (gpt2_num_params floats); synchronous. */
+gpt2_status gpt2_get_params(const gpt2_t* h, float* host);
+gpt2_status gpt2_set_params(gpt2_t* h, const float* host); /* also refreshes the bf16 copy */
+gpt2_status gpt2_get_grads(const gpt2_t* h, float* host);
+
+/* Checkpoint state: params, m, v (each gpt2_num_params floats) and the step
+ * counter t.  Any pointer may be NULL to skip that part. Synchronous. */
+gpt2_status gpt2_get_state(const gpt2_t* h, float* params, float* m, float* v, long* t);
+gpt2_status gpt2_set_state(gpt2_t* h, const float* params, const float* m, const float* v,
+                           long t);
+
+/* Tensor i (0..15) of the flat layout: name, 1 or 2 (or 3 for per-layer
+ * matrices) dims, shape, offset in floats.  Order: wte[Vpad,C] wpe[Tmax,C]
+ * ln1_g[L,C] ln1_b[L,C] w_qkv[L,3C,C] b_qkv[L,3C] w_o[L,C,C] b_o[L,C]
+ * ln2_g[L,C] ln2_b[L,C] w_fc[L,4C,C] b_fc[L,4C] w_p[L,C,4C] b_p[L,C]
+ * lnf_g[C] lnf_b[C]; matrices are (out, in) row-major, y = x W^T + b. */
+gpt2_status gpt2_tensor_info(const gpt2_t* h, int i, const char** name, int* ndim,
+                             int64_t shape[3], size_t* offset);
+
+/* Device pointer to the logits of the last forward without targets,
+ * [B*T, Vpad] row-major in the activation dtype (bf16 / fp32 build). */
+gpt2_status gpt2_logits(const gpt2_t* h, const void** dev_ptr);
+
+/* Per-position losses of the last forward with targets (B*T floats, host). */
+gpt2_status gpt2_get_losses(const gpt2_t* h, float* host, size_t n);
+
+/* Copy an activation of the last forward to the host as fp32 (for tests):
+ * kind 0 residual input of layer `layer` (layer == L: the final residual),
+ * 1 ln1 out, 2 qkv, 3 attention out, 4 residual after attention, 5 ln2 out,
+ * 6 fc pre-activation, 7 GELU out, 8 lnf out.  n = number of floats. */
+gpt2_status gpt2_read_activation(const gpt2_t* h, int kind, int layer, float* host, size_t n);
+
+/* Text of the last error on this handle ("" if none). */
+const char* gpt2_last_error(const gpt2_t* h);
+
+/* Number of kernel launches this library has made in the process so far
+ * (all handles); differences across a region count its launches. */
+long gpt2_launch_count(void);
+
+/* Per-kernel-family timing with CUDA events on the handle's stream.  Kinds:
+ * 0 GEMM, 1 attention forward, 2 attention backward, 3 LayerNorm (fwd+bwd),
+ * 4 classifier, 5 encoder (fwd+bwd), 6 bias-gradient column sums,
+ * 7 optimiser (norm, clip, AdamW).  gpt2_profile_read synchronises the
+ * stream, writes for each kind the summed milliseconds, the number of timed
+ * regions and the algorithmic FLOPs (GEMM: 2MNK; attention: causal products),
+ * and clears the records.  `kinds` is the length of the arrays (>= 8). */
+gpt2_status gpt2_profile_enable(gpt2_t* h, int on);
+gpt2_status gpt2_profile_read(gpt2_t* h, double* ms, long* launches, double* flops, int kinds);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPT2_B200_H */

@@ -96,6 +96,9 @@ def lib(openmp: bool = False) -> ctypes.CDLL:
             fn = getattr(L, f"orc_{name}_{sfx}")
             fn.argtypes = [R]
             fn.restype = R
+        fn = getattr(L, f"orc_gelu_tanh_vec_{sfx}")
+        fn.argtypes = [P, P, sz, i]
+        fn.restype = None
         fn = getattr(L, f"orc_layernorm_fwd_{sfx}")
         fn.argtypes = [P, P, P, P, P, P, i, i]
         fn.restype = None
@@ -226,13 +229,22 @@ class Oracle:
             _ptr(m, self.ct), _ptr(v, self.ct), t, lr, b1, b2, eps, wd)
 
     # primitives ---------------------------------------------------------
+    def _gelu_vec(self, x, grad):
+        x = np.ascontiguousarray(x, self.dtype)
+        y = np.empty_like(x)
+        getattr(self.lib, f"orc_gelu_tanh_vec_{self.sfx}")(_ptr(x, self.ct), _ptr(y, self.ct),
+                                                           x.size, int(grad))
+        return y
+
     def gelu_tanh(self, x):
-        f = getattr(self.lib, f"orc_gelu_tanh_{self.sfx}")
-        return np.array([f(float(v)) for v in np.ravel(x)], self.dtype).reshape(np.shape(x))
+        if np.ndim(x) == 0:
+            return float(getattr(self.lib, f"orc_gelu_tanh_{self.sfx}")(float(x)))
+        return self._gelu_vec(x, False)
 
     def gelu_tanh_grad(self, x):
-        f = getattr(self.lib, f"orc_gelu_tanh_grad_{self.sfx}")
-        return np.array([f(float(v)) for v in np.ravel(x)], self.dtype).reshape(np.shape(x))
+        if np.ndim(x) == 0:
+            return float(getattr(self.lib, f"orc_gelu_tanh_grad_{self.sfx}")(float(x)))
+        return self._gelu_vec(x, True)
 
     def gelu_erf(self, x):
         f = getattr(self.lib, f"orc_gelu_erf_{self.sfx}")

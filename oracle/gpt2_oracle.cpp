@@ -626,6 +626,10 @@ uint64_t orc_splitmix64(uint64_t seed, uint64_t n) { return sm_output(seed, n); 
   R orc_gelu_tanh_##SFX(R x) { return gelu_tanh<R>(x); }                       \
   R orc_gelu_tanh_grad_##SFX(R x) { return gelu_tanh_grad<R>(x); }             \
   R orc_gelu_erf_##SFX(R x) { return gelu_erf<R>(x); }                         \
+  void orc_gelu_tanh_vec_##SFX(const R* x, R* y, size_t n, int grad) {         \
+    for (size_t i = 0; i < n; ++i)                                             \
+      y[i] = grad ? gelu_tanh_grad<R>(x[i]) : gelu_tanh<R>(x[i]);              \
+  }                                                                            \
   void orc_layernorm_fwd_##SFX(const R* x, const R* g, const R* b, R* y,       \
                                R* mean, R* rstd, int M, int C) {               \
     layernorm_fwd<R>(x, g, b, y, mean, rstd, M, C);                            \

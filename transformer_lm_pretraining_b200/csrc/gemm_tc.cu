@@ -1,0 +1,568 @@
+// bf16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Persistent, warp-specialised kernel, one CTA per SM:
+//   warp 0     TMA producer: 128x64 A and BNx64 B tiles (128-byte swizzle)
+//              into a STAGES-deep shared-memory ring;
+//   warp 1     allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16)
+//              from one elected lane, accumulating fp32 in TMEM;
+//   warps 2-5  epilogue: tcgen05.ld of the 128 x BN accumulator (one row per
+//              thread), bias / GELU / residual / GELU-backward / fp32
+//              accumulate, global stores.
+// The TMEM accumulator is double-buffered so the epilogue of one tile runs
+// under the main loop of the next.  Both operands may be K-major or
+// MN-major (the tensor core reads either from the descriptor), which covers
+// the forward (A, B K-major), data-gradient (B MN-major) and
+// weight-gradient (both MN-major) products without any transpose copies.
+//
+// Every mbarrier wait is bounded: after ~2 s a role sets an abort flag and
+// the device error word (ERR_TIMEOUT), the other roles see the flag and
+// leave their loops, the producer waits (bounded) for its copies in flight,
+// and TMEM is freed before the kernel returns.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "gemm_epi.cuh"
+
+namespace gpt2k {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for the phase with the given parity.  false = gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 127u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(err, ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives
+// row (lane base + i), columns taddr.col .. +31.
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// Shared-memory matrix descriptors (tcgen05 format, 128-byte swizzle).
+//  K-major tile: rows of 64 bf16 (128 B), 8-row groups 1024 B apart (SBO);
+//    the k-th 16-element slice starts 32 B further in.
+//  MN-major tile: 64(MN) x 64(K) boxes of 8 KB, k rows of 128 B; 8-row
+//    groups 1024 B apart (SBO), next 64 MN elements 8 KB on (LBO);
+//    the k-th 16-row slice starts 2048 B further in.
+__device__ __forceinline__ uint64_t desc_common(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int k16) {
+  return desc_common(tile + 32u * k16, 16u, 1024u);
+}
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int k16) {
+  return desc_common(tile + 2048u * k16, 8192u, 1024u);
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, M = 128, N = BN.
+template <int BN, bool A_MN, bool B_MN>
+__host__ __device__ constexpr uint32_t make_idesc() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((A_MN ? 1u : 0u) << 15) |
+         ((B_MN ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+template <int BN>
+constexpr uint32_t tmem_cols() {
+  return 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+}
+
+template <int BN, int STAGES>
+constexpr size_t smem_bytes() {
+  return 1024 + (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 256;
+}
+
+template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const EpiParams ep, int K, int tiles_m, int tiles_n, int splits, int kb_per_split,
+                   int n_fast, int vec_ok, long split_stride, int* err) {
+  constexpr int A_BYTES = BM * BK * 2;
+  constexpr int B_BYTES = BN * BK * 2;
+  constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
+  constexpr uint32_t TMEM_COLS = tmem_cols<BN>();
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * (A_BYTES + B_BYTES));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kb_total = (K + BK - 1) / BK;
+  const int tiles = tiles_m * tiles_n;
+  const int units = tiles * splits;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 128);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto decode = [&](int u, int& tm, int& tn, int& kb0, int& kb1, int& sp) {
+    sp = u / tiles;
+    const int r = u - sp * tiles;
+    if (n_fast) {
+      tm = r / tiles_n;
+      tn = r - tm * tiles_n;
+    } else {
+      tn = r / tiles_m;
+      tm = r - tn * tiles_m;
+    }
+    kb0 = sp * kb_per_split;
+    kb1 = min(kb0 + kb_per_split, kb_total);
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- producer --
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0;  // stages that received at least one load
+      uint32_t last_parity = 0;  // parity of the latest fill of each stage
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tm, tn, kb0, kb1, sp;
+        decode(u, tm, tn, kb0, kb1, sp);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_expect_tx(fb, STAGE_TX);
+          const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
+          if (!A_MN) {
+            tma_load_2d(a_dst, &tmA, fb, kb * BK, tm * BM);
+          } else {
+            tma_load_2d(a_dst, &tmA, fb, tm * BM, kb * BK);
+            tma_load_2d(a_dst + 8192, &tmA, fb, tm * BM + 64, kb * BK);
+          }
+          if (!B_MN) {
+            tma_load_2d(b_dst, &tmB, fb, kb * BK, tn * BN);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + 8192 * j, &tmB, fb, tn * BN + 64 * j, kb * BK);
+          }
+          issued_mask |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Give the copies already issued a bounded time to land before the
+        // shared memory they target is released.
+        const uint64_t t0 = global_ns();
+        for (int s = 0; s < STAGES; ++s) {
+          if (!(issued_mask & (1u << s))) continue;
+          const uint32_t par = (last_parity >> s) & 1u;
+          while (!mbar_try_wait(full0 + 8 * s, par)) {
+            if (global_ns() - t0 > kWaitLimitNs) break;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // --------------------------------------------------------- MMA --
+      constexpr uint32_t idesc = make_idesc<BN, A_MN, B_MN>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int tm, tn, kb0, kb1, sp;
+        decode(u, tm, tn, kb0, kb1, sp);
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_MN ? desc_mnmajor(a_base, k) : desc_kmajor(a_base, k);
+            const uint64_t bd = B_MN ? desc_mnmajor(b_base, k) : desc_kmajor(b_base, k);
+            tc_mma(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull0 + 8 * acc);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        // let MMAs already issued finish before TMEM is released
+        tc_commit(tfull0 + 8 * acc);
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(tfull0 + 8 * acc, acc_phase)) {
+          if (global_ns() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue --
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      int tm, tn, kb0, kb1, sp;
+      decode(u, tm, tn, kb0, kb1, sp);
+      // warp-uniform decision: the TMEM loads below are warp-collective
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, err));
+      if (!ok) break;
+      tc_fence_after();
+      const int m = tm * BM + row;
+      EpiParams e = ep;
+      if (EPI == EPI_F32_STORE) e.out32 += (size_t)sp * split_stride;
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        const int n0 = tn * BN + c0;
+        if (n0 >= ep.N) break;  // uniform across the warp
+        uint32_t r[32];
+        tc_ld32(t_row + (uint32_t)c0, r);
+        tc_wait_ld();
+        if (m < ep.M) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          epi_row32<EPI>(e, m, n0, v, vec_ok != 0);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * acc);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS));
+  }
+}
+
+// ------------------------------------------------------------ host side --
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::mutex g_mu;
+
+static cudaError_t get_encoder() {
+  if (g_encode) return cudaSuccess;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess) return e;
+  if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return cudaSuccess;
+}
+
+// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows
+// `ld` elements apart; box of 64 x box_outer with 128-byte swizzle.
+static cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer,
+                             uint64_t ld, uint32_t box_outer) {
+  using Key = std::tuple<const void*, uint64_t, uint64_t, uint64_t, uint32_t>;
+  static std::map<Key, CUtensorMap> cache;
+  const Key key{ptr, inner, outer, ld, box_outer};
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *tm = it->second;
+      return cudaSuccess;
+    }
+  }
+  cudaError_t e = get_encoder();
+  if (e != cudaSuccess) return e;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64u, box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  std::lock_guard<std::mutex> g(g_mu);
+  if (cache.size() > 4096) cache.clear();
+  cache[key] = *tm;
+  return cudaSuccess;
+}
+
+static int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = kNumSMs;
+  }
+  return n;
+}
+
+template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI>
+static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const EpiParams& ep, int K,
+                          int splits, int kb_per_split, int n_fast, int vec_ok, long split_stride,
+                          cudaStream_t s, int* err) {
+  auto kern = gemm_tc_kernel<BN, STAGES, A_MN, B_MN, EPI>;
+  constexpr size_t smem = smem_bytes<BN, STAGES>();
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const int tiles_m = (ep.M + BM - 1) / BM;
+  const int tiles_n = (ep.N + BN - 1) / BN;
+  const int units = tiles_m * tiles_n * splits;
+  const int grid = units < num_sms() ? units : num_sms();
+  kern<<<grid, kThreads, smem, s>>>(ta, tb, ep, K, tiles_m, tiles_n, splits, kb_per_split, n_fast,
+                                    vec_ok, split_stride, err);
+  note_launch();
+  return cudaGetLastError();
+}
+
+template <int BN, int STAGES>
+static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb,
+                            const EpiParams& ep, int epi, int splits, int kb_per_split, int n_fast,
+                            int vec_ok, long split_stride, cudaStream_t s, int* err) {
+#define GPT2_TC(AM, BMJ, E)                                                                     \
+  if (a.a_mn == AM && a.b_mn == BMJ && epi == E)                                                \
+    return launch<BN, STAGES, AM, BMJ, E>(ta, tb, ep, a.K, splits, kb_per_split, n_fast, vec_ok, \
+                                          split_stride, s, err);
+  GPT2_TC(0, 0, EPI_STORE)
+  GPT2_TC(0, 0, EPI_BIAS)
+  GPT2_TC(0, 0, EPI_BIAS_GELU)
+  GPT2_TC(0, 0, EPI_BIAS_RESID)
+  GPT2_TC(0, 1, EPI_STORE)
+  GPT2_TC(0, 1, EPI_DGELU)
+  GPT2_TC(1, 1, EPI_F32_ACC)
+  GPT2_TC(1, 1, EPI_F32_STORE)
+  GPT2_TC(1, 0, EPI_STORE)
+  GPT2_TC(0, 0, EPI_F32_STORE)
+#undef GPT2_TC
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace tc
+
+__global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, int splits, int M,
+                                     int N) {
+  const size_t total = (size_t)M * N;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int m = (int)(i / N), n = (int)(i % N);
+    float s = 0.f;
+    for (int k = 0; k < splits; ++k) s += ws[(size_t)k * total + i];
+    out32[(size_t)m * ldo32 + n] += s;
+  }
+}
+
+cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
+  using namespace tc;
+  if (a.M <= 0 || a.N <= 0 || a.K <= 0) return cudaSuccess;
+  // TMA: 16-byte aligned bases and row strides.
+  if ((reinterpret_cast<uintptr_t>(a.A) & 15) || (reinterpret_cast<uintptr_t>(a.B) & 15) ||
+      (a.lda % 8) || (a.ldb % 8))
+    return cudaErrorInvalidValue;
+  const int BN = a.N >= 256 ? 256 : 128;
+  CUtensorMap ta, tb;
+  cudaError_t e;
+  if (!a.a_mn) e = make_tmap(&ta, a.A, a.K, a.M, a.lda, BM);
+  else e = make_tmap(&ta, a.A, a.M, a.K, a.lda, 64);
+  if (e != cudaSuccess) return e;
+  if (!a.b_mn) e = make_tmap(&tb, a.B, a.K, a.N, a.ldb, BN);
+  else e = make_tmap(&tb, a.B, a.N, a.K, a.ldb, 64);
+  if (e != cudaSuccess) return e;
+
+  EpiParams ep{a.M, a.N, a.alpha, a.out, a.ldo, a.out32, a.ldo32, a.bias, a.resid, a.ldr, a.aux, a.ldaux};
+  const int tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  const int kb_total = (a.K + BK - 1) / BK;
+
+  // split-K for the weight-gradient products with few output tiles
+  int splits = 1;
+  int epi = a.epi;
+  if (a.epi == EPI_F32_ACC && a.max_splits > 1 && a.split_ws) {
+    const int want = (num_sms() + tiles - 1) / tiles;
+    splits = want < a.max_splits ? want : a.max_splits;
+    if (splits > kb_total / 4) splits = kb_total / 4;
+    while (splits > 1 && (size_t)splits * a.M * a.N > a.split_ws_floats) --splits;
+    if (splits < 1) splits = 1;
+  }
+  int kb_per_split = (kb_total + splits - 1) / splits;
+  splits = (kb_total + kb_per_split - 1) / kb_per_split;  // no empty split
+  long split_stride = 0;
+  if (splits > 1) {
+    epi = EPI_F32_STORE;
+    ep.out32 = a.split_ws;
+    ep.ldo32 = a.N;
+    ep.alpha = a.alpha;
+    split_stride = (long)a.M * a.N;
+  }
+  // The larger operand is reused by consecutive tiles (L2 locality).
+  const double a_bytes = (double)a.M * a.K, b_bytes = (double)a.N * a.K;
+  const int n_fast = a_bytes > b_bytes ? 1 : 0;
+  const int vec_ok = (ep.ldo % 8 == 0) && (ep.ldo32 % 4 == 0) && (ep.ldr % 8 == 0) &&
+                     (ep.ldaux % 8 == 0) && ((reinterpret_cast<uintptr_t>(ep.out) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(ep.out32) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(ep.resid) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(ep.aux) & 15) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(ep.bias) & 15) == 0);
+  if (BN == 256)
+    e = dispatch<256, 4>(a, ta, tb, ep, epi, splits, kb_per_split, n_fast, vec_ok, split_stride, s, err);
+  else
+    e = dispatch<128, 6>(a, ta, tb, ep, epi, splits, kb_per_split, n_fast, vec_ok, split_stride, s, err);
+  if (e != cudaSuccess) return e;
+  if (splits > 1) {
+    const size_t total = (size_t)a.M * a.N;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
+    splitk_reduce_kernel<<<blocks, 256, 0, s>>>(a.out32, a.ldo32, a.split_ws, splits, a.M, a.N);
+    note_launch();
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace gpt2k

@@ -1,0 +1,853 @@
+// GPT-2 step engine behind the C ABI of include/gpt2.h: parameter/optimiser
+// state layout, activation workspace layout, and the sequence of kernel
+// launches for forward, backward, clip and AdamW.
+
+#include <cmath>
+#include <cstdio>
+#include <algorithm>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/gpt2.h"
+#include "kernels.h"
+
+using namespace gpt2k;
+
+namespace {
+
+size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Carves consecutive 256-byte aligned regions out of one allocation.
+struct Carver {
+  char* base;
+  size_t used = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <class T>
+  T* take(size_t n) {
+    T* p = reinterpret_cast<T*>(base ? base + used : nullptr);
+    used += align256(n * sizeof(T));
+    return p;
+  }
+};
+
+struct Acts {
+  act_t *res, *h1, *qkv, *att, *xmid, *h2, *u, *g, *hf, *logits;
+  float *mean1, *rstd1, *lse, *mean2, *rstd2, *meanf, *rstdf, *losses;
+  int* tok;
+  act_t *dres, *dh, *datt, *dqkv, *dbig;
+  float *dsum, *partials, *splitk;
+  void* enc_scratch;
+  size_t splitk_floats;
+};
+
+constexpr int kMaxSplits = 8;
+
+// Optional per-kernel-family timing with CUDA events on the handle's stream.
+enum ProfKind {
+  PK_GEMM, PK_ATTN_FWD, PK_ATTN_BWD, PK_LAYERNORM, PK_CLASSIFIER, PK_ENCODER, PK_COLSUM,
+  PK_OPTIMIZER, PK_COUNT
+};
+
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  double flops;
+};
+
+}  // namespace
+
+struct gpt2 {
+  Layout lay;
+  uint64_t seed = 0;
+  cudaStream_t stream = nullptr;
+  // state
+  void* state = nullptr;
+  size_t state_bytes = 0;
+  bool own_state = false;
+  float *params = nullptr, *grads = nullptr, *m = nullptr, *v = nullptr;
+  act_t* pact = nullptr;
+  float* scalars = nullptr;
+  double* norm_partials = nullptr;
+  int* err = nullptr;
+  long t = 0;
+  // workspace
+  void* work = nullptr;
+  size_t work_bytes = 0;
+  bool own_work = false;
+  // forward record
+  int B = 0, T = 0;
+  bool have_grad_logits = false;
+  bool have_logits = false;
+  Acts a{};
+  std::string last_error;
+  // profiling
+  bool prof = false;
+  std::vector<cudaEvent_t> ev_pool;
+  std::vector<ProfRec> recs;
+};
+
+namespace {
+
+gpt2_status fail(gpt2_t* h, gpt2_status code, const std::string& msg) {
+  if (h) h->last_error = msg;
+  return code;
+}
+
+gpt2_status cuda_fail(gpt2_t* h, cudaError_t e, const char* where) {
+  return fail(h, GPT2_ERR_CUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+#define GPT2_CUDA(h, call)                                   \
+  do {                                                       \
+    cudaError_t e_ = (call);                                 \
+    if (e_ != cudaSuccess) return cuda_fail(h, e_, #call);   \
+  } while (0)
+
+// Layout of the state allocation.
+size_t carve_state(const Layout& lay, void* base, gpt2_t* h) {
+  Carver c(base);
+  float* params = c.take<float>(lay.total);
+  float* grads = c.take<float>(lay.total);
+  float* m = c.take<float>(lay.total);
+  float* v = c.take<float>(lay.total);
+#if GPT2_ACT_BF16
+  act_t* pact = c.take<act_t>(lay.total);
+#else
+  act_t* pact = params;
+#endif
+  float* scalars = c.take<float>(S_COUNT);
+  double* np = c.take<double>(kNormBlocks);
+  int* err = c.take<int>(16);
+  if (h) {
+    h->params = params; h->grads = grads; h->m = m; h->v = v; h->pact = pact;
+    h->scalars = scalars; h->norm_partials = np; h->err = err;
+  }
+  return c.used;
+}
+
+// Layout of the workspace for B x T tokens.
+size_t carve_work(const Layout& lay, int B, int T, void* base, Acts* a) {
+  const size_t M = (size_t)B * T, C = lay.C, L = lay.L, H = lay.H;
+  Carver c(base);
+  Acts x{};
+  x.res = c.take<act_t>((L + 1) * M * C);
+  x.h1 = c.take<act_t>(L * M * C);
+  x.qkv = c.take<act_t>(L * M * 3 * C);
+  x.att = c.take<act_t>(L * M * C);
+  x.xmid = c.take<act_t>(L * M * C);
+  x.h2 = c.take<act_t>(L * M * C);
+  x.u = c.take<act_t>(L * M * 4 * C);
+  x.g = c.take<act_t>(L * M * 4 * C);
+  x.hf = c.take<act_t>(M * C);
+  x.logits = c.take<act_t>(M * (size_t)lay.Vp);
+  x.mean1 = c.take<float>(L * M);
+  x.rstd1 = c.take<float>(L * M);
+  x.lse = c.take<float>(L * M * H);
+  x.mean2 = c.take<float>(L * M);
+  x.rstd2 = c.take<float>(L * M);
+  x.meanf = c.take<float>(M);
+  x.rstdf = c.take<float>(M);
+  x.losses = c.take<float>(M);
+  x.tok = c.take<int>(M);
+  x.dres = c.take<act_t>(M * C);
+  x.dh = c.take<act_t>(M * C);
+  x.datt = c.take<act_t>(M * C);
+  x.dqkv = c.take<act_t>(M * 3 * C);
+  x.dbig = c.take<act_t>(M * 4 * C);
+  x.dsum = c.take<float>(M * H);
+  const size_t part = std::max((size_t)kColsumChunks * 4 * C, (size_t)kLnBlocks * 2 * C);
+  x.partials = c.take<float>(part);
+  x.splitk_floats = (size_t)kMaxSplits * 4 * C * C;
+  x.splitk = c.take<float>(x.splitk_floats);
+  x.enc_scratch = c.take<char>(encoder_scratch_bytes((int)M, (int)C));
+  if (a) *a = x;
+  return c.used;
+}
+
+gpt2_status check_err_word(gpt2_t* h) {
+  int e = 0;
+  GPT2_CUDA(h, cudaMemcpyAsync(&e, h->err, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  if (e) {
+    GPT2_CUDA(h, cudaMemsetAsync(h->err, 0, sizeof(int), h->stream));
+    if (e & ERR_TIMEOUT) return fail(h, GPT2_ERR_TIMEOUT, "a kernel's bounded wait expired");
+    if (e & ERR_TOKEN) return fail(h, GPT2_ERR_TOKEN, "token id outside [0, V)");
+    if (e & ERR_TARGET) return fail(h, GPT2_ERR_TOKEN, "target id outside [0, V)");
+  }
+  return GPT2_OK;
+}
+
+gpt2_status ensure_state(gpt2_t* h) {
+  if (h->state) return GPT2_OK;
+  const size_t bytes = carve_state(h->lay, nullptr, nullptr);
+  void* p = nullptr;
+  GPT2_CUDA(h, cudaMalloc(&p, bytes));
+  gpt2_status st = gpt2_bind_memory(h, p, bytes, nullptr, 0);
+  if (st != GPT2_OK) {
+    cudaFree(p);
+    return st;
+  }
+  h->own_state = true;
+  return GPT2_OK;
+}
+
+gpt2_status ensure_work(gpt2_t* h, int B, int T) {
+  const size_t need = carve_work(h->lay, B, T, nullptr, nullptr);
+  if (h->work && h->work_bytes >= need) return GPT2_OK;
+  if (h->work && !h->own_work)
+    return fail(h, GPT2_ERR_ARG, "bound workspace is smaller than gpt2_workspace_bytes(B, T)");
+  if (h->own_work) {
+    cudaFree(h->work);
+    h->work = nullptr;
+  }
+  void* p = nullptr;
+  GPT2_CUDA(h, cudaMalloc(&p, need));
+  h->work = p;
+  h->work_bytes = need;
+  h->own_work = true;
+  return GPT2_OK;
+}
+
+#define GPT2_TRY(expr)            \
+  do {                            \
+    gpt2_status st_ = (expr);     \
+    if (st_ != GPT2_OK) return st_; \
+  } while (0)
+
+cudaEvent_t prof_event(gpt2_t* h) {
+  if (!h->ev_pool.empty()) {
+    cudaEvent_t e = h->ev_pool.back();
+    h->ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Timeline marks: with profiling on, each mark records an event on the
+// stream; the time up to the next mark is charged to the mark's kernel
+// family (only that family's launches sit between two marks).
+void mark(gpt2_t* h, int kind, double flops = 0) {
+  if (!h->prof) return;
+  cudaEvent_t e = prof_event(h);
+  cudaEventRecord(e, h->stream);
+  if (!h->recs.empty() && h->recs.back().b == nullptr) h->recs.back().b = e;
+  h->recs.push_back({kind, e, nullptr, flops});
+}
+void mark_end(gpt2_t* h) {
+  if (!h->prof || h->recs.empty() || h->recs.back().b != nullptr) return;
+  cudaEvent_t e = prof_event(h);
+  cudaEventRecord(e, h->stream);
+  h->recs.back().b = e;
+}
+
+gpt2_status run_gemm(gpt2_t* h, const GemmArgs& ga) {
+  mark(h, PK_GEMM, 2.0 * ga.M * ga.N * ga.K);
+  GPT2_CUDA(h, gemm(ga, h->stream, h->err));
+  return GPT2_OK;
+}
+
+GemmArgs gemm_args(int M, int N, int K) {
+  GemmArgs g{};
+  g.M = M; g.N = N; g.K = K;
+  g.alpha = 1.f;
+  g.max_splits = 1;
+  return g;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gpt2_build_is_bf16(void) { return GPT2_ACT_BF16; }
+
+gpt2_status gpt2_create(int L, int H, int C, int V, int Vpad, int Tmax, uint64_t seed,
+                        gpt2_t** out) {
+  if (!out) return GPT2_ERR_ARG;
+  *out = nullptr;
+  if (L < 1 || H < 1 || C < 8 || V < 1 || Tmax < 1 || C % H || C % 8 || Vpad < V || Vpad % 64 ||
+      C > 2048)
+    return GPT2_ERR_ARG;
+  const int hd = C / H;
+#if GPT2_ACT_BF16
+  if (hd != 32 && hd != 64 && hd != 128) return GPT2_ERR_ARG;
+#else
+  if (hd > 128 || hd % 8) return GPT2_ERR_ARG;
+#endif
+  gpt2_t* h = new gpt2_t();
+  h->lay = make_layout(L, H, C, V, Vpad, Tmax);
+  h->seed = seed;
+  *out = h;
+  return GPT2_OK;
+}
+
+void gpt2_destroy(gpt2_t* h) {
+  if (!h) return;
+  if (h->own_state && h->state) cudaFree(h->state);
+  if (h->own_work && h->work) cudaFree(h->work);
+  std::vector<cudaEvent_t> evs = h->ev_pool;
+  for (const ProfRec& r : h->recs) {
+    evs.push_back(r.a);
+    if (r.b) evs.push_back(r.b);
+  }
+  std::sort(evs.begin(), evs.end());
+  evs.erase(std::unique(evs.begin(), evs.end()), evs.end());
+  for (cudaEvent_t e : evs) cudaEventDestroy(e);
+  delete h;
+}
+
+size_t gpt2_num_params(const gpt2_t* h) { return h ? h->lay.total : 0; }
+
+size_t gpt2_state_bytes(const gpt2_t* h) { return h ? carve_state(h->lay, nullptr, nullptr) : 0; }
+
+size_t gpt2_workspace_bytes(const gpt2_t* h, int B, int T) {
+  if (!h || B < 1 || T < 1) return 0;
+  return carve_work(h->lay, B, T, nullptr, nullptr);
+}
+
+gpt2_status gpt2_bind_memory(gpt2_t* h, void* dev_state, size_t state_bytes, void* dev_work,
+                             size_t work_bytes) {
+  if (!h) return GPT2_ERR_ARG;
+  if (dev_state) {
+    if (reinterpret_cast<uintptr_t>(dev_state) & 255)
+      return fail(h, GPT2_ERR_ARG, "state memory must be 256-byte aligned");
+    if (state_bytes < gpt2_state_bytes(h)) return fail(h, GPT2_ERR_ARG, "state memory too small");
+    if (h->own_state && h->state) cudaFree(h->state);
+    h->own_state = false;
+    h->state = dev_state;
+    h->state_bytes = state_bytes;
+    carve_state(h->lay, dev_state, h);
+    const size_t P = h->lay.total;
+    init_params(h->params, h->lay, h->seed, h->stream);
+    GPT2_CUDA(h, cudaGetLastError());
+    GPT2_CUDA(h, cudaMemsetAsync(h->grads, 0, P * sizeof(float), h->stream));
+    GPT2_CUDA(h, cudaMemsetAsync(h->m, 0, P * sizeof(float), h->stream));
+    GPT2_CUDA(h, cudaMemsetAsync(h->v, 0, P * sizeof(float), h->stream));
+    GPT2_CUDA(h, cudaMemsetAsync(h->scalars, 0, S_COUNT * sizeof(float), h->stream));
+    reset_clip(h->scalars, h->stream);
+    GPT2_CUDA(h, cudaMemsetAsync(h->err, 0, 16 * sizeof(int), h->stream));
+#if GPT2_ACT_BF16
+    f32_to_act(h->pact, h->params, P, h->stream);
+    GPT2_CUDA(h, cudaGetLastError());
+#endif
+    h->t = 0;
+    h->have_grad_logits = h->have_logits = false;
+  }
+  if (dev_work) {
+    if (reinterpret_cast<uintptr_t>(dev_work) & 255)
+      return fail(h, GPT2_ERR_ARG, "workspace must be 256-byte aligned");
+    if (h->own_work && h->work) cudaFree(h->work);
+    h->own_work = false;
+    h->work = dev_work;
+    h->work_bytes = work_bytes;
+    h->have_grad_logits = h->have_logits = false;
+  }
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_set_stream(gpt2_t* h, void* cuda_stream) {
+  if (!h) return GPT2_ERR_ARG;
+  h->stream = static_cast<cudaStream_t>(cuda_stream);
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int B, int T,
+                         float* loss_host) {
+  if (!h || !tok || B < 1 || T < 1) return fail(h, GPT2_ERR_ARG, "bad forward arguments");
+  const Layout& y = h->lay;
+  if (T > y.Tmax) return fail(h, GPT2_ERR_ARG, "T > Tmax");
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  st = ensure_work(h, B, T);
+  if (st) return st;
+  Acts& a = h->a;
+  carve_work(y, B, T, h->work, &a);
+  h->B = B;
+  h->T = T;
+  const int M = B * T, C = y.C, L = y.L, H = y.H;
+  const size_t MC = (size_t)M * C;
+  cudaStream_t s = h->stream;
+  const float* P = h->params;
+  const act_t* W = h->pact;
+
+  mark(h, PK_ENCODER);
+  encoder_fwd(a.res, a.tok, tok, W + y.off[T_WTE], W + y.off[T_WPE], B, T, C, y.V, h->err, s);
+  for (int l = 0; l < L; ++l) {
+    act_t* x = a.res + (size_t)l * MC;
+    act_t* h1 = a.h1 + (size_t)l * MC;
+    act_t* qkv = a.qkv + (size_t)l * 3 * MC;
+    act_t* att = a.att + (size_t)l * MC;
+    act_t* xm = a.xmid + (size_t)l * MC;
+    act_t* h2 = a.h2 + (size_t)l * MC;
+    act_t* u = a.u + (size_t)l * 4 * MC;
+    act_t* g = a.g + (size_t)l * 4 * MC;
+    mark(h, PK_LAYERNORM);
+    layernorm_fwd(h1, a.mean1 + (size_t)l * M, a.rstd1 + (size_t)l * M, x,
+                  P + y.off[T_LN1G] + (size_t)l * C, P + y.off[T_LN1B] + (size_t)l * C, M, C, s);
+    {  // qkv = h1 W_qkv^T + b_qkv
+      GemmArgs ga = gemm_args(M, 3 * C, C);
+      ga.A = h1; ga.lda = C;
+      ga.B = W + y.off[T_WQKV] + (size_t)l * 3 * C * C; ga.ldb = C;
+      ga.epi = EPI_BIAS; ga.bias = P + y.off[T_BQKV] + (size_t)l * 3 * C;
+      ga.out = qkv; ga.ldo = 3 * C;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    mark(h, PK_ATTN_FWD, 4.0 * B * H * (double)T * (T + 1) / 2 * (C / H));
+    GPT2_CUDA(h, attention_fwd(att, a.lse + (size_t)l * M * H, qkv, B, T, C, H, s));
+    {  // xmid = x + att W_o^T + b_o
+      GemmArgs ga = gemm_args(M, C, C);
+      ga.A = att; ga.lda = C;
+      ga.B = W + y.off[T_WO] + (size_t)l * C * C; ga.ldb = C;
+      ga.epi = EPI_BIAS_RESID; ga.bias = P + y.off[T_BO] + (size_t)l * C;
+      ga.resid = x; ga.ldr = C;
+      ga.out = xm; ga.ldo = C;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    mark(h, PK_LAYERNORM);
+    layernorm_fwd(h2, a.mean2 + (size_t)l * M, a.rstd2 + (size_t)l * M, xm,
+                  P + y.off[T_LN2G] + (size_t)l * C, P + y.off[T_LN2B] + (size_t)l * C, M, C, s);
+    {  // u = h2 W_fc^T + b_fc; g = gelu(u)
+      GemmArgs ga = gemm_args(M, 4 * C, C);
+      ga.A = h2; ga.lda = C;
+      ga.B = W + y.off[T_WFC] + (size_t)l * 4 * C * C; ga.ldb = C;
+      ga.epi = EPI_BIAS_GELU; ga.bias = P + y.off[T_BFC] + (size_t)l * 4 * C;
+      ga.aux = u; ga.ldaux = 4 * C;
+      ga.out = g; ga.ldo = 4 * C;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    {  // x_next = xmid + g W_p^T + b_p
+      GemmArgs ga = gemm_args(M, C, 4 * C);
+      ga.A = g; ga.lda = 4 * C;
+      ga.B = W + y.off[T_WP] + (size_t)l * 4 * C * C; ga.ldb = 4 * C;
+      ga.epi = EPI_BIAS_RESID; ga.bias = P + y.off[T_BP] + (size_t)l * C;
+      ga.resid = xm; ga.ldr = C;
+      ga.out = a.res + (size_t)(l + 1) * MC; ga.ldo = C;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+  }
+  mark(h, PK_LAYERNORM);
+  layernorm_fwd(a.hf, a.meanf, a.rstdf, a.res + (size_t)L * MC, P + y.off[T_LNFG],
+                P + y.off[T_LNFB], M, C, s);
+  {  // logits = hf wte^T over all Vpad rows (padded rows are 0)
+    GemmArgs ga = gemm_args(M, y.Vp, C);
+    ga.A = a.hf; ga.lda = C;
+    ga.B = W + y.off[T_WTE]; ga.ldb = C;
+    ga.epi = EPI_STORE;
+    ga.out = a.logits; ga.ldo = y.Vp;
+    GPT2_TRY(run_gemm(h, ga));
+  }
+  h->have_grad_logits = false;
+  h->have_logits = false;
+  if (tgt) {
+    mark(h, PK_CLASSIFIER);
+    classifier(a.logits, a.losses, tgt, M, y.V, y.Vp, h->err, s);
+    mean_loss(h->scalars + S_LOSS, a.losses, M, s);
+    h->have_grad_logits = true;
+  } else {
+    h->have_logits = true;
+  }
+  mark_end(h);
+  GPT2_CUDA(h, cudaGetLastError());
+  if (loss_host) {
+    GPT2_CUDA(h, cudaMemcpyAsync(loss_host, h->scalars + S_LOSS, sizeof(float),
+                                 cudaMemcpyDeviceToHost, s));
+    st = check_err_word(h);
+    if (st) return st;
+    if (tgt && !std::isfinite(*loss_host)) return fail(h, GPT2_ERR_NONFINITE, "loss is not finite");
+  }
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_read_loss(gpt2_t* h, float* loss_host) {
+  if (!h || !loss_host || !h->scalars) return GPT2_ERR_ARG;
+  GPT2_CUDA(h, cudaMemcpyAsync(loss_host, h->scalars + S_LOSS, sizeof(float),
+                               cudaMemcpyDeviceToHost, h->stream));
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_zero_grad(gpt2_t* h) {
+  if (!h) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  GPT2_CUDA(h, cudaMemsetAsync(h->grads, 0, h->lay.total * sizeof(float), h->stream));
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
+  if (!h) return GPT2_ERR_ARG;
+  if (!h->have_grad_logits)
+    return fail(h, GPT2_ERR_STATE, "backward needs a preceding forward with targets");
+  const Layout& y = h->lay;
+  Acts& a = h->a;
+  const int B = h->B, T = h->T, M = B * T, C = y.C, L = y.L, H = y.H;
+  const size_t MC = (size_t)M * C;
+  cudaStream_t s = h->stream;
+  const float* P = h->params;
+  const act_t* W = h->pact;
+  float* G = h->grads;
+  EncoderScratch es;
+  encoder_scratch_carve(&es, a.enc_scratch, M, C);
+
+  {  // dhf = scale * dz wte  (dz: the logits buffer)
+    GemmArgs ga = gemm_args(M, C, y.Vp);
+    ga.A = a.logits; ga.lda = y.Vp;
+    ga.B = W + y.off[T_WTE]; ga.ldb = C; ga.b_mn = 1;
+    ga.epi = EPI_STORE; ga.alpha = loss_scale;
+    ga.out = a.dh; ga.ldo = C;
+    GPT2_TRY(run_gemm(h, ga));
+  }
+  {  // dwte += scale * dz^T hf
+    GemmArgs ga = gemm_args(y.Vp, C, M);
+    ga.A = a.logits; ga.lda = y.Vp; ga.a_mn = 1;
+    ga.B = a.hf; ga.ldb = C; ga.b_mn = 1;
+    ga.epi = EPI_F32_ACC; ga.alpha = loss_scale;
+    ga.out32 = G + y.off[T_WTE]; ga.ldo32 = C;
+    ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+    GPT2_TRY(run_gemm(h, ga));
+  }
+  mark(h, PK_LAYERNORM);
+  layernorm_bwd(a.dres, a.dh, a.res + (size_t)L * MC, a.meanf, a.rstdf, P + y.off[T_LNFG],
+                G + y.off[T_LNFG], G + y.off[T_LNFB], a.partials, M, C, 0, s);
+
+  for (int l = L - 1; l >= 0; --l) {
+    const act_t* x = a.res + (size_t)l * MC;
+    const act_t* h1 = a.h1 + (size_t)l * MC;
+    const act_t* qkv = a.qkv + (size_t)l * 3 * MC;
+    const act_t* att = a.att + (size_t)l * MC;
+    const act_t* xm = a.xmid + (size_t)l * MC;
+    const act_t* h2 = a.h2 + (size_t)l * MC;
+    const act_t* u = a.u + (size_t)l * 4 * MC;
+    const act_t* g = a.g + (size_t)l * 4 * MC;
+    // ---- MLP: x_next = xm + gelu(h2 Wfc^T + bfc) Wp^T + bp
+    {  // du = (dres Wp) * gelu'(u)
+      GemmArgs ga = gemm_args(M, 4 * C, C);
+      ga.A = a.dres; ga.lda = C;
+      ga.B = W + y.off[T_WP] + (size_t)l * 4 * C * C; ga.ldb = 4 * C; ga.b_mn = 1;
+      ga.epi = EPI_DGELU; ga.aux = const_cast<act_t*>(u); ga.ldaux = 4 * C;
+      ga.out = a.dbig; ga.ldo = 4 * C;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    {  // dWp += dres^T g
+      GemmArgs ga = gemm_args(C, 4 * C, M);
+      ga.A = a.dres; ga.lda = C; ga.a_mn = 1;
+      ga.B = g; ga.ldb = 4 * C; ga.b_mn = 1;
+      ga.epi = EPI_F32_ACC;
+      ga.out32 = G + y.off[T_WP] + (size_t)l * 4 * C * C; ga.ldo32 = 4 * C;
+      ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    mark(h, PK_COLSUM);
+    colsum_acc(G + y.off[T_BP] + (size_t)l * C, a.dres, M, C, a.partials, s);
+    {  // dh = du Wfc
+      GemmArgs ga = gemm_args(M, C, 4 * C);
+      ga.A = a.dbig; ga.lda = 4 * C;
+      ga.B = W + y.off[T_WFC] + (size_t)l * 4 * C * C; ga.ldb = C; ga.b_mn = 1;
+      ga.epi = EPI_STORE;
+      ga.out = a.dh; ga.ldo = C;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    {  // dWfc += du^T h2
+      GemmArgs ga = gemm_args(4 * C, C, M);
+      ga.A = a.dbig; ga.lda = 4 * C; ga.a_mn = 1;
+      ga.B = h2; ga.ldb = C; ga.b_mn = 1;
+      ga.epi = EPI_F32_ACC;
+      ga.out32 = G + y.off[T_WFC] + (size_t)l * 4 * C * C; ga.ldo32 = C;
+      ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    mark(h, PK_COLSUM);
+    colsum_acc(G + y.off[T_BFC] + (size_t)l * 4 * C, a.dbig, M, 4 * C, a.partials, s);
+    mark(h, PK_LAYERNORM);
+    layernorm_bwd(a.dres, a.dh, xm, a.mean2 + (size_t)l * M, a.rstd2 + (size_t)l * M,
+                  P + y.off[T_LN2G] + (size_t)l * C, G + y.off[T_LN2G] + (size_t)l * C,
+                  G + y.off[T_LN2B] + (size_t)l * C, a.partials, M, C, 1, s);
+    // ---- attention: xm = x + att Wo^T + bo
+    {  // datt = dres Wo
+      GemmArgs ga = gemm_args(M, C, C);
+      ga.A = a.dres; ga.lda = C;
+      ga.B = W + y.off[T_WO] + (size_t)l * C * C; ga.ldb = C; ga.b_mn = 1;
+      ga.epi = EPI_STORE;
+      ga.out = a.datt; ga.ldo = C;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    {  // dWo += dres^T att
+      GemmArgs ga = gemm_args(C, C, M);
+      ga.A = a.dres; ga.lda = C; ga.a_mn = 1;
+      ga.B = att; ga.ldb = C; ga.b_mn = 1;
+      ga.epi = EPI_F32_ACC;
+      ga.out32 = G + y.off[T_WO] + (size_t)l * C * C; ga.ldo32 = C;
+      ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    mark(h, PK_COLSUM);
+    colsum_acc(G + y.off[T_BO] + (size_t)l * C, a.dres, M, C, a.partials, s);
+    mark(h, PK_ATTN_BWD, 10.0 * B * H * (double)T * (T + 1) / 2 * (C / H));
+    GPT2_CUDA(h, attention_bwd(a.dqkv, a.dsum, a.datt, qkv, att, a.lse + (size_t)l * M * H, B, T,
+                               C, H, s));
+    {  // dh = dqkv Wqkv
+      GemmArgs ga = gemm_args(M, C, 3 * C);
+      ga.A = a.dqkv; ga.lda = 3 * C;
+      ga.B = W + y.off[T_WQKV] + (size_t)l * 3 * C * C; ga.ldb = C; ga.b_mn = 1;
+      ga.epi = EPI_STORE;
+      ga.out = a.dh; ga.ldo = C;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    {  // dWqkv += dqkv^T h1
+      GemmArgs ga = gemm_args(3 * C, C, M);
+      ga.A = a.dqkv; ga.lda = 3 * C; ga.a_mn = 1;
+      ga.B = h1; ga.ldb = C; ga.b_mn = 1;
+      ga.epi = EPI_F32_ACC;
+      ga.out32 = G + y.off[T_WQKV] + (size_t)l * 3 * C * C; ga.ldo32 = C;
+      ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    mark(h, PK_COLSUM);
+    colsum_acc(G + y.off[T_BQKV] + (size_t)l * 3 * C, a.dqkv, M, 3 * C, a.partials, s);
+    mark(h, PK_LAYERNORM);
+    layernorm_bwd(a.dres, a.dh, x, a.mean1 + (size_t)l * M, a.rstd1 + (size_t)l * M,
+                  P + y.off[T_LN1G] + (size_t)l * C, G + y.off[T_LN1G] + (size_t)l * C,
+                  G + y.off[T_LN1B] + (size_t)l * C, a.partials, M, C, 1, s);
+  }
+  mark(h, PK_ENCODER);
+  encoder_bwd(G + y.off[T_WTE], G + y.off[T_WPE], a.dres, a.tok, B, T, C, y.Vp, es, s);
+  mark_end(h);
+  GPT2_CUDA(h, cudaGetLastError());
+  h->have_grad_logits = false;
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_grad_norm_clip(gpt2_t* h, float max_norm, float* norm_host) {
+  if (!h) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  mark(h, PK_OPTIMIZER);
+  grad_norm_clip(h->scalars, h->grads, h->lay.total, max_norm, h->norm_partials, h->stream);
+  mark_end(h);
+  GPT2_CUDA(h, cudaGetLastError());
+  if (norm_host) {
+    GPT2_CUDA(h, cudaMemcpyAsync(norm_host, h->scalars + S_NORM, sizeof(float),
+                                 cudaMemcpyDeviceToHost, h->stream));
+    st = check_err_word(h);
+    if (st) return st;
+    if (!std::isfinite(*norm_host))
+      return fail(h, GPT2_ERR_NONFINITE, "gradient norm is not finite");
+  }
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_adamw_step(gpt2_t* h, float lr, float beta1, float beta2, float eps,
+                            float weight_decay) {
+  if (!h) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  h->t += 1;
+  AdamArgs a;
+  a.lr = lr; a.b1 = beta1; a.b2 = beta2; a.eps = eps; a.wd = weight_decay;
+  a.bc1 = (float)(1.0 - std::pow((double)beta1, (double)h->t));
+  a.bc2 = (float)(1.0 - std::pow((double)beta2, (double)h->t));
+  mark(h, PK_OPTIMIZER);
+  adamw(h->params, h->pact, h->grads, h->m, h->v, h->lay, a, h->scalars, h->stream);
+  GPT2_CUDA(h, cudaGetLastError());
+  reset_clip(h->scalars, h->stream);  // the clip scale applies to one step only
+  mark_end(h);
+  GPT2_CUDA(h, cudaGetLastError());
+  return GPT2_OK;
+}
+
+double gpt2_lr(long step, double max_lr, double min_lr, long warmup, long max_steps) {
+  if (step < warmup) return max_lr * (double)(step + 1) / (double)warmup;
+  if (step > max_steps || max_steps <= warmup) return min_lr;
+  const double ratio = (double)(step - warmup) / (double)(max_steps - warmup);
+  return min_lr + 0.5 * (1.0 + std::cos(M_PI * ratio)) * (max_lr - min_lr);
+}
+
+gpt2_status gpt2_get_params(const gpt2_t* hc, float* host) {
+  gpt2_t* h = const_cast<gpt2_t*>(hc);
+  if (!h || !host) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  GPT2_CUDA(h, cudaMemcpyAsync(host, h->params, h->lay.total * 4, cudaMemcpyDeviceToHost, h->stream));
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_set_params(gpt2_t* h, const float* host) {
+  if (!h || !host) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  GPT2_CUDA(h, cudaMemcpyAsync(h->params, host, h->lay.total * 4, cudaMemcpyHostToDevice, h->stream));
+#if GPT2_ACT_BF16
+  f32_to_act(h->pact, h->params, h->lay.total, h->stream);
+  GPT2_CUDA(h, cudaGetLastError());
+#endif
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_get_grads(const gpt2_t* hc, float* host) {
+  gpt2_t* h = const_cast<gpt2_t*>(hc);
+  if (!h || !host) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  GPT2_CUDA(h, cudaMemcpyAsync(host, h->grads, h->lay.total * 4, cudaMemcpyDeviceToHost, h->stream));
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_get_state(const gpt2_t* hc, float* params, float* m, float* v, long* t) {
+  gpt2_t* h = const_cast<gpt2_t*>(hc);
+  if (!h) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  const size_t n = h->lay.total * 4;
+  if (params) GPT2_CUDA(h, cudaMemcpyAsync(params, h->params, n, cudaMemcpyDeviceToHost, h->stream));
+  if (m) GPT2_CUDA(h, cudaMemcpyAsync(m, h->m, n, cudaMemcpyDeviceToHost, h->stream));
+  if (v) GPT2_CUDA(h, cudaMemcpyAsync(v, h->v, n, cudaMemcpyDeviceToHost, h->stream));
+  if (t) *t = h->t;
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_set_state(gpt2_t* h, const float* params, const float* m, const float* v, long t) {
+  if (!h || t < 0) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  const size_t n = h->lay.total * 4;
+  if (params) {
+    GPT2_CUDA(h, cudaMemcpyAsync(h->params, params, n, cudaMemcpyHostToDevice, h->stream));
+#if GPT2_ACT_BF16
+    f32_to_act(h->pact, h->params, h->lay.total, h->stream);
+    GPT2_CUDA(h, cudaGetLastError());
+#endif
+  }
+  if (m) GPT2_CUDA(h, cudaMemcpyAsync(h->m, m, n, cudaMemcpyHostToDevice, h->stream));
+  if (v) GPT2_CUDA(h, cudaMemcpyAsync(h->v, v, n, cudaMemcpyHostToDevice, h->stream));
+  h->t = t;
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_tensor_info(const gpt2_t* h, int i, const char** name, int* ndim,
+                             int64_t shape[3], size_t* offset) {
+  static const char* names[T_COUNT] = {"wte", "wpe", "ln1_g", "ln1_b", "w_qkv", "b_qkv",
+                                       "w_o", "b_o", "ln2_g", "ln2_b", "w_fc", "b_fc",
+                                       "w_p", "b_p", "lnf_g", "lnf_b"};
+  if (!h || i < 0 || i >= T_COUNT) return GPT2_ERR_ARG;
+  const Layout& y = h->lay;
+  int64_t sh[3] = {0, 0, 0};
+  int nd = 0;
+  const int64_t L = y.L, C = y.C;
+  switch (i) {
+    case T_WTE: nd = 2; sh[0] = y.Vp; sh[1] = C; break;
+    case T_WPE: nd = 2; sh[0] = y.Tmax; sh[1] = C; break;
+    case T_WQKV: nd = 3; sh[0] = L; sh[1] = 3 * C; sh[2] = C; break;
+    case T_BQKV: nd = 2; sh[0] = L; sh[1] = 3 * C; break;
+    case T_WO: nd = 3; sh[0] = L; sh[1] = C; sh[2] = C; break;
+    case T_WFC: nd = 3; sh[0] = L; sh[1] = 4 * C; sh[2] = C; break;
+    case T_BFC: nd = 2; sh[0] = L; sh[1] = 4 * C; break;
+    case T_WP: nd = 3; sh[0] = L; sh[1] = C; sh[2] = 4 * C; break;
+    case T_LNFG: case T_LNFB: nd = 1; sh[0] = C; break;
+    default: nd = 2; sh[0] = L; sh[1] = C; break;
+  }
+  if (name) *name = names[i];
+  if (ndim) *ndim = nd;
+  if (shape) for (int k = 0; k < 3; ++k) shape[k] = sh[k];
+  if (offset) *offset = y.off[i];
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_logits(const gpt2_t* h, const void** dev_ptr) {
+  if (!h || !dev_ptr) return GPT2_ERR_ARG;
+  if (!h->have_logits) return GPT2_ERR_STATE;
+  *dev_ptr = h->a.logits;
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_get_losses(const gpt2_t* hc, float* host, size_t n) {
+  gpt2_t* h = const_cast<gpt2_t*>(hc);
+  if (!h || !host || !h->work) return GPT2_ERR_ARG;
+  if (n > (size_t)h->B * h->T) return fail(h, GPT2_ERR_ARG, "n > B*T");
+  GPT2_CUDA(h, cudaMemcpyAsync(host, h->a.losses, n * 4, cudaMemcpyDeviceToHost, h->stream));
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_read_activation(const gpt2_t* hc, int kind, int layer, float* host, size_t n) {
+  gpt2_t* h = const_cast<gpt2_t*>(hc);
+  if (!h || !host || !h->work) return GPT2_ERR_ARG;
+  const Layout& y = h->lay;
+  const size_t M = (size_t)h->B * h->T, C = y.C;
+  const Acts& a = h->a;
+  const act_t* src = nullptr;
+  size_t cnt = 0;
+  if (layer < 0 || layer > y.L || (kind != 0 && kind != 8 && layer == y.L)) return GPT2_ERR_ARG;
+  switch (kind) {
+    case 0: src = a.res + layer * M * C; cnt = M * C; break;
+    case 1: src = a.h1 + layer * M * C; cnt = M * C; break;
+    case 2: src = a.qkv + layer * 3 * M * C; cnt = 3 * M * C; break;
+    case 3: src = a.att + layer * M * C; cnt = M * C; break;
+    case 4: src = a.xmid + layer * M * C; cnt = M * C; break;
+    case 5: src = a.h2 + layer * M * C; cnt = M * C; break;
+    case 6: src = a.u + layer * 4 * M * C; cnt = 4 * M * C; break;
+    case 7: src = a.g + layer * 4 * M * C; cnt = 4 * M * C; break;
+    case 8: src = a.hf; cnt = M * C; break;
+    default: return GPT2_ERR_ARG;
+  }
+  if (n != cnt) return fail(h, GPT2_ERR_ARG, "n does not match the activation size");
+#if GPT2_ACT_BF16
+  std::vector<uint16_t> tmp(cnt);
+  GPT2_CUDA(h, cudaMemcpyAsync(tmp.data(), src, cnt * 2, cudaMemcpyDeviceToHost, h->stream));
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  for (size_t i = 0; i < cnt; ++i) {
+    const uint32_t bits = (uint32_t)tmp[i] << 16;
+    std::memcpy(host + i, &bits, 4);
+  }
+#else
+  GPT2_CUDA(h, cudaMemcpyAsync(host, src, cnt * 4, cudaMemcpyDeviceToHost, h->stream));
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+#endif
+  return GPT2_OK;
+}
+
+const char* gpt2_last_error(const gpt2_t* h) { return h ? h->last_error.c_str() : "null handle"; }
+
+long gpt2_launch_count(void) { return launch_count(); }
+
+gpt2_status gpt2_profile_enable(gpt2_t* h, int on) {
+  if (!h) return GPT2_ERR_ARG;
+  h->prof = on != 0;
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_profile_read(gpt2_t* h, double* ms, long* launches, double* flops, int kinds) {
+  if (!h || kinds < PK_COUNT) return GPT2_ERR_ARG;
+  for (int k = 0; k < kinds; ++k) {
+    if (ms) ms[k] = 0;
+    if (launches) launches[k] = 0;
+    if (flops) flops[k] = 0;
+  }
+  mark_end(h);
+  GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  std::vector<cudaEvent_t> used;
+  for (const ProfRec& r : h->recs) {
+    if (r.b) {
+      float t = 0.f;
+      GPT2_CUDA(h, cudaEventElapsedTime(&t, r.a, r.b));
+      if (ms) ms[r.kind] += t;
+      if (launches) launches[r.kind] += 1;
+      if (flops) flops[r.kind] += r.flops;
+      used.push_back(r.b);
+    }
+    used.push_back(r.a);
+  }
+  std::sort(used.begin(), used.end());
+  used.erase(std::unique(used.begin(), used.end()), used.end());
+  h->ev_pool.insert(h->ev_pool.end(), used.begin(), used.end());
+  h->recs.clear();
+  return GPT2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// Kernel-level C entry points (include/gpt2_kernels.h).
+
+#include "../../include/gpt2.h"
+#include "../../include/gpt2_kernels.h"
+#include "kernels.h"
+
+using namespace gpt2k;
+
+namespace {
+
+int* err_word() {
+  static int* e = nullptr;
+  if (!e) {
+    if (cudaMalloc(&e, sizeof(int)) != cudaSuccess) return nullptr;
+    cudaMemset(e, 0, sizeof(int));
+  }
+  return e;
+}
+
+int status(cudaError_t e) { return e == cudaSuccess ? GPT2_OK : (e == cudaErrorInvalidValue ? GPT2_ERR_ARG : GPT2_ERR_CUDA); }
+
+}  // namespace
+
+extern "C" {
+
+int gpt2k_gemm(void* stream, int epi, int M, int N, int K, const void* A, long lda, int a_mn,
+               const void* B, long ldb, int b_mn, float alpha, void* out, long ldo, float* out32,
+               long ldo32, const float* bias, const void* resid, long ldr, void* aux, long ldaux,
+               float* split_ws, size_t split_ws_floats) {
+  if (M < 0 || N < 0 || K < 0 || epi < 0 || epi > EPI_F32_ACC) return GPT2_ERR_ARG;
+  int* err = err_word();
+  if (!err) return GPT2_ERR_CUDA;
+  GemmArgs g{};
+  g.M = M; g.N = N; g.K = K;
+  g.A = static_cast<const act_t*>(A); g.lda = lda; g.a_mn = a_mn;
+  g.B = static_cast<const act_t*>(B); g.ldb = ldb; g.b_mn = b_mn;
+  g.epi = epi; g.alpha = alpha;
+  g.out = static_cast<act_t*>(out); g.ldo = ldo;
+  g.out32 = out32; g.ldo32 = ldo32;
+  g.bias = bias;
+  g.resid = static_cast<const act_t*>(resid); g.ldr = ldr;
+  g.aux = static_cast<act_t*>(aux); g.ldaux = ldaux;
+  g.split_ws = split_ws; g.split_ws_floats = split_ws_floats;
+  g.max_splits = split_ws ? 8 : 1;
+  return status(gemm(g, static_cast<cudaStream_t>(stream), err));
+}
+
+int gpt2k_attention_fwd(void* stream, void* att, float* lse, const void* qkv, int B, int T, int C,
+                        int H) {
+  if (B < 1 || T < 1 || H < 1 || C % H) return GPT2_ERR_ARG;
+  return status(attention_fwd(static_cast<act_t*>(att), lse, static_cast<const act_t*>(qkv), B, T,
+                              C, H, static_cast<cudaStream_t>(stream)));
+}
+
+int gpt2k_attention_bwd(void* stream, void* dqkv, float* dsum, const void* datt, const void* qkv,
+                        const void* att, const float* lse, int B, int T, int C, int H) {
+  if (B < 1 || T < 1 || H < 1 || C % H) return GPT2_ERR_ARG;
+  return status(attention_bwd(static_cast<act_t*>(dqkv), dsum, static_cast<const act_t*>(datt),
+                              static_cast<const act_t*>(qkv), static_cast<const act_t*>(att), lse,
+                              B, T, C, H, static_cast<cudaStream_t>(stream)));
+}
+
+int gpt2k_take_error(void) {
+  int* err = err_word();
+  if (!err) return GPT2_ERR_CUDA;
+  int e = 0;
+  if (cudaMemcpy(&e, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GPT2_ERR_CUDA;
+  cudaMemset(err, 0, sizeof(int));
+  return e;
+}
+
+}  // extern "C"

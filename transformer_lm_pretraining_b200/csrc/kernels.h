@@ -1,0 +1,141 @@
+// Launch interface of the GPT-2 step kernels (internal to the library).
+#pragma once
+
+#include "common.cuh"
+
+namespace gpt2k {
+
+// ------------------------------------------------------------- layout --
+// Flat parameter order (one slice per tensor, row-major, y = x W^T + b).
+enum Tensor {
+  T_WTE, T_WPE, T_LN1G, T_LN1B, T_WQKV, T_BQKV, T_WO, T_BO, T_LN2G, T_LN2B,
+  T_WFC, T_BFC, T_WP, T_BP, T_LNFG, T_LNFB, T_COUNT
+};
+
+struct Layout {
+  int L, H, C, V, Vp, Tmax;
+  size_t off[T_COUNT];
+  size_t num[T_COUNT];
+  size_t total;
+};
+
+Layout make_layout(int L, int H, int C, int V, int Vp, int Tmax);
+bool tensor_decayed(int t);
+
+// ---------------------------------------------------------------- GEMM --
+// D[m, n] = alpha * sum_k A(m, k) B(n, k), then the epilogue.
+//   A(m, k) = A[m * lda + k]  (a_mn = 0, "K-major")  or A[k * lda + m] (a_mn = 1)
+//   B(n, k) = B[n * ldb + k]  (b_mn = 0)             or B[k * ldb + n] (b_mn = 1)
+enum Epi {
+  EPI_STORE = 0,       // out = D
+  EPI_BIAS = 1,        // out = D + bias[n]
+  EPI_BIAS_GELU = 2,   // aux = D + bias[n]; out = gelu(aux)
+  EPI_BIAS_RESID = 3,  // out = resid + D + bias[n]
+  EPI_DGELU = 4,       // out = D * gelu'(aux)
+  EPI_F32_ACC = 5,     // out32 += D
+  EPI_F32_STORE = 6,   // out32 = D
+};
+
+struct GemmArgs {
+  int M, N, K;
+  const act_t* A; long lda; int a_mn;
+  const act_t* B; long ldb; int b_mn;
+  int epi;
+  float alpha;
+  act_t* out; long ldo;
+  float* out32; long ldo32;
+  const float* bias;
+  const act_t* resid; long ldr;
+  act_t* aux; long ldaux;
+  // split-K (EPI_F32_ACC only): partial sums go to split_ws, then a
+  // fixed-order reduction adds them into out32.  max_splits = 1 disables.
+  float* split_ws; size_t split_ws_floats; int max_splits;
+};
+
+cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err_flag);
+
+// ------------------------------------------------------------- encoder --
+// x0[m, :] = wte[tok[m], :] + wpe[m % T, :]; saves the (range-checked)
+// tokens for the backward pass; bad ids set err bit 1 and read row 0.
+void encoder_fwd(act_t* x0, int* tok_saved, const int* tok, const act_t* wte,
+                 const act_t* wpe, int B, int T, int C, int V, int* err, cudaStream_t s);
+
+struct EncoderScratch {
+  int* keys[2];     // [M] each
+  int* vals[2];     // [M] each
+  int* hist;        // [256 * ceil(M / 1024)]
+  float* partial;   // [M * C]
+};
+size_t encoder_scratch_bytes(int M, int C);
+void encoder_scratch_carve(EncoderScratch* es, void* base, int M, int C);
+
+// dwpe[t, :] += sum_b dx0[b T + t, :];  dwte[v, :] += sum_{m: tok[m] = v} dx0[m, :]
+// in ascending m (stable radix sort by token, fixed-chunk partial sums).
+void encoder_bwd(float* dwte, float* dwpe, const act_t* dx0, const int* tok_saved,
+                 int B, int T, int C, int Vp, const EncoderScratch& es, cudaStream_t s);
+
+// ----------------------------------------------------------- layernorm --
+void layernorm_fwd(act_t* y, float* mean, float* rstd, const act_t* x, const float* g,
+                   const float* b, int M, int C, cudaStream_t s);
+// dres = (accumulate ? dres : 0) + LN backward of dy;  dg, db += column sums
+// (per-block partials in `partials` [kLnBlocks * 2C], reduced in fixed order).
+constexpr int kLnBlocks = 296;
+void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
+                   const float* rstd, const float* g, float* dg, float* db, float* partials,
+                   int M, int C, int accumulate, cudaStream_t s);
+
+// ------------------------------------------------------------ column sums --
+constexpr int kColsumChunks = 128;
+// db[n] += sum_m dy[m, n] (fixed order); partials: [kColsumChunks * N] floats
+void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s);
+
+// ----------------------------------------------------------- attention --
+// qkv [B*T, 3C] = [q | k | v], head h at columns h*hd..; att [B*T, C];
+// lse [B, H, T] (natural log).
+cudaError_t attention_fwd(act_t* att, float* lse, const act_t* qkv, int B, int T, int C, int H,
+                          cudaStream_t s);
+// dqkv [B*T, 3C] (overwritten); dsum [B, H, T] scratch.
+cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
+                          const act_t* att, const float* lse, int B, int T, int C, int H,
+                          cudaStream_t s);
+
+// ---------------------------------------------------------- classifier --
+// In place over logits [M, Vp]: per row lse over the first V columns,
+// losses[m] = lse - z[tgt[m]], and z <- (softmax(z) - onehot(tgt)) / M for
+// columns < V, 0 for the padded columns.  Bad targets set err bit 2.
+void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int Vp, int* err,
+                cudaStream_t s);
+// out[0] = mean of losses[0..M) (fixed-order reduction)
+void mean_loss(float* out, const float* losses, int M, cudaStream_t s);
+
+// ----------------------------------------------------------- optimizer --
+void init_params(float* p, const Layout& lay, uint64_t seed, cudaStream_t s);
+void f32_to_act(act_t* out, const float* in, size_t n, cudaStream_t s);
+void act_to_f32(float* out, const act_t* in, size_t n, cudaStream_t s);
+
+// scalars layout (device floats)
+enum Scalar { S_NORM = 0, S_CLIP = 1, S_LOSS = 2, S_COUNT = 16 };
+constexpr int kNormBlocks = 592;
+// scalars[S_NORM] = ||g||_2, scalars[S_CLIP] = max_norm / (norm + 1e-6) or 1
+void grad_norm_clip(float* scalars, const float* g, size_t n, float max_norm, double* partials,
+                    cudaStream_t s);
+
+// scalars[S_NORM] = 0, scalars[S_CLIP] = 1 (no clipping pending)
+void reset_clip(float* scalars, cudaStream_t s);
+
+struct AdamArgs {
+  float lr, b1, b2, eps, wd;
+  float bc1, bc2;  // 1 - b1^t, 1 - b2^t
+};
+// Decay applies to the tensors flagged in `decay_mask` (bit per tensor).
+void adamw(float* p, act_t* pact, const float* g, float* m, float* v, const Layout& lay,
+           const AdamArgs& a, const float* scalars, cudaStream_t s);
+
+// Process-wide count of kernel launches made by this library.
+void note_launch(int n = 1);
+long launch_count();
+
+// Error bits in the device error word.
+enum ErrBits { ERR_TOKEN = 1, ERR_TARGET = 2, ERR_TIMEOUT = 4 };
+
+}  // namespace gpt2k

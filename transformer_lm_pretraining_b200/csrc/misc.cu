@@ -1,0 +1,427 @@
+// Bias-gradient column sums, the fused softmax cross-entropy, the mean
+// loss, parameter init, the global gradient norm and AdamW.
+
+#include <atomic>
+
+#include "kernels.h"
+
+namespace gpt2k {
+
+// ------------------------------------------------------------ layout --
+Layout make_layout(int L, int H, int C, int V, int Vp, int Tmax) {
+  Layout g;
+  g.L = L; g.H = H; g.C = C; g.V = V; g.Vp = Vp; g.Tmax = Tmax;
+  const size_t l = (size_t)L, c = (size_t)C;
+  g.num[T_WTE] = (size_t)Vp * c;
+  g.num[T_WPE] = (size_t)Tmax * c;
+  g.num[T_LN1G] = l * c;
+  g.num[T_LN1B] = l * c;
+  g.num[T_WQKV] = l * 3 * c * c;
+  g.num[T_BQKV] = l * 3 * c;
+  g.num[T_WO] = l * c * c;
+  g.num[T_BO] = l * c;
+  g.num[T_LN2G] = l * c;
+  g.num[T_LN2B] = l * c;
+  g.num[T_WFC] = l * 4 * c * c;
+  g.num[T_BFC] = l * 4 * c;
+  g.num[T_WP] = l * 4 * c * c;
+  g.num[T_BP] = l * c;
+  g.num[T_LNFG] = c;
+  g.num[T_LNFB] = c;
+  size_t o = 0;
+  for (int i = 0; i < T_COUNT; ++i) {
+    g.off[i] = o;
+    o += g.num[i];
+  }
+  g.total = o;
+  return g;
+}
+
+static std::atomic<long> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+long launch_count() { return g_launches.load(std::memory_order_relaxed); }
+
+bool tensor_decayed(int t) {
+  return t == T_WTE || t == T_WPE || t == T_WQKV || t == T_WO || t == T_WFC || t == T_WP;
+}
+
+namespace {
+
+// ------------------------------------------------------------ colsum --
+// partials[chunk][n] = sum over the chunk's rows (ascending) of dy[m, n];
+// block = 32 x 8 threads, 64 columns (2 per thread).
+__global__ void colsum_partial_kernel(float* __restrict__ partials, const act_t* __restrict__ dy,
+                                      int M, int N, int rows_per_chunk) {
+  __shared__ float red[8][64];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int n = blockIdx.x * 64 + 2 * tx;
+  const int r0 = blockIdx.y * rows_per_chunk;
+  const int r1 = min(M, r0 + rows_per_chunk);
+  float s0 = 0.f, s1 = 0.f;
+  if (n < N) {
+    for (int r = r0 + ty; r < r1; r += 8) {
+      const act_t* p = dy + (size_t)r * N + n;
+      s0 += to_f(p[0]);
+      if (n + 1 < N) s1 += to_f(p[1]);
+    }
+  }
+  red[ty][2 * tx] = s0;
+  red[ty][2 * tx + 1] = s1;
+  __syncthreads();
+  if (ty == 0) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float s = 0.f;
+      for (int k = 0; k < 8; ++k) s += red[k][2 * tx + j];
+      if (n + j < N) partials[(size_t)blockIdx.y * N + n + j] = s;
+    }
+  }
+}
+
+__global__ void colsum_reduce_kernel(float* __restrict__ db, const float* __restrict__ partials,
+                                     int chunks, int N) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  float s = 0.f;
+  for (int c = 0; c < chunks; ++c) s += partials[(size_t)c * N + n];
+  db[n] += s;
+}
+
+// -------------------------------------------------------- classifier --
+// One block per row.  Pass 1: max and sum of exp over the first V logits
+// (per-thread online, then block reduction in fixed order).  Pass 2:
+// z <- (exp(z - lse) - [col == tgt]) / M for col < V, 0 for padding.
+constexpr int kClsThreads = 512;
+
+__device__ __forceinline__ void online_merge(float& m, float& s, float m2, float s2) {
+  if (m2 > m) {
+    s = s * __expf(m - m2) + s2;
+    m = m2;
+  } else if (m2 > -INFINITY) {
+    s += s2 * __expf(m2 - m);
+  }
+}
+
+__global__ void __launch_bounds__(kClsThreads)
+    classifier_kernel(act_t* __restrict__ logits, float* __restrict__ losses,
+                      const int* __restrict__ tgt, int M, int V, int Vp, int* err) {
+  const int row = blockIdx.x;
+  act_t* z = logits + (size_t)row * Vp;
+  const int vec = (Vp % 8 == 0) ? 8 : 1;
+  float mx = -INFINITY, sm = 0.f;
+  if (vec == 8) {
+    for (int c = threadIdx.x * 8; c < Vp; c += kClsThreads * 8) {
+      float v[8];
+      load8(z + c, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (c + i < V) online_merge(mx, sm, v[i], 1.f);
+    }
+  } else {
+    for (int c = threadIdx.x; c < V; c += kClsThreads) online_merge(mx, sm, to_f(z[c]), 1.f);
+  }
+  // warp then block reduction (fixed order)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, mx, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, sm, o);
+    online_merge(mx, sm, m2, s2);
+  }
+  __shared__ float wm[kClsThreads / 32], ws[kClsThreads / 32];
+  __shared__ float lse_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    wm[warp] = mx;
+    ws[warp] = sm;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = wm[0], s = ws[0];
+    for (int w = 1; w < kClsThreads / 32; ++w) online_merge(m, s, wm[w], ws[w]);
+    lse_s = m + logf(s);
+  }
+  __syncthreads();
+  const float lse = lse_s;
+  int t = tgt[row];
+  if (t < 0 || t >= V) {
+    if (threadIdx.x == 0) atomicOr(err, ERR_TARGET);
+    t = 0;
+  }
+  if (threadIdx.x == 0) losses[row] = lse - to_f(z[t]);
+  __syncthreads();  // the target logit is read before it is overwritten
+  const float inv = 1.0f / (float)M;
+  if (vec == 8) {
+    for (int c = threadIdx.x * 8; c < Vp; c += kClsThreads * 8) {
+      float v[8];
+      load8(z + c, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int col = c + i;
+        v[i] = col < V ? (__expf(v[i] - lse) - (col == t ? 1.f : 0.f)) * inv : 0.f;
+      }
+      store8(z + c, v);
+    }
+  } else {
+    for (int c = threadIdx.x; c < Vp; c += kClsThreads) {
+      const float v = to_f(z[c]);
+      z[c] = from_f<act_t>(c < V ? (__expf(v - lse) - (c == t ? 1.f : 0.f)) * inv : 0.f);
+    }
+  }
+}
+
+__global__ void mean_loss_kernel(float* out, const float* __restrict__ losses, int M) {
+  __shared__ float red[1024];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) s += losses[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[0] = red[0] / (float)M;
+}
+
+// -------------------------------------------------------------- init --
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): output n of a generator
+// seeded with s is mix(s + n * 0x9E3779B97F4A7C15).  Tensor t uses the
+// generator seeded with output t+1 of the master generator seeded with
+// `seed`; element i takes outputs 2i+1, 2i+2 as the two uniforms of one
+// Box-Muller normal (cosine branch), evaluated in double, rounded once.
+__device__ __forceinline__ uint64_t sm64_mix(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+__device__ __forceinline__ uint64_t sm64_out(uint64_t seed, uint64_t n) {
+  return sm64_mix(seed + n * 0x9E3779B97F4A7C15ull);
+}
+
+struct InitSeg {
+  size_t off, count;  // elements [off, off + count) get normals
+  uint64_t tseed;
+  double sd;
+};
+struct InitTable {
+  InitSeg seg[6];
+  int n;
+};
+
+__global__ void init_normal_kernel(float* __restrict__ p, InitTable tab) {
+  const InitSeg sg = tab.seg[blockIdx.y];
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < sg.count;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const uint64_t r1 = sm64_out(sg.tseed, 2 * i + 1);
+    const uint64_t r2 = sm64_out(sg.tseed, 2 * i + 2);
+    const double u1 = (double)((r1 >> 11) + 1) * 0x1.0p-53;
+    const double u2 = (double)(r2 >> 11) * 0x1.0p-53;
+    const double z = sqrt(-2.0 * log(u1)) * cos(6.283185307179586476925286766559 * u2);
+    p[sg.off + i] = (float)(sg.sd * z);
+  }
+}
+
+__global__ void fill_kernel(float* p, size_t n, float v) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    p[i] = v;
+}
+
+template <class TO, class TI>
+__global__ void convert_kernel(TO* __restrict__ out, const TI* __restrict__ in, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    out[i] = from_f<TO>(to_f(in[i]));
+}
+
+// -------------------------------------------------------- grad norm --
+// Stage 1: block b sums g^2 over the fixed strided set of float4s
+// i = b * 256 + tid + k * (gridDim.x * 256) in double, then reduces over the
+// block in a fixed tree.  Stage 2 (one block) adds the block sums in order.
+__global__ void __launch_bounds__(256) norm_partial_kernel(double* __restrict__ partials,
+                                                           const float* __restrict__ g,
+                                                           size_t n) {
+  __shared__ double red[256];
+  double s = 0.0;
+  const size_t n4 = n / 4;
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n4; i += (size_t)gridDim.x * 256) {
+    const float4 v = g4[i];
+    s += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+  }
+  if (blockIdx.x == 0)
+    for (size_t i = n4 * 4 + threadIdx.x; i < n; i += 256) s += (double)g[i] * g[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) partials[blockIdx.x] = red[0];
+}
+
+__global__ void norm_final_kernel(float* __restrict__ scalars, const double* __restrict__ partials,
+                                  int nblk, float max_norm) {
+  if (threadIdx.x != 0) return;
+  double s = 0.0;
+  for (int b = 0; b < nblk; ++b) s += partials[b];
+  const float nrm = (float)sqrt(s);
+  scalars[S_NORM] = nrm;
+  scalars[S_CLIP] = (nrm > max_norm) ? max_norm / (nrm + 1e-6f) : 1.0f;
+}
+
+// ------------------------------------------------------------- AdamW --
+struct DecayTable {
+  size_t begin[T_COUNT];
+  size_t end[T_COUNT];
+  int n;
+};
+
+__global__ void __launch_bounds__(256)
+    adamw_kernel(float* __restrict__ p, act_t* __restrict__ pact, const float* __restrict__ g,
+                 float* __restrict__ m, float* __restrict__ v, size_t n, AdamArgs a,
+                 DecayTable dt, const float* __restrict__ scalars) {
+  const float nrm = scalars[S_NORM];
+  if (!isfinite(nrm)) return;  // never apply a non-finite update
+  const float clip = scalars[S_CLIP];
+  const size_t n4 = n / 4;
+  for (size_t i4 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4;
+       i4 += (size_t)gridDim.x * blockDim.x) {
+    const size_t i = i4 * 4;
+    float wd = 0.f;
+    for (int k = 0; k < dt.n; ++k)
+      if (i >= dt.begin[k] && i < dt.end[k]) wd = a.wd;
+    float4 pp = reinterpret_cast<float4*>(p)[i4];
+    const float4 gg = reinterpret_cast<const float4*>(g)[i4];
+    float4 mm = reinterpret_cast<float4*>(m)[i4];
+    float4 vv = reinterpret_cast<float4*>(v)[i4];
+    float* pe = &pp.x;
+    const float* ge = &gg.x;
+    float* me = &mm.x;
+    float* ve = &vv.x;
+    float outv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float gr = ge[j] * clip;
+      me[j] = a.b1 * me[j] + (1.f - a.b1) * gr;
+      ve[j] = a.b2 * ve[j] + (1.f - a.b2) * gr * gr;
+      const float mh = me[j] / a.bc1;
+      const float vh = ve[j] / a.bc2;
+      pe[j] -= a.lr * (mh / (sqrtf(vh) + a.eps) + wd * pe[j]);
+      outv[j] = pe[j];
+    }
+    reinterpret_cast<float4*>(p)[i4] = pp;
+    reinterpret_cast<float4*>(m)[i4] = mm;
+    reinterpret_cast<float4*>(v)[i4] = vv;
+#if GPT2_ACT_BF16
+    __nv_bfloat162 lo = __floats2bfloat162_rn(outv[0], outv[1]);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(outv[2], outv[3]);
+    uint2 packed;
+    packed.x = *reinterpret_cast<uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(pact)[i4] = packed;
+#else
+    (void)pact;
+    (void)outv;
+#endif
+  }
+}
+
+__global__ void reset_clip_kernel(float* scalars) {
+  scalars[S_NORM] = 0.f;
+  scalars[S_CLIP] = 1.f;
+}
+
+int grid_for(size_t n, int threads, int max_blocks) {
+  size_t b = (n + threads - 1) / threads;
+  if (b > (size_t)max_blocks) b = max_blocks;
+  if (b < 1) b = 1;
+  return (int)b;
+}
+
+}  // namespace
+
+void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s) {
+  const int rows = (M + kColsumChunks - 1) / kColsumChunks;
+  const int chunks = (M + rows - 1) / rows;
+  dim3 g((N + 63) / 64, chunks);
+  colsum_partial_kernel<<<g, 256, 0, s>>>(partials, dy, M, N, rows);
+  colsum_reduce_kernel<<<(N + 255) / 256, 256, 0, s>>>(db, partials, chunks, N);
+  note_launch(2);
+}
+
+void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int Vp, int* err,
+                cudaStream_t s) {
+  classifier_kernel<<<M, kClsThreads, 0, s>>>(logits, losses, tgt, M, V, Vp, err);
+  note_launch();
+}
+
+void mean_loss(float* out, const float* losses, int M, cudaStream_t s) {
+  mean_loss_kernel<<<1, 1024, 0, s>>>(out, losses, M);
+  note_launch();
+}
+
+void init_params(float* p, const Layout& lay, uint64_t seed, cudaStream_t s) {
+  cudaMemsetAsync(p, 0, lay.total * sizeof(float), s);
+  const int gains[3] = {T_LN1G, T_LN2G, T_LNFG};
+  for (int t : gains)
+    fill_kernel<<<grid_for(lay.num[t], 256, 1024), 256, 0, s>>>(p + lay.off[t], lay.num[t], 1.0f);
+  InitTable tab;
+  tab.n = 0;
+  const double sd = 0.02, sd_res = 0.02 / sqrt(2.0 * lay.L);
+  const int normals[6] = {T_WTE, T_WPE, T_WQKV, T_WO, T_WFC, T_WP};
+  size_t maxc = 0;
+  for (int t : normals) {
+    InitSeg& sg = tab.seg[tab.n++];
+    sg.off = lay.off[t];
+    sg.count = (t == T_WTE) ? (size_t)lay.V * lay.C : lay.num[t];  // pad rows stay 0
+    // tensor seed = output (t + 1) of the master SplitMix64 seeded with `seed`
+    uint64_t z = seed + (uint64_t)(t + 1) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    sg.tseed = z ^ (z >> 31);
+    sg.sd = (t == T_WO || t == T_WP) ? sd_res : sd;
+    if (sg.count > maxc) maxc = sg.count;
+  }
+  dim3 grid(grid_for(maxc, 256, 2048), tab.n);
+  init_normal_kernel<<<grid, 256, 0, s>>>(p, tab);
+  note_launch(4);
+}
+
+void f32_to_act(act_t* out, const float* in, size_t n, cudaStream_t s) {
+  convert_kernel<act_t, float><<<grid_for(n, 256, 4096), 256, 0, s>>>(out, in, n);
+  note_launch();
+}
+
+void act_to_f32(float* out, const act_t* in, size_t n, cudaStream_t s) {
+  convert_kernel<float, act_t><<<grid_for(n, 256, 4096), 256, 0, s>>>(out, in, n);
+  note_launch();
+}
+
+void grad_norm_clip(float* scalars, const float* g, size_t n, float max_norm, double* partials,
+                    cudaStream_t s) {
+  norm_partial_kernel<<<kNormBlocks, 256, 0, s>>>(partials, g, n);
+  norm_final_kernel<<<1, 32, 0, s>>>(scalars, partials, kNormBlocks, max_norm);
+  note_launch(2);
+}
+
+void reset_clip(float* scalars, cudaStream_t s) {
+  reset_clip_kernel<<<1, 1, 0, s>>>(scalars);
+  note_launch();
+}
+
+void adamw(float* p, act_t* pact, const float* g, float* m, float* v, const Layout& lay,
+           const AdamArgs& a, const float* scalars, cudaStream_t s) {
+  DecayTable dt;
+  dt.n = 0;
+  for (int t = 0; t < T_COUNT; ++t)
+    if (tensor_decayed(t)) {
+      dt.begin[dt.n] = lay.off[t];
+      dt.end[dt.n] = lay.off[t] + lay.num[t];
+      ++dt.n;
+    }
+  adamw_kernel<<<grid_for(lay.total / 4, 256, kNumSMs * 8), 256, 0, s>>>(p, pact, g, m, v,
+                                                                         lay.total, a, dt, scalars);
+  note_launch();
+}
+
+}  // namespace gpt2k
