@@ -188,12 +188,17 @@ def test_attention_forward_backward(B, T, C, H):
     dabs = np.abs(datt * o_bf).reshape(B * T, H, hd).sum(-1)
     kmax = np.abs(qkv[:, C:2 * C]).reshape(B, T, H, hd).max(axis=1)
     extra_q = (2 ** -8 / np.sqrt(hd)) * dabs.reshape(B, T, H, 1) * kmax[:, None]
+    # dK_j = scale sum_i P_ij (dP_ij - D_i) q_i sums the same D_i errors over
+    # the queries attending to key j: allow 6e-2 rms there, and check the
+    # whole of each part in relative L2 as well.
     extra = [extra_q.reshape(B * T, C), 0.0, 0.0]
+    frac = [5e-2, 6e-2, 5e-2]
     for part in range(3):
         sl = slice(part * C, (part + 1) * C)
         err = np.abs(got[:, sl] - ref_d[:, sl])
-        bound = 2 ** -6 * np.abs(ref_d[:, sl]) + 5e-2 * rms(ref_d[:, sl]) + extra[part]
+        bound = 2 ** -6 * np.abs(ref_d[:, sl]) + frac[part] * rms(ref_d[:, sl]) + extra[part]
         assert (err <= bound).all(), (part, (err / bound).max())
+        assert np.linalg.norm(got[:, sl] - ref_d[:, sl]) <= 1e-2 * np.linalg.norm(ref_d[:, sl])
 
 
 def test_attention_backward_is_deterministic():
