@@ -60,6 +60,43 @@ int gpt2k_attention_bwd(void* stream, void* dqkv, float* dsum, const void* datt,
  * GEMM expired); read and cleared.  Synchronous. */
 int gpt2k_take_error(void);
 
+/* Size, in floats, of the fixed scratch array behind
+ * gpt2k_gemm_wgrad_noalloc (16 MiB). */
+#define GPT2K_NOALLOC_SCRATCH_FLOATS (4u << 20)
+
+/* The weight-gradient product of gpt2k_gemm (a_mn = b_mn = 1, fp32
+ * accumulate: out32[m, n] += alpha * sum_k A[k lda + m] B[k ldb + n]) for
+ * callers that cannot give the library device memory.  The pages have no
+ * counterpart of this call; it exists for the host side of this library.
+ *
+ * Who needs it: a caller whose device memory all belongs to its own
+ * allocator -- for instance PyTorch's caching allocator, which may already
+ * hold nearly all free memory, so that any cudaMalloc made behind its back
+ * fails or fragments the pool -- and which therefore cannot hand over a
+ * split-K workspace, nor let the library allocate one.
+ *
+ * What it does instead: the split-K partial sums go to a file-scope device
+ * array of GPT2K_NOALLOC_SCRATCH_FLOATS floats that every GPU holds from the
+ * moment it loads the library until the process exits.  The call allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *  - At most max_splits (1..8) K-slices are used; max_splits * M * N must
+ *    not exceed GPT2K_NOALLOC_SCRATCH_FLOATS, else GPT2_ERR_ARG is returned
+ *    before any work is enqueued.  The result is the same as gpt2k_gemm's
+ *    weight-gradient form given a workspace of max_splits * M * N floats.
+ *  - The first call on a device looks up the array's device address on that
+ *    (current) device; make that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves its last
+ *    partial sums in it; each call writes every partial it later reads, and
+ *    clears its own error word.  Calls whose work overlaps on the GPU (other
+ *    streams, other threads) race on the array: serialise them.
+ *  - err_dev (may be NULL) is a device int that receives bit 2 if a bounded
+ *    wait inside the GEMM expired; with NULL that report goes to a private
+ *    word and is dropped.
+ * Operands and strides as for gpt2k_gemm; asynchronous on `stream`. */
+int gpt2k_gemm_wgrad_noalloc(void* stream, int M, int N, int K, const void* A, long lda,
+                             const void* B, long ldb, float alpha, float* out32, long ldo32,
+                             int max_splits, int* err_dev);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
          "-I", CSRC, "-I", os.path.join(ROOT, "include")]
 
-COMMON = ["gpt2.cu", "kernel_abi.cu", "encoder.cu", "layernorm.cu", "misc.cu", "attention.cu"]
+COMMON = ["gpt2.cu", "kernel_abi.cu", "noalloc.cu", "encoder.cu", "layernorm.cu", "misc.cu",
+          "attention.cu"]
 VARIANTS = {
     "libgpt2.so": (COMMON + ["gemm_tc.cu"], []),
     "libgpt2_fp32.so": (COMMON + ["gemm_simt.cu"], ["-DGPT2_FP32_VALIDATE"]),

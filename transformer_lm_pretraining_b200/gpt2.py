@@ -68,6 +68,7 @@ SIGNATURES = {
     "gpt2k_attention_fwd": (_i, [_vp, _vp, _fp, _vp, _i, _i, _i, _i]),
     "gpt2k_attention_bwd": (_i, [_vp, _vp, _fp, _vp, _vp, _vp, _fp, _i, _i, _i, _i]),
     "gpt2k_take_error": (_i, []),
+    "gpt2k_gemm_wgrad_noalloc": (_i, [_vp, _i, _i, _i, _vp, _l, _vp, _l, _f, _fp, _l, _i, _vp]),
 }
 
 _LIBS: dict = {}
@@ -301,3 +302,17 @@ def gpt2k_attention_bwd(dqkv, dsum, datt, qkv, att, lse, B, T, C, H, precision="
 
 def gpt2k_take_error(precision="bf16") -> int:
     return int(load(precision).gpt2k_take_error())
+
+
+def gpt2k_gemm_wgrad_noalloc(M, N, K, A, lda, B, ldb, alpha, out32, ldo32, max_splits=8,
+                             err=None, precision="bf16", stream=None) -> int:
+    """Weight-gradient GEMM whose split-K scratch is the library's fixed
+    device array (no device memory is allocated or passed in); returns the
+    C status code (0 = OK)."""
+    import torch
+
+    L = load(precision)
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(L.gpt2k_gemm_wgrad_noalloc(
+        s.cuda_stream, M, N, K, _dptr(A), lda, _dptr(B), ldb, alpha,
+        ctypes.cast(ctypes.c_void_p(out32.data_ptr()), _fp), ldo32, max_splits, _dptr(err)))
