@@ -183,12 +183,13 @@ const char* gpt2_last_error(const gpt2_t* h);
 long gpt2_launch_count(void);
 
 /* Per-kernel-family timing with CUDA events on the handle's stream.  Kinds:
- * 0 GEMM, 1 attention forward, 2 attention backward, 3 LayerNorm (fwd+bwd),
- * 4 classifier, 5 encoder (fwd+bwd), 6 bias-gradient column sums,
- * 7 optimiser (norm, clip, AdamW).  gpt2_profile_read synchronises the
- * stream, writes for each kind the summed milliseconds, the number of timed
- * regions and the algorithmic FLOPs (GEMM: 2MNK; attention: causal products),
- * and clears the records.  `kinds` is the length of the arrays (>= 8). */
+ * 0 GEMM, 1 attention forward, 2 attention backward, 3 LayerNorm forward,
+ * 4 LayerNorm backward, 5 classifier, 6 encoder (fwd+bwd), 7 bias-gradient
+ * column sums, 8 optimiser (norm, clip, AdamW).  gpt2_profile_read
+ * synchronises the stream, writes for each kind the summed milliseconds, the
+ * number of timed regions and the algorithmic FLOPs (GEMM: 2MNK; attention:
+ * causal products), and clears the records.  `kinds` is the length of the
+ * arrays (>= 9). */
 gpt2_status gpt2_profile_enable(gpt2_t* h, int on);
 gpt2_status gpt2_profile_read(gpt2_t* h, double* ms, long* launches, double* flops, int kinds);
 

@@ -67,8 +67,26 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float* v) {
   *reinterpret_cast<uint4*>(p) = u;
 }
 
-// GPT-2's GELU: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) and its
-// derivative (the tanh form named on the condensed GPT-2 page).
+// GPT-2's GELU: 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3), and
+// its derivative (the tanh form named on the condensed GPT-2 page).
+#if GPT2_ACT_BF16
+// bf16 build: the same function through the identity 0.5 (1 + tanh(u)) =
+// 1 / (1 + exp(-2u)), evaluated with the fast exp and divide intrinsics (two
+// special-function ops per element, accurate to a few fp32 ulps even where
+// 1 + tanh(u) is tiny), which keeps the GEMM epilogues off the critical path.
+__device__ __forceinline__ float gelu_sigmoid_arg(float x) {
+  const float k2 = 1.5957691216057308f;  // 2 sqrt(2/pi)
+  return fmaxf(k2 * (x + 0.044715f * x * x * x), -80.0f);  // exp(-2u) stays finite
+}
+__device__ __forceinline__ float gelu_tanh(float x) {
+  return __fdividef(x, 1.0f + __expf(-gelu_sigmoid_arg(x)));
+}
+__device__ __forceinline__ float gelu_tanh_grad(float x) {
+  const float s = __fdividef(1.0f, 1.0f + __expf(-gelu_sigmoid_arg(x)));
+  const float du = 1.5957691216057308f * (1.0f + 3.0f * 0.044715f * x * x);  // d(2u)/dx
+  return s + x * s * (1.0f - s) * du;
+}
+#else
 __device__ __forceinline__ float gelu_tanh(float x) {
   const float k = 0.7978845608028654f;
   return 0.5f * x * (1.0f + tanhf(k * (x + 0.044715f * x * x * x)));
@@ -79,5 +97,6 @@ __device__ __forceinline__ float gelu_tanh_grad(float x) {
   const float dinner = k * (1.0f + 3.0f * 0.044715f * x * x);
   return 0.5f * (1.0f + th) + 0.5f * x * (1.0f - th * th) * dinner;
 }
+#endif
 
 }  // namespace gpt2k

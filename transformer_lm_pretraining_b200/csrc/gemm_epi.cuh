@@ -52,6 +52,7 @@ template <int EPI>
 __device__ __forceinline__ void epi_row32(const EpiParams& e, int m, int n0, float* v,
                                           bool vec_ok) {
   if (!(vec_ok && n0 + 32 <= e.N)) {
+#pragma unroll
     for (int i = 0; i < 32; ++i)
       if (n0 + i < e.N) epi_scalar<EPI>(e, m, n0 + i, v[i]);
     return;

@@ -5,9 +5,12 @@
 //              into a STAGES-deep shared-memory ring;
 //   warp 1     allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16)
 //              from one elected lane, accumulating fp32 in TMEM;
-//   warps 2-5  epilogue: tcgen05.ld of the 128 x BN accumulator (one row per
-//              thread), bias / GELU / residual / GELU-backward / fp32
-//              accumulate, global stores.
+//   warps 2-5  epilogue, 64 columns at a time: tcgen05.ld of the accumulator
+//              (thread = row), bias / GELU / residual / GELU-backward, then
+//              the results are written to a 128-byte-swizzled shared-memory
+//              box and leave with one TMA bulk store (TMA reduce-add for the
+//              fp32 gradient accumulation).  Residual and pre-activation
+//              inputs arrive by TMA into the same kind of box.
 // The TMEM accumulator is double-buffered so the epilogue of one tile runs
 // under the main loop of the next.  Both operands may be K-major or
 // MN-major (the tensor core reads either from the descriptor), which covers
@@ -22,6 +25,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -34,6 +38,7 @@ namespace tc {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int kThreads = 192;
+constexpr int kStageBox = 16384;  // one 128-row x 128-byte epilogue box
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -93,6 +98,59 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm,
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                            int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, uint32_t src, int x, int y,
+                                             int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tm)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* tm, uint32_t src, int x,
+                                                  int y, int z) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::
+          "l"(reinterpret_cast<uint64_t>(tm)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void epi_bar() {  // the 128 epilogue threads
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// Barrier of the 128 epilogue threads that also ANDs a predicate over them,
+// so that every epilogue warp takes the same branch after a bounded wait.
+__device__ __forceinline__ bool epi_bar_and(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -118,7 +176,7 @@ __device__ __forceinline__ void tc_wait_ld() {
 }
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives
 // row (lane base + i), columns taddr.col .. +31.
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -162,32 +220,44 @@ constexpr uint32_t tmem_cols() {
 
 template <int BN, int STAGES>
 constexpr size_t smem_bytes() {
-  return 1024 + (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 256;
+  return 1024 + (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 2 * kStageBox + 256;
+}
+
+// Byte offset of 16-byte chunk j of row r in a 128-byte-swizzled box.
+__device__ __forceinline__ uint32_t swz(int r, int j) {
+  return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
 }
 
 template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const EpiParams ep, int K, int tiles_m, int tiles_n, int splits, int kb_per_split,
-                   int n_fast, int vec_ok, long split_stride, int* err) {
+                   const __grid_constant__ CUtensorMap tmOut,
+                   const __grid_constant__ CUtensorMap tmX, const EpiParams ep, int K,
+                   int tiles_m, int tiles_n, int splits, int kb_per_split, int n_fast, int* err) {
   constexpr int A_BYTES = BM * BK * 2;
   constexpr int B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = tmem_cols<BN>();
+  constexpr bool HAS_IN = (EPI == EPI_BIAS_RESID || EPI == EPI_DGELU);
+  constexpr bool F32_OUT = (EPI == EPI_F32_ACC || EPI == EPI_F32_STORE);
+  constexpr bool HAS_BIAS = (EPI == EPI_BIAS || EPI == EPI_BIAS_GELU || EPI == EPI_BIAS_RESID);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * (A_BYTES + B_BYTES));
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  uint8_t* st0 = smem + STAGES * (A_BYTES + B_BYTES);  // epilogue boxes (1024-aligned)
+  uint8_t* st1 = st0 + kStageBox;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(st1 + kStageBox);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
   const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t in_full = smem_u32(bars + 2 * STAGES + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -204,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, 128);
     }
+    mbar_init(in_full, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -340,38 +411,123 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- epilogue --
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
+    const int etid = threadIdx.x - 64;  // 0 .. 127
+    const uint32_t st0_u = smem_u32(st0), st1_u = smem_u32(st1);
+    if (etid == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmOut)) : "memory");
+      if (HAS_IN || EPI == EPI_BIAS_GELU)
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
+    }
     int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    uint32_t acc_phase = 0, in_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       int tm, tn, kb0, kb1, sp;
       decode(u, tm, tn, kb0, kb1, sp);
-      // warp-uniform decision: the TMEM loads below are warp-collective
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, err));
+      const int m0 = tm * BM, nt0 = tn * BN;
+      const int ngroups = (min(BN, ep.N - nt0) + 63) >> 6;  // 64-column groups in range
+      if (HAS_IN && etid == 0) {
+        mbar_expect_tx(in_full, kStageBox);
+        tma_load_3d(st1_u, &tmX, in_full, nt0, m0, 0);
+      }
+      // uniform decision over the epilogue warps (TMEM loads are
+      // warp-collective and the named barriers below need all 128 threads)
+      ok = epi_bar_and(mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, err));
       if (!ok) break;
       tc_fence_after();
-      const int m = tm * BM + row;
-      EpiParams e = ep;
-      if (EPI == EPI_F32_STORE) e.out32 += (size_t)sp * split_stride;
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        const int n0 = tn * BN + c0;
-        if (n0 >= ep.N) break;  // uniform across the warp
-        uint32_t r[32];
-        tc_ld32(t_row + (uint32_t)c0, r);
-        tc_wait_ld();
-        if (m < ep.M) {
-          float v[32];
+      for (int g = 0; g < ngroups; ++g) {
+        const int nb = nt0 + 64 * g;
+        float v[64];
+        {
+          uint32_t r[64];
+          tc_ld32(t_row + (uint32_t)(64 * g), r);
+          tc_ld32(t_row + (uint32_t)(64 * g + 32), r + 32);
+          tc_wait_ld();
+          if (g == ngroups - 1) {  // every TMEM read of this tile is done
+            tc_fence_before();
+            mbar_arrive(tempty0 + 8 * acc);
+          }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          epi_row32<EPI>(e, m, n0, v, vec_ok != 0);
+          for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]) * ep.alpha;
+        }
+        if (HAS_BIAS && ep.bias) {
+          if (nb + 64 <= ep.N) {
+            const float4* b4 = reinterpret_cast<const float4*>(ep.bias + nb);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float4 b = b4[j];
+              v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (nb + i < ep.N) v[i] += ep.bias[nb + i];
+          }
+        }
+        if (HAS_IN) {
+          ok = epi_bar_and(mbar_wait(in_full, in_phase, abort_flag, err));
+          if (!ok) break;
+          in_phase ^= 1u;
+          float x[64];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) load8(reinterpret_cast<const act_t*>(st1 + swz(row, j)), x + 8 * j);
+          epi_bar();  // everyone has read the input box
+          if (etid == 0 && g + 1 < ngroups) {
+            fence_async_smem();
+            mbar_expect_tx(in_full, kStageBox);
+            tma_load_3d(st1_u, &tmX, in_full, nb + 64, m0, 0);
+          }
+          if (EPI == EPI_BIAS_RESID) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] += x[i];
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] *= gelu_tanh_grad(x[i]);
+          }
+        }
+        // the previous group's stores must have read the boxes
+        if (etid == 0) bulk_wait_read_all();
+        epi_bar();
+        if (F32_OUT) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            *reinterpret_cast<float4*>(st0 + swz(row, j)) =
+                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            *reinterpret_cast<float4*>(st1 + swz(row, j)) =
+                make_float4(v[32 + 4 * j], v[33 + 4 * j], v[34 + 4 * j], v[35 + 4 * j]);
+          }
+        } else {
+          if (EPI == EPI_BIAS_GELU) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(st1 + swz(row, j)), v + 8 * j);
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = gelu_tanh(v[i]);
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(st0 + swz(row, j)), v + 8 * j);
+        }
+        fence_async_smem();
+        epi_bar();
+        if (etid == 0) {
+          if (EPI == EPI_F32_ACC) {
+            tma_reduce_add_3d(&tmOut, st0_u, nb, m0, 0);
+            if (nb + 32 < ep.N) tma_reduce_add_3d(&tmOut, st1_u, nb + 32, m0, 0);
+          } else if (EPI == EPI_F32_STORE) {
+            tma_store_3d(&tmOut, st0_u, nb, m0, sp);
+            if (nb + 32 < ep.N) tma_store_3d(&tmOut, st1_u, nb + 32, m0, sp);
+          } else {
+            tma_store_3d(&tmOut, st0_u, nb, m0, 0);
+            if (EPI == EPI_BIAS_GELU) tma_store_3d(&tmX, st1_u, nb, m0, 0);
+          }
+          bulk_commit();
         }
       }
-      tc_fence_before();
-      mbar_arrive(tempty0 + 8 * acc);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (etid == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -398,13 +554,18 @@ static cudaError_t get_encoder() {
   return cudaSuccess;
 }
 
-// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows
-// `ld` elements apart; box of 64 x box_outer with 128-byte swizzle.
-static cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t outer,
-                             uint64_t ld, uint32_t box_outer) {
-  using Key = std::tuple<const void*, uint64_t, uint64_t, uint64_t, uint32_t>;
+// Tensor map with 128-byte swizzle over a row-major [outer][inner] array
+// (`ld` elements between rows), box box_inner x box_outer.  depth = 0 gives
+// a rank-2 map (GEMM operands); depth >= 1 a rank-3 map over `depth` such
+// arrays `dstride` elements apart (epilogue boxes, addressed with 3-D
+// coordinates), box depth 1.  fp32 = element type float, else bf16.
+static cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, bool fp32, uint64_t inner,
+                             uint64_t outer, uint64_t ld, uint32_t box_inner, uint32_t box_outer,
+                             uint64_t depth = 0, uint64_t dstride = 0) {
+  using Key = std::tuple<const void*, bool, uint64_t, uint64_t, uint64_t, uint32_t, uint32_t,
+                         uint64_t, uint64_t>;
   static std::map<Key, CUtensorMap> cache;
-  const Key key{ptr, inner, outer, ld, box_outer};
+  const Key key{ptr, fp32, inner, outer, ld, box_inner, box_outer, depth, dstride};
   {
     std::lock_guard<std::mutex> g(g_mu);
     auto it = cache.find(key);
@@ -415,14 +576,16 @@ static cudaError_t make_tmap(CUtensorMap* tm, const void* ptr, uint64_t inner, u
   }
   cudaError_t e = get_encoder();
   if (e != cudaSuccess) return e;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64u, box_outer};
-  cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const uint64_t es = fp32 ? 4 : 2;
+  const cuuint32_t rank = depth >= 1 ? 3 : 2;
+  cuuint64_t dims[3] = {inner, outer, depth >= 1 ? depth : 1};
+  cuuint64_t strides[2] = {ld * es, (depth > 1 ? dstride : ld * outer) * es};
+  cuuint32_t box[3] = {box_inner, box_outer, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = g_encode(tm, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        rank, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   std::lock_guard<std::mutex> g(g_mu);
   if (cache.size() > 4096) cache.clear();
@@ -442,11 +605,12 @@ static int num_sms() {
 }
 
 template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI>
-static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const EpiParams& ep, int K,
-                          int splits, int kb_per_split, int n_fast, int vec_ok, long split_stride,
-                          cudaStream_t s, int* err) {
+static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                          const CUtensorMap& tx, const EpiParams& ep, int K, int splits,
+                          int kb_per_split, int n_fast, cudaStream_t s, int* err) {
   auto kern = gemm_tc_kernel<BN, STAGES, A_MN, B_MN, EPI>;
   constexpr size_t smem = smem_bytes<BN, STAGES>();
+  static_assert(smem <= 232448, "shared memory budget");
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -457,20 +621,21 @@ static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const Ep
   const int tiles_n = (ep.N + BN - 1) / BN;
   const int units = tiles_m * tiles_n * splits;
   const int grid = units < num_sms() ? units : num_sms();
-  kern<<<grid, kThreads, smem, s>>>(ta, tb, ep, K, tiles_m, tiles_n, splits, kb_per_split, n_fast,
-                                    vec_ok, split_stride, err);
+  kern<<<grid, kThreads, smem, s>>>(ta, tb, to, tx, ep, K, tiles_m, tiles_n, splits, kb_per_split,
+                                    n_fast, err);
   note_launch();
   return cudaGetLastError();
 }
 
 template <int BN, int STAGES>
 static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb,
-                            const EpiParams& ep, int epi, int splits, int kb_per_split, int n_fast,
-                            int vec_ok, long split_stride, cudaStream_t s, int* err) {
-#define GPT2_TC(AM, BMJ, E)                                                                     \
-  if (a.a_mn == AM && a.b_mn == BMJ && epi == E)                                                \
-    return launch<BN, STAGES, AM, BMJ, E>(ta, tb, ep, a.K, splits, kb_per_split, n_fast, vec_ok, \
-                                          split_stride, s, err);
+                            const CUtensorMap& to, const CUtensorMap& tx, const EpiParams& ep,
+                            int epi, int splits, int kb_per_split, int n_fast, cudaStream_t s,
+                            int* err) {
+#define GPT2_TC(AM, BMJ, E)                                                                      \
+  if (a.a_mn == AM && a.b_mn == BMJ && epi == E)                                                 \
+    return launch<BN, STAGES, AM, BMJ, E>(ta, tb, to, tx, ep, a.K, splits, kb_per_split, n_fast, \
+                                          s, err);
   GPT2_TC(0, 0, EPI_STORE)
   GPT2_TC(0, 0, EPI_BIAS)
   GPT2_TC(0, 0, EPI_BIAS_GELU)
@@ -480,7 +645,6 @@ static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUte
   GPT2_TC(1, 1, EPI_F32_ACC)
   GPT2_TC(1, 1, EPI_F32_STORE)
   GPT2_TC(1, 0, EPI_STORE)
-  GPT2_TC(0, 0, EPI_F32_STORE)
 #undef GPT2_TC
   return cudaErrorInvalidValue;
 }
@@ -490,6 +654,21 @@ static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUte
 __global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, int splits, int M,
                                      int N) {
   const size_t total = (size_t)M * N;
+  if (ldo32 == N && (total & 3) == 0) {  // contiguous output: float4 path
+    const size_t t4 = total / 4;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < t4;
+         i += (size_t)gridDim.x * blockDim.x) {
+      float4 s = reinterpret_cast<const float4*>(ws)[i];
+      for (int k = 1; k < splits; ++k) {
+        const float4 w = reinterpret_cast<const float4*>(ws + (size_t)k * total)[i];
+        s.x += w.x; s.y += w.y; s.z += w.z; s.w += w.w;
+      }
+      float4 o = reinterpret_cast<float4*>(out32)[i];
+      o.x += s.x; o.y += s.y; o.z += s.z; o.w += s.w;
+      reinterpret_cast<float4*>(out32)[i] = o;
+    }
+    return;
+  }
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {
     const int m = (int)(i / N), n = (int)(i % N);
@@ -499,65 +678,89 @@ __global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, 
   }
 }
 
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   using namespace tc;
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return cudaSuccess;
-  // TMA: 16-byte aligned bases and row strides.
-  if ((reinterpret_cast<uintptr_t>(a.A) & 15) || (reinterpret_cast<uintptr_t>(a.B) & 15) ||
-      (a.lda % 8) || (a.ldb % 8))
+  // TMA: 16-byte aligned bases and row strides for every operand and output
+  if (!aligned16(a.A) || !aligned16(a.B) || (a.lda % 8) || (a.ldb % 8)) return cudaErrorInvalidValue;
+  const bool f32_out = a.epi == EPI_F32_ACC || a.epi == EPI_F32_STORE;
+  if (f32_out ? (!a.out32 || !aligned16(a.out32) || (a.ldo32 % 4))
+              : (!a.out || !aligned16(a.out) || (a.ldo % 8)))
     return cudaErrorInvalidValue;
+  if (a.epi == EPI_BIAS_RESID && (!a.resid || !aligned16(a.resid) || (a.ldr % 8)))
+    return cudaErrorInvalidValue;
+  if ((a.epi == EPI_BIAS_GELU || a.epi == EPI_DGELU) && (!a.aux || !aligned16(a.aux) || (a.ldaux % 8)))
+    return cudaErrorInvalidValue;
+  if (a.bias && !aligned16(a.bias)) return cudaErrorInvalidValue;
   const int BN = a.N >= 256 ? 256 : 128;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, to, tx;
+  std::memset(&to, 0, sizeof(to));
+  std::memset(&tx, 0, sizeof(tx));
   cudaError_t e;
-  if (!a.a_mn) e = make_tmap(&ta, a.A, a.K, a.M, a.lda, BM);
-  else e = make_tmap(&ta, a.A, a.M, a.K, a.lda, 64);
+  if (!a.a_mn) e = make_tmap(&ta, a.A, false, a.K, a.M, a.lda, 64, BM);
+  else e = make_tmap(&ta, a.A, false, a.M, a.K, a.lda, 64, 64);
   if (e != cudaSuccess) return e;
-  if (!a.b_mn) e = make_tmap(&tb, a.B, a.K, a.N, a.ldb, BN);
-  else e = make_tmap(&tb, a.B, a.N, a.K, a.ldb, 64);
+  if (!a.b_mn) e = make_tmap(&tb, a.B, false, a.K, a.N, a.ldb, 64, BN);
+  else e = make_tmap(&tb, a.B, false, a.N, a.K, a.ldb, 64, 64);
   if (e != cudaSuccess) return e;
 
   EpiParams ep{a.M, a.N, a.alpha, a.out, a.ldo, a.out32, a.ldo32, a.bias, a.resid, a.ldr, a.aux, a.ldaux};
   const int tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
   const int kb_total = (a.K + BK - 1) / BK;
 
-  // split-K for the weight-gradient products with few output tiles
+  // split-K for the weight-gradient products with few output tiles: pick the
+  // split count with the lowest estimated time = whole waves of units at
+  // ~8.5 TFLOP/s per SM + the partials' write/read and the output update
+  // at ~6 TB/s (at least 4 k-blocks per split; partials must fit)
   int splits = 1;
   int epi = a.epi;
-  if (a.epi == EPI_F32_ACC && a.max_splits > 1 && a.split_ws) {
-    const int want = (num_sms() + tiles - 1) / tiles;
-    splits = want < a.max_splits ? want : a.max_splits;
-    if (splits > kb_total / 4) splits = kb_total / 4;
-    while (splits > 1 && (size_t)splits * a.M * a.N > a.split_ws_floats) --splits;
-    if (splits < 1) splits = 1;
+  if (a.epi == EPI_F32_ACC && a.max_splits > 1 && a.split_ws && tiles < num_sms() &&
+      aligned16(a.split_ws) && a.N % 4 == 0) {
+    double best = 1e30;
+    const double out_bytes = 4.0 * a.M * a.N;
+    for (int sp = 1; sp <= a.max_splits; ++sp) {
+      if (sp > 1 && (sp > kb_total / 4 || (size_t)sp * a.M * a.N > a.split_ws_floats)) break;
+      const int waves = (tiles * sp + num_sms() - 1) / num_sms();
+      const double t_unit = 2.0 * BM * BN * ((double)kb_total * BK / sp) / 8.5e12;
+      const double t_red = sp > 1 ? (2.0 * sp + 2.0) * out_bytes / 6.0e12 : 0.0;
+      const double t = waves * t_unit + t_red;
+      if (t < best * 0.98) {
+        best = t;
+        splits = sp;
+      }
+    }
   }
   int kb_per_split = (kb_total + splits - 1) / splits;
   splits = (kb_total + kb_per_split - 1) / kb_per_split;  // no empty split
-  long split_stride = 0;
+  // epilogue tensor maps
   if (splits > 1) {
     epi = EPI_F32_STORE;
-    ep.out32 = a.split_ws;
-    ep.ldo32 = a.N;
-    ep.alpha = a.alpha;
-    split_stride = (long)a.M * a.N;
+    e = make_tmap(&to, a.split_ws, true, a.N, a.M, a.N, 32, BM, splits, (uint64_t)a.M * a.N);
+  } else if (f32_out) {
+    e = make_tmap(&to, a.out32, true, a.N, a.M, a.ldo32, 32, BM, 1);
+  } else {
+    e = make_tmap(&to, a.out, false, a.N, a.M, a.ldo, 64, BM, 1);
   }
+  if (e != cudaSuccess) return e;
+  if (a.epi == EPI_BIAS_RESID) e = make_tmap(&tx, a.resid, false, a.N, a.M, a.ldr, 64, BM, 1);
+  else if (a.epi == EPI_BIAS_GELU || a.epi == EPI_DGELU)
+    e = make_tmap(&tx, a.aux, false, a.N, a.M, a.ldaux, 64, BM, 1);
+  if (e != cudaSuccess) return e;
   // The larger operand is reused by consecutive tiles (L2 locality).
   const double a_bytes = (double)a.M * a.K, b_bytes = (double)a.N * a.K;
   const int n_fast = a_bytes > b_bytes ? 1 : 0;
-  const int vec_ok = (ep.ldo % 8 == 0) && (ep.ldo32 % 4 == 0) && (ep.ldr % 8 == 0) &&
-                     (ep.ldaux % 8 == 0) && ((reinterpret_cast<uintptr_t>(ep.out) & 15) == 0) &&
-                     ((reinterpret_cast<uintptr_t>(ep.out32) & 15) == 0) &&
-                     ((reinterpret_cast<uintptr_t>(ep.resid) & 15) == 0) &&
-                     ((reinterpret_cast<uintptr_t>(ep.aux) & 15) == 0) &&
-                     ((reinterpret_cast<uintptr_t>(ep.bias) & 15) == 0);
   if (BN == 256)
-    e = dispatch<256, 4>(a, ta, tb, ep, epi, splits, kb_per_split, n_fast, vec_ok, split_stride, s, err);
+    e = dispatch<256, 4>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
   else
-    e = dispatch<128, 6>(a, ta, tb, ep, epi, splits, kb_per_split, n_fast, vec_ok, split_stride, s, err);
+    e = dispatch<128, 6>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
   if (e != cudaSuccess) return e;
   if (splits > 1) {
     const size_t total = (size_t)a.M * a.N;
-    int blocks = (int)((total + 255) / 256);
+    int blocks = (int)((total / 4 + 255) / 256);
     if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
+    if (blocks < 1) blocks = 1;
     splitk_reduce_kernel<<<blocks, 256, 0, s>>>(a.out32, a.ldo32, a.split_ws, splits, a.M, a.N);
     note_launch();
     e = cudaGetLastError();

@@ -45,8 +45,8 @@ constexpr int kMaxSplits = 8;
 
 // Optional per-kernel-family timing with CUDA events on the handle's stream.
 enum ProfKind {
-  PK_GEMM, PK_ATTN_FWD, PK_ATTN_BWD, PK_LAYERNORM, PK_CLASSIFIER, PK_ENCODER, PK_COLSUM,
-  PK_OPTIMIZER, PK_COUNT
+  PK_GEMM, PK_ATTN_FWD, PK_ATTN_BWD, PK_LAYERNORM, PK_LN_BWD, PK_CLASSIFIER, PK_ENCODER,
+  PK_COLSUM, PK_OPTIMIZER, PK_COUNT
 };
 
 struct ProfRec {
@@ -156,7 +156,7 @@ size_t carve_work(const Layout& lay, int B, int T, void* base, Acts* a) {
   x.dqkv = c.take<act_t>(M * 3 * C);
   x.dbig = c.take<act_t>(M * 4 * C);
   x.dsum = c.take<float>(M * H);
-  const size_t part = std::max((size_t)kColsumChunks * 4 * C, (size_t)kLnBlocks * 2 * C);
+  const size_t part = std::max((size_t)kColsumChunks * 4 * C, (size_t)kLnBlocks * 3 * C);
   x.partials = c.take<float>(part);
   x.splitk_floats = (size_t)kMaxSplits * 4 * C * C;
   x.splitk = c.take<float>(x.splitk_floats);
@@ -508,9 +508,11 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
     GPT2_TRY(run_gemm(h, ga));
   }
-  mark(h, PK_LAYERNORM);
+  mark(h, PK_LN_BWD);
+  // dres = d x_L; its column sum is the bias gradient of the last W_p
   layernorm_bwd(a.dres, a.dh, a.res + (size_t)L * MC, a.meanf, a.rstdf, P + y.off[T_LNFG],
-                G + y.off[T_LNFG], G + y.off[T_LNFB], a.partials, M, C, 0, s);
+                G + y.off[T_LNFG], G + y.off[T_LNFB], G + y.off[T_BP] + (size_t)(L - 1) * C,
+                a.partials, M, C, 0, s);
 
   for (int l = L - 1; l >= 0; --l) {
     const act_t* x = a.res + (size_t)l * MC;
@@ -539,8 +541,6 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
       GPT2_TRY(run_gemm(h, ga));
     }
-    mark(h, PK_COLSUM);
-    colsum_acc(G + y.off[T_BP] + (size_t)l * C, a.dres, M, C, a.partials, s);
     {  // dh = du Wfc
       GemmArgs ga = gemm_args(M, C, 4 * C);
       ga.A = a.dbig; ga.lda = 4 * C;
@@ -560,10 +560,12 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     }
     mark(h, PK_COLSUM);
     colsum_acc(G + y.off[T_BFC] + (size_t)l * 4 * C, a.dbig, M, 4 * C, a.partials, s);
-    mark(h, PK_LAYERNORM);
+    mark(h, PK_LN_BWD);
+    // dres = d x_mid; its column sum is the bias gradient of W_o
     layernorm_bwd(a.dres, a.dh, xm, a.mean2 + (size_t)l * M, a.rstd2 + (size_t)l * M,
                   P + y.off[T_LN2G] + (size_t)l * C, G + y.off[T_LN2G] + (size_t)l * C,
-                  G + y.off[T_LN2B] + (size_t)l * C, a.partials, M, C, 1, s);
+                  G + y.off[T_LN2B] + (size_t)l * C, G + y.off[T_BO] + (size_t)l * C,
+                  a.partials, M, C, 1, s);
     // ---- attention: xm = x + att Wo^T + bo
     {  // datt = dres Wo
       GemmArgs ga = gemm_args(M, C, C);
@@ -582,8 +584,6 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
       GPT2_TRY(run_gemm(h, ga));
     }
-    mark(h, PK_COLSUM);
-    colsum_acc(G + y.off[T_BO] + (size_t)l * C, a.dres, M, C, a.partials, s);
     mark(h, PK_ATTN_BWD, 10.0 * B * H * (double)T * (T + 1) / 2 * (C / H));
     GPT2_CUDA(h, attention_bwd(a.dqkv, a.dsum, a.datt, qkv, att, a.lse + (size_t)l * M * H, B, T,
                                C, H, s));
@@ -606,10 +606,12 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     }
     mark(h, PK_COLSUM);
     colsum_acc(G + y.off[T_BQKV] + (size_t)l * 3 * C, a.dqkv, M, 3 * C, a.partials, s);
-    mark(h, PK_LAYERNORM);
+    mark(h, PK_LN_BWD);
+    // dres = d x_l = gradient at the output of layer l-1: bias of its W_p
     layernorm_bwd(a.dres, a.dh, x, a.mean1 + (size_t)l * M, a.rstd1 + (size_t)l * M,
                   P + y.off[T_LN1G] + (size_t)l * C, G + y.off[T_LN1G] + (size_t)l * C,
-                  G + y.off[T_LN1B] + (size_t)l * C, a.partials, M, C, 1, s);
+                  G + y.off[T_LN1B] + (size_t)l * C,
+                  l > 0 ? G + y.off[T_BP] + (size_t)(l - 1) * C : nullptr, a.partials, M, C, 1, s);
   }
   mark(h, PK_ENCODER);
   encoder_bwd(G + y.off[T_WTE], G + y.off[T_WPE], a.dres, a.tok, B, T, C, y.Vp, es, s);

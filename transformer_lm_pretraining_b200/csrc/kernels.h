@@ -78,14 +78,16 @@ void encoder_bwd(float* dwte, float* dwpe, const act_t* dx0, const int* tok_save
 void layernorm_fwd(act_t* y, float* mean, float* rstd, const act_t* x, const float* g,
                    const float* b, int M, int C, cudaStream_t s);
 // dres = (accumulate ? dres : 0) + LN backward of dy;  dg, db += column sums
-// (per-block partials in `partials` [kLnBlocks * 2C], reduced in fixed order).
-constexpr int kLnBlocks = 296;
+// of dy * xhat and dy; dbias_out (may be null) += column sums of the written
+// dres.  Per-block partials in `partials` [kLnBlocks * 3C], reduced in a
+// fixed order.
+constexpr int kLnBlocks = 592;
 void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
-                   const float* rstd, const float* g, float* dg, float* db, float* partials,
-                   int M, int C, int accumulate, cudaStream_t s);
+                   const float* rstd, const float* g, float* dg, float* db, float* dbias_out,
+                   float* partials, int M, int C, int accumulate, cudaStream_t s);
 
 // ------------------------------------------------------------ column sums --
-constexpr int kColsumChunks = 128;
+constexpr int kColsumChunks = 192;
 // db[n] += sum_m dy[m, n] (fixed order); partials: [kColsumChunks * N] floats
 void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s);
 

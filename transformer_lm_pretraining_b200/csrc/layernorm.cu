@@ -1,8 +1,11 @@
 // LayerNorm forward and backward: one warp per row, 16-byte vector loads,
-// fp32 statistics (biased variance, eps = 1e-5).  The backward's dgamma /
-// dbeta column sums are accumulated per warp in registers over a fixed row
-// assignment, reduced per block in warp order, and summed over blocks in
-// block order: no atomics, fixed summation order.
+// fp32 statistics (biased variance, eps = 1e-5).
+//
+// The backward's column sums -- dgamma, dbeta and, optionally, the column
+// sum of the residual gradient it writes (the bias gradient of the
+// projection that produced that residual) -- are accumulated per warp in
+// registers over a fixed row assignment, reduced per block in warp order,
+// and summed over blocks in block order: no atomics, fixed summation order.
 
 #include "kernels.h"
 
@@ -12,20 +15,20 @@ namespace {
 
 constexpr float kLnEps = 1e-5f;
 
-// kMaxChunks = ceil(C / 256): the 8-element chunks each lane owns.
-template <int kMaxChunks>
-__global__ void ln_fwd_kernel(act_t* __restrict__ y, float* __restrict__ mean,
-                              float* __restrict__ rstd, const act_t* __restrict__ x,
-                              const float* __restrict__ g, const float* __restrict__ b, int M,
-                              int C) {
+// kChunks = ceil(C / 256): the 8-element chunks each lane owns.
+template <int kChunks>
+__global__ void __launch_bounds__(256)
+    ln_fwd_kernel(act_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
+                  const act_t* __restrict__ x, const float* __restrict__ g,
+                  const float* __restrict__ b, int M, int C) {
   const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (row >= M) return;
   const int lane = threadIdx.x & 31;
   const act_t* xr = x + (size_t)row * C;
-  float v[kMaxChunks][8];
+  float v[kChunks][8];
   float s = 0.f;
 #pragma unroll
-  for (int k = 0; k < kMaxChunks; ++k) {
+  for (int k = 0; k < kChunks; ++k) {
     const int c = (k * 32 + lane) * 8;
     if (c < C) {
       load8(xr + c, v[k]);
@@ -36,7 +39,7 @@ __global__ void ln_fwd_kernel(act_t* __restrict__ y, float* __restrict__ mean,
   const float mu = warp_sum(s) / C;
   float q = 0.f;
 #pragma unroll
-  for (int k = 0; k < kMaxChunks; ++k) {
+  for (int k = 0; k < kChunks; ++k) {
     const int c = (k * 32 + lane) * 8;
     if (c < C) {
 #pragma unroll
@@ -49,12 +52,14 @@ __global__ void ln_fwd_kernel(act_t* __restrict__ y, float* __restrict__ mean,
   const float rs = rsqrtf(warp_sum(q) / C + kLnEps);
   act_t* yr = y + (size_t)row * C;
 #pragma unroll
-  for (int k = 0; k < kMaxChunks; ++k) {
+  for (int k = 0; k < kChunks; ++k) {
     const int c = (k * 32 + lane) * 8;
     if (c < C) {
-      float o[8];
+      float gg[8], bb[8], o[8];
+      load8(g + c, gg);
+      load8(b + c, bb);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = (v[k][i] - mu) * rs * g[c + i] + b[c + i];
+      for (int i = 0; i < 8; ++i) o[i] = (v[k][i] - mu) * rs * gg[i] + bb[i];
       store8(yr + c, o);
     }
   }
@@ -65,99 +70,141 @@ __global__ void ln_fwd_kernel(act_t* __restrict__ y, float* __restrict__ mean,
 }
 
 // grid = kLnBlocks blocks of 8 warps; warp w of block blk handles rows
-// (blk * 8 + w) + k * (kLnBlocks * 8).  partials[blk][0..C) = dgamma,
-// partials[blk][C..2C) = dbeta.
-template <int kMaxChunks>
+// (blk * 8 + w) + k * (kLnBlocks * 8).  partials[blk][0][..C) = dgamma,
+// [1] = dbeta, [2] = column sums of the written dres (when NSUMS == 3).
+template <int kChunks, int NSUMS>
 __global__ void __launch_bounds__(256)
     ln_bwd_kernel(act_t* __restrict__ dres, const act_t* __restrict__ dy,
                   const act_t* __restrict__ x, const float* __restrict__ mean,
                   const float* __restrict__ rstd, const float* __restrict__ g,
                   float* __restrict__ partials, int M, int C, int accumulate) {
-  extern __shared__ float red[];  // [8 warps][2C]
+  extern __shared__ float red[];  // [8 warps][C]
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nw = blockDim.x / 32;
-  float dg[kMaxChunks][8], db[kMaxChunks][8], gv[kMaxChunks][8];
+  float acc[NSUMS][kChunks][8], gv[kChunks][8];
 #pragma unroll
-  for (int k = 0; k < kMaxChunks; ++k)
+  for (int k = 0; k < kChunks; ++k) {
+    const int c = (k * 32 + lane) * 8;
+    if (c < C) load8(g + c, gv[k]);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      dg[k][i] = 0.f;
-      db[k][i] = 0.f;
-      const int c = (k * 32 + lane) * 8 + i;
-      gv[k][i] = c < C ? g[c] : 0.f;
+      if (c >= C) gv[k][i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < NSUMS; ++j) acc[j][k][i] = 0.f;
     }
+  }
   for (int row = blockIdx.x * nw + warp; row < M; row += gridDim.x * nw) {
     const act_t* xr = x + (size_t)row * C;
     const act_t* dyr = dy + (size_t)row * C;
+    act_t* dr = dres + (size_t)row * C;
     const float mu = mean[row], rs = rstd[row];
-    float xh[kMaxChunks][8], dxh[kMaxChunks][8];
-    float a = 0.f, bsum = 0.f;
+    float xv[kChunks][8], dv[kChunks][8], ov[kChunks][8];
 #pragma unroll
-    for (int k = 0; k < kMaxChunks; ++k) {
+    for (int k = 0; k < kChunks; ++k) {
       const int c = (k * 32 + lane) * 8;
       if (c < C) {
-        float xv[8], dv[8];
-        load8(xr + c, xv);
-        load8(dyr + c, dv);
+        load8(xr + c, xv[k]);
+        load8(dyr + c, dv[k]);
+        if (accumulate) load8(dr + c, ov[k]);
+      }
+    }
+    float a = 0.f, bsum = 0.f;
+#pragma unroll
+    for (int k = 0; k < kChunks; ++k) {
+      const int c = (k * 32 + lane) * 8;
+      if (c < C) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          xh[k][i] = (xv[i] - mu) * rs;
-          dxh[k][i] = dv[i] * gv[k][i];
-          a += dxh[k][i];
-          bsum += dxh[k][i] * xh[k][i];
-          dg[k][i] += dv[i] * xh[k][i];
-          db[k][i] += dv[i];
+          const float xh = (xv[k][i] - mu) * rs;
+          const float dxh = dv[k][i] * gv[k][i];
+          a += dxh;
+          bsum += dxh * xh;
+          acc[0][k][i] += dv[k][i] * xh;
+          acc[1][k][i] += dv[k][i];
+          xv[k][i] = xh;
+          dv[k][i] = dxh;
         }
       }
     }
     a = warp_sum(a) / C;
     bsum = warp_sum(bsum) / C;
-    act_t* dr = dres + (size_t)row * C;
 #pragma unroll
-    for (int k = 0; k < kMaxChunks; ++k) {
+    for (int k = 0; k < kChunks; ++k) {
       const int c = (k * 32 + lane) * 8;
       if (c < C) {
         float o[8];
-        if (accumulate) load8(dr + c, o);
-        else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = 0.f;
+        for (int i = 0; i < 8; ++i)
+          o[i] = (accumulate ? ov[k][i] : 0.f) + rs * (dv[k][i] - a - xv[k][i] * bsum);
+        if (NSUMS == 3) {
+          // the bias gradient sums the values as stored (activation dtype)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[NSUMS - 1][k][i] += to_f(from_f<act_t>(o[i]));
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] += rs * (dxh[k][i] - a - xh[k][i] * bsum);
         store8(dr + c, o);
       }
     }
   }
-  // block reduction of the column partials in warp order
+  // block reduction of each column sum in warp order, one sum at a time
 #pragma unroll
-  for (int k = 0; k < kMaxChunks; ++k) {
-    const int c = (k * 32 + lane) * 8;
-    if (c < C) {
+  for (int j = 0; j < NSUMS; ++j) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        red[(size_t)warp * 2 * C + c + i] = dg[k][i];
-        red[(size_t)warp * 2 * C + C + c + i] = db[k][i];
+    for (int k = 0; k < kChunks; ++k) {
+      const int c = (k * 32 + lane) * 8;
+      if (c < C) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[(size_t)warp * C + c + i] = acc[j][k][i];
       }
     }
-  }
-  __syncthreads();
-  for (int j = threadIdx.x; j < 2 * C; j += blockDim.x) {
-    float s = 0.f;
-    for (int w = 0; w < nw; ++w) s += red[(size_t)w * 2 * C + j];
-    partials[(size_t)blockIdx.x * 2 * C + j] = s;
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      float s = 0.f;
+      for (int w = 0; w < nw; ++w) s += red[(size_t)w * C + c];
+      partials[((size_t)blockIdx.x * NSUMS + j) * C + c] = s;
+    }
+    __syncthreads();
   }
 }
 
-// dg[c] += sum_blk partials[blk][c]; db[c] += sum_blk partials[blk][C + c]
+// out_j[c] += sum over blocks (in order) of partials[blk][j][c]: thread
+// (tx, ty) takes column tx of a 32-column group and blocks ty, ty+8, ...;
+// the 8 partial sums are then added in ty order.
 __global__ void ln_bwd_reduce_kernel(float* __restrict__ dg, float* __restrict__ db,
-                                     const float* __restrict__ partials, int nblk, int C) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= 2 * C) return;
+                                     float* __restrict__ dsum3,
+                                     const float* __restrict__ partials, int nblk, int nsums,
+                                     int C) {
+  __shared__ float red[8][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int col = blockIdx.x * 32 + tx;  // over nsums * C
   float s = 0.f;
-  for (int b = 0; b < nblk; ++b) s += partials[(size_t)b * 2 * C + j];
-  if (j < C) dg[j] += s;
-  else db[j - C] += s;
+  if (col < nsums * C) {
+    const int j = col / C, c = col % C;
+    for (int b = ty; b < nblk; b += 8) s += partials[((size_t)b * nsums + j) * C + c];
+  }
+  red[ty][tx] = s;
+  __syncthreads();
+  if (ty == 0 && col < nsums * C) {
+    float t = 0.f;
+    for (int k = 0; k < 8; ++k) t += red[k][tx];
+    const int j = col / C, c = col % C;
+    float* dst = j == 0 ? dg : (j == 1 ? db : dsum3);
+    dst[c] += t;
+  }
+}
+
+template <int N, int S>
+void ln_bwd_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
+                   const float* rstd, const float* g, float* partials, int M, int C,
+                   int accumulate, cudaStream_t s) {
+  const size_t smem = (size_t)8 * C * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(ln_bwd_kernel<N, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         8 * 2048 * 4);
+    attr = true;
+  }
+  ln_bwd_kernel<N, S><<<kLnBlocks, 256, smem, s>>>(dres, dy, x, mean, rstd, g, partials, M, C,
+                                                   accumulate);
 }
 
 }  // namespace
@@ -176,30 +223,24 @@ void layernorm_fwd(act_t* y, float* mean, float* rstd, const act_t* x, const flo
   note_launch();
 }
 
-template <int N>
-static void ln_bwd_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
-                          const float* rstd, const float* g, float* partials, int M, int C,
-                          int accumulate, cudaStream_t s) {
-  const size_t smem = (size_t)8 * 2 * C * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(ln_bwd_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * 2 * 2048 * 4);
-    attr = true;
-  }
-  ln_bwd_kernel<N><<<kLnBlocks, 256, smem, s>>>(dres, dy, x, mean, rstd, g, partials, M, C, accumulate);
-}
-
 void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
-                   const float* rstd, const float* g, float* dg, float* db, float* partials,
-                   int M, int C, int accumulate, cudaStream_t s) {
-  switch ((C + 255) / 256) {
-#define GPT2_LNB(N) \
-  case N: ln_bwd_launch<N>(dres, dy, x, mean, rstd, g, partials, M, C, accumulate, s); break;
+                   const float* rstd, const float* g, float* dg, float* db, float* dbias_out,
+                   float* partials, int M, int C, int accumulate, cudaStream_t s) {
+  const int nsums = dbias_out ? 3 : 2;
+  switch ((C + 255) / 256 * 4 + nsums) {
+#define GPT2_LNB(N)                                                                          \
+  case 4 * N + 2:                                                                            \
+    ln_bwd_launch<N, 2>(dres, dy, x, mean, rstd, g, partials, M, C, accumulate, s);          \
+    break;                                                                                   \
+  case 4 * N + 3:                                                                            \
+    ln_bwd_launch<N, 3>(dres, dy, x, mean, rstd, g, partials, M, C, accumulate, s);          \
+    break;
     GPT2_LNB(1) GPT2_LNB(2) GPT2_LNB(3) GPT2_LNB(4) GPT2_LNB(5) GPT2_LNB(6) GPT2_LNB(7) GPT2_LNB(8)
 #undef GPT2_LNB
     default: break;
   }
-  ln_bwd_reduce_kernel<<<(2 * C + 255) / 256, 256, 0, s>>>(dg, db, partials, kLnBlocks, C);
+  ln_bwd_reduce_kernel<<<(nsums * C + 31) / 32, 256, 0, s>>>(dg, db, dbias_out, partials,
+                                                              kLnBlocks, nsums, C);
   note_launch(2);
 }
 

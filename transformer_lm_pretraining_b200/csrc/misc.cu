@@ -48,43 +48,65 @@ bool tensor_decayed(int t) {
 namespace {
 
 // ------------------------------------------------------------ colsum --
-// partials[chunk][n] = sum over the chunk's rows (ascending) of dy[m, n];
-// block = 32 x 8 threads, 64 columns (2 per thread).
-__global__ void colsum_partial_kernel(float* __restrict__ partials, const act_t* __restrict__ dy,
-                                      int M, int N, int rows_per_chunk) {
-  __shared__ float red[8][64];
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int n = blockIdx.x * 64 + 2 * tx;
+// partials[chunk][n] = sum over the chunk's rows of dy[m, n] (row set of
+// warp w: r0 + w, r0 + w + 8, ...; then the 8 warps in order).  A warp
+// covers 256 columns, 8 per lane (16-byte loads); N % 8 == 0.
+__global__ void __launch_bounds__(256)
+    colsum_partial_kernel(float* __restrict__ partials, const act_t* __restrict__ dy, int M, int N,
+                          int rows_per_chunk) {
+  __shared__ float red[8][256];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int n = blockIdx.x * 256 + lane * 8;
   const int r0 = blockIdx.y * rows_per_chunk;
   const int r1 = min(M, r0 + rows_per_chunk);
-  float s0 = 0.f, s1 = 0.f;
+  float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (n < N) {
-    for (int r = r0 + ty; r < r1; r += 8) {
-      const act_t* p = dy + (size_t)r * N + n;
-      s0 += to_f(p[0]);
-      if (n + 1 < N) s1 += to_f(p[1]);
+    int r = r0 + w;
+    for (; r + 24 < r1; r += 32) {  // four rows in flight
+      float a[8], b[8], c[8], d[8];
+      load8(dy + (size_t)r * N + n, a);
+      load8(dy + (size_t)(r + 8) * N + n, b);
+      load8(dy + (size_t)(r + 16) * N + n, c);
+      load8(dy + (size_t)(r + 24) * N + n, d);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[i] = (((s[i] + a[i]) + b[i]) + c[i]) + d[i];
+    }
+    for (; r < r1; r += 8) {
+      float a[8];
+      load8(dy + (size_t)r * N + n, a);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[i] += a[i];
     }
   }
-  red[ty][2 * tx] = s0;
-  red[ty][2 * tx + 1] = s1;
-  __syncthreads();
-  if (ty == 0) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      float s = 0.f;
-      for (int k = 0; k < 8; ++k) s += red[k][2 * tx + j];
-      if (n + j < N) partials[(size_t)blockIdx.y * N + n + j] = s;
-    }
+  for (int i = 0; i < 8; ++i) red[w][lane * 8 + i] = s[i];
+  __syncthreads();
+  const int col = blockIdx.x * 256 + threadIdx.x;
+  if (col < N) {
+    float t = 0.f;
+    for (int k = 0; k < 8; ++k) t += red[k][threadIdx.x];
+    partials[(size_t)blockIdx.y * N + col] = t;
   }
 }
 
+// db[n] += sum over chunks (in order) of partials[chunk][n]: thread (tx, ty)
+// takes column tx of a 32-column group and chunks ty, ty+8, ...; the 8
+// partial sums are added in ty order.
 __global__ void colsum_reduce_kernel(float* __restrict__ db, const float* __restrict__ partials,
                                      int chunks, int N) {
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
+  __shared__ float red[8][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int n = blockIdx.x * 32 + tx;
   float s = 0.f;
-  for (int c = 0; c < chunks; ++c) s += partials[(size_t)c * N + n];
-  db[n] += s;
+  if (n < N)
+    for (int c = ty; c < chunks; c += 8) s += partials[(size_t)c * N + n];
+  red[ty][tx] = s;
+  __syncthreads();
+  if (ty == 0 && n < N) {
+    float t = 0.f;
+    for (int k = 0; k < 8; ++k) t += red[k][tx];
+    db[n] += t;
+  }
 }
 
 // -------------------------------------------------------- classifier --
@@ -341,11 +363,15 @@ int grid_for(size_t n, int threads, int max_blocks) {
 }  // namespace
 
 void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s) {
-  const int rows = (M + kColsumChunks - 1) / kColsumChunks;
+  // enough chunks for ~4 blocks per SM
+  const int colgroups = (N + 255) / 256;
+  int want = (4 * kNumSMs + colgroups - 1) / colgroups;
+  if (want > kColsumChunks) want = kColsumChunks;
+  const int rows = (M + want - 1) / want;
   const int chunks = (M + rows - 1) / rows;
-  dim3 g((N + 63) / 64, chunks);
+  dim3 g(colgroups, chunks);
   colsum_partial_kernel<<<g, 256, 0, s>>>(partials, dy, M, N, rows);
-  colsum_reduce_kernel<<<(N + 255) / 256, 256, 0, s>>>(db, partials, chunks, N);
+  colsum_reduce_kernel<<<(N + 31) / 32, 256, 0, s>>>(db, partials, chunks, N);
   note_launch(2);
 }
 

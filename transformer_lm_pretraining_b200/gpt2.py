@@ -26,8 +26,8 @@ ACT_NAMES = {"residual": 0, "ln1": 1, "qkv": 2, "attn": 3, "xmid": 4, "ln2": 5,
 
 EPI = {"store": 0, "bias": 1, "bias_gelu": 2, "bias_resid": 3, "dgelu": 4, "f32_acc": 5}
 
-PROF_KINDS = ("gemm", "attn_fwd", "attn_bwd", "layernorm", "classifier", "encoder", "colsum",
-              "optimizer")
+PROF_KINDS = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "classifier", "encoder",
+              "colsum", "optimizer")
 
 # name -> (restype, argtypes)
 _vp, _sz, _i, _f, _d, _l, _u64 = (ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float,
