@@ -621,12 +621,12 @@ __global__ void naive_bwd_dkdv_kernel(float* __restrict__ dqkv, const float* __r
 }  // namespace
 
 cudaError_t attention_fwd(act_t* att, float* lse, const act_t* qkv, int B, int T, int C, int H,
-                          cudaStream_t s) {
+                          int* err, cudaStream_t s) {
   const int hd = C / H;
 #if GPT2_ACT_BF16
   switch (hd) {
     case 32: return fwd_launch<32>(att, lse, qkv, B, T, C, H, s);
-    case 64: return fwd_launch<64>(att, lse, qkv, B, T, C, H, s);
+    case 64: return attention_fwd_tc(att, lse, qkv, B, T, C, H, err, s);  // tcgen05
     case 128: return fwd_launch<128>(att, lse, qkv, B, T, C, H, s);
     default: return cudaErrorInvalidValue;
   }

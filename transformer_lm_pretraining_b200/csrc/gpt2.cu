@@ -395,7 +395,7 @@ gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int 
       GPT2_TRY(run_gemm(h, ga));
     }
     mark(h, PK_ATTN_FWD, 4.0 * B * H * (double)T * (T + 1) / 2 * (C / H));
-    GPT2_CUDA(h, attention_fwd(att, a.lse + (size_t)l * M * H, qkv, B, T, C, H, s));
+    GPT2_CUDA(h, attention_fwd(att, a.lse + (size_t)l * M * H, qkv, B, T, C, H, h->err, s));
     {  // xmid = x + att W_o^T + b_o
       GemmArgs ga = gemm_args(M, C, C);
       ga.A = att; ga.lda = C;

@@ -48,8 +48,10 @@ int gpt2k_gemm(void* stream, int epi, int M, int N, int K, const void* A, long l
 int gpt2k_attention_fwd(void* stream, void* att, float* lse, const void* qkv, int B, int T, int C,
                         int H) {
   if (B < 1 || T < 1 || H < 1 || C % H) return GPT2_ERR_ARG;
+  int* err = err_word();
+  if (!err) return GPT2_ERR_CUDA;
   return status(attention_fwd(static_cast<act_t*>(att), lse, static_cast<const act_t*>(qkv), B, T,
-                              C, H, static_cast<cudaStream_t>(stream)));
+                              C, H, err, static_cast<cudaStream_t>(stream)));
 }
 
 int gpt2k_attention_bwd(void* stream, void* dqkv, float* dsum, const void* datt, const void* qkv,

@@ -95,7 +95,11 @@ void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaS
 // qkv [B*T, 3C] = [q | k | v], head h at columns h*hd..; att [B*T, C];
 // lse [B, H, T] (natural log).
 cudaError_t attention_fwd(act_t* att, float* lse, const act_t* qkv, int B, int T, int C, int H,
-                          cudaStream_t s);
+                          int* err, cudaStream_t s);
+// tcgen05 forward (head dim 64; bf16 build)
+bool attention_fwd_tc_supported(int C, int H);
+cudaError_t attention_fwd_tc(act_t* att, float* lse, const act_t* qkv, int B, int T, int C, int H,
+                             int* err, cudaStream_t s);
 // dqkv [B*T, 3C] (overwritten); dsum [B, H, T] scratch.
 cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
                           const act_t* att, const float* lse, int B, int T, int C, int H,

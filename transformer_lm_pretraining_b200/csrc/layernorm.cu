@@ -72,40 +72,34 @@ __global__ void __launch_bounds__(256)
 // grid = kLnBlocks blocks of 8 warps; warp w of block blk handles rows
 // (blk * 8 + w) + k * (kLnBlocks * 8).  partials[blk][0][..C) = dgamma,
 // [1] = dbeta, [2] = column sums of the written dres (when NSUMS == 3).
+// The per-column running sums live in shared memory, one private slice per
+// warp (each lane owns its columns, so no two threads touch the same word),
+// which keeps the row loop's register footprint small enough for several
+// blocks per SM.
 template <int kChunks, int NSUMS>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
     ln_bwd_kernel(act_t* __restrict__ dres, const act_t* __restrict__ dy,
                   const act_t* __restrict__ x, const float* __restrict__ mean,
                   const float* __restrict__ rstd, const float* __restrict__ g,
                   float* __restrict__ partials, int M, int C, int accumulate) {
-  extern __shared__ float red[];  // [8 warps][C]
+  extern __shared__ float red[];  // [8 warps][NSUMS][C]
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nw = blockDim.x / 32;
-  float acc[NSUMS][kChunks][8], gv[kChunks][8];
-#pragma unroll
-  for (int k = 0; k < kChunks; ++k) {
-    const int c = (k * 32 + lane) * 8;
-    if (c < C) load8(g + c, gv[k]);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (c >= C) gv[k][i] = 0.f;
-#pragma unroll
-      for (int j = 0; j < NSUMS; ++j) acc[j][k][i] = 0.f;
-    }
-  }
+  float* mine = red + (size_t)warp * NSUMS * C;
+  for (int i = lane; i < NSUMS * C; i += 32) mine[i] = 0.f;
+  __syncwarp();
   for (int row = blockIdx.x * nw + warp; row < M; row += gridDim.x * nw) {
     const act_t* xr = x + (size_t)row * C;
     const act_t* dyr = dy + (size_t)row * C;
     act_t* dr = dres + (size_t)row * C;
     const float mu = mean[row], rs = rstd[row];
-    float xv[kChunks][8], dv[kChunks][8], ov[kChunks][8];
+    float xv[kChunks][8], dv[kChunks][8];
 #pragma unroll
     for (int k = 0; k < kChunks; ++k) {
       const int c = (k * 32 + lane) * 8;
       if (c < C) {
         load8(xr + c, xv[k]);
         load8(dyr + c, dv[k]);
-        if (accumulate) load8(dr + c, ov[k]);
       }
     }
     float a = 0.f, bsum = 0.f;
@@ -113,17 +107,23 @@ __global__ void __launch_bounds__(256)
     for (int k = 0; k < kChunks; ++k) {
       const int c = (k * 32 + lane) * 8;
       if (c < C) {
+        float gg[8], s0[8], s1[8];
+        load8(g + c, gg);
+        load8(mine + c, s0);
+        load8(mine + C + c, s1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float xh = (xv[k][i] - mu) * rs;
-          const float dxh = dv[k][i] * gv[k][i];
+          const float dxh = dv[k][i] * gg[i];
           a += dxh;
           bsum += dxh * xh;
-          acc[0][k][i] += dv[k][i] * xh;
-          acc[1][k][i] += dv[k][i];
+          s0[i] += dv[k][i] * xh;
+          s1[i] += dv[k][i];
           xv[k][i] = xh;
           dv[k][i] = dxh;
         }
+        store8(mine + c, s0);
+        store8(mine + C + c, s1);
       }
     }
     a = warp_sum(a) / C;
@@ -133,36 +133,28 @@ __global__ void __launch_bounds__(256)
       const int c = (k * 32 + lane) * 8;
       if (c < C) {
         float o[8];
+        if (accumulate) load8(dr + c, o);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          o[i] = (accumulate ? ov[k][i] : 0.f) + rs * (dv[k][i] - a - xv[k][i] * bsum);
+          o[i] = (accumulate ? o[i] : 0.f) + rs * (dv[k][i] - a - xv[k][i] * bsum);
         if (NSUMS == 3) {
           // the bias gradient sums the values as stored (activation dtype)
+          float s2[8];
+          load8(mine + 2 * C + c, s2);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[NSUMS - 1][k][i] += to_f(from_f<act_t>(o[i]));
+          for (int i = 0; i < 8; ++i) s2[i] += to_f(from_f<act_t>(o[i]));
+          store8(mine + 2 * C + c, s2);
         }
         store8(dr + c, o);
       }
     }
   }
-  // block reduction of each column sum in warp order, one sum at a time
-#pragma unroll
-  for (int j = 0; j < NSUMS; ++j) {
-#pragma unroll
-    for (int k = 0; k < kChunks; ++k) {
-      const int c = (k * 32 + lane) * 8;
-      if (c < C) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) red[(size_t)warp * C + c + i] = acc[j][k][i];
-      }
-    }
-    __syncthreads();
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
-      float s = 0.f;
-      for (int w = 0; w < nw; ++w) s += red[(size_t)w * C + c];
-      partials[((size_t)blockIdx.x * NSUMS + j) * C + c] = s;
-    }
-    __syncthreads();
+  __syncthreads();
+  // block reduction of each column sum in warp order
+  for (int i = threadIdx.x; i < NSUMS * C; i += blockDim.x) {
+    float s = 0.f;
+    for (int w = 0; w < nw; ++w) s += red[(size_t)w * NSUMS * C + i];
+    partials[(size_t)blockIdx.x * NSUMS * C + i] = s;
   }
 }
 
@@ -196,11 +188,11 @@ template <int N, int S>
 void ln_bwd_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
                    const float* rstd, const float* g, float* partials, int M, int C,
                    int accumulate, cudaStream_t s) {
-  const size_t smem = (size_t)8 * C * sizeof(float);
+  const size_t smem = (size_t)8 * S * C * sizeof(float);
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(ln_bwd_kernel<N, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         8 * 2048 * 4);
+                         8 * S * 2048 * 4 > 227 * 1024 ? 227 * 1024 : 8 * S * 2048 * 4);
     attr = true;
   }
   ln_bwd_kernel<N, S><<<kLnBlocks, 256, smem, s>>>(dres, dy, x, mean, rstd, g, partials, M, C,
