@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float mnew = fmaxf(mrow[r], mx);
-      const float alpha = exp2f(mrow[r] - mnew);
+      const float alpha = fast_exp2(mrow[r] - mnew);
       lrow[r] *= alpha;
 #pragma unroll
       for (int dt = 0; dt < HD / 8; ++dt) {
@@ -227,8 +227,8 @@ __global__ void __launch_bounds__(kWarps * 32)
       }
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
-        s[nt][2 * r] = exp2f(s[nt][2 * r] - mnew);
-        s[nt][2 * r + 1] = exp2f(s[nt][2 * r + 1] - mnew);
+        s[nt][2 * r] = fast_exp2(s[nt][2 * r] - mnew);
+        s[nt][2 * r + 1] = fast_exp2(s[nt][2 * r + 1] - mnew);
         lrow[r] += s[nt][2 * r] + s[nt][2 * r + 1];
       }
       mrow[r] = mnew;
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         const int q = i * kTile + ql;
         const int key = k0 + warp * 16 + g + 8 * (e >> 1);
         const bool live = q < T && q >= key;
-        st[nt][e] = live ? exp2f(st[nt][e] * sl2 - sm.r0[buf][ql]) : 0.f;
+        st[nt][e] = live ? fast_exp2(st[nt][e] * sl2 - sm.r0[buf][ql]) : 0.f;
       }
     // dV += P^T dO
     mma_pv<HD>(dv, st, sm.y[buf]);
@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         const int key = j * kTile + nt * 8 + 2 * c4 + (e & 1);
         const int qr = q0 + warp * 16 + g + 8 * (e >> 1);
         const bool live = key <= qr && qr < T;
-        s[nt][e] = live ? exp2f(s[nt][e] * sl2 - lse2[e >> 1]) : 0.f;
+        s[nt][e] = live ? fast_exp2(s[nt][e] * sl2 - lse2[e >> 1]) : 0.f;
       }
     float dp[8][4];
 #pragma unroll
@@ -649,7 +649,7 @@ cudaError_t attention_fwd(act_t* att, float* lse, const act_t* qkv, int B, int T
 
 cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
                           const act_t* att, const float* lse, int B, int T, int C, int H,
-                          cudaStream_t s) {
+                          int* err, cudaStream_t s) {
   const size_t n = (size_t)B * T * H;
   attn_rowdot_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dsum, datt, att, B, T, C, H);
   note_launch();
@@ -657,7 +657,7 @@ cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act
 #if GPT2_ACT_BF16
   switch (hd) {
     case 32: return bwd_launch<32>(dqkv, dsum, datt, qkv, lse, B, T, C, H, s);
-    case 64: return bwd_launch<64>(dqkv, dsum, datt, qkv, lse, B, T, C, H, s);
+    case 64: return attention_bwd_tc(dqkv, dsum, datt, qkv, lse, B, T, C, H, err, s);  // tcgen05
     case 128: return bwd_launch<128>(dqkv, dsum, datt, qkv, lse, B, T, C, H, s);
     default: return cudaErrorInvalidValue;
   }

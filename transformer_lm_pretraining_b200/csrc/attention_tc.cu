@@ -1,7 +1,7 @@
 // Causal flash-attention forward on the sm_100a tensor cores (head dim 64).
 //
 // One CTA per (query tile of 128 rows, batch, head), heaviest tiles first;
-// 6 warps:
+// 10 warps:
 //   warp 0     TMA: the Q tile once, then K/V tiles of 128 keys into a
 //              3-stage shared-memory ring (128-byte swizzle, zero fill past
 //              the sequence);
@@ -9,12 +9,15 @@
 //              K=64) into one of two TMEM buffers, and O_j = P_j V_j
 //              (M=128, N=64, K=128; V read MN-major straight from its tile)
 //              into one of two more;
-//   warps 2-5  softmax, one query row per thread: read S_j from TMEM, online
-//              max/sum in base 2, write P_j = exp2(S_j - m) as bf16 into a
-//              swizzled shared-memory tile (the next MMA's A operand), and
-//              fold O_{j-1} into the fp32 row accumulator held in registers
-//              with the pending rescale factor.  S_{j+1} and O_{j-1} are
-//              computed by the tensor core while row j's softmax runs.
+//   warps 2-9  softmax: two threads per query row (warps w and w+4 share a
+//              TMEM lane quarter), each owning 64 of the 128 key columns and
+//              32 of the 64 output dimensions.  They read S_j from TMEM,
+//              agree on the running row max through shared memory, write
+//              P_j = 2^(S_j log2e/sqrt(d) - m) as bf16 into a swizzled tile
+//              (the next MMA's A operand), and fold O_{j-1} into fp32 row
+//              accumulators held in registers with the pending rescale
+//              factor.  S_{j+1} and O_{j-1} are computed by the tensor core
+//              while tile j's softmax runs.
 // T x T is never materialised.  The output row is normalised by the
 // running sum; the natural-log log-sum-exp of each row is stored for the
 // backward pass.  Every wait is bounded (error word ERR_TIMEOUT).
@@ -26,31 +29,32 @@
 #include <mutex>
 #include <tuple>
 
-#include "tc_util.cuh"
+#include "attention_tc.cuh"
 
 namespace gpt2k {
 
 namespace {
 
 using namespace tc;
+using attn::kHD;
+using attn::kBox;
 
-constexpr int kHD = 64;
-constexpr int kTileQ = 128;
-constexpr int kTileK = 128;
+constexpr int kTileQ = attn::kTile;
+constexpr int kTileK = attn::kTile;
 constexpr int kKVStages = 3;
-constexpr int kBox = 16384;  // 128 rows x 64 bf16
-constexpr int kThreadsAttn = 192;
+constexpr int kSoftmaxThreads = attn::kComputeThreads;
+constexpr int kThreadsAttn = 64 + kSoftmaxThreads;
 constexpr uint32_t kTmemCols = 512;  // S: 2 x 128, O: 2 x 64
+constexpr int kAux = 4096;           // barriers + cross-thread row scratch
 
 constexpr size_t attn_smem_bytes() {
-  // Q, K ring, V ring, P double buffer (two 64-key boxes each), barriers
-  return 1024 + kBox + 2 * (size_t)kKVStages * kBox + 2 * 2 * (size_t)kBox + 512;
+  // Q, K ring, V ring, P double buffer (two 64-key boxes each), aux
+  return 1024 + kBox + 2 * (size_t)kKVStages * kBox + 2 * 2 * (size_t)kBox + kAux;
 }
 
-// bf16 x bf16 -> fp32, M = 128, N = n, A K-major, B K- or MN-major
-__host__ __device__ constexpr uint32_t attn_idesc(int n, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) |
-         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+__device__ __forceinline__ void sm_bar() { named_bar<1, kSoftmaxThreads>(); }
+__device__ __forceinline__ bool sm_bar_and(bool pred) {
+  return named_bar_and<1, kSoftmaxThreads>(pred);
 }
 
 __global__ void __launch_bounds__(kThreadsAttn, 1)
@@ -63,8 +67,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   uint8_t* sK = sQ + kBox;                      // [kKVStages][kBox]
   uint8_t* sV = sK + kKVStages * kBox;          // [kKVStages][kBox]
   uint8_t* sP = sV + kKVStages * kBox;          // [2][2 boxes]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 4 * kBox);
-  // barrier slots
+  uint8_t* aux = sP + 4 * kBox;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
   const uint32_t q_full = smem_u32(bars + 0);
   const uint32_t kv_full0 = smem_u32(bars + 1);                  // [3]
   const uint32_t kv_empty0 = smem_u32(bars + 1 + kKVStages);     // [3]
@@ -77,6 +81,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   const uint32_t drain = s_full0 + 96;                           // abort path only
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1 + 2 * kKVStages + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red_max = reinterpret_cast<float*>(aux + 512);   // [2 parity][2 halves][128 rows]
+  float* red_l = red_max + 2 * 2 * kTileQ;                // [2 halves][128 rows]
 
   const int qb = gridDim.x - 1 - blockIdx.x;  // heaviest query tiles first
   const int b = blockIdx.y / H, h = blockIdx.y % H;
@@ -92,11 +98,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full0 + 8 * i, 1);
-      mbar_init(s_empty0 + 8 * i, 128);
-      mbar_init(p_full0 + 8 * i, 128);
+      mbar_init(s_empty0 + 8 * i, kSoftmaxThreads);
+      mbar_init(p_full0 + 8 * i, kSoftmaxThreads);
       mbar_init(p_empty0 + 8 * i, 1);
       mbar_init(o_full0 + 8 * i, 1);
-      mbar_init(o_empty0 + 8 * i, 128);
+      mbar_init(o_empty0 + 8 * i, kSoftmaxThreads);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -150,8 +156,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA --
-      constexpr uint32_t idS = attn_idesc(kTileK, false);
-      constexpr uint32_t idO = attn_idesc(kHD, true);
+      constexpr uint32_t idS = attn::idesc(kTileK, false);
+      constexpr uint32_t idO = attn::idesc(kHD, true);
       bool ok = mbar_wait(q_full, 0, abort_flag, err);
       tc_fence_after();
       const uint32_t q_base = smem_u32(sQ);
@@ -201,90 +207,107 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else {
     // -------------------------------------------------------- softmax --
-    const int qw = warp & 3;  // TMEM lane quarter
+    const int qw = warp & 3;           // TMEM lane quarter
+    const int half = (warp - 2) >> 2;  // 0: key columns 0-63 / dims 0-31; 1: 64-127 / 32-63
     const int r = qw * 32 + lane;
     const int qi = q0 + r;  // query index in the sequence
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    float o[kHD];
+    float o[kHD / 2];
 #pragma unroll
-    for (int i = 0; i < kHD; ++i) o[i] = 0.f;
+    for (int i = 0; i < kHD / 2; ++i) o[i] = 0.f;
     float m = -INFINITY, l = 0.f, a_pend = 1.f;
     bool ok = true;
     for (int j = 0; j <= nkv && ok; ++j) {
       float a_new = 1.f;
       if (j < nkv) {
         const int sb = j & 1;
-        ok = epi_bar_and(mbar_wait(s_full0 + 8 * sb, (uint32_t)(j >> 1) & 1u, abort_flag, err));
+        ok = sm_bar_and(mbar_wait(s_full0 + 8 * sb, (uint32_t)(j >> 1) & 1u, abort_flag, err));
         if (!ok) break;
         tc_fence_after();
-        float s[kTileK];
+        float s[64];
         {
-          uint32_t rr[kTileK];
-#pragma unroll
-          for (int c = 0; c < kTileK / 32; ++c)
-            tc_ld32(lane_base + (uint32_t)(sb * kTileK + 32 * c), rr + 32 * c);
+          uint32_t rr[64];
+          const uint32_t col = (uint32_t)(sb * kTileK + 64 * half);
+          tc_ld32(lane_base + col, rr);
+          tc_ld32(lane_base + col + 32, rr + 32);
           tc_wait_ld();
           tc_fence_before();
           mbar_arrive(s_empty0 + 8 * sb);
 #pragma unroll
-          for (int c = 0; c < kTileK; ++c) s[c] = __uint_as_float(rr[c]) * sl2;
+          for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(rr[c]);
         }
+        const int key0 = j * kTileK + 64 * half;
         if (j == qb) {  // diagonal tile: keys after the query (and past T) are masked
 #pragma unroll
-          for (int c = 0; c < kTileK; ++c)
-            if (j * kTileK + c > qi || j * kTileK + c >= T) s[c] = -INFINITY;
+          for (int c = 0; c < 64; ++c)
+            if (key0 + c > qi || key0 + c >= T) s[c] = -INFINITY;
         }
-        float mx = m;
+        // row max over this thread's 64 columns (8 independent chains),
+        // then with the partner thread's half through shared memory
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < kTileK; ++c) mx = fmaxf(mx, s[c]);
-        a_new = (mx == -INFINITY) ? 1.f : exp2f(m - mx);
-        const float mref = (mx == -INFINITY) ? 0.f : mx;
-        float sum = 0.f;
+        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-        for (int c = 0; c < kTileK; ++c) {
-          s[c] = exp2f(s[c] - mref);
-          sum += s[c];
+        for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        float* rm = red_max + (j & 1) * 2 * kTileQ;
+        rm[half * kTileQ + r] = mx;
+        sm_bar();
+        mx = fmaxf(mx, rm[(half ^ 1) * kTileQ + r]) * sl2;  // scaled (log2 units)
+        const float mnew = fmaxf(m, mx);
+        a_new = (mnew == -INFINITY) ? 1.f : fast_exp2(m - mnew);
+        const float mref = (mnew == -INFINITY) ? 0.f : mnew;
+        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          s[c] = fast_exp2(fmaf(s[c], sl2, -mref));
+          sum8[c & 7] += s[c];
         }
-        l = l * a_new + sum;
-        m = mx;
-        // P_j into its shared-memory tile (two 64-key boxes, 128-byte swizzle)
+        l = l * a_new + (((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
+                         ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
+        m = mnew;
+        // P_j (this half's 64 keys = one 128-byte-swizzled box)
         const int pb = j & 1;
-        ok = epi_bar_and(mbar_wait(p_empty0 + 8 * pb, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, err));
+        ok = sm_bar_and(mbar_wait(p_empty0 + 8 * pb, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, err));
         if (!ok) break;
-        uint8_t* pt = sP + pb * 2 * kBox;
+        uint8_t* pt = sP + (pb * 2 + half) * kBox;
 #pragma unroll
-        for (int c8 = 0; c8 < kTileK / 8; ++c8)
-          store8(reinterpret_cast<__nv_bfloat16*>(pt + (c8 >> 3) * kBox + swz(r, c8 & 7)), s + 8 * c8);
+        for (int c8 = 0; c8 < 8; ++c8)
+          store8(reinterpret_cast<__nv_bfloat16*>(pt + swz(r, c8)), s + 8 * c8);
         fence_async_smem();
         mbar_arrive(p_full0 + 8 * pb);
       }
       if (j >= 1) {  // fold O_{j-1} (computed with the max of tile j-1)
         const int ob = (j - 1) & 1;
-        ok = epi_bar_and(mbar_wait(o_full0 + 8 * ob, (uint32_t)((j - 1) >> 1) & 1u, abort_flag, err));
+        ok = sm_bar_and(mbar_wait(o_full0 + 8 * ob, (uint32_t)((j - 1) >> 1) & 1u, abort_flag, err));
         if (!ok) break;
         tc_fence_after();
-        uint32_t rr[kHD];
-        tc_ld32(lane_base + 2u * kTileK + (uint32_t)(ob * kHD), rr);
-        tc_ld32(lane_base + 2u * kTileK + (uint32_t)(ob * kHD + 32), rr + 32);
+        uint32_t rr[32];
+        tc_ld32(lane_base + 2u * kTileK + (uint32_t)(ob * kHD + 32 * half), rr);
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(o_empty0 + 8 * ob);
 #pragma unroll
-        for (int i = 0; i < kHD; ++i) o[i] = o[i] * a_pend + __uint_as_float(rr[i]);
+        for (int i = 0; i < kHD / 2; ++i) o[i] = o[i] * a_pend + __uint_as_float(rr[i]);
       }
       a_pend = a_new;
     }
+    // row sum = the two halves' partial sums
+    red_l[half * kTileQ + r] = l;
+    sm_bar();
+    l += red_l[(half ^ 1) * kTileQ + r];
     if (ok && qi < T) {
       const float inv = 1.f / l;
-      __nv_bfloat16* dst = att + ((size_t)b * T + qi) * C + (size_t)h * kHD;
+      __nv_bfloat16* dst = att + ((size_t)b * T + qi) * C + (size_t)h * kHD + 32 * half;
 #pragma unroll
-      for (int i = 0; i < kHD; i += 8) {
+      for (int i = 0; i < kHD / 2; i += 8) {
         float t[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) t[k] = o[i + k] * inv;
         store8(dst + i, t);
       }
-      lse[((size_t)b * H + h) * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
+      if (half == 0) lse[((size_t)b * H + h) * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
     }
   }
 
@@ -297,37 +320,35 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encoder_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
+}  // namespace
 
-// qkv viewed as [B][T][3C] bf16; box = 64 columns x 128 rows of one sequence
-cudaError_t qkv_map(CUtensorMap* tm, const void* qkv, int B, int T, int C) {
+namespace attn {
+
+cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols) {
   using Key = std::tuple<const void*, int, int, int>;
   static std::map<Key, CUtensorMap> cache;
   static std::mutex mu;
-  const Key key{qkv, B, T, C};
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  const Key key{base, B, T, cols};
   std::lock_guard<std::mutex> g(mu);
   auto it = cache.find(key);
   if (it != cache.end()) {
     *tm = it->second;
     return cudaSuccess;
   }
-  auto enc = encoder_fn();
-  if (!enc) return cudaErrorNotSupported;
-  cuuint64_t dims[3] = {(cuuint64_t)3 * C, (cuuint64_t)T, (cuuint64_t)B};
-  cuuint64_t strides[2] = {(cuuint64_t)3 * C * 2, (cuuint64_t)T * 3 * C * 2};
+  if (!enc) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return cudaErrorNotSupported;
+    enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)T * cols * 2};
   cuuint32_t box[3] = {64u, 128u, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
-  if (enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(qkv), dims, strides, box, estr,
+  if (enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
@@ -336,7 +357,7 @@ cudaError_t qkv_map(CUtensorMap* tm, const void* qkv, int B, int T, int C) {
   return cudaSuccess;
 }
 
-}  // namespace
+}  // namespace attn
 
 bool attention_fwd_tc_supported(int C, int H) {
   return C / H == kHD && (C * 2) % 16 == 0;
@@ -347,7 +368,7 @@ cudaError_t attention_fwd_tc(act_t* att, float* lse, const act_t* qkv, int B, in
   if (!attention_fwd_tc_supported(C, H) || (reinterpret_cast<uintptr_t>(qkv) & 15))
     return cudaErrorInvalidValue;
   CUtensorMap tm;
-  cudaError_t e = qkv_map(&tm, qkv, B, T, C);
+  cudaError_t e = attn::seq_map(&tm, qkv, B, T, 3 * C);
   if (e != cudaSuccess) return e;
   constexpr size_t smem = attn_smem_bytes();
   static_assert(smem <= 232448, "shared memory budget");

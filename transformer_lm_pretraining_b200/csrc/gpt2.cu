@@ -586,7 +586,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     }
     mark(h, PK_ATTN_BWD, 10.0 * B * H * (double)T * (T + 1) / 2 * (C / H));
     GPT2_CUDA(h, attention_bwd(a.dqkv, a.dsum, a.datt, qkv, att, a.lse + (size_t)l * M * H, B, T,
-                               C, H, s));
+                               C, H, h->err, s));
     {  // dh = dqkv Wqkv
       GemmArgs ga = gemm_args(M, C, 3 * C);
       ga.A = a.dqkv; ga.lda = 3 * C;

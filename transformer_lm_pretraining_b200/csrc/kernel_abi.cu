@@ -57,9 +57,11 @@ int gpt2k_attention_fwd(void* stream, void* att, float* lse, const void* qkv, in
 int gpt2k_attention_bwd(void* stream, void* dqkv, float* dsum, const void* datt, const void* qkv,
                         const void* att, const float* lse, int B, int T, int C, int H) {
   if (B < 1 || T < 1 || H < 1 || C % H) return GPT2_ERR_ARG;
+  int* err = err_word();
+  if (!err) return GPT2_ERR_CUDA;
   return status(attention_bwd(static_cast<act_t*>(dqkv), dsum, static_cast<const act_t*>(datt),
                               static_cast<const act_t*>(qkv), static_cast<const act_t*>(att), lse,
-                              B, T, C, H, static_cast<cudaStream_t>(stream)));
+                              B, T, C, H, err, static_cast<cudaStream_t>(stream)));
 }
 
 int gpt2k_take_error(void) {
