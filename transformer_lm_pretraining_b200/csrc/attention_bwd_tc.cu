@@ -57,8 +57,10 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t par, uint64_t 
 // ------------------------------------------------------------------ dK/dV --
 constexpr int kQStages = 2;
 constexpr size_t dkdv_smem_bytes() {
-  // K, V, [Q, dO] x stages, P^T and dS^T tiles (two boxes each), aux
-  return 1024 + 2 * (size_t)kBox + 2 * (size_t)kQStages * kBox + 4 * (size_t)kBox + kAux;
+  // K, V, [Q, dO] x stages, P^T and dS^T tiles (two boxes each), per-column
+  // L and D of two query tiles, aux
+  return 1024 + 2 * (size_t)kBox + 2 * (size_t)kQStages * kBox + 4 * (size_t)kBox +
+         4 * kTile * sizeof(float) + kAux;
 }
 
 __global__ void __launch_bounds__(kThreadsBwd, 1)
@@ -75,7 +77,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   uint8_t* sDO = sQ + kQStages * kBox;    // [kQStages]
   uint8_t* sPT = sDO + kQStages * kBox;   // 2 boxes (query columns 0-63, 64-127)
   uint8_t* sDST = sPT + 2 * kBox;         // 2 boxes
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDST + 2 * kBox);
+  float* col_lse = reinterpret_cast<float*>(sDST + 2 * kBox);  // [2 tiles][L 128, D 128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(col_lse + 4 * kTile);
   const uint32_t kv_full = smem_u32(bars + 0);
   const uint32_t qd_full0 = smem_u32(bars + 1);   // [2]
   const uint32_t qd_empty0 = smem_u32(bars + 3);  // [2]
@@ -196,9 +199,18 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
     const float* lse_bh = lse + ((size_t)b * H + h) * T;
     const float* d_bh = dsum + ((size_t)b * H + h) * T;
+    const int ct = threadIdx.x - 64;  // 0 .. 255
     bool ok = true;
     for (int t = 0; t < n && ok; ++t) {
       const int qc0 = (j + t) * kTile + 64 * half;  // first query column of this half
+      // this tile's per-column L (log2 units) and D into shared memory,
+      // loaded while the tensor core computes S^T and dP^T
+      float* cl = col_lse + (t & 1) * 2 * kTile;
+      {
+        const int q = (j + t) * kTile + (ct & (kTile - 1));
+        const float v = q < T ? (ct < kTile ? lse_bh[q] * kLog2e : d_bh[q]) : 0.f;
+        cl[ct] = v;  // [0, 128): L, [128, 256): D
+      }
       ok = cbar_and(mbar_wait(sd_full, (uint32_t)t & 1u, abort_flag, err));
       if (!ok) break;
       ok = cbar_and(mbar_wait(pd_empty, ((uint32_t)t & 1u) ^ 1u, abort_flag, err));
@@ -211,12 +223,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         tc_ld32(lane_base + col, rs);
         tc_ld32(lane_base + kTile + col, rp);
         float pv[32], dv[32];
-        // per-column L (log2 units) and D, shared by every row of the warp
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int q = qc0 + 32 * ch + c;
-          pv[c] = q < T ? lse_bh[q] * kLog2e : 0.f;
-          dv[c] = q < T ? d_bh[q] : 0.f;
+        for (int c = 0; c < 32; c += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(cl + col + c);
+          const float4 d = *reinterpret_cast<const float4*>(cl + kTile + col + c);
+          pv[c] = a.x; pv[c + 1] = a.y; pv[c + 2] = a.z; pv[c + 3] = a.w;
+          dv[c] = d.x; dv[c + 1] = d.y; dv[c + 2] = d.z; dv[c + 3] = d.w;
         }
         tc_wait_ld();
 #pragma unroll

@@ -158,26 +158,34 @@ __global__ void __launch_bounds__(256, 3)
   }
 }
 
-// out_j[c] += sum over blocks (in order) of partials[blk][j][c]: thread
-// (tx, ty) takes column tx of a 32-column group and blocks ty, ty+8, ...;
-// the 8 partial sums are then added in ty order.
-__global__ void ln_bwd_reduce_kernel(float* __restrict__ dg, float* __restrict__ db,
-                                     float* __restrict__ dsum3,
-                                     const float* __restrict__ partials, int nblk, int nsums,
-                                     int C) {
-  __shared__ float red[8][33];
+// out_j[c] += sum over blocks of partials[blk][j][c] in a fixed order:
+// thread (tx, ty) of a 32 x 32 block takes column tx of a 32-column group
+// and blocks ty, ty+32, ... (four independent running sums, combined in a
+// fixed order); the 32 partial sums are then added in ty order.
+__global__ void __launch_bounds__(1024)
+    ln_bwd_reduce_kernel(float* __restrict__ dg, float* __restrict__ db, float* __restrict__ dsum3,
+                         const float* __restrict__ partials, int nblk, int nsums, int C) {
+  __shared__ float red[32][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + tx;  // over nsums * C
-  float s = 0.f;
+  const size_t stride = (size_t)nsums * C;
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
   if (col < nsums * C) {
-    const int j = col / C, c = col % C;
-    for (int b = ty; b < nblk; b += 8) s += partials[((size_t)b * nsums + j) * C + c];
+    const float* p = partials + col;
+    int b = ty;
+    for (; b + 96 < nblk; b += 128) {
+      s[0] += p[(size_t)b * stride];
+      s[1] += p[(size_t)(b + 32) * stride];
+      s[2] += p[(size_t)(b + 64) * stride];
+      s[3] += p[(size_t)(b + 96) * stride];
+    }
+    for (int k = 0; b < nblk; b += 32, ++k) s[k] += p[(size_t)b * stride];
   }
-  red[ty][tx] = s;
+  red[ty][tx] = (s[0] + s[1]) + (s[2] + s[3]);
   __syncthreads();
   if (ty == 0 && col < nsums * C) {
     float t = 0.f;
-    for (int k = 0; k < 8; ++k) t += red[k][tx];
+    for (int k = 0; k < 32; ++k) t += red[k][tx];
     const int j = col / C, c = col % C;
     float* dst = j == 0 ? dg : (j == 1 ? db : dsum3);
     dst[c] += t;
@@ -231,8 +239,8 @@ void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* me
 #undef GPT2_LNB
     default: break;
   }
-  ln_bwd_reduce_kernel<<<(nsums * C + 31) / 32, 256, 0, s>>>(dg, db, dbias_out, partials,
-                                                              kLnBlocks, nsums, C);
+  ln_bwd_reduce_kernel<<<(nsums * C + 31) / 32, 1024, 0, s>>>(dg, db, dbias_out, partials,
+                                                               kLnBlocks, nsums, C);
   note_launch(2);
 }
 

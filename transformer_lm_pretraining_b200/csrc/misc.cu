@@ -89,22 +89,23 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// db[n] += sum over chunks (in order) of partials[chunk][n]: thread (tx, ty)
-// takes column tx of a 32-column group and chunks ty, ty+8, ...; the 8
-// partial sums are added in ty order.
-__global__ void colsum_reduce_kernel(float* __restrict__ db, const float* __restrict__ partials,
-                                     int chunks, int N) {
-  __shared__ float red[8][33];
+// db[n] += sum over chunks of partials[chunk][n] in a fixed order: thread
+// (tx, ty) of a 32 x 32 block takes column tx of a 32-column group and
+// chunks ty, ty+32, ...; the 32 partial sums are added in ty order.
+__global__ void __launch_bounds__(1024)
+    colsum_reduce_kernel(float* __restrict__ db, const float* __restrict__ partials, int chunks,
+                         int N) {
+  __shared__ float red[32][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int n = blockIdx.x * 32 + tx;
   float s = 0.f;
   if (n < N)
-    for (int c = ty; c < chunks; c += 8) s += partials[(size_t)c * N + n];
+    for (int c = ty; c < chunks; c += 32) s += partials[(size_t)c * N + n];
   red[ty][tx] = s;
   __syncthreads();
   if (ty == 0 && n < N) {
     float t = 0.f;
-    for (int k = 0; k < 8; ++k) t += red[k][tx];
+    for (int k = 0; k < 32; ++k) t += red[k][tx];
     db[n] += t;
   }
 }
@@ -371,7 +372,7 @@ void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaS
   const int chunks = (M + rows - 1) / rows;
   dim3 g(colgroups, chunks);
   colsum_partial_kernel<<<g, 256, 0, s>>>(partials, dy, M, N, rows);
-  colsum_reduce_kernel<<<(N + 31) / 32, 256, 0, s>>>(db, partials, chunks, N);
+  colsum_reduce_kernel<<<(N + 31) / 32, 1024, 0, s>>>(db, partials, chunks, N);
   note_launch(2);
 }
 
