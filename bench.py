@@ -39,6 +39,27 @@ from transformer_lm_pretraining_b200.workloads import WORKLOADS  # noqa: E402
 PAGES_A100_TOK_S = 16384 / 0.090  # 90 ms per 16x1024 step on 1x A100 SXM 80GB (pages)
 SPEC_BF16_DENSE = 2.25e15
 
+# DRAM bytes (read + write) per GEMM launch, averaged over the launches of a
+# gpt2_124m step, from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum, profiles/gemm_tc_dram_traffic_gpt2_124m_step.md).
+# Valid only for the GEMM sources it was taken on: reported as null as soon
+# as their hash differs.
+GEMM_TRAFFIC = {"bytes_per_launch": 1.398e8,
+                "sources_sha256": "faf889710ae8d57cd083392a2e9353af33ed4afac34b385b9aa1a878c362ee7f"}
+GEMM_SOURCES = ("gemm_tc.cu", "gemm_epi.cuh", "tc_util.cuh")
+
+
+def gemm_traffic(workload):
+    import hashlib
+
+    if workload != "gpt2_124m":
+        return None
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(HERE, "transformer_lm_pretraining_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return GEMM_TRAFFIC["bytes_per_launch"] if h.hexdigest() == GEMM_TRAFFIC["sources_sha256"] else None
+
 
 def load_peaks():
     p = os.path.join(HERE, "MEASURED_PEAKS.json")
@@ -228,7 +249,6 @@ def run_ours(args, wl):
 
     clocks = ClockSampler(local)
     clocks.start()
-    model.profile_enable(True)
     n0 = g2.gpt2_launch_count()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
@@ -237,11 +257,21 @@ def run_ours(args, wl):
     ev1.record(stream)
     torch.cuda.synchronize()
     launches = (g2.gpt2_launch_count() - n0) // args.steps
-    prof = model.profile_read()
-    model.profile_enable(False)
     clk = clocks.stop()
     barrier()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+
+    # per-kernel-family device time: a second timed pass over the same
+    # batches with CUDA events around every launch on the step's stream
+    # (kept out of the headline loop, whose time the events would inflate)
+    n_prof = min(args.steps, 20)
+    torch.cuda.synchronize()
+    model.profile_enable(True)
+    for k in range(args.warmup, args.warmup + n_prof):
+        step(k, dev[k])
+    torch.cuda.synchronize()
+    prof = model.profile_read()
+    model.profile_enable(False)
     ms_step = ms_total / args.steps
     tokens = wl.tokens_per_step * args.steps * world
     value = tokens / (ms_total / 1e3)
@@ -281,7 +311,7 @@ def run_ours(args, wl):
     mfu = fpt * value / world / SPEC_BF16_DENSE
     gemm_ms, gemm_n, gemm_fl = prof["gemm"]
     achieved = gemm_fl / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
-    fam_ms = {k: v[0] / args.steps for k, v in prof.items()}
+    fam_ms = {k: v[0] / n_prof for k, v in prof.items()}
     fam_total = sum(fam_ms.values())
     out = {
         "metric": "training tokens/s and MFU, GPT-2 124M bf16, B=16xT=1024, 1xB200"
@@ -307,8 +337,12 @@ def run_ours(args, wl):
                      "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops_sustained"] if achieved else None,
                      "peak_source": f"{peaks['source']} sustained bf16",
-                     "launches_per_step": gemm_n / args.steps,
-                     "traffic": None},
+                     "launches_per_step": gemm_n / n_prof,
+                     "timing": f"CUDA events around each GEMM launch on the step's stream, "
+                               f"second timed pass of {n_prof} steps",
+                     "traffic": gemm_traffic(wl.name),
+                     "traffic_unit": "bytes per launch (ncu dram read + write, averaged over the "
+                                     "step's GEMM launches)"},
         "kernel_breakdown_ms_per_step": {k: round(v, 4) for k, v in fam_ms.items()},
         "kernel_breakdown_share": {k: round(v / fam_total, 4) for k, v in fam_ms.items()}
         if fam_total > 0 else None,
