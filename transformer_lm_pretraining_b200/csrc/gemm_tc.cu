@@ -5,12 +5,16 @@
 //              into a STAGES-deep shared-memory ring;
 //   warp 1     allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16)
 //              from one elected lane, accumulating fp32 in TMEM;
-//   warps 2-5  epilogue, 64 columns at a time: tcgen05.ld of the accumulator
-//              (thread = row), bias / GELU / residual / GELU-backward, then
-//              the results are written to a 128-byte-swizzled shared-memory
-//              box and leave with one TMA bulk store (TMA reduce-add for the
-//              fp32 gradient accumulation).  Residual and pre-activation
-//              inputs arrive by TMA into the same kind of box.
+//   warps 2-9  epilogue, two warps per TMEM lane quarter: each warp owns
+//              32 rows and every other 64-column group of the tile.  Per
+//              group: tcgen05.ld of the accumulator (thread = row), bias /
+//              GELU / residual / GELU-backward, the result written to the
+//              warp's own 128-byte-swizzled shared-memory box and sent with
+//              one TMA bulk store (TMA reduce-add for the fp32 gradient
+//              accumulation).  Residual and pre-activation inputs arrive by
+//              TMA in the same box ahead of the accumulator read.  Warps
+//              synchronise only within themselves, so no epilogue step
+//              waits for another warp.
 // The TMEM accumulator is double-buffered so the epilogue of one tile runs
 // under the main loop of the next.  Both operands may be K-major or
 // MN-major (the tensor core reads either from the descriptor), which covers
@@ -38,8 +42,15 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 192;
-constexpr int kStageBox = 16384;  // one 128-row x 128-byte epilogue box
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;
+constexpr int kWarpBox = 4096;  // one warp's epilogue box: 32 rows x 128 bytes
+
+// Epilogues that read a second [M, N] input (residual or pre-activation).
+constexpr bool epi_has_input(int epi) { return epi == EPI_BIAS_RESID || epi == EPI_DGELU; }
+// Operand ring depth: what the shared memory holds next to the epilogue boxes.
+constexpr int ring_stages(int bn, int /*epi*/) { return bn == 256 ? 4 : 6; }
 
 // Instruction descriptor: bf16 x bf16 -> fp32, M = 128, N = BN.
 template <int BN, bool A_MN, bool B_MN>
@@ -53,9 +64,10 @@ constexpr uint32_t tmem_cols() {
   return 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
 }
 
-template <int BN, int STAGES>
+template <int BN, int EPI>
 constexpr size_t smem_bytes() {
-  return 1024 + (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 2 * kStageBox + 256;
+  return 1024 + (size_t)ring_stages(BN, EPI) * (BM * BK * 2 + BN * BK * 2) +
+         (size_t)kEpiWarps * kWarpBox + 256;
 }
 
 template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI>
@@ -68,7 +80,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = tmem_cols<BN>();
-  constexpr bool HAS_IN = (EPI == EPI_BIAS_RESID || EPI == EPI_DGELU);
+  constexpr bool HAS_IN = epi_has_input(EPI);
+  static_assert(STAGES == ring_stages(BN, EPI), "ring depth");
   constexpr bool F32_OUT = (EPI == EPI_F32_ACC || EPI == EPI_F32_STORE);
   constexpr bool HAS_BIAS = (EPI == EPI_BIAS || EPI == EPI_BIAS_GELU || EPI == EPI_BIAS_RESID);
 
@@ -77,17 +90,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint8_t* st0 = smem + STAGES * (A_BYTES + B_BYTES);  // epilogue boxes (1024-aligned)
-  uint8_t* st1 = st0 + kStageBox;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(st1 + kStageBox);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  uint8_t* sBox = smem + STAGES * (A_BYTES + B_BYTES);  // [kEpiWarps] boxes, 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sBox + kEpiWarps * kWarpBox);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4 + kEpiWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
   const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
-  const uint32_t in_full = smem_u32(bars + 2 * STAGES + 4);
+  const uint32_t in_full0 = smem_u32(bars + 2 * STAGES + 4);  // [kEpiWarps]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -102,9 +114,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, 128);
+      mbar_init(tempty0 + 8 * b, kEpiThreads);
     }
-    mbar_init(in_full, 1);
+    for (int w = 0; w < kEpiWarps; ++w) mbar_init(in_full0 + 8 * w, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -239,43 +251,69 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue --
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;
-    const int etid = threadIdx.x - 64;  // 0 .. 127
-    const uint32_t st0_u = smem_u32(st0), st1_u = smem_u32(st1);
-    if (etid == 0) {
+    const int q = warp & 3;          // TMEM lane quarter this warp may access
+    const int h = (warp - 2) >> 2;   // groups h, h + 2, ... of each tile
+    uint8_t* box = sBox + (warp - 2) * kWarpBox;
+    const uint32_t box_u = smem_u32(box);
+    const uint32_t in_full = in_full0 + 8 * (warp - 2);
+    uint32_t in_phase = 0;
+    bool in_pend = false;  // an input copy into the box is in flight
+    if (warp == 2 && lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmOut)) : "memory");
-      if (HAS_IN || EPI == EPI_BIAS_GELU)
+      if (EPI == EPI_BIAS_GELU || HAS_IN)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
     }
+    // Write 8 16-byte chunks of this thread's row into the warp's box and
+    // send the box with `send` from lane 0 once every lane's writes are
+    // visible to the async proxy.  The box is reused only after the
+    // previous store has read it.
+    auto put_box = [&](auto write_row, auto send) {
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+      write_row();
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        send();
+        bulk_commit();
+      }
+    };
     int acc = 0;
-    uint32_t acc_phase = 0, in_phase = 0;
+    uint32_t acc_phase = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       int tm, tn, kb0, kb1, sp;
       decode(u, tm, tn, kb0, kb1, sp);
       const int m0 = tm * BM, nt0 = tn * BN;
+      const int r0 = m0 + q * 32;  // first row of this warp's slab
       const int ngroups = (min(BN, ep.N - nt0) + 63) >> 6;  // 64-column groups in range
-      if (HAS_IN && etid == 0) {
-        mbar_expect_tx(in_full, kStageBox);
-        tma_load_3d(st1_u, &tmX, in_full, nt0, m0, 0);
-      }
-      // uniform decision over the epilogue warps (TMEM loads are
-      // warp-collective and the named barriers below need all 128 threads)
-      ok = epi_bar_and(mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, err));
+      ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, err));
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      if (h >= ngroups) {  // no group for this warp in a narrow tile
+        tc_fence_before();
+        mbar_arrive(tempty0 + 8 * acc);
+      }
 #pragma unroll 1
-      for (int g = 0; g < ngroups; ++g) {
-        const int nb = nt0 + 64 * g;
+      for (int g = h; g < ngroups; g += 2) {
+        const int nb = nt0 + 64 * g;  // first column of the group
+        const bool live = r0 < ep.M;  // rows of this slab exist
+        if (HAS_IN && live && lane == 0) {
+          // the group's input slab into the box, ahead of the accumulator
+          // read (the box is free once the previous store has read it)
+          bulk_wait_read<0>();
+          mbar_expect_tx(in_full, kWarpBox);
+          tma_load_3d(box_u, &tmX, in_full, nb, r0, 0);
+          in_pend = true;
+        }
         float v[64];
         {
           uint32_t r[64];
           tc_ld32(t_row + (uint32_t)(64 * g), r);
           tc_ld32(t_row + (uint32_t)(64 * g + 32), r + 32);
           tc_wait_ld();
-          if (g == ngroups - 1) {  // every TMEM read of this tile is done
+          if (g + 2 >= ngroups) {  // every TMEM read of this warp for the tile is done
             tc_fence_before();
             mbar_arrive(tempty0 + 8 * acc);
           }
@@ -287,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float4* b4 = reinterpret_cast<const float4*>(ep.bias + nb);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const float4 b = b4[j];
+              const float4 b = __ldg(b4 + j);
               v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
             }
           } else {
@@ -296,68 +334,80 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (nb + i < ep.N) v[i] += ep.bias[nb + i];
           }
         }
+        if (!live) continue;  // slab entirely below the matrix: nothing to store
         if (HAS_IN) {
-          ok = epi_bar_and(mbar_wait(in_full, in_phase, abort_flag, err));
+          ok = __all_sync(0xffffffffu, mbar_wait(in_full, in_phase, abort_flag, err));
           if (!ok) break;
           in_phase ^= 1u;
-          float x[64];
+          in_pend = false;
+          uint4 xin[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) load8(reinterpret_cast<const act_t*>(st1 + swz(row, j)), x + 8 * j);
-          epi_bar();  // everyone has read the input box
-          if (etid == 0 && g + 1 < ngroups) {
-            fence_async_smem();
-            mbar_expect_tx(in_full, kStageBox);
-            tma_load_3d(st1_u, &tmX, in_full, nb + 64, m0, 0);
-          }
-          if (EPI == EPI_BIAS_RESID) {
+          for (int c = 0; c < 8; ++c) xin[c] = *reinterpret_cast<const uint4*>(box + swz(lane, c));
+          __syncwarp();  // the box is rewritten below
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] += x[i];
-          } else {
+          for (int c = 0; c < 8; ++c) {
+            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xin[c]);
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] *= gelu_tanh_grad(x[i]);
+            for (int i = 0; i < 4; ++i) {
+              const float2 x = __bfloat1622float2(x2[i]);
+              if (EPI == EPI_BIAS_RESID) {
+                v[8 * c + 2 * i] += x.x;
+                v[8 * c + 2 * i + 1] += x.y;
+              } else {
+                v[8 * c + 2 * i] *= gelu_tanh_grad(x.x);
+                v[8 * c + 2 * i + 1] *= gelu_tanh_grad(x.y);
+              }
+            }
           }
         }
-        // the previous group's stores must have read the boxes
-        if (etid == 0) bulk_wait_read_all();
-        epi_bar();
         if (F32_OUT) {
+          // two 32-column fp32 boxes, one after the other
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            *reinterpret_cast<float4*>(st0 + swz(row, j)) =
-                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            *reinterpret_cast<float4*>(st1 + swz(row, j)) =
-                make_float4(v[32 + 4 * j], v[33 + 4 * j], v[34 + 4 * j], v[35 + 4 * j]);
+          for (int half = 0; half < 2; ++half) {
+            if (half == 1 && nb + 32 >= ep.N) break;
+            put_box(
+                [&] {
+#pragma unroll
+                  for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<float4*>(box + swz(lane, j)) =
+                        make_float4(v[32 * half + 4 * j], v[32 * half + 4 * j + 1],
+                                    v[32 * half + 4 * j + 2], v[32 * half + 4 * j + 3]);
+                },
+                [&] {
+                  if (EPI == EPI_F32_ACC) tma_reduce_add_3d(&tmOut, box_u, nb + 32 * half, r0, 0);
+                  else tma_store_3d(&tmOut, box_u, nb + 32 * half, r0, sp);
+                });
           }
         } else {
           if (EPI == EPI_BIAS_GELU) {
+            // the pre-activation u first (saved for the backward), then GELU(u)
+            put_box(
+                [&] {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(st1 + swz(row, j)), v + 8 * j);
+                  for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(box + swz(lane, j)), v + 8 * j);
+                },
+                [&] { tma_store_3d(&tmX, box_u, nb, r0, 0); });
 #pragma unroll
             for (int i = 0; i < 64; ++i) v[i] = gelu_tanh(v[i]);
           }
+          put_box(
+              [&] {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(st0 + swz(row, j)), v + 8 * j);
-        }
-        fence_async_smem();
-        epi_bar();
-        if (etid == 0) {
-          if (EPI == EPI_F32_ACC) {
-            tma_reduce_add_3d(&tmOut, st0_u, nb, m0, 0);
-            if (nb + 32 < ep.N) tma_reduce_add_3d(&tmOut, st1_u, nb + 32, m0, 0);
-          } else if (EPI == EPI_F32_STORE) {
-            tma_store_3d(&tmOut, st0_u, nb, m0, sp);
-            if (nb + 32 < ep.N) tma_store_3d(&tmOut, st1_u, nb + 32, m0, sp);
-          } else {
-            tma_store_3d(&tmOut, st0_u, nb, m0, 0);
-            if (EPI == EPI_BIAS_GELU) tma_store_3d(&tmX, st1_u, nb, m0, 0);
-          }
-          bulk_commit();
+                for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(box + swz(lane, j)), v + 8 * j);
+              },
+              [&] { tma_store_3d(&tmOut, box_u, nb, r0, 0); });
         }
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    if (etid == 0) bulk_wait_all();
+    if (lane == 0) {
+      bulk_wait_all();
+      // an input copy still in flight lands before the shared memory is released
+      const uint64_t t0 = global_ns();
+      while (in_pend && !mbar_try_wait(in_full, in_phase) && global_ns() - t0 < kWaitLimitNs) {
+      }
+    }
   }
 
   tc_fence_before();
@@ -434,12 +484,12 @@ static int num_sms() {
   return n;
 }
 
-template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI>
+template <int BN, bool A_MN, bool B_MN, int EPI>
 static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
                           const CUtensorMap& tx, const EpiParams& ep, int K, int splits,
                           int kb_per_split, int n_fast, cudaStream_t s, int* err) {
-  auto kern = gemm_tc_kernel<BN, STAGES, A_MN, B_MN, EPI>;
-  constexpr size_t smem = smem_bytes<BN, STAGES>();
+  auto kern = gemm_tc_kernel<BN, ring_stages(BN, EPI), A_MN, B_MN, EPI>;
+  constexpr size_t smem = smem_bytes<BN, EPI>();
   static_assert(smem <= 232448, "shared memory budget");
   static bool attr_done = false;
   if (!attr_done) {
@@ -457,15 +507,14 @@ static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CU
   return cudaGetLastError();
 }
 
-template <int BN, int STAGES>
+template <int BN>
 static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb,
                             const CUtensorMap& to, const CUtensorMap& tx, const EpiParams& ep,
                             int epi, int splits, int kb_per_split, int n_fast, cudaStream_t s,
                             int* err) {
 #define GPT2_TC(AM, BMJ, E)                                                                      \
   if (a.a_mn == AM && a.b_mn == BMJ && epi == E)                                                 \
-    return launch<BN, STAGES, AM, BMJ, E>(ta, tb, to, tx, ep, a.K, splits, kb_per_split, n_fast, \
-                                          s, err);
+    return launch<BN, AM, BMJ, E>(ta, tb, to, tx, ep, a.K, splits, kb_per_split, n_fast, s, err);
   GPT2_TC(0, 0, EPI_STORE)
   GPT2_TC(0, 0, EPI_BIAS)
   GPT2_TC(0, 0, EPI_BIAS_GELU)
@@ -565,26 +614,27 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   int kb_per_split = (kb_total + splits - 1) / splits;
   splits = (kb_total + kb_per_split - 1) / kb_per_split;  // no empty split
   // epilogue tensor maps
+  // epilogue tensor maps: one warp's 32-row slab per box
   if (splits > 1) {
     epi = EPI_F32_STORE;
-    e = make_tmap(&to, a.split_ws, true, a.N, a.M, a.N, 32, BM, splits, (uint64_t)a.M * a.N);
+    e = make_tmap(&to, a.split_ws, true, a.N, a.M, a.N, 32, 32, splits, (uint64_t)a.M * a.N);
   } else if (f32_out) {
-    e = make_tmap(&to, a.out32, true, a.N, a.M, a.ldo32, 32, BM, 1);
+    e = make_tmap(&to, a.out32, true, a.N, a.M, a.ldo32, 32, 32, 1);
   } else {
-    e = make_tmap(&to, a.out, false, a.N, a.M, a.ldo, 64, BM, 1);
+    e = make_tmap(&to, a.out, false, a.N, a.M, a.ldo, 64, 32, 1);
   }
   if (e != cudaSuccess) return e;
-  if (a.epi == EPI_BIAS_RESID) e = make_tmap(&tx, a.resid, false, a.N, a.M, a.ldr, 64, BM, 1);
+  if (a.epi == EPI_BIAS_RESID) e = make_tmap(&tx, a.resid, false, a.N, a.M, a.ldr, 64, 32, 1);
   else if (a.epi == EPI_BIAS_GELU || a.epi == EPI_DGELU)
-    e = make_tmap(&tx, a.aux, false, a.N, a.M, a.ldaux, 64, BM, 1);
+    e = make_tmap(&tx, a.aux, false, a.N, a.M, a.ldaux, 64, 32, 1);
   if (e != cudaSuccess) return e;
   // The larger operand is reused by consecutive tiles (L2 locality).
   const double a_bytes = (double)a.M * a.K, b_bytes = (double)a.N * a.K;
   const int n_fast = a_bytes > b_bytes ? 1 : 0;
   if (BN == 256)
-    e = dispatch<256, 4>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
+    e = dispatch<256>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
   else
-    e = dispatch<128, 6>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
+    e = dispatch<128>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
   if (e != cudaSuccess) return e;
   if (splits > 1) {
     const size_t total = (size_t)a.M * a.N;
