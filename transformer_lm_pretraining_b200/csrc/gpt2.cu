@@ -442,7 +442,7 @@ gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int 
   h->have_logits = false;
   if (tgt) {
     mark(h, PK_CLASSIFIER);
-    classifier(a.logits, a.losses, tgt, M, y.V, y.Vp, h->err, s);
+    classifier(a.logits, a.losses, tgt, M, y.V, y.Vp, 1, h->err, s);
     mean_loss(h->scalars + S_LOSS, a.losses, M, s);
     h->have_grad_logits = true;
   } else {

@@ -111,10 +111,11 @@ cudaError_t attention_bwd_tc(act_t* dqkv, const float* dsum, const act_t* datt, 
 
 // ---------------------------------------------------------- classifier --
 // In place over logits [M, Vp]: per row lse over the first V columns,
-// losses[m] = lse - z[tgt[m]], and z <- (softmax(z) - onehot(tgt)) / M for
-// columns < V, 0 for the padded columns.  Bad targets set err bit 2.
-void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int Vp, int* err,
-                cudaStream_t s);
+// losses[m] = lse - z[tgt[m]], and (write_grad != 0) z <- (softmax(z) -
+// onehot(tgt)) / M for columns < V, 0 for the padded columns.  Bad targets
+// set err bit 2.
+void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int Vp, int write_grad,
+                int* err, cudaStream_t s);
 // out[0] = mean of losses[0..M) (fixed-order reduction)
 void mean_loss(float* out, const float* losses, int M, cudaStream_t s);
 

@@ -69,15 +69,21 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// grid = kLnBlocks blocks of 8 warps; warp w of block blk handles rows
-// (blk * 8 + w) + k * (kLnBlocks * 8).  partials[blk][0][..C) = dgamma,
+// grid = nblk blocks of 8 warps; warp w of block blk handles rows
+// (blk * 8 + w) + k * (nblk * 8).  partials[blk][0][..C) = dgamma,
 // [1] = dbeta, [2] = column sums of the written dres (when NSUMS == 3).
 // The per-column running sums live in shared memory, one private slice per
 // warp (each lane owns its columns, so no two threads touch the same word),
 // which keeps the row loop's register footprint small enough for several
 // blocks per SM.
+// 8 activations as loaded (16 bytes in the bf16 build): rows are kept in
+// this form and converted where used.
+struct alignas(16) Pack8 {
+  act_t v[8];
+};
+
 template <int kChunks, int NSUMS>
-__global__ void __launch_bounds__(256, 3)
+__global__ void __launch_bounds__(256, 2)
     ln_bwd_kernel(act_t* __restrict__ dres, const act_t* __restrict__ dy,
                   const act_t* __restrict__ x, const float* __restrict__ mean,
                   const float* __restrict__ rstd, const float* __restrict__ g,
@@ -92,16 +98,18 @@ __global__ void __launch_bounds__(256, 3)
     const act_t* xr = x + (size_t)row * C;
     const act_t* dyr = dy + (size_t)row * C;
     act_t* dr = dres + (size_t)row * C;
-    const float mu = mean[row], rs = rstd[row];
-    float xv[kChunks][8], dv[kChunks][8];
+    // every load of the row is issued before any of it is used
+    Pack8 px[kChunks], pd[kChunks], po[kChunks];
 #pragma unroll
     for (int k = 0; k < kChunks; ++k) {
       const int c = (k * 32 + lane) * 8;
       if (c < C) {
-        load8(xr + c, xv[k]);
-        load8(dyr + c, dv[k]);
+        px[k] = *reinterpret_cast<const Pack8*>(xr + c);
+        pd[k] = *reinterpret_cast<const Pack8*>(dyr + c);
+        if (accumulate) po[k] = *reinterpret_cast<const Pack8*>(dr + c);
       }
     }
+    const float mu = mean[row], rs = rstd[row];
     float a = 0.f, bsum = 0.f;
 #pragma unroll
     for (int k = 0; k < kChunks; ++k) {
@@ -113,14 +121,13 @@ __global__ void __launch_bounds__(256, 3)
         load8(mine + C + c, s1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float xh = (xv[k][i] - mu) * rs;
-          const float dxh = dv[k][i] * gg[i];
+          const float xh = (to_f(px[k].v[i]) - mu) * rs;
+          const float d = to_f(pd[k].v[i]);
+          const float dxh = d * gg[i];
           a += dxh;
           bsum += dxh * xh;
-          s0[i] += dv[k][i] * xh;
-          s1[i] += dv[k][i];
-          xv[k][i] = xh;
-          dv[k][i] = dxh;
+          s0[i] += d * xh;
+          s1[i] += d;
         }
         store8(mine + c, s0);
         store8(mine + C + c, s1);
@@ -132,11 +139,14 @@ __global__ void __launch_bounds__(256, 3)
     for (int k = 0; k < kChunks; ++k) {
       const int c = (k * 32 + lane) * 8;
       if (c < C) {
-        float o[8];
-        if (accumulate) load8(dr + c, o);
+        float gg[8], o[8];
+        load8(g + c, gg);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          o[i] = (accumulate ? o[i] : 0.f) + rs * (dv[k][i] - a - xv[k][i] * bsum);
+        for (int i = 0; i < 8; ++i) {
+          const float xh = (to_f(px[k].v[i]) - mu) * rs;
+          const float dxh = to_f(pd[k].v[i]) * gg[i];
+          o[i] = (accumulate ? to_f(po[k].v[i]) : 0.f) + rs * (dxh - a - xh * bsum);
+        }
         if (NSUMS == 3) {
           // the bias gradient sums the values as stored (activation dtype)
           float s2[8];
@@ -192,19 +202,32 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
+// Launches one wave: as many blocks as are resident at once (at most
+// kLnBlocks), so no block waits for a second wave.  Returns the grid used.
 template <int N, int S>
-void ln_bwd_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
-                   const float* rstd, const float* g, float* partials, int M, int C,
-                   int accumulate, cudaStream_t s) {
+int ln_bwd_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
+                  const float* rstd, const float* g, float* partials, int M, int C,
+                  int accumulate, cudaStream_t s) {
   const size_t smem = (size_t)8 * S * C * sizeof(float);
   static bool attr = false;
+  static int grid_c = -1, grid = kLnBlocks;
   if (!attr) {
     cudaFuncSetAttribute(ln_bwd_kernel<N, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          8 * S * 2048 * 4 > 227 * 1024 ? 227 * 1024 : 8 * S * 2048 * 4);
     attr = true;
   }
-  ln_bwd_kernel<N, S><<<kLnBlocks, 256, smem, s>>>(dres, dy, x, mean, rstd, g, partials, M, C,
-                                                   accumulate);
+  if (grid_c != C) {
+    int per_sm = 0, sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_bwd_kernel<N, S>, 256, smem);
+    grid = per_sm * sms;
+    if (grid < 1 || grid > kLnBlocks) grid = kLnBlocks;
+    grid_c = C;
+  }
+  ln_bwd_kernel<N, S><<<grid, 256, smem, s>>>(dres, dy, x, mean, rstd, g, partials, M, C,
+                                              accumulate);
+  return grid;
 }
 
 }  // namespace
@@ -227,20 +250,21 @@ void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* me
                    const float* rstd, const float* g, float* dg, float* db, float* dbias_out,
                    float* partials, int M, int C, int accumulate, cudaStream_t s) {
   const int nsums = dbias_out ? 3 : 2;
+  int nblk = kLnBlocks;
   switch ((C + 255) / 256 * 4 + nsums) {
 #define GPT2_LNB(N)                                                                          \
   case 4 * N + 2:                                                                            \
-    ln_bwd_launch<N, 2>(dres, dy, x, mean, rstd, g, partials, M, C, accumulate, s);          \
+    nblk = ln_bwd_launch<N, 2>(dres, dy, x, mean, rstd, g, partials, M, C, accumulate, s);   \
     break;                                                                                   \
   case 4 * N + 3:                                                                            \
-    ln_bwd_launch<N, 3>(dres, dy, x, mean, rstd, g, partials, M, C, accumulate, s);          \
+    nblk = ln_bwd_launch<N, 3>(dres, dy, x, mean, rstd, g, partials, M, C, accumulate, s);   \
     break;
     GPT2_LNB(1) GPT2_LNB(2) GPT2_LNB(3) GPT2_LNB(4) GPT2_LNB(5) GPT2_LNB(6) GPT2_LNB(7) GPT2_LNB(8)
 #undef GPT2_LNB
     default: break;
   }
-  ln_bwd_reduce_kernel<<<(nsums * C + 31) / 32, 1024, 0, s>>>(dg, db, dbias_out, partials,
-                                                               kLnBlocks, nsums, C);
+  ln_bwd_reduce_kernel<<<(nsums * C + 31) / 32, 1024, 0, s>>>(dg, db, dbias_out, partials, nblk,
+                                                               nsums, C);
   note_launch(2);
 }
 

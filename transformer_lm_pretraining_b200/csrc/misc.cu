@@ -4,6 +4,7 @@
 #include <atomic>
 
 #include "kernels.h"
+#include "tc_util.cuh"
 
 namespace gpt2k {
 
@@ -127,7 +128,8 @@ __device__ __forceinline__ void online_merge(float& m, float& s, float m2, float
 
 __global__ void __launch_bounds__(kClsThreads)
     classifier_kernel(act_t* __restrict__ logits, float* __restrict__ losses,
-                      const int* __restrict__ tgt, int M, int V, int Vp, int* err) {
+                      const int* __restrict__ tgt, int M, int V, int Vp, int write_grad,
+                      int* err) {
   const int row = blockIdx.x;
   act_t* z = logits + (size_t)row * Vp;
   const int vec = (Vp % 8 == 0) ? 8 : 1;
@@ -171,6 +173,7 @@ __global__ void __launch_bounds__(kClsThreads)
     t = 0;
   }
   if (threadIdx.x == 0) losses[row] = lse - to_f(z[t]);
+  if (!write_grad) return;
   __syncthreads();  // the target logit is read before it is overwritten
   const float inv = 1.0f / (float)M;
   if (vec == 8) {
@@ -188,6 +191,130 @@ __global__ void __launch_bounds__(kClsThreads)
     for (int c = threadIdx.x; c < Vp; c += kClsThreads) {
       const float v = to_f(z[c]);
       z[c] = from_f<act_t>(c < V ? (__expf(v - lse) - (c == t ? 1.f : 0.f)) * inv : 0.f);
+    }
+  }
+}
+
+// Persistent variant for rows that fit twice in shared memory: one CTA per
+// SM takes rows blockIdx.x, + gridDim.x, ...; each row arrives with one
+// bulk copy, a row ahead of its use (two buffers), so HBM sees one read and
+// one write of the logits.  Three passes over shared memory: the max, the
+// sum of exponentials (per-thread partials over a fixed column assignment,
+// then warps in order), then z <- (softmax - onehot) / M written straight to
+// global memory (skipped when write_grad == 0).  Separate max and sum
+// passes keep every exponential independent of the others (a running max
+// would chain them).
+constexpr int kClsBulkThreads = 1024;
+
+__device__ __forceinline__ float block_reduce_cls(float v, float* red, bool is_max) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? fmaxf(v, w) : v + w;
+  }
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int w = 1; w < kClsBulkThreads / 32; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  __syncthreads();  // red is reused by the next reduction
+  return r;
+}
+
+__global__ void __launch_bounds__(kClsBulkThreads, 1)
+    classifier_bulk_kernel(act_t* __restrict__ logits, float* __restrict__ losses,
+                           const int* __restrict__ tgt, int M, int V, int Vp, int write_grad,
+                           int* err) {
+  using namespace tc;
+  extern __shared__ __align__(128) uint8_t cls_smem[];
+  __shared__ float red[kClsBulkThreads / 32];
+  __shared__ uint64_t bars[2];
+  __shared__ int abort_s;
+  const uint32_t row_bytes = (uint32_t)Vp * sizeof(act_t);
+  const uint32_t buf_stride = (row_bytes + 127u) & ~127u;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    mbar_init(smem_u32(&bars[0]), 1);
+    mbar_init(smem_u32(&bars[1]), 1);
+    abort_s = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto issue = [&](int b, int r) {
+    const uint32_t bar = smem_u32(&bars[b]);
+    mbar_expect_tx(bar, row_bytes);
+    bulk_load_1d(smem_u32(cls_smem + b * buf_stride), logits + (size_t)r * Vp, row_bytes, bar);
+  };
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b)
+      if (blockIdx.x + b * gridDim.x < M) issue(b, blockIdx.x + b * gridDim.x);
+  }
+  const float inv = 1.0f / (float)M;
+  constexpr float kLog2e = 1.4426950408889634f;
+  uint32_t phase = 0;  // bit b: parity of buffer b's next fill
+  int it = 0;
+  for (int row = blockIdx.x; row < M; row += gridDim.x, ++it) {
+    const int b = it & 1;
+    const bool got = mbar_wait(smem_u32(&bars[b]), (phase >> b) & 1u, &abort_s, err);
+    if (!__syncthreads_and(got)) break;
+    phase ^= 1u << b;
+    const act_t* z = reinterpret_cast<const act_t*>(cls_smem + b * buf_stride);
+    float mx = -INFINITY;
+    for (int c = tid * 8; c < Vp; c += kClsBulkThreads * 8) {
+      float v[8];
+      load8(z + c, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (c + i < V) mx = fmaxf(mx, v[i]);
+    }
+    mx = block_reduce_cls(mx, red, true);
+    const float mx2 = mx * kLog2e;
+    float sm = 0.f;
+    for (int c = tid * 8; c < Vp; c += kClsBulkThreads * 8) {
+      float v[8];
+      load8(z + c, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (c + i < V) sm += fast_exp2(fmaf(v[i], kLog2e, -mx2));
+    }
+    sm = block_reduce_cls(sm, red, false);
+    const float lse = mx + logf(sm);
+    int t = tgt[row];
+    if (t < 0 || t >= V) {
+      if (tid == 0) atomicOr(err, ERR_TARGET);
+      t = 0;
+    }
+    if (tid == 0) losses[row] = lse - to_f(z[t]);
+    if (write_grad) {
+      const float lse2 = lse * kLog2e;
+      act_t* out = logits + (size_t)row * Vp;
+      for (int c = tid * 8; c < Vp; c += kClsBulkThreads * 8) {
+        float v[8];
+        load8(z + c, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int col = c + i;
+          v[i] = col < V ? (fast_exp2(fmaf(v[i], kLog2e, -lse2)) - (col == t ? 1.f : 0.f)) * inv
+                         : 0.f;
+        }
+        store8(out + c, v);
+      }
+    }
+    __syncthreads();  // every read of buffer b is done
+    if (tid == 0 && row + 2 * gridDim.x < M) {
+      fence_async_smem();
+      issue(b, row + 2 * gridDim.x);
+    }
+  }
+  // copies still in flight land before the shared memory is released
+  if (tid == 0) {
+    const uint64_t t0 = global_ns();
+    for (int k = 0; k < 2; ++k) {
+      const int r = blockIdx.x + (it + k) * gridDim.x;
+      if (r >= M) break;
+      while (!mbar_try_wait(smem_u32(&bars[(it + k) & 1]), (phase >> ((it + k) & 1)) & 1u) &&
+             global_ns() - t0 < kWaitLimitNs) {
+      }
     }
   }
 }
@@ -376,9 +503,28 @@ void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaS
   note_launch(2);
 }
 
-void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int Vp, int* err,
-                cudaStream_t s) {
-  classifier_kernel<<<M, kClsThreads, 0, s>>>(logits, losses, tgt, M, V, Vp, err);
+void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int Vp, int write_grad,
+                int* err, cudaStream_t s) {
+  if (M <= 0) return;
+  const size_t row_bytes = (size_t)Vp * sizeof(act_t);
+  const size_t smem = 2 * ((row_bytes + 127) & ~(size_t)127);
+  if (smem <= 200 * 1024 && row_bytes % 16 == 0 &&
+      (reinterpret_cast<uintptr_t>(logits) & 15) == 0) {
+    static size_t attr = 0;
+    if (attr < smem) {
+      cudaFuncSetAttribute(classifier_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+      attr = smem;
+    }
+    int sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = M < sms ? M : sms;
+    classifier_bulk_kernel<<<grid, kClsBulkThreads, smem, s>>>(logits, losses, tgt, M, V, Vp,
+                                                                 write_grad, err);
+  } else {
+    classifier_kernel<<<M, kClsThreads, 0, s>>>(logits, losses, tgt, M, V, Vp, write_grad, err);
+  }
   note_launch();
 }
 
