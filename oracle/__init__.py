@@ -102,6 +102,12 @@ def lib(openmp: bool = False) -> ctypes.CDLL:
         fn = getattr(L, f"orc_layernorm_fwd_{sfx}")
         fn.argtypes = [P, P, P, P, P, P, i, i]
         fn.restype = None
+        fn = getattr(L, f"orc_layernorm_bwd_{sfx}")
+        fn.argtypes = [P, P, P, P, P, P, P, P, i, i]
+        fn.restype = None
+        fn = getattr(L, f"orc_softmax_xent_{sfx}")
+        fn.argtypes = [P, i, i, _I32, R, P, P]
+        fn.restype = None
         fn = getattr(L, f"orc_attention_fwd_{sfx}")
         fn.argtypes = [P, P, i, i, i, i]
         fn.restype = None
@@ -277,6 +283,34 @@ class Oracle:
             _ptr(np.ascontiguousarray(b, self.dtype), self.ct), _ptr(y, self.ct),
             _ptr(mean, self.ct), _ptr(rstd, self.ct), M, C)
         return y, mean, rstd
+
+    def layernorm_bwd(self, x, g, mean, rstd, dy):
+        """(dx, dg, db) of the LayerNorm backward (dx from zero)."""
+        x = np.ascontiguousarray(x, self.dtype)
+        M, C = x.shape
+        dx = np.zeros_like(x)
+        dg = np.zeros(C, self.dtype)
+        db = np.zeros(C, self.dtype)
+        getattr(self.lib, f"orc_layernorm_bwd_{self.sfx}")(
+            _ptr(x, self.ct), _ptr(np.ascontiguousarray(g, self.dtype), self.ct),
+            _ptr(np.ascontiguousarray(mean, self.dtype), self.ct),
+            _ptr(np.ascontiguousarray(rstd, self.dtype), self.ct),
+            _ptr(np.ascontiguousarray(dy, self.dtype), self.ct), _ptr(dx, self.ct),
+            _ptr(dg, self.ct), _ptr(db, self.ct), M, C)
+        return dx, dg, db
+
+    def softmax_xent(self, z, tgt, scale=1.0, grad=True):
+        """(losses, dz) of softmax cross-entropy over rows of z [M, V]; dz =
+        (softmax - onehot) * scale / M, or None when grad is False."""
+        z = np.ascontiguousarray(z, self.dtype)
+        M, V = z.shape
+        t = np.ascontiguousarray(tgt, np.int32)
+        losses = np.zeros(M, self.dtype)
+        dz = np.zeros_like(z) if grad else None
+        getattr(self.lib, f"orc_softmax_xent_{self.sfx}")(
+            _ptr(z, self.ct), M, V, t.ctypes.data_as(_I32),
+            self.ct(scale), _ptr(losses, self.ct), _ptr(dz, self.ct) if grad else None)
+        return losses, dz
 
     def linear_fwd(self, x, W, b=None):
         x = np.ascontiguousarray(x, self.dtype)

@@ -353,6 +353,33 @@ void attention_bwd(const R* qkv, const R* dy, R* dqkv, int B, int T, int C,
 }
 
 // ----------------------------------------------------------------- model --
+// log sum_v exp(z[v]) over the first V logits of a row (max-shifted).
+template <class R>
+R row_lse(const R* z, int V) {
+  R mx = -INFINITY;
+  for (int v = 0; v < V; ++v) mx = std::max(mx, z[v]);
+  R s = 0;
+  for (int v = 0; v < V; ++v) s += std::exp(z[v] - mx);
+  return mx + std::log(s);
+}
+
+// Softmax cross-entropy of M rows of V logits: losses[m] = lse_m - z[tgt[m]]
+// and, when dz is given, dz = (softmax - onehot(tgt)) * scale / M.
+template <class R>
+void softmax_xent(const R* z, int M, int V, const int* tgt, R scale, R* losses, R* dz) {
+  for (int m = 0; m < M; ++m) {
+    const R* zr = z + (size_t)m * V;
+    const R lse = row_lse(zr, V);
+    if (losses) losses[m] = lse - zr[tgt[m]];
+    if (!dz) continue;
+    for (int v = 0; v < V; ++v) {
+      R d = std::exp(zr[v] - lse);
+      if (v == tgt[m]) d -= R(1);
+      dz[(size_t)m * V + v] = d * scale / R(M);
+    }
+  }
+}
+
 template <class R>
 struct Model {
   Cfg g;
@@ -429,17 +456,9 @@ struct Model {
                C, V);
     if (!tgt) return 0;
     lossv.resize(M);
+    softmax_xent(logits.data(), M, V, tgt, R(1), lossv.data(), (R*)nullptr);
     R total = 0;
-    for (int m = 0; m < M; ++m) {
-      const R* z = logits.data() + (size_t)m * V;
-      R mx = -INFINITY;
-      for (int v = 0; v < V; ++v) mx = std::max(mx, z[v]);
-      R s = 0;
-      for (int v = 0; v < V; ++v) s += std::exp(z[v] - mx);
-      const R lse = mx + std::log(s);
-      lossv[m] = lse - z[tgt[m]];
-      total += lossv[m];
-    }
+    for (int m = 0; m < M; ++m) total += lossv[m];
     return total / M;
   }
 
@@ -449,19 +468,7 @@ struct Model {
     const size_t MC = (size_t)M * C;
     // softmax cross-entropy: dz = (softmax - onehot) * scale / M
     std::vector<R> dz((size_t)M * V);
-    for (int m = 0; m < M; ++m) {
-      const R* z = logits.data() + (size_t)m * V;
-      R mx = -INFINITY;
-      for (int v = 0; v < V; ++v) mx = std::max(mx, z[v]);
-      R s = 0;
-      for (int v = 0; v < V; ++v) s += std::exp(z[v] - mx);
-      const R lse = mx + std::log(s);
-      for (int v = 0; v < V; ++v) {
-        R d = std::exp(z[v] - lse);
-        if (v == tgt[m]) d -= R(1);
-        dz[(size_t)m * V + v] = d * loss_scale / R(M);
-      }
-    }
+    softmax_xent(logits.data(), M, V, tgt, loss_scale, (R*)nullptr, dz.data());
     std::vector<R> dhf(MC, 0), dx(MC, 0);
     linear_bwd(hf.data(), p + g.off[WTE], dz.data(), dhf.data(),
                grad + g.off[WTE], (R*)nullptr, M, C, V);
@@ -633,6 +640,15 @@ uint64_t orc_splitmix64(uint64_t seed, uint64_t n) { return sm_output(seed, n); 
   void orc_layernorm_fwd_##SFX(const R* x, const R* g, const R* b, R* y,       \
                                R* mean, R* rstd, int M, int C) {               \
     layernorm_fwd<R>(x, g, b, y, mean, rstd, M, C);                            \
+  }                                                                            \
+  void orc_layernorm_bwd_##SFX(const R* x, const R* g, const R* mean,         \
+                               const R* rstd, const R* dy, R* dx, R* dg, R* db, \
+                               int M, int C) {                                 \
+    layernorm_bwd<R>(x, g, mean, rstd, dy, dx, dg, db, M, C);                  \
+  }                                                                            \
+  void orc_softmax_xent_##SFX(const R* z, int M, int V, const int* tgt,        \
+                              R scale, R* losses, R* dz) {                     \
+    softmax_xent<R>(z, M, V, tgt, scale, losses, dz);                          \
   }                                                                            \
   void orc_attention_fwd_##SFX(const R* qkv, R* y, int B, int T, int C,        \
                                int H) {                                        \

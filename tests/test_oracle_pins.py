@@ -209,6 +209,61 @@ def test_layernorm_output_moments():
 
 
 # ------------------------------------------------------------------ GELU ---
+def test_layernorm_backward_matches_central_differences():
+    # L = sum(w * LN(x)) for a fixed w: dL/dx, dL/dg, dL/db by central
+    # differences of the forward against the backward with dy = w
+    o = Oracle(Config(1, 1, 8, 11, 11, 4))
+    rng = np.random.default_rng(5)
+    M, C = 3, 8
+    x = rng.standard_normal((M, C))
+    g = 1.0 + 0.3 * rng.standard_normal(C)
+    b = 0.1 * rng.standard_normal(C)
+    w = rng.standard_normal((M, C))
+    _, mean, rstd = o.layernorm_fwd(x, g, b)
+    dx, dg, db = o.layernorm_bwd(x, g, mean, rstd, w)
+
+    def loss(x_, g_, b_):
+        return float((w * o.layernorm_fwd(x_, g_, b_)[0]).sum())
+
+    h = 1e-6
+    for arr, grad in ((x, dx), (g, dg), (b, db)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            e = np.zeros_like(arr)
+            e[idx] = h
+            args = [x, g, b]
+            k = next(i for i, a in enumerate(args) if a is arr)
+            args_p = list(args); args_p[k] = arr + e
+            args_m = list(args); args_m[k] = arr - e
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        assert np.allclose(grad, num, rtol=1e-6, atol=1e-7)
+    # shifting a row leaves LN unchanged: each row of dx sums to zero
+    assert np.allclose(dx.sum(axis=1), 0.0, atol=1e-12)
+
+
+def test_softmax_xent_closed_forms():
+    o = Oracle(Config(1, 1, 8, 11, 11, 4))
+    # uniform logits: loss = ln V, dz = (1/V - onehot) * scale / M exactly
+    M, V, scale = 4, 7, 0.5
+    z = np.full((M, V), 1.25)
+    t = np.array([0, 3, 6, 2])
+    losses, dz = o.softmax_xent(z, t, scale)
+    assert np.allclose(losses, math.log(V), rtol=0, atol=1e-15)
+    want = (np.full((M, V), 1.0 / V) - np.eye(V)[t]) * scale / M
+    assert np.allclose(dz, want, rtol=0, atol=1e-16)
+    # two classes: loss = softplus(z_other - z_target); rows of dz sum to 0
+    rng = np.random.default_rng(6)
+    z2 = rng.standard_normal((5, 2)) * 3
+    t2 = rng.integers(0, 2, 5)
+    l2, d2 = o.softmax_xent(z2, t2, 1.0)
+    other = z2[np.arange(5), 1 - t2] - z2[np.arange(5), t2]
+    assert np.allclose(l2, np.log1p(np.exp(other)), rtol=1e-14)
+    assert np.allclose(d2.sum(axis=1), 0.0, atol=1e-16)
+    # no gradient requested: losses only
+    l3, d3 = o.softmax_xent(z2, t2, 1.0, grad=False)
+    assert d3 is None and np.array_equal(l3, l2)
+
+
 def test_gelu_identities():
     o = Oracle(Config(1, 1, 8, 11, 11, 4))
     xs = np.linspace(-8, 8, 321)
