@@ -56,8 +56,38 @@ int gpt2k_attention_fwd(void* stream, void* att, float* lse, const void* qkv, in
 int gpt2k_attention_bwd(void* stream, void* dqkv, float* dsum, const void* datt, const void* qkv,
                         const void* att, const float* lse, int B, int T, int C, int H);
 
-/* Device error word of the kernel-level calls (bit 2: a bounded wait in a
- * GEMM expired); read and cleared.  Synchronous. */
+/* LayerNorm forward over the rows of x [M, C] (first page, layer structure;
+ * eps 1e-5, biased variance): y = (x - mean) rstd g + b in the activation
+ * dtype, mean and rstd [M] fp32 kept for the backward; g, b fp32 [C].
+ * C must be a multiple of 8 and at most 2048; x, y 16-byte aligned. */
+int gpt2k_layernorm_fwd(void* stream, void* y, float* mean, float* rstd, const void* x,
+                        const float* g, const float* b, int M, int C);
+
+/* Its backward (the chain rule through y): with dxhat = dy g and xhat =
+ * (x - mean) rstd, dx = (accumulate ? dx : 0) + rstd (dxhat - mean_c(dxhat)
+ * - xhat mean_c(dxhat xhat)); dg += sum_m dy xhat; db += sum_m dy; and, if
+ * dsum is not NULL, dsum += sum_m dx as stored (the bias gradient of the
+ * projection that produced x's residual).  The column sums add per-block
+ * partials in a fixed order (bit-reproducible).  partials is fp32 scratch
+ * of gpt2k_layernorm_bwd_scratch(C) floats.  Shape rules as the forward. */
+int gpt2k_layernorm_bwd(void* stream, void* dx, const void* dy, const void* x, const float* mean,
+                        const float* rstd, const float* g, float* dg, float* db, float* dsum,
+                        float* partials, int M, int C, int accumulate);
+size_t gpt2k_layernorm_bwd_scratch(int C);
+
+/* Softmax cross-entropy over the rows of logits [M, Vp] (activation dtype),
+ * classes 0 .. V-1 (the padded columns V .. Vp-1 are excluded; condensed
+ * GPT-2 page, vocabulary padding): losses[m] = logsumexp(z_m[0:V]) -
+ * z_m[tgt[m]] (fp32); if write_grad, the logits are overwritten with
+ * (softmax - onehot(tgt)) / M for columns < V and 0 for the padding.  A
+ * target outside [0, V) is read as 0 and sets error bit value 2.  Vp must
+ * be a multiple of 8 and logits 16-byte aligned. */
+int gpt2k_classifier(void* stream, void* logits, float* losses, const int* tgt, int M, int V,
+                     int Vp, int write_grad);
+
+/* Device error word of the kernel-level calls (bit value 2: a bad target;
+ * 4: a bounded wait in a tensor-core kernel expired); read and cleared.
+ * Synchronous. */
 int gpt2k_take_error(void);
 
 /* Size, in floats, of the fixed scratch array behind

@@ -1,23 +1,26 @@
 // Causal flash-attention forward on the sm_100a tensor cores (head dim 64).
 //
-// One CTA per (query tile of 128 rows, batch, head), heaviest tiles first;
-// 10 warps:
-//   warp 0     TMA: the Q tile once, then K/V tiles of 128 keys into a
-//              3-stage shared-memory ring (128-byte swizzle, zero fill past
-//              the sequence);
-//   warp 1     TMEM owner and MMA issuer: S_j = Q K_j^T (M=128, N=128,
-//              K=64) into one of two TMEM buffers, and O_j = P_j V_j
-//              (M=128, N=64, K=128; V read MN-major straight from its tile)
-//              into one of two more;
-//   warps 2-9  softmax: two threads per query row (warps w and w+4 share a
-//              TMEM lane quarter), each owning 64 of the 128 key columns and
-//              32 of the 64 output dimensions.  They read S_j from TMEM,
-//              agree on the running row max through shared memory, write
-//              P_j = 2^(S_j log2e/sqrt(d) - m) as bf16 into a swizzled tile
-//              (the next MMA's A operand), and fold O_{j-1} into fp32 row
-//              accumulators held in registers with the pending rescale
-//              factor.  S_{j+1} and O_{j-1} are computed by the tensor core
-//              while tile j's softmax runs.
+// Persistent: one CTA per SM walks a static list of work items, each a pair
+// of adjacent 128-row query tiles (A = 2p, B = 2p + 1) of one (batch, head).
+// Items are ordered heaviest first and dealt to the CTAs in a snake order,
+// which balances the causal work across SMs.  10 warps:
+//   warp 0     TMA: the item's two Q tiles, then its K/V tiles of 128 keys
+//              into a 3-stage ring (128-byte swizzle, zero fill past the
+//              sequence), running ahead into the next item;
+//   warp 1     TMEM owner and MMA issuer: S_t = Q_t K_j^T (M=128, N=128,
+//              K=64) into one TMEM buffer per tile t, and O_t += P_t V_j
+//              (M=128, N=64, K=128; V read MN-major from its tile), O_t
+//              accumulated in TMEM over the item's key tiles.  S for key
+//              tile j+1 is issued before PV for key tile j, so the next
+//              scores are ready when a softmax ends;
+//   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: one thread
+//              per query row.  Each reads its row of S from TMEM twice (the
+//              max, then the exponentials) and writes P = 2^(S log2e /
+//              sqrt(d) - m) as bf16 into a swizzled tile (the next MMA's A
+//              operand).  The reference max m is raised only when a tile's
+//              max exceeds it by more than 2^8 (P stays below 256); then the
+//              row of O in TMEM and the running sum are rescaled first.  No
+//              thread waits for another thread's row.
 // T x T is never materialised.  The output row is normalised by the
 // running sum; the natural-log log-sum-exp of each row is stored for the
 // backward pass.  Every wait is bounded (error word ERR_TIMEOUT).
@@ -38,71 +41,80 @@ namespace {
 using namespace tc;
 using attn::kHD;
 using attn::kBox;
+using attn::kTile;
 
-constexpr int kTileQ = attn::kTile;
-constexpr int kTileK = attn::kTile;
 constexpr int kKVStages = 3;
-constexpr int kSoftmaxThreads = attn::kComputeThreads;
-constexpr int kThreadsAttn = 64 + kSoftmaxThreads;
-constexpr uint32_t kTmemCols = 512;  // S: 2 x 128, O: 2 x 64
-constexpr int kAux = 4096;           // barriers + cross-thread row scratch
+constexpr int kRowThreads = 128;  // softmax threads per query tile
+constexpr int kThreadsAttn = 64 + 2 * kRowThreads;
+constexpr uint32_t kTmemCols = 512;  // S: 2 tiles x 128; O: 2 tiles x 64
+constexpr uint32_t kOCol = 2 * kTile;
+constexpr float kRescaleLog2 = 8.0f;  // raise the reference max past this margin
+constexpr int kAux = 1024;  // barriers
 
 constexpr size_t attn_smem_bytes() {
-  // Q, K ring, V ring, P double buffer (two 64-key boxes each), aux
-  return 1024 + kBox + 2 * (size_t)kKVStages * kBox + 2 * 2 * (size_t)kBox + kAux;
+  // Q (two tiles), K ring, V ring, P (two tiles of two 64-key boxes), aux
+  return 1024 + 2 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + 4 * (size_t)kBox + kAux;
 }
 
-__device__ __forceinline__ void sm_bar() { named_bar<1, kSoftmaxThreads>(); }
-__device__ __forceinline__ bool sm_bar_and(bool pred) {
-  return named_bar_and<1, kSoftmaxThreads>(pred);
+// Work item k of this CTA (snake order over the heaviest-first item list);
+// false when the CTA has no item k.
+struct FwdItem {
+  int b, h, qa, qb, nkv_a, nkv_b;  // nkv_b = 0: no tile B
+};
+__device__ __forceinline__ bool fwd_item(int k, int B, int H, int nq, FwdItem& it) {
+  const int G = gridDim.x;
+  const int w = k * G + ((k & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+  const int BH = B * H;
+  const int npairs = (nq + 1) >> 1;
+  if (w >= npairs * BH) return false;
+  const int p = npairs - 1 - w / BH, bh = w % BH;
+  it.b = bh / H;
+  it.h = bh % H;
+  it.qa = 2 * p;
+  it.qb = 2 * p + 1;
+  it.nkv_a = it.qa + 1;
+  it.nkv_b = it.qb < nq ? it.qb + 1 : 0;
+  return true;
 }
 
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     flash_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, __nv_bfloat16* __restrict__ att,
-                        float* __restrict__ lse, int T, int C, int H, float sl2, int* err) {
+                        float* __restrict__ lse, int B, int T, int C, int H, float sl2, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kBox;                      // [kKVStages][kBox]
+  uint8_t* sQ = smem;                           // [2 tiles][kBox]
+  uint8_t* sK = sQ + 2 * kBox;                  // [kKVStages][kBox]
   uint8_t* sV = sK + kKVStages * kBox;          // [kKVStages][kBox]
-  uint8_t* sP = sV + kKVStages * kBox;          // [2][2 boxes]
-  uint8_t* aux = sP + 4 * kBox;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
+  uint8_t* sP = sV + kKVStages * kBox;          // [2 tiles][2 boxes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 4 * kBox);
   const uint32_t q_full = smem_u32(bars + 0);
-  const uint32_t kv_full0 = smem_u32(bars + 1);                  // [3]
-  const uint32_t kv_empty0 = smem_u32(bars + 1 + kKVStages);     // [3]
-  const uint32_t s_full0 = smem_u32(bars + 1 + 2 * kKVStages);   // [2]
-  const uint32_t s_empty0 = s_full0 + 16;                        // [2]
-  const uint32_t p_full0 = s_full0 + 32;                         // [2]
-  const uint32_t p_empty0 = s_full0 + 48;                        // [2]
-  const uint32_t o_full0 = s_full0 + 64;                         // [2]
-  const uint32_t o_empty0 = s_full0 + 80;                        // [2]
-  const uint32_t drain = s_full0 + 96;                           // abort path only
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 1 + 2 * kKVStages + 13);
+  const uint32_t q_empty = smem_u32(bars + 1);
+  const uint32_t kv_full0 = smem_u32(bars + 2);                  // [3]
+  const uint32_t kv_empty0 = smem_u32(bars + 2 + kKVStages);     // [3]
+  const uint32_t s_full0 = smem_u32(bars + 2 + 2 * kKVStages);   // [2 tiles]
+  const uint32_t s_empty0 = s_full0 + 16;                        // [2 tiles]
+  const uint32_t p_full0 = s_full0 + 32;                         // [2 tiles]
+  const uint32_t o_full0 = s_full0 + 48;                         // [2 tiles]
+  const uint32_t drain = s_full0 + 64;                           // abort path only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red_max = reinterpret_cast<float*>(aux + 512);   // [2 parity][2 halves][128 rows]
-  float* red_l = red_max + 2 * 2 * kTileQ;                // [2 halves][128 rows]
 
-  const int qb = gridDim.x - 1 - blockIdx.x;  // heaviest query tiles first
-  const int b = blockIdx.y / H, h = blockIdx.y % H;
-  const int q0 = qb * kTileQ;
-  const int nkv = qb + 1;  // causal: key tiles 0 .. qb
+  const int nq = (T + kTile - 1) / kTile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < kKVStages; ++s) {
       mbar_init(kv_full0 + 8 * s, 1);
       mbar_init(kv_empty0 + 8 * s, 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full0 + 8 * i, 1);
-      mbar_init(s_empty0 + 8 * i, kSoftmaxThreads);
-      mbar_init(p_full0 + 8 * i, kSoftmaxThreads);
-      mbar_init(p_empty0 + 8 * i, 1);
-      mbar_init(o_full0 + 8 * i, 1);
-      mbar_init(o_empty0 + 8 * i, kSoftmaxThreads);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(s_full0 + 8 * t, 1);
+      mbar_init(s_empty0 + 8 * t, kRowThreads);
+      mbar_init(p_full0 + 8 * t, kRowThreads);
+      mbar_init(o_full0 + 8 * t, 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -123,29 +135,39 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     if (lane == 0) {
       // ------------------------------------------------------------ TMA --
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
-      mbar_expect_tx(q_full, kBox);
-      tma_load_3d(smem_u32(sQ), &tmQKV, q_full, h * kHD, q0, b);
-      int stage = 0;
-      uint32_t phase = 0;
+      uint32_t n_item = 0, q_issued = 0;
+      uint32_t g = 0;  // K/V tiles loaded so far (ring position)
       uint32_t issued = 0, last_parity = 0;
-      for (int j = 0; j < nkv; ++j) {
-        if (!mbar_wait(kv_empty0 + 8 * stage, phase ^ 1u, abort_flag, err)) break;
-        const uint32_t fb = kv_full0 + 8 * stage;
-        mbar_expect_tx(fb, 2 * kBox);
-        tma_load_3d(smem_u32(sK + stage * kBox), &tmQKV, fb, C + h * kHD, j * kTileK, b);
-        tma_load_3d(smem_u32(sV + stage * kBox), &tmQKV, fb, 2 * C + h * kHD, j * kTileK, b);
-        issued |= 1u << stage;
-        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kKVStages) {
-          stage = 0;
-          phase ^= 1u;
+      bool ok = true;
+      FwdItem it;
+      for (int k = 0; ok && fwd_item(k, B, H, nq, it); ++k, ++n_item) {
+        if (!mbar_wait(q_empty, (n_item & 1u) ^ 1u, abort_flag, err)) break;
+        mbar_expect_tx(q_full, it.nkv_b ? 2 * kBox : kBox);
+        tma_load_3d(smem_u32(sQ), &tmQKV, q_full, it.h * kHD, it.qa * kTile, it.b);
+        if (it.nkv_b) tma_load_3d(smem_u32(sQ + kBox), &tmQKV, q_full, it.h * kHD, it.qb * kTile, it.b);
+        q_issued = n_item + 1;
+        const int nkv = it.nkv_b ? it.nkv_b : it.nkv_a;
+        for (int j = 0; j < nkv; ++j, ++g) {
+          const int st = g % kKVStages;
+          const uint32_t ph = (g / kKVStages) & 1u;
+          if (!mbar_wait(kv_empty0 + 8 * st, ph ^ 1u, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = kv_full0 + 8 * st;
+          mbar_expect_tx(fb, 2 * kBox);
+          tma_load_3d(smem_u32(sK + st * kBox), &tmQKV, fb, C + it.h * kHD, j * kTile, it.b);
+          tma_load_3d(smem_u32(sV + st * kBox), &tmQKV, fb, 2 * C + it.h * kHD, j * kTile, it.b);
+          issued |= 1u << st;
+          last_parity = (last_parity & ~(1u << st)) | (ph << st);
         }
       }
       // every copy issued lands before the shared memory is released (the
       // MMA warp has already waited for all of them unless it gave up)
       const uint64_t t0 = global_ns();
-      while (!mbar_try_wait(q_full, 0) && global_ns() - t0 < kWaitLimitNs) {
-      }
+      if (q_issued)
+        while (!mbar_try_wait(q_full, (q_issued - 1) & 1u) && global_ns() - t0 < kWaitLimitNs) {
+        }
       for (int s2 = 0; s2 < kKVStages; ++s2) {
         if (!(issued & (1u << s2))) continue;
         while (!mbar_try_wait(kv_full0 + 8 * s2, (last_parity >> s2) & 1u) &&
@@ -156,47 +178,61 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA --
-      constexpr uint32_t idS = attn::idesc(kTileK, false);
+      constexpr uint32_t idS = attn::idesc(kTile, false);
       constexpr uint32_t idO = attn::idesc(kHD, true);
-      bool ok = mbar_wait(q_full, 0, abort_flag, err);
-      tc_fence_after();
-      const uint32_t q_base = smem_u32(sQ);
-      // S_j: stage j % 3, S buffer j % 2
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kKVStages, sb = j & 1;
-        if (!mbar_wait(kv_full0 + 8 * st, (uint32_t)(j / kKVStages) & 1u, abort_flag, err)) return false;
-        if (!mbar_wait(s_empty0 + 8 * sb, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, err)) return false;
+      uint32_t n_item = 0, g = 0;
+      uint32_t cs[2] = {0, 0}, co[2] = {0, 0};  // S / PV products issued per tile
+      bool ok = true;
+      // S_t = Q_t K (key tile in ring stage st)
+      auto issue_s = [&](int t, int st) -> bool {
+        if (!mbar_wait(s_empty0 + 8 * t, (cs[t] & 1u) ^ 1u, abort_flag, err)) return false;
         tc_fence_after();
-        const uint32_t k_base = smem_u32(sK + st * kBox);
+        const uint32_t q_base = smem_u32(sQ + t * kBox), k_base = smem_u32(sK + st * kBox);
 #pragma unroll
         for (int k = 0; k < kHD / 16; ++k)
-          tc_mma(tmem + (uint32_t)(sb * kTileK), desc_kmajor(q_base, k), desc_kmajor(k_base, k), idS,
+          tc_mma(tmem + (uint32_t)(t * kTile), desc_kmajor(q_base, k), desc_kmajor(k_base, k), idS,
                  k > 0 ? 1u : 0u);
-        tc_commit(s_full0 + 8 * sb);
+        tc_commit(s_full0 + 8 * t);
+        ++cs[t];
         return true;
       };
-      // O_j = P_j V_j: P buffer j % 2, V stage j % 3, O buffer j % 2
-      auto issue_o = [&](int j) -> bool {
-        const int st = j % kKVStages, pb = j & 1;
-        if (!mbar_wait(p_full0 + 8 * pb, (uint32_t)(j >> 1) & 1u, abort_flag, err)) return false;
-        if (!mbar_wait(o_empty0 + 8 * pb, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, err)) return false;
+      // O_t (+)= P_t V (value tile in ring stage st); the item's first
+      // product initialises O_t
+      auto issue_pv = [&](int t, int st, bool first) -> bool {
+        if (!mbar_wait(p_full0 + 8 * t, co[t] & 1u, abort_flag, err)) return false;
         tc_fence_after();
-        const uint32_t p_base = smem_u32(sP + pb * 2 * kBox);
-        const uint32_t v_base = smem_u32(sV + st * kBox);
+        const uint32_t p_base = smem_u32(sP + t * 2 * kBox), v_base = smem_u32(sV + st * kBox);
 #pragma unroll
-        for (int k = 0; k < kTileK / 16; ++k)
-          tc_mma(tmem + 2u * kTileK + (uint32_t)(pb * kHD),
-                 desc_kmajor(p_base + (uint32_t)((k >> 2) * kBox), k & 3), desc_mnmajor(v_base, k), idO,
-                 k > 0 ? 1u : 0u);
-        tc_commit(o_full0 + 8 * pb);
-        tc_commit(p_empty0 + 8 * pb);
-        tc_commit(kv_empty0 + 8 * st);  // K_j and V_j are no longer read
+        for (int k = 0; k < kTile / 16; ++k)
+          tc_mma(tmem + kOCol + (uint32_t)(t * kHD),
+                 desc_kmajor(p_base + (uint32_t)((k >> 2) * kBox), k & 3), desc_mnmajor(v_base, k),
+                 idO, (k > 0 || !first) ? 1u : 0u);
+        tc_commit(o_full0 + 8 * t);
+        ++co[t];
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 1; j <= nkv && ok; ++j) {
-        if (j < nkv) ok = issue_s(j);
-        if (ok) ok = issue_o(j - 1);
+      FwdItem it;
+      for (int k = 0; ok && fwd_item(k, B, H, nq, it); ++k, ++n_item) {
+        ok = mbar_wait(q_full, n_item & 1u, abort_flag, err);
+        if (!ok) break;
+        tc_fence_after();
+        const int nkv = it.nkv_b ? it.nkv_b : it.nkv_a;
+        for (int j = 0; j <= nkv && ok; ++j) {
+          if (j < nkv) {
+            const uint32_t gj = g + j;
+            ok = mbar_wait(kv_full0 + 8 * (gj % kKVStages), (gj / kKVStages) & 1u, abort_flag, err);
+            if (ok && j < it.nkv_a) ok = issue_s(0, gj % kKVStages);
+            if (ok && j < it.nkv_b) ok = issue_s(1, gj % kKVStages);
+            if (ok && j == nkv - 1) tc_commit(q_empty);  // the item's Q tiles are read
+          }
+          if (ok && j >= 1) {
+            const uint32_t st = (g + j - 1) % kKVStages;
+            if (j - 1 < it.nkv_a) ok = issue_pv(0, st, j == 1);
+            if (ok && j - 1 < it.nkv_b) ok = issue_pv(1, st, j == 1);
+            if (ok) tc_commit(kv_empty0 + 8 * st);  // K and V of key tile j-1 are no longer read
+          }
+        }
+        g += nkv;
       }
       if (!ok) {  // let issued MMAs finish before TMEM is released
         tc_commit(drain);
@@ -207,107 +243,148 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else {
     // -------------------------------------------------------- softmax --
-    const int qw = warp & 3;           // TMEM lane quarter
-    const int half = (warp - 2) >> 2;  // 0: key columns 0-63 / dims 0-31; 1: 64-127 / 32-63
-    const int r = qw * 32 + lane;
-    const int qi = q0 + r;  // query index in the sequence
+    const int t = (warp - 2) >> 2;  // query tile of the item: 0 = A, 1 = B
+    const int qw = warp & 3;        // TMEM lane quarter
+    const int r = qw * 32 + lane;   // row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    float o[kHD / 2];
-#pragma unroll
-    for (int i = 0; i < kHD / 2; ++i) o[i] = 0.f;
-    float m = -INFINITY, l = 0.f, a_pend = 1.f;
+    const uint32_t s_col = (uint32_t)(t * kTile);
+    const uint32_t o_col = kOCol + (uint32_t)(t * kHD);
+    const uint32_t p_row = smem_u32(sP + t * 2 * kBox) + (uint32_t)(r * 128);  // this row of P
+    uint32_t cs = 0, co = 0;  // S tiles read / PV products waited for by this tile's threads
     bool ok = true;
-    for (int j = 0; j <= nkv && ok; ++j) {
-      float a_new = 1.f;
-      if (j < nkv) {
-        const int sb = j & 1;
-        ok = sm_bar_and(mbar_wait(s_full0 + 8 * sb, (uint32_t)(j >> 1) & 1u, abort_flag, err));
+    // wait for the next PV product of this tile (every completion is
+    // waited for, in order, so that the barrier parity stays in step)
+    auto wait_pv = [&]() -> bool {
+      const bool r2 = __all_sync(0xffffffffu, mbar_wait(o_full0 + 8 * t, co & 1u, abort_flag, err));
+      ++co;
+      return r2;
+    };
+    FwdItem it;
+    for (int k = 0; ok && fwd_item(k, B, H, nq, it); ++k) {
+      const int nk = t ? it.nkv_b : it.nkv_a;
+      if (nk == 0) continue;  // the item has no tile B
+      const int qt = t ? it.qb : it.qa;
+      const int qi = qt * kTile + r;  // query index in the sequence
+      float m = -INFINITY, l = 0.f;  // reference max (log2 units) and the sum against it
+      for (int j = 0; j < nk && ok; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * t, cs & 1u, abort_flag, err));
         if (!ok) break;
         tc_fence_after();
-        float s[64];
-        {
-          uint32_t rr[64];
-          const uint32_t col = (uint32_t)(sb * kTileK + 64 * half);
-          tc_ld32(lane_base + col, rr);
-          tc_ld32(lane_base + col + 32, rr + 32);
-          tc_wait_ld();
-          tc_fence_before();
-          mbar_arrive(s_empty0 + 8 * sb);
+        const bool diag = (j == nk - 1);  // keys after the query are masked
+        const int key0 = j * kTile;
+        // pass 1: the row max, 32 columns per TMEM load, the next load in
+        // flight while the current chunk is scanned
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // columns c > lim of chunk ch are masked (keys after the query)
+        auto mask_lim = [&](int ch) { return diag ? qi - key0 - 32 * ch : 1 << 30; };
+        auto scan_max = [&](const uint32_t* rr, int ch) {
+          const int lim = mask_lim(ch);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(rr[c]);
+          for (int c = 0; c < 32; ++c) {
+            const float v = c > lim ? -INFINITY : __uint_as_float(rr[c]);
+            mx4[c & 3] = fmaxf(mx4[c & 3], v);
+          }
+        };
+        uint32_t ra[32], rb[32];
+        tc_ld32(lane_base + s_col, ra);
+        tc_wait_ld();
+        tc_ld32(lane_base + s_col + 32, rb);
+        scan_max(ra, 0);
+        tc_wait_ld();
+        tc_ld32(lane_base + s_col + 64, ra);
+        scan_max(rb, 1);
+        tc_wait_ld();
+        tc_ld32(lane_base + s_col + 96, rb);
+        scan_max(ra, 2);
+        tc_wait_ld();
+        scan_max(rb, 3);
+        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+        // the previous product is complete: P is free and O may be rescaled
+        if (j >= 1) {
+          ok = wait_pv();
+          if (!ok) break;
+          tc_fence_after();
         }
-        const int key0 = j * kTileK + 64 * half;
-        if (j == qb) {  // diagonal tile: keys after the query (and past T) are masked
+        if (mt > m + kRescaleLog2) {
+          if (j >= 1) {  // rescale the row of O and the sum to the new reference
+            const float f = fast_exp2(m - mt);
+            l *= f;
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (key0 + c > qi || key0 + c >= T) s[c] = -INFINITY;
+            for (int hf = 0; hf < 2; ++hf) {
+              tc_ld32(lane_base + o_col + 32 * hf, ra);
+              tc_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) ra[c] = __float_as_uint(__uint_as_float(ra[c]) * f);
+              attn::tc_st32(lane_base + o_col + 32 * hf, ra);
+            }
+            attn::tc_wait_st();
+          }
+          m = mt;
         }
-        // row max over this thread's 64 columns (8 independent chains),
-        // then with the partner thread's half through shared memory
-        float mx8[8];
+        // pass 2: P into the shared-memory tile, row sum
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        // key columns 32ch .. 32ch+31: box ch / 2, 16-byte chunks 4 (ch % 2) ..
+        auto emit = [&](const uint32_t* rr, int ch) {
+          const int lim = mask_lim(ch);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float pv[8];
 #pragma unroll
-        for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        float* rm = red_max + (j & 1) * 2 * kTileQ;
-        rm[half * kTileQ + r] = mx;
-        sm_bar();
-        mx = fmaxf(mx, rm[(half ^ 1) * kTileQ + r]) * sl2;  // scaled (log2 units)
-        const float mnew = fmaxf(m, mx);
-        a_new = (mnew == -INFINITY) ? 1.f : fast_exp2(m - mnew);
-        const float mref = (mnew == -INFINITY) ? 0.f : mnew;
-        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          s[c] = fast_exp2(fmaf(s[c], sl2, -mref));
-          sum8[c & 7] += s[c];
-        }
-        l = l * a_new + (((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
-                         ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7])));
-        m = mnew;
-        // P_j (this half's 64 keys = one 128-byte-swizzled box)
-        const int pb = j & 1;
-        ok = sm_bar_and(mbar_wait(p_empty0 + 8 * pb, ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, err));
-        if (!ok) break;
-        uint8_t* pt = sP + (pb * 2 + half) * kBox;
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8)
-          store8(reinterpret_cast<__nv_bfloat16*>(pt + swz(r, c8)), s + 8 * c8);
-        fence_async_smem();
-        mbar_arrive(p_full0 + 8 * pb);
-      }
-      if (j >= 1) {  // fold O_{j-1} (computed with the max of tile j-1)
-        const int ob = (j - 1) & 1;
-        ok = sm_bar_and(mbar_wait(o_full0 + 8 * ob, (uint32_t)((j - 1) >> 1) & 1u, abort_flag, err));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t rr[32];
-        tc_ld32(lane_base + 2u * kTileK + (uint32_t)(ob * kHD + 32 * half), rr);
+            for (int q = 0; q < 8; ++q) {
+              const int c = 8 * c8 + q;
+              const float v = c > lim ? -INFINITY : __uint_as_float(rr[c]);
+              pv[q] = fast_exp2(fmaf(v, sl2, -m));
+              sum4[q & 3] += pv[q];
+            }
+            attn::st_shared_bf16x8(
+                p_row + (uint32_t)((ch >> 1) * kBox) + ((uint32_t)((4 * (ch & 1) + c8) ^ (r & 7)) << 4),
+                pv);
+          }
+        };
+        tc_ld32(lane_base + s_col, ra);
+        tc_wait_ld();
+        tc_ld32(lane_base + s_col + 32, rb);
+        emit(ra, 0);
+        tc_wait_ld();
+        tc_ld32(lane_base + s_col + 64, ra);
+        emit(rb, 1);
+        tc_wait_ld();
+        tc_ld32(lane_base + s_col + 96, rb);
+        emit(ra, 2);
         tc_wait_ld();
         tc_fence_before();
-        mbar_arrive(o_empty0 + 8 * ob);
-#pragma unroll
-        for (int i = 0; i < kHD / 2; ++i) o[i] = o[i] * a_pend + __uint_as_float(rr[i]);
+        mbar_arrive(s_empty0 + 8 * t);  // S_t is read: the next S_t may be computed
+        emit(rb, 3);
+        fence_async_smem();
+        mbar_arrive(p_full0 + 8 * t);  // (after the TMEM fence above: O's rescale is ordered too)
+        l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        ++cs;
       }
-      a_pend = a_new;
-    }
-    // row sum = the two halves' partial sums
-    red_l[half * kTileQ + r] = l;
-    sm_bar();
-    l += red_l[(half ^ 1) * kTileQ + r];
-    if (ok && qi < T) {
-      const float inv = 1.f / l;
-      __nv_bfloat16* dst = att + ((size_t)b * T + qi) * C + (size_t)h * kHD + 32 * half;
+      if (!ok) break;
+      // the item's last product, then the normalised output row
+      ok = wait_pv();
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t ra[32], rb[32];
+      tc_ld32(lane_base + o_col, ra);
+      tc_ld32(lane_base + o_col + 32, rb);
+      tc_wait_ld();
+      tc_fence_before();  // O is read before the next item's first product overwrites it
+      if (qi < T) {
+        const float inv = 1.f / l;
+        __nv_bfloat16* dst = att + ((size_t)it.b * T + qi) * C + (size_t)it.h * kHD;
 #pragma unroll
-      for (int i = 0; i < kHD / 2; i += 8) {
-        float t[8];
+        for (int i = 0; i < 32; i += 8) {
+          float v[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) t[k] = o[i + k] * inv;
-        store8(dst + i, t);
+          for (int q = 0; q < 8; ++q) v[q] = __uint_as_float(ra[i + q]) * inv;
+          store8(dst + i, v);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) v[q] = __uint_as_float(rb[i + q]) * inv;
+          store8(dst + 32 + i, v);
+        }
+        lse[((size_t)it.b * H + it.h) * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
       }
-      if (half == 0) lse[((size_t)b * H + h) * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
     }
   }
 
@@ -380,8 +457,12 @@ cudaError_t attention_fwd_tc(act_t* att, float* lse, const act_t* qkv, int B, in
     attr = true;
   }
   const float sl2 = 1.4426950408889634f / sqrtf((float)kHD);
-  dim3 grid((T + kTileQ - 1) / kTileQ, B * H);
-  flash_fwd_tc_kernel<<<grid, kThreadsAttn, smem, s>>>(tm, att, lse, T, C, H, sl2, err);
+  const int items = (((T + kTile - 1) / kTile + 1) / 2) * B * H;
+  int sms = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = items < sms ? items : sms;
+  flash_fwd_tc_kernel<<<grid, kThreadsAttn, smem, s>>>(tm, att, lse, B, T, C, H, sl2, err);
   note_launch();
   return cudaGetLastError();
 }

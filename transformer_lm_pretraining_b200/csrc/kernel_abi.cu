@@ -17,6 +17,8 @@ int* err_word() {
   return e;
 }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 int status(cudaError_t e) { return e == cudaSuccess ? GPT2_OK : (e == cudaErrorInvalidValue ? GPT2_ERR_ARG : GPT2_ERR_CUDA); }
 
 }  // namespace
@@ -62,6 +64,41 @@ int gpt2k_attention_bwd(void* stream, void* dqkv, float* dsum, const void* datt,
   return status(attention_bwd(static_cast<act_t*>(dqkv), dsum, static_cast<const act_t*>(datt),
                               static_cast<const act_t*>(qkv), static_cast<const act_t*>(att), lse,
                               B, T, C, H, err, static_cast<cudaStream_t>(stream)));
+}
+
+int gpt2k_layernorm_fwd(void* stream, void* y, float* mean, float* rstd, const void* x,
+                        const float* g, const float* b, int M, int C) {
+  if (M < 0 || C < 8 || C > 2048 || C % 8 || !aligned16(x) || !aligned16(y)) return GPT2_ERR_ARG;
+  if (M == 0) return GPT2_OK;
+  layernorm_fwd(static_cast<act_t*>(y), mean, rstd, static_cast<const act_t*>(x), g, b, M, C,
+                static_cast<cudaStream_t>(stream));
+  return status(cudaGetLastError());
+}
+
+size_t gpt2k_layernorm_bwd_scratch(int C) { return (size_t)kLnBlocks * 3 * (C > 0 ? C : 0); }
+
+int gpt2k_layernorm_bwd(void* stream, void* dx, const void* dy, const void* x, const float* mean,
+                        const float* rstd, const float* g, float* dg, float* db, float* dsum,
+                        float* partials, int M, int C, int accumulate) {
+  if (M < 0 || C < 8 || C > 2048 || C % 8 || !aligned16(x) || !aligned16(dy) || !aligned16(dx) ||
+      !partials)
+    return GPT2_ERR_ARG;
+  if (M == 0) return GPT2_OK;
+  layernorm_bwd(static_cast<act_t*>(dx), static_cast<const act_t*>(dy),
+                static_cast<const act_t*>(x), mean, rstd, g, dg, db, dsum, partials, M, C,
+                accumulate ? 1 : 0, static_cast<cudaStream_t>(stream));
+  return status(cudaGetLastError());
+}
+
+int gpt2k_classifier(void* stream, void* logits, float* losses, const int* tgt, int M, int V,
+                     int Vp, int write_grad) {
+  if (M < 0 || V < 1 || Vp < V || Vp % 8 || !aligned16(logits)) return GPT2_ERR_ARG;
+  if (M == 0) return GPT2_OK;
+  int* err = err_word();
+  if (!err) return GPT2_ERR_CUDA;
+  classifier(static_cast<act_t*>(logits), losses, tgt, M, V, Vp, write_grad ? 1 : 0, err,
+             static_cast<cudaStream_t>(stream));
+  return status(cudaGetLastError());
 }
 
 int gpt2k_take_error(void) {

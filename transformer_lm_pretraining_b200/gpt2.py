@@ -67,6 +67,10 @@ SIGNATURES = {
                         _vp, _l, _vp, _l, _fp, _sz]),
     "gpt2k_attention_fwd": (_i, [_vp, _vp, _fp, _vp, _i, _i, _i, _i]),
     "gpt2k_attention_bwd": (_i, [_vp, _vp, _fp, _vp, _vp, _vp, _fp, _i, _i, _i, _i]),
+    "gpt2k_layernorm_fwd": (_i, [_vp, _vp, _fp, _fp, _vp, _fp, _fp, _i, _i]),
+    "gpt2k_layernorm_bwd": (_i, [_vp, _vp, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _i, _i, _i]),
+    "gpt2k_layernorm_bwd_scratch": (_sz, [_i]),
+    "gpt2k_classifier": (_i, [_vp, _vp, _fp, _vp, _i, _i, _i, _i]),
     "gpt2k_take_error": (_i, []),
     "gpt2k_gemm_wgrad_noalloc": (_i, [_vp, _i, _i, _i, _vp, _l, _vp, _l, _f, _fp, _l, _i, _vp]),
 }
@@ -298,6 +302,44 @@ def gpt2k_attention_bwd(dqkv, dsum, datt, qkv, att, lse, B, T, C, H, precision="
                                _dptr(att), cf(lse), B, T, C, H)
     if rc:
         raise GPT2Error(rc, "gpt2k_attention_bwd")
+
+
+def _f32p(t):
+    return None if t is None else ctypes.cast(ctypes.c_void_p(t.data_ptr()), _fp)
+
+
+def _stream(stream):
+    import torch
+
+    return (stream if stream is not None else torch.cuda.current_stream()).cuda_stream
+
+
+def gpt2k_layernorm_fwd(y, mean, rstd, x, g, b, M, C, precision="bf16", stream=None):
+    rc = load(precision).gpt2k_layernorm_fwd(_stream(stream), _dptr(y), _f32p(mean), _f32p(rstd),
+                                             _dptr(x), _f32p(g), _f32p(b), M, C)
+    if rc:
+        raise GPT2Error(rc, "gpt2k_layernorm_fwd")
+
+
+def gpt2k_layernorm_bwd_scratch(C, precision="bf16") -> int:
+    return int(load(precision).gpt2k_layernorm_bwd_scratch(C))
+
+
+def gpt2k_layernorm_bwd(dx, dy, x, mean, rstd, g, dg, db, dsum, partials, M, C, accumulate,
+                        precision="bf16", stream=None):
+    rc = load(precision).gpt2k_layernorm_bwd(
+        _stream(stream), _dptr(dx), _dptr(dy), _dptr(x), _f32p(mean), _f32p(rstd), _f32p(g),
+        _f32p(dg), _f32p(db), _f32p(dsum), _f32p(partials), M, C, 1 if accumulate else 0)
+    if rc:
+        raise GPT2Error(rc, "gpt2k_layernorm_bwd")
+
+
+def gpt2k_classifier(logits, losses, tgt, M, V, Vp, write_grad=True, precision="bf16",
+                     stream=None):
+    rc = load(precision).gpt2k_classifier(_stream(stream), _dptr(logits), _f32p(losses),
+                                          _dptr(tgt), M, V, Vp, 1 if write_grad else 0)
+    if rc:
+        raise GPT2Error(rc, "gpt2k_classifier")
 
 
 def gpt2k_take_error(precision="bf16") -> int:

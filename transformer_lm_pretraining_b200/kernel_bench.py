@@ -8,8 +8,11 @@ GEMM forms (the three products of a projection y = x W^T + b):
   fwd    out[M, N] = x[M, K] W[N, K]^T            (epi: store, bias, bias_gelu, bias_resid)
   dgrad  out[M, N] = dy[M, K] W[K, N]             (epi: store, dgelu)
   wgrad  out32[M, N] += dy[K, M]^T x[K, N]        (fp32 accumulate, split-K when few tiles)
+  python -m transformer_lm_pretraining_b200.kernel_bench ln --M 16384 --C 768 --form bwd
+  python -m transformer_lm_pretraining_b200.kernel_bench cls --M 16384 --V 50257 --Vp 50304
 Prints one JSON line with the mean time per call (CUDA events, after one
-warm-up call) and the achieved TFLOP/s.  Inputs are random bf16.
+warm-up call) and the achieved TFLOP/s (GEMM, attention) or GB/s of
+algorithmic traffic (LayerNorm, classifier).  Inputs are random bf16.
 """
 from __future__ import annotations
 
@@ -79,6 +82,39 @@ def bench_attn(a):
     return call, 4.0 * tri
 
 
+def bench_ln(a):
+    M, C = a.M, a.C
+    x, dy = _rand((M, C)), _rand((M, C))
+    g = torch.ones(C, device="cuda")
+    b = torch.zeros(C, device="cuda")
+    y = torch.empty((M, C), dtype=torch.bfloat16, device="cuda")
+    mean = torch.empty(M, dtype=torch.float32, device="cuda")
+    rstd = torch.empty(M, dtype=torch.float32, device="cuda")
+    g2.gpt2k_layernorm_fwd(y, mean, rstd, x, g, b, M, C)
+    if a.form == "fwd":
+        def call():
+            g2.gpt2k_layernorm_fwd(y, mean, rstd, x, g, b, M, C)
+        return call, 4.0 * M * C + 8.0 * M  # bytes: read x, write y, mean, rstd
+    dx = _rand((M, C))
+    dg, db, ds = (torch.zeros(C, device="cuda") for _ in range(3))
+    part = torch.empty(g2.gpt2k_layernorm_bwd_scratch(C), dtype=torch.float32, device="cuda")
+
+    def call():
+        g2.gpt2k_layernorm_bwd(dx, dy, x, mean, rstd, g, dg, db, ds, part, M, C, 1)
+    return call, 8.0 * M * C + 8.0 * M  # bytes: read x, dy, dx; write dx; mean, rstd
+
+
+def bench_cls(a):
+    M, V, Vp = a.M, a.V, a.Vp
+    z = _rand((M, Vp))
+    losses = torch.empty(M, dtype=torch.float32, device="cuda")
+    tgt = torch.randint(0, V, (M,), dtype=torch.int32, device="cuda")
+
+    def call():
+        g2.gpt2k_classifier(z, losses, tgt, M, V, Vp, write_grad=True)
+    return call, 4.0 * M * Vp  # bytes: read and write the logits
+
+
 def main():
     ap = argparse.ArgumentParser()
     sub = ap.add_subparsers(dest="kind", required=True)
@@ -96,9 +132,20 @@ def main():
     t.add_argument("--H", type=int, default=12)
     t.add_argument("--form", default="fwd", choices=["fwd", "bwd"])
     t.add_argument("--iters", type=int, default=20)
+    n = sub.add_parser("ln")
+    n.add_argument("--M", type=int, default=16384)
+    n.add_argument("--C", type=int, default=768)
+    n.add_argument("--form", default="bwd", choices=["fwd", "bwd"])
+    n.add_argument("--iters", type=int, default=20)
+    c = sub.add_parser("cls")
+    c.add_argument("--M", type=int, default=16384)
+    c.add_argument("--V", type=int, default=50257)
+    c.add_argument("--Vp", type=int, default=50304)
+    c.add_argument("--iters", type=int, default=5)
+    c.set_defaults(form="fwd+grad")
     a = ap.parse_args()
     torch.manual_seed(0)
-    call, flops = bench_gemm(a) if a.kind == "gemm" else bench_attn(a)
+    call, work = {"gemm": bench_gemm, "attn": bench_attn, "ln": bench_ln, "cls": bench_cls}[a.kind](a)
     call()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -109,8 +156,10 @@ def main():
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.iters
     err = g2.gpt2k_take_error()
-    print(json.dumps({"kernel": a.kind, "form": a.form, "args": vars(a), "ms": ms,
-                      "tflops": flops / (ms / 1e3) / 1e12, "error_word": err}))
+    rate = ({"gbs": work / (ms / 1e3) / 1e9} if a.kind in ("ln", "cls")
+            else {"tflops": work / (ms / 1e3) / 1e12})
+    print(json.dumps({"kernel": a.kind, "form": a.form, "args": vars(a), "ms": ms, **rate,
+                      "error_word": err}))
     if err:
         raise SystemExit(f"kernel error word {err}")
 
