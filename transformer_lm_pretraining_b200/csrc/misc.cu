@@ -3,6 +3,8 @@
 
 #include <atomic>
 
+#include <cuda_fp16.h>
+
 #include "kernels.h"
 #include "tc_util.cuh"
 
@@ -198,12 +200,14 @@ __global__ void __launch_bounds__(kClsThreads)
 // Persistent variant for rows that fit twice in shared memory: one CTA per
 // SM takes rows blockIdx.x, + gridDim.x, ...; each row arrives with one
 // bulk copy, a row ahead of its use (two buffers), so HBM sees one read and
-// one write of the logits.  Three passes over shared memory: the max, the
-// sum of exponentials (per-thread partials over a fixed column assignment,
-// then warps in order), then z <- (softmax - onehot) / M written straight to
-// global memory (skipped when write_grad == 0).  Separate max and sum
-// passes keep every exponential independent of the others (a running max
-// would chain them).
+// one write of the logits.  Three passes over shared memory: the max (on
+// packed bf16 pairs); the exponentials e = exp(z - max), summed in fp32
+// (per-thread partials over a fixed column assignment, then warps in order)
+// and kept in place as fp16; then z <- e / sum / M - onehot / M written
+// straight to global memory (skipped when write_grad == 0).  Separate max
+// and sum passes keep every exponential independent of the others (a
+// running max would chain them), and each logit is exponentiated once.
+// The bf16 build only (rows of 2-byte logits).
 constexpr int kClsBulkThreads = 1024;
 
 __device__ __forceinline__ float block_reduce_cls(float v, float* red, bool is_max) {
@@ -258,44 +262,77 @@ __global__ void __launch_bounds__(kClsBulkThreads, 1)
     const bool got = mbar_wait(smem_u32(&bars[b]), (phase >> b) & 1u, &abort_s, err);
     if (!__syncthreads_and(got)) break;
     phase ^= 1u << b;
-    const act_t* z = reinterpret_cast<const act_t*>(cls_smem + b * buf_stride);
-    float mx = -INFINITY;
-    for (int c = tid * 8; c < Vp; c += kClsBulkThreads * 8) {
-      float v[8];
-      load8(z + c, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (c + i < V) mx = fmaxf(mx, v[i]);
-    }
-    mx = block_reduce_cls(mx, red, true);
-    const float mx2 = mx * kLog2e;
-    float sm = 0.f;
-    for (int c = tid * 8; c < Vp; c += kClsBulkThreads * 8) {
-      float v[8];
-      load8(z + c, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (c + i < V) sm += fast_exp2(fmaf(v[i], kLog2e, -mx2));
-    }
-    sm = block_reduce_cls(sm, red, false);
-    const float lse = mx + logf(sm);
+    uint8_t* zb = cls_smem + b * buf_stride;
+    const act_t* z = reinterpret_cast<const act_t*>(zb);
     int t = tgt[row];
     if (t < 0 || t >= V) {
       if (tid == 0) atomicOr(err, ERR_TARGET);
       t = 0;
     }
-    if (tid == 0) losses[row] = lse - to_f(z[t]);
-    if (write_grad) {
-      const float lse2 = lse * kLog2e;
-      act_t* out = logits + (size_t)row * Vp;
+    const float zt = to_f(z[t]);  // read before pass 2 overwrites the row
+    // pass 1: the max over columns < V, on packed bf16 pairs
+    float mx = -INFINITY;
+    {
+      __nv_bfloat162 m2 = __floats2bfloat162_rn(-INFINITY, -INFINITY);
       for (int c = tid * 8; c < Vp; c += kClsBulkThreads * 8) {
-        float v[8];
-        load8(z + c, v);
+        if (c + 8 <= V) {
+          const uint4 u = *reinterpret_cast<const uint4*>(z + c);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+          m2 = __hmax2(__hmax2(m2, h2[0]), __hmax2(h2[1], __hmax2(h2[2], h2[3])));
+        } else {
+          for (int i = 0; i < 8 && c + i < V; ++i) mx = fmaxf(mx, to_f(z[c + i]));
+        }
+      }
+      mx = fmaxf(mx, fmaxf(__low2float(m2), __high2float(m2)));
+    }
+    mx = block_reduce_cls(mx, red, true);
+    const float mx2 = mx * kLog2e;
+    // pass 2: e = exp(z - max) summed in fp32 and kept in place as fp16
+    // (0 for the padded columns), so that pass 3 needs no exponential
+    float sm = 0.f;
+    for (int c = tid * 8; c < Vp; c += kClsBulkThreads * 8) {
+      float v[8];
+      load8(z + c, v);
+      if (c + 8 <= V) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int col = c + i;
-          v[i] = col < V ? (fast_exp2(fmaf(v[i], kLog2e, -lse2)) - (col == t ? 1.f : 0.f)) * inv
-                         : 0.f;
+          v[i] = fast_exp2(fmaf(v[i], kLog2e, -mx2));
+          sm += v[i];
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v[i] = c + i < V ? fast_exp2(fmaf(v[i], kLog2e, -mx2)) : 0.f;
+          sm += v[i];
+        }
+      }
+      uint4 o;
+      __half2* o2 = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o2[i] = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+      *reinterpret_cast<uint4*>(zb + (size_t)c * 2) = o;
+    }
+    sm = block_reduce_cls(sm, red, false);
+    const float lse = mx + logf(sm);
+    if (tid == 0) losses[row] = lse - zt;
+    if (write_grad) {
+      // pass 3: z <- e / sum / M, minus 1 / M at the target
+      const float sc = inv / sm;
+      act_t* out = logits + (size_t)row * Vp;
+      for (int c = tid * 8; c < Vp; c += kClsBulkThreads * 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(zb + (size_t)c * 2);
+        const __half2* e2 = reinterpret_cast<const __half2*>(&u);
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __half22float2(e2[i]);
+          v[2 * i] = f.x * sc;
+          v[2 * i + 1] = f.y * sc;
+        }
+        if (t >= c && t < c + 8) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (c + i == t) v[i] -= inv;
         }
         store8(out + c, v);
       }
@@ -508,7 +545,7 @@ void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int 
   if (M <= 0) return;
   const size_t row_bytes = (size_t)Vp * sizeof(act_t);
   const size_t smem = 2 * ((row_bytes + 127) & ~(size_t)127);
-  if (smem <= 200 * 1024 && row_bytes % 16 == 0 &&
+  if (sizeof(act_t) == 2 && smem <= 200 * 1024 && row_bytes % 16 == 0 &&
       (reinterpret_cast<uintptr_t>(logits) & 15) == 0) {
     static size_t attr = 0;
     if (attr < smem) {
