@@ -49,8 +49,17 @@ constexpr int kWarpBox = 4096;  // one warp's epilogue box: 32 rows x 128 bytes
 
 // Epilogues that read a second [M, N] input (residual or pre-activation).
 constexpr bool epi_has_input(int epi) { return epi == EPI_BIAS_RESID || epi == EPI_DGELU; }
+// Boxes per epilogue warp.  With two, a warp writes one box while TMA still
+// reads the other (output epilogues), or the next group's input streams into
+// a box of its own while the current group is computed (input epilogues).
+// The second box costs a ring stage, which is worth it only for the GELU
+// backward (measured: one ring stage less slows the store, bias, GELU and
+// fp32 forms more than the second box gains).
+constexpr int epi_boxes(int epi) { return epi == EPI_DGELU ? 2 : 1; }
 // Operand ring depth: what the shared memory holds next to the epilogue boxes.
-constexpr int ring_stages(int bn, int /*epi*/) { return bn == 256 ? 4 : 6; }
+constexpr int ring_stages(int bn, int epi) {
+  return bn == 256 ? (epi_boxes(epi) == 2 ? 3 : 4) : (epi_boxes(epi) == 2 ? 5 : 6);
+}
 
 // Instruction descriptor: bf16 x bf16 -> fp32, M = 128, N = BN.
 template <int BN, bool A_MN, bool B_MN>
@@ -67,7 +76,7 @@ constexpr uint32_t tmem_cols() {
 template <int BN, int EPI>
 constexpr size_t smem_bytes() {
   return 1024 + (size_t)ring_stages(BN, EPI) * (BM * BK * 2 + BN * BK * 2) +
-         (size_t)kEpiWarps * kWarpBox + 256;
+         (size_t)kEpiWarps * epi_boxes(EPI) * kWarpBox + 256;
 }
 
 template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI>
@@ -90,8 +99,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint8_t* sBox = smem + STAGES * (A_BYTES + B_BYTES);  // [kEpiWarps] boxes, 1024-aligned
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sBox + kEpiWarps * kWarpBox);
+  constexpr int NBOX = epi_boxes(EPI);
+  uint8_t* sBox = smem + STAGES * (A_BYTES + B_BYTES);  // [kEpiWarps][NBOX] boxes, 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sBox + kEpiWarps * NBOX * kWarpBox);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4 + kEpiWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -253,11 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- epilogue --
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int h = (warp - 2) >> 2;   // groups h, h + 2, ... of each tile
-    uint8_t* box = sBox + (warp - 2) * kWarpBox;
-    const uint32_t box_u = smem_u32(box);
+    uint8_t* wbox = sBox + (warp - 2) * NBOX * kWarpBox;  // this warp's boxes
+    // input epilogues: the input box (the second box, or the only one)
+    uint8_t* ibox = wbox + (NBOX - 1) * kWarpBox;
+    const uint32_t ibox_u = smem_u32(ibox);
+    int ob = 0;  // output box of the next store (alternates when the output has two)
     const uint32_t in_full = in_full0 + 8 * (warp - 2);
     uint32_t in_phase = 0;
-    bool in_pend = false;  // an input copy into the box is in flight
+    bool in_pend = false;  // an input copy is in flight
+    bool pre = false;      // the input of this warp's next group is already requested
     if (warp == 2 && lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmOut)) : "memory");
       if (EPI == EPI_BIAS_GELU || HAS_IN)
@@ -267,16 +281,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     // send the box with `send` from lane 0 once every lane's writes are
     // visible to the async proxy.  The box is reused only after the
     // previous store has read it.
+    // With two output boxes used in turn, every store but the latest (which
+    // read the other box) must have read its box.
+    constexpr int OUT_BOXES = HAS_IN ? 1 : NBOX;
     auto put_box = [&](auto write_row, auto send) {
-      if (lane == 0) bulk_wait_read<0>();
+      uint8_t* box = wbox + ob * kWarpBox;
+      if (lane == 0) {
+        if (OUT_BOXES == 2) bulk_wait_read<1>();
+        else bulk_wait_read<0>();
+      }
       __syncwarp();
-      write_row();
+      write_row(box);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        send();
+        send(smem_u32(box));
         bulk_commit();
       }
+      if (OUT_BOXES == 2) ob ^= 1;
     };
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -299,14 +321,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = h; g < ngroups; g += 2) {
         const int nb = nt0 + 64 * g;  // first column of the group
         const bool live = r0 < ep.M;  // rows of this slab exist
-        if (HAS_IN && live && lane == 0) {
-          // the group's input slab into the box, ahead of the accumulator
-          // read (the box is free once the previous store has read it)
-          bulk_wait_read<0>();
+        if (HAS_IN && live && !pre && lane == 0) {
+          // the group's input slab, ahead of the accumulator read (a shared
+          // box is free once the previous store has read it)
+          if (NBOX == 1) bulk_wait_read<0>();
           mbar_expect_tx(in_full, kWarpBox);
-          tma_load_3d(box_u, &tmX, in_full, nb, r0, 0);
+          tma_load_3d(ibox_u, &tmX, in_full, nb, r0, 0);
           in_pend = true;
         }
+        pre = false;
         float v[64];
         {
           uint32_t r[64];
@@ -342,8 +365,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           in_pend = false;
           uint4 xin[8];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) xin[c] = *reinterpret_cast<const uint4*>(box + swz(lane, c));
-          __syncwarp();  // the box is rewritten below
+          for (int c = 0; c < 8; ++c) xin[c] = *reinterpret_cast<const uint4*>(ibox + swz(lane, c));
+          __syncwarp();  // every lane has read the input box
+          if (NBOX == 2) {
+            // request this warp's next input now: group g + 2 of this tile, or
+            // group h of the next tile
+            int pn = -1, pr = 0;
+            if (g + 2 < ngroups) {
+              pn = nb + 128;
+              pr = r0;
+            } else if (u + (int)gridDim.x < units) {
+              int tm2, tn2, kb02, kb12, sp2;
+              decode(u + gridDim.x, tm2, tn2, kb02, kb12, sp2);
+              const int nt2 = tn2 * BN, r2 = tm2 * BM + q * 32;
+              if (h < ((min(BN, ep.N - nt2) + 63) >> 6) && r2 < ep.M) {
+                pn = nt2 + 64 * h;
+                pr = r2;
+              }
+            }
+            if (pn >= 0) {
+              if (lane == 0) {
+                fence_async_smem();  // the reads above come before the copy's writes
+                mbar_expect_tx(in_full, kWarpBox);
+                tma_load_3d(ibox_u, &tmX, in_full, pn, pr, 0);
+                in_pend = true;
+              }
+              pre = true;
+            }
+          }
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xin[c]);
@@ -366,14 +415,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int half = 0; half < 2; ++half) {
             if (half == 1 && nb + 32 >= ep.N) break;
             put_box(
-                [&] {
+                [&](uint8_t* box) {
 #pragma unroll
                   for (int j = 0; j < 8; ++j)
                     *reinterpret_cast<float4*>(box + swz(lane, j)) =
                         make_float4(v[32 * half + 4 * j], v[32 * half + 4 * j + 1],
                                     v[32 * half + 4 * j + 2], v[32 * half + 4 * j + 3]);
                 },
-                [&] {
+                [&](uint32_t box_u) {
                   if (EPI == EPI_F32_ACC) tma_reduce_add_3d(&tmOut, box_u, nb + 32 * half, r0, 0);
                   else tma_store_3d(&tmOut, box_u, nb + 32 * half, r0, sp);
                 });
@@ -382,20 +431,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (EPI == EPI_BIAS_GELU) {
             // the pre-activation u first (saved for the backward), then GELU(u)
             put_box(
-                [&] {
+                [&](uint8_t* box) {
 #pragma unroll
                   for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(box + swz(lane, j)), v + 8 * j);
                 },
-                [&] { tma_store_3d(&tmX, box_u, nb, r0, 0); });
+                [&](uint32_t box_u) { tma_store_3d(&tmX, box_u, nb, r0, 0); });
 #pragma unroll
             for (int i = 0; i < 64; ++i) v[i] = gelu_tanh(v[i]);
           }
           put_box(
-              [&] {
+              [&](uint8_t* box) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(box + swz(lane, j)), v + 8 * j);
               },
-              [&] { tma_store_3d(&tmOut, box_u, nb, r0, 0); });
+              [&](uint32_t box_u) { tma_store_3d(&tmOut, box_u, nb, r0, 0); });
         }
       }
       acc ^= 1;
