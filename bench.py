@@ -222,7 +222,8 @@ def run_ours(args, wl):
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
     model = g2.GPT2(wl.L, wl.H, wl.C, wl.V, wl.Vp, wl.Tmax, seed=0, precision="bf16",
-                    B=wl.B, T=wl.T)
+                    B=wl.B, T=wl.T, recompute=args.recompute)
+    evaluate = args.mode == "eval"
     model.set_stream(stream)
     n_steps = args.warmup + args.steps
     host = make_batches(wl, n_steps, seed=1 + rank)
@@ -234,6 +235,10 @@ def run_ours(args, wl):
         return g2.gpt2_lr(k, wl.lr_max, 0.1 * wl.lr_max, wl.warmup, wl.max_steps)
 
     def step(k, batches):
+        if evaluate:  # forward-only evaluation: loss of every micro-batch
+            for tok, tgt in batches:
+                model.evaluate(tok, tgt, sync_loss=False)
+            return
         model.zero_grad()
         for tok, tgt in batches:
             model.forward(tok, tgt, sync_loss=False)
@@ -291,14 +296,19 @@ def run_ours(args, wl):
         e0.record(stream)
         for k in range(n_e2e):
             hb = pinned[(args.warmup + k) % n_steps]
-            model.zero_grad()
+            if not evaluate:
+                model.zero_grad()
             for j, (t, y) in enumerate(hb):
                 bufs[j][0].copy_(t, non_blocking=True)
                 bufs[j][1].copy_(y, non_blocking=True)
-                model.forward(bufs[j][0], bufs[j][1], sync_loss=False)
-                model.backward(scale)
-            model.grad_norm_clip(1.0, sync=False)
-            model.adamw_step(lr(args.warmup + k), 0.9, 0.95, 1e-8, 0.1)
+                if evaluate:
+                    model.evaluate(bufs[j][0], bufs[j][1], sync_loss=False)
+                else:
+                    model.forward(bufs[j][0], bufs[j][1], sync_loss=False)
+                    model.backward(scale)
+            if not evaluate:
+                model.grad_norm_clip(1.0, sync=False)
+                model.adamw_step(lr(args.warmup + k), 0.9, 0.95, 1e-8, 0.1)
             model.read_loss()
         e1.record(stream)
         torch.cuda.synchronize()
@@ -307,28 +317,31 @@ def run_ours(args, wl):
                "h2d_bytes_per_step": 2 * 4 * wl.B * wl.T * wl.n_micro, "d2h_bytes_per_step": 4}
 
     peaks = load_peaks()
-    fpt = wl.flops_per_token()
+    fpt = wl.flops_per_token() / (3.0 if evaluate else 1.0)  # the forward is a third
     mfu = fpt * value / world / SPEC_BF16_DENSE
     gemm_ms, gemm_n, gemm_fl = prof["gemm"]
     achieved = gemm_fl / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
     fam_ms = {k: v[0] / n_prof for k, v in prof.items()}
     fam_total = sum(fam_ms.values())
     out = {
-        "metric": "training tokens/s and MFU, GPT-2 124M bf16, B=16xT=1024, 1xB200"
-        if wl.name == "gpt2_124m" else f"training tokens/s and MFU, {wl.name} bf16",
+        "metric": ("evaluation" if evaluate else "training")
+        + (" tokens/s and MFU, GPT-2 124M bf16, B=16xT=1024, 1xB200" if wl.name == "gpt2_124m"
+           else f" tokens/s and MFU, {wl.name} bf16"),
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak",
-        "vs_baseline": value / PAGES_A100_TOK_S if wl.name == "gpt2_124m" else None,
+        "vs_baseline": value / PAGES_A100_TOK_S if wl.name == "gpt2_124m" and not evaluate else None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "global_batch": wl.B * wl.n_micro * world, "seq_len": wl.T,
                    "micro_batch": wl.B, "n_micro": wl.n_micro,
                    "tokens_per_step": wl.tokens_per_step * world,
                    "parallelism": "replicas" if world > 1 else "single-gpu",
+                   "mode": args.mode, "recompute": args.recompute,
                    "l2": "no explicit flush: every step streams ~10 GB of activations, logits and "
                          "optimizer state through HBM, far above the 126 MB L2"},
         "mfu": mfu,
-        "mfu_basis": f"{fpt / 1e6:.2f} MFLOP/token (6N + 6LCT, N = 12LC^2 + Vpad C) over "
+        "mfu_basis": f"{fpt / 1e6:.2f} MFLOP/token ({'2N + 2LCT' if evaluate else '6N + 6LCT'}, "
+                     f"N = 12LC^2 + Vpad C) over "
                      f"2.25 PFLOP/s dense bf16 spec; {fpt * value / world / (peaks['bf16_tflops'] * 1e12):.3f} "
                      f"of the {peaks['source']} cuBLAS bf16 peak",
         "gpu_launches": int(launches),
@@ -349,7 +362,7 @@ def run_ours(args, wl):
         "clocks": clk,
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not evaluate:
         out["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_T)
     if world > 1:
         barrier()
@@ -368,6 +381,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-T", type=int, default=256)
+    ap.add_argument("--mode", default="train", choices=["train", "eval"],
+                    help="train: the training step; eval: forward-only evaluation (loss)")
+    ap.add_argument("--recompute", type=int, default=0, choices=[0, 1],
+                    help="1: recompute GELU in the backward instead of keeping it")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -90,6 +90,16 @@ size_t gpt2_workspace_bytes(const gpt2_t* h, int B, int T);
 gpt2_status gpt2_bind_memory(gpt2_t* h, void* dev_state, size_t state_bytes, void* dev_work,
                              size_t work_bytes);
 
+/* Activation recompute (the recompute option of the first page's training
+ * loop): level 1 keeps no GELU output per layer (one layer's buffer is
+ * reused) and the backward recomputes GELU(u) from the stored pre-activation
+ * u before the projection's weight gradient; level 0 (the default) keeps
+ * them.  Results are bit-identical at both levels (the forward applies GELU
+ * to u as stored).  Level 1 shrinks gpt2_workspace_bytes by (L-1) B T 4C
+ * activations; set it before sizing and binding the workspace.  Errors:
+ * GPT2_ERR_ARG (level not 0 or 1). */
+gpt2_status gpt2_set_recompute(gpt2_t* h, int level);
+
 /* Stream (a cudaStream_t) on which every later call enqueues its work. */
 gpt2_status gpt2_set_stream(gpt2_t* h, void* cuda_stream);
 
@@ -105,6 +115,17 @@ gpt2_status gpt2_set_stream(gpt2_t* h, void* cuda_stream);
  * GPT2_ERR_STATE (no memory), GPT2_ERR_TOKEN, GPT2_ERR_NONFINITE. */
 gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok_dev, const int32_t* tgt_dev, int B, int T,
                          float* loss_host);
+
+/* Forward-only evaluation (the validation loop of the TinyStories page and
+ * the evaluation of the condensed GPT-2 page): the forward of gpt2_forward
+ * with targets, giving the same per-position and mean losses, but the
+ * logits [B*T, Vpad] are left as computed (no gradient is written into
+ * them) and no gpt2_backward may follow (GPT2_ERR_STATE until the next
+ * forward with targets).  B*T may be anything up to what the workspace was
+ * sized for.  loss_host (may be NULL) receives the mean loss and makes the
+ * call synchronous; the perplexity is exp(loss).  Errors as gpt2_forward. */
+gpt2_status gpt2_evaluate(gpt2_t* h, const int32_t* tok_dev, const int32_t* tgt_dev, int B, int T,
+                          float* loss_host);
 
 /* Mean loss of the last forward with targets, read back to the host
  * (synchronises the stream). */
@@ -185,11 +206,11 @@ long gpt2_launch_count(void);
 /* Per-kernel-family timing with CUDA events on the handle's stream.  Kinds:
  * 0 GEMM, 1 attention forward, 2 attention backward, 3 LayerNorm forward,
  * 4 LayerNorm backward, 5 classifier, 6 encoder (fwd+bwd), 7 bias-gradient
- * column sums, 8 optimiser (norm, clip, AdamW).  gpt2_profile_read
- * synchronises the stream, writes for each kind the summed milliseconds, the
- * number of timed regions and the algorithmic FLOPs (GEMM: 2MNK; attention:
- * causal products), and clears the records.  `kinds` is the length of the
- * arrays (>= 9). */
+ * column sums, 8 optimiser (norm, clip, AdamW), 9 GELU recompute.
+ * gpt2_profile_read synchronises the stream, writes for each kind the summed
+ * milliseconds, the number of timed regions and the algorithmic FLOPs (GEMM:
+ * 2MNK; attention: causal products), and clears the records.  `kinds` is the
+ * length of the arrays (>= 10). */
 gpt2_status gpt2_profile_enable(gpt2_t* h, int on);
 gpt2_status gpt2_profile_read(gpt2_t* h, double* ms, long* launches, double* flops, int kinds);
 

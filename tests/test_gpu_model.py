@@ -308,3 +308,89 @@ def test_clip_scale_matches_oracle_and_applies_once():
     assert t2 == t1 + 1
     assert np.allclose(m2, 0.9 * m1 + 0.1 * m.get_grads(), rtol=1e-5, atol=1e-12)
     m.close()
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_evaluate_matches_oracle_forward(precision):
+    # forward-only evaluation: the loss of the oracle's forward, the same
+    # per-position losses as the training forward, logits left as computed,
+    # no backward after it, and no effect on a training step that follows
+    name, cfg, B, T, iid = CASES[1]
+    tok, tgt = batch_for(cfg, B, T, iid, seed=3)
+    params = Oracle(cfg).init(0).astype(np.float32)
+    rloss, rlosses, _ = Oracle(cfg, openmp=True).forward(params.astype(np.float64), tok, tgt, B, T)
+    m = g2.GPT2(*cfg.args, seed=0, precision=precision, B=B, T=T)
+    m.set_params(params)
+    t, y = tok_tensors(tok, tgt)
+    loss = m.evaluate(t, y)
+    tol = 1e-4 if precision == "fp32" else 2e-2
+    assert abs(loss - rloss) <= tol, (loss, rloss)
+    assert abs(math.exp(loss) - math.exp(rloss)) <= 2 * tol * math.exp(rloss)  # perplexity
+    eval_losses = m.get_losses(B * T)
+    eval_logits = m.logits(B, T).clone()
+    with pytest.raises(g2.GPT2Error):
+        m.backward(1.0)
+    m.forward(t)  # no targets: logits only
+    assert torch.equal(m.logits(B, T), eval_logits)
+    # the training forward gives the same losses bit for bit; a step after
+    # an evaluation equals a step without one
+    m.zero_grad()
+    assert m.forward(t, y) == loss
+    assert np.array_equal(m.get_losses(B * T), eval_losses)
+    m.backward(1.0)
+    g_after = m.get_grads()
+    m.close()
+    m2 = g2.GPT2(*cfg.args, seed=0, precision=precision, B=B, T=T)
+    m2.set_params(params)
+    m2.zero_grad()
+    m2.forward(t, y)
+    m2.backward(1.0)
+    assert np.array_equal(m2.get_grads(), g_after)
+    m2.close()
+
+
+def test_evaluate_at_a_smaller_batch_than_reserved():
+    name, cfg, B, T, iid = CASES[0]
+    tok, tgt = batch_for(cfg, B, T, iid, seed=4)
+    params = Oracle(cfg).init(0).astype(np.float32)
+    m = g2.GPT2(*cfg.args, seed=0, precision="bf16", B=B, T=T)
+    m.set_params(params)
+    t, y = tok_tensors(tok[:1, : T // 2], tgt[:1, : T // 2])
+    loss = m.evaluate(t.contiguous(), y.contiguous())
+    rloss, _, _ = Oracle(cfg).forward(params.astype(np.float64), tok[:1, : T // 2], tgt[:1, : T // 2],
+                                      1, T // 2)
+    assert abs(loss - rloss) <= 2e-2
+    m.close()
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_recompute_is_bit_identical(precision):
+    # GELU recomputed in the backward from the stored pre-activation gives
+    # the same loss, gradients and updated parameters bit for bit, in a
+    # workspace smaller by (L - 1) B T 4C activations
+    name, cfg, B, T, iid = CASES[1]
+    tok, tgt = batch_for(cfg, B, T, iid, seed=5)
+    params = Oracle(cfg).init(0).astype(np.float32)
+    out = []
+    for level in (0, 1):
+        m = g2.GPT2(*cfg.args, seed=0, precision=precision, B=B, T=T, recompute=level)
+        m.set_params(params)
+        t, y = tok_tensors(tok, tgt)
+        m.zero_grad()
+        loss = m.forward(t, y)
+        m.backward(1.0)
+        grads = m.get_grads()
+        m.grad_norm_clip(1.0)
+        m.adamw_step(6e-4, 0.9, 0.95, 1e-8, 0.1)
+        out.append((loss, grads, m.get_params(), m.workspace_bytes(B, T)))
+        if level:
+            with pytest.raises(g2.GPT2Error):
+                m.read_activation("gelu", 0, B * T * 4 * cfg.C)
+        m.close()
+    (l0, g0, p0, w0), (l1, g1, p1, w1) = out
+    assert l0 == l1
+    assert np.array_equal(g0, g1)
+    assert np.array_equal(p0, p1)
+    elt = 4 if precision == "fp32" else 2
+    saved = (cfg.L - 1) * B * T * 4 * cfg.C * elt
+    assert saved - 1024 <= w0 - w1 <= saved + 1024

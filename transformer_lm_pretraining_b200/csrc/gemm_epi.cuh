@@ -37,10 +37,10 @@ __device__ __forceinline__ void epi_scalar(const EpiParams& e, int m, int n, flo
     if (e.bias) v += e.bias[n];
   }
   if (EPI == EPI_BIAS_RESID) v += to_f(e.resid[(size_t)m * e.ldr + n]);
-  if (EPI == EPI_BIAS_GELU) {
+  if (EPI == EPI_BIAS_GELU) {  // GELU of u as stored, so that it can be recomputed from u
     const act_t u = from_f<act_t>(v);
     e.aux[(size_t)m * e.ldaux + n] = u;
-    v = gelu_tanh(v);
+    v = gelu_tanh(to_f(u));
   }
   e.out[(size_t)m * e.ldo + n] = from_f<act_t>(v);
 }
@@ -100,12 +100,12 @@ __device__ __forceinline__ void epi_row32(const EpiParams& e, int m, int n0, flo
         for (int i = 0; i < 8; ++i) v[8 * j + i] += x[i];
       }
     }
-    if (EPI == EPI_BIAS_GELU) {
+    if (EPI == EPI_BIAS_GELU) {  // GELU of u as stored, so that it can be recomputed from u
       act_t* a = e.aux + (size_t)m * e.ldaux + n0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) store8(a + 8 * j, v + 8 * j);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+      for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(to_f(from_f<act_t>(v[i])));
     }
   }
   act_t* o = e.out + (size_t)m * e.ldo + n0;

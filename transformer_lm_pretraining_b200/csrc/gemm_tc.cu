@@ -429,11 +429,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           if (EPI == EPI_BIAS_GELU) {
-            // the pre-activation u first (saved for the backward), then GELU(u)
+            // the pre-activation u first (saved for the backward), then GELU
+            // of u as stored (bf16), which a backward that recomputes GELU
+            // from u reproduces bit for bit
+            uint4 up[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&up[j]);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                h2[i] = __floats2bfloat162_rn(v[8 * j + 2 * i], v[8 * j + 2 * i + 1]);
+                const float2 f = __bfloat1622float2(h2[i]);
+                v[8 * j + 2 * i] = f.x;
+                v[8 * j + 2 * i + 1] = f.y;
+              }
+            }
             put_box(
                 [&](uint8_t* box) {
 #pragma unroll
-                  for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(box + swz(lane, j)), v + 8 * j);
+                  for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4*>(box + swz(lane, j)) = up[j];
                 },
                 [&](uint32_t box_u) { tma_store_3d(&tmX, box_u, nb, r0, 0); });
 #pragma unroll

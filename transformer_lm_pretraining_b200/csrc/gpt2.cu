@@ -46,7 +46,7 @@ constexpr int kMaxSplits = 8;
 // Optional per-kernel-family timing with CUDA events on the handle's stream.
 enum ProfKind {
   PK_GEMM, PK_ATTN_FWD, PK_ATTN_BWD, PK_LAYERNORM, PK_LN_BWD, PK_CLASSIFIER, PK_ENCODER,
-  PK_COLSUM, PK_OPTIMIZER, PK_COUNT
+  PK_COLSUM, PK_OPTIMIZER, PK_RECOMPUTE, PK_COUNT
 };
 
 struct ProfRec {
@@ -75,6 +75,7 @@ struct gpt2 {
   void* work = nullptr;
   size_t work_bytes = 0;
   bool own_work = false;
+  int recompute = 0;  // 1: GELU outputs are not kept; the backward recomputes them
   // forward record
   int B = 0, T = 0;
   bool have_grad_logits = false;
@@ -127,7 +128,7 @@ size_t carve_state(const Layout& lay, void* base, gpt2_t* h) {
 }
 
 // Layout of the workspace for B x T tokens.
-size_t carve_work(const Layout& lay, int B, int T, void* base, Acts* a) {
+size_t carve_work(const Layout& lay, int B, int T, int recompute, void* base, Acts* a) {
   const size_t M = (size_t)B * T, C = lay.C, L = lay.L, H = lay.H;
   Carver c(base);
   Acts x{};
@@ -138,7 +139,7 @@ size_t carve_work(const Layout& lay, int B, int T, void* base, Acts* a) {
   x.xmid = c.take<act_t>(L * M * C);
   x.h2 = c.take<act_t>(L * M * C);
   x.u = c.take<act_t>(L * M * 4 * C);
-  x.g = c.take<act_t>(L * M * 4 * C);
+  x.g = c.take<act_t>((recompute ? 1 : L) * M * 4 * C);  // one layer's worth when recomputed
   x.hf = c.take<act_t>(M * C);
   x.logits = c.take<act_t>(M * (size_t)lay.Vp);
   x.mean1 = c.take<float>(L * M);
@@ -193,7 +194,7 @@ gpt2_status ensure_state(gpt2_t* h) {
 }
 
 gpt2_status ensure_work(gpt2_t* h, int B, int T) {
-  const size_t need = carve_work(h->lay, B, T, nullptr, nullptr);
+  const size_t need = carve_work(h->lay, B, T, h->recompute, nullptr, nullptr);
   if (h->work && h->work_bytes >= need) return GPT2_OK;
   if (h->work && !h->own_work)
     return fail(h, GPT2_ERR_ARG, "bound workspace is smaller than gpt2_workspace_bytes(B, T)");
@@ -304,7 +305,7 @@ size_t gpt2_state_bytes(const gpt2_t* h) { return h ? carve_state(h->lay, nullpt
 
 size_t gpt2_workspace_bytes(const gpt2_t* h, int B, int T) {
   if (!h || B < 1 || T < 1) return 0;
-  return carve_work(h->lay, B, T, nullptr, nullptr);
+  return carve_work(h->lay, B, T, h->recompute, nullptr, nullptr);
 }
 
 gpt2_status gpt2_bind_memory(gpt2_t* h, void* dev_state, size_t state_bytes, void* dev_work,
@@ -347,14 +348,27 @@ gpt2_status gpt2_bind_memory(gpt2_t* h, void* dev_state, size_t state_bytes, voi
   return GPT2_OK;
 }
 
+gpt2_status gpt2_set_recompute(gpt2_t* h, int level) {
+  if (!h || level < 0 || level > 1) return fail(h, GPT2_ERR_ARG, "recompute level is 0 or 1");
+  if (level != h->recompute) {
+    h->recompute = level;
+    h->have_grad_logits = h->have_logits = false;  // the workspace layout changed
+  }
+  return GPT2_OK;
+}
+
 gpt2_status gpt2_set_stream(gpt2_t* h, void* cuda_stream) {
   if (!h) return GPT2_ERR_ARG;
   h->stream = static_cast<cudaStream_t>(cuda_stream);
   return GPT2_OK;
 }
 
-gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int B, int T,
-                         float* loss_host) {
+namespace {
+
+// The forward pass; `train` leaves dL/dlogits in the logits buffer for the
+// backward, otherwise (evaluation) the logits are kept as computed.
+gpt2_status forward_impl(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int B, int T,
+                         float* loss_host, bool train) {
   if (!h || !tok || B < 1 || T < 1) return fail(h, GPT2_ERR_ARG, "bad forward arguments");
   const Layout& y = h->lay;
   if (T > y.Tmax) return fail(h, GPT2_ERR_ARG, "T > Tmax");
@@ -363,7 +377,7 @@ gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int 
   st = ensure_work(h, B, T);
   if (st) return st;
   Acts& a = h->a;
-  carve_work(y, B, T, h->work, &a);
+  carve_work(y, B, T, h->recompute, h->work, &a);
   h->B = B;
   h->T = T;
   const int M = B * T, C = y.C, L = y.L, H = y.H;
@@ -382,7 +396,7 @@ gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int 
     act_t* xm = a.xmid + (size_t)l * MC;
     act_t* h2 = a.h2 + (size_t)l * MC;
     act_t* u = a.u + (size_t)l * 4 * MC;
-    act_t* g = a.g + (size_t)l * 4 * MC;
+    act_t* g = a.g + (h->recompute ? 0 : (size_t)l * 4 * MC);
     mark(h, PK_LAYERNORM);
     layernorm_fwd(h1, a.mean1 + (size_t)l * M, a.rstd1 + (size_t)l * M, x,
                   P + y.off[T_LN1G] + (size_t)l * C, P + y.off[T_LN1B] + (size_t)l * C, M, C, s);
@@ -442,9 +456,10 @@ gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int 
   h->have_logits = false;
   if (tgt) {
     mark(h, PK_CLASSIFIER);
-    classifier(a.logits, a.losses, tgt, M, y.V, y.Vp, 1, h->err, s);
+    classifier(a.logits, a.losses, tgt, M, y.V, y.Vp, train ? 1 : 0, h->err, s);
     mean_loss(h->scalars + S_LOSS, a.losses, M, s);
-    h->have_grad_logits = true;
+    h->have_grad_logits = train;
+    h->have_logits = !train;
   } else {
     h->have_logits = true;
   }
@@ -458,6 +473,19 @@ gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int 
     if (tgt && !std::isfinite(*loss_host)) return fail(h, GPT2_ERR_NONFINITE, "loss is not finite");
   }
   return GPT2_OK;
+}
+
+}  // namespace
+
+gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int B, int T,
+                         float* loss_host) {
+  return forward_impl(h, tok, tgt, B, T, loss_host, true);
+}
+
+gpt2_status gpt2_evaluate(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int B, int T,
+                          float* loss_host) {
+  if (!tgt) return fail(h, GPT2_ERR_ARG, "evaluation needs targets");
+  return forward_impl(h, tok, tgt, B, T, loss_host, false);
 }
 
 gpt2_status gpt2_read_loss(gpt2_t* h, float* loss_host) {
@@ -522,7 +550,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     const act_t* xm = a.xmid + (size_t)l * MC;
     const act_t* h2 = a.h2 + (size_t)l * MC;
     const act_t* u = a.u + (size_t)l * 4 * MC;
-    const act_t* g = a.g + (size_t)l * 4 * MC;
+    const act_t* g = a.g + (h->recompute ? 0 : (size_t)l * 4 * MC);
     // ---- MLP: x_next = xm + gelu(h2 Wfc^T + bfc) Wp^T + bp
     {  // du = (dres Wp) * gelu'(u)
       GemmArgs ga = gemm_args(M, 4 * C, C);
@@ -531,6 +559,10 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.epi = EPI_DGELU; ga.aux = const_cast<act_t*>(u); ga.ldaux = 4 * C;
       ga.out = a.dbig; ga.ldo = 4 * C;
       GPT2_TRY(run_gemm(h, ga));
+    }
+    if (h->recompute) {  // g = gelu(u), as the forward's epilogue computed it
+      mark(h, PK_RECOMPUTE);
+      gelu_fwd(const_cast<act_t*>(g), u, 4 * MC, s);
     }
     {  // dWp += dres^T g
       GemmArgs ga = gemm_args(C, 4 * C, M);
@@ -794,7 +826,11 @@ gpt2_status gpt2_read_activation(const gpt2_t* hc, int kind, int layer, float* h
     case 4: src = a.xmid + layer * M * C; cnt = M * C; break;
     case 5: src = a.h2 + layer * M * C; cnt = M * C; break;
     case 6: src = a.u + layer * 4 * M * C; cnt = 4 * M * C; break;
-    case 7: src = a.g + layer * 4 * M * C; cnt = 4 * M * C; break;
+    case 7:
+      if (h->recompute) return fail(h, GPT2_ERR_STATE, "GELU outputs are not kept (recompute)");
+      src = a.g + layer * 4 * M * C;
+      cnt = 4 * M * C;
+      break;
     case 8: src = a.hf; cnt = M * C; break;
     default: return GPT2_ERR_ARG;
   }

@@ -119,6 +119,10 @@ void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int 
 // out[0] = mean of losses[0..M) (fixed-order reduction)
 void mean_loss(float* out, const float* losses, int M, cudaStream_t s);
 
+// g = GELU_tanh(u) elementwise (n elements, activation dtype); the same
+// function the fc GEMM's epilogue applies to the stored u.
+void gelu_fwd(act_t* g, const act_t* u, size_t n, cudaStream_t s);
+
 // ----------------------------------------------------------- optimizer --
 void init_params(float* p, const Layout& lay, uint64_t seed, cudaStream_t s);
 void f32_to_act(act_t* out, const float* in, size_t n, cudaStream_t s);

@@ -570,6 +570,29 @@ void mean_loss(float* out, const float* losses, int M, cudaStream_t s) {
   note_launch();
 }
 
+namespace {
+__global__ void gelu_fwd_kernel(act_t* __restrict__ g, const act_t* __restrict__ u, size_t n) {
+  const size_t n8 = n / 8;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float v[8];
+    load8(u + 8 * i, v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = gelu_tanh(v[k]);
+    store8(g + 8 * i, v);
+  }
+  for (size_t i = 8 * n8 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    g[i] = from_f<act_t>(gelu_tanh(to_f(u[i])));
+}
+}  // namespace
+
+void gelu_fwd(act_t* g, const act_t* u, size_t n, cudaStream_t s) {
+  if (!n) return;
+  gelu_fwd_kernel<<<grid_for(n / 8 + 1, 256, 8 * kNumSMs), 256, 0, s>>>(g, u, n);
+  note_launch();
+}
+
 void init_params(float* p, const Layout& lay, uint64_t seed, cudaStream_t s) {
   cudaMemsetAsync(p, 0, lay.total * sizeof(float), s);
   const int gains[3] = {T_LN1G, T_LN2G, T_LNFG};

@@ -27,7 +27,7 @@ ACT_NAMES = {"residual": 0, "ln1": 1, "qkv": 2, "attn": 3, "xmid": 4, "ln2": 5,
 EPI = {"store": 0, "bias": 1, "bias_gelu": 2, "bias_resid": 3, "dgelu": 4, "f32_acc": 5}
 
 PROF_KINDS = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "classifier", "encoder",
-              "colsum", "optimizer")
+              "colsum", "optimizer", "recompute")
 
 # name -> (restype, argtypes)
 _vp, _sz, _i, _f, _d, _l, _u64 = (ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float,
@@ -43,6 +43,8 @@ SIGNATURES = {
     "gpt2_bind_memory": (_i, [_vp, _vp, _sz, _vp, _sz]),
     "gpt2_set_stream": (_i, [_vp, _vp]),
     "gpt2_forward": (_i, [_vp, _vp, _vp, _i, _i, _fp]),
+    "gpt2_evaluate": (_i, [_vp, _vp, _vp, _i, _i, _fp]),
+    "gpt2_set_recompute": (_i, [_vp, _i]),
     "gpt2_zero_grad": (_i, [_vp]),
     "gpt2_read_loss": (_i, [_vp, _fp]),
     "gpt2_backward": (_i, [_vp, _f]),
@@ -117,7 +119,8 @@ def _dptr(t) -> int | None:
 class GPT2:
     """One model + optimiser state on the current CUDA device."""
 
-    def __init__(self, L, H, C, V, Vp, Tmax, seed=0, precision="bf16", B=None, T=None):
+    def __init__(self, L, H, C, V, Vp, Tmax, seed=0, precision="bf16", B=None, T=None,
+                 recompute=0):
         import torch
 
         self.torch = torch
@@ -134,6 +137,7 @@ class GPT2:
         self._work = None
         self.set_stream()
         self._check(self.lib.gpt2_bind_memory(h, self._state.data_ptr(), self._state.numel(), None, 0))
+        self._check(self.lib.gpt2_set_recompute(h, int(recompute)))
         if B is not None:
             self.reserve(B, T)
 
@@ -176,6 +180,31 @@ class GPT2:
         self._check(self.lib.gpt2_forward(self.h, _dptr(tok), _dptr(tgt), B, T,
                                           ctypes.byref(out) if sync_loss else None))
         return out.value if sync_loss else None
+
+    def evaluate(self, tok, tgt, sync_loss=True):
+        """Mean loss of a forward-only pass (no gradient is written, no
+        backward may follow); perplexity = exp(loss)."""
+        B, T = tok.shape
+        self.reserve(B, T)
+        out = ctypes.c_float(float("nan"))
+        self._check(self.lib.gpt2_evaluate(self.h, _dptr(tok), _dptr(tgt), B, T,
+                                           ctypes.byref(out) if sync_loss else None))
+        return out.value if sync_loss else None
+
+    def logits(self, B, T):
+        """The logits buffer [B*T, Vpad] (a view into the workspace, activation
+        dtype) after a forward without targets or an evaluation."""
+        torch = self.torch
+        ptr = ctypes.c_void_p()
+        self._check(self.lib.gpt2_logits(self.h, ctypes.byref(ptr)))
+        bf16 = self.precision == "bf16"
+
+        class _View:  # CUDA array interface over the library's buffer
+            __cuda_array_interface__ = {"shape": (B * T, self.cfg[4]), "typestr": "<i2" if bf16 else "<f4",
+                                        "data": (ptr.value, False), "version": 2}
+
+        t = torch.as_tensor(_View(), device="cuda")
+        return t.view(torch.bfloat16) if bf16 else t
 
     def zero_grad(self):
         self._check(self.lib.gpt2_zero_grad(self.h))
