@@ -168,6 +168,126 @@ __global__ void __launch_bounds__(256, 2)
   }
 }
 
+// Row-group variant for C = 8 * TPR with TPR (threads per row) a multiple
+// of 32: a block takes RPB rows at a time, TPR threads to a row and 8
+// columns to a thread, so every thread keeps the three column sums of its 8
+// columns in registers across all its rows, and gamma in registers too.
+// The two row reductions go through a warp shuffle and, across the row's
+// warps, shared memory (one barrier per group of rows, double-buffered).
+// The next group's rows are loaded while the current one is computed.
+// partials[blk][0..NSUMS) as the per-warp kernel.
+template <int TPR, int NSUMS>
+__global__ void __launch_bounds__(TPR * (TPR >= 256 ? 1 : 256 / TPR), 2)
+    ln_bwd_rows_kernel(act_t* __restrict__ dres, const act_t* __restrict__ dy,
+                       const act_t* __restrict__ x, const float* __restrict__ mean,
+                       const float* __restrict__ rstd, const float* __restrict__ g,
+                       float* __restrict__ partials, int M, int accumulate) {
+  constexpr int RPB = TPR >= 256 ? 1 : 256 / TPR;  // rows per group
+  constexpr int WPR = TPR / 32;                      // warps per row
+  constexpr int C = 8 * TPR;
+  __shared__ float red[2][RPB][WPR][2];
+  extern __shared__ float sums[];  // [RPB][NSUMS][C] at the end
+  const int slot = threadIdx.x / TPR, tc = threadIdx.x % TPR;
+  const int wr = tc / 32, lane = threadIdx.x & 31;
+  const int c = tc * 8;
+  const int stride = gridDim.x * RPB;
+  float gg[8], s0[8], s1[8], s2[8];
+  load8(g + c, gg);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s0[i] = s1[i] = s2[i] = 0.f;
+  Pack8 px, pd, po;
+  float mu = 0.f, rs = 0.f;
+  auto fetch = [&](int row) {
+    if (row >= M) return;
+    px = *reinterpret_cast<const Pack8*>(x + (size_t)row * C + c);
+    pd = *reinterpret_cast<const Pack8*>(dy + (size_t)row * C + c);
+    if (accumulate) po = *reinterpret_cast<const Pack8*>(dres + (size_t)row * C + c);
+    mu = mean[row];
+    rs = rstd[row];
+  };
+  int row = blockIdx.x * RPB + slot;
+  fetch(row);
+  for (int it = 0; blockIdx.x * RPB + it * stride < M; ++it, row += stride) {
+    const Pack8 cx = px, cd = pd, co = po;
+    const float crs = rs, nmr = -mu * rs;
+    const bool live = row < M;
+    fetch(row + stride);  // in flight while this group is computed
+    float xh[8], dxh[8], a = 0.f, b = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      xh[i] = fmaf(to_f(cx.v[i]), crs, nmr);
+      const float d = live ? to_f(cd.v[i]) : 0.f;
+      dxh[i] = d * gg[i];
+      a += dxh[i];
+      b = fmaf(dxh[i], xh[i], b);
+      s0[i] = fmaf(d, xh[i], s0[i]);
+      s1[i] += d;
+    }
+    a = warp_sum(a);
+    b = warp_sum(b);
+    float* rr = &red[it & 1][slot][0][0];
+    if (lane == 0) {
+      rr[2 * wr] = a;
+      rr[2 * wr + 1] = b;
+    }
+    __syncthreads();
+    a = 0.f;
+    b = 0.f;
+#pragma unroll
+    for (int w = 0; w < WPR; ++w) {
+      a += rr[2 * w];
+      b += rr[2 * w + 1];
+    }
+    a *= 1.0f / C;
+    b *= 1.0f / C;
+    if (live) {
+      Pack8 q;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float t = fmaf(-xh[i], b, dxh[i] - a);
+        const float o = accumulate ? fmaf(crs, t, to_f(co.v[i])) : crs * t;
+        q.v[i] = from_f<act_t>(o);
+        if (NSUMS == 3) s2[i] += to_f(q.v[i]);  // the bias gradient sums the values as stored
+      }
+      *reinterpret_cast<Pack8*>(dres + (size_t)row * C + c) = q;
+    }
+  }
+  // block reduction over the row slots, in slot order
+  float* mine = sums + (size_t)slot * NSUMS * C;
+  store8(mine + c, s0);
+  store8(mine + C + c, s1);
+  if (NSUMS == 3) store8(mine + 2 * C + c, s2);
+  __syncthreads();
+  for (int i = threadIdx.x; i < NSUMS * C; i += blockDim.x) {
+    float t = 0.f;
+    for (int k = 0; k < RPB; ++k) t += sums[(size_t)k * NSUMS * C + i];
+    partials[(size_t)blockIdx.x * NSUMS * C + i] = t;
+  }
+}
+
+template <int TPR, int S>
+int ln_bwd_rows_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
+                       const float* rstd, const float* g, float* partials, int M,
+                       int accumulate, cudaStream_t s) {
+  constexpr int RPB = TPR >= 256 ? 1 : 256 / TPR;
+  constexpr int threads = TPR * RPB;
+  constexpr size_t smem = (size_t)RPB * S * 8 * TPR * sizeof(float);
+  static int grid = 0;
+  if (!grid) {
+    cudaFuncSetAttribute(ln_bwd_rows_kernel<TPR, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    int per_sm = 0, sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_bwd_rows_kernel<TPR, S>, threads, smem);
+    grid = per_sm * sms;
+    if (grid < 1 || grid > kLnBlocks) grid = kLnBlocks;
+  }
+  ln_bwd_rows_kernel<TPR, S><<<grid, threads, smem, s>>>(dres, dy, x, mean, rstd, g, partials, M,
+                                                         accumulate);
+  return grid;
+}
+
 // out_j[c] += sum over blocks of partials[blk][j][c] in a fixed order:
 // thread (tx, ty) of a 32 x 32 block takes column tx of a 32-column group
 // and blocks ty, ty+32, ... (four independent running sums, combined in a
@@ -251,6 +371,18 @@ void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* me
                    float* partials, int M, int C, int accumulate, cudaStream_t s) {
   const int nsums = dbias_out ? 3 : 2;
   int nblk = kLnBlocks;
+  switch (C * 4 + nsums) {  // widths with a row-group kernel
+#define GPT2_LNR(W)                                                                            \
+  case 4 * W + 2:                                                                              \
+    nblk = ln_bwd_rows_launch<W / 8, 2>(dres, dy, x, mean, rstd, g, partials, M, accumulate, s); \
+    goto reduce;                                                                               \
+  case 4 * W + 3:                                                                              \
+    nblk = ln_bwd_rows_launch<W / 8, 3>(dres, dy, x, mean, rstd, g, partials, M, accumulate, s); \
+    goto reduce;
+    GPT2_LNR(256) GPT2_LNR(512) GPT2_LNR(768) GPT2_LNR(1024) GPT2_LNR(2048)
+#undef GPT2_LNR
+    default: break;
+  }
   switch ((C + 255) / 256 * 4 + nsums) {
 #define GPT2_LNB(N)                                                                          \
   case 4 * N + 2:                                                                            \
@@ -263,6 +395,7 @@ void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* me
 #undef GPT2_LNB
     default: break;
   }
+reduce:
   ln_bwd_reduce_kernel<<<(nsums * C + 31) / 32, 1024, 0, s>>>(dg, db, dbias_out, partials, nblk,
                                                                nsums, C);
   note_launch(2);
