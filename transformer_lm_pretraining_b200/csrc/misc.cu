@@ -65,20 +65,25 @@ __global__ void __launch_bounds__(256)
   float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (n < N) {
     int r = r0 + w;
-    for (; r + 24 < r1; r += 32) {  // four rows in flight
-      float a[8], b[8], c[8], d[8];
-      load8(dy + (size_t)r * N + n, a);
-      load8(dy + (size_t)(r + 8) * N + n, b);
-      load8(dy + (size_t)(r + 16) * N + n, c);
-      load8(dy + (size_t)(r + 24) * N + n, d);
+    // eight rows in flight, loaded as raw 16-byte vectors and converted after
+    struct alignas(16) Row8 {
+      act_t v[8];
+    };
+    for (; r < r1; r += 64) {  // one round trip per 8 rows, the last batch guarded
+      Row8 q[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) s[i] = (((s[i] + a[i]) + b[i]) + c[i]) + d[i];
-    }
-    for (; r < r1; r += 8) {
-      float a[8];
-      load8(dy + (size_t)r * N + n, a);
+      for (int k = 0; k < 8; ++k) {
+        if (r + 8 * k < r1) {
+          q[k] = *reinterpret_cast<const Row8*>(dy + (size_t)(r + 8 * k) * N + n);
+        } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) s[i] += a[i];
+          for (int i = 0; i < 8; ++i) q[k].v[i] = from_f<act_t>(0.f);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[i] += to_f(q[k].v[i]);
     }
   }
 #pragma unroll
@@ -528,9 +533,9 @@ int grid_for(size_t n, int threads, int max_blocks) {
 }  // namespace
 
 void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s) {
-  // enough chunks for ~4 blocks per SM
+  // enough chunks for ~8 blocks per SM
   const int colgroups = (N + 255) / 256;
-  int want = (4 * kNumSMs + colgroups - 1) / colgroups;
+  int want = (8 * kNumSMs + colgroups - 1) / colgroups;
   if (want > kColsumChunks) want = kColsumChunks;
   const int rows = (M + want - 1) / want;
   const int chunks = (M + rows - 1) / rows;
