@@ -276,44 +276,58 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         ok = cbar_and(mbar_wait(sd_full, gt & 1u, abort_flag, err));
         if (!ok) break;
         tc_fence_after();
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {  // 32 query columns at a time
-          uint32_t rs[32], rp[32];
-          const uint32_t col = (uint32_t)(64 * half + 32 * ch);
-          tc_ld32(lane_base + col, rs);
-          tc_ld32(lane_base + kTile + col, rp);
-          float pv[32], dv[32];
+        // 16 query columns per chunk; the next chunk's TMEM loads are in
+        // flight while the current chunk is computed
+        uint32_t sa[16], pa[16], sb[16], pb[16];
+        auto ld_chunk = [&](int ch, uint32_t* s_, uint32_t* p_) {
+          const uint32_t col = (uint32_t)(64 * half + 16 * ch);
+          attn::tc_ld16(lane_base + col, s_);
+          attn::tc_ld16(lane_base + kTile + col, p_);
+        };
+        auto do_chunk = [&](int ch, const uint32_t* s_, const uint32_t* p_) -> bool {
+          const int col = 64 * half + 16 * ch;
+          float pv[16], dv[16];
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
+          for (int c = 0; c < 16; c += 4) {
             const float4 a = *reinterpret_cast<const float4*>(cl + col + c);
             const float4 d = *reinterpret_cast<const float4*>(cl + kTile + col + c);
             pv[c] = a.x; pv[c + 1] = a.y; pv[c + 2] = a.z; pv[c + 3] = a.w;
             dv[c] = d.x; dv[c + 1] = d.y; dv[c + 2] = d.z; dv[c + 3] = d.w;
           }
-          tc_wait_ld();
-          if (ch == 1) {  // both score buffers are read: the next tile's may be computed
-            tc_fence_before();
-            mbar_arrive(sd_empty);
-          }
-          const int lim = kj - qc0 - 32 * ch;  // columns c < lim are queries before the key
-          const int tcut = T - qc0 - 32 * ch;  // columns c >= tcut are past the sequence
+          const int lim = kj - qc0 - 16 * ch;  // columns c < lim are queries before the key
+          const int tcut = T - qc0 - 16 * ch;  // columns c >= tcut are past the sequence
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float p = fast_exp2(fmaf(__uint_as_float(rs[c]), sl2, -pv[c]));
+          for (int c = 0; c < 16; ++c) {
+            float p = fast_exp2(fmaf(__uint_as_float(s_[c]), sl2, -pv[c]));
             if (c < lim || c >= tcut) p = 0.f;  // causal (only bites when i == j) and padding
             pv[c] = p;
-            dv[c] = p * (__uint_as_float(rp[c]) - dv[c]);
+            dv[c] = p * (__uint_as_float(p_[c]) - dv[c]);
           }
-          if (ch == 0) {  // the previous tile's products have read P^T and dS^T
-            ok = cbar_and(mbar_wait(pd_empty, (gt & 1u) ^ 1u, abort_flag, err));
-            if (!ok) break;
-          }
+          // the previous tile's products have read P^T and dS^T
+          if (ch == 0 && !cbar_and(mbar_wait(pd_empty, (gt & 1u) ^ 1u, abort_flag, err))) return false;
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            const uint32_t off = (uint32_t)(((4 * ch + c8) ^ (r & 7)) << 4);
+          for (int c8 = 0; c8 < 2; ++c8) {
+            const uint32_t off = (uint32_t)(((2 * ch + c8) ^ (r & 7)) << 4);
             attn::st_shared_bf16x8(pt_row + off, pv + 8 * c8);
             attn::st_shared_bf16x8(dst_row + off, dv + 8 * c8);
           }
+          return true;
+        };
+        ld_chunk(0, sa, pa);
+        tc_wait_ld();
+        ld_chunk(1, sb, pb);
+        ok = do_chunk(0, sa, pa);
+        tc_wait_ld();
+        if (ok) {
+          ld_chunk(2, sa, pa);
+          do_chunk(1, sb, pb);
+          tc_wait_ld();
+          ld_chunk(3, sb, pb);
+          do_chunk(2, sa, pa);
+          tc_wait_ld();
+          tc_fence_before();
+          mbar_arrive(sd_empty);  // both score buffers are read: the next tile's may be computed
+          do_chunk(3, sb, pb);
         }
         if (!ok) break;
         fence_async_smem();
@@ -543,33 +557,48 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         ok = warp_and(mbar_wait(sd_full, gg & 1u, abort_flag, err));
         if (!ok) break;
         tc_fence_after();
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {  // 32 key columns at a time
-          uint32_t rs[32], rp[32];
-          const uint32_t col = (uint32_t)(64 * half + 32 * ch);
-          tc_ld32(lane_base + col, rs);
-          tc_ld32(lane_base + kTile + col, rp);
-          tc_wait_ld();
-          if (ch == 1) {  // both score buffers are read: the next tile's may be computed
-            tc_fence_before();
-            mbar_arrive(sd_empty);
-          }
-          const int lim = qi - key0 - 32 * ch;  // columns c > lim are keys after the query
-          const int tcut = T - key0 - 32 * ch;  // columns c >= tcut are past the sequence
-          float ds[32];
+        // 16 key columns per chunk; the next chunk's TMEM loads are in
+        // flight while the current chunk is computed
+        uint32_t sa[16], pa[16], sb[16], pb[16];
+        auto ld_chunk = [&](int ch, uint32_t* s_, uint32_t* p_) {
+          const uint32_t col = (uint32_t)(64 * half + 16 * ch);
+          attn::tc_ld16(lane_base + col, s_);
+          attn::tc_ld16(lane_base + kTile + col, p_);
+        };
+        auto do_chunk = [&](int ch, const uint32_t* s_, const uint32_t* p_) -> bool {
+          const int lim = qi - key0 - 16 * ch;  // columns c > lim are keys after the query
+          const int tcut = T - key0 - 16 * ch;  // columns c >= tcut are past the sequence
+          float ds[16];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float p = fast_exp2(fmaf(__uint_as_float(rs[c]), sl2, -lse2));
+          for (int c = 0; c < 16; ++c) {
+            float p = fast_exp2(fmaf(__uint_as_float(s_[c]), sl2, -lse2));
             if (c > lim || c >= tcut) p = 0.f;  // causal (only bites on the diagonal) and padding
-            ds[c] = p * (__uint_as_float(rp[c]) - drow);
+            ds[c] = p * (__uint_as_float(p_[c]) - drow);
           }
-          if (ch == 0) {  // the product two tiles back has read this dS buffer
-            ok = warp_and(mbar_wait(ds_empty0 + 8 * db, ((gg >> 1) & 1u) ^ 1u, abort_flag, err));
-            if (!ok) break;
-          }
+          // the product two tiles back has read this dS buffer
+          if (ch == 0 &&
+              !warp_and(mbar_wait(ds_empty0 + 8 * db, ((gg >> 1) & 1u) ^ 1u, abort_flag, err)))
+            return false;
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8)
-            attn::st_shared_bf16x8(ds_row + (uint32_t)(((4 * ch + c8) ^ (r & 7)) << 4), ds + 8 * c8);
+          for (int c8 = 0; c8 < 2; ++c8)
+            attn::st_shared_bf16x8(ds_row + (uint32_t)(((2 * ch + c8) ^ (r & 7)) << 4), ds + 8 * c8);
+          return true;
+        };
+        ld_chunk(0, sa, pa);
+        tc_wait_ld();
+        ld_chunk(1, sb, pb);
+        ok = do_chunk(0, sa, pa);
+        tc_wait_ld();
+        if (ok) {
+          ld_chunk(2, sa, pa);
+          do_chunk(1, sb, pb);
+          tc_wait_ld();
+          ld_chunk(3, sb, pb);
+          do_chunk(2, sa, pa);
+          tc_wait_ld();
+          tc_fence_before();
+          mbar_arrive(sd_empty);  // both score buffers are read: the next tile's may be computed
+          do_chunk(3, sb, pb);
         }
         if (!ok) break;
         fence_async_smem();

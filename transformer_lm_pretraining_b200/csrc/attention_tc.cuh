@@ -23,6 +23,17 @@ __host__ __device__ constexpr uint32_t idesc(int n, bool b_mn) {
 // one sequence (rows past T read as zero).
 cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols);
 
+// 32 lanes x 16 consecutive 32-bit TMEM columns (thread i: row lane base + i).
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 // 8 floats -> 8 bf16 (round to nearest) stored as 16 bytes at a 32-bit
 // shared-memory address (no 64-bit generic addresses to keep live).
 __device__ __forceinline__ void st_shared_bf16x8(uint32_t addr, const float* v) {
