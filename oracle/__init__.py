@@ -108,6 +108,9 @@ def lib(openmp: bool = False) -> ctypes.CDLL:
         fn = getattr(L, f"orc_softmax_xent_{sfx}")
         fn.argtypes = [P, i, i, _I32, R, P, P]
         fn.restype = None
+        fn = getattr(L, f"orc_sample_token_{sfx}")
+        fn.argtypes = [P, i, R, i, d]
+        fn.restype = i
         fn = getattr(L, f"orc_attention_fwd_{sfx}")
         fn.argtypes = [P, P, i, i, i, i]
         fn.restype = None
@@ -312,6 +315,14 @@ class Oracle:
             self.ct(scale), _ptr(losses, self.ct), _ptr(dz, self.ct) if grad else None)
         return losses, dz
 
+    def sample_token(self, z, temperature=0.0, top_k=0, u=0.0):
+        """Next token from one row of logits: argmax at temperature 0, else
+        the first index where the cumulative softmax(z / temperature) over
+        the top_k logits exceeds u."""
+        z = np.ascontiguousarray(z, self.dtype)
+        return int(getattr(self.lib, f"orc_sample_token_{self.sfx}")(
+            _ptr(z, self.ct), z.size, self.ct(temperature), int(top_k), float(u)))
+
     def linear_fwd(self, x, W, b=None):
         x = np.ascontiguousarray(x, self.dtype)
         W = np.ascontiguousarray(W, self.dtype)
@@ -330,6 +341,12 @@ def lr(step, max_lr, min_lr, warmup, max_steps) -> float:
 
 def splitmix64(seed: int, n: int) -> int:
     return int(lib().orc_splitmix64(seed, n))
+
+
+def sample_uniform(seed: int, position: int, row: int) -> float:
+    """The uniform draw for the token at `position` of sequence `row`:
+    the SplitMix64 output n = position * 65536 + row of `seed`, top 53 bits."""
+    return (splitmix64(seed, position * 65536 + row) >> 11) * 2.0 ** -53
 
 
 def std_normal(seed: int, tensor: int, i: int) -> float:

@@ -41,6 +41,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <vector>
 #include <algorithm>
 #ifdef _OPENMP
@@ -380,6 +381,40 @@ void softmax_xent(const R* z, int M, int V, const int* tgt, R scale, R* losses, 
   }
 }
 
+// The next token from one row of V logits (generation loop of the pages).
+// temperature 0: the argmax (lowest index among equal maxima).  Otherwise
+// the softmax of z / temperature over the top_k largest logits (top_k <= 0
+// or >= V: all of them; logits equal to the k-th largest are kept), and the
+// token is the smallest v at which the cumulative probability exceeds u
+// (u uniform in [0, 1), a draw the caller passes in).
+template <class R>
+int sample_token(const R* z, int V, R temperature, int top_k, double u) {
+  int best = 0;
+  for (int v = 1; v < V; ++v)
+    if (z[v] > z[best]) best = v;
+  if (temperature <= R(0)) return best;
+  R thr = -INFINITY;
+  if (top_k > 0 && top_k < V) {
+    std::vector<R> sorted(z, z + V);
+    std::nth_element(sorted.begin(), sorted.begin() + (top_k - 1), sorted.end(), std::greater<R>());
+    thr = sorted[top_k - 1];
+  }
+  const R mx = z[best];
+  R total = 0;
+  for (int v = 0; v < V; ++v)
+    if (z[v] >= thr) total += std::exp((z[v] - mx) / temperature);
+  const R target = R(u) * total;
+  R cum = 0;
+  int last = best;
+  for (int v = 0; v < V; ++v) {
+    if (z[v] < thr) continue;
+    cum += std::exp((z[v] - mx) / temperature);
+    last = v;
+    if (cum > target) return v;
+  }
+  return last;
+}
+
 template <class R>
 struct Model {
   Cfg g;
@@ -649,6 +684,10 @@ uint64_t orc_splitmix64(uint64_t seed, uint64_t n) { return sm_output(seed, n); 
   void orc_softmax_xent_##SFX(const R* z, int M, int V, const int* tgt,        \
                               R scale, R* losses, R* dz) {                     \
     softmax_xent<R>(z, M, V, tgt, scale, losses, dz);                          \
+  }                                                                            \
+  int orc_sample_token_##SFX(const R* z, int V, R temperature, int top_k,     \
+                             double u) {                                       \
+    return sample_token<R>(z, V, temperature, top_k, u);                       \
   }                                                                            \
   void orc_attention_fwd_##SFX(const R* qkv, R* y, int B, int T, int C,        \
                                int H) {                                        \

@@ -464,3 +464,28 @@ def test_fp32_oracle_tracks_fp64():
         if np.abs(a).max() == 0:
             continue
         assert np.abs(a - b).max() <= 1e-4 * np.abs(a).max(), name
+
+
+def test_sample_token_is_the_inverse_cdf_of_the_tempered_softmax():
+    o = Oracle(Config(1, 1, 8, 11, 11, 4))
+    rng = np.random.default_rng(7)
+    z = rng.standard_normal(9) * 2.0
+    z[3] = z[6] = z.max() + 0.5  # a tie for the maximum
+    # temperature 0: the argmax, the lowest index among equal maxima
+    assert o.sample_token(z) == 3
+    # a uniform grid of draws reproduces the softmax(z / T) masses exactly
+    # (inverse-CDF construction), to within one grid step per token
+    n = 20000
+    for temp, k in ((1.0, 0), (0.7, 0), (2.0, 4)):
+        counts = np.zeros(z.size)
+        for i in range(n):
+            counts[o.sample_token(z, temp, k, (i + 0.5) / n)] += 1
+        keep = np.ones(z.size, bool)
+        if k:
+            keep = z >= np.sort(z)[::-1][k - 1]
+        w = np.where(keep, np.exp((z - z.max()) / temp), 0.0)
+        want = w / w.sum()
+        assert np.all(np.abs(counts / n - want) <= 1.5 / n), (temp, k)
+        assert np.all(counts[~keep] == 0)
+    # a very low temperature concentrates on the (first) maximum
+    assert all(o.sample_token(z, 1e-3, 0, u) in (3, 6) for u in (0.0, 0.3, 0.99))
