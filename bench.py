@@ -371,6 +371,63 @@ def run_ours(args, wl):
     return out if rank == 0 else None
 
 
+def run_generate(args, wl):
+    """Autoregressive generation with the key/value cache: B sequences, a
+    prompt of T/8 tokens, generated to T/4 (both from the workload's T);
+    tokens/s = B * new tokens / device time of one gpt2_generate call."""
+    import torch
+
+    from transformer_lm_pretraining_b200 import gpt2 as g2
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    Tp, Ttot = max(1, wl.T // 8), max(2, wl.T // 4)
+    model = g2.GPT2(wl.L, wl.H, wl.C, wl.V, wl.Vp, wl.Tmax, seed=0, precision="bf16", B=wl.B, T=Tp)
+    model.set_stream(stream)
+    prompt = ZipfStream(wl.V, 1).next_batch(wl.B, Tp)[0]
+    tok = torch.zeros((wl.B, Ttot), dtype=torch.int32, device="cuda")
+    tok[:, :Tp] = torch.from_numpy(prompt).cuda()
+    for _ in range(args.warmup):
+        model.generate(tok, Tp, 0.8, 40, 7)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    n0 = g2.gpt2_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(args.steps):
+        model.generate(tok, Tp, 0.8, 40, 7 + k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    new = Ttot - Tp
+    value = wl.B * new / (ms / 1e3)
+    launches = (g2.gpt2_launch_count() - n0) // args.steps
+    # each decode step streams the bf16 weights once plus the cached keys
+    # and values of the positions so far (prefill excluded from the bytes)
+    peaks = load_peaks()
+    w_bytes = 2.0 * model.P
+    kv_bytes = 2.0 * wl.L * wl.B * 2 * wl.C * sum(range(Tp + 1, Ttot))
+    step_ms = ms / new
+    achieved = (w_bytes * (new - 1) + kv_bytes) / (ms / 1e3) / 1e9
+    model.close()
+    return {"metric": f"generation tokens/s (key/value cache), {wl.name} bf16",
+            "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.B, "prompt": Tp, "total": Ttot,
+                       "temperature": 0.8, "top_k": 40, "mode": "generate",
+                       "l2": "weights (249 MB) stream through HBM every decode step, above L2"},
+            "gpu_launches": int(launches),
+            "roofline": {"kernel": "whole decode step (weights + key/value cache per step)",
+                         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "peak_source": peaks["source"], "traffic": None},
+            "clocks": clk}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -381,15 +438,21 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-T", type=int, default=256)
-    ap.add_argument("--mode", default="train", choices=["train", "eval"],
-                    help="train: the training step; eval: forward-only evaluation (loss)")
+    ap.add_argument("--mode", default="train", choices=["train", "eval", "generate"],
+                    help="train: the training step; eval: forward-only evaluation (loss); "
+                         "generate: autoregressive generation with the key/value cache")
     ap.add_argument("--recompute", type=int, default=0, choices=[0, 1],
                     help="1: recompute GELU in the backward instead of keeping it")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = WORKLOADS[args.workload]
-    out = run_reference(args, wl) if args.impl == "reference" else run_ours(args, wl)
+    if args.impl == "reference":
+        out = run_reference(args, wl)
+    elif args.mode == "generate":
+        out = run_generate(args, wl)
+    else:
+        out = run_ours(args, wl)
     if out is not None:
         print(json.dumps(out), flush=True)
 

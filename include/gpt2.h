@@ -127,6 +127,26 @@ gpt2_status gpt2_forward(gpt2_t* h, const int32_t* tok_dev, const int32_t* tgt_d
 gpt2_status gpt2_evaluate(gpt2_t* h, const int32_t* tok_dev, const int32_t* tgt_dev, int B, int T,
                           float* loss_host);
 
+/* Autoregressive generation with a key/value cache (the sampling loop of
+ * the pages).  tok_dev is a device int32 buffer [B][T_total] whose first
+ * T_prompt columns hold the prompts; the call fills columns T_prompt ..
+ * T_total-1, one token per position: the forward over the prompts (as
+ * gpt2_forward without targets) leaves their keys and values in a cache,
+ * then each new position runs one-position layers against it.  Each token
+ * is drawn from the logits over the first V classes: temperature 0 takes
+ * the argmax (lowest index among equal maxima); otherwise the softmax of
+ * logits / temperature over the top_k largest logits (top_k <= 0: all; ties
+ * at the k-th value kept) is inverted at the uniform draw u = (SplitMix64
+ * output n = position * 65536 + row of `seed`) >> 11, times 2^-53.
+ * step_logits (may be NULL) is device fp32 [T_total - T_prompt][B][V] and
+ * receives the logits each token was drawn from.  The cache and the
+ * one-position buffers are device memory the library allocates and keeps
+ * until gpt2_destroy; the forward record afterwards holds the prompts (no
+ * gpt2_backward).  Asynchronous.  Errors: GPT2_ERR_ARG (T_prompt < 1,
+ * T_total <= T_prompt or > Tmax, head dim above 128), GPT2_ERR_CUDA. */
+gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok_dev, int B, int T_prompt, int T_total,
+                          float temperature, int top_k, uint64_t seed, float* step_logits);
+
 /* Mean loss of the last forward with targets, read back to the host
  * (synchronises the stream). */
 gpt2_status gpt2_read_loss(gpt2_t* h, float* loss_host);

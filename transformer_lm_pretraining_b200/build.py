@@ -25,7 +25,7 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-re
          "-I", CSRC, "-I", os.path.join(ROOT, "include")]
 
 COMMON = ["gpt2.cu", "kernel_abi.cu", "noalloc.cu", "encoder.cu", "layernorm.cu", "misc.cu",
-          "attention.cu"]
+          "attention.cu", "generate.cu"]
 VARIANTS = {
     "libgpt2.so": (COMMON + ["gemm_tc.cu", "attention_tc.cu", "attention_bwd_tc.cu"], []),
     "libgpt2_fp32.so": (COMMON + ["gemm_simt.cu"], ["-DGPT2_FP32_VALIDATE"]),

@@ -46,6 +46,17 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): output n of the generator
+// seeded with s is mix(s + n * 0x9E3779B97F4A7C15).
+__host__ __device__ __forceinline__ uint64_t sm64_mix(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+__host__ __device__ __forceinline__ uint64_t sm64_out(uint64_t seed, uint64_t n) {
+  return sm64_mix(seed + n * 0x9E3779B97F4A7C15ull);
+}
+
 // 8 consecutive activations <-> 8 floats (16 B of bf16 or 32 B of fp32).
 __device__ __forceinline__ void load8(const float* p, float* v) {
   const float4 a = *reinterpret_cast<const float4*>(p);

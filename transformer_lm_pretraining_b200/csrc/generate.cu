@@ -1,0 +1,244 @@
+// Kernels of autoregressive generation with a key/value cache: the
+// embedding of one position per sequence, single-query causal attention over
+// the cached keys and values, and the next-token sampler.
+
+#include <climits>
+
+#include "kernels.h"
+
+namespace gpt2k {
+
+namespace {
+
+constexpr int kSampleThreads = 1024;
+
+// x[b] = wte[tok[b * ld_tok + p]] + wpe[p]; ids outside [0, V) read as 0 and
+// set ERR_TOKEN.
+__global__ void decode_embed_kernel(act_t* __restrict__ x, const int* __restrict__ tok, int ld_tok,
+                                    int p, const act_t* __restrict__ wte,
+                                    const act_t* __restrict__ wpe, int C, int V, int* err) {
+  const int b = blockIdx.x;
+  int t = tok[(size_t)b * ld_tok + p];
+  if (t < 0 || t >= V) {
+    if (threadIdx.x == 0) atomicOr(err, ERR_TOKEN);
+    t = 0;
+  }
+  for (int c = threadIdx.x * 8; c < C; c += blockDim.x * 8) {
+    float a[8], w[8];
+    load8(wte + (size_t)t * C + c, a);
+    load8(wpe + (size_t)p * C + c, w);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] += w[i];
+    store8(x + (size_t)b * C + c, a);
+  }
+}
+
+// One block per (head, sequence): the query q[b, head] against the n cached
+// keys of that sequence: scores in shared memory, softmax in fp32, then the
+// value average (threads split the keys in two halves per output dimension).
+// kv rows: [b][Ttot][2C] = [k | v].
+__global__ void __launch_bounds__(128)
+    decode_attention_kernel(act_t* __restrict__ att, const act_t* __restrict__ q,
+                            const act_t* __restrict__ kv, int Ttot, int n, int C, int H,
+                            float scale) {
+  extern __shared__ float sc[];  // [n] scores, then [128 / hd][hd] partial outputs
+  __shared__ float red[4], qv[256];
+  const int h = blockIdx.x, b = blockIdx.y, hd = C / H;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int d = tid; d < hd; d += blockDim.x) qv[d] = to_f(q[(size_t)b * C + h * hd + d]);
+  __syncthreads();
+  const act_t* kb = kv + (size_t)b * Ttot * 2 * C + (size_t)h * hd;
+  float mx = -INFINITY;
+  for (int k = tid; k < n; k += blockDim.x) {
+    const act_t* kr = kb + (size_t)k * 2 * C;
+    float s = 0.f;
+    for (int d = 0; d < hd; d += 8) {
+      float kk[8];
+      load8(kr + d, kk);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s = fmaf(qv[d + i], kk[i], s);
+    }
+    s *= scale;
+    sc[k] = s;
+    mx = fmaxf(mx, s);
+  }
+  mx = warp_max(mx);
+  if (lane == 0) red[w] = mx;
+  __syncthreads();
+  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  float sum = 0.f;
+  for (int k = tid; k < n; k += blockDim.x) {
+    const float e = __expf(sc[k] - mx);
+    sc[k] = e;
+    sum += e;
+  }
+  sum = warp_sum(sum);
+  if (lane == 0) red[w] = sum;
+  __syncthreads();
+  sum = (red[0] + red[1]) + (red[2] + red[3]);
+  // output dimension d = tid % hd, key half = tid / hd (hd <= 64 uses both halves)
+  float* part = sc + n;
+  const int d = tid % hd, half = tid / hd, halves = blockDim.x / hd;
+  if (half < halves) {
+    float o = 0.f;
+    for (int k = half; k < n; k += halves)
+      o = fmaf(sc[k], to_f(kb[(size_t)k * 2 * C + C + d]), o);
+    part[half * hd + d] = o;
+  }
+  __syncthreads();
+  if (tid < hd) {
+    float o = 0.f;
+    for (int hh = 0; hh < halves; ++hh) o += part[hh * hd + tid];
+    att[(size_t)b * C + h * hd + tid] = from_f<act_t>(o / sum);
+  }
+}
+
+// Order-preserving map of a float to an unsigned integer.
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float block_max_f(float v, float* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  v = warp_max(v);
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int i = 1; i < kSampleThreads / 32; ++i) r = fmaxf(r, red[i]);
+  __syncthreads();
+  return r;
+}
+__device__ __forceinline__ float block_sum_f(float v, float* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  v = warp_sum(v);
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int i = 1; i < kSampleThreads / 32; ++i) r += red[i];
+  __syncthreads();
+  return r;
+}
+__device__ __forceinline__ int block_min_i(int v, int* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  int r = red[0];
+  for (int i = 1; i < kSampleThreads / 32; ++i) r = min(r, red[i]);
+  __syncthreads();
+  return r;
+}
+
+// One block per sequence b: the next token from the row of V logits at
+// logits + b * ld_logits, written to tok[b * ld_tok + p_out].  Temperature
+// 0: the argmax (lowest index among equal maxima).  Otherwise the softmax of
+// z / temperature over the top_k largest logits (threshold found by
+// bisection over order-preserving keys; ties kept), inverted at the uniform
+// u = SplitMix64(seed, p_out * 65536 + b) (top 53 bits): each thread owns a
+// contiguous run of columns, the runs' sums are scanned in a fixed order,
+// and the run where the cumulative mass first exceeds u * total is walked.
+// logits_out (may be null) receives the row as fp32.
+__global__ void __launch_bounds__(kSampleThreads)
+    sample_kernel(int* __restrict__ tok, int ld_tok, int p_out, const act_t* __restrict__ logits,
+                  long ld_logits, int V, float temperature, int top_k, uint64_t seed,
+                  float* __restrict__ logits_out) {
+  __shared__ float redf[kSampleThreads / 32];
+  __shared__ int redi[kSampleThreads / 32];
+  __shared__ float scan[kSampleThreads];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const act_t* z = logits + (size_t)b * ld_logits;
+  if (logits_out)
+    for (int v = tid; v < V; v += kSampleThreads) logits_out[(size_t)b * V + v] = to_f(z[v]);
+  float mx = -INFINITY;
+  for (int v = tid; v < V; v += kSampleThreads) mx = fmaxf(mx, to_f(z[v]));
+  mx = block_max_f(mx, redf);
+  int chosen;
+  if (temperature <= 0.f) {
+    int first = INT_MAX;
+    for (int v = tid; v < V; v += kSampleThreads)
+      if (to_f(z[v]) == mx) first = min(first, v);
+    chosen = block_min_i(first, redi);
+  } else {
+    // keep z >= the k-th largest value: the largest key t with count(key >= t) >= k
+    uint32_t thr = 0;
+    if (top_k > 0 && top_k < V) {
+      uint32_t lo = 0, hi = 0xFFFFFFFFu;  // count(key >= lo) >= k always
+      while (lo < hi) {
+        const uint32_t mid = lo + (uint32_t)(((uint64_t)hi - lo + 1) >> 1);
+        int cnt = 0;
+        for (int v = tid; v < V; v += kSampleThreads) cnt += ord_key(to_f(z[v])) >= mid;
+        const float tot = block_sum_f((float)cnt, redf);
+        if (tot >= (float)top_k) lo = mid;
+        else hi = mid - 1;
+      }
+      thr = lo;
+    }
+    const float inv_t = 1.0f / temperature;
+    const int chunk = (V + kSampleThreads - 1) / kSampleThreads;
+    const int v0 = min(V, tid * chunk), v1 = min(V, v0 + chunk);
+    float s = 0.f;
+    for (int v = v0; v < v1; ++v) {
+      const float zv = to_f(z[v]);
+      if (ord_key(zv) >= thr) s += __expf((zv - mx) * inv_t);
+    }
+    // exclusive scan of the runs' sums in thread order
+    scan[tid] = s;
+    __syncthreads();
+    if (tid == 0) {
+      float acc = 0.f;
+      for (int i = 0; i < kSampleThreads; ++i) {
+        const float x = scan[i];
+        scan[i] = acc;
+        acc += x;
+      }
+      redf[0] = acc;
+    }
+    __syncthreads();
+    const float total = redf[0];
+    const double u = (double)(sm64_out(seed, (uint64_t)p_out * 65536u + (uint64_t)b) >> 11) *
+                     1.1102230246251565e-16;  // 2^-53
+    const float target = (float)u * total;
+    int found = INT_MAX, last = -1;
+    float cum = scan[tid];
+    for (int v = v0; v < v1; ++v) {
+      const float zv = to_f(z[v]);
+      if (ord_key(zv) < thr) continue;
+      cum += __expf((zv - mx) * inv_t);
+      last = v;
+      if (cum > target && found == INT_MAX) found = v;
+    }
+    chosen = block_min_i(found, redi);
+    if (chosen == INT_MAX) chosen = -block_min_i(-last, redi);  // rounding: the last kept token
+  }
+  if (tid == 0) tok[(size_t)b * ld_tok + p_out] = chosen;
+}
+
+}  // namespace
+
+void decode_embed(act_t* x, const int* tok, int ld_tok, int p, const act_t* wte, const act_t* wpe,
+                  int B, int C, int V, int* err, cudaStream_t s) {
+  decode_embed_kernel<<<B, 128, 0, s>>>(x, tok, ld_tok, p, wte, wpe, C, V, err);
+  note_launch();
+}
+
+void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int n, int B, int C,
+                      int H, cudaStream_t s) {
+  const int hd = C / H;  // <= 128 (checked by the caller)
+  const size_t smem = ((size_t)n + 128) * sizeof(float);
+  decode_attention_kernel<<<dim3(H, B), 128, smem, s>>>(att, q, kv, Ttot, n, C, H,
+                                                         1.0f / sqrtf((float)hd));
+  note_launch();
+}
+
+void sample_tokens(int* tok, int ld_tok, int p_out, const act_t* logits, long ld_logits, int B,
+                   int V, float temperature, int top_k, uint64_t seed, float* logits_out,
+                   cudaStream_t s) {
+  sample_kernel<<<B, kSampleThreads, 0, s>>>(tok, ld_tok, p_out, logits, ld_logits, V, temperature,
+                                             top_k, seed, logits_out);
+  note_launch();
+}
+
+}  // namespace gpt2k

@@ -76,6 +76,9 @@ struct gpt2 {
   size_t work_bytes = 0;
   bool own_work = false;
   int recompute = 0;  // 1: GELU outputs are not kept; the backward recomputes them
+  // generation: key/value cache and one-position scratch (library-owned)
+  void* gen = nullptr;
+  size_t gen_bytes = 0;
   // forward record
   int B = 0, T = 0;
   bool have_grad_logits = false;
@@ -288,6 +291,7 @@ void gpt2_destroy(gpt2_t* h) {
   if (!h) return;
   if (h->own_state && h->state) cudaFree(h->state);
   if (h->own_work && h->work) cudaFree(h->work);
+  if (h->gen) cudaFree(h->gen);
   std::vector<cudaEvent_t> evs = h->ev_pool;
   for (const ProfRec& r : h->recs) {
     evs.push_back(r.a);
@@ -486,6 +490,152 @@ gpt2_status gpt2_evaluate(gpt2_t* h, const int32_t* tok, const int32_t* tgt, int
                           float* loss_host) {
   if (!tgt) return fail(h, GPT2_ERR_ARG, "evaluation needs targets");
   return forward_impl(h, tok, tgt, B, T, loss_host, false);
+}
+
+namespace {
+
+// Generation buffers: the key/value cache [L][B][Ttot][2C] and the
+// one-position activations of a decode step.
+struct GenBufs {
+  act_t *cache, *x0, *x1, *hb, *q, *att, *xm, *u, *g, *logits;
+  float *mean, *rstd;
+  int* prompt;
+};
+
+size_t carve_gen(const Layout& y, int B, int Tp, int Ttot, void* base, GenBufs* out) {
+  const size_t C = y.C;
+  Carver c(base);
+  GenBufs g{};
+  g.cache = c.take<act_t>((size_t)y.L * B * Ttot * 2 * C);
+  g.x0 = c.take<act_t>(B * C);
+  g.x1 = c.take<act_t>(B * C);
+  g.hb = c.take<act_t>(B * C);
+  g.q = c.take<act_t>(B * C);
+  g.att = c.take<act_t>(B * C);
+  g.xm = c.take<act_t>(B * C);
+  g.u = c.take<act_t>(B * 4 * C);
+  g.g = c.take<act_t>(B * 4 * C);
+  g.logits = c.take<act_t>((size_t)B * y.Vp);
+  g.mean = c.take<float>(B);
+  g.rstd = c.take<float>(B);
+  g.prompt = c.take<int>((size_t)B * Tp);
+  if (out) *out = g;
+  return c.used;
+}
+
+}  // namespace
+
+gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, float temperature,
+                          int top_k, uint64_t seed, float* step_logits) {
+  if (!h || !tok || B < 1 || Tp < 1 || Ttot <= Tp) return fail(h, GPT2_ERR_ARG, "bad generate arguments");
+  const Layout& y = h->lay;
+  if (Ttot > y.Tmax) return fail(h, GPT2_ERR_ARG, "T_total > Tmax");
+  if (y.C / y.H > 128) return fail(h, GPT2_ERR_ARG, "generation supports head dims up to 128");
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  const size_t need = carve_gen(y, B, Tp, Ttot, nullptr, nullptr);
+  if (h->gen_bytes < need) {
+    if (h->gen) cudaFree(h->gen);
+    h->gen = nullptr;
+    h->gen_bytes = 0;
+    GPT2_CUDA(h, cudaMalloc(&h->gen, need));
+    h->gen_bytes = need;
+  }
+  GenBufs gb;
+  carve_gen(y, B, Tp, Ttot, h->gen, &gb);
+  cudaStream_t s = h->stream;
+  const int C = y.C, L = y.L, H = y.H;
+  const float* P = h->params;
+  const act_t* W = h->pact;
+  // prefill: the training forward over the prompt (contiguous copy), then
+  // its keys and values into the cache
+  GPT2_CUDA(h, cudaMemcpy2DAsync(gb.prompt, (size_t)Tp * sizeof(int), tok, (size_t)Ttot * sizeof(int),
+                                 (size_t)Tp * sizeof(int), B, cudaMemcpyDeviceToDevice, s));
+  st = forward_impl(h, gb.prompt, nullptr, B, Tp, nullptr, true);
+  if (st) return st;
+  const Acts& a = h->a;
+  const size_t MCp = (size_t)B * Tp * C;
+  for (int l = 0; l < L; ++l)
+    for (int b = 0; b < B; ++b)
+      GPT2_CUDA(h, cudaMemcpy2DAsync(gb.cache + ((size_t)l * B + b) * Ttot * 2 * C, 2 * C * sizeof(act_t),
+                                     a.qkv + (size_t)l * 3 * MCp + (size_t)b * Tp * 3 * C + C,
+                                     3 * C * sizeof(act_t), 2 * C * sizeof(act_t), Tp,
+                                     cudaMemcpyDeviceToDevice, s));
+  const size_t Vs = (size_t)y.V;
+  sample_tokens(tok, Ttot, Tp, a.logits + (size_t)(Tp - 1) * y.Vp, (long)Tp * y.Vp, B, y.V,
+                temperature, top_k, seed, step_logits, s);
+  // decode: position p takes token p and yields token p + 1
+  for (int p = Tp; p < Ttot - 1; ++p) {
+    decode_embed(gb.x0, tok, Ttot, p, W + y.off[T_WTE], W + y.off[T_WPE], B, C, y.V, h->err, s);
+    act_t* x = gb.x0;
+    act_t* xn = gb.x1;
+    for (int l = 0; l < L; ++l) {
+      act_t* kv = gb.cache + (size_t)l * B * Ttot * 2 * C;
+      layernorm_fwd(gb.hb, gb.mean, gb.rstd, x, P + y.off[T_LN1G] + (size_t)l * C,
+                    P + y.off[T_LN1B] + (size_t)l * C, B, C, s);
+      {  // q = h W_q^T + b_q
+        GemmArgs ga = gemm_args(B, C, C);
+        ga.A = gb.hb; ga.lda = C;
+        ga.B = W + y.off[T_WQKV] + (size_t)l * 3 * C * C; ga.ldb = C;
+        ga.epi = EPI_BIAS; ga.bias = P + y.off[T_BQKV] + (size_t)l * 3 * C;
+        ga.out = gb.q; ga.ldo = C;
+        GPT2_TRY(run_gemm(h, ga));
+      }
+      {  // [k | v] of position p straight into the cache
+        GemmArgs ga = gemm_args(B, 2 * C, C);
+        ga.A = gb.hb; ga.lda = C;
+        ga.B = W + y.off[T_WQKV] + (size_t)l * 3 * C * C + (size_t)C * C; ga.ldb = C;
+        ga.epi = EPI_BIAS; ga.bias = P + y.off[T_BQKV] + (size_t)l * 3 * C + C;
+        ga.out = kv + (size_t)p * 2 * C; ga.ldo = (long)Ttot * 2 * C;
+        GPT2_TRY(run_gemm(h, ga));
+      }
+      decode_attention(gb.att, gb.q, kv, Ttot, p + 1, B, C, H, s);
+      {  // xm = x + att W_o^T + b_o
+        GemmArgs ga = gemm_args(B, C, C);
+        ga.A = gb.att; ga.lda = C;
+        ga.B = W + y.off[T_WO] + (size_t)l * C * C; ga.ldb = C;
+        ga.epi = EPI_BIAS_RESID; ga.bias = P + y.off[T_BO] + (size_t)l * C;
+        ga.resid = x; ga.ldr = C;
+        ga.out = gb.xm; ga.ldo = C;
+        GPT2_TRY(run_gemm(h, ga));
+      }
+      layernorm_fwd(gb.hb, gb.mean, gb.rstd, gb.xm, P + y.off[T_LN2G] + (size_t)l * C,
+                    P + y.off[T_LN2B] + (size_t)l * C, B, C, s);
+      {  // u = h W_fc^T + b_fc; g = gelu(u)
+        GemmArgs ga = gemm_args(B, 4 * C, C);
+        ga.A = gb.hb; ga.lda = C;
+        ga.B = W + y.off[T_WFC] + (size_t)l * 4 * C * C; ga.ldb = C;
+        ga.epi = EPI_BIAS_GELU; ga.bias = P + y.off[T_BFC] + (size_t)l * 4 * C;
+        ga.aux = gb.u; ga.ldaux = 4 * C;
+        ga.out = gb.g; ga.ldo = 4 * C;
+        GPT2_TRY(run_gemm(h, ga));
+      }
+      {  // x_next = xm + g W_p^T + b_p
+        GemmArgs ga = gemm_args(B, C, 4 * C);
+        ga.A = gb.g; ga.lda = 4 * C;
+        ga.B = W + y.off[T_WP] + (size_t)l * 4 * C * C; ga.ldb = 4 * C;
+        ga.epi = EPI_BIAS_RESID; ga.bias = P + y.off[T_BP] + (size_t)l * C;
+        ga.resid = gb.xm; ga.ldr = C;
+        ga.out = xn; ga.ldo = C;
+        GPT2_TRY(run_gemm(h, ga));
+      }
+      std::swap(x, xn);
+    }
+    layernorm_fwd(gb.hb, gb.mean, gb.rstd, x, P + y.off[T_LNFG], P + y.off[T_LNFB], B, C, s);
+    {  // logits of position p
+      GemmArgs ga = gemm_args(B, y.Vp, C);
+      ga.A = gb.hb; ga.lda = C;
+      ga.B = W + y.off[T_WTE]; ga.ldb = C;
+      ga.epi = EPI_STORE;
+      ga.out = gb.logits; ga.ldo = y.Vp;
+      GPT2_TRY(run_gemm(h, ga));
+    }
+    sample_tokens(tok, Ttot, p + 1, gb.logits, y.Vp, B, y.V, temperature, top_k, seed,
+                  step_logits ? step_logits + (size_t)(p + 1 - Tp) * B * Vs : nullptr, s);
+  }
+  h->have_logits = h->have_grad_logits = false;  // the forward record now holds the prompt only
+  GPT2_CUDA(h, cudaGetLastError());
+  return GPT2_OK;
 }
 
 gpt2_status gpt2_read_loss(gpt2_t* h, float* loss_host) {

@@ -119,6 +119,21 @@ void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int 
 // out[0] = mean of losses[0..M) (fixed-order reduction)
 void mean_loss(float* out, const float* losses, int M, cudaStream_t s);
 
+// ------------------------------------------------------------ generation --
+// x[b] = wte[tok[b * ld_tok + p]] + wpe[p] for b < B (bad ids: ERR_TOKEN, read as 0)
+void decode_embed(act_t* x, const int* tok, int ld_tok, int p, const act_t* wte, const act_t* wpe,
+                  int B, int C, int V, int* err, cudaStream_t s);
+// att[b] = causal attention of the single query q[b] over the first n
+// cached positions kv[b][0..n) ([b][Ttot][2C] rows of [k | v]); C / H <= 128
+void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int n, int B, int C,
+                      int H, cudaStream_t s);
+// tok[b * ld_tok + p_out] = the next token drawn from the V logits of row
+// b (greedy at temperature 0; else top-k tempered softmax at the SplitMix64
+// uniform of (seed, p_out * 65536 + b)); logits_out (may be null): [B][V] fp32
+void sample_tokens(int* tok, int ld_tok, int p_out, const act_t* logits, long ld_logits, int B,
+                   int V, float temperature, int top_k, uint64_t seed, float* logits_out,
+                   cudaStream_t s);
+
 // g = GELU_tanh(u) elementwise (n elements, activation dtype); the same
 // function the fc GEMM's epilogue applies to the stored u.
 void gelu_fwd(act_t* g, const act_t* u, size_t n, cudaStream_t s);

@@ -380,14 +380,6 @@ __global__ void mean_loss_kernel(float* out, const float* __restrict__ losses, i
 // generator seeded with output t+1 of the master generator seeded with
 // `seed`; element i takes outputs 2i+1, 2i+2 as the two uniforms of one
 // Box-Muller normal (cosine branch), evaluated in double, rounded once.
-__device__ __forceinline__ uint64_t sm64_mix(uint64_t z) {
-  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-  return z ^ (z >> 31);
-}
-__device__ __forceinline__ uint64_t sm64_out(uint64_t seed, uint64_t n) {
-  return sm64_mix(seed + n * 0x9E3779B97F4A7C15ull);
-}
 
 struct InitSeg {
   size_t off, count;  // elements [off, off + count) get normals

@@ -45,6 +45,7 @@ SIGNATURES = {
     "gpt2_forward": (_i, [_vp, _vp, _vp, _i, _i, _fp]),
     "gpt2_evaluate": (_i, [_vp, _vp, _vp, _i, _i, _fp]),
     "gpt2_set_recompute": (_i, [_vp, _i]),
+    "gpt2_generate": (_i, [_vp, _vp, _i, _i, _i, _f, _i, _u64, _fp]),
     "gpt2_zero_grad": (_i, [_vp]),
     "gpt2_read_loss": (_i, [_vp, _fp]),
     "gpt2_backward": (_i, [_vp, _f]),
@@ -205,6 +206,15 @@ class GPT2:
 
         t = torch.as_tensor(_View(), device="cuda")
         return t.view(torch.bfloat16) if bf16 else t
+
+    def generate(self, tok, T_prompt, temperature=0.0, top_k=0, seed=0, step_logits=None):
+        """Fill tok[:, T_prompt:] (a device int32 tensor [B, T_total]) by
+        autoregressive generation with a key/value cache."""
+        B, T_total = tok.shape
+        self.reserve(B, T_prompt)
+        sl = None if step_logits is None else ctypes.cast(ctypes.c_void_p(step_logits.data_ptr()), _fp)
+        self._check(self.lib.gpt2_generate(self.h, _dptr(tok), B, T_prompt, T_total, temperature,
+                                           top_k, seed, sl))
 
     def zero_grad(self):
         self._check(self.lib.gpt2_zero_grad(self.h))
