@@ -6,23 +6,28 @@
 //   dV = P^T dO,  dK = dS^T Q / sqrt(d),  dQ = dS K / sqrt(d)
 //
 // Two persistent kernels, one CTA per SM walking a static snake order over
-// work items (heaviest first), 10 warps each (TMA, MMA, 8 compute warps =
-// two threads per 128-row tile row, each owning 64 of the 128 columns):
-//   dK/dV: item = (batch, head, key tile j); streams the query tiles i >= j.
-//          The tensor core computes S^T = K Q^T and dP^T = V dO^T into
-//          TMEM; the compute warps turn them into P^T and dS^T (bf16,
-//          swizzled shared-memory tiles); the tensor core then accumulates
-//          dV += P^T dO and dK += dS^T Q in TMEM (dO and Q read MN-major
-//          straight from their tiles).
+// work items (heaviest first), 10 warps each (TMA, MMA, 8 compute warps,
+// two threads per tile row):
+//   dK/dV: item = (batch, head, key tile j); streams the query tiles i >= j
+//          in 64-query halves (sub-tiles).  The tensor core computes
+//          S^T = K Q^T and dP^T = V dO^T of a sub-tile into one of two TMEM
+//          score buffers; the compute warps turn them into P^T and dS^T
+//          (bf16, swizzled shared-memory tiles, also double-buffered); the
+//          tensor core then accumulates dV += P^T dO and dK += dS^T Q in
+//          TMEM (dO and Q read MN-major straight from their tiles).  K and V
+//          are double-buffered across items.
 //   dQ:    item = (batch, head, query tile i); streams the key tiles j <= i:
 //          S = Q K^T and dP = dO V^T into TMEM, dS into shared memory,
 //          dQ += dS K in TMEM (K read MN-major).
 // The compute warps hand the score buffers back to the tensor core as soon
-// as they have read them, so the next tile's scores are computed while the
-// current tile is finished; the gradient accumulators are double-buffered in
-// TMEM, so an item's result is written while the next item runs, and the
-// next item's operands load as soon as the current item's last score
-// product is issued.  Every wait is bounded (error word ERR_TIMEOUT).
+// as they have read them, so the next scores are computed while the current
+// ones are finished; the gradient accumulators are double-buffered in TMEM,
+// so an item's result is written while the next item runs.  Compute warps
+// wait per warp (no block-wide barrier in the loop), and the causal mask is
+// applied only on the diagonal tile and the one holding the end of the
+// sequence.  Every wait is bounded (error word ERR_TIMEOUT).
+
+#include <type_traits>
 
 #include "attention_tc.cuh"
 
@@ -42,7 +47,6 @@ constexpr uint32_t kAccCol = 2 * kTile;  // accumulators after the two score buf
 constexpr int kAux = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ bool cbar_and(bool p) { return named_bar_and<1, kCT>(p); }
 __device__ __forceinline__ bool warp_and(bool p) { return __all_sync(0xffffffffu, p); }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot) {
@@ -71,12 +75,20 @@ __device__ __forceinline__ int snake_item(int k, int count) {
 }
 
 // ------------------------------------------------------------------ dK/dV --
+// The query tiles are processed in 64-query halves ("sub-tiles"), so that the
+// score products of two sub-tiles fit in TMEM next to the two accumulator
+// pairs: while the compute warps turn one sub-tile's S^T and dP^T into P^T
+// and dS^T, the tensor core already holds (or is computing) the next
+// sub-tile's scores and runs the previous sub-tile's dV and dK products.
+// TMEM columns: [0,128) and [128,256) score buffers (S^T 64 | dP^T 64),
+// [256,512) two accumulator pairs (dV 64 | dK 64).
 constexpr int kQStages = 2;
+constexpr int kSub = 64;  // queries per sub-tile
 constexpr size_t dkdv_smem_bytes() {
-  // K, V, [Q, dO] x stages, P^T and dS^T tiles (two boxes each), per-column
-  // L and D of two query tiles, aux
-  return 1024 + 2 * (size_t)kBox + 2 * (size_t)kQStages * kBox + 4 * (size_t)kBox +
-         4 * kTile * sizeof(float) + kAux;
+  // [K, V] x 2 items, [Q, dO] x stages, P^T and dS^T x 2 sub-tiles (one box
+  // each), each compute warp's per-column L and D of two sub-tiles, aux
+  return 1024 + 4 * (size_t)kBox + 2 * (size_t)kQStages * kBox + 4 * (size_t)kBox +
+         (kCT / 32) * 2 * 64 * sizeof(float) + kAux;
 }
 
 __global__ void __launch_bounds__(kThreadsBwd, 1)
@@ -87,26 +99,25 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sK = smem;
-  uint8_t* sV = sK + kBox;
-  uint8_t* sQ = sV + kBox;                // [kQStages]
+  uint8_t* sKV = smem;                    // [2 items][K box, V box]
+  uint8_t* sQ = sKV + 4 * kBox;           // [kQStages]
   uint8_t* sDO = sQ + kQStages * kBox;    // [kQStages]
-  uint8_t* sPT = sDO + kQStages * kBox;   // 2 boxes (query columns 0-63, 64-127)
-  uint8_t* sDST = sPT + 2 * kBox;         // 2 boxes
-  float* col_lse = reinterpret_cast<float*>(sDST + 2 * kBox);  // [2 tiles][L 128, D 128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(col_lse + 4 * kTile);
-  const uint32_t kv_full = smem_u32(bars + 0);
-  const uint32_t kv_empty = smem_u32(bars + 1);
-  const uint32_t qd_full0 = smem_u32(bars + 2);   // [2]
-  const uint32_t qd_empty0 = smem_u32(bars + 4);  // [2]
-  const uint32_t sd_full = smem_u32(bars + 6);
-  const uint32_t sd_empty = smem_u32(bars + 7);
-  const uint32_t pd_full = smem_u32(bars + 8);
-  const uint32_t pd_empty = smem_u32(bars + 9);
-  const uint32_t acc_full0 = smem_u32(bars + 10);   // [2]
-  const uint32_t acc_empty0 = smem_u32(bars + 12);  // [2]
-  const uint32_t drain = smem_u32(bars + 14);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint8_t* sPT = sDO + kQStages * kBox;   // [2 sub-tiles]: 128 keys x 64 queries
+  uint8_t* sDST = sPT + 2 * kBox;         // [2 sub-tiles]
+  float* col_lse = reinterpret_cast<float*>(sDST + 2 * kBox);  // [warp][2][L 32, D 32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(col_lse + (kCT / 32) * 2 * 64);
+  const uint32_t kv_full0 = smem_u32(bars + 0);     // [2]
+  const uint32_t kv_empty0 = smem_u32(bars + 2);    // [2]
+  const uint32_t qd_full0 = smem_u32(bars + 4);     // [2]
+  const uint32_t qd_empty0 = smem_u32(bars + 6);    // [2]
+  const uint32_t sd_full0 = smem_u32(bars + 8);     // [2]
+  const uint32_t sd_empty0 = smem_u32(bars + 10);   // [2]
+  const uint32_t pd_full0 = smem_u32(bars + 12);    // [2]
+  const uint32_t pd_empty0 = smem_u32(bars + 14);   // [2]
+  const uint32_t acc_full0 = smem_u32(bars + 16);   // [2]
+  const uint32_t acc_empty0 = smem_u32(bars + 18);  // [2]
+  const uint32_t drain = smem_u32(bars + 20);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int nq = (T + kTile - 1) / kTile;
@@ -114,17 +125,15 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
-    mbar_init(kv_empty, 1);
-    for (int s = 0; s < kQStages; ++s) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(kv_full0 + 8 * s, 1);
+      mbar_init(kv_empty0 + 8 * s, 1);
       mbar_init(qd_full0 + 8 * s, 1);
       mbar_init(qd_empty0 + 8 * s, 1);
-    }
-    mbar_init(sd_full, 1);
-    mbar_init(sd_empty, kCT);
-    mbar_init(pd_full, kCT);
-    mbar_init(pd_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+      mbar_init(sd_full0 + 8 * s, 1);
+      mbar_init(sd_empty0 + 8 * s, kCT);
+      mbar_init(pd_full0 + 8 * s, kCT);
+      mbar_init(pd_empty0 + 8 * s, 1);
       mbar_init(acc_full0 + 8 * s, 1);
       mbar_init(acc_empty0 + 8 * s, kCT);
     }
@@ -144,17 +153,22 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmDO)) : "memory");
       uint32_t n_item = 0, g = 0;  // items started, query tiles loaded
-      uint32_t issued = 0, last_par = 0;
+      uint32_t kv_issued = 0, kv_par = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int k = 0; ok; ++k, ++n_item) {
         const int w = snake_item(k, items);
         if (w < 0) break;
         const int j = w / BH, bh = w % BH, b = bh / H, h = bh % H;
         const int n = nq - j;  // query tiles i = j .. nq-1
-        if (!mbar_wait(kv_empty, (n_item & 1u) ^ 1u, abort_flag, err)) break;
-        mbar_expect_tx(kv_full, 2 * kBox);
-        tma_load_3d(smem_u32(sK), &tmQKV, kv_full, C + h * kHD, j * kTile, b);
-        tma_load_3d(smem_u32(sV), &tmQKV, kv_full, 2 * C + h * kHD, j * kTile, b);
+        const int ks = n_item & 1;
+        const uint32_t kpar = (n_item >> 1) & 1u;
+        if (!mbar_wait(kv_empty0 + 8 * ks, kpar ^ 1u, abort_flag, err)) break;
+        const uint32_t kb = kv_full0 + 8 * ks;
+        mbar_expect_tx(kb, 2 * kBox);
+        tma_load_3d(smem_u32(sKV + ks * 2 * kBox), &tmQKV, kb, C + h * kHD, j * kTile, b);
+        tma_load_3d(smem_u32(sKV + ks * 2 * kBox + kBox), &tmQKV, kb, 2 * C + h * kHD, j * kTile, b);
+        kv_issued |= 1u << ks;
+        kv_par = (kv_par & ~(1u << ks)) | (kpar << ks);
         for (int t = 0; t < n; ++t, ++g) {
           const int st = g & 1;
           const uint32_t par = (g >> 1) & 1u;
@@ -172,74 +186,93 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       }
       // every copy issued lands before the shared memory is released
       const uint64_t t0 = global_ns();
-      if (n_item) drain_wait(kv_full, (n_item - 1) & 1u, t0);
-      for (int s = 0; s < kQStages; ++s)
+      for (int s = 0; s < 2; ++s) {
+        if (kv_issued & (1u << s)) drain_wait(kv_full0 + 8 * s, (kv_par >> s) & 1u, t0);
         if (issued & (1u << s)) drain_wait(qd_full0 + 8 * s, (last_par >> s) & 1u, t0);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA --
-      constexpr uint32_t idS = attn::idesc(kTile, false);
+      constexpr uint32_t idS = attn::idesc(kSub, false);
       constexpr uint32_t idA = attn::idesc(kHD, true);
-      const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
-      uint32_t n_item = 0, g = 0;
-      bool ok = true;
-      // S^T and dP^T of the query tile with global index gt
-      auto issue_sd = [&](uint32_t gt) -> bool {
-        const int st = gt & 1;
-        if (!mbar_wait(qd_full0 + 8 * st, (gt >> 1) & 1u, abort_flag, err)) return false;
-        if (!mbar_wait(sd_empty, (gt & 1u) ^ 1u, abort_flag, err)) return false;
+      // S^T = K Q_s^T and dP^T = V dO_s^T of sub-tile s (half hs of the
+      // query tile in stage st) into score buffer s % 2
+      auto issue_sd = [&](uint32_t s, int st, uint32_t tpar, int hs, int ks) -> bool {
+        const uint32_t sb = s & 1u;
+        if (!mbar_wait(qd_full0 + 8 * st, tpar, abort_flag, err)) return false;
+        if (!mbar_wait(sd_empty0 + 8 * sb, ((s >> 1) & 1u) ^ 1u, abort_flag, err)) return false;
         tc_fence_after();
-        const uint32_t q_base = smem_u32(sQ + st * kBox), do_base = smem_u32(sDO + st * kBox);
+        const uint32_t k_base = smem_u32(sKV + ks * 2 * kBox), v_base = k_base + kBox;
+        const uint32_t q_base = smem_u32(sQ + st * kBox) + hs * (kSub * 128);
+        const uint32_t do_base = smem_u32(sDO + st * kBox) + hs * (kSub * 128);
+        const uint32_t d = tmem + sb * 2 * kSub;
 #pragma unroll
-        for (int k = 0; k < kHD / 16; ++k)  // S^T = K Q^T
-          tc_mma(tmem, desc_kmajor(k_base, k), desc_kmajor(q_base, k), idS, k > 0 ? 1u : 0u);
+        for (int k = 0; k < kHD / 16; ++k)
+          tc_mma(d, desc_kmajor(k_base, k), desc_kmajor(q_base, k), idS, k > 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < kHD / 16; ++k)  // dP^T = V dO^T
-          tc_mma(tmem + kTile, desc_kmajor(v_base, k), desc_kmajor(do_base, k), idS, k > 0 ? 1u : 0u);
-        tc_commit(sd_full);
+        for (int k = 0; k < kHD / 16; ++k)
+          tc_mma(d + kSub, desc_kmajor(v_base, k), desc_kmajor(do_base, k), idS, k > 0 ? 1u : 0u);
+        tc_commit(sd_full0 + 8 * sb);
         return true;
       };
-      // dV += P^T dO, dK += dS^T Q into the accumulator pair at column acc
-      auto issue_acc = [&](uint32_t gt, uint32_t acc, bool first) -> bool {
-        const int st = gt & 1;
-        if (!mbar_wait(pd_full, gt & 1u, abort_flag, err)) return false;
+      // dV += P^T dO_s, dK += dS^T Q_s of a sub-tile whose P^T and dS^T are
+      // (being) written; releases the query tile after its second half and
+      // hands the accumulators over after the item's last sub-tile
+      struct Pend {
+        uint32_t s, acc, ab;
+        int st, hs;
+        bool first, last;
+      };
+      auto issue_acc = [&](const Pend& p) -> bool {
+        const uint32_t sb = p.s & 1u;
+        if (!mbar_wait(pd_full0 + 8 * sb, (p.s >> 1) & 1u, abort_flag, err)) return false;
         tc_fence_after();
-        const uint32_t q_base = smem_u32(sQ + st * kBox), do_base = smem_u32(sDO + st * kBox);
-        const uint32_t pt = smem_u32(sPT), dst = smem_u32(sDST);
+        const uint32_t q_base = smem_u32(sQ + p.st * kBox), do_base = smem_u32(sDO + p.st * kBox);
+        const uint32_t pt = smem_u32(sPT + sb * kBox), dst = smem_u32(sDST + sb * kBox);
 #pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)
-          tc_mma(tmem + acc, desc_kmajor(pt + (uint32_t)((k >> 2) * kBox), k & 3),
-                 desc_mnmajor(do_base, k), idA, (!first || k > 0) ? 1u : 0u);
+        for (int k = 0; k < kSub / 16; ++k)
+          tc_mma(tmem + p.acc, desc_kmajor(pt, k), desc_mnmajor(do_base, 4 * p.hs + k), idA,
+                 (!p.first || k > 0) ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)
-          tc_mma(tmem + acc + kHD, desc_kmajor(dst + (uint32_t)((k >> 2) * kBox), k & 3),
-                 desc_mnmajor(q_base, k), idA, (!first || k > 0) ? 1u : 0u);
-        tc_commit(pd_empty);
-        tc_commit(qd_empty0 + 8 * st);
+        for (int k = 0; k < kSub / 16; ++k)
+          tc_mma(tmem + p.acc + kHD, desc_kmajor(dst, k), desc_mnmajor(q_base, 4 * p.hs + k), idA,
+                 (!p.first || k > 0) ? 1u : 0u);
+        tc_commit(pd_empty0 + 8 * sb);
+        if (p.hs == 1) tc_commit(qd_empty0 + 8 * p.st);
+        if (p.last) tc_commit(acc_full0 + 8 * p.ab);
         return true;
       };
+      // One flat sequence over every sub-tile of every item: the scores of
+      // sub-tile s are issued before the products of sub-tile s - 1.
+      uint32_t n_item = 0, gs = 0, gt = 0;
+      Pend pend{};
+      bool have = false, ok = true;
       for (int k = 0; ok; ++k, ++n_item) {
         const int w = snake_item(k, items);
         if (w < 0) break;
         const int n = nq - w / BH;
+        const int ks = n_item & 1;
         const uint32_t ab = n_item & 1u, acc = kAccCol + ab * 2 * kHD;
-        ok = mbar_wait(kv_full, n_item & 1u, abort_flag, err);
+        ok = mbar_wait(kv_full0 + 8 * ks, (n_item >> 1) & 1u, abort_flag, err);
         if (ok) ok = mbar_wait(acc_empty0 + 8 * ab, ((n_item >> 1) & 1u) ^ 1u, abort_flag, err);
         if (!ok) break;
         tc_fence_after();
-        ok = issue_sd(g);
-        if (ok && n == 1) tc_commit(kv_empty);  // K and V are no longer read
-        for (int t = 1; t <= n && ok; ++t) {
-          if (t < n) {
-            ok = issue_sd(g + t);
-            if (ok && t == n - 1) tc_commit(kv_empty);
+        for (int t = 0; t < n && ok; ++t, ++gt) {
+          const int st = gt & 1;
+          const uint32_t tpar = (gt >> 1) & 1u;
+          for (int hs = 0; hs < 2; ++hs, ++gs) {
+            ok = issue_sd(gs, st, tpar, hs, ks);
+            if (!ok) break;
+            if (t == n - 1 && hs == 1) tc_commit(kv_empty0 + 8 * ks);  // K, V no longer read
+            if (have) ok = issue_acc(pend);
+            if (!ok) break;
+            pend = Pend{gs, acc, ab, st, hs, t == 0 && hs == 0, t == n - 1 && hs == 1};
+            have = true;
           }
-          if (ok) ok = issue_acc(g + t - 1, acc, t == 1);
         }
-        if (ok) tc_commit(acc_full0 + 8 * ab);
-        g += n;
       }
+      if (ok && have) ok = issue_acc(pend);
       if (!ok) {  // let issued MMAs finish before TMEM is released
         tc_commit(drain);
         drain_wait(drain, 0, global_ns());
@@ -247,13 +280,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     }
   } else {
     // -------------------------------------------------------- compute --
+    // thread = key row r, owning 32 of a sub-tile's 64 query columns.  Every
+    // wait is per warp (warps drift apart and overlap their latencies); each
+    // warp stages the L and D of its own 32 columns.
     const int qw = warp & 3, half = (warp - 2) >> 2;
     const int r = qw * 32 + lane;
-    const int ct = threadIdx.x - 64;  // 0 .. 255
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    const uint32_t pt_row = smem_u32(sPT + half * kBox) + (uint32_t)(r * 128);
-    const uint32_t dst_row = smem_u32(sDST + half * kBox) + (uint32_t)(r * 128);
-    uint32_t n_item = 0, g = 0;
+    float* wcl = col_lse + (warp - 2) * 2 * 64;  // [2 sub-tiles][L 32 | D 32]
+    uint32_t n_item = 0, gs = 0;
     bool ok = true;
     for (int k = 0; ok; ++k, ++n_item) {
       const int w = snake_item(k, items);
@@ -264,79 +298,80 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const float* lse_bh = lse + (size_t)bh * T;
       const float* d_bh = dsum + (size_t)bh * T;
       for (int t = 0; t < n && ok; ++t) {
-        const uint32_t gt = g + t;
-        const int qc0 = (j + t) * kTile + 64 * half;  // first query column of this half
-        // this tile's per-column L (log2 units) and D into shared memory,
-        // loaded while the tensor core computes S^T and dP^T
-        float* cl = col_lse + (gt & 1) * 2 * kTile;
-        {
-          const int q = (j + t) * kTile + (ct & (kTile - 1));
-          cl[ct] = q < T ? (ct < kTile ? lse_bh[q] * kLog2e : d_bh[q]) : 0.f;  // [0,128): L, [128,256): D
-        }
-        ok = cbar_and(mbar_wait(sd_full, gt & 1u, abort_flag, err));
-        if (!ok) break;
-        tc_fence_after();
-        // 16 query columns per chunk; the next chunk's TMEM loads are in
-        // flight while the current chunk is computed
-        uint32_t sa[16], pa[16], sb[16], pb[16];
-        auto ld_chunk = [&](int ch, uint32_t* s_, uint32_t* p_) {
-          const uint32_t col = (uint32_t)(64 * half + 16 * ch);
-          attn::tc_ld16(lane_base + col, s_);
-          attn::tc_ld16(lane_base + kTile + col, p_);
-        };
-        auto do_chunk = [&](int ch, const uint32_t* s_, const uint32_t* p_) -> bool {
-          const int col = 64 * half + 16 * ch;
-          float pv[16], dv[16];
-#pragma unroll
-          for (int c = 0; c < 16; c += 4) {
-            const float4 a = *reinterpret_cast<const float4*>(cl + col + c);
-            const float4 d = *reinterpret_cast<const float4*>(cl + kTile + col + c);
-            pv[c] = a.x; pv[c + 1] = a.y; pv[c + 2] = a.z; pv[c + 3] = a.w;
-            dv[c] = d.x; dv[c + 1] = d.y; dv[c + 2] = d.z; dv[c + 3] = d.w;
+        for (int hs = 0; hs < 2; ++hs, ++gs) {
+          const uint32_t sb = gs & 1u;
+          const int cq = kSub * hs + 32 * half;  // first column of this thread in the tile
+          const int qc0 = (j + t) * kTile + cq;  // its query index
+          // L (log2 units) and D of the warp's 32 columns, loaded while the
+          // tensor core computes the scores
+          float* cl = wcl + sb * 64;
+          {
+            const int q = qc0 + lane;
+            cl[lane] = q < T ? lse_bh[q] * kLog2e : 0.f;
+            cl[32 + lane] = q < T ? d_bh[q] : 0.f;
           }
-          const int lim = kj - qc0 - 16 * ch;  // columns c < lim are queries before the key
-          const int tcut = T - qc0 - 16 * ch;  // columns c >= tcut are past the sequence
+          __syncwarp();
+          // causal mask on the diagonal tile, padding past T on the last one
+          const bool masked = t == 0 || qc0 - cq + kSub * (hs + 1) > T;
+          ok = warp_and(mbar_wait(sd_full0 + 8 * sb, (gs >> 1) & 1u, abort_flag, err));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t s_col = lane_base + sb * 2 * kSub + 32 * half;
+          const uint32_t pt_row = smem_u32(sPT + sb * kBox) + (uint32_t)(r * 128);
+          const uint32_t dst_row = smem_u32(sDST + sb * kBox) + (uint32_t)(r * 128);
+          uint32_t sa[16], pa[16], sb16[16], pb[16];
+          auto ld_chunk = [&](int ch, uint32_t* s_, uint32_t* p_) {
+            attn::tc_ld16(s_col + 16 * ch, s_);
+            attn::tc_ld16(s_col + kSub + 16 * ch, p_);
+          };
+          auto do_chunk = [&](int ch, const uint32_t* s_, const uint32_t* p_, auto mask) -> bool {
+            float pv[16], dv[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float p = fast_exp2(fmaf(__uint_as_float(s_[c]), sl2, -pv[c]));
-            if (c < lim || c >= tcut) p = 0.f;  // causal (only bites when i == j) and padding
-            pv[c] = p;
-            dv[c] = p * (__uint_as_float(p_[c]) - dv[c]);
-          }
-          // the previous tile's products have read P^T and dS^T
-          if (ch == 0 && !cbar_and(mbar_wait(pd_empty, (gt & 1u) ^ 1u, abort_flag, err))) return false;
+            for (int c = 0; c < 16; c += 4) {
+              const float4 a = *reinterpret_cast<const float4*>(cl + 16 * ch + c);
+              const float4 d = *reinterpret_cast<const float4*>(cl + 32 + 16 * ch + c);
+              pv[c] = a.x; pv[c + 1] = a.y; pv[c + 2] = a.z; pv[c + 3] = a.w;
+              dv[c] = d.x; dv[c + 1] = d.y; dv[c + 2] = d.z; dv[c + 3] = d.w;
+            }
+            const int lim = kj - qc0 - 16 * ch;  // columns c < lim are queries before the key
+            const int tcut = T - qc0 - 16 * ch;  // columns c >= tcut are past the sequence
 #pragma unroll
-          for (int c8 = 0; c8 < 2; ++c8) {
-            const uint32_t off = (uint32_t)(((2 * ch + c8) ^ (r & 7)) << 4);
-            attn::st_shared_bf16x8(pt_row + off, pv + 8 * c8);
-            attn::st_shared_bf16x8(dst_row + off, dv + 8 * c8);
-          }
-          return true;
-        };
-        ld_chunk(0, sa, pa);
-        tc_wait_ld();
-        ld_chunk(1, sb, pb);
-        ok = do_chunk(0, sa, pa);
-        tc_wait_ld();
-        if (ok) {
-          ld_chunk(2, sa, pa);
-          do_chunk(1, sb, pb);
+            for (int c = 0; c < 16; ++c) {
+              float p = fast_exp2(fmaf(__uint_as_float(s_[c]), sl2, -pv[c]));
+              if (decltype(mask)::value && (c < lim || c >= tcut)) p = 0.f;
+              pv[c] = p;
+              dv[c] = p * (__uint_as_float(p_[c]) - dv[c]);
+            }
+            // the products of sub-tile gs - 2 have read this P^T / dS^T buffer
+            if (ch == 0 &&
+                !warp_and(mbar_wait(pd_empty0 + 8 * sb, ((gs >> 1) & 1u) ^ 1u, abort_flag, err)))
+              return false;
+#pragma unroll
+            for (int c8 = 0; c8 < 2; ++c8) {
+              const uint32_t off = (uint32_t)(((4 * half + 2 * ch + c8) ^ (r & 7)) << 4);
+              attn::st_shared_bf16x8(pt_row + off, pv + 8 * c8);
+              attn::st_shared_bf16x8(dst_row + off, dv + 8 * c8);
+            }
+            return true;
+          };
+          ld_chunk(0, sa, pa);
           tc_wait_ld();
-          ld_chunk(3, sb, pb);
-          do_chunk(2, sa, pa);
+          ld_chunk(1, sb16, pb);
+          ok = masked ? do_chunk(0, sa, pa, std::true_type{}) : do_chunk(0, sa, pa, std::false_type{});
           tc_wait_ld();
           tc_fence_before();
-          mbar_arrive(sd_empty);  // both score buffers are read: the next tile's may be computed
-          do_chunk(3, sb, pb);
+          mbar_arrive(sd_empty0 + 8 * sb);  // the scores are read: sub-tile gs + 2 may be computed
+          if (!ok) break;
+          if (masked) do_chunk(1, sb16, pb, std::true_type{});
+          else do_chunk(1, sb16, pb, std::false_type{});
+          fence_async_smem();
+          mbar_arrive(pd_full0 + 8 * sb);
         }
-        if (!ok) break;
-        fence_async_smem();
-        mbar_arrive(pd_full);
       }
       if (!ok) break;
       // the item's dV and dK (accumulator pair n_item % 2)
       const uint32_t ab = n_item & 1u, acc = kAccCol + ab * 2 * kHD;
-      ok = cbar_and(mbar_wait(acc_full0 + 8 * ab, (n_item >> 1) & 1u, abort_flag, err));
+      ok = warp_and(mbar_wait(acc_full0 + 8 * ab, (n_item >> 1) & 1u, abort_flag, err));
       if (!ok) break;
       tc_fence_after();
       uint32_t rv[32], rk[32];
@@ -359,7 +394,6 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           store8(row + 2 * C + i, d);
         }
       }
-      g += n;
     }
   }
 
@@ -554,6 +588,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         const int db = gg & 1;
         const int key0 = jj * kTile + 64 * half;
         const uint32_t ds_row = smem_u32(sDS + (db * 2 + half) * kBox) + (uint32_t)(r * 128);
+        // causal mask on the diagonal tile, padding past T on the last one
+        const bool masked = jj == i || (jj + 1) * kTile > T;
         ok = warp_and(mbar_wait(sd_full, gg & 1u, abort_flag, err));
         if (!ok) break;
         tc_fence_after();
@@ -565,14 +601,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           attn::tc_ld16(lane_base + col, s_);
           attn::tc_ld16(lane_base + kTile + col, p_);
         };
-        auto do_chunk = [&](int ch, const uint32_t* s_, const uint32_t* p_) -> bool {
+        auto do_chunk = [&](int ch, const uint32_t* s_, const uint32_t* p_, auto mask) -> bool {
           const int lim = qi - key0 - 16 * ch;  // columns c > lim are keys after the query
           const int tcut = T - key0 - 16 * ch;  // columns c >= tcut are past the sequence
           float ds[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             float p = fast_exp2(fmaf(__uint_as_float(s_[c]), sl2, -lse2));
-            if (c > lim || c >= tcut) p = 0.f;  // causal (only bites on the diagonal) and padding
+            if (decltype(mask)::value && (c > lim || c >= tcut)) p = 0.f;
             ds[c] = p * (__uint_as_float(p_[c]) - drow);
           }
           // the product two tiles back has read this dS buffer
@@ -584,22 +620,26 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
             attn::st_shared_bf16x8(ds_row + (uint32_t)(((2 * ch + c8) ^ (r & 7)) << 4), ds + 8 * c8);
           return true;
         };
-        ld_chunk(0, sa, pa);
-        tc_wait_ld();
-        ld_chunk(1, sb, pb);
-        ok = do_chunk(0, sa, pa);
-        tc_wait_ld();
-        if (ok) {
-          ld_chunk(2, sa, pa);
-          do_chunk(1, sb, pb);
+        auto run = [&](auto mask) {
+          ld_chunk(0, sa, pa);
           tc_wait_ld();
-          ld_chunk(3, sb, pb);
-          do_chunk(2, sa, pa);
+          ld_chunk(1, sb, pb);
+          ok = do_chunk(0, sa, pa, mask);
           tc_wait_ld();
-          tc_fence_before();
-          mbar_arrive(sd_empty);  // both score buffers are read: the next tile's may be computed
-          do_chunk(3, sb, pb);
-        }
+          if (ok) {
+            ld_chunk(2, sa, pa);
+            do_chunk(1, sb, pb, mask);
+            tc_wait_ld();
+            ld_chunk(3, sb, pb);
+            do_chunk(2, sa, pa, mask);
+            tc_wait_ld();
+            tc_fence_before();
+            mbar_arrive(sd_empty);  // both score buffers are read: the next tile's may be computed
+            do_chunk(3, sb, pb, mask);
+          }
+        };
+        if (masked) run(std::true_type{});
+        else run(std::false_type{});
         if (!ok) break;
         fence_async_smem();
         mbar_arrive(ds_full0 + 8 * db);
