@@ -45,6 +45,15 @@ int gpt2k_gemm(void* stream, int epi, int M, int N, int K, const void* A, long l
                long ldo32, const float* bias, const void* resid, long ldr, void* aux, long ldaux,
                float* split_ws, size_t split_ws_floats);
 
+/* Whether gpt2k_gemm (and the model's products) run the products with
+ * N >= 256, M > 128 and no split-K as 256 x 256 tiles over pairs of CTAs on
+ * neighbouring SMs (tcgen05 cta_group::2: each CTA stages half of the B
+ * tile, halving its shared-memory operand traffic) instead of 128 x 256
+ * tiles on single CTAs.  enable = 0 or 1; the default is 1; the fp32
+ * validation build has no pairs.  Process-wide, not thread-safe against
+ * concurrent launches; returns the previous setting. */
+int gpt2k_gemm_set_cta_pairs(int enable);
+
 /* Causal attention forward over qkv [B*T, 3C] = [q | k | v] (head h in
  * columns h*C/H .. of each part): att [B*T, C], lse [B, H, T] (natural-log
  * log-sum-exp of the scaled scores, fp32). */

@@ -58,12 +58,21 @@ def ref_linear(x, W, b=None):
 
 
 GEMM_SHAPES = [(128, 256, 64), (256, 384, 192), (300, 200, 136), (1000, 768, 768),
-               (64, 2304, 768), (513, 50304 // 8, 768)]
+               (64, 2304, 768), (513, 50304 // 8, 768), (16384, 768, 64)]
+
+
+@pytest.fixture(params=[1, 0], ids=["pairs", "single"])
+def cta_pairs(request):
+    """Both tilings of the wide products: 256 x 256 tiles over CTA pairs
+    (the default) and 128 x 256 tiles on single CTAs."""
+    prev = g2.gpt2k_gemm_set_cta_pairs(request.param)
+    yield request.param
+    g2.gpt2k_gemm_set_cta_pairs(prev)
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
 @pytest.mark.parametrize("epi", ["store", "bias", "bias_gelu", "bias_resid"])
-def test_gemm_forward(M, N, K, epi):
+def test_gemm_forward(M, N, K, epi, cta_pairs):
     rng = np.random.default_rng(M * 7 + N + K)
     x = bf16(rng.standard_normal((M, K)))
     W = bf16(rng.standard_normal((N, K)) * 0.05)
@@ -91,7 +100,7 @@ def test_gemm_forward(M, N, K, epi):
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 200, 136), (1000, 768, 3072), (256, 3072, 768)])
 @pytest.mark.parametrize("epi", ["store", "dgelu"])
-def test_gemm_dgrad(M, N, K, epi):
+def test_gemm_dgrad(M, N, K, epi, cta_pairs):
     """out[M, N] = dy[M, K] W[K, N] (W read MN-major, as the weight is stored)."""
     rng = np.random.default_rng(M + 3 * N + K)
     dy = bf16(rng.standard_normal((M, K)))
@@ -111,7 +120,7 @@ def test_gemm_dgrad(M, N, K, epi):
 @pytest.mark.parametrize("M,N,K,split", [(256, 128, 192, False), (200, 136, 300, False),
                                          (768, 768, 4096, True), (2304, 768, 2048, True),
                                          (3072, 768, 1000, True), (1024, 512, 520, False)])
-def test_gemm_wgrad_accumulates(M, N, K, split):
+def test_gemm_wgrad_accumulates(M, N, K, split, cta_pairs):
     """out32[M, N] += sum_k dy[k, M] x[k, N]: both operands MN-major (tokens
     are the reduction), fp32 accumulate, optional fixed-order split-K."""
     rng = np.random.default_rng(M + N + 5 * K)
@@ -127,6 +136,58 @@ def test_gemm_wgrad_accumulates(M, N, K, split):
     ref = g0 + 0.25 * ref_linear(np.ascontiguousarray(dy.T), np.ascontiguousarray(x.T))
     got = out32.cpu().double().numpy()
     assert np.abs(got - ref).max() <= 1e-5 * rms(ref) * np.sqrt(K / 64)
+
+
+@pytest.mark.parametrize("M,N,K", [(1000, 768, 768), (16384, 3072, 768)])
+def test_gemm_forward_is_deterministic(M, N, K, cta_pairs):
+    rng = np.random.default_rng(M + N)
+    A = dev(bf16(rng.standard_normal((M, K))))
+    B = dev(bf16(rng.standard_normal((N, K)) * 0.05))
+    bias = torch.tensor(rng.standard_normal(N).astype(np.float32), device="cuda")
+    outs = []
+    for _ in range(2):
+        o = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        u = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        g2.gpt2k_gemm("bias_gelu", M, N, K, A, K, 0, B, K, 0, 1.0, out=o, ldo=N, bias=bias,
+                      aux=u, ldaux=N)
+        outs.append((o.view(torch.int16).cpu().numpy(), u.view(torch.int16).cpu().numpy()))
+    assert g2.gpt2k_take_error() == 0
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("form", ["dgrad", "bias_resid", "wgrad"])
+def test_gemm_pairs_match_single_ctas(form):
+    """The two tilings accumulate every output in the same k order, so they
+    agree bit for bit."""
+    rng = np.random.default_rng(17)
+    M, N, K = 1000, 768, 3072
+    outs = []
+    for pairs in (1, 0):
+        prev = g2.gpt2k_gemm_set_cta_pairs(pairs)
+        if form == "dgrad":
+            dy = dev(bf16(np.random.default_rng(1).standard_normal((M, K))))
+            W = dev(bf16(np.random.default_rng(2).standard_normal((K, N)) * 0.05))
+            o = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            g2.gpt2k_gemm("store", M, N, K, dy, K, 0, W, N, 1, 0.5, out=o, ldo=N)
+            outs.append(o.view(torch.int16).cpu().numpy())
+        elif form == "bias_resid":
+            x = dev(bf16(np.random.default_rng(3).standard_normal((M, K))))
+            W = dev(bf16(np.random.default_rng(4).standard_normal((N, K)) * 0.05))
+            r = dev(bf16(np.random.default_rng(5).standard_normal((M, N))))
+            b = torch.tensor(np.random.default_rng(6).standard_normal(N).astype(np.float32), device="cuda")
+            o = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            g2.gpt2k_gemm("bias_resid", M, N, K, x, K, 0, W, K, 0, 1.0, out=o, ldo=N, bias=b,
+                          resid=r, ldr=N)
+            outs.append(o.view(torch.int16).cpu().numpy())
+        else:  # weight gradient without split-K: M = 768 output rows, tokens reduced
+            dy = dev(bf16(np.random.default_rng(7).standard_normal((K, N))))
+            x = dev(bf16(np.random.default_rng(8).standard_normal((K, 512))))
+            o = torch.zeros((N, 512), dtype=torch.float32, device="cuda")
+            g2.gpt2k_gemm("f32_acc", N, 512, K, dy, N, 1, x, 512, 1, 1.0, out32=o, ldo32=512)
+            outs.append(o.cpu().numpy())
+        g2.gpt2k_gemm_set_cta_pairs(prev)
+    assert g2.gpt2k_take_error() == 0
+    assert np.array_equal(outs[0], outs[1])
 
 
 def test_gemm_is_deterministic():

@@ -81,6 +81,8 @@ __global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, 
   }
 }
 
+int gemm_set_cta_pairs(int) { return 0; }  // no CTA pairs in this build
+
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   (void)err;
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return cudaSuccess;

@@ -56,16 +56,20 @@ constexpr bool epi_has_input(int epi) { return epi == EPI_BIAS_RESID || epi == E
 // backward (measured: one ring stage less slows the store, bias, GELU and
 // fp32 forms more than the second box gains).
 constexpr int epi_boxes(int epi) { return epi == EPI_DGELU ? 2 : 1; }
-// Operand ring depth: what the shared memory holds next to the epilogue boxes.
-constexpr int ring_stages(int bn, int epi) {
-  return bn == 256 ? (epi_boxes(epi) == 2 ? 3 : 4) : (epi_boxes(epi) == 2 ? 5 : 6);
+// Operand ring depth: what the shared memory holds next to the epilogue boxes
+// (a CTA of a pair holds half of the B tile, so its stages are smaller).
+constexpr int ring_stages(int bn, int epi, int cg) {
+  return cg == 2 ? (epi_boxes(epi) == 2 ? 5 : 6)
+                 : bn == 256 ? (epi_boxes(epi) == 2 ? 3 : 4) : (epi_boxes(epi) == 2 ? 5 : 6);
 }
 
-// Instruction descriptor: bf16 x bf16 -> fp32, M = 128, N = BN.
-template <int BN, bool A_MN, bool B_MN>
+// Instruction descriptor: bf16 x bf16 -> fp32, M = 128 per CTA (256 for a
+// pair), N = BN.
+template <int BN, bool A_MN, bool B_MN, int CG>
 __host__ __device__ constexpr uint32_t make_idesc() {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((A_MN ? 1u : 0u) << 15) |
-         ((B_MN ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+         ((B_MN ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)((BM * CG) >> 4) << 24);
 }
 
 template <int BN>
@@ -73,24 +77,30 @@ constexpr uint32_t tmem_cols() {
   return 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int CG>
 constexpr size_t smem_bytes() {
-  return 1024 + (size_t)ring_stages(BN, EPI) * (BM * BK * 2 + BN * BK * 2) +
+  return 1024 + (size_t)ring_stages(BN, EPI, CG) * (BM * BK * 2 + (BN / CG) * BK * 2) +
          (size_t)kEpiWarps * epi_boxes(EPI) * kWarpBox + 256;
 }
 
-template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI>
+template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmOut,
                    const __grid_constant__ CUtensorMap tmX, const EpiParams ep, int K,
                    int tiles_m, int tiles_n, int splits, int kb_per_split, int n_fast, int* err) {
   constexpr int A_BYTES = BM * BK * 2;
-  constexpr int B_BYTES = BN * BK * 2;
+  constexpr int B_BYTES = (BN / CG) * BK * 2;  // this CTA's rows of the B tile
   constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = tmem_cols<BN>();
   constexpr bool HAS_IN = epi_has_input(EPI);
-  static_assert(STAGES == ring_stages(BN, EPI), "ring depth");
+  static_assert(STAGES == ring_stages(BN, EPI, CG), "ring depth");
+  static_assert(CG == 1 || (CG == 2 && BN == 256), "CTA pairs use 256 x 256 tiles");
+  // CTA pair: rank 0 (the leader) issues the MMAs for both CTAs; each CTA
+  // loads its 128 rows of A and BN / 2 rows of B and runs the epilogue of
+  // its 128 rows of the tile.
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
   constexpr bool F32_OUT = (EPI == EPI_F32_ACC || EPI == EPI_F32_STORE);
   constexpr bool HAS_BIAS = (EPI == EPI_BIAS || EPI == EPI_BIAS_GELU || EPI == EPI_BIAS_RESID);
 
@@ -116,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kb_total = (K + BK - 1) / BK;
   const int tiles = tiles_m * tiles_n;
   const int units = tiles * splits;
+  const int unit0 = blockIdx.x / CG, unit_step = gridDim.x / CG;  // a pair shares its units
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -124,20 +135,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, kEpiThreads);
+      mbar_init(tempty0 + 8 * b, CG * kEpiWarps);  // one arrival per epilogue warp of the pair
     }
     for (int w = 0; w < kEpiWarps; ++w) mbar_init(in_full0 + 8 * w, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  if (warp == 1) {  // for a pair: one warp of each CTA allocates collectively
+    if (CG == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(TMEM_COLS));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync();  // the peer's barriers are initialised before any remote use
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -165,29 +184,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued_mask = 0;  // stages that received at least one load
       uint32_t last_parity = 0;  // parity of the latest fill of each stage
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = unit0; u < units && ok; u += unit_step) {
         int tm, tn, kb0, kb1, sp;
         decode(u, tm, tn, kb0, kb1, sp);
+        const int am = tm * BM * CG + (int)rank * BM;          // this CTA's rows of A
+        const int bn0 = tn * BN + (int)rank * (BN / CG);       // and of B
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, err)) {
             ok = false;
             break;
           }
           const uint32_t fb = full0 + 8 * stage;
-          mbar_expect_tx(fb, STAGE_TX);
           const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
-          if (!A_MN) {
-            tma_load_2d(a_dst, &tmA, fb, kb * BK, tm * BM);
-          } else {
-            tma_load_2d(a_dst, &tmA, fb, tm * BM, kb * BK);
-            tma_load_2d(a_dst + 8192, &tmA, fb, tm * BM + 64, kb * BK);
-          }
-          if (!B_MN) {
-            tma_load_2d(b_dst, &tmB, fb, kb * BK, tn * BN);
-          } else {
+          if (CG == 1) {
+            mbar_expect_tx(fb, STAGE_TX);
+            if (!A_MN) {
+              tma_load_2d(a_dst, &tmA, fb, kb * BK, am);
+            } else {
+              tma_load_2d(a_dst, &tmA, fb, am, kb * BK);
+              tma_load_2d(a_dst + 8192, &tmA, fb, am + 64, kb * BK);
+            }
+            if (!B_MN) {
+              tma_load_2d(b_dst, &tmB, fb, kb * BK, bn0);
+            } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + 8192 * j, &tmB, fb, tn * BN + 64 * j, kb * BK);
+              for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + 8192 * j, &tmB, fb, bn0 + 64 * j, kb * BK);
+            }
+          } else {
+            // both CTAs' copies complete on the leader's full barrier, which
+            // expects the pair's bytes
+            if (leader) mbar_expect_tx(fb, CG * STAGE_TX);
+            const uint32_t lfb = map_shared(fb, 0);
+            if (!A_MN) {
+              tma_load_2d_pair(a_dst, &tmA, lfb, kb * BK, am);
+            } else {
+              tma_load_2d_pair(a_dst, &tmA, lfb, am, kb * BK);
+              tma_load_2d_pair(a_dst + 8192, &tmA, lfb, am + 64, kb * BK);
+            }
+            if (!B_MN) {
+              tma_load_2d_pair(b_dst, &tmB, lfb, kb * BK, bn0);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BN / CG / 64; ++j)
+                tma_load_2d_pair(b_dst + 8192 * j, &tmB, lfb, bn0 + 64 * j, kb * BK);
+            }
           }
           issued_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -197,7 +238,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) {
+      if (!ok && CG == 2 && !leader) {
+        // this CTA's copies complete on the leader's barriers: give them a
+        // short bounded time to land
+        const uint64_t t0 = global_ns();
+        while (global_ns() - t0 < 200000ull) {
+        }
+      } else if (!ok) {
         // Give the copies already issued a bounded time to land before the
         // shared memory they target is released.
         const uint64_t t0 = global_ns();
@@ -211,18 +258,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // --------------------------------------------------------- MMA --
-      constexpr uint32_t idesc = make_idesc<BN, A_MN, B_MN>();
+      constexpr uint32_t idesc = make_idesc<BN, A_MN, B_MN, CG>();
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = unit0; u < units && ok; u += unit_step) {
         int tm, tn, kb0, kb1, sp;
         decode(u, tm, tn, kb0, kb1, sp);
-        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, err)) break;
+        if (CG == 2 ? !mbar_wait_cluster(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, err)
+                    : !mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, err))
+          break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -237,22 +286,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = A_MN ? desc_mnmajor(a_base, k) : desc_kmajor(a_base, k);
             const uint64_t bd = B_MN ? desc_mnmajor(b_base, k) : desc_kmajor(b_base, k);
-            tc_mma(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            if (CG == 1) tc_mma(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            else tc_mma_pair(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
           }
-          tc_commit(empty0 + 8 * stage);
+          if (CG == 1) tc_commit(empty0 + 8 * stage);
+          else tc_commit_pair(empty0 + 8 * stage, 0x3);  // the stage is free in both CTAs
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(tfull0 + 8 * acc);
+        if (CG == 1) tc_commit(tfull0 + 8 * acc);
+        else tc_commit_pair(tfull0 + 8 * acc, 0x3);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       if (!ok) {
         // let MMAs already issued finish before TMEM is released
-        tc_commit(tfull0 + 8 * acc);
+        if (CG == 1) tc_commit(tfull0 + 8 * acc);
+        else tc_commit_pair(tfull0 + 8 * acc, 0x1);
         const uint64_t t0 = global_ns();
         while (!mbar_try_wait(tfull0 + 8 * acc, acc_phase)) {
           if (global_ns() - t0 > kWaitLimitNs) break;
@@ -300,23 +353,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (OUT_BOXES == 2) ob ^= 1;
     };
+    // This warp has read its accumulator columns of the tile: one arrival
+    // per warp on the leader's barrier (the peer CTA's warps arrive remotely).
+    const uint32_t tempty_leader = CG == 2 ? map_shared(tempty0, 0) : 0u;
+    auto release_acc = [&](int a) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (CG == 1) mbar_arrive(tempty0 + 8 * a);
+        else mbar_arrive_cluster(tempty_leader + 8 * a);
+      }
+    };
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (int u = unit0; u < units && ok; u += unit_step) {
       int tm, tn, kb0, kb1, sp;
       decode(u, tm, tn, kb0, kb1, sp);
-      const int m0 = tm * BM, nt0 = tn * BN;
+      const int m0 = tm * BM * CG + (int)rank * BM, nt0 = tn * BN;
       const int r0 = m0 + q * 32;  // first row of this warp's slab
       const int ngroups = (min(BN, ep.N - nt0) + 63) >> 6;  // 64-column groups in range
       ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, err));
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if (h >= ngroups) {  // no group for this warp in a narrow tile
-        tc_fence_before();
-        mbar_arrive(tempty0 + 8 * acc);
-      }
+      if (h >= ngroups) release_acc(acc);  // no group for this warp in a narrow tile
 #pragma unroll 1
       for (int g = h; g < ngroups; g += 2) {
         const int nb = nt0 + 64 * g;  // first column of the group
@@ -336,10 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_ld32(t_row + (uint32_t)(64 * g), r);
           tc_ld32(t_row + (uint32_t)(64 * g + 32), r + 32);
           tc_wait_ld();
-          if (g + 2 >= ngroups) {  // every TMEM read of this warp for the tile is done
-            tc_fence_before();
-            mbar_arrive(tempty0 + 8 * acc);
-          }
+          if (g + 2 >= ngroups) release_acc(acc);  // every TMEM read of this warp for the tile is done
 #pragma unroll
           for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]) * ep.alpha;
         }
@@ -374,10 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (g + 2 < ngroups) {
               pn = nb + 128;
               pr = r0;
-            } else if (u + (int)gridDim.x < units) {
+            } else if (u + unit_step < units) {
               int tm2, tn2, kb02, kb12, sp2;
-              decode(u + gridDim.x, tm2, tn2, kb02, kb12, sp2);
-              const int nt2 = tn2 * BN, r2 = tm2 * BM + q * 32;
+              decode(u + unit_step, tm2, tn2, kb02, kb12, sp2);
+              const int nt2 = tn2 * BN, r2 = tm2 * BM * CG + (int)rank * BM + q * 32;
               if (h < ((min(BN, ep.N - nt2) + 63) >> 6) && r2 < ep.M) {
                 pn = nt2 + 64 * h;
                 pr = r2;
@@ -474,11 +532,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  // a pair leaves together: no MMA of the leader, copy or remote arrival
+  // still targets the peer when it exits
+  if (CG == 2) cluster_sync();
+  else __syncthreads();
   tc_fence_after();
   if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(TMEM_COLS));
+    if (CG == 1)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(TMEM_COLS));
+    else
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(TMEM_COLS));
   }
 }
 
@@ -547,12 +612,12 @@ static int num_sms() {
   return n;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
+template <int BN, bool A_MN, bool B_MN, int EPI, int CG>
 static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
                           const CUtensorMap& tx, const EpiParams& ep, int K, int splits,
                           int kb_per_split, int n_fast, cudaStream_t s, int* err) {
-  auto kern = gemm_tc_kernel<BN, ring_stages(BN, EPI), A_MN, B_MN, EPI>;
-  constexpr size_t smem = smem_bytes<BN, EPI>();
+  auto kern = gemm_tc_kernel<BN, ring_stages(BN, EPI, CG), A_MN, B_MN, EPI, CG>;
+  constexpr size_t smem = smem_bytes<BN, EPI, CG>();
   static_assert(smem <= 232448, "shared memory budget");
   static bool attr_done = false;
   if (!attr_done) {
@@ -560,24 +625,44 @@ static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CU
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  const int tiles_m = (ep.M + BM - 1) / BM;
+  const int tiles_m = (ep.M + BM * CG - 1) / (BM * CG);
   const int tiles_n = (ep.N + BN - 1) / BN;
   const int units = tiles_m * tiles_n * splits;
-  const int grid = units < num_sms() ? units : num_sms();
-  kern<<<grid, kThreads, smem, s>>>(ta, tb, to, tx, ep, K, tiles_m, tiles_n, splits, kb_per_split,
-                                    n_fast, err);
+  const int slots = num_sms() / CG;  // persistent CTAs (pairs)
+  const int grid = CG * (units < slots ? units : slots);
+  if (CG == 1) {
+    kern<<<grid, kThreads, smem, s>>>(ta, tb, to, tx, ep, K, tiles_m, tiles_n, splits,
+                                      kb_per_split, n_fast, err);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, to, tx, ep, K, tiles_m, tiles_n, splits,
+                                       kb_per_split, n_fast, err);
+    if (e != cudaSuccess) return e;
+  }
   note_launch();
   return cudaGetLastError();
 }
 
-template <int BN>
+template <int BN, int CG>
 static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb,
                             const CUtensorMap& to, const CUtensorMap& tx, const EpiParams& ep,
                             int epi, int splits, int kb_per_split, int n_fast, cudaStream_t s,
                             int* err) {
 #define GPT2_TC(AM, BMJ, E)                                                                      \
-  if (a.a_mn == AM && a.b_mn == BMJ && epi == E)                                                 \
-    return launch<BN, AM, BMJ, E>(ta, tb, to, tx, ep, a.K, splits, kb_per_split, n_fast, s, err);
+  if constexpr (CG == 1 || (E != EPI_BIAS_GELU && E != EPI_DGELU))                               \
+    if (a.a_mn == AM && a.b_mn == BMJ && epi == E)                                               \
+      return launch<BN, AM, BMJ, E, CG>(ta, tb, to, tx, ep, a.K, splits, kb_per_split, n_fast, s, err);
   GPT2_TC(0, 0, EPI_STORE)
   GPT2_TC(0, 0, EPI_BIAS)
   GPT2_TC(0, 0, EPI_BIAS_GELU)
@@ -622,6 +707,13 @@ __global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, 
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+static int g_cta_pairs = 1;
+int gemm_set_cta_pairs(int enable) {
+  const int prev = g_cta_pairs;
+  g_cta_pairs = enable ? 1 : 0;
+  return prev;
+}
+
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   using namespace tc;
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return cudaSuccess;
@@ -643,9 +735,6 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   cudaError_t e;
   if (!a.a_mn) e = make_tmap(&ta, a.A, false, a.K, a.M, a.lda, 64, BM);
   else e = make_tmap(&ta, a.A, false, a.M, a.K, a.lda, 64, 64);
-  if (e != cudaSuccess) return e;
-  if (!a.b_mn) e = make_tmap(&tb, a.B, false, a.K, a.N, a.ldb, 64, BN);
-  else e = make_tmap(&tb, a.B, false, a.N, a.K, a.ldb, 64, 64);
   if (e != cudaSuccess) return e;
 
   EpiParams ep{a.M, a.N, a.alpha, a.out, a.ldo, a.out32, a.ldo32, a.bias, a.resid, a.ldr, a.aux, a.ldaux};
@@ -676,6 +765,16 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   }
   int kb_per_split = (kb_total + splits - 1) / splits;
   splits = (kb_total + kb_per_split - 1) / kb_per_split;  // no empty split
+  // 256 x 256 tiles over CTA pairs for the wide products without split-K
+  // (measured: 5-11 % faster where the main loop sets the pace).  The GELU
+  // and GELU-backward epilogues set the pace of their products; there the
+  // pair waits for the slower of its two epilogues and single CTAs are
+  // faster (measured 3-6 %).
+  const bool epi_bound = a.epi == EPI_BIAS_GELU || a.epi == EPI_DGELU;
+  const int CG = (g_cta_pairs && BN == 256 && splits == 1 && a.M > BM && !epi_bound) ? 2 : 1;
+  if (!a.b_mn) e = make_tmap(&tb, a.B, false, a.K, a.N, a.ldb, 64, BN / CG);
+  else e = make_tmap(&tb, a.B, false, a.N, a.K, a.ldb, 64, 64);
+  if (e != cudaSuccess) return e;
   // epilogue tensor maps
   // epilogue tensor maps: one warp's 32-row slab per box
   if (splits > 1) {
@@ -694,10 +793,12 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   // The larger operand is reused by consecutive tiles (L2 locality).
   const double a_bytes = (double)a.M * a.K, b_bytes = (double)a.N * a.K;
   const int n_fast = a_bytes > b_bytes ? 1 : 0;
-  if (BN == 256)
-    e = dispatch<256>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
+  if (CG == 2)
+    e = dispatch<256, 2>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
+  else if (BN == 256)
+    e = dispatch<256, 1>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
   else
-    e = dispatch<128>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
+    e = dispatch<128, 1>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
   if (e != cudaSuccess) return e;
   if (splits > 1) {
     const size_t total = (size_t)a.M * a.N;

@@ -25,6 +25,8 @@ int status(cudaError_t e) { return e == cudaSuccess ? GPT2_OK : (e == cudaErrorI
 
 extern "C" {
 
+int gpt2k_gemm_set_cta_pairs(int enable) { return gemm_set_cta_pairs(enable); }
+
 int gpt2k_gemm(void* stream, int epi, int M, int N, int K, const void* A, long lda, int a_mn,
                const void* B, long ldb, int b_mn, float alpha, void* out, long ldo, float* out32,
                long ldo32, const float* bias, const void* resid, long ldr, void* aux, long ldaux,

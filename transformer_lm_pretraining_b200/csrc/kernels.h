@@ -53,6 +53,9 @@ struct GemmArgs {
 };
 
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err_flag);
+// Whether wide products run as 256 x 256 tiles over CTA pairs (default on;
+// the fp32 build has no pairs).  Returns the previous setting.
+int gemm_set_cta_pairs(int enable);
 
 // ------------------------------------------------------------- encoder --
 // x0[m, :] = wte[tok[m], :] + wpe[m % T, :]; saves the (range-checked)

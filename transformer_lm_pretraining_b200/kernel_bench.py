@@ -125,6 +125,7 @@ def main():
     g.add_argument("--form", default="fwd", choices=["fwd", "dgrad", "wgrad"])
     g.add_argument("--epi", default="bias")
     g.add_argument("--iters", type=int, default=20)
+    g.add_argument("--pairs", type=int, default=1, help="256 x 256 tiles over CTA pairs (1) or not (0)")
     t = sub.add_parser("attn")
     t.add_argument("--B", type=int, default=16)
     t.add_argument("--T", type=int, default=1024)
@@ -145,6 +146,8 @@ def main():
     c.set_defaults(form="fwd+grad")
     a = ap.parse_args()
     torch.manual_seed(0)
+    if a.kind == "gemm":
+        g2.gpt2k_gemm_set_cta_pairs(a.pairs)
     call, work = {"gemm": bench_gemm, "attn": bench_attn, "ln": bench_ln, "cls": bench_cls}[a.kind](a)
     call()
     torch.cuda.synchronize()
