@@ -46,7 +46,8 @@ int gpt2k_gemm(void* stream, int epi, int M, int N, int K, const void* A, long l
                float* split_ws, size_t split_ws_floats);
 
 /* Whether gpt2k_gemm (and the model's products) run the products with
- * N >= 256, M > 128 and no split-K as 256 x 256 tiles over pairs of CTAs on
+ * N >= 256 and M > 128 (other than the GELU epilogues, whose pace their
+ * epilogue sets) as 256 x 256 tiles over pairs of CTAs on
  * neighbouring SMs (tcgen05 cta_group::2: each CTA stages half of the B
  * tile, halving its shared-memory operand traffic) instead of 128 x 256
  * tiles on single CTAs.  enable = 0 or 1; the default is 1; the fp32

@@ -738,7 +738,14 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   if (e != cudaSuccess) return e;
 
   EpiParams ep{a.M, a.N, a.alpha, a.out, a.ldo, a.out32, a.ldo32, a.bias, a.resid, a.ldr, a.aux, a.ldaux};
-  const int tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  // 256 x 256 tiles over CTA pairs for the wide products (measured: 5-11 %
+  // faster where the main loop sets the pace).  The GELU and GELU-backward
+  // epilogues set the pace of their products; there the pair waits for the
+  // slower of its two epilogues and single CTAs are faster (measured 3-6 %).
+  const bool epi_bound = a.epi == EPI_BIAS_GELU || a.epi == EPI_DGELU;
+  const int CG = (g_cta_pairs && BN == 256 && a.M > BM && !epi_bound) ? 2 : 1;
+  const int slots = num_sms() / CG;  // persistent CTAs or pairs
+  const int tiles = ((a.M + BM * CG - 1) / (BM * CG)) * ((a.N + BN - 1) / BN);
   const int kb_total = (a.K + BK - 1) / BK;
 
   // split-K for the weight-gradient products with few output tiles: pick the
@@ -747,13 +754,13 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   // at ~6 TB/s (at least 4 k-blocks per split; partials must fit)
   int splits = 1;
   int epi = a.epi;
-  if (a.epi == EPI_F32_ACC && a.max_splits > 1 && a.split_ws && tiles < num_sms() &&
+  if (a.epi == EPI_F32_ACC && a.max_splits > 1 && a.split_ws && tiles < slots &&
       aligned16(a.split_ws) && a.N % 4 == 0) {
     double best = 1e30;
     const double out_bytes = 4.0 * a.M * a.N;
     for (int sp = 1; sp <= a.max_splits; ++sp) {
       if (sp > 1 && (sp > kb_total / 4 || (size_t)sp * a.M * a.N > a.split_ws_floats)) break;
-      const int waves = (tiles * sp + num_sms() - 1) / num_sms();
+      const int waves = (tiles * sp + slots - 1) / slots;
       const double t_unit = 2.0 * BM * BN * ((double)kb_total * BK / sp) / 8.5e12;
       const double t_red = sp > 1 ? (2.0 * sp + 2.0) * out_bytes / 6.0e12 : 0.0;
       const double t = waves * t_unit + t_red;
@@ -765,13 +772,6 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   }
   int kb_per_split = (kb_total + splits - 1) / splits;
   splits = (kb_total + kb_per_split - 1) / kb_per_split;  // no empty split
-  // 256 x 256 tiles over CTA pairs for the wide products without split-K
-  // (measured: 5-11 % faster where the main loop sets the pace).  The GELU
-  // and GELU-backward epilogues set the pace of their products; there the
-  // pair waits for the slower of its two epilogues and single CTAs are
-  // faster (measured 3-6 %).
-  const bool epi_bound = a.epi == EPI_BIAS_GELU || a.epi == EPI_DGELU;
-  const int CG = (g_cta_pairs && BN == 256 && splits == 1 && a.M > BM && !epi_bound) ? 2 : 1;
   if (!a.b_mn) e = make_tmap(&tb, a.B, false, a.K, a.N, a.ldb, 64, BN / CG);
   else e = make_tmap(&tb, a.B, false, a.N, a.K, a.ldb, 64, 64);
   if (e != cudaSuccess) return e;
