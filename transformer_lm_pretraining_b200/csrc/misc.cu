@@ -525,9 +525,16 @@ int grid_for(size_t n, int threads, int max_blocks) {
 }  // namespace
 
 void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s) {
-  // enough chunks for ~8 blocks per SM
+  // as many blocks as are resident at once and no more: a block past the
+  // first wave would run on its own after it
+  static int per_sm = 0;
+  if (!per_sm) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, colsum_partial_kernel, 256, 0);
+    if (per_sm < 1) per_sm = 1;
+  }
   const int colgroups = (N + 255) / 256;
-  int want = (8 * kNumSMs + colgroups - 1) / colgroups;
+  int want = per_sm * kNumSMs / colgroups;
+  if (want < 1) want = 1;
   if (want > kColsumChunks) want = kColsumChunks;
   const int rows = (M + want - 1) / want;
   const int chunks = (M + rows - 1) / rows;
