@@ -19,7 +19,6 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
-import datetime
 import json
 import os
 import statistics
@@ -197,27 +196,14 @@ def run_reference(args, wl):
 
 def run_ours(args, wl):
     import torch
-    import torch.distributed as dist
 
     from transformer_lm_pretraining_b200 import gpt2 as g2
+    from transformer_lm_pretraining_b200.replicas import Replicas
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    reps = Replicas("nccl", timeout_s=120)
+    world, rank, local = reps.world, reps.rank, reps.local_rank
+    barrier, max_over_ranks = reps.barrier, reps.max
 
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
@@ -226,7 +212,7 @@ def run_ours(args, wl):
     evaluate = args.mode == "eval"
     model.set_stream(stream)
     n_steps = args.warmup + args.steps
-    host = make_batches(wl, n_steps, seed=1 + rank)
+    host = make_batches(wl, n_steps, seed=reps.data_seed(1))
     # inputs resident in HBM before the timed region
     dev = [[(torch.from_numpy(t).cuda(), torch.from_numpy(y).cuda()) for t, y in st] for st in host]
     scale = 1.0 / wl.n_micro
@@ -278,8 +264,7 @@ def run_ours(args, wl):
     prof = model.profile_read()
     model.profile_enable(False)
     ms_step = ms_total / args.steps
-    tokens = wl.tokens_per_step * args.steps * world
-    value = tokens / (ms_total / 1e3)
+    value = reps.throughput(wl.tokens_per_step * args.steps, ms_total)
 
     # end to end through the public API: pinned host inputs copied in and the
     # loss read back every step
@@ -313,7 +298,7 @@ def run_ours(args, wl):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-        e2e = {"value": wl.tokens_per_step * n_e2e * world / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": reps.throughput(wl.tokens_per_step * n_e2e, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": 2 * 4 * wl.B * wl.T * wl.n_micro, "d2h_bytes_per_step": 4}
 
     peaks = load_peaks()
@@ -364,11 +349,9 @@ def run_ours(args, wl):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not evaluate:
         out["cpu_baseline"] = cpu_baseline(wl, args.cpu_sample_T)
-    if world > 1:
-        barrier()
-        dist.destroy_process_group()
+    reps.close()
     model.close()
-    return out if rank == 0 else None
+    return out if reps.is_root else None
 
 
 def run_generate(args, wl):
@@ -378,20 +361,24 @@ def run_generate(args, wl):
     import torch
 
     from transformer_lm_pretraining_b200 import gpt2 as g2
+    from transformer_lm_pretraining_b200.replicas import Replicas
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    reps = Replicas("nccl", timeout_s=120)
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
     Tp, Ttot = max(1, wl.T // 8), max(2, wl.T // 4)
     model = g2.GPT2(wl.L, wl.H, wl.C, wl.V, wl.Vp, wl.Tmax, seed=0, precision="bf16", B=wl.B, T=Tp)
     model.set_stream(stream)
-    prompt = ZipfStream(wl.V, 1).next_batch(wl.B, Tp)[0]
+    prompt = ZipfStream(wl.V, reps.data_seed(1)).next_batch(wl.B, Tp)[0]
     tok = torch.zeros((wl.B, Ttot), dtype=torch.int32, device="cuda")
     tok[:, :Tp] = torch.from_numpy(prompt).cuda()
     for _ in range(args.warmup):
         model.generate(tok, Tp, 0.8, 40, 7)
     torch.cuda.synchronize()
-    clocks = ClockSampler(0)
+    reps.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(reps.local_rank)
     clocks.start()
     n0 = g2.gpt2_launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -401,9 +388,11 @@ def run_generate(args, wl):
     e1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
+    reps.barrier()
+    ms_total = reps.max(e0.elapsed_time(e1))
+    ms = ms_total / args.steps
     new = Ttot - Tp
-    value = wl.B * new / (ms / 1e3)
+    value = reps.throughput(wl.B * new * args.steps, ms_total)
     launches = (g2.gpt2_launch_count() - n0) // args.steps
     # each decode step streams the bf16 weights once plus the cached keys
     # and values of the positions so far (prefill excluded from the bytes)
@@ -412,9 +401,12 @@ def run_generate(args, wl):
     kv_bytes = 2.0 * wl.L * wl.B * 2 * wl.C * sum(range(Tp + 1, Ttot))
     step_ms = ms / new
     achieved = (w_bytes * (new - 1) + kv_bytes) / (ms / 1e3) / 1e9
+    reps.close()
     model.close()
+    if not reps.is_root:
+        return None
     return {"metric": f"generation tokens/s (key/value cache), {wl.name} bf16",
-            "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "value": value, "unit": "tokens/s", "n_gpus": reps.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.B, "prompt": Tp, "total": Ttot,
