@@ -15,6 +15,17 @@
 //              TMA in the same box ahead of the accumulator read.  Warps
 //              synchronise only within themselves, so no epilogue step
 //              waits for another warp.
+// CTA pairs (template argument CG = 2, a cluster of two CTAs on neighbouring
+// SMs): 256 x 256 output tiles.  Each CTA stages its own 128 rows of A and
+// half of the B tile (its ring stages are 32 KB, six of them), its TMA
+// copies completing on the even CTA's full barrier; the even CTA's MMA
+// thread issues tcgen05.mma.cta_group::2 (M = 256), so each SM computes its
+// 128 x 256 half of the tile while reading only half of B from shared
+// memory.  Stage releases and tile completions reach both CTAs through
+// multicast tcgen05.commit; each epilogue warp of either CTA returns the
+// accumulator with one arrival on the even CTA's barrier.  TMEM is
+// allocated and freed by one warp of each CTA together, after cluster
+// barriers.  No TMA load multicasts.
 // The TMEM accumulator is double-buffered so the epilogue of one tile runs
 // under the main loop of the next.  Both operands may be K-major or
 // MN-major (the tensor core reads either from the descriptor), which covers
