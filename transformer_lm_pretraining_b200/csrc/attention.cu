@@ -650,14 +650,17 @@ cudaError_t attention_fwd(act_t* att, float* lse, const act_t* qkv, int B, int T
 cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
                           const act_t* att, const float* lse, int B, int T, int C, int H,
                           int* err, cudaStream_t s) {
+  const int hd = C / H;
+#if GPT2_ACT_BF16
+  // the tcgen05 kernels form D themselves (head dim 64)
+  if (hd == 64) return attention_bwd_tc(dqkv, dsum, datt, qkv, att, lse, B, T, C, H, err, s);
+#endif
   const size_t n = (size_t)B * T * H;
   attn_rowdot_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dsum, datt, att, B, T, C, H);
   note_launch();
-  const int hd = C / H;
 #if GPT2_ACT_BF16
   switch (hd) {
     case 32: return bwd_launch<32>(dqkv, dsum, datt, qkv, lse, B, T, C, H, s);
-    case 64: return attention_bwd_tc(dqkv, dsum, datt, qkv, lse, B, T, C, H, err, s);  // tcgen05
     case 128: return bwd_launch<128>(dqkv, dsum, datt, qkv, lse, B, T, C, H, s);
     default: return cudaErrorInvalidValue;
   }

@@ -18,7 +18,9 @@
 //          are double-buffered across items.
 //   dQ:    item = (batch, head, query tile i); streams the key tiles j <= i:
 //          S = Q K^T and dP = dO V^T into TMEM, dS into shared memory,
-//          dQ += dS K in TMEM (K read MN-major).
+//          dQ += dS K in TMEM (K read MN-major).  It runs first and also
+//          forms D = rowsum(dO * O) of its rows from the dO and O tiles it
+//          loads, storing it for the dK/dV kernel.
 // The compute warps hand the score buffers back to the tensor core as soon
 // as they have read them, so the next scores are computed while the current
 // ones are finished; the gradient accumulators are double-buffered in TMEM,
@@ -406,21 +408,23 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 // --------------------------------------------------------------------- dQ --
 constexpr int kKVStages = 3;
 constexpr size_t dq_smem_bytes() {
-  // Q, dO, [K, V] x stages, dS (two buffers of two boxes), aux
-  return 1024 + 2 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + 4 * (size_t)kBox + kAux;
+  // Q, dO, O, [K, V] x stages, dS (two buffers of two boxes), aux
+  return 1024 + 3 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + 4 * (size_t)kBox + kAux;
 }
 
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     flash_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
-                           const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse,
-                           const float* __restrict__ dsum, __nv_bfloat16* __restrict__ dqkv, int B,
+                           const __grid_constant__ CUtensorMap tmDO,
+                           const __grid_constant__ CUtensorMap tmO, const float* __restrict__ lse,
+                           float* __restrict__ dsum, __nv_bfloat16* __restrict__ dqkv, int B,
                            int T, int C, int H, float sl2, float scale, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
   uint8_t* sDO = sQ + kBox;
-  uint8_t* sK = sDO + kBox;                // [kKVStages]
+  uint8_t* sO = sDO + kBox;                // the forward's output rows (for D)
+  uint8_t* sK = sO + kBox;                 // [kKVStages]
   uint8_t* sV = sK + kKVStages * kBox;     // [kKVStages]
   uint8_t* sDS = sV + kKVStages * kBox;    // [2 buffers][2 boxes]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + 4 * kBox);
@@ -444,7 +448,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
-    mbar_init(qd_empty, 1);
+    mbar_init(qd_empty, 1 + kCT);  // the last S/dP product, and every compute thread's D
     for (int s = 0; s < kKVStages; ++s) {
       mbar_init(kv_full0 + 8 * s, 1);
       mbar_init(kv_empty0 + 8 * s, 1);
@@ -472,6 +476,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       // ------------------------------------------------------------ TMA --
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQKV)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmDO)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmO)) : "memory");
       uint32_t n_item = 0, gk = 0;  // items started, key tiles loaded
       uint32_t issued = 0, last_par = 0;
       bool ok = true;
@@ -481,9 +486,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         const int i = nq - 1 - w / BH, bh = w % BH, b = bh / H, h = bh % H;
         const int n = i + 1;  // key tiles 0 .. i
         if (!mbar_wait(qd_empty, (n_item & 1u) ^ 1u, abort_flag, err)) break;
-        mbar_expect_tx(qd_full, 2 * kBox);
+        mbar_expect_tx(qd_full, 3 * kBox);
         tma_load_3d(smem_u32(sQ), &tmQKV, qd_full, h * kHD, i * kTile, b);
         tma_load_3d(smem_u32(sDO), &tmDO, qd_full, h * kHD, i * kTile, b);
+        tma_load_3d(smem_u32(sO), &tmO, qd_full, h * kHD, i * kTile, b);
         for (int jj = 0; jj < n; ++jj, ++gk) {
           const int st = gk % kKVStages;
           const uint32_t par = (gk / kKVStages) & 1u;
@@ -582,7 +588,21 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const int n = i + 1;
       const int qi = i * kTile + r;  // this thread's query row
       const float lse2 = qi < T ? lse[(size_t)bh * T + qi] * kLog2e : 0.f;
-      const float drow = qi < T ? dsum[(size_t)bh * T + qi] : 0.f;
+      // D = rowsum(dO * O) of this row from the item's dO and O tiles (rows
+      // past T are zero-filled); stored for the dK/dV kernel, which runs next
+      ok = warp_and(mbar_wait(qd_full, n_item & 1u, abort_flag, err));
+      if (!ok) break;
+      float drow = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float a[8], o[8];
+        load8(reinterpret_cast<const __nv_bfloat16*>(sDO + swz(r, c)), a);
+        load8(reinterpret_cast<const __nv_bfloat16*>(sO + swz(r, c)), o);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) drow = fmaf(a[e], o[e], drow);
+      }
+      mbar_arrive(qd_empty);  // this thread is done with dO and O
+      if (half == 0 && qi < T) dsum[(size_t)bh * T + qi] = drow;
       for (int jj = 0; jj < n && ok; ++jj) {
         const uint32_t gg = gk + jj;
         const int db = gg & 1;
@@ -676,15 +696,18 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 
 }  // namespace
 
-cudaError_t attention_bwd_tc(act_t* dqkv, const float* dsum, const act_t* datt, const act_t* qkv,
-                             const float* lse, int B, int T, int C, int H, int* err,
-                             cudaStream_t s) {
-  if (C / H != kHD || (reinterpret_cast<uintptr_t>(qkv) & 15) || (reinterpret_cast<uintptr_t>(datt) & 15))
+cudaError_t attention_bwd_tc(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
+                             const act_t* att, const float* lse, int B, int T, int C, int H,
+                             int* err, cudaStream_t s) {
+  if (C / H != kHD || (reinterpret_cast<uintptr_t>(qkv) & 15) ||
+      (reinterpret_cast<uintptr_t>(datt) & 15) || (reinterpret_cast<uintptr_t>(att) & 15))
     return cudaErrorInvalidValue;
-  CUtensorMap tq, td;
+  CUtensorMap tq, td, to;
   cudaError_t e = attn::seq_map(&tq, qkv, B, T, 3 * C);
   if (e != cudaSuccess) return e;
   e = attn::seq_map(&td, datt, B, T, C);
+  if (e != cudaSuccess) return e;
+  e = attn::seq_map(&to, att, B, T, C);
   if (e != cudaSuccess) return e;
   constexpr size_t sm_a = dkdv_smem_bytes(), sm_b = dq_smem_bytes();
   static_assert(sm_a <= 232448 && sm_b <= 232448, "shared memory budget");
@@ -704,10 +727,11 @@ cudaError_t attention_bwd_tc(act_t* dqkv, const float* dsum, const act_t* datt, 
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = items < sms ? items : sms;
+  // dQ first: it forms D = rowsum(dO * O) of its query tiles for dK/dV
+  flash_bwd_dq_tc_kernel<<<grid, kThreadsBwd, sm_b, s>>>(tq, td, to, lse, dsum, dqkv, B, T, C, H,
+                                                         sl2, scale, err);
   flash_bwd_dkdv_tc_kernel<<<grid, kThreadsBwd, sm_a, s>>>(tq, td, lse, dsum, dqkv, B, T, C, H, sl2,
                                                            scale, err);
-  flash_bwd_dq_tc_kernel<<<grid, kThreadsBwd, sm_b, s>>>(tq, td, lse, dsum, dqkv, B, T, C, H, sl2,
-                                                         scale, err);
   note_launch(2);
   return cudaGetLastError();
 }

@@ -107,10 +107,11 @@ cudaError_t attention_fwd_tc(act_t* att, float* lse, const act_t* qkv, int B, in
 cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
                           const act_t* att, const float* lse, int B, int T, int C, int H,
                           int* err, cudaStream_t s);
-// tcgen05 backward (head dim 64; bf16 build); dsum holds D = rowsum(dO * O)
-cudaError_t attention_bwd_tc(act_t* dqkv, const float* dsum, const act_t* datt, const act_t* qkv,
-                             const float* lse, int B, int T, int C, int H, int* err,
-                             cudaStream_t s);
+// tcgen05 backward (head dim 64; bf16 build); it writes D = rowsum(dO * O)
+// (B*H*T floats) to dsum itself, from datt and the forward's output att
+cudaError_t attention_bwd_tc(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
+                             const act_t* att, const float* lse, int B, int T, int C, int H,
+                             int* err, cudaStream_t s);
 
 // ---------------------------------------------------------- classifier --
 // In place over logits [M, Vp]: per row lse over the first V columns,
