@@ -57,8 +57,11 @@ def ref_linear(x, W, b=None):
     return ORC_MP.linear_fwd(x, W, b)
 
 
+# (129, 512, 64): a pair tile whose second CTA holds one live row;
+# (257, 256, 520): one row past a pair tile, N one tile wide, K ragged
 GEMM_SHAPES = [(128, 256, 64), (256, 384, 192), (300, 200, 136), (1000, 768, 768),
-               (64, 2304, 768), (513, 50304 // 8, 768), (16384, 768, 64)]
+               (64, 2304, 768), (513, 50304 // 8, 768), (16384, 768, 64), (129, 512, 64),
+               (257, 256, 520)]
 
 
 @pytest.fixture(params=[1, 0], ids=["pairs", "single"])
@@ -98,7 +101,8 @@ def test_gemm_forward(M, N, K, epi, cta_pairs):
     assert_bf16_close(got, ref)
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 200, 136), (1000, 768, 3072), (256, 3072, 768)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 200, 136), (1000, 768, 3072), (256, 3072, 768),
+                                   (129, 512, 200)])
 @pytest.mark.parametrize("epi", ["store", "dgelu"])
 def test_gemm_dgrad(M, N, K, epi, cta_pairs):
     """out[M, N] = dy[M, K] W[K, N] (W read MN-major, as the weight is stored)."""
