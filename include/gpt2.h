@@ -189,6 +189,15 @@ gpt2_status gpt2_get_params(const gpt2_t* h, float* host);
 gpt2_status gpt2_set_params(gpt2_t* h, const float* host); /* also refreshes the bf16 copy */
 gpt2_status gpt2_get_grads(const gpt2_t* h, float* host);
 
+/* Device pointer to the fp32 gradient buffer itself (gpt2_num_params floats,
+ * the layout of gpt2_tensor_info), owned by the model.  For replicas that
+ * exchange gradients: after every replica's gpt2_backward calls, a sum
+ * all-reduce of this buffer (on the model's stream, or ordered after it)
+ * and then gpt2_grad_norm_clip / gpt2_adamw_step on every replica keep the
+ * replicas' parameters identical.  Valid until gpt2_destroy or
+ * gpt2_bind_memory. */
+gpt2_status gpt2_grads_device(gpt2_t* h, float** dev_ptr);
+
 /* Checkpoint state: params, m, v (each gpt2_num_params floats) and the step
  * counter t.  Any pointer may be NULL to skip that part. Synchronous. */
 gpt2_status gpt2_get_state(const gpt2_t* h, float* params, float* m, float* v, long* t);

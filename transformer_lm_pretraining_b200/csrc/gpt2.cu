@@ -881,6 +881,14 @@ gpt2_status gpt2_get_grads(const gpt2_t* hc, float* host) {
   return GPT2_OK;
 }
 
+gpt2_status gpt2_grads_device(gpt2_t* h, float** dev_ptr) {
+  if (!h || !dev_ptr) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  *dev_ptr = h->grads;
+  return GPT2_OK;
+}
+
 gpt2_status gpt2_get_state(const gpt2_t* hc, float* params, float* m, float* v, long* t) {
   gpt2_t* h = const_cast<gpt2_t*>(hc);
   if (!h) return GPT2_ERR_ARG;

@@ -60,6 +60,7 @@ SIGNATURES = {
     "gpt2_tensor_info": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_i),
                               ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(_sz)]),
     "gpt2_logits": (_i, [_vp, ctypes.POINTER(_vp)]),
+    "gpt2_grads_device": (_i, [_vp, ctypes.POINTER(_fp)]),
     "gpt2_get_losses": (_i, [_vp, _fp, _sz]),
     "gpt2_read_activation": (_i, [_vp, _i, _i, _fp, _sz]),
     "gpt2_last_error": (ctypes.c_char_p, [_vp]),
@@ -246,6 +247,20 @@ class GPT2:
         p = np.ascontiguousarray(p, np.float32)
         assert p.size == self.P
         self._check(self.lib.gpt2_set_params(self.h, _fptr(p)))
+
+    def grads_tensor(self):
+        """The model's fp32 gradient buffer [P] as a torch CUDA tensor (a
+        view, no copy): what replicas all-reduce between backward and clip."""
+        torch = self.torch
+        ptr = _fp()
+        self._check(self.lib.gpt2_grads_device(self.h, ctypes.byref(ptr)))
+        addr = ctypes.cast(ptr, ctypes.c_void_p).value
+
+        class _View:  # CUDA array interface over the library's buffer
+            __cuda_array_interface__ = {"shape": (self.P,), "typestr": "<f4",
+                                        "data": (addr, False), "version": 2}
+
+        return torch.as_tensor(_View(), device="cuda")
 
     def get_grads(self) -> np.ndarray:
         a = np.empty(self.P, np.float32)
