@@ -96,8 +96,9 @@ int gpt2k_classifier(void* stream, void* logits, float* losses, const int* tgt, 
                      int Vp, int write_grad);
 
 /* Device error word of the kernel-level calls (bit value 2: a bad target;
- * 4: a bounded wait in a tensor-core kernel expired); read and cleared.
- * Synchronous. */
+ * 4: a bounded wait in a tensor-core kernel expired), ORed with the private
+ * error word of gpt2k_gemm_wgrad_noalloc on the current device (calls made
+ * with err_dev = NULL); both are read and cleared.  Synchronous. */
 int gpt2k_take_error(void);
 
 /* Size, in floats, of the fixed scratch array behind
@@ -116,22 +117,27 @@ int gpt2k_take_error(void);
  * split-K workspace, nor let the library allocate one.
  *
  * What it does instead: the split-K partial sums go to a file-scope device
- * array of GPT2K_NOALLOC_SCRATCH_FLOATS floats that every GPU holds from the
- * moment it loads the library until the process exits.  The call allocates
- * nothing (no cudaMalloc, cudaFree or allocating library routine).
+ * array of GPT2K_NOALLOC_SCRATCH_FLOATS floats.  The call itself makes no
+ * cudaMalloc, cudaFree or allocating library routine call.
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    with that device current.  CUDA loads modules lazily by default, so
+ *    that lookup is also when the driver places the 16 MiB array on the
+ *    device: the first call needs 16 MiB free.  Make it early -- before the
+ *    caller's allocator has taken the memory -- and outside any stream
+ *    capture.  From then on the array stays on that device until the
+ *    process exits.
  *  - At most max_splits (1..8) K-slices are used; max_splits * M * N must
  *    not exceed GPT2K_NOALLOC_SCRATCH_FLOATS, else GPT2_ERR_ARG is returned
  *    before any work is enqueued.  The result is the same as gpt2k_gemm's
  *    weight-gradient form given a workspace of max_splits * M * N floats.
- *  - The first call on a device looks up the array's device address on that
- *    (current) device; make that first call before any stream capture.
  *  - Every call on a device shares the one array and leaves its last
- *    partial sums in it; each call writes every partial it later reads, and
- *    clears its own error word.  Calls whose work overlaps on the GPU (other
- *    streams, other threads) race on the array: serialise them.
- *  - err_dev (may be NULL) is a device int that receives bit 2 if a bounded
- *    wait inside the GEMM expired; with NULL that report goes to a private
- *    word and is dropped.
+ *    partial sums in it; each call writes every partial it later reads.
+ *    Calls whose work overlaps on the GPU (other streams, other threads)
+ *    race on the array: serialise them.
+ *  - err_dev (may be NULL) is a device int that receives bit value 4 if a
+ *    bounded wait inside the GEMM expired (the output is then incomplete).
+ *    With NULL the bit goes to a private word of the device, which
+ *    accumulates until gpt2k_take_error reads and clears it.
  * Operands and strides as for gpt2k_gemm; asynchronous on `stream`. */
 int gpt2k_gemm_wgrad_noalloc(void* stream, int M, int N, int K, const void* A, long lda,
                              const void* B, long ldb, float alpha, float* out32, long ldo32,

@@ -31,7 +31,11 @@ def _rms(a):
 
 
 def test_noalloc_matches_workspace_gemm_on_two_calls():
-    for M, N, K, seed in [(768, 512, 4096, 1), (256, 768, 2048, 2)]:
+    # the first shape's calls pass an error word of their own; the second
+    # shape's calls pass none, so a bounded-wait expiry would land in the
+    # library's private word, which gpt2k_take_error reads and clears
+    g2.gpt2k_take_error()
+    for M, N, K, seed, own_err in [(768, 512, 4096, 1, True), (256, 768, 2048, 2, False)]:
         rng = np.random.default_rng(seed)
         dy = _bf16_dev(rng.standard_normal((K, M)))
         x = _bf16_dev(rng.standard_normal((K, N)))
@@ -40,14 +44,21 @@ def test_noalloc_matches_workspace_gemm_on_two_calls():
         want = torch.tensor(g0, device="cuda")
         ws = torch.zeros(8 * M * N, dtype=torch.float32, device="cuda")
         g2.gpt2k_gemm("f32_acc", M, N, K, dy, M, 1, x, N, 1, 0.5, out32=want, ldo32=N, split_ws=ws)
-
-        got = torch.tensor(g0, device="cuda")
-        rc = g2.gpt2k_gemm_wgrad_noalloc(M, N, K, dy, M, x, N, 0.5, got, N, max_splits=8)
-        assert rc == 0
         torch.cuda.synchronize()
-        assert g2.gpt2k_take_error() == 0
-        w, g = want.cpu().double().numpy(), got.cpu().double().numpy()
-        assert np.abs(g - w).max() <= 1e-5 * _rms(w) * np.sqrt(K / 64)
+        assert g2.gpt2k_take_error() == 0  # the workspace-taking reference call
+
+        err = torch.zeros(1, dtype=torch.int32, device="cuda") if own_err else None
+        for call in range(2):  # the second call finds the array as the first left it
+            got = torch.tensor(g0, device="cuda")
+            rc = g2.gpt2k_gemm_wgrad_noalloc(M, N, K, dy, M, x, N, 0.5, got, N, max_splits=8,
+                                             err=err)
+            assert rc == 0
+            torch.cuda.synchronize()
+            if own_err:
+                assert int(err.item()) == 0, call
+            assert g2.gpt2k_take_error() == 0, call
+            w, g = want.cpu().double().numpy(), got.cpu().double().numpy()
+            assert np.abs(g - w).max() <= 1e-5 * _rms(w) * np.sqrt(K / 64), call
 
 
 def test_noalloc_refuses_sizes_beyond_its_array():

@@ -109,7 +109,7 @@ int gpt2k_take_error(void) {
   int e = 0;
   if (cudaMemcpy(&e, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GPT2_ERR_CUDA;
   cudaMemset(err, 0, sizeof(int));
-  return e;
+  return e | noalloc_take_error();
 }
 
 }  // extern "C"

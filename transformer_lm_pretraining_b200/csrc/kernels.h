@@ -172,4 +172,8 @@ long launch_count();
 // Error bits in the device error word.
 enum ErrBits { ERR_TOKEN = 1, ERR_TARGET = 2, ERR_TIMEOUT = 4 };
 
+// Error bits left by gpt2k_gemm_wgrad_noalloc calls made without an error
+// word of their own, on the current device; read and cleared (synchronous).
+int noalloc_take_error();
+
 }  // namespace gpt2k

@@ -12,8 +12,11 @@ using namespace gpt2k;
 
 namespace {
 
-// 4 Mi floats = 16 MiB on every GPU that loads this library, held until the
-// process exits; every call of the entry point shares it.
+// 4 Mi floats = 16 MiB on every GPU where the entry point has run, held
+// until the process exits; every call of the entry point shares it.  With
+// lazy module loading (the CUDA default since 12.2) the driver places the
+// array on a device when the first call there looks up its address, so
+// that first call needs 16 MiB of free device memory.
 static __device__ __align__(256) float g_wgrad_scratch[GPT2K_NOALLOC_SCRATCH_FLOATS];
 static __device__ __align__(256) int g_wgrad_err[1];
 
@@ -49,6 +52,28 @@ int device_slots(DeviceSlots* out) {
 
 }  // namespace
 
+namespace gpt2k {
+
+// Error bits that calls made with err_dev = NULL left in the private error
+// word of the current device, read and cleared (synchronous); 0 when the
+// entry point has not been set up on this device.
+int noalloc_take_error() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  int* err = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_slots[dev].ready) return 0;
+    err = g_slots[dev].err;
+  }
+  int e = 0;
+  if (cudaMemcpy(&e, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return 0;
+  cudaMemset(err, 0, sizeof(int));
+  return e;
+}
+
+}  // namespace gpt2k
+
 extern "C" int gpt2k_gemm_wgrad_noalloc(void* stream, int M, int N, int K, const void* A,
                                         long lda, const void* B, long ldb, float alpha,
                                         float* out32, long ldo32, int max_splits, int* err_dev) {
@@ -60,8 +85,9 @@ extern "C" int gpt2k_gemm_wgrad_noalloc(void* stream, int M, int N, int K, const
   const int st = device_slots(&slots);
   if (st != GPT2_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Without err_dev the expiry bit goes to the private word, which keeps
+  // accumulating until gpt2k_take_error reads and clears it.
   int* err = err_dev ? err_dev : slots.err;
-  if (!err_dev && cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return GPT2_ERR_CUDA;
   GemmArgs g{};
   g.M = M; g.N = N; g.K = K;
   g.A = static_cast<const act_t*>(A); g.lda = lda; g.a_mn = 1;
