@@ -134,26 +134,114 @@ def make_batches(wl, n_steps, seed):
     return out
 
 
-def cpu_baseline(wl, sample_T, threads_note=True):
-    """The oracle (OpenMP build, all host cores) on a bounded sample of the
-    workload: one B=1 x sample_T micro-batch forward+backward of the full
-    model plus one AdamW over every parameter; tokens/s = sample_T / time."""
+def metric_name(wl, mode="train"):
+    """The metric string both arms print for a workload (so that the two
+    lines can be compared)."""
+    kind = "evaluation" if mode == "eval" else "training"
+    if wl.name == "gpt2_124m":
+        return f"{kind} tokens/sec and MFU, GPT-2 124M bf16, B=16×T=1024, 1×B200"
+    return f"{kind} tokens/s and MFU, {wl.name} bf16"
+
+
+def _oracle_row_and_opt(wl, T, openmp):
+    """Time the fp32 oracle on one B=1 x T micro-batch forward+backward, and
+    on one clip + AdamW over every parameter.  Returns (t_row, t_opt,
+    threads, num_params)."""
     import oracle
 
     cfg = oracle.Config(wl.L, wl.H, wl.C, wl.V, wl.Vp, wl.Tmax)
-    o = oracle.Oracle(cfg, np.float32, openmp=True)
+    o = oracle.Oracle(cfg, np.float32, openmp=openmp)
     p = o.init(0)
-    tok, tgt = ZipfStream(wl.V, 0).next_batch(1, sample_T)
+    tok, tgt = ZipfStream(wl.V, 0).next_batch(1, T)
     m, v = np.zeros_like(p), np.zeros_like(p)
     t0 = time.perf_counter()
-    _, g, _ = o.forward_backward(p, tok, tgt, 1, sample_T, 1.0)
+    _, g, _ = o.forward_backward(p, tok, tgt, 1, T, 1.0)
+    t1 = time.perf_counter()
     o.clip(g, 1.0)
     o.adamw(p, g, m, v, 1, wl.lr_max)
-    dt = time.perf_counter() - t0
-    return {"value": sample_T / dt, "unit": "tokens/s", "cores": oracle.openmp_threads(),
-            "kind": "oracle",
-            "sample": f"fp32 oracle, {wl.name} model, B=1 x T={sample_T} forward+backward + "
-                      f"clip + one AdamW over all {o.num_params()} params, {dt:.1f} s"}
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1, (oracle.openmp_threads() if openmp else 1), o.num_params()
+
+
+def cpu_baseline(wl, sample_T_1core=64):
+    """The oracle as it stands on the host cores, on a bounded sample of the
+    workload, scaled to one optimizer step of it.
+
+    All cores (the OpenMP build, which parallelises only over independent
+    outputs): one full-length B=1 x T row forward+backward and one clip +
+    AdamW over every parameter; the step is B*n_micro rows + one clip/AdamW.
+    One core (the single-threaded build): a B=1 x sample_T_1core row and the
+    clip/AdamW, the row scaled to full length by its FLOP count (6N + 6LCT
+    per token, N = 12LC^2 + Vpad C)."""
+    rows = wl.B * wl.n_micro
+    t_row, t_opt, threads, P = _oracle_row_and_opt(wl, wl.T, True)
+    step = rows * t_row + t_opt
+    out = {"value": wl.tokens_per_step / step, "unit": "tokens/s", "cores": threads,
+           "kind": "oracle",
+           "sample": f"fp32 oracle (OpenMP, {threads} threads), {wl.name}: one B=1 x T={wl.T} row "
+                     f"forward+backward {t_row:.2f} s and one clip + AdamW over {P} params "
+                     f"{t_opt:.2f} s, step extrapolated as {rows} rows + 1 optimizer update = "
+                     f"{step:.1f} s"}
+    Ts = min(sample_T_1core, wl.T)
+    t_row1, t_opt1, _, _ = _oracle_row_and_opt(wl, Ts, False)
+    n_mm = 12 * wl.L * wl.C ** 2 + wl.Vp * wl.C
+
+    def row_flops(T):
+        return T * (6.0 * n_mm + 6.0 * wl.L * wl.C * T)
+
+    step1 = rows * t_row1 * row_flops(wl.T) / row_flops(Ts) + t_opt1
+    out["value_1core"] = wl.tokens_per_step / step1
+    out["sample_1core"] = (f"single-threaded fp32 oracle: one B=1 x T={Ts} row forward+backward "
+                           f"{t_row1:.2f} s, scaled by FLOP count to a T={wl.T} row, x {rows} rows, "
+                           f"+ clip/AdamW {t_opt1:.2f} s = {step1:.0f} s per step (extrapolated)")
+    return out
+
+
+def family_roofline(wl, fam, peaks, distinct_ids, recompute):
+    """Per kernel family of one optimizer step: device time, algorithmic
+    work and the fraction of the measured peak it reaches.  fam = {family:
+    (ms per step, launches per step, flops per step)} from the profiling
+    pass.  Algorithmic bytes (bf16 activations, fp32 statistics and
+    parameters), per micro-batch of M = B*T tokens unless stated:
+      encoder     M(6C + 8) forward + M 2C + (T + distinct ids) 8C backward
+      ln_fwd      (2L + 1) M (4C + 8)
+      ln_bwd      (2L + 1) M (8C + 8)
+      classifier  M (4 Vpad + 8)
+      colsum      L M 2 (4C + 3C)   (bias gradients of W_fc and W_qkv)
+      recompute   L M 4C 4          (read u, write GELU(u))
+      optimizer   34 bytes per parameter per step (norm: 4; AdamW: 30)
+    gemm and attention are tensor-bound: their algorithmic FLOPs come from
+    the profiling pass (2MNK per GEMM; causal 4 B H T(T+1)/2 hd forward and
+    10 B H T(T+1)/2 hd backward)."""
+    L, C, Vp, T = wl.L, wl.C, wl.Vp, wl.T
+    M = wl.B * wl.T
+    nm = wl.n_micro
+    P = 12 * L * C * C + 13 * L * C + 2 * C + Vp * C + wl.Tmax * C
+    hbm = {
+        "encoder": nm * (M * (6 * C + 8) + M * 2 * C + (T + distinct_ids) * 8 * C),
+        "ln_fwd": nm * (2 * L + 1) * M * (4 * C + 8),
+        "ln_bwd": nm * (2 * L + 1) * M * (8 * C + 8),
+        "classifier": nm * M * (4 * Vp + 8),
+        "colsum": nm * L * M * 2 * (4 * C + 3 * C),
+        "recompute": nm * L * M * 4 * C * 4 if recompute else 0,
+        "optimizer": 34 * P,
+    }
+    out = {}
+    for k, (ms, n, fl) in fam.items():
+        if ms <= 0:
+            continue
+        if k in hbm:
+            ach = hbm[k] / (ms / 1e3) / 1e9
+            out[k] = {"ms": round(ms, 4), "launches": n, "bound": "hbm",
+                      "algorithmic": hbm[k], "unit": "GB/s", "achieved": round(ach, 1),
+                      "peak": peaks["hbm_gbs"], "frac": round(ach / peaks["hbm_gbs"], 3)}
+        else:
+            ach = fl / (ms / 1e3) / 1e12
+            out[k] = {"ms": round(ms, 4), "launches": n, "bound": "tensor",
+                      "algorithmic": fl, "unit": "TFLOP/s", "achieved": round(ach, 1),
+                      "peak": peaks["bf16_tflops_sustained"],
+                      "frac": round(ach / peaks["bf16_tflops_sustained"], 3)}
+    return out
 
 
 def run_reference(args, wl):
@@ -181,7 +269,7 @@ def run_reference(args, wl):
             times.append(time.perf_counter() - t0)
     tot = sum(times)
     value = T * len(times) / tot
-    return {"impl": "reference", "metric": "training tokens/s, GPT-2 step (fwd+bwd+clip+AdamW)",
+    return {"impl": "reference", "metric": metric_name(wl, args.mode),
             "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -303,15 +391,18 @@ def run_ours(args, wl):
 
     peaks = load_peaks()
     fpt = wl.flops_per_token() / (3.0 if evaluate else 1.0)  # the forward is a third
-    mfu = fpt * value / world / SPEC_BF16_DENSE
+    mfu_spec = fpt * value / world / SPEC_BF16_DENSE
+    peak_mfu = peaks["bf16_tflops"] * 1e12 if peaks["source"] == "measured" else SPEC_BF16_DENSE
+    mfu = fpt * value / world / peak_mfu
     gemm_ms, gemm_n, gemm_fl = prof["gemm"]
     achieved = gemm_fl / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
     fam_ms = {k: v[0] / n_prof for k, v in prof.items()}
+    distinct = float(np.mean([len(np.unique(t)) for st in host[args.warmup:] for t, _ in st]))
+    fam_roof = family_roofline(wl, {k: (v[0] / n_prof, v[1] / n_prof, v[2] / n_prof)
+                                    for k, v in prof.items()}, peaks, distinct, args.recompute)
     fam_total = sum(fam_ms.values())
     out = {
-        "metric": ("evaluation" if evaluate else "training")
-        + (" tokens/s and MFU, GPT-2 124M bf16, B=16xT=1024, 1xB200" if wl.name == "gpt2_124m"
-           else f" tokens/s and MFU, {wl.name} bf16"),
+        "metric": metric_name(wl, args.mode),
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak",
@@ -325,10 +416,13 @@ def run_ours(args, wl):
                    "l2": "no explicit flush: every step streams ~10 GB of activations, logits and "
                          "optimizer state through HBM, far above the 126 MB L2"},
         "mfu": mfu,
+        "mfu_spec": mfu_spec,
         "mfu_basis": f"{fpt / 1e6:.2f} MFLOP/token ({'2N + 2LCT' if evaluate else '6N + 6LCT'}, "
-                     f"N = 12LC^2 + Vpad C) over "
-                     f"2.25 PFLOP/s dense bf16 spec; {fpt * value / world / (peaks['bf16_tflops'] * 1e12):.3f} "
-                     f"of the {peaks['source']} cuBLAS bf16 peak",
+                     f"N = 12LC^2 + Vpad C); mfu over "
+                     + (f"the measured dense bf16 burst peak {peaks['bf16_tflops']:.0f} TFLOP/s"
+                        if peaks["source"] == "measured" else "the 2.25 PFLOP/s dense bf16 spec "
+                        "(no measured peak on this box)")
+                     + "; mfu_spec over the 2.25 PFLOP/s dense bf16 spec",
         "gpu_launches": int(launches),
         "roofline": {"kernel": "gemm_tc_kernel (all projection GEMM launches of a step)",
                      "bound": "tensor", "achieved": achieved,
@@ -344,6 +438,10 @@ def run_ours(args, wl):
         "kernel_breakdown_ms_per_step": {k: round(v, 4) for k, v in fam_ms.items()},
         "kernel_breakdown_share": {k: round(v / fam_total, 4) for k, v in fam_ms.items()}
         if fam_total > 0 else None,
+        "kernel_roofline": fam_roof,
+        "kernel_roofline_basis": "device time per family from CUDA events around its launches "
+                                 "(second pass); HBM families against the measured copy bandwidth, "
+                                 "tensor families against the sustained bf16 peak",
         "clocks": clk,
         "e2e": e2e,
     }
@@ -429,7 +527,8 @@ def main():
     ap.add_argument("--workload", default="gpt2_124m", choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-T", type=int, default=256)
+    ap.add_argument("--cpu-sample-T", type=int, default=64,
+                    help="row length of the single-threaded oracle sample")
     ap.add_argument("--mode", default="train", choices=["train", "eval", "generate"],
                     help="train: the training step; eval: forward-only evaluation (loss); "
                          "generate: autoregressive generation with the key/value cache")
