@@ -289,7 +289,7 @@ def run_ours(args, wl):
     from transformer_lm_pretraining_b200.replicas import Replicas
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    reps = Replicas("nccl", timeout_s=120)
+    reps = Replicas("nccl", timeout_s=120, group=args.mode in ("dp", "zero1"))
     world, rank, local = reps.world, reps.rank, reps.local_rank
     barrier, max_over_ranks = reps.barrier, reps.max
 
@@ -308,10 +308,29 @@ def run_ours(args, wl):
     def lr(k):
         return g2.gpt2_lr(k, wl.lr_max, 0.1 * wl.lr_max, wl.warmup, wl.max_steps)
 
+    dp_step = None
+    if args.mode in ("dp", "zero1"):
+        # data-parallel step: each rank its own micro-batches, gradients
+        # summed over NCCL (per layer, overlapped with the backward) or
+        # reduce-scattered with a sharded AdamW and an all-gather (ZeRO-1)
+        import torch.distributed as dist
+
+        from transformer_lm_pretraining_b200.data_parallel import DataParallelStep
+
+        dp_step = DataParallelStep(
+            model, world, rank, mode="zero1" if args.mode == "zero1" else "allreduce",
+            overlap=args.mode == "dp", sync=False,
+            all_reduce=lambda t: dist.all_reduce(t),
+            reduce_scatter=lambda out, t: dist.reduce_scatter_tensor(out, t),
+            all_gather=lambda out, shard: dist.all_gather_into_tensor(out, shard))
+
     def step(k, batches):
         if evaluate:  # forward-only evaluation: loss of every micro-batch
             for tok, tgt in batches:
                 model.evaluate(tok, tgt, sync_loss=False)
+            return
+        if dp_step is not None:
+            dp_step(batches, lr(k), 1.0, 0.9, 0.95, 1e-8, 0.1)
             return
         model.zero_grad()
         for tok, tgt in batches:
@@ -323,6 +342,30 @@ def run_ours(args, wl):
     for k in range(args.warmup):
         step(k, dev[k])
     torch.cuda.synchronize()
+
+    # The training step as one CUDA graph (gpt2_step_graph_capture): its token
+    # buffers receive each step's micro-batches, then the graph is replayed;
+    # the learning rate follows the schedule from the device step counter.
+    use_graph = args.graph and args.mode == "train"
+    graph_kernels = None
+    if use_graph:
+        n_tok = wl.n_micro * wl.B * wl.T
+        stok = torch.empty(n_tok, dtype=torch.int32, device="cuda")
+        stgt = torch.empty(n_tok, dtype=torch.int32, device="cuda")
+        graph_kernels = model.capture_step(stok, stgt, wl.B, wl.T, wl.n_micro, 1.0, wl.lr_max,
+                                           0.1 * wl.lr_max, wl.warmup, wl.max_steps)
+
+        def load_tokens(batches):
+            for j, (t, y) in enumerate(batches):
+                stok[j * wl.B * wl.T:(j + 1) * wl.B * wl.T].copy_(t.view(-1), non_blocking=True)
+                stgt[j * wl.B * wl.T:(j + 1) * wl.B * wl.T].copy_(y.view(-1), non_blocking=True)
+
+        def timed_step(k, batches):
+            load_tokens(batches)
+            model.launch_step()
+    else:
+        timed_step = step
+    torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
 
@@ -332,10 +375,10 @@ def run_ours(args, wl):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for k in range(args.warmup, n_steps):
-        step(k, dev[k])
+        timed_step(k, dev[k])
     ev1.record(stream)
     torch.cuda.synchronize()
-    launches = (g2.gpt2_launch_count() - n0) // args.steps
+    launches = graph_kernels if use_graph else (g2.gpt2_launch_count() - n0) // args.steps
     clk = clocks.stop()
     barrier()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1))
@@ -369,6 +412,19 @@ def run_ours(args, wl):
         e0.record(stream)
         for k in range(n_e2e):
             hb = pinned[(args.warmup + k) % n_steps]
+            if use_graph:  # pinned host tokens into the graph's buffers, replay, loss back
+                load_tokens(hb)
+                model.launch_step()
+                model.read_loss()
+                continue
+            if dp_step is not None:
+                for j, (t, y) in enumerate(hb):
+                    bufs[j][0].copy_(t, non_blocking=True)
+                    bufs[j][1].copy_(y, non_blocking=True)
+                dp_step([(bufs[j][0], bufs[j][1]) for j in range(wl.n_micro)],
+                        lr(args.warmup + k), 1.0, 0.9, 0.95, 1e-8, 0.1)
+                model.read_loss()
+                continue
             if not evaluate:
                 model.zero_grad()
             for j, (t, y) in enumerate(hb):
@@ -411,8 +467,12 @@ def run_ours(args, wl):
         "config": {"workload": wl.name, "global_batch": wl.B * wl.n_micro * world, "seq_len": wl.T,
                    "micro_batch": wl.B, "n_micro": wl.n_micro,
                    "tokens_per_step": wl.tokens_per_step * world,
-                   "parallelism": "replicas" if world > 1 else "single-gpu",
+                   "parallelism": ({"dp": f"dp{world} (per-layer all-reduce overlapped with "
+                                          "the backward)",
+                                    "zero1": f"dp{world} ZeRO-1"}.get(args.mode)
+                                   or ("replicas" if world > 1 else "single-gpu")),
                    "mode": args.mode, "recompute": args.recompute,
+                   "cuda_graph": bool(use_graph),
                    "l2": "no explicit flush: every step streams ~10 GB of activations, logits and "
                          "optimizer state through HBM, far above the 126 MB L2"},
         "mfu": mfu,
@@ -529,9 +589,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-T", type=int, default=64,
                     help="row length of the single-threaded oracle sample")
-    ap.add_argument("--mode", default="train", choices=["train", "eval", "generate"],
+    ap.add_argument("--mode", default="train", choices=["train", "eval", "generate", "dp", "zero1"],
                     help="train: the training step; eval: forward-only evaluation (loss); "
-                         "generate: autoregressive generation with the key/value cache")
+                         "generate: autoregressive generation with the key/value cache; "
+                         "dp: data-parallel step over the ranks (NCCL all-reduce per layer, "
+                         "overlapped with the backward); zero1: data-parallel with the "
+                         "optimizer sharded (reduce-scatter, AdamW on a shard, all-gather)")
+    ap.add_argument("--graph", type=int, default=1, choices=[0, 1],
+                    help="1: time the training step replayed as one captured CUDA graph; "
+                         "0: the eager calls")
     ap.add_argument("--recompute", type=int, default=0, choices=[0, 1],
                     help="1: recompute GELU in the backward instead of keeping it")
     args = ap.parse_args()

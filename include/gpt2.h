@@ -173,9 +173,37 @@ gpt2_status gpt2_grad_norm_clip(gpt2_t* h, float max_norm, float* norm_host);
  * p -= lr (mhat / (sqrt(vhat) + eps) + wd p) with wd applied to the 2-D
  * tensors wte, wpe, W_qkv, W_o, W_fc, W_p only), using the clip scale of the
  * last gpt2_grad_norm_clip (1 if none since the last step).  Refreshes the
- * bf16 weight copy.  Gradients are left as they are. */
+ * bf16 weight copy.  Gradients are left as they are.  The step counter t
+ * lives on the device (gpt2_get_state reads it). */
 gpt2_status gpt2_adamw_step(gpt2_t* h, float lr, float beta1, float beta2, float eps,
                             float weight_decay);
+
+/* The same step with lr = gpt2_lr(t - 1, max_lr, min_lr, warmup, max_steps)
+ * evaluated on the device from its own step counter (after t += 1), so that
+ * a captured step (gpt2_step_graph_capture) follows the schedule when it is
+ * replayed.  warmup >= 1. */
+gpt2_status gpt2_adamw_step_scheduled(gpt2_t* h, double max_lr, double min_lr, long warmup,
+                                      long max_steps, float beta1, float beta2, float eps,
+                                      float weight_decay);
+
+/* One whole optimizer step captured as a CUDA graph owned by the handle and
+ * replayed with gpt2_step_graph_launch, in place of the ~370 separate
+ * launches of the eager calls: gpt2_zero_grad; for i < n_micro,
+ * gpt2_forward(tok_dev + i B T, tgt_dev + i B T, B, T) and
+ * gpt2_backward(1 / n_micro); gpt2_grad_norm_clip(max_norm);
+ * gpt2_adamw_step_scheduled(...).  tok_dev and tgt_dev (n_micro B T ids
+ * each) are read at every replay: write the next step's tokens there before
+ * launching it.  Capturing enqueues no work.  Requirements: a stream set with
+ * gpt2_set_stream (not the legacy default stream), profiling off, and one
+ * eager step of the same B and T run before (first-use set-up of the kernels
+ * is not captured).  A new capture replaces the previous graph.
+ * gpt2_step_graph_kernels gives the number of kernels one replay runs. */
+gpt2_status gpt2_step_graph_capture(gpt2_t* h, const int32_t* tok_dev, const int32_t* tgt_dev,
+                                    int B, int T, int n_micro, float max_norm, double max_lr,
+                                    double min_lr, long warmup, long max_steps, float beta1,
+                                    float beta2, float eps, float weight_decay);
+gpt2_status gpt2_step_graph_launch(gpt2_t* h);
+long gpt2_step_graph_kernels(const gpt2_t* h);
 
 /* Host-side schedule: lr = max_lr (step+1)/warmup for step < warmup, then a
  * cosine from max_lr at step = warmup to min_lr at step = max_steps, and
@@ -197,6 +225,43 @@ gpt2_status gpt2_get_grads(const gpt2_t* h, float* host);
  * replicas' parameters identical.  Valid until gpt2_destroy or
  * gpt2_bind_memory. */
 gpt2_status gpt2_grads_device(gpt2_t* h, float** dev_ptr);
+
+/* Data-parallel building blocks (condensed GPT-2 page, section 3: each GPU
+ * runs its own micro-batches and the gradients are averaged before the
+ * update; the llm.c page's ZeRO-1 option shards the optimizer state).
+ *
+ * gpt2_padded_params: length of the device buffers behind
+ * gpt2_grads_device / gpt2_params_device, gpt2_num_params rounded up to a
+ * multiple of 2048 with zeros, so that R ranks (R a power of two up to 2048)
+ * can take equal contiguous shards of them.
+ * gpt2_grad_sumsq: sum of the squared gradient elements [begin, end) (a
+ * shard; begin a multiple of 4, end <= gpt2_padded_params), as a double at
+ * sumsq_dev (device, 8-byte aligned), in a fixed-order two-stage reduction.
+ * gpt2_clip_from_sumsq: the global norm n = sqrt(*sumsq_dev) (e.g. the sum of
+ * every rank's shard sums) and the clip scale of gpt2_grad_norm_clip from it;
+ * norm_host as there.
+ * gpt2_adamw_step_range: gpt2_adamw_step on the parameters [begin, end) only
+ * (begin and end - begin multiples of 4, unless end is the number of
+ * parameters; also advances the step counter), refreshing the bf16 copy of
+ * that range only.
+ * gpt2_params_device: device pointer to the fp32 parameters (padded length),
+ * e.g. for an all-gather of every rank's updated shard.
+ * gpt2_refresh_weights: rewrite the bf16 weight copy the GEMMs read from the
+ * fp32 parameters (after such an all-gather).
+ * gpt2_set_backward_events: n = L + 1 cudaEvent_t handles (or n = 0 to stop)
+ * that gpt2_backward records on its stream: event l once layer l's gradients
+ * are final (every per-layer tensor slice of layer l), event L after the last
+ * kernel (wte, wpe, lnf); a caller can start the gradient exchange of each
+ * layer on another stream while the backward of the layers below runs. */
+size_t gpt2_padded_params(const gpt2_t* h);
+gpt2_status gpt2_grad_sumsq(gpt2_t* h, size_t begin, size_t end, double* sumsq_dev);
+gpt2_status gpt2_clip_from_sumsq(gpt2_t* h, const double* sumsq_dev, float max_norm,
+                                 float* norm_host);
+gpt2_status gpt2_adamw_step_range(gpt2_t* h, float lr, float beta1, float beta2, float eps,
+                                  float weight_decay, size_t begin, size_t end);
+gpt2_status gpt2_params_device(gpt2_t* h, float** dev_ptr);
+gpt2_status gpt2_refresh_weights(gpt2_t* h);
+gpt2_status gpt2_set_backward_events(gpt2_t* h, void* const* events, int n);
 
 /* Checkpoint state: params, m, v (each gpt2_num_params floats) and the step
  * counter t.  Any pointer may be NULL to skip that part. Synchronous. */

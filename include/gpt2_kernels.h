@@ -45,6 +45,18 @@ int gpt2k_gemm(void* stream, int epi, int M, int N, int K, const void* A, long l
                long ldo32, const float* bias, const void* resid, long ldr, void* aux, long ldaux,
                float* split_ws, size_t split_ws_floats);
 
+/* Test of the bounded waits (no counterpart on the pages): the forward
+ * product out[M, N] = A[M, K] B[N, K]^T (store epilogue, row-major, ld = K
+ * and N) with CTA 0's TMA producer skipping the load of k-block `kblock` of
+ * its first tile, so that the MMA issuer's wait for it runs out after the
+ * kernels' wait limit (about 2 s).  The kernel then takes its abort path:
+ * the device error word of the kernel-level calls receives bit value 4
+ * (read it with gpt2k_take_error), every role leaves its loop, the copies in
+ * flight land, TMEM is freed and the kernel returns; `out` holds garbage.
+ * The context stays usable.  Never part of the training step. */
+int gpt2k_gemm_expiry_test(void* stream, int M, int N, int K, const void* A, const void* B,
+                           void* out, int kblock);
+
 /* Whether gpt2k_gemm (and the model's products) run the products with
  * N >= 256 and M > 128 (other than the GELU epilogues, whose pace their
  * epilogue sets) as 256 x 256 tiles over pairs of CTAs on
@@ -62,7 +74,11 @@ int gpt2k_attention_fwd(void* stream, void* att, float* lse, const void* qkv, in
                         int H);
 
 /* Its backward: dqkv [B*T, 3C] (overwritten) from datt [B*T, C], the
- * forward's qkv, att and lse; dsum is fp32 scratch of B*H*T floats. */
+ * forward's qkv, att and lse; dsum is 16-byte aligned fp32 scratch of
+ * gpt2k_attention_bwd_scratch(B, T, H) floats (per-row softmax statistics:
+ * D = rowsum(datt * att) and, for head dim 64, the log-sum-exp beside it,
+ * over T rounded up to whole 128-row tiles). */
+size_t gpt2k_attention_bwd_scratch(int B, int T, int H);
 int gpt2k_attention_bwd(void* stream, void* dqkv, float* dsum, const void* datt, const void* qkv,
                         const void* att, const float* lse, int B, int T, int C, int H);
 

@@ -32,17 +32,24 @@ def _batches(step):
 
 
 class OracleReplica:
-    """The oracle behind the model interface the data-parallel step uses."""
+    """The oracle behind the model interface the data-parallel step uses.
+    Its flat buffers carry the library's zero padding to a multiple of 2048
+    (the ZeRO-1 shards split the padded length)."""
 
     def __init__(self):
         sys.path.insert(0, ROOT)
         from oracle import Config, Oracle
 
         self.o = Oracle(Config(*CFG))
-        self.p = self.o.init(0)
-        self.g = np.zeros_like(self.p)
-        self.m, self.v = np.zeros_like(self.p), np.zeros_like(self.p)
+        P = self.o.num_params()
+        self.padded_params = (P + 2047) // 2048 * 2048
+        self._p = np.zeros(self.padded_params)
+        self._p[:P] = self.o.init(0)
+        self._g = np.zeros(self.padded_params)
+        self.p, self.g = self._p[:P], self._g[:P]
+        self.m, self.v = np.zeros(P), np.zeros(P)
         self.t = 0
+        self.clip_scale = 1.0
         self._batch = None
 
     def zero_grad(self):
@@ -55,8 +62,32 @@ class OracleReplica:
         tok, tgt = self._batch
         self.o.forward_backward(self.p, tok, tgt, B, T, scale, grads=self.g)
 
-    def grads_tensor(self):
-        return torch.from_numpy(self.g)  # shares memory: the all-reduce writes self.g
+    def grads_tensor(self, padded=False):
+        return torch.from_numpy(self._g if padded else self.g)  # shares memory with the buffer
+
+    def params_tensor(self, padded=True):
+        return torch.from_numpy(self._p if padded else self.p)
+
+    def grad_sumsq(self, begin, end, out):
+        out[0] = float(np.sum(self._g[begin:end] ** 2))
+
+    def clip_from_sumsq(self, sumsq, max_norm):
+        n = float(np.sqrt(float(sumsq[0])))
+        self.clip_scale = max_norm / (n + 1e-6) if n > max_norm else 1.0
+        return n
+
+    def adamw_step_range(self, lr, b1, b2, eps, wd, begin, end):
+        # AdamW is elementwise: run it on copies and keep this range only
+        self.t += 1
+        p, g = self.p.copy(), self.g * self.clip_scale
+        m, v = self.m.copy(), self.v.copy()
+        self.o.adamw(p, g, m, v, self.t, lr, b1, b2, eps, wd)
+        end = min(end, self.p.size)
+        self.p[begin:end], self.m[begin:end], self.v[begin:end] = p[begin:end], m[begin:end], v[begin:end]
+        self.clip_scale = 1.0
+
+    def refresh_weights(self):
+        pass
 
     def grad_norm_clip(self, max_norm):
         return self.o.clip(self.g, max_norm)
@@ -72,7 +103,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, mode="allreduce"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
                       RANK=str(rank), LOCAL_RANK=str(rank))
     sys.path.insert(0, ROOT)
@@ -82,7 +113,21 @@ def _worker(rank, world, port, q):
 
     dist.init_process_group("gloo", timeout=__import__("datetime").timedelta(seconds=60))
     model = OracleReplica()
-    step = DataParallelStep(model, world)
+    if mode == "zero1":
+        # gloo has no reduce-scatter: the in-place shard of an all-reduce is
+        # the same sum; the all-gather goes through a list of shards
+        def reduce_scatter(out, t):
+            dist.all_reduce(t)
+
+        def all_gather(out, shard):
+            parts = [torch.empty_like(shard) for _ in range(world)]
+            dist.all_gather(parts, shard.clone())
+            out.copy_(torch.cat(parts))
+
+        step = DataParallelStep(model, world, rank, mode="zero1", reduce_scatter=reduce_scatter,
+                                all_gather=all_gather)
+    else:
+        step = DataParallelStep(model, world)
     norms = []
     for s in range(STEPS):
         mine = _batches(s)[rank::world]  # this rank's micro-batches
@@ -92,11 +137,12 @@ def _worker(rank, world, port, q):
     dist.destroy_process_group()
 
 
-def test_two_rank_data_parallel_equals_full_batch_step():
+@pytest.mark.parametrize("mode", ["allreduce", "zero1"])
+def test_two_rank_data_parallel_equals_full_batch_step(mode):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q, mode)) for r in range(2)]
     for p in procs:
         p.start()
     out = []

@@ -31,7 +31,13 @@ def _port():
         return s.getsockname()[1]
 
 
-def test_grads_buffer_and_nccl_step_match_the_plain_step():
+@pytest.mark.parametrize("mode,overlap", [("allreduce", False), ("allreduce", True),
+                                          ("zero1", False)])
+def test_grads_buffer_and_nccl_step_match_the_plain_step(mode, overlap):
+    """allreduce: one NCCL sum of the whole buffer, or (overlap) one per
+    layer's gradient ranges on a second stream, each started by the event the
+    backward records after that layer; zero1: reduce-scatter, shard norm,
+    AdamW on the shard, all-gather of the parameters, bf16 refresh."""
     import torch.distributed as dist
 
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_port()))
@@ -61,12 +67,21 @@ def test_grads_buffer_and_nccl_step_match_the_plain_step():
         assert np.array_equal(g_view, plain.get_grads())  # the view is the buffer
         n_plain = plain.grad_norm_clip(1.0)
         plain.adamw_step(1e-3, 0.9, 0.95, 1e-8, 0.1)
-        # the data-parallel step with the NCCL sum forced on
-        dp = DataParallelStep(models[1], 1, all_reduce=lambda t: dist.all_reduce(t))
+        # the data-parallel step with the NCCL collectives forced on
+        dp = DataParallelStep(
+            models[1], 1, 0, mode=mode, overlap=overlap,
+            all_reduce=lambda t: dist.all_reduce(t),
+            reduce_scatter=lambda out, t: dist.reduce_scatter_tensor(out, t),
+            all_gather=lambda out, shard: dist.all_gather_into_tensor(out, shard))
         n_dp = dp(batches, 1e-3)
         torch.cuda.synchronize()
-        assert n_dp == n_plain
-        assert np.array_equal(models[1].get_params(), plain.get_params())
+        dp.close()
+        if mode == "zero1":  # the norm from the shard's sum of squares (another summation order)
+            assert abs(n_dp - n_plain) <= 1e-6 * n_plain
+            assert np.abs(models[1].get_params() - plain.get_params()).max() <= 1e-6
+        else:
+            assert n_dp == n_plain
+            assert np.array_equal(models[1].get_params(), plain.get_params())
         for m in models:
             m.close()
     finally:

@@ -246,7 +246,7 @@ def test_attention_forward_backward(B, T, C, H):
     # backward with the GPU's own (bf16) forward output, as in training
     ref_d = o.attention_bwd(qkv, datt, B, T)
     dqkv = torch.zeros((B * T, 3 * C), dtype=torch.bfloat16, device="cuda")
-    dsum = torch.zeros(B * H * T, dtype=torch.float32, device="cuda")
+    dsum = torch.zeros(g2.gpt2k_attention_bwd_scratch(B, T, H), dtype=torch.float32, device="cuda")
     g2.gpt2k_attention_bwd(dqkv, dsum, dev(datt), q, att, lse, B, T, C, H)
     torch.cuda.synchronize()
     got = host(dqkv)
@@ -293,7 +293,29 @@ def test_attention_backward_is_deterministic():
     outs = []
     for _ in range(2):
         dq = torch.zeros((B * T, 3 * C), dtype=torch.bfloat16, device="cuda")
-        ds = torch.zeros(B * H * T, dtype=torch.float32, device="cuda")
+        ds = torch.zeros(g2.gpt2k_attention_bwd_scratch(B, T, H), dtype=torch.float32, device="cuda")
         g2.gpt2k_attention_bwd(dq, ds, d, q, att, lse, B, T, C, H)
         outs.append(dq.view(torch.int16).cpu().numpy())
     assert np.array_equal(outs[0], outs[1])
+
+
+def test_bounded_wait_expiry_reports_and_recovers():
+    """The bounded waits' abort path, made to run: a GEMM whose TMA producer
+    (CTA 0) skips one k-block, so that the MMA issuer's wait for it runs out
+    (about 2 s).  The kernel reports ERR_TIMEOUT (bit value 4) in the error
+    word, every role leaves, TMEM is freed and the launch completes; the
+    next product on the same context is correct and reports nothing."""
+    M, N, K = 256, 128, 512  # single-CTA 128 x 128 tiles: a few CTAs, one withholds
+    rng = np.random.default_rng(5)
+    x = bf16(rng.standard_normal((M, K)))
+    w = bf16(rng.standard_normal((N, K)) * 0.05)
+    out = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    g2.gpt2k_take_error()  # start from a clear error word
+    assert g2.gpt2k_gemm_expiry_test(M, N, K, dev(x), dev(w), out, kblock=0) == 0
+    torch.cuda.synchronize()  # the launch completes: no hang
+    assert g2.gpt2k_take_error() & 4
+    out2 = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    g2.gpt2k_gemm("store", M, N, K, dev(x), K, 0, dev(w), K, 0, 1.0, out=out2, ldo=N)
+    torch.cuda.synchronize()
+    assert g2.gpt2k_take_error() == 0
+    assert_bf16_close(host(out2), ref_linear(x, w))

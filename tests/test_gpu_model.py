@@ -394,3 +394,53 @@ def test_recompute_is_bit_identical(precision):
     elt = 4 if precision == "fp32" else 2
     saved = (cfg.L - 1) * B * T * 4 * cfg.C * elt
     assert saved - 1024 <= w0 - w1 <= saved + 1024
+
+
+def test_captured_step_equals_eager_steps():
+    """The step captured as one CUDA graph (gpt2_step_graph_capture: zero
+    grad, two micro-batches at loss scale 1/2, clip, AdamW with the schedule
+    on the device) replays bit-identically to the same eager calls with the
+    host's gpt2_lr, through the warmup and into the cosine phase."""
+    cfg = Config(2, 2, 128, 1000, 1024, 128)
+    B, T, n_micro = 2, 128, 2
+    sched = (1e-3, 1e-4, 3, 10)  # steps 0-2 warm up, step 3 starts the cosine
+    s = ZipfStream(cfg.V, 0)
+    steps = [[s.next_batch(B, T) for _ in range(n_micro)] for _ in range(4)]
+    stream = torch.cuda.Stream()
+
+    def eager(m, k):
+        m.zero_grad()
+        for tok, tgt in steps[k]:
+            t, y = tok_tensors(tok, tgt)
+            m.forward(t, y, sync_loss=False)
+            m.backward(1.0 / n_micro)
+        m.grad_norm_clip(1.0, sync=False)
+        m.adamw_step(g2.gpt2_lr(k, *sched), 0.9, 0.95, 1e-8, 0.1)
+        return m.read_loss()
+
+    with torch.cuda.stream(stream):
+        a = g2.GPT2(*cfg.args, seed=7, precision="bf16", B=B, T=T)
+        a.set_stream(stream)
+        want = [eager(a, k) for k in range(4)]
+        pa, ma, va, ta = a.get_state()
+        a.close()
+
+        b = g2.GPT2(*cfg.args, seed=7, precision="bf16", B=B, T=T)
+        b.set_stream(stream)
+        got = [eager(b, 0)]  # one eager step first: kernels set up outside the capture
+        stok = torch.empty(n_micro * B * T, dtype=torch.int32, device="cuda")
+        stgt = torch.empty(n_micro * B * T, dtype=torch.int32, device="cuda")
+        kernels = b.capture_step(stok, stgt, B, T, n_micro, 1.0, *sched)
+        assert kernels > 10
+        for k in range(1, 4):
+            for j, (tok, tgt) in enumerate(steps[k]):
+                t, y = tok_tensors(tok, tgt)
+                stok[j * B * T:(j + 1) * B * T].copy_(t.view(-1))
+                stgt[j * B * T:(j + 1) * B * T].copy_(y.view(-1))
+            b.launch_step()
+            got.append(b.read_loss())
+        pb, mb, vb, tb = b.get_state()
+        b.close()
+    assert got == want
+    assert ta == tb == 4
+    assert np.array_equal(pa, pb) and np.array_equal(ma, mb) and np.array_equal(va, vb)

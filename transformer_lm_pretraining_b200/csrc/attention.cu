@@ -647,6 +647,15 @@ cudaError_t attention_fwd(act_t* att, float* lse, const act_t* qkv, int B, int T
 #endif
 }
 
+size_t attention_bwd_scratch_floats(int B, int T, int H) {
+  size_t n = (size_t)B * H * T;  // D = rowsum(dO * O) of every row
+#if GPT2_ACT_BF16
+  const size_t tc = attention_bwd_tc_scratch_floats(B, T, H);
+  if (tc > n) n = tc;
+#endif
+  return n;
+}
+
 cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
                           const act_t* att, const float* lse, int B, int T, int C, int H,
                           int* err, cudaStream_t s) {

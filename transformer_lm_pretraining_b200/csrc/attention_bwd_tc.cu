@@ -7,27 +7,31 @@
 //
 // Two persistent kernels, one CTA per SM walking a static snake order over
 // work items (heaviest first), 10 warps each (TMA, MMA, 8 compute warps,
-// two threads per tile row):
+// two threads per tile row).  In both, the second product of each step
+// takes its A operand (P^T and dS^T, or dS) from TMEM, where the compute
+// warps write it as packed bf16, so shared memory only feeds the tensor core
+// the operands that TMA brings in:
+//   dQ:    item = (batch, head, query tile i); streams the key tiles j <= i:
+//          S = Q K^T and dP = dO V^T into TMEM, dS into one of two TMEM
+//          buffers, dQ += dS K in one of two TMEM accumulators (K read
+//          MN-major).  It runs first: it also forms D = rowsum(dO * O) of
+//          its rows from the dO and O tiles it loads, and stores, per query
+//          row, the pair (L log2(e), D) for the dK/dV kernel in a layout
+//          padded to whole 128-row tiles (rows past T get L = +inf, D = 0,
+//          which makes their P exactly 0 there).
 //   dK/dV: item = (batch, head, key tile j); streams the query tiles i >= j
 //          in 64-query halves (sub-tiles).  The tensor core computes
 //          S^T = K Q^T and dP^T = V dO^T of a sub-tile into one of two TMEM
-//          score buffers; the compute warps turn them into P^T and dS^T
-//          (bf16, swizzled shared-memory tiles, also double-buffered); the
-//          tensor core then accumulates dV += P^T dO and dK += dS^T Q in
-//          TMEM (dO and Q read MN-major straight from their tiles).  K and V
-//          are double-buffered across items.
-//   dQ:    item = (batch, head, query tile i); streams the key tiles j <= i:
-//          S = Q K^T and dP = dO V^T into TMEM, dS into shared memory,
-//          dQ += dS K in TMEM (K read MN-major).  It runs first and also
-//          forms D = rowsum(dO * O) of its rows from the dO and O tiles it
-//          loads, storing it for the dK/dV kernel.
-// The compute warps hand the score buffers back to the tensor core as soon
-// as they have read them, so the next scores are computed while the current
-// ones are finished; the gradient accumulators are double-buffered in TMEM,
-// so an item's result is written while the next item runs.  Compute warps
-// wait per warp (no block-wide barrier in the loop), and the causal mask is
-// applied only on the diagonal tile and the one holding the end of the
-// sequence.  Every wait is bounded (error word ERR_TIMEOUT).
+//          score buffers; the compute warps turn them into P^T and dS^T in
+//          one of two TMEM operand buffers; the tensor core then accumulates
+//          dV += P^T dO and dK += dS^T Q in TMEM (dO and Q read MN-major
+//          straight from their tiles).  The (L, D) pairs of each query tile
+//          arrive by a bulk copy next to its Q and dO tiles.
+// Each compute thread loads its part of the scores from TMEM in one round
+// trip and hands the buffer straight back, so the tensor core computes the
+// next scores while the current ones are exponentiated.  The causal mask is
+// applied only on the diagonal tile.  Every wait is bounded (error word
+// ERR_TIMEOUT).
 
 #include <type_traits>
 
@@ -45,9 +49,9 @@ using attn::kTile;
 constexpr int kCT = attn::kComputeThreads;
 constexpr int kThreadsBwd = 64 + kCT;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCol = 2 * kTile;  // accumulators after the two score buffers
 constexpr int kAux = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kNegInf = 0xff800000u;
 
 __device__ __forceinline__ bool warp_and(bool p) { return __all_sync(0xffffffffu, p); }
 
@@ -60,6 +64,16 @@ __device__ __forceinline__ void tmem_alloc(uint32_t* slot) {
 __device__ __forceinline__ void tmem_dealloc(uint32_t base) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base),
                "r"(kTmemCols));
+}
+
+// 32 lanes x 16 consecutive 32-bit columns from registers into TMEM.
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
 }
 
 // Bounded wait for copies issued to `bar` (latest fill parity `par`).
@@ -77,52 +91,49 @@ __device__ __forceinline__ int snake_item(int k, int count) {
 }
 
 // ------------------------------------------------------------------ dK/dV --
-// The query tiles are processed in 64-query halves ("sub-tiles"), so that the
-// score products of two sub-tiles fit in TMEM next to the two accumulator
-// pairs: while the compute warps turn one sub-tile's S^T and dP^T into P^T
-// and dS^T, the tensor core already holds (or is computing) the next
-// sub-tile's scores and runs the previous sub-tile's dV and dK products.
-// TMEM columns: [0,128) and [128,256) score buffers (S^T 64 | dP^T 64),
-// [256,512) two accumulator pairs (dV 64 | dK 64).
-constexpr int kQStages = 2;
+// TMEM columns: [0, 256) two score buffers (S^T 64 | dP^T 64, fp32);
+// [256, 384) two operand buffers (P^T 32 | dS^T 32, bf16 pairs of the 64
+// sub-tile queries); [384, 512) the accumulators dV 64 | dK 64.
+constexpr int kQStages = 3;
 constexpr int kSub = 64;  // queries per sub-tile
+constexpr uint32_t kOpCol = 256;
+constexpr uint32_t kAccColKV = 384;
+constexpr int kPairBytes = kTile * 8;  // (L log2e, D) of one query tile
 constexpr size_t dkdv_smem_bytes() {
-  // [K, V] x 2 items, [Q, dO] x stages, P^T and dS^T x 2 sub-tiles (one box
-  // each), each compute warp's per-column L and D of two sub-tiles, aux
-  return 1024 + 4 * (size_t)kBox + 2 * (size_t)kQStages * kBox + 4 * (size_t)kBox +
-         (kCT / 32) * 2 * 64 * sizeof(float) + kAux;
+  // [K, V] x 2 items, [Q, dO] x stages, (L, D) pairs x stages, aux
+  return 1024 + 4 * (size_t)kBox + 2 * (size_t)kQStages * kBox + (size_t)kQStages * kPairBytes +
+         kAux;
 }
 
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     flash_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
-                             const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ lse,
-                             const float* __restrict__ dsum, __nv_bfloat16* __restrict__ dqkv, int B,
-                             int T, int C, int H, float sl2, float scale, int* err) {
+                             const __grid_constant__ CUtensorMap tmDO,
+                             const float2* __restrict__ pairs, __nv_bfloat16* __restrict__ dqkv,
+                             int B, int T, int C, int H, float sl2, float scale, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sKV = smem;                    // [2 items][K box, V box]
   uint8_t* sQ = sKV + 4 * kBox;           // [kQStages]
   uint8_t* sDO = sQ + kQStages * kBox;    // [kQStages]
-  uint8_t* sPT = sDO + kQStages * kBox;   // [2 sub-tiles]: 128 keys x 64 queries
-  uint8_t* sDST = sPT + 2 * kBox;         // [2 sub-tiles]
-  float* col_lse = reinterpret_cast<float*>(sDST + 2 * kBox);  // [warp][2][L 32, D 32]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(col_lse + (kCT / 32) * 2 * 64);
+  uint8_t* sLD = sDO + kQStages * kBox;   // [kQStages][128 pairs]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sLD + kQStages * kPairBytes);
   const uint32_t kv_full0 = smem_u32(bars + 0);     // [2]
   const uint32_t kv_empty0 = smem_u32(bars + 2);    // [2]
-  const uint32_t qd_full0 = smem_u32(bars + 4);     // [2]
-  const uint32_t qd_empty0 = smem_u32(bars + 6);    // [2]
-  const uint32_t sd_full0 = smem_u32(bars + 8);     // [2]
-  const uint32_t sd_empty0 = smem_u32(bars + 10);   // [2]
-  const uint32_t pd_full0 = smem_u32(bars + 12);    // [2]
-  const uint32_t pd_empty0 = smem_u32(bars + 14);   // [2]
-  const uint32_t acc_full0 = smem_u32(bars + 16);   // [2]
-  const uint32_t acc_empty0 = smem_u32(bars + 18);  // [2]
-  const uint32_t drain = smem_u32(bars + 20);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  const uint32_t qd_full0 = smem_u32(bars + 4);     // [kQStages]
+  const uint32_t qd_empty0 = smem_u32(bars + 4 + kQStages);   // [kQStages]
+  const uint32_t sd_full0 = smem_u32(bars + 4 + 2 * kQStages);   // [2]
+  const uint32_t sd_empty0 = sd_full0 + 16;         // [2]
+  const uint32_t pd_full0 = sd_full0 + 32;          // [2]
+  const uint32_t pd_empty0 = sd_full0 + 48;         // [2]
+  const uint32_t acc_full = sd_full0 + 64;
+  const uint32_t acc_empty = sd_full0 + 72;
+  const uint32_t drain = sd_full0 + 80;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 + 2 * kQStages + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int nq = (T + kTile - 1) / kTile;
+  const int Tp = nq * kTile;
   const int BH = B * H, items = nq * BH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -130,15 +141,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(kv_full0 + 8 * s, 1);
       mbar_init(kv_empty0 + 8 * s, 1);
-      mbar_init(qd_full0 + 8 * s, 1);
-      mbar_init(qd_empty0 + 8 * s, 1);
       mbar_init(sd_full0 + 8 * s, 1);
       mbar_init(sd_empty0 + 8 * s, kCT);
       mbar_init(pd_full0 + 8 * s, kCT);
       mbar_init(pd_empty0 + 8 * s, 1);
-      mbar_init(acc_full0 + 8 * s, 1);
-      mbar_init(acc_empty0 + 8 * s, kCT);
     }
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(qd_full0 + 8 * s, 1);
+      mbar_init(qd_empty0 + 8 * s, 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kCT);
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -172,26 +185,28 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         kv_issued |= 1u << ks;
         kv_par = (kv_par & ~(1u << ks)) | (kpar << ks);
         for (int t = 0; t < n; ++t, ++g) {
-          const int st = g & 1;
-          const uint32_t par = (g >> 1) & 1u;
+          const int st = g % kQStages;
+          const uint32_t par = (g / kQStages) & 1u;
           if (!mbar_wait(qd_empty0 + 8 * st, par ^ 1u, abort_flag, err)) {
             ok = false;
             break;
           }
           const uint32_t fb = qd_full0 + 8 * st;
-          mbar_expect_tx(fb, 2 * kBox);
+          mbar_expect_tx(fb, 2 * kBox + kPairBytes);
           tma_load_3d(smem_u32(sQ + st * kBox), &tmQKV, fb, h * kHD, (j + t) * kTile, b);
           tma_load_3d(smem_u32(sDO + st * kBox), &tmDO, fb, h * kHD, (j + t) * kTile, b);
+          bulk_load_1d(smem_u32(sLD + st * kPairBytes),
+                       pairs + (size_t)bh * Tp + (size_t)(j + t) * kTile, kPairBytes, fb);
           issued |= 1u << st;
           last_par = (last_par & ~(1u << st)) | (par << st);
         }
       }
       // every copy issued lands before the shared memory is released
       const uint64_t t0 = global_ns();
-      for (int s = 0; s < 2; ++s) {
+      for (int s = 0; s < 2; ++s)
         if (kv_issued & (1u << s)) drain_wait(kv_full0 + 8 * s, (kv_par >> s) & 1u, t0);
+      for (int s = 0; s < kQStages; ++s)
         if (issued & (1u << s)) drain_wait(qd_full0 + 8 * s, (last_par >> s) & 1u, t0);
-      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -219,30 +234,35 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         return true;
       };
       // dV += P^T dO_s, dK += dS^T Q_s of a sub-tile whose P^T and dS^T are
-      // (being) written; releases the query tile after its second half and
-      // hands the accumulators over after the item's last sub-tile
+      // (being) written to TMEM; releases the query tile after its second
+      // half and hands the accumulators over after the item's last sub-tile
       struct Pend {
-        uint32_t s, acc, ab;
+        uint32_t s;
         int st, hs;
         bool first, last;
       };
+      uint32_t n_acc = 0;  // items whose accumulators have been started
       auto issue_acc = [&](const Pend& p) -> bool {
         const uint32_t sb = p.s & 1u;
+        if (p.first) {  // the previous item's dV and dK have been read out
+          if (!mbar_wait(acc_empty, (n_acc & 1u) ^ 1u, abort_flag, err)) return false;
+          ++n_acc;
+        }
         if (!mbar_wait(pd_full0 + 8 * sb, (p.s >> 1) & 1u, abort_flag, err)) return false;
         tc_fence_after();
         const uint32_t q_base = smem_u32(sQ + p.st * kBox), do_base = smem_u32(sDO + p.st * kBox);
-        const uint32_t pt = smem_u32(sPT + sb * kBox), dst = smem_u32(sDST + sb * kBox);
+        const uint32_t pt = tmem + kOpCol + sb * kSub, dst = pt + kSub / 2;
 #pragma unroll
         for (int k = 0; k < kSub / 16; ++k)
-          tc_mma(tmem + p.acc, desc_kmajor(pt, k), desc_mnmajor(do_base, 4 * p.hs + k), idA,
-                 (!p.first || k > 0) ? 1u : 0u);
+          attn::tc_mma_ts(tmem + kAccColKV, pt + (uint32_t)(8 * k),
+                          desc_mnmajor(do_base, 4 * p.hs + k), idA, (!p.first || k > 0) ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < kSub / 16; ++k)
-          tc_mma(tmem + p.acc + kHD, desc_kmajor(dst, k), desc_mnmajor(q_base, 4 * p.hs + k), idA,
-                 (!p.first || k > 0) ? 1u : 0u);
+          attn::tc_mma_ts(tmem + kAccColKV + kHD, dst + (uint32_t)(8 * k),
+                          desc_mnmajor(q_base, 4 * p.hs + k), idA, (!p.first || k > 0) ? 1u : 0u);
         tc_commit(pd_empty0 + 8 * sb);
         if (p.hs == 1) tc_commit(qd_empty0 + 8 * p.st);
-        if (p.last) tc_commit(acc_full0 + 8 * p.ab);
+        if (p.last) tc_commit(acc_full);
         return true;
       };
       // One flat sequence over every sub-tile of every item: the scores of
@@ -255,21 +275,19 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (w < 0) break;
         const int n = nq - w / BH;
         const int ks = n_item & 1;
-        const uint32_t ab = n_item & 1u, acc = kAccCol + ab * 2 * kHD;
         ok = mbar_wait(kv_full0 + 8 * ks, (n_item >> 1) & 1u, abort_flag, err);
-        if (ok) ok = mbar_wait(acc_empty0 + 8 * ab, ((n_item >> 1) & 1u) ^ 1u, abort_flag, err);
         if (!ok) break;
         tc_fence_after();
         for (int t = 0; t < n && ok; ++t, ++gt) {
-          const int st = gt & 1;
-          const uint32_t tpar = (gt >> 1) & 1u;
+          const int st = gt % kQStages;
+          const uint32_t tpar = (gt / kQStages) & 1u;
           for (int hs = 0; hs < 2; ++hs, ++gs) {
             ok = issue_sd(gs, st, tpar, hs, ks);
             if (!ok) break;
             if (t == n - 1 && hs == 1) tc_commit(kv_empty0 + 8 * ks);  // K, V no longer read
             if (have) ok = issue_acc(pend);
             if (!ok) break;
-            pend = Pend{gs, acc, ab, st, hs, t == 0 && hs == 0, t == n - 1 && hs == 1};
+            pend = Pend{gs, st, hs, t == 0 && hs == 0, t == n - 1 && hs == 1};
             have = true;
           }
         }
@@ -283,13 +301,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   } else {
     // -------------------------------------------------------- compute --
     // thread = key row r, owning 32 of a sub-tile's 64 query columns.  Every
-    // wait is per warp (warps drift apart and overlap their latencies); each
-    // warp stages the L and D of its own 32 columns.
+    // wait is per warp (warps drift apart and overlap their latencies).
     const int qw = warp & 3, half = (warp - 2) >> 2;
     const int r = qw * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    float* wcl = col_lse + (warp - 2) * 2 * 64;  // [2 sub-tiles][L 32 | D 32]
-    uint32_t n_item = 0, gs = 0;
+    uint32_t n_item = 0, gs = 0, gt = 0;
     bool ok = true;
     for (int k = 0; ok; ++k, ++n_item) {
       const int w = snake_item(k, items);
@@ -297,91 +313,68 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const int j = w / BH, bh = w % BH, b = bh / H, h = bh % H;
       const int n = nq - j;
       const int kj = j * kTile + r;  // this thread's key row
-      const float* lse_bh = lse + (size_t)bh * T;
-      const float* d_bh = dsum + (size_t)bh * T;
-      for (int t = 0; t < n && ok; ++t) {
+      for (int t = 0; t < n && ok; ++t, ++gt) {
+        const int st = gt % kQStages;
+        const float4* ld4 = reinterpret_cast<const float4*>(sLD + st * kPairBytes);
         for (int hs = 0; hs < 2; ++hs, ++gs) {
           const uint32_t sb = gs & 1u;
-          const int cq = kSub * hs + 32 * half;  // first column of this thread in the tile
-          const int qc0 = (j + t) * kTile + cq;  // its query index
-          // L (log2 units) and D of the warp's 32 columns, loaded while the
-          // tensor core computes the scores
-          float* cl = wcl + sb * 64;
-          {
-            const int q = qc0 + lane;
-            cl[lane] = q < T ? lse_bh[q] * kLog2e : 0.f;
-            cl[32 + lane] = q < T ? d_bh[q] : 0.f;
-          }
-          __syncwarp();
-          // causal mask on the diagonal tile, padding past T on the last one
-          const bool masked = t == 0 || qc0 - cq + kSub * (hs + 1) > T;
+          const int cq = kSub * hs + 32 * half;  // first query column of this thread in the tile
           ok = warp_and(mbar_wait(sd_full0 + 8 * sb, (gs >> 1) & 1u, abort_flag, err));
           if (!ok) break;
           tc_fence_after();
-          const uint32_t s_col = lane_base + sb * 2 * kSub + 32 * half;
-          const uint32_t pt_row = smem_u32(sPT + sb * kBox) + (uint32_t)(r * 128);
-          const uint32_t dst_row = smem_u32(sDST + sb * kBox) + (uint32_t)(r * 128);
-          uint32_t sa[16], pa[16], sb16[16], pb[16];
-          auto ld_chunk = [&](int ch, uint32_t* s_, uint32_t* p_) {
-            attn::tc_ld16(s_col + 16 * ch, s_);
-            attn::tc_ld16(s_col + kSub + 16 * ch, p_);
-          };
-          auto do_chunk = [&](int ch, const uint32_t* s_, const uint32_t* p_, auto mask) -> bool {
-            float pv[16], dv[16];
-#pragma unroll
-            for (int c = 0; c < 16; c += 4) {
-              const float4 a = *reinterpret_cast<const float4*>(cl + 16 * ch + c);
-              const float4 d = *reinterpret_cast<const float4*>(cl + 32 + 16 * ch + c);
-              pv[c] = a.x; pv[c + 1] = a.y; pv[c + 2] = a.z; pv[c + 3] = a.w;
-              dv[c] = d.x; dv[c + 1] = d.y; dv[c + 2] = d.z; dv[c + 3] = d.w;
-            }
-            const int lim = kj - qc0 - 16 * ch;  // columns c < lim are queries before the key
-            const int tcut = T - qc0 - 16 * ch;  // columns c >= tcut are past the sequence
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              float p = fast_exp2(fmaf(__uint_as_float(s_[c]), sl2, -pv[c]));
-              if (decltype(mask)::value && (c < lim || c >= tcut)) p = 0.f;
-              pv[c] = p;
-              dv[c] = p * (__uint_as_float(p_[c]) - dv[c]);
-            }
-            // the products of sub-tile gs - 2 have read this P^T / dS^T buffer
-            if (ch == 0 &&
-                !warp_and(mbar_wait(pd_empty0 + 8 * sb, ((gs >> 1) & 1u) ^ 1u, abort_flag, err)))
-              return false;
-#pragma unroll
-            for (int c8 = 0; c8 < 2; ++c8) {
-              const uint32_t off = (uint32_t)(((4 * half + 2 * ch + c8) ^ (r & 7)) << 4);
-              attn::st_shared_bf16x8(pt_row + off, pv + 8 * c8);
-              attn::st_shared_bf16x8(dst_row + off, dv + 8 * c8);
-            }
-            return true;
-          };
-          ld_chunk(0, sa, pa);
-          tc_wait_ld();
-          ld_chunk(1, sb16, pb);
-          ok = masked ? do_chunk(0, sa, pa, std::true_type{}) : do_chunk(0, sa, pa, std::false_type{});
+          uint32_t sr[32], dp[32];
+          tc_ld32(lane_base + sb * 2 * kSub + 32 * half, sr);
+          tc_ld32(lane_base + sb * 2 * kSub + kSub + 32 * half, dp);
           tc_wait_ld();
           tc_fence_before();
           mbar_arrive(sd_empty0 + 8 * sb);  // the scores are read: sub-tile gs + 2 may be computed
+          if (t == 0) {  // the diagonal tile: queries before the key are masked
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (cq + c < r) sr[c] = kNegInf;
+          }
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            // (L log2e, D) of queries cq + c .. cq + c + 3 (query-tile stage st)
+            const float4 a = ld4[(cq + c) / 2];
+            const float4 bq = ld4[(cq + c) / 2 + 1];
+            const float lq[4] = {a.x, a.z, bq.x, bq.z};
+            const float dq[4] = {a.y, a.w, bq.y, bq.w};
+            float p[4], ds[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              p[e] = fast_exp2(fmaf(__uint_as_float(sr[c + e]), sl2, -lq[e]));
+              ds[e] = p[e] * (__uint_as_float(dp[c + e]) - dq[e]);
+            }
+            pk[c / 2] = attn::pack_bf16x2(p[0], p[1]);
+            pk[c / 2 + 1] = attn::pack_bf16x2(p[2], p[3]);
+            dk[c / 2] = attn::pack_bf16x2(ds[0], ds[1]);
+            dk[c / 2 + 1] = attn::pack_bf16x2(ds[2], ds[3]);
+          }
+          // the products of sub-tile gs - 2 have read this operand buffer
+          ok = warp_and(mbar_wait(pd_empty0 + 8 * sb, ((gs >> 1) & 1u) ^ 1u, abort_flag, err));
           if (!ok) break;
-          if (masked) do_chunk(1, sb16, pb, std::true_type{});
-          else do_chunk(1, sb16, pb, std::false_type{});
-          fence_async_smem();
+          tc_fence_after();
+          const uint32_t op = lane_base + kOpCol + sb * kSub + 16 * half;
+          tc_st16(op, pk);
+          tc_st16(op + kSub / 2, dk);
+          attn::tc_wait_st();
+          tc_fence_before();
           mbar_arrive(pd_full0 + 8 * sb);
         }
       }
       if (!ok) break;
-      // the item's dV and dK (accumulator pair n_item % 2)
-      const uint32_t ab = n_item & 1u, acc = kAccCol + ab * 2 * kHD;
-      ok = warp_and(mbar_wait(acc_full0 + 8 * ab, (n_item >> 1) & 1u, abort_flag, err));
+      // the item's dV and dK
+      ok = warp_and(mbar_wait(acc_full, n_item & 1u, abort_flag, err));
       if (!ok) break;
       tc_fence_after();
       uint32_t rv[32], rk[32];
-      tc_ld32(lane_base + acc + 32 * half, rv);
-      tc_ld32(lane_base + acc + kHD + 32 * half, rk);
+      tc_ld32(lane_base + kAccColKV + 32 * half, rv);
+      tc_ld32(lane_base + kAccColKV + kHD + 32 * half, rk);
       tc_wait_ld();
       tc_fence_before();
-      mbar_arrive(acc_empty0 + 8 * ab);
+      mbar_arrive(acc_empty);
       if (kj < T) {
         __nv_bfloat16* row = dqkv + ((size_t)b * T + kj) * 3 * C + (size_t)h * kHD + 32 * half;
 #pragma unroll
@@ -406,17 +399,21 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 }
 
 // --------------------------------------------------------------------- dQ --
-constexpr int kKVStages = 3;
+// TMEM columns: [0, 128) S, [128, 256) dP (fp32); [256, 384) two dS buffers
+// (bf16 pairs of 128 keys); [384, 512) two dQ accumulators.
+constexpr int kKVStages = 4;
+constexpr uint32_t kDSCol = 256;
+constexpr uint32_t kAccColQ = 384;
 constexpr size_t dq_smem_bytes() {
-  // Q, dO, O, [K, V] x stages, dS (two buffers of two boxes), aux
-  return 1024 + 3 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + 4 * (size_t)kBox + kAux;
+  // Q, dO, O, [K, V] x stages, aux
+  return 1024 + 3 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + kAux;
 }
 
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     flash_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
                            const __grid_constant__ CUtensorMap tmDO,
                            const __grid_constant__ CUtensorMap tmO, const float* __restrict__ lse,
-                           float* __restrict__ dsum, __nv_bfloat16* __restrict__ dqkv, int B,
+                           float2* __restrict__ pairs, __nv_bfloat16* __restrict__ dqkv, int B,
                            int T, int C, int H, float sl2, float scale, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -426,23 +423,23 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   uint8_t* sO = sDO + kBox;                // the forward's output rows (for D)
   uint8_t* sK = sO + kBox;                 // [kKVStages]
   uint8_t* sV = sK + kKVStages * kBox;     // [kKVStages]
-  uint8_t* sDS = sV + kKVStages * kBox;    // [2 buffers][2 boxes]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + 4 * kBox);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kKVStages * kBox);
   const uint32_t qd_full = smem_u32(bars + 0);
   const uint32_t qd_empty = smem_u32(bars + 1);
-  const uint32_t kv_full0 = smem_u32(bars + 2);              // [3]
-  const uint32_t kv_empty0 = smem_u32(bars + 2 + kKVStages); // [3]
-  const uint32_t sd_full = smem_u32(bars + 8);
-  const uint32_t sd_empty = smem_u32(bars + 9);
-  const uint32_t ds_full0 = smem_u32(bars + 10);             // [2]
-  const uint32_t ds_empty0 = smem_u32(bars + 12);            // [2]
-  const uint32_t acc_full0 = smem_u32(bars + 14);            // [2]
-  const uint32_t acc_empty0 = smem_u32(bars + 16);           // [2]
-  const uint32_t drain = smem_u32(bars + 18);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  const uint32_t kv_full0 = smem_u32(bars + 2);              // [kKVStages]
+  const uint32_t kv_empty0 = smem_u32(bars + 2 + kKVStages); // [kKVStages]
+  const uint32_t sd_full = smem_u32(bars + 2 + 2 * kKVStages);
+  const uint32_t sd_empty = sd_full + 8;
+  const uint32_t ds_full0 = sd_full + 16;                    // [2]
+  const uint32_t ds_empty0 = sd_full + 32;                   // [2]
+  const uint32_t acc_full0 = sd_full + 48;                   // [2]
+  const uint32_t acc_empty0 = sd_full + 64;                  // [2]
+  const uint32_t drain = sd_full + 80;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int nq = (T + kTile - 1) / kTile;
+  const int Tp = nq * kTile;
   const int BH = B * H, items = nq * BH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -534,16 +531,16 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         tc_commit(sd_full);
         return true;
       };
-      // dQ (+)= dS K into the accumulator at column acc
+      // dQ (+)= dS K into the accumulator at column acc (dS from TMEM)
       auto issue_dq = [&](uint32_t gg, uint32_t acc, bool first) -> bool {
         const int st = gg % kKVStages, db = gg & 1;
         if (!mbar_wait(ds_full0 + 8 * db, (gg >> 1) & 1u, abort_flag, err)) return false;
         tc_fence_after();
-        const uint32_t ds = smem_u32(sDS + db * 2 * kBox), k_base = smem_u32(sK + st * kBox);
+        const uint32_t ds = tmem + kDSCol + (uint32_t)(db * kHD), k_base = smem_u32(sK + st * kBox);
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k)
-          tc_mma(tmem + acc, desc_kmajor(ds + (uint32_t)((k >> 2) * kBox), k & 3),
-                 desc_mnmajor(k_base, k), idQ, (!first || k > 0) ? 1u : 0u);
+          attn::tc_mma_ts(tmem + acc, ds + (uint32_t)(8 * k), desc_mnmajor(k_base, k), idQ,
+                          (!first || k > 0) ? 1u : 0u);
         tc_commit(ds_empty0 + 8 * db);
         tc_commit(kv_empty0 + 8 * st);
         return true;
@@ -552,7 +549,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         const int w = snake_item(k, items);
         if (w < 0) break;
         const int n = nq - w / BH;  // i + 1
-        const uint32_t ab = n_item & 1u, acc = kAccCol + ab * kHD;
+        const uint32_t ab = n_item & 1u, acc = kAccColQ + ab * kHD;
         ok = mbar_wait(qd_full, n_item & 1u, abort_flag, err);
         if (ok) ok = mbar_wait(acc_empty0 + 8 * ab, ((n_item >> 1) & 1u) ^ 1u, abort_flag, err);
         if (!ok) break;
@@ -576,6 +573,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     }
   } else {
     // -------------------------------------------------------- compute --
+    // thread = query row r, owning 64 of a key tile's 128 columns
     const int qw = warp & 3, half = (warp - 2) >> 2;
     const int r = qw * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
@@ -589,7 +587,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const int qi = i * kTile + r;  // this thread's query row
       const float lse2 = qi < T ? lse[(size_t)bh * T + qi] * kLog2e : 0.f;
       // D = rowsum(dO * O) of this row from the item's dO and O tiles (rows
-      // past T are zero-filled); stored for the dK/dV kernel, which runs next
+      // past T are zero-filled); stored with L for the dK/dV kernel
       ok = warp_and(mbar_wait(qd_full, n_item & 1u, abort_flag, err));
       if (!ok) break;
       float drow = 0.f;
@@ -602,70 +600,46 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         for (int e = 0; e < 8; ++e) drow = fmaf(a[e], o[e], drow);
       }
       mbar_arrive(qd_empty);  // this thread is done with dO and O
-      if (half == 0 && qi < T) dsum[(size_t)bh * T + qi] = drow;
+      if (half == 0)
+        pairs[(size_t)bh * Tp + qi] = qi < T ? make_float2(lse2, drow) : make_float2(INFINITY, 0.f);
       for (int jj = 0; jj < n && ok; ++jj) {
         const uint32_t gg = gk + jj;
         const int db = gg & 1;
-        const int key0 = jj * kTile + 64 * half;
-        const uint32_t ds_row = smem_u32(sDS + (db * 2 + half) * kBox) + (uint32_t)(r * 128);
-        // causal mask on the diagonal tile, padding past T on the last one
-        const bool masked = jj == i || (jj + 1) * kTile > T;
         ok = warp_and(mbar_wait(sd_full, gg & 1u, abort_flag, err));
         if (!ok) break;
         tc_fence_after();
-        // 16 key columns per chunk; the next chunk's TMEM loads are in
-        // flight while the current chunk is computed
-        uint32_t sa[16], pa[16], sb[16], pb[16];
-        auto ld_chunk = [&](int ch, uint32_t* s_, uint32_t* p_) {
-          const uint32_t col = (uint32_t)(64 * half + 16 * ch);
-          attn::tc_ld16(lane_base + col, s_);
-          attn::tc_ld16(lane_base + kTile + col, p_);
-        };
-        auto do_chunk = [&](int ch, const uint32_t* s_, const uint32_t* p_, auto mask) -> bool {
-          const int lim = qi - key0 - 16 * ch;  // columns c > lim are keys after the query
-          const int tcut = T - key0 - 16 * ch;  // columns c >= tcut are past the sequence
-          float ds[16];
+        uint32_t sr[64], dp[64];
+        tc_ld32(lane_base + 64 * half, sr);
+        tc_ld32(lane_base + 64 * half + 32, sr + 32);
+        tc_ld32(lane_base + kTile + 64 * half, dp);
+        tc_ld32(lane_base + kTile + 64 * half + 32, dp + 32);
+        tc_wait_ld();
+        tc_fence_before();
+        mbar_arrive(sd_empty);  // S and dP are read: the next key tile's may be computed
+        if (jj == i) {  // the diagonal tile: keys after the query are masked
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float p = fast_exp2(fmaf(__uint_as_float(s_[c]), sl2, -lse2));
-            if (decltype(mask)::value && (c > lim || c >= tcut)) p = 0.f;
-            ds[c] = p * (__uint_as_float(p_[c]) - drow);
-          }
-          // the product two tiles back has read this dS buffer
-          if (ch == 0 &&
-              !warp_and(mbar_wait(ds_empty0 + 8 * db, ((gg >> 1) & 1u) ^ 1u, abort_flag, err)))
-            return false;
+          for (int c = 0; c < 64; ++c)
+            if (64 * half + c > r) sr[c] = kNegInf;
+        }
+        uint32_t dk[32];
 #pragma unroll
-          for (int c8 = 0; c8 < 2; ++c8)
-            attn::st_shared_bf16x8(ds_row + (uint32_t)(((2 * ch + c8) ^ (r & 7)) << 4), ds + 8 * c8);
-          return true;
-        };
-        auto run = [&](auto mask) {
-          ld_chunk(0, sa, pa);
-          tc_wait_ld();
-          ld_chunk(1, sb, pb);
-          ok = do_chunk(0, sa, pa, mask);
-          tc_wait_ld();
-          if (ok) {
-            ld_chunk(2, sa, pa);
-            do_chunk(1, sb, pb, mask);
-            tc_wait_ld();
-            ld_chunk(3, sb, pb);
-            do_chunk(2, sa, pa, mask);
-            tc_wait_ld();
-            tc_fence_before();
-            mbar_arrive(sd_empty);  // both score buffers are read: the next tile's may be computed
-            do_chunk(3, sb, pb, mask);
-          }
-        };
-        if (masked) run(std::true_type{});
-        else run(std::false_type{});
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -lse2));
+          dk[c / 2] = attn::pack_bf16x2(p0 * (__uint_as_float(dp[c]) - drow),
+                                        p1 * (__uint_as_float(dp[c + 1]) - drow));
+        }
+        // the product two tiles back has read this dS buffer
+        ok = warp_and(mbar_wait(ds_empty0 + 8 * db, ((gg >> 1) & 1u) ^ 1u, abort_flag, err));
         if (!ok) break;
-        fence_async_smem();
+        tc_fence_after();
+        attn::tc_st32(lane_base + kDSCol + (uint32_t)(db * kHD) + 32 * half, dk);
+        attn::tc_wait_st();
+        tc_fence_before();
         mbar_arrive(ds_full0 + 8 * db);
       }
       if (!ok) break;
-      const uint32_t ab = n_item & 1u, acc = kAccCol + ab * kHD;
+      const uint32_t ab = n_item & 1u, acc = kAccColQ + ab * kHD;
       ok = warp_and(mbar_wait(acc_full0 + 8 * ab, (n_item >> 1) & 1u, abort_flag, err));
       if (!ok) break;
       tc_fence_after();
@@ -696,11 +670,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 
 }  // namespace
 
-cudaError_t attention_bwd_tc(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
+size_t attention_bwd_tc_scratch_floats(int B, int T, int H) {
+  const size_t Tp = (size_t)(T + kTile - 1) / kTile * kTile;
+  return 2 * (size_t)B * H * Tp;
+}
+
+cudaError_t attention_bwd_tc(act_t* dqkv, float* scratch, const act_t* datt, const act_t* qkv,
                              const act_t* att, const float* lse, int B, int T, int C, int H,
                              int* err, cudaStream_t s) {
   if (C / H != kHD || (reinterpret_cast<uintptr_t>(qkv) & 15) ||
-      (reinterpret_cast<uintptr_t>(datt) & 15) || (reinterpret_cast<uintptr_t>(att) & 15))
+      (reinterpret_cast<uintptr_t>(datt) & 15) || (reinterpret_cast<uintptr_t>(att) & 15) ||
+      (reinterpret_cast<uintptr_t>(scratch) & 15))
     return cudaErrorInvalidValue;
   CUtensorMap tq, td, to;
   cudaError_t e = attn::seq_map(&tq, qkv, B, T, 3 * C);
@@ -727,10 +707,12 @@ cudaError_t attention_bwd_tc(act_t* dqkv, float* dsum, const act_t* datt, const 
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = items < sms ? items : sms;
-  // dQ first: it forms D = rowsum(dO * O) of its query tiles for dK/dV
-  flash_bwd_dq_tc_kernel<<<grid, kThreadsBwd, sm_b, s>>>(tq, td, to, lse, dsum, dqkv, B, T, C, H,
+  float2* pairs = reinterpret_cast<float2*>(scratch);
+  // dQ first: it forms D = rowsum(dO * O) of its query tiles and stores the
+  // (L, D) pairs for dK/dV
+  flash_bwd_dq_tc_kernel<<<grid, kThreadsBwd, sm_b, s>>>(tq, td, to, lse, pairs, dqkv, B, T, C, H,
                                                          sl2, scale, err);
-  flash_bwd_dkdv_tc_kernel<<<grid, kThreadsBwd, sm_a, s>>>(tq, td, lse, dsum, dqkv, B, T, C, H, sl2,
+  flash_bwd_dkdv_tc_kernel<<<grid, kThreadsBwd, sm_a, s>>>(tq, td, pairs, dqkv, B, T, C, H, sl2,
                                                            scale, err);
   note_launch(2);
   return cudaGetLastError();

@@ -5,25 +5,30 @@
 // Items are ordered heaviest first and dealt to the CTAs in a snake order,
 // which balances the causal work across SMs.  10 warps:
 //   warp 0     TMA: the item's two Q tiles, then its K/V tiles of 128 keys
-//              into a 3-stage ring (128-byte swizzle, zero fill past the
+//              into a 4-stage ring (128-byte swizzle, zero fill past the
 //              sequence), running ahead into the next item;
 //   warp 1     TMEM owner and MMA issuer: S_t = Q_t K_j^T (M=128, N=128,
 //              K=64) into one TMEM buffer per tile t, and O_t += P_t V_j
-//              (M=128, N=64, K=128; V read MN-major from its tile), O_t
-//              accumulated in TMEM over the item's key tiles.  S for key
-//              tile j+1 is issued before PV for key tile j, so the next
-//              scores are ready when a softmax ends;
+//              (M=128, N=64, K=128) with P_t read from TMEM as the A operand
+//              and V read MN-major from its shared-memory tile; O_t
+//              accumulates in TMEM over the item's key tiles.  S for key
+//              tile j+1 is issued before PV for key tile j;
 //   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: one thread
-//              per query row.  Each reads its row of S from TMEM twice (the
-//              max, then the exponentials) and writes P = 2^(S log2e /
-//              sqrt(d) - m) as bf16 into a swizzled tile (the next MMA's A
-//              operand).  The reference max m is raised only when a tile's
-//              max exceeds it by more than 2^8 (P stays below 256); then the
-//              row of O in TMEM and the running sum are rescaled first.  No
-//              thread waits for another thread's row.
+//              per query row.  A thread loads its whole row of S from TMEM
+//              into registers at once and hands the buffer straight back (so
+//              the next S is computed while this one is exponentiated),
+//              takes the row max, forms P = 2^(S log2e / sqrt(d) - m) and
+//              writes it as packed bf16 into its tile's P columns of TMEM.
+//              The reference max m is raised only when a tile's max exceeds
+//              it by more than 2^8 (P stays below 256); then the row of O in
+//              TMEM and the running sum are rescaled first.  No thread waits
+//              for another thread's row.
 // T x T is never materialised.  The output row is normalised by the
 // running sum; the natural-log log-sum-exp of each row is stored for the
 // backward pass.  Every wait is bounded (error word ERR_TIMEOUT).
+//
+// TMEM columns: [0, 256) S_A | S_B (fp32), [256, 384) O_A | O_B (fp32),
+// [384, 512) P_A | P_B (128 keys as 64 columns of bf16 pairs).
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -43,17 +48,19 @@ using attn::kHD;
 using attn::kBox;
 using attn::kTile;
 
-constexpr int kKVStages = 3;
+constexpr int kKVStages = 4;
 constexpr int kRowThreads = 128;  // softmax threads per query tile
 constexpr int kThreadsAttn = 64 + 2 * kRowThreads;
-constexpr uint32_t kTmemCols = 512;  // S: 2 tiles x 128; O: 2 tiles x 64
-constexpr uint32_t kOCol = 2 * kTile;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kOCol = 2 * kTile;         // O_t at kOCol + t * kHD
+constexpr uint32_t kPCol = kOCol + 2 * kHD;   // P_t at kPCol + t * kHD (bf16 pairs)
 constexpr float kRescaleLog2 = 8.0f;  // raise the reference max past this margin
 constexpr int kAux = 1024;  // barriers
+constexpr uint32_t kNegInf = 0xff800000u;
 
 constexpr size_t attn_smem_bytes() {
-  // Q (two tiles), K ring, V ring, P (two tiles of two 64-key boxes), aux
-  return 1024 + 2 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + 4 * (size_t)kBox + kAux;
+  // Q (two tiles), K ring, V ring, aux
+  return 1024 + 2 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + kAux;
 }
 
 // Work item k of this CTA (snake order over the heaviest-first item list);
@@ -86,12 +93,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   uint8_t* sQ = smem;                           // [2 tiles][kBox]
   uint8_t* sK = sQ + 2 * kBox;                  // [kKVStages][kBox]
   uint8_t* sV = sK + kKVStages * kBox;          // [kKVStages][kBox]
-  uint8_t* sP = sV + kKVStages * kBox;          // [2 tiles][2 boxes]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 4 * kBox);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kKVStages * kBox);
   const uint32_t q_full = smem_u32(bars + 0);
   const uint32_t q_empty = smem_u32(bars + 1);
-  const uint32_t kv_full0 = smem_u32(bars + 2);                  // [3]
-  const uint32_t kv_empty0 = smem_u32(bars + 2 + kKVStages);     // [3]
+  const uint32_t kv_full0 = smem_u32(bars + 2);                  // [kKVStages]
+  const uint32_t kv_empty0 = smem_u32(bars + 2 + kKVStages);     // [kKVStages]
   const uint32_t s_full0 = smem_u32(bars + 2 + 2 * kKVStages);   // [2 tiles]
   const uint32_t s_empty0 = s_full0 + 16;                        // [2 tiles]
   const uint32_t p_full0 = s_full0 + 32;                         // [2 tiles]
@@ -196,17 +202,17 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         ++cs[t];
         return true;
       };
-      // O_t (+)= P_t V (value tile in ring stage st); the item's first
-      // product initialises O_t
+      // O_t (+)= P_t V (P_t from TMEM, value tile in ring stage st); the
+      // item's first product initialises O_t
       auto issue_pv = [&](int t, int st, bool first) -> bool {
         if (!mbar_wait(p_full0 + 8 * t, co[t] & 1u, abort_flag, err)) return false;
         tc_fence_after();
-        const uint32_t p_base = smem_u32(sP + t * 2 * kBox), v_base = smem_u32(sV + st * kBox);
+        const uint32_t v_base = smem_u32(sV + st * kBox);
+        const uint32_t p_t = tmem + kPCol + (uint32_t)(t * kHD);
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k)
-          tc_mma(tmem + kOCol + (uint32_t)(t * kHD),
-                 desc_kmajor(p_base + (uint32_t)((k >> 2) * kBox), k & 3), desc_mnmajor(v_base, k),
-                 idO, (k > 0 || !first) ? 1u : 0u);
+          attn::tc_mma_ts(tmem + kOCol + (uint32_t)(t * kHD), p_t + (uint32_t)(8 * k),
+                          desc_mnmajor(v_base, k), idO, (k > 0 || !first) ? 1u : 0u);
         tc_commit(o_full0 + 8 * t);
         ++co[t];
         return true;
@@ -247,9 +253,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const int qw = warp & 3;        // TMEM lane quarter
     const int r = qw * 32 + lane;   // row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    const uint32_t s_col = (uint32_t)(t * kTile);
-    const uint32_t o_col = kOCol + (uint32_t)(t * kHD);
-    const uint32_t p_row = smem_u32(sP + t * 2 * kBox) + (uint32_t)(r * 128);  // this row of P
+    const uint32_t s_col = lane_base + (uint32_t)(t * kTile);
+    const uint32_t o_col = lane_base + kOCol + (uint32_t)(t * kHD);
+    const uint32_t p_col = lane_base + kPCol + (uint32_t)(t * kHD);
     uint32_t cs = 0, co = 0;  // S tiles read / PV products waited for by this tile's threads
     bool ok = true;
     // wait for the next PV product of this tile (every completion is
@@ -269,96 +275,65 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       for (int j = 0; j < nk && ok; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * t, cs & 1u, abort_flag, err));
         if (!ok) break;
+        ++cs;
         tc_fence_after();
-        const bool diag = (j == nk - 1);  // keys after the query are masked
-        const int key0 = j * kTile;
-        // pass 1: the row max, 32 columns per TMEM load, the next load in
-        // flight while the current chunk is scanned
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        // columns c > lim of chunk ch are masked (keys after the query)
-        auto mask_lim = [&](int ch) { return diag ? qi - key0 - 32 * ch : 1 << 30; };
-        auto scan_max = [&](const uint32_t* rr, int ch) {
-          const int lim = mask_lim(ch);
+        // the whole row of S in one round trip; the buffer goes straight back
+        uint32_t sr[kTile];
+        tc_ld32(s_col, sr);
+        tc_ld32(s_col + 32, sr + 32);
+        tc_ld32(s_col + 64, sr + 64);
+        tc_ld32(s_col + 96, sr + 96);
+        tc_wait_ld();
+        tc_fence_before();
+        mbar_arrive(s_empty0 + 8 * t);  // S_t is read: the next S_t may be computed
+        if (j == nk - 1) {  // the diagonal tile: keys after the query are masked
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float v = c > lim ? -INFINITY : __uint_as_float(rr[c]);
-            mx4[c & 3] = fmaxf(mx4[c & 3], v);
-          }
-        };
-        uint32_t ra[32], rb[32];
-        tc_ld32(lane_base + s_col, ra);
-        tc_wait_ld();
-        tc_ld32(lane_base + s_col + 32, rb);
-        scan_max(ra, 0);
-        tc_wait_ld();
-        tc_ld32(lane_base + s_col + 64, ra);
-        scan_max(rb, 1);
-        tc_wait_ld();
-        tc_ld32(lane_base + s_col + 96, rb);
-        scan_max(ra, 2);
-        tc_wait_ld();
-        scan_max(rb, 3);
+          for (int c = 0; c < kTile; ++c)
+            if (c > r) sr[c] = kNegInf;
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(sr[c]));
         const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
-        // the previous product is complete: P is free and O may be rescaled
+        const bool raise = mt > m + kRescaleLog2;  // always on the first key tile
+        const float mn = raise ? mt : m;
+        // P in registers (bf16 pairs) and its row sum
+        uint32_t pk[kTile / 2];
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < kTile / 2; ++c) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), sl2, -mn));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -mn));
+          sum4[(2 * c) & 3] += p0;
+          sum4[(2 * c + 1) & 3] += p1;
+          pk[c] = attn::pack_bf16x2(p0, p1);
+        }
+        // the previous product is complete: P_t is free and O_t may be rescaled
         if (j >= 1) {
           ok = wait_pv();
           if (!ok) break;
           tc_fence_after();
-        }
-        if (mt > m + kRescaleLog2) {
-          if (j >= 1) {  // rescale the row of O and the sum to the new reference
-            const float f = fast_exp2(m - mt);
+          if (raise) {  // rescale the row of O and the sum to the new reference
+            const float f = fast_exp2(m - mn);
             l *= f;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-              tc_ld32(lane_base + o_col + 32 * hf, ra);
+              uint32_t o[32];
+              tc_ld32(o_col + 32 * hf, o);
               tc_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 32; ++c) ra[c] = __float_as_uint(__uint_as_float(ra[c]) * f);
-              attn::tc_st32(lane_base + o_col + 32 * hf, ra);
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+              attn::tc_st32(o_col + 32 * hf, o);
             }
-            attn::tc_wait_st();
           }
-          m = mt;
         }
-        // pass 2: P into the shared-memory tile, row sum
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-        // key columns 32ch .. 32ch+31: box ch / 2, 16-byte chunks 4 (ch % 2) ..
-        auto emit = [&](const uint32_t* rr, int ch) {
-          const int lim = mask_lim(ch);
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            float pv[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int c = 8 * c8 + q;
-              const float v = c > lim ? -INFINITY : __uint_as_float(rr[c]);
-              pv[q] = fast_exp2(fmaf(v, sl2, -m));
-              sum4[q & 3] += pv[q];
-            }
-            attn::st_shared_bf16x8(
-                p_row + (uint32_t)((ch >> 1) * kBox) + ((uint32_t)((4 * (ch & 1) + c8) ^ (r & 7)) << 4),
-                pv);
-          }
-        };
-        tc_ld32(lane_base + s_col, ra);
-        tc_wait_ld();
-        tc_ld32(lane_base + s_col + 32, rb);
-        emit(ra, 0);
-        tc_wait_ld();
-        tc_ld32(lane_base + s_col + 64, ra);
-        emit(rb, 1);
-        tc_wait_ld();
-        tc_ld32(lane_base + s_col + 96, rb);
-        emit(ra, 2);
-        tc_wait_ld();
+        m = mn;
+        attn::tc_st32(p_col, pk);
+        attn::tc_st32(p_col + 32, pk + 32);
+        attn::tc_wait_st();
         tc_fence_before();
-        mbar_arrive(s_empty0 + 8 * t);  // S_t is read: the next S_t may be computed
-        emit(rb, 3);
-        fence_async_smem();
-        mbar_arrive(p_full0 + 8 * t);  // (after the TMEM fence above: O's rescale is ordered too)
+        mbar_arrive(p_full0 + 8 * t);  // P_t (and a rescaled O_t) may be consumed
         l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-        ++cs;
       }
       if (!ok) break;
       // the item's last product, then the normalised output row
@@ -366,8 +341,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       if (!ok) break;
       tc_fence_after();
       uint32_t ra[32], rb[32];
-      tc_ld32(lane_base + o_col, ra);
-      tc_ld32(lane_base + o_col + 32, rb);
+      tc_ld32(o_col, ra);
+      tc_ld32(o_col + 32, rb);
       tc_wait_ld();
       tc_fence_before();  // O is read before the next item's first product overwrites it
       if (qi < T) {

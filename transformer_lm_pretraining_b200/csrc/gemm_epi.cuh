@@ -14,6 +14,7 @@ struct EpiParams {
   const float* bias;
   const act_t* resid; long ldr;
   act_t* aux; long ldaux;
+  int expiry_test;  // GemmArgs::expiry_test
 };
 
 // One output element (any epilogue kind).

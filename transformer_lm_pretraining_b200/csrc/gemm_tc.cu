@@ -205,6 +205,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if (ep.expiry_test > 0 && blockIdx.x == 0 && u == unit0 && kb == kb0 + ep.expiry_test - 1) {
+            // test of the bounded waits: this stage is never filled
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           const uint32_t fb = full0 + 8 * stage;
           const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
@@ -748,7 +756,8 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   else e = make_tmap(&ta, a.A, false, a.M, a.K, a.lda, 64, 64);
   if (e != cudaSuccess) return e;
 
-  EpiParams ep{a.M, a.N, a.alpha, a.out, a.ldo, a.out32, a.ldo32, a.bias, a.resid, a.ldr, a.aux, a.ldaux};
+  EpiParams ep{a.M, a.N, a.alpha, a.out, a.ldo, a.out32, a.ldo32, a.bias, a.resid, a.ldr, a.aux, a.ldaux,
+               a.expiry_test};
   // 256 x 256 tiles over CTA pairs for the wide products (measured: 5-11 %
   // faster where the main loop sets the pace).  The GELU and GELU-backward
   // epilogues set the pace of their products; there the pair waits for the

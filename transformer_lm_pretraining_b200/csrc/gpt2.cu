@@ -70,7 +70,7 @@ struct gpt2 {
   float* scalars = nullptr;
   double* norm_partials = nullptr;
   int* err = nullptr;
-  long t = 0;
+  int* dstep = nullptr;  // the optimizer step counter t, on the device
   // workspace
   void* work = nullptr;
   size_t work_bytes = 0;
@@ -85,6 +85,13 @@ struct gpt2 {
   bool have_logits = false;
   Acts a{};
   std::string last_error;
+  // events recorded after each layer's backward (and the last one after the
+  // embedding's), for callers overlapping gradient communication
+  std::vector<cudaEvent_t> bwd_events;
+  // a captured optimizer step (gpt2_step_graph_capture)
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t graph_exec = nullptr;
+  long graph_launches = 0;
   // profiling
   bool prof = false;
   std::vector<cudaEvent_t> ev_pool;
@@ -108,15 +115,21 @@ gpt2_status cuda_fail(gpt2_t* h, cudaError_t e, const char* where) {
     if (e_ != cudaSuccess) return cuda_fail(h, e_, #call);   \
   } while (0)
 
+// Parameters per buffer, padded with zeros to a multiple of 2048 so that
+// data-parallel ranks (up to 2048 of them, in powers of two) can take equal
+// shards of the flat buffers.
+size_t padded_params(const Layout& lay) { return (lay.total + 2047) / 2048 * 2048; }
+
 // Layout of the state allocation.
 size_t carve_state(const Layout& lay, void* base, gpt2_t* h) {
   Carver c(base);
-  float* params = c.take<float>(lay.total);
-  float* grads = c.take<float>(lay.total);
-  float* m = c.take<float>(lay.total);
-  float* v = c.take<float>(lay.total);
+  const size_t Pp = padded_params(lay);
+  float* params = c.take<float>(Pp);
+  float* grads = c.take<float>(Pp);
+  float* m = c.take<float>(Pp);
+  float* v = c.take<float>(Pp);
 #if GPT2_ACT_BF16
-  act_t* pact = c.take<act_t>(lay.total);
+  act_t* pact = c.take<act_t>(Pp);
 #else
   act_t* pact = params;
 #endif
@@ -126,6 +139,7 @@ size_t carve_state(const Layout& lay, void* base, gpt2_t* h) {
   if (h) {
     h->params = params; h->grads = grads; h->m = m; h->v = v; h->pact = pact;
     h->scalars = scalars; h->norm_partials = np; h->err = err;
+    h->dstep = err + 8;
   }
   return c.used;
 }
@@ -159,7 +173,7 @@ size_t carve_work(const Layout& lay, int B, int T, int recompute, void* base, Ac
   x.datt = c.take<act_t>(M * C);
   x.dqkv = c.take<act_t>(M * 3 * C);
   x.dbig = c.take<act_t>(M * 4 * C);
-  x.dsum = c.take<float>(M * H);
+  x.dsum = c.take<float>(attention_bwd_scratch_floats(B, T, (int)H));
   const size_t part = std::max((size_t)kColsumChunks * 4 * C, (size_t)kLnBlocks * 3 * C);
   x.partials = c.take<float>(part);
   x.splitk_floats = (size_t)kMaxSplits * 4 * C * C;
@@ -292,6 +306,8 @@ void gpt2_destroy(gpt2_t* h) {
   if (h->own_state && h->state) cudaFree(h->state);
   if (h->own_work && h->work) cudaFree(h->work);
   if (h->gen) cudaFree(h->gen);
+  if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+  if (h->graph) cudaGraphDestroy(h->graph);
   std::vector<cudaEvent_t> evs = h->ev_pool;
   for (const ProfRec& r : h->recs) {
     evs.push_back(r.a);
@@ -323,21 +339,18 @@ gpt2_status gpt2_bind_memory(gpt2_t* h, void* dev_state, size_t state_bytes, voi
     h->own_state = false;
     h->state = dev_state;
     h->state_bytes = state_bytes;
-    carve_state(h->lay, dev_state, h);
+    const size_t used = carve_state(h->lay, dev_state, h);
     const size_t P = h->lay.total;
+    // everything zero (gradients, moments, the zero padding of every buffer,
+    // scalars, error word, step counter), then the seeded parameters
+    GPT2_CUDA(h, cudaMemsetAsync(dev_state, 0, used, h->stream));
     init_params(h->params, h->lay, h->seed, h->stream);
     GPT2_CUDA(h, cudaGetLastError());
-    GPT2_CUDA(h, cudaMemsetAsync(h->grads, 0, P * sizeof(float), h->stream));
-    GPT2_CUDA(h, cudaMemsetAsync(h->m, 0, P * sizeof(float), h->stream));
-    GPT2_CUDA(h, cudaMemsetAsync(h->v, 0, P * sizeof(float), h->stream));
-    GPT2_CUDA(h, cudaMemsetAsync(h->scalars, 0, S_COUNT * sizeof(float), h->stream));
     reset_clip(h->scalars, h->stream);
-    GPT2_CUDA(h, cudaMemsetAsync(h->err, 0, 16 * sizeof(int), h->stream));
 #if GPT2_ACT_BF16
     f32_to_act(h->pact, h->params, P, h->stream);
     GPT2_CUDA(h, cudaGetLastError());
 #endif
-    h->t = 0;
     h->have_grad_logits = h->have_logits = false;
   }
   if (dev_work) {
@@ -794,10 +807,12 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
                   P + y.off[T_LN1G] + (size_t)l * C, G + y.off[T_LN1G] + (size_t)l * C,
                   G + y.off[T_LN1B] + (size_t)l * C,
                   l > 0 ? G + y.off[T_BP] + (size_t)(l - 1) * C : nullptr, a.partials, M, C, 1, s);
+    if (!h->bwd_events.empty()) GPT2_CUDA(h, cudaEventRecord(h->bwd_events[l], s));
   }
   mark(h, PK_ENCODER);
   encoder_bwd(G + y.off[T_WTE], G + y.off[T_WPE], a.dres, a.tok, B, T, C, y.Vp, es, s);
   mark_end(h);
+  if (!h->bwd_events.empty()) GPT2_CUDA(h, cudaEventRecord(h->bwd_events[L], s));
   GPT2_CUDA(h, cudaGetLastError());
   h->have_grad_logits = false;
   return GPT2_OK;
@@ -822,24 +837,173 @@ gpt2_status gpt2_grad_norm_clip(gpt2_t* h, float max_norm, float* norm_host) {
   return GPT2_OK;
 }
 
-gpt2_status gpt2_adamw_step(gpt2_t* h, float lr, float beta1, float beta2, float eps,
-                            float weight_decay) {
+}  // extern "C"
+
+namespace {
+
+// One AdamW step: the device step counter advances, the step's learning
+// rate (given, or from the schedule on the device) and bias corrections
+// land in device scalars, then the fused update runs.
+gpt2_status adamw_impl(gpt2_t* h, float lr, const double* sched, float beta1, float beta2,
+                       float eps, float weight_decay, size_t begin = 0, size_t end = (size_t)-1) {
   if (!h) return GPT2_ERR_ARG;
   gpt2_status st = ensure_state(h);
   if (st) return st;
-  h->t += 1;
+  if (end > h->lay.total) end = h->lay.total;
   AdamArgs a;
-  a.lr = lr; a.b1 = beta1; a.b2 = beta2; a.eps = eps; a.wd = weight_decay;
-  a.bc1 = (float)(1.0 - std::pow((double)beta1, (double)h->t));
-  a.bc2 = (float)(1.0 - std::pow((double)beta2, (double)h->t));
+  a.b1 = beta1; a.b2 = beta2; a.eps = eps; a.wd = weight_decay;
   mark(h, PK_OPTIMIZER);
-  adamw(h->params, h->pact, h->grads, h->m, h->v, h->lay, a, h->scalars, h->stream);
+  adam_prep(h->scalars, h->dstep, lr, sched != nullptr, sched, beta1, beta2, h->stream);
+  adamw(h->params, h->pact, h->grads, h->m, h->v, h->lay, a, h->scalars, h->stream, begin, end);
   GPT2_CUDA(h, cudaGetLastError());
   reset_clip(h->scalars, h->stream);  // the clip scale applies to one step only
   mark_end(h);
   GPT2_CUDA(h, cudaGetLastError());
   return GPT2_OK;
 }
+
+}  // namespace
+
+extern "C" {
+
+gpt2_status gpt2_adamw_step(gpt2_t* h, float lr, float beta1, float beta2, float eps,
+                            float weight_decay) {
+  return adamw_impl(h, lr, nullptr, beta1, beta2, eps, weight_decay);
+}
+
+gpt2_status gpt2_adamw_step_scheduled(gpt2_t* h, double max_lr, double min_lr, long warmup,
+                                      long max_steps, float beta1, float beta2, float eps,
+                                      float weight_decay) {
+  if (warmup < 1 || max_steps < 0) return fail(h, GPT2_ERR_ARG, "bad schedule");
+  const double sched[4] = {max_lr, min_lr, (double)warmup, (double)max_steps};
+  return adamw_impl(h, 0.f, sched, beta1, beta2, eps, weight_decay);
+}
+
+gpt2_status gpt2_adamw_step_range(gpt2_t* h, float lr, float beta1, float beta2, float eps,
+                                  float weight_decay, size_t begin, size_t end) {
+  if (!h || begin > end || (begin & 3) || (end < h->lay.total && ((end - begin) & 3)))
+    return fail(h, GPT2_ERR_ARG, "AdamW range: begin and length must be multiples of 4");
+  return adamw_impl(h, lr, nullptr, beta1, beta2, eps, weight_decay, begin, end);
+}
+
+size_t gpt2_padded_params(const gpt2_t* h) { return h ? padded_params(h->lay) : 0; }
+
+gpt2_status gpt2_grad_sumsq(gpt2_t* h, size_t begin, size_t end, double* sumsq_dev) {
+  if (!h || !sumsq_dev || begin > end) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  if (end > padded_params(h->lay)) return fail(h, GPT2_ERR_ARG, "range past the padded buffer");
+  if ((begin & 3) || (reinterpret_cast<uintptr_t>(sumsq_dev) & 7))
+    return fail(h, GPT2_ERR_ARG, "begin must be a multiple of 4, sumsq_dev 8-byte aligned");
+  mark(h, PK_OPTIMIZER);
+  grad_sumsq(sumsq_dev, h->grads + begin, end - begin, h->norm_partials, h->stream);
+  mark_end(h);
+  GPT2_CUDA(h, cudaGetLastError());
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_clip_from_sumsq(gpt2_t* h, const double* sumsq_dev, float max_norm,
+                                 float* norm_host) {
+  if (!h || !sumsq_dev) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  clip_from_sumsq(h->scalars, sumsq_dev, max_norm, h->stream);
+  GPT2_CUDA(h, cudaGetLastError());
+  if (norm_host) {
+    GPT2_CUDA(h, cudaMemcpyAsync(norm_host, h->scalars + S_NORM, sizeof(float),
+                                 cudaMemcpyDeviceToHost, h->stream));
+    st = check_err_word(h);
+    if (st) return st;
+    if (!std::isfinite(*norm_host))
+      return fail(h, GPT2_ERR_NONFINITE, "gradient norm is not finite");
+  }
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_params_device(gpt2_t* h, float** dev_ptr) {
+  if (!h || !dev_ptr) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  *dev_ptr = h->params;
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_refresh_weights(gpt2_t* h) {
+  if (!h) return GPT2_ERR_ARG;
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+#if GPT2_ACT_BF16
+  f32_to_act(h->pact, h->params, h->lay.total, h->stream);
+  GPT2_CUDA(h, cudaGetLastError());
+#endif
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_set_backward_events(gpt2_t* h, void* const* events, int n) {
+  if (!h || n < 0 || (n > 0 && !events)) return GPT2_ERR_ARG;
+  if (n && n != h->lay.L + 1) return fail(h, GPT2_ERR_ARG, "backward events: n must be L + 1 or 0");
+  h->bwd_events.clear();
+  for (int i = 0; i < n; ++i) h->bwd_events.push_back(static_cast<cudaEvent_t>(events[i]));
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_step_graph_capture(gpt2_t* h, const int32_t* tok_dev, const int32_t* tgt_dev,
+                                    int B, int T, int n_micro, float max_norm, double max_lr,
+                                    double min_lr, long warmup, long max_steps, float beta1,
+                                    float beta2, float eps, float weight_decay) {
+  if (!h || !tok_dev || !tgt_dev || B < 1 || T < 1 || n_micro < 1 || warmup < 1)
+    return fail(h, GPT2_ERR_ARG, "bad step-graph arguments");
+  if (!h->stream) return fail(h, GPT2_ERR_STATE, "capturing needs a stream set by gpt2_set_stream");
+  if (h->prof) return fail(h, GPT2_ERR_STATE, "capturing with profiling on");
+  if (!h->bwd_events.empty()) return fail(h, GPT2_ERR_STATE, "capturing with backward events set");
+  if (T > h->lay.Tmax) return fail(h, GPT2_ERR_ARG, "T > Tmax");
+  gpt2_status st = ensure_state(h);
+  if (st) return st;
+  st = ensure_work(h, B, T);  // no allocation may happen while capturing
+  if (st) return st;
+  if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+  if (h->graph) cudaGraphDestroy(h->graph);
+  h->graph_exec = nullptr;
+  h->graph = nullptr;
+  const long n0 = launch_count();
+  GPT2_CUDA(h, cudaStreamBeginCapture(h->stream, cudaStreamCaptureModeThreadLocal));
+  const size_t M = (size_t)B * T;
+  st = gpt2_zero_grad(h);
+  for (int i = 0; i < n_micro && !st; ++i) {
+    st = forward_impl(h, tok_dev + i * M, tgt_dev + i * M, B, T, nullptr, true);
+    if (!st) st = gpt2_backward(h, 1.0f / (float)n_micro);
+  }
+  if (!st) st = gpt2_grad_norm_clip(h, max_norm, nullptr);
+  if (!st)
+    st = gpt2_adamw_step_scheduled(h, max_lr, min_lr, warmup, max_steps, beta1, beta2, eps,
+                                   weight_decay);
+  cudaGraph_t g = nullptr;
+  const cudaError_t ec = cudaStreamEndCapture(h->stream, &g);
+  if (st) {
+    if (g) cudaGraphDestroy(g);
+    return st;
+  }
+  if (ec != cudaSuccess) return cuda_fail(h, ec, "cudaStreamEndCapture");
+  cudaGraphExec_t ex = nullptr;
+  const cudaError_t ei = cudaGraphInstantiate(&ex, g, 0);
+  if (ei != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return cuda_fail(h, ei, "cudaGraphInstantiate");
+  }
+  h->graph = g;
+  h->graph_exec = ex;
+  h->graph_launches = launch_count() - n0;
+  return GPT2_OK;
+}
+
+gpt2_status gpt2_step_graph_launch(gpt2_t* h) {
+  if (!h) return GPT2_ERR_ARG;
+  if (!h->graph_exec) return fail(h, GPT2_ERR_STATE, "no captured step");
+  GPT2_CUDA(h, cudaGraphLaunch(h->graph_exec, h->stream));
+  return GPT2_OK;
+}
+
+long gpt2_step_graph_kernels(const gpt2_t* h) { return h ? h->graph_launches : 0; }
 
 double gpt2_lr(long step, double max_lr, double min_lr, long warmup, long max_steps) {
   if (step < warmup) return max_lr * (double)(step + 1) / (double)warmup;
@@ -898,13 +1062,15 @@ gpt2_status gpt2_get_state(const gpt2_t* hc, float* params, float* m, float* v, 
   if (params) GPT2_CUDA(h, cudaMemcpyAsync(params, h->params, n, cudaMemcpyDeviceToHost, h->stream));
   if (m) GPT2_CUDA(h, cudaMemcpyAsync(m, h->m, n, cudaMemcpyDeviceToHost, h->stream));
   if (v) GPT2_CUDA(h, cudaMemcpyAsync(v, h->v, n, cudaMemcpyDeviceToHost, h->stream));
-  if (t) *t = h->t;
+  int ti = 0;
+  GPT2_CUDA(h, cudaMemcpyAsync(&ti, h->dstep, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
   GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
+  if (t) *t = ti;
   return GPT2_OK;
 }
 
 gpt2_status gpt2_set_state(gpt2_t* h, const float* params, const float* m, const float* v, long t) {
-  if (!h || t < 0) return GPT2_ERR_ARG;
+  if (!h || t < 0 || t > 0x7fffffffL) return GPT2_ERR_ARG;
   gpt2_status st = ensure_state(h);
   if (st) return st;
   const size_t n = h->lay.total * 4;
@@ -917,7 +1083,8 @@ gpt2_status gpt2_set_state(gpt2_t* h, const float* params, const float* m, const
   }
   if (m) GPT2_CUDA(h, cudaMemcpyAsync(h->m, m, n, cudaMemcpyHostToDevice, h->stream));
   if (v) GPT2_CUDA(h, cudaMemcpyAsync(h->v, v, n, cudaMemcpyHostToDevice, h->stream));
-  h->t = t;
+  const int ti = (int)t;
+  GPT2_CUDA(h, cudaMemcpyAsync(h->dstep, &ti, sizeof(int), cudaMemcpyHostToDevice, h->stream));
   GPT2_CUDA(h, cudaStreamSynchronize(h->stream));
   return GPT2_OK;
 }

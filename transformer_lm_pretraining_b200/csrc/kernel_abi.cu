@@ -49,6 +49,22 @@ int gpt2k_gemm(void* stream, int epi, int M, int N, int K, const void* A, long l
   return status(gemm(g, static_cast<cudaStream_t>(stream), err));
 }
 
+int gpt2k_gemm_expiry_test(void* stream, int M, int N, int K, const void* A, const void* B,
+                           void* out, int kblock) {
+  if (M < 1 || N < 1 || K < 1 || kblock < 0 || kblock >= (K + 63) / 64) return GPT2_ERR_ARG;
+  int* err = err_word();
+  if (!err) return GPT2_ERR_CUDA;
+  GemmArgs g{};
+  g.M = M; g.N = N; g.K = K;
+  g.A = static_cast<const act_t*>(A); g.lda = K;
+  g.B = static_cast<const act_t*>(B); g.ldb = K;
+  g.epi = EPI_STORE; g.alpha = 1.f;
+  g.out = static_cast<act_t*>(out); g.ldo = N;
+  g.max_splits = 1;
+  g.expiry_test = kblock + 1;
+  return status(gemm(g, static_cast<cudaStream_t>(stream), err));
+}
+
 int gpt2k_attention_fwd(void* stream, void* att, float* lse, const void* qkv, int B, int T, int C,
                         int H) {
   if (B < 1 || T < 1 || H < 1 || C % H) return GPT2_ERR_ARG;
@@ -56,6 +72,11 @@ int gpt2k_attention_fwd(void* stream, void* att, float* lse, const void* qkv, in
   if (!err) return GPT2_ERR_CUDA;
   return status(attention_fwd(static_cast<act_t*>(att), lse, static_cast<const act_t*>(qkv), B, T,
                               C, H, err, static_cast<cudaStream_t>(stream)));
+}
+
+size_t gpt2k_attention_bwd_scratch(int B, int T, int H) {
+  if (B < 1 || T < 1 || H < 1) return 0;
+  return attention_bwd_scratch_floats(B, T, H);
 }
 
 int gpt2k_attention_bwd(void* stream, void* dqkv, float* dsum, const void* datt, const void* qkv,

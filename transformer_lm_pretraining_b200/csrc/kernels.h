@@ -50,6 +50,11 @@ struct GemmArgs {
   // split-K (EPI_F32_ACC only): partial sums go to split_ws, then a
   // fixed-order reduction adds them into out32.  max_splits = 1 disables.
   float* split_ws; size_t split_ws_floats; int max_splits;
+  // Test of the bounded waits only: n > 0 makes CTA 0's producer skip the
+  // load of k-block n - 1 of its first tile, so that the MMA's wait for it
+  // expires (error word ERR_TIMEOUT) and the kernel takes its abort path.
+  // 0 (the value of a zero-initialised GemmArgs) in every product call.
+  int expiry_test;
 };
 
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err_flag);
@@ -103,13 +108,18 @@ cudaError_t attention_fwd(act_t* att, float* lse, const act_t* qkv, int B, int T
 bool attention_fwd_tc_supported(int C, int H);
 cudaError_t attention_fwd_tc(act_t* att, float* lse, const act_t* qkv, int B, int T, int C, int H,
                              int* err, cudaStream_t s);
-// dqkv [B*T, 3C] (overwritten); dsum [B, H, T] scratch.
+// dqkv [B*T, 3C] (overwritten); dsum: fp32 scratch of
+// attention_bwd_scratch_floats(B, T, H) floats, 16-byte aligned.
+size_t attention_bwd_scratch_floats(int B, int T, int H);
 cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
                           const act_t* att, const float* lse, int B, int T, int C, int H,
                           int* err, cudaStream_t s);
-// tcgen05 backward (head dim 64; bf16 build); it writes D = rowsum(dO * O)
-// (B*H*T floats) to dsum itself, from datt and the forward's output att
-cudaError_t attention_bwd_tc(act_t* dqkv, float* dsum, const act_t* datt, const act_t* qkv,
+// tcgen05 backward (head dim 64; bf16 build); it forms D = rowsum(dO * O)
+// itself, from datt and the forward's output att, and keeps the per-row
+// (L log2 e, D) pairs in `scratch` (attention_bwd_tc_scratch_floats floats:
+// B*H rows of T rounded up to 128 pairs)
+size_t attention_bwd_tc_scratch_floats(int B, int T, int H);
+cudaError_t attention_bwd_tc(act_t* dqkv, float* scratch, const act_t* datt, const act_t* qkv,
                              const act_t* att, const float* lse, int B, int T, int C, int H,
                              int* err, cudaStream_t s);
 
@@ -148,7 +158,7 @@ void f32_to_act(act_t* out, const float* in, size_t n, cudaStream_t s);
 void act_to_f32(float* out, const act_t* in, size_t n, cudaStream_t s);
 
 // scalars layout (device floats)
-enum Scalar { S_NORM = 0, S_CLIP = 1, S_LOSS = 2, S_COUNT = 16 };
+enum Scalar { S_NORM = 0, S_CLIP = 1, S_LOSS = 2, S_LR = 3, S_BC1 = 4, S_BC2 = 5, S_COUNT = 16 };
 constexpr int kNormBlocks = 592;
 // scalars[S_NORM] = ||g||_2, scalars[S_CLIP] = max_norm / (norm + 1e-6) or 1
 void grad_norm_clip(float* scalars, const float* g, size_t n, float max_norm, double* partials,
@@ -158,12 +168,24 @@ void grad_norm_clip(float* scalars, const float* g, size_t n, float max_norm, do
 void reset_clip(float* scalars, cudaStream_t s);
 
 struct AdamArgs {
-  float lr, b1, b2, eps, wd;
-  float bc1, bc2;  // 1 - b1^t, 1 - b2^t
+  float b1, b2, eps, wd;  // the learning rate and bias corrections are device scalars
 };
+
+// The optimizer step counter and its learning rate, on the device: t =
+// ++*step; scalars[S_LR] = lr, or with `scheduled` the warmup-then-cosine
+// schedule lr(t - 1) (sched = {max_lr, min_lr, warmup, max_steps});
+// scalars[S_BC1] = 1 - b1^t, scalars[S_BC2] = 1 - b2^t.
+void adam_prep(float* scalars, int* step, float lr, bool scheduled, const double* sched, float b1,
+               float b2, cudaStream_t s);
 // Decay applies to the tensors flagged in `decay_mask` (bit per tensor).
+// over the flat parameter range [begin, end) (begin and end - begin multiples
+// of 4 unless end is the total)
 void adamw(float* p, act_t* pact, const float* g, float* m, float* v, const Layout& lay,
-           const AdamArgs& a, const float* scalars, cudaStream_t s);
+           const AdamArgs& a, const float* scalars, cudaStream_t s, size_t begin, size_t end);
+// *out = sum of g[i]^2 over n elements (fixed-order two-stage reduction in double)
+void grad_sumsq(double* out, const float* g, size_t n, double* partials, cudaStream_t s);
+// scalars[S_NORM] = sqrt(*sumsq), scalars[S_CLIP] as grad_norm_clip
+void clip_from_sumsq(float* scalars, const double* sumsq, float max_norm, cudaStream_t s);
 
 // Process-wide count of kernel launches made by this library.
 void note_launch(int n = 1);

@@ -8,6 +8,7 @@
 // and summed over blocks in block order: no atomics, fixed summation order.
 
 #include "kernels.h"
+#include "tc_util.cuh"
 
 namespace gpt2k {
 
@@ -69,6 +70,166 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// 8 activations as loaded (16 bytes in the bf16 build): rows are kept in
+// this form and converted where used.
+struct alignas(16) Pack8 {
+  act_t v[8];
+};
+
+// Rows staged through shared memory by bulk copies: TEAMS teams of TPR
+// threads per block, one row per team at a time, 8 columns per thread.  One
+// thread of each team keeps D of the team's next rows in flight (one
+// cp.async.bulk per row tensor, completing on the slot's mbarrier), so the
+// bytes in flight do not depend on registers; the team reads a row from its
+// slot, and the slot is refilled once every thread of the team has passed
+// the team's named barrier (or, for one-warp rows, its __syncwarp).  Row
+// sums go through a warp shuffle and, across the team's warps, shared memory
+// behind the named barrier: no block-wide barrier in the row loop.
+template <int TPR>
+constexpr int ln_teams() {
+  return TPR >= 256 ? 2 : (768 / TPR > 8 ? 8 : 768 / TPR);
+}
+constexpr int kLnStages = 4;  // rows in flight per team
+
+// Bounded wait for the bulk copies of a slot: the copies always complete, so
+// the limit only guards against a broken device; after it the row is
+// processed with whatever the slot holds and the kernel still ends.
+__device__ __forceinline__ void ln_slot_wait(uint32_t bar, uint32_t parity) {
+  if (tc::mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = tc::global_ns();
+  while (!tc::mbar_try_wait(bar, parity))
+    if (tc::global_ns() - t0 > tc::kWaitLimitNs) return;
+}
+
+// Chan, Golub & LeVeque (1979), parallel variance: parts a, b of sizes na, nb
+// with means ma, mb and squared-deviation sums Sa, Sb form a union of mean
+// ma + d nb / n and sum Sa + Sb + d^2 na nb / n, d = mb - ma.  For equal
+// sizes, written symmetrically so that both partners of a butterfly step get
+// the same bits.
+__device__ __forceinline__ void chan_merge(float& mean, float& m2, float n, float mean_b, float m2_b) {
+  const float d = mean_b - mean;
+  mean = 0.5f * (mean + mean_b);
+  m2 = (m2 + m2_b) + d * d * (0.5f * n);
+}
+
+template <int TPR>
+__global__ void __launch_bounds__(TPR * ln_teams<TPR>())
+    ln_fwd_staged_kernel(act_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
+                         const act_t* __restrict__ x, const float* __restrict__ g,
+                         const float* __restrict__ b, int M) {
+  constexpr int TEAMS = ln_teams<TPR>();
+  constexpr int WPR = TPR / 32;
+  constexpr int C = 8 * TPR;
+  constexpr uint32_t kRowBytes = C * sizeof(act_t);
+  extern __shared__ __align__(128) uint8_t ln_smem[];
+  act_t* ring = reinterpret_cast<act_t*>(ln_smem);  // [TEAMS][kLnStages][C]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ln_smem + (size_t)TEAMS * kLnStages * kRowBytes);
+  __shared__ float red[TEAMS][2][WPR][2];
+  const int team = threadIdx.x / TPR, tc = threadIdx.x % TPR;
+  const int wr = tc / 32, lane = threadIdx.x & 31;
+  const int c = tc * 8;
+  const int stride = gridDim.x * TEAMS;
+  const int row0 = blockIdx.x * TEAMS + team;
+  const uint32_t bar0 = tc::smem_u32(bars + team * kLnStages);
+  const uint32_t slot0 = tc::smem_u32(ring + (size_t)team * kLnStages * C);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < TEAMS * kLnStages; ++i) tc::mbar_init(tc::smem_u32(bars + i), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto issue = [&](int k) {  // row k of this team into slot k % kLnStages
+    const int row = row0 + k * stride;
+    if (row >= M) return;
+    const uint32_t bar = bar0 + 8 * (k % kLnStages);
+    tc::mbar_expect_tx(bar, kRowBytes);
+    tc::bulk_load_1d(slot0 + (uint32_t)(k % kLnStages) * kRowBytes, x + (size_t)row * C, kRowBytes,
+                     bar);
+  };
+  if (tc == 0)
+    for (int k = 0; k < kLnStages; ++k) issue(k);
+  float gg[8], bb[8];
+  load8(g + c, gg);
+  load8(b + c, bb);
+  for (int k = 0;; ++k) {
+    const int row = row0 + k * stride;
+    if (row >= M) break;  // uniform over the team
+    const int st = k % kLnStages;
+    ln_slot_wait(bar0 + 8 * st, (uint32_t)(k / kLnStages) & 1u);
+    float v[8];
+    load8(ring + ((size_t)team * kLnStages + st) * C + c, v);
+    float mu = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mu += v[i];
+    mu *= 0.125f;
+    float m2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m2 = fmaf(v[i] - mu, v[i] - mu, m2);
+    float n = 8.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {  // pairwise merges over the warp
+      const float mb = __shfl_xor_sync(0xffffffffu, mu, o);
+      const float sb = __shfl_xor_sync(0xffffffffu, m2, o);
+      chan_merge(mu, m2, n, mb, sb);
+      n *= 2.f;
+    }
+    if (WPR > 1) {  // the team's warps, merged in warp order
+      float* rr = &red[team][k & 1][0][0];
+      if (lane == 0) {
+        rr[2 * wr] = mu;
+        rr[2 * wr + 1] = m2;
+      }
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "n"(TPR) : "memory");
+      mu = rr[0];
+      m2 = rr[1];
+      float na = 256.f;
+#pragma unroll
+      for (int w = 1; w < WPR; ++w) {
+        const float d = rr[2 * w] - mu;
+        const float nn = na + 256.f;
+        mu = fmaf(d, 256.f / nn, mu);
+        m2 = m2 + rr[2 * w + 1] + d * d * (na * 256.f / nn);
+        na = nn;
+      }
+    } else {
+      __syncwarp();
+    }
+    if (tc == 0) issue(k + kLnStages);  // every thread of the team has read the slot
+    const float rs = rsqrtf(m2 * (1.0f / C) + kLnEps);
+    Pack8 q;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q.v[i] = from_f<act_t>(fmaf((v[i] - mu) * rs, gg[i], bb[i]));
+    *reinterpret_cast<Pack8*>(y + (size_t)row * C + c) = q;
+    if (tc == 0) {
+      mean[row] = mu;
+      rstd[row] = rs;
+    }
+  }
+}
+
+template <int TPR>
+constexpr size_t ln_fwd_smem() {
+  return (size_t)ln_teams<TPR>() * kLnStages * (8 * TPR * sizeof(act_t) + 8);
+}
+
+template <int TPR>
+void ln_fwd_staged_launch(act_t* y, float* mean, float* rstd, const act_t* x, const float* g,
+                          const float* b, int M, cudaStream_t s) {
+  constexpr int threads = TPR * ln_teams<TPR>();
+  constexpr size_t smem = ln_fwd_smem<TPR>();
+  static int grid = 0;
+  if (!grid) {
+    cudaFuncSetAttribute(ln_fwd_staged_kernel<TPR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    int per_sm = 0, sms = 0, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_fwd_staged_kernel<TPR>, threads, smem);
+    grid = per_sm * sms;
+    if (grid < 1) grid = sms;
+  }
+  ln_fwd_staged_kernel<TPR><<<grid, threads, smem, s>>>(y, mean, rstd, x, g, b, M);
+}
+
 // grid = nblk blocks of 8 warps; warp w of block blk handles rows
 // (blk * 8 + w) + k * (nblk * 8).  partials[blk][0][..C) = dgamma,
 // [1] = dbeta, [2] = column sums of the written dres (when NSUMS == 3).
@@ -76,11 +237,6 @@ __global__ void __launch_bounds__(256)
 // warp (each lane owns its columns, so no two threads touch the same word),
 // which keeps the row loop's register footprint small enough for several
 // blocks per SM.
-// 8 activations as loaded (16 bytes in the bf16 build): rows are kept in
-// this form and converted where used.
-struct alignas(16) Pack8 {
-  act_t v[8];
-};
 
 template <int kChunks, int NSUMS>
 __global__ void __launch_bounds__(256, 2)
@@ -168,123 +324,160 @@ __global__ void __launch_bounds__(256, 2)
   }
 }
 
-// Row-group variant for C = 8 * TPR with TPR (threads per row) a multiple
-// of 32: a block takes RPB rows at a time, TPR threads to a row and 8
-// columns to a thread, so every thread keeps the three column sums of its 8
-// columns in registers across all its rows, and gamma in registers too.
-// The two row reductions go through a warp shuffle and, across the row's
-// warps, shared memory (one barrier per group of rows, double-buffered).
-// The next group's rows are loaded while the current one is computed.
-// partials[blk][0..NSUMS) as the per-warp kernel.
+// The backward with the same staging as ln_fwd_staged_kernel: a slot holds
+// the row of x, of dy and (when accumulating) of dres, brought by one bulk
+// copy each; mean and rstd of the next rows are loaded into registers ahead.
+// Every thread keeps the column sums of its 8 columns (and gamma) in
+// registers across its rows.  partials[blk][0..NSUMS) as the per-warp
+// kernel (teams added in team order).
+template <int TPR>
+constexpr int ln_bwd_teams() {
+  return TPR >= 256 ? 2 : (384 / TPR > 8 ? 8 : 384 / TPR);
+}
+
 template <int TPR, int NSUMS>
-__global__ void __launch_bounds__(TPR * (TPR >= 256 ? 1 : 256 / TPR), 2)
-    ln_bwd_rows_kernel(act_t* __restrict__ dres, const act_t* __restrict__ dy,
-                       const act_t* __restrict__ x, const float* __restrict__ mean,
-                       const float* __restrict__ rstd, const float* __restrict__ g,
-                       float* __restrict__ partials, int M, int accumulate) {
-  constexpr int RPB = TPR >= 256 ? 1 : 256 / TPR;  // rows per group
-  constexpr int WPR = TPR / 32;                      // warps per row
+__global__ void __launch_bounds__(TPR * ln_bwd_teams<TPR>())
+    ln_bwd_staged_kernel(act_t* __restrict__ dres, const act_t* __restrict__ dy,
+                         const act_t* __restrict__ x, const float* __restrict__ mean,
+                         const float* __restrict__ rstd, const float* __restrict__ g,
+                         float* __restrict__ partials, int M, int accumulate) {
+  constexpr int TEAMS = ln_bwd_teams<TPR>();
+  constexpr int WPR = TPR / 32;
   constexpr int C = 8 * TPR;
-  __shared__ float red[2][RPB][WPR][2];
-  extern __shared__ float sums[];  // [RPB][NSUMS][C] at the end
-  const int slot = threadIdx.x / TPR, tc = threadIdx.x % TPR;
+  constexpr uint32_t kRowBytes = C * sizeof(act_t);
+  constexpr uint32_t kSlotBytes = 3 * kRowBytes;  // x | dy | dres
+  extern __shared__ __align__(128) uint8_t ln_smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ln_smem + (size_t)TEAMS * kLnStages * kSlotBytes);
+  float* sums = reinterpret_cast<float*>(bars + TEAMS * kLnStages);  // [TEAMS][NSUMS][C] at the end
+  __shared__ float red[TEAMS][2][WPR][2];
+  const int team = threadIdx.x / TPR, tc = threadIdx.x % TPR;
   const int wr = tc / 32, lane = threadIdx.x & 31;
   const int c = tc * 8;
-  const int stride = gridDim.x * RPB;
+  const int stride = gridDim.x * TEAMS;
+  const int row0 = blockIdx.x * TEAMS + team;
+  const uint32_t bar0 = tc::smem_u32(bars + team * kLnStages);
+  uint8_t* slots = ln_smem + (size_t)team * kLnStages * kSlotBytes;
+  const uint32_t slot0 = tc::smem_u32(slots);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < TEAMS * kLnStages; ++i) tc::mbar_init(tc::smem_u32(bars + i), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  auto issue = [&](int k) {  // row k of this team into slot k % kLnStages
+    const int row = row0 + k * stride;
+    if (row >= M) return;
+    const uint32_t bar = bar0 + 8 * (k % kLnStages);
+    const uint32_t dst = slot0 + (uint32_t)(k % kLnStages) * kSlotBytes;
+    tc::mbar_expect_tx(bar, accumulate ? 3 * kRowBytes : 2 * kRowBytes);
+    tc::bulk_load_1d(dst, x + (size_t)row * C, kRowBytes, bar);
+    tc::bulk_load_1d(dst + kRowBytes, dy + (size_t)row * C, kRowBytes, bar);
+    if (accumulate) tc::bulk_load_1d(dst + 2 * kRowBytes, dres + (size_t)row * C, kRowBytes, bar);
+  };
+  if (tc == 0)
+    for (int k = 0; k < kLnStages; ++k) issue(k);
   float gg[8], s0[8], s1[8], s2[8];
   load8(g + c, gg);
 #pragma unroll
   for (int i = 0; i < 8; ++i) s0[i] = s1[i] = s2[i] = 0.f;
-  Pack8 px, pd, po;
-  float mu = 0.f, rs = 0.f;
-  auto fetch = [&](int row) {
-    if (row >= M) return;
-    px = *reinterpret_cast<const Pack8*>(x + (size_t)row * C + c);
-    pd = *reinterpret_cast<const Pack8*>(dy + (size_t)row * C + c);
-    if (accumulate) po = *reinterpret_cast<const Pack8*>(dres + (size_t)row * C + c);
-    mu = mean[row];
-    rs = rstd[row];
-  };
-  int row = blockIdx.x * RPB + slot;
-  fetch(row);
-  for (int it = 0; blockIdx.x * RPB + it * stride < M; ++it, row += stride) {
-    const Pack8 cx = px, cd = pd, co = po;
-    const float crs = rs, nmr = -mu * rs;
-    const bool live = row < M;
-    fetch(row + stride);  // in flight while this group is computed
-    float xh[8], dxh[8], a = 0.f, b = 0.f;
+  // mean and rstd one row ahead
+  float mu_n = 0.f, rs_n = 0.f;
+  if (row0 < M) {
+    mu_n = mean[row0];
+    rs_n = rstd[row0];
+  }
+  for (int k = 0;; ++k) {
+    const int row = row0 + k * stride;
+    if (row >= M) break;  // uniform over the team
+    const float crs = rs_n, nmr = -mu_n * rs_n;
+    if (row + stride < M) {
+      mu_n = mean[row + stride];
+      rs_n = rstd[row + stride];
+    }
+    const int st = k % kLnStages;
+    ln_slot_wait(bar0 + 8 * st, (uint32_t)(k / kLnStages) & 1u);
+    const uint8_t* slot = slots + (size_t)st * kSlotBytes;
+    const Pack8 cx = *reinterpret_cast<const Pack8*>(slot + c * sizeof(act_t));
+    const Pack8 cd = *reinterpret_cast<const Pack8*>(slot + kRowBytes + c * sizeof(act_t));
+    Pack8 co;
+    if (accumulate) co = *reinterpret_cast<const Pack8*>(slot + 2 * kRowBytes + c * sizeof(act_t));
+    float xh[8], dxh[8], a = 0.f, bsum = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       xh[i] = fmaf(to_f(cx.v[i]), crs, nmr);
-      const float d = live ? to_f(cd.v[i]) : 0.f;
+      const float d = to_f(cd.v[i]);
       dxh[i] = d * gg[i];
       a += dxh[i];
-      b = fmaf(dxh[i], xh[i], b);
+      bsum = fmaf(dxh[i], xh[i], bsum);
       s0[i] = fmaf(d, xh[i], s0[i]);
       s1[i] += d;
     }
     a = warp_sum(a);
-    b = warp_sum(b);
-    float* rr = &red[it & 1][slot][0][0];
-    if (lane == 0) {
-      rr[2 * wr] = a;
-      rr[2 * wr + 1] = b;
-    }
-    __syncthreads();
-    a = 0.f;
-    b = 0.f;
-#pragma unroll
-    for (int w = 0; w < WPR; ++w) {
-      a += rr[2 * w];
-      b += rr[2 * w + 1];
-    }
-    a *= 1.0f / C;
-    b *= 1.0f / C;
-    if (live) {
-      Pack8 q;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float t = fmaf(-xh[i], b, dxh[i] - a);
-        const float o = accumulate ? fmaf(crs, t, to_f(co.v[i])) : crs * t;
-        q.v[i] = from_f<act_t>(o);
-        if (NSUMS == 3) s2[i] += to_f(q.v[i]);  // the bias gradient sums the values as stored
+    bsum = warp_sum(bsum);
+    if (WPR > 1) {
+      float* rr = &red[team][k & 1][0][0];
+      if (lane == 0) {
+        rr[2 * wr] = a;
+        rr[2 * wr + 1] = bsum;
       }
-      *reinterpret_cast<Pack8*>(dres + (size_t)row * C + c) = q;
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "n"(TPR) : "memory");
+      a = 0.f;
+      bsum = 0.f;
+#pragma unroll
+      for (int w = 0; w < WPR; ++w) {
+        a += rr[2 * w];
+        bsum += rr[2 * w + 1];
+      }
+    } else {
+      __syncwarp();
     }
+    if (tc == 0) issue(k + kLnStages);  // every thread of the team has read the slot
+    a *= 1.0f / C;
+    bsum *= 1.0f / C;
+    Pack8 q;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float t = fmaf(-xh[i], bsum, dxh[i] - a);
+      const float o = accumulate ? fmaf(crs, t, to_f(co.v[i])) : crs * t;
+      q.v[i] = from_f<act_t>(o);
+      if (NSUMS == 3) s2[i] += to_f(q.v[i]);  // the bias gradient sums the values as stored
+    }
+    *reinterpret_cast<Pack8*>(dres + (size_t)row * C + c) = q;
   }
-  // block reduction over the row slots, in slot order
-  float* mine = sums + (size_t)slot * NSUMS * C;
+  // block reduction over the teams, in team order
+  float* mine = sums + (size_t)team * NSUMS * C;
   store8(mine + c, s0);
   store8(mine + C + c, s1);
   if (NSUMS == 3) store8(mine + 2 * C + c, s2);
   __syncthreads();
   for (int i = threadIdx.x; i < NSUMS * C; i += blockDim.x) {
     float t = 0.f;
-    for (int k = 0; k < RPB; ++k) t += sums[(size_t)k * NSUMS * C + i];
+    for (int k = 0; k < TEAMS; ++k) t += sums[(size_t)k * NSUMS * C + i];
     partials[(size_t)blockIdx.x * NSUMS * C + i] = t;
   }
 }
 
 template <int TPR, int S>
-int ln_bwd_rows_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
-                       const float* rstd, const float* g, float* partials, int M,
-                       int accumulate, cudaStream_t s) {
-  constexpr int RPB = TPR >= 256 ? 1 : 256 / TPR;
-  constexpr int threads = TPR * RPB;
-  constexpr size_t smem = (size_t)RPB * S * 8 * TPR * sizeof(float);
+int ln_bwd_staged_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
+                         const float* rstd, const float* g, float* partials, int M,
+                         int accumulate, cudaStream_t s) {
+  constexpr int TEAMS = ln_bwd_teams<TPR>();
+  constexpr int threads = TPR * TEAMS;
+  constexpr size_t smem = (size_t)TEAMS * kLnStages * (3 * 8 * TPR * sizeof(act_t) + 8) +
+                          (size_t)TEAMS * S * 8 * TPR * sizeof(float);
   static int grid = 0;
   if (!grid) {
-    cudaFuncSetAttribute(ln_bwd_rows_kernel<TPR, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(ln_bwd_staged_kernel<TPR, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     int per_sm = 0, sms = 0, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_bwd_rows_kernel<TPR, S>, threads, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_bwd_staged_kernel<TPR, S>, threads,
+                                                  smem);
     grid = per_sm * sms;
     if (grid < 1 || grid > kLnBlocks) grid = kLnBlocks;
   }
-  ln_bwd_rows_kernel<TPR, S><<<grid, threads, smem, s>>>(dres, dy, x, mean, rstd, g, partials, M,
-                                                         accumulate);
+  ln_bwd_staged_kernel<TPR, S><<<grid, threads, smem, s>>>(dres, dy, x, mean, rstd, g, partials,
+                                                           M, accumulate);
   return grid;
 }
 
@@ -354,6 +547,16 @@ int ln_bwd_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mea
 
 void layernorm_fwd(act_t* y, float* mean, float* rstd, const act_t* x, const float* g,
                    const float* b, int M, int C, cudaStream_t s) {
+  switch (C) {  // widths with a team kernel
+#define GPT2_LNFT(W)                                           \
+  case W:                                                    \
+    ln_fwd_staged_launch<W / 8>(y, mean, rstd, x, g, b, M, s); \
+    note_launch();                                           \
+    return;
+    GPT2_LNFT(256) GPT2_LNFT(512) GPT2_LNFT(768) GPT2_LNFT(1024) GPT2_LNFT(2048)
+#undef GPT2_LNFT
+    default: break;
+  }
   const int warps = 8;
   const int grid = (M + warps - 1) / warps;
   switch ((C + 255) / 256) {
@@ -374,10 +577,10 @@ void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* me
   switch (C * 4 + nsums) {  // widths with a row-group kernel
 #define GPT2_LNR(W)                                                                            \
   case 4 * W + 2:                                                                              \
-    nblk = ln_bwd_rows_launch<W / 8, 2>(dres, dy, x, mean, rstd, g, partials, M, accumulate, s); \
+    nblk = ln_bwd_staged_launch<W / 8, 2>(dres, dy, x, mean, rstd, g, partials, M, accumulate, s); \
     goto reduce;                                                                               \
   case 4 * W + 3:                                                                              \
-    nblk = ln_bwd_rows_launch<W / 8, 3>(dres, dy, x, mean, rstd, g, partials, M, accumulate, s); \
+    nblk = ln_bwd_staged_launch<W / 8, 3>(dres, dy, x, mean, rstd, g, partials, M, accumulate, s); \
     goto reduce;
     GPT2_LNR(256) GPT2_LNR(512) GPT2_LNR(768) GPT2_LNR(1024) GPT2_LNR(2048)
 #undef GPT2_LNR

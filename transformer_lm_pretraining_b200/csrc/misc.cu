@@ -449,6 +449,21 @@ __global__ void __launch_bounds__(256) norm_partial_kernel(double* __restrict__ 
   if (threadIdx.x == 0) partials[blockIdx.x] = red[0];
 }
 
+__global__ void sumsq_final_kernel(double* __restrict__ out, const double* __restrict__ partials,
+                                   int nblk) {
+  if (threadIdx.x != 0) return;
+  double s = 0.0;
+  for (int b = 0; b < nblk; ++b) s += partials[b];
+  *out = s;
+}
+
+__global__ void clip_from_sumsq_kernel(float* __restrict__ scalars, const double* __restrict__ sumsq,
+                                       float max_norm) {
+  const float nrm = (float)sqrt(*sumsq);
+  scalars[S_NORM] = nrm;
+  scalars[S_CLIP] = (nrm > max_norm) ? max_norm / (nrm + 1e-6f) : 1.0f;
+}
+
 __global__ void norm_final_kernel(float* __restrict__ scalars, const double* __restrict__ partials,
                                   int nblk, float max_norm) {
   if (threadIdx.x != 0) return;
@@ -468,15 +483,21 @@ struct DecayTable {
 
 __global__ void __launch_bounds__(256)
     adamw_kernel(float* __restrict__ p, act_t* __restrict__ pact, const float* __restrict__ g,
-                 float* __restrict__ m, float* __restrict__ v, size_t n, AdamArgs a,
+                 float* __restrict__ m, float* __restrict__ v, size_t base, size_t n, AdamArgs a,
                  DecayTable dt, const float* __restrict__ scalars) {
   const float nrm = scalars[S_NORM];
   if (!isfinite(nrm)) return;  // never apply a non-finite update
   const float clip = scalars[S_CLIP];
+  const float lr = scalars[S_LR], bc1 = scalars[S_BC1], bc2 = scalars[S_BC2];
   const size_t n4 = n / 4;
+  p += base;
+  pact += base;
+  g += base;
+  m += base;
+  v += base;
   for (size_t i4 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4;
        i4 += (size_t)gridDim.x * blockDim.x) {
-    const size_t i = i4 * 4;
+    const size_t i = base + i4 * 4;  // index in the flat parameter order
     float wd = 0.f;
     for (int k = 0; k < dt.n; ++k)
       if (i >= dt.begin[k] && i < dt.end[k]) wd = a.wd;
@@ -494,9 +515,9 @@ __global__ void __launch_bounds__(256)
       const float gr = ge[j] * clip;
       me[j] = a.b1 * me[j] + (1.f - a.b1) * gr;
       ve[j] = a.b2 * ve[j] + (1.f - a.b2) * gr * gr;
-      const float mh = me[j] / a.bc1;
-      const float vh = ve[j] / a.bc2;
-      pe[j] -= a.lr * (mh / (sqrtf(vh) + a.eps) + wd * pe[j]);
+      const float mh = me[j] / bc1;
+      const float vh = ve[j] / bc2;
+      pe[j] -= lr * (mh / (sqrtf(vh) + a.eps) + wd * pe[j]);
       outv[j] = pe[j];
     }
     reinterpret_cast<float4*>(p)[i4] = pp;
@@ -514,6 +535,31 @@ __global__ void __launch_bounds__(256)
     (void)outv;
 #endif
   }
+}
+
+// The step's learning rate: warmup lr_max (s + 1) / W for s < W, then a
+// cosine from lr_max down to lr_min at s = S, lr_min after (condensed GPT-2
+// page, section 3; the same formula as the host's gpt2_lr).
+struct Sched {
+  double max_lr, min_lr, warmup, max_steps;
+};
+__global__ void adam_prep_kernel(float* scalars, int* step, float lr, int scheduled, Sched sc,
+                                 float b1, float b2) {
+  const int t = *step + 1;
+  *step = t;
+  double l = lr;
+  if (scheduled) {
+    const double s = (double)(t - 1);
+    if (s < sc.warmup) l = sc.max_lr * (s + 1.0) / sc.warmup;
+    else if (s > sc.max_steps || sc.max_steps <= sc.warmup) l = sc.min_lr;
+    else {
+      const double ratio = (s - sc.warmup) / (sc.max_steps - sc.warmup);
+      l = sc.min_lr + 0.5 * (1.0 + cos(3.14159265358979323846 * ratio)) * (sc.max_lr - sc.min_lr);
+    }
+  }
+  scalars[S_LR] = (float)l;
+  scalars[S_BC1] = (float)(1.0 - pow((double)b1, (double)t));
+  scalars[S_BC2] = (float)(1.0 - pow((double)b2, (double)t));
 }
 
 __global__ void reset_clip_kernel(float* scalars) {
@@ -650,13 +696,32 @@ void grad_norm_clip(float* scalars, const float* g, size_t n, float max_norm, do
   note_launch(2);
 }
 
+void grad_sumsq(double* out, const float* g, size_t n, double* partials, cudaStream_t s) {
+  norm_partial_kernel<<<kNormBlocks, 256, 0, s>>>(partials, g, n);
+  sumsq_final_kernel<<<1, 32, 0, s>>>(out, partials, kNormBlocks);
+  note_launch(2);
+}
+
+void clip_from_sumsq(float* scalars, const double* sumsq, float max_norm, cudaStream_t s) {
+  clip_from_sumsq_kernel<<<1, 1, 0, s>>>(scalars, sumsq, max_norm);
+  note_launch();
+}
+
+void adam_prep(float* scalars, int* step, float lr, bool scheduled, const double* sched, float b1,
+               float b2, cudaStream_t s) {
+  Sched sc{0.0, 0.0, 1.0, 1.0};
+  if (scheduled) sc = Sched{sched[0], sched[1], sched[2], sched[3]};
+  adam_prep_kernel<<<1, 1, 0, s>>>(scalars, step, lr, scheduled ? 1 : 0, sc, b1, b2);
+  note_launch();
+}
+
 void reset_clip(float* scalars, cudaStream_t s) {
   reset_clip_kernel<<<1, 1, 0, s>>>(scalars);
   note_launch();
 }
 
 void adamw(float* p, act_t* pact, const float* g, float* m, float* v, const Layout& lay,
-           const AdamArgs& a, const float* scalars, cudaStream_t s) {
+           const AdamArgs& a, const float* scalars, cudaStream_t s, size_t begin, size_t end) {
   DecayTable dt;
   dt.n = 0;
   for (int t = 0; t < T_COUNT; ++t)
@@ -665,8 +730,10 @@ void adamw(float* p, act_t* pact, const float* g, float* m, float* v, const Layo
       dt.end[dt.n] = lay.off[t] + lay.num[t];
       ++dt.n;
     }
-  adamw_kernel<<<grid_for(lay.total / 4, 256, kNumSMs * 8), 256, 0, s>>>(p, pact, g, m, v,
-                                                                         lay.total, a, dt, scalars);
+  if (end > lay.total) end = lay.total;
+  if (begin >= end) return;
+  adamw_kernel<<<grid_for((end - begin) / 4, 256, kNumSMs * 8), 256, 0, s>>>(
+      p, pact, g, m, v, begin, end - begin, a, dt, scalars);
   note_launch();
 }
 

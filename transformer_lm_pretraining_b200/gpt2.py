@@ -51,6 +51,18 @@ SIGNATURES = {
     "gpt2_backward": (_i, [_vp, _f]),
     "gpt2_grad_norm_clip": (_i, [_vp, _f, _fp]),
     "gpt2_adamw_step": (_i, [_vp, _f, _f, _f, _f, _f]),
+    "gpt2_adamw_step_scheduled": (_i, [_vp, _d, _d, _l, _l, _f, _f, _f, _f]),
+    "gpt2_step_graph_capture": (_i, [_vp, _vp, _vp, _i, _i, _i, _f, _d, _d, _l, _l, _f, _f, _f,
+                                     _f]),
+    "gpt2_step_graph_launch": (_i, [_vp]),
+    "gpt2_padded_params": (_sz, [_vp]),
+    "gpt2_grad_sumsq": (_i, [_vp, _sz, _sz, _vp]),
+    "gpt2_clip_from_sumsq": (_i, [_vp, _vp, _f, _fp]),
+    "gpt2_adamw_step_range": (_i, [_vp, _f, _f, _f, _f, _f, _sz, _sz]),
+    "gpt2_params_device": (_i, [_vp, ctypes.POINTER(_fp)]),
+    "gpt2_refresh_weights": (_i, [_vp]),
+    "gpt2_set_backward_events": (_i, [_vp, ctypes.POINTER(_vp), _i]),
+    "gpt2_step_graph_kernels": (_l, [_vp]),
     "gpt2_lr": (_d, [_l, _d, _d, _l, _l]),
     "gpt2_get_params": (_i, [_vp, _fp]),
     "gpt2_set_params": (_i, [_vp, _fp]),
@@ -71,12 +83,14 @@ SIGNATURES = {
     "gpt2k_gemm": (_i, [_vp, _i, _i, _i, _i, _vp, _l, _i, _vp, _l, _i, _f, _vp, _l, _fp, _l, _fp,
                         _vp, _l, _vp, _l, _fp, _sz]),
     "gpt2k_attention_fwd": (_i, [_vp, _vp, _fp, _vp, _i, _i, _i, _i]),
+    "gpt2k_attention_bwd_scratch": (_sz, [_i, _i, _i]),
     "gpt2k_attention_bwd": (_i, [_vp, _vp, _fp, _vp, _vp, _vp, _fp, _i, _i, _i, _i]),
     "gpt2k_layernorm_fwd": (_i, [_vp, _vp, _fp, _fp, _vp, _fp, _fp, _i, _i]),
     "gpt2k_layernorm_bwd": (_i, [_vp, _vp, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _i, _i, _i]),
     "gpt2k_layernorm_bwd_scratch": (_sz, [_i]),
     "gpt2k_classifier": (_i, [_vp, _vp, _fp, _vp, _i, _i, _i, _i]),
     "gpt2k_take_error": (_i, []),
+    "gpt2k_gemm_expiry_test": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _i]),
     "gpt2k_gemm_wgrad_noalloc": (_i, [_vp, _i, _i, _i, _vp, _l, _vp, _l, _f, _fp, _l, _i, _vp]),
 }
 
@@ -237,6 +251,25 @@ class GPT2:
     def adamw_step(self, lr, b1=0.9, b2=0.95, eps=1e-8, wd=0.1):
         self._check(self.lib.gpt2_adamw_step(self.h, lr, b1, b2, eps, wd))
 
+    def adamw_step_scheduled(self, max_lr, min_lr, warmup, max_steps, b1=0.9, b2=0.95, eps=1e-8,
+                             wd=0.1):
+        self._check(self.lib.gpt2_adamw_step_scheduled(self.h, max_lr, min_lr, warmup, max_steps,
+                                                       b1, b2, eps, wd))
+
+    def capture_step(self, tok, tgt, B, T, n_micro, max_norm, max_lr, min_lr, warmup, max_steps,
+                     b1=0.9, b2=0.95, eps=1e-8, wd=0.1):
+        """Capture one optimizer step over the device token buffers tok, tgt
+        (n_micro * B * T int32 each) as a CUDA graph; returns the number of
+        kernels a replay runs."""
+        self._check(self.lib.gpt2_step_graph_capture(self.h, _dptr(tok), _dptr(tgt), B, T, n_micro,
+                                                     max_norm, max_lr, min_lr, warmup, max_steps,
+                                                     b1, b2, eps, wd))
+        return int(self.lib.gpt2_step_graph_kernels(self.h))
+
+    def launch_step(self):
+        """Replay the captured step on the model's stream (asynchronous)."""
+        self._check(self.lib.gpt2_step_graph_launch(self.h))
+
     # ------------------------------------------------------------- state --
     def get_params(self) -> np.ndarray:
         a = np.empty(self.P, np.float32)
@@ -248,19 +281,61 @@ class GPT2:
         assert p.size == self.P
         self._check(self.lib.gpt2_set_params(self.h, _fptr(p)))
 
-    def grads_tensor(self):
-        """The model's fp32 gradient buffer [P] as a torch CUDA tensor (a
-        view, no copy): what replicas all-reduce between backward and clip."""
+    def _device_view(self, getter, n):
+        """A torch CUDA tensor over n fp32 elements of a library buffer (no copy)."""
         torch = self.torch
         ptr = _fp()
-        self._check(self.lib.gpt2_grads_device(self.h, ctypes.byref(ptr)))
+        self._check(getter(self.h, ctypes.byref(ptr)))
         addr = ctypes.cast(ptr, ctypes.c_void_p).value
 
         class _View:  # CUDA array interface over the library's buffer
-            __cuda_array_interface__ = {"shape": (self.P,), "typestr": "<f4",
+            __cuda_array_interface__ = {"shape": (n,), "typestr": "<f4",
                                         "data": (addr, False), "version": 2}
 
         return torch.as_tensor(_View(), device="cuda")
+
+    @property
+    def padded_params(self) -> int:
+        return int(self.lib.gpt2_padded_params(self.h))
+
+    def grads_tensor(self, padded=False):
+        """The model's fp32 gradient buffer [P] (or [padded_params] with the
+        zero padding) as a torch CUDA tensor (a view, no copy): what replicas
+        all-reduce, or reduce-scatter, between backward and clip."""
+        return self._device_view(self.lib.gpt2_grads_device,
+                                 self.padded_params if padded else self.P)
+
+    def params_tensor(self, padded=False):
+        """The fp32 parameter buffer as a torch CUDA tensor view (for the
+        all-gather of updated shards; call refresh_weights afterwards)."""
+        return self._device_view(self.lib.gpt2_params_device,
+                                 self.padded_params if padded else self.P)
+
+    def grad_sumsq(self, begin, end, out):
+        """out (a float64 CUDA tensor of one element) = sum of squared
+        gradients [begin, end)."""
+        self._check(self.lib.gpt2_grad_sumsq(self.h, begin, end, _dptr(out)))
+
+    def clip_from_sumsq(self, sumsq, max_norm=1.0, sync=True):
+        out = ctypes.c_float(float("nan"))
+        self._check(self.lib.gpt2_clip_from_sumsq(self.h, _dptr(sumsq), max_norm,
+                                                  ctypes.byref(out) if sync else None))
+        return out.value if sync else None
+
+    def adamw_step_range(self, lr, b1, b2, eps, wd, begin, end):
+        self._check(self.lib.gpt2_adamw_step_range(self.h, lr, b1, b2, eps, wd, begin, end))
+
+    def refresh_weights(self):
+        self._check(self.lib.gpt2_refresh_weights(self.h))
+
+    def set_backward_events(self, events):
+        """events: L + 1 torch.cuda.Event objects (recorded at least once, so
+        that they exist) or None to stop recording."""
+        if not events:
+            self._check(self.lib.gpt2_set_backward_events(self.h, None, 0))
+            return
+        arr = (_vp * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        self._check(self.lib.gpt2_set_backward_events(self.h, arr, len(events)))
 
     def get_grads(self) -> np.ndarray:
         a = np.empty(self.P, np.float32)
@@ -353,6 +428,11 @@ def gpt2k_attention_fwd(att, lse, qkv, B, T, C, H, precision="bf16", stream=None
         raise GPT2Error(rc, "gpt2k_attention_fwd")
 
 
+def gpt2k_attention_bwd_scratch(B, T, H, precision="bf16") -> int:
+    """Floats of fp32 scratch gpt2k_attention_bwd needs."""
+    return int(load(precision).gpt2k_attention_bwd_scratch(B, T, H))
+
+
 def gpt2k_attention_bwd(dqkv, dsum, datt, qkv, att, lse, B, T, C, H, precision="bf16", stream=None):
     import torch
 
@@ -401,6 +481,13 @@ def gpt2k_classifier(logits, losses, tgt, M, V, Vp, write_grad=True, precision="
                                           _dptr(tgt), M, V, Vp, 1 if write_grad else 0)
     if rc:
         raise GPT2Error(rc, "gpt2k_classifier")
+
+
+def gpt2k_gemm_expiry_test(M, N, K, A, B, out, kblock=0, precision="bf16", stream=None) -> int:
+    """The GEMM with one withheld k-block (test of the bounded waits);
+    returns the C status."""
+    return int(load(precision).gpt2k_gemm_expiry_test(_stream(stream), M, N, K, _dptr(A), _dptr(B),
+                                                      _dptr(out), kblock))
 
 
 def gpt2k_take_error(precision="bf16") -> int:

@@ -71,7 +71,7 @@ def bench_attn(a):
         g2.gpt2k_attention_fwd(att, lse, qkv, B, T, C, H)
         datt = _rand((B * T, C))
         dqkv = torch.empty((B * T, 3 * C), dtype=torch.bfloat16, device="cuda")
-        dsum = torch.empty(B * H * T, dtype=torch.float32, device="cuda")
+        dsum = torch.empty(g2.gpt2k_attention_bwd_scratch(B, T, H), dtype=torch.float32, device="cuda")
 
         def call():
             g2.gpt2k_attention_bwd(dqkv, dsum, datt, qkv, att, lse, B, T, C, H)

@@ -17,16 +17,28 @@ import os
 
 
 class Replicas:
-    def __init__(self, backend: str = "nccl", timeout_s: float = 120.0):
+    def __init__(self, backend: str = "nccl", timeout_s: float = 120.0, group: bool = False):
+        """group=True starts the process group even on one rank (for the
+        data-parallel step, whose collectives then run as one-rank NCCL
+        calls)."""
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
         self.backend = backend
         self._dist = None
-        if self.world > 1:
+        if self.world > 1 or group:
             import torch.distributed as dist
 
-            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+            if self.world == 1:
+                os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+                if "MASTER_PORT" not in os.environ:
+                    import socket
+
+                    with socket.socket() as s:
+                        s.bind(("127.0.0.1", 0))
+                        os.environ["MASTER_PORT"] = str(s.getsockname()[1])
+            dist.init_process_group(backend, rank=self.rank, world_size=self.world,
+                                    timeout=datetime.timedelta(seconds=timeout_s))
             self._dist = dist
 
     @property
