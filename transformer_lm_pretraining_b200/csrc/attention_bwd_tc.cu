@@ -47,7 +47,8 @@ using attn::kHD;
 using attn::kTile;
 
 constexpr int kCT = attn::kComputeThreads;
-constexpr int kThreadsBwd = 64 + kCT;
+constexpr int kThreadsBwd = 64 + kCT + 32;  // + a second MMA-issuing warp (the last one)
+constexpr int kMma2 = kThreadsBwd / 32 - 1;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAux = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -128,8 +129,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   const uint32_t pd_empty0 = sd_full0 + 48;         // [2]
   const uint32_t acc_full = sd_full0 + 64;
   const uint32_t acc_empty = sd_full0 + 72;
-  const uint32_t drain = sd_full0 + 80;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 + 2 * kQStages + 11);
+  const uint32_t drain0 = sd_full0 + 80;  // [2] abort path only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 + 2 * kQStages + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int nq = (T + kTile - 1) / kTile;
@@ -148,11 +149,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     }
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(qd_full0 + 8 * s, 1);
-      mbar_init(qd_empty0 + 8 * s, 1);
+      mbar_init(qd_empty0 + 8 * s, 2);  // the scores and the products read Q and dO
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kCT);
-    mbar_init(drain, 1);
+    mbar_init(drain0, 1);
+    mbar_init(drain0 + 8, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -210,66 +212,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ------------------------------------------------------------ MMA --
-      constexpr uint32_t idS = attn::idesc(kSub, false);
-      constexpr uint32_t idA = attn::idesc(kHD, true);
+      // -------------------------------------------------- MMA: scores --
       // S^T = K Q_s^T and dP^T = V dO_s^T of sub-tile s (half hs of the
-      // query tile in stage st) into score buffer s % 2
-      auto issue_sd = [&](uint32_t s, int st, uint32_t tpar, int hs, int ks) -> bool {
-        const uint32_t sb = s & 1u;
-        if (!mbar_wait(qd_full0 + 8 * st, tpar, abort_flag, err)) return false;
-        if (!mbar_wait(sd_empty0 + 8 * sb, ((s >> 1) & 1u) ^ 1u, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(sKV + ks * 2 * kBox), v_base = k_base + kBox;
-        const uint32_t q_base = smem_u32(sQ + st * kBox) + hs * (kSub * 128);
-        const uint32_t do_base = smem_u32(sDO + st * kBox) + hs * (kSub * 128);
-        const uint32_t d = tmem + sb * 2 * kSub;
-#pragma unroll
-        for (int k = 0; k < kHD / 16; ++k)
-          tc_mma(d, desc_kmajor(k_base, k), desc_kmajor(q_base, k), idS, k > 0 ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < kHD / 16; ++k)
-          tc_mma(d + kSub, desc_kmajor(v_base, k), desc_kmajor(do_base, k), idS, k > 0 ? 1u : 0u);
-        tc_commit(sd_full0 + 8 * sb);
-        return true;
-      };
-      // dV += P^T dO_s, dK += dS^T Q_s of a sub-tile whose P^T and dS^T are
-      // (being) written to TMEM; releases the query tile after its second
-      // half and hands the accumulators over after the item's last sub-tile
-      struct Pend {
-        uint32_t s;
-        int st, hs;
-        bool first, last;
-      };
-      uint32_t n_acc = 0;  // items whose accumulators have been started
-      auto issue_acc = [&](const Pend& p) -> bool {
-        const uint32_t sb = p.s & 1u;
-        if (p.first) {  // the previous item's dV and dK have been read out
-          if (!mbar_wait(acc_empty, (n_acc & 1u) ^ 1u, abort_flag, err)) return false;
-          ++n_acc;
-        }
-        if (!mbar_wait(pd_full0 + 8 * sb, (p.s >> 1) & 1u, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t q_base = smem_u32(sQ + p.st * kBox), do_base = smem_u32(sDO + p.st * kBox);
-        const uint32_t pt = tmem + kOpCol + sb * kSub, dst = pt + kSub / 2;
-#pragma unroll
-        for (int k = 0; k < kSub / 16; ++k)
-          attn::tc_mma_ts(tmem + kAccColKV, pt + (uint32_t)(8 * k),
-                          desc_mnmajor(do_base, 4 * p.hs + k), idA, (!p.first || k > 0) ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < kSub / 16; ++k)
-          attn::tc_mma_ts(tmem + kAccColKV + kHD, dst + (uint32_t)(8 * k),
-                          desc_mnmajor(q_base, 4 * p.hs + k), idA, (!p.first || k > 0) ? 1u : 0u);
-        tc_commit(pd_empty0 + 8 * sb);
-        if (p.hs == 1) tc_commit(qd_empty0 + 8 * p.st);
-        if (p.last) tc_commit(acc_full);
-        return true;
-      };
-      // One flat sequence over every sub-tile of every item: the scores of
-      // sub-tile s are issued before the products of sub-tile s - 1.
+      // query tile in stage st) into score buffer s % 2.  The products run
+      // from their own warp, so the scores of the next sub-tiles never wait
+      // behind them.
+      constexpr uint32_t idS = attn::idesc(kSub, false);
       uint32_t n_item = 0, gs = 0, gt = 0;
-      Pend pend{};
-      bool have = false, ok = true;
+      bool ok = true;
       for (int k = 0; ok; ++k, ++n_item) {
         const int w = snake_item(k, items);
         if (w < 0) break;
@@ -277,25 +227,79 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         const int ks = n_item & 1;
         ok = mbar_wait(kv_full0 + 8 * ks, (n_item >> 1) & 1u, abort_flag, err);
         if (!ok) break;
-        tc_fence_after();
+        const uint32_t k_base = smem_u32(sKV + ks * 2 * kBox), v_base = k_base + kBox;
         for (int t = 0; t < n && ok; ++t, ++gt) {
           const int st = gt % kQStages;
-          const uint32_t tpar = (gt / kQStages) & 1u;
-          for (int hs = 0; hs < 2; ++hs, ++gs) {
-            ok = issue_sd(gs, st, tpar, hs, ks);
+          ok = mbar_wait(qd_full0 + 8 * st, (gt / kQStages) & 1u, abort_flag, err);
+          for (int hs = 0; hs < 2 && ok; ++hs, ++gs) {
+            const uint32_t sb = gs & 1u;
+            ok = mbar_wait(sd_empty0 + 8 * sb, ((gs >> 1) & 1u) ^ 1u, abort_flag, err);
             if (!ok) break;
-            if (t == n - 1 && hs == 1) tc_commit(kv_empty0 + 8 * ks);  // K, V no longer read
-            if (have) ok = issue_acc(pend);
-            if (!ok) break;
-            pend = Pend{gs, st, hs, t == 0 && hs == 0, t == n - 1 && hs == 1};
-            have = true;
+            tc_fence_after();
+            const uint32_t q_base = smem_u32(sQ + st * kBox) + hs * (kSub * 128);
+            const uint32_t do_base = smem_u32(sDO + st * kBox) + hs * (kSub * 128);
+            const uint32_t d = tmem + sb * 2 * kSub;
+#pragma unroll
+            for (int kk = 0; kk < kHD / 16; ++kk)
+              tc_mma(d, desc_kmajor(k_base, kk), desc_kmajor(q_base, kk), idS, kk > 0 ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < kHD / 16; ++kk)
+              tc_mma(d + kSub, desc_kmajor(v_base, kk), desc_kmajor(do_base, kk), idS,
+                     kk > 0 ? 1u : 0u);
+            tc_commit(sd_full0 + 8 * sb);
+            if (hs == 1) tc_commit(qd_empty0 + 8 * st);  // the scores are done with Q, dO
           }
         }
+        if (ok) tc_commit(kv_empty0 + 8 * ks);  // K, V no longer read
       }
-      if (ok && have) ok = issue_acc(pend);
       if (!ok) {  // let issued MMAs finish before TMEM is released
-        tc_commit(drain);
-        drain_wait(drain, 0, global_ns());
+        tc_commit(drain0);
+        drain_wait(drain0, 0, global_ns());
+      }
+    }
+  } else if (warp == kMma2) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA: products --
+      // dV += P^T dO_s, dK += dS^T Q_s of each sub-tile once its P^T and
+      // dS^T are in TMEM; the accumulators go to the compute warps after the
+      // item's last sub-tile.
+      constexpr uint32_t idA = attn::idesc(kHD, true);
+      uint32_t n_item = 0, gs = 0, gt = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k, ++n_item) {
+        const int w = snake_item(k, items);
+        if (w < 0) break;
+        const int n = nq - w / BH;
+        // the previous item's dV and dK have been read out
+        ok = mbar_wait(acc_empty, (n_item & 1u) ^ 1u, abort_flag, err);
+        for (int t = 0; t < n && ok; ++t, ++gt) {
+          const int st = gt % kQStages;
+          ok = mbar_wait(qd_full0 + 8 * st, (gt / kQStages) & 1u, abort_flag, err);
+          const uint32_t q_base = smem_u32(sQ + st * kBox), do_base = smem_u32(sDO + st * kBox);
+          for (int hs = 0; hs < 2 && ok; ++hs, ++gs) {
+            const uint32_t sb = gs & 1u;
+            ok = mbar_wait(pd_full0 + 8 * sb, (gs >> 1) & 1u, abort_flag, err);
+            if (!ok) break;
+            tc_fence_after();
+            const bool first = t == 0 && hs == 0;
+            const uint32_t pt = tmem + kOpCol + sb * kSub, dst = pt + kSub / 2;
+#pragma unroll
+            for (int kk = 0; kk < kSub / 16; ++kk)
+              attn::tc_mma_ts(tmem + kAccColKV, pt + (uint32_t)(8 * kk),
+                              desc_mnmajor(do_base, 4 * hs + kk), idA, (!first || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int kk = 0; kk < kSub / 16; ++kk)
+              attn::tc_mma_ts(tmem + kAccColKV + kHD, dst + (uint32_t)(8 * kk),
+                              desc_mnmajor(q_base, 4 * hs + kk), idA, (!first || kk > 0) ? 1u : 0u);
+            tc_commit(pd_empty0 + 8 * sb);
+            if (hs == 1) tc_commit(qd_empty0 + 8 * st);  // the products are done with Q, dO
+          }
+        }
+        if (ok) tc_commit(acc_full);
+      }
+      if (!ok) {
+        tc_commit(drain0 + 8);
+        drain_wait(drain0 + 8, 0, global_ns());
       }
     }
   } else {
@@ -434,8 +438,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   const uint32_t ds_empty0 = sd_full + 32;                   // [2]
   const uint32_t acc_full0 = sd_full + 48;                   // [2]
   const uint32_t acc_empty0 = sd_full + 64;                  // [2]
-  const uint32_t drain = sd_full + 80;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 11);
+  const uint32_t drain0 = sd_full + 80;                      // [2] abort path only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int nq = (T + kTile - 1) / kTile;
@@ -448,7 +452,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     mbar_init(qd_empty, 1 + kCT);  // the last S/dP product, and every compute thread's D
     for (int s = 0; s < kKVStages; ++s) {
       mbar_init(kv_full0 + 8 * s, 1);
-      mbar_init(kv_empty0 + 8 * s, 1);
+      mbar_init(kv_empty0 + 8 * s, 2);  // the scores read K, V; the products K
     }
     mbar_init(sd_full, 1);
     mbar_init(sd_empty, kCT);
@@ -457,8 +461,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       mbar_init(ds_empty0 + 8 * s, 1);
       mbar_init(acc_full0 + 8 * s, 1);
       mbar_init(acc_empty0 + 8 * s, kCT);
+      mbar_init(drain0 + 8 * s, 1);
     }
-    mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -509,66 +513,78 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ------------------------------------------------------------ MMA --
+      // -------------------------------------------------- MMA: scores --
+      // S = Q K_j^T and dP = dO V_j^T for every key tile j of every item;
+      // the dQ products run from their own warp.
       constexpr uint32_t idS = attn::idesc(kTile, false);
-      constexpr uint32_t idQ = attn::idesc(kHD, true);
       const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO);
       uint32_t n_item = 0, gk = 0;
       bool ok = true;
-      // S and dP against the key tile with global index gg
-      auto issue_sd = [&](uint32_t gg) -> bool {
-        const int st = gg % kKVStages;
-        if (!mbar_wait(kv_full0 + 8 * st, (gg / kKVStages) & 1u, abort_flag, err)) return false;
-        if (!mbar_wait(sd_empty, (gg & 1u) ^ 1u, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(sK + st * kBox), v_base = smem_u32(sV + st * kBox);
-#pragma unroll
-        for (int k = 0; k < kHD / 16; ++k)  // S = Q K^T
-          tc_mma(tmem, desc_kmajor(q_base, k), desc_kmajor(k_base, k), idS, k > 0 ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < kHD / 16; ++k)  // dP = dO V^T
-          tc_mma(tmem + kTile, desc_kmajor(do_base, k), desc_kmajor(v_base, k), idS, k > 0 ? 1u : 0u);
-        tc_commit(sd_full);
-        return true;
-      };
-      // dQ (+)= dS K into the accumulator at column acc (dS from TMEM)
-      auto issue_dq = [&](uint32_t gg, uint32_t acc, bool first) -> bool {
-        const int st = gg % kKVStages, db = gg & 1;
-        if (!mbar_wait(ds_full0 + 8 * db, (gg >> 1) & 1u, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t ds = tmem + kDSCol + (uint32_t)(db * kHD), k_base = smem_u32(sK + st * kBox);
-#pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)
-          attn::tc_mma_ts(tmem + acc, ds + (uint32_t)(8 * k), desc_mnmajor(k_base, k), idQ,
-                          (!first || k > 0) ? 1u : 0u);
-        tc_commit(ds_empty0 + 8 * db);
-        tc_commit(kv_empty0 + 8 * st);
-        return true;
-      };
       for (int k = 0; ok; ++k, ++n_item) {
         const int w = snake_item(k, items);
         if (w < 0) break;
         const int n = nq - w / BH;  // i + 1
-        const uint32_t ab = n_item & 1u, acc = kAccColQ + ab * kHD;
         ok = mbar_wait(qd_full, n_item & 1u, abort_flag, err);
-        if (ok) ok = mbar_wait(acc_empty0 + 8 * ab, ((n_item >> 1) & 1u) ^ 1u, abort_flag, err);
-        if (!ok) break;
-        tc_fence_after();
-        ok = issue_sd(gk);
-        if (ok && n == 1) tc_commit(qd_empty);  // Q and dO are no longer read
-        for (int jj = 1; jj <= n && ok; ++jj) {
-          if (jj < n) {
-            ok = issue_sd(gk + jj);
-            if (ok && jj == n - 1) tc_commit(qd_empty);
-          }
-          if (ok) ok = issue_dq(gk + jj - 1, acc, jj == 1);
+        for (int jj = 0; jj < n && ok; ++jj) {
+          const uint32_t gg = gk + jj;
+          const int st = gg % kKVStages;
+          ok = mbar_wait(kv_full0 + 8 * st, (gg / kKVStages) & 1u, abort_flag, err);
+          if (ok) ok = mbar_wait(sd_empty, (gg & 1u) ^ 1u, abort_flag, err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(sK + st * kBox), v_base = smem_u32(sV + st * kBox);
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk)  // S = Q K^T
+            tc_mma(tmem, desc_kmajor(q_base, kk), desc_kmajor(k_base, kk), idS, kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk)  // dP = dO V^T
+            tc_mma(tmem + kTile, desc_kmajor(do_base, kk), desc_kmajor(v_base, kk), idS,
+                   kk > 0 ? 1u : 0u);
+          tc_commit(sd_full);
+          tc_commit(kv_empty0 + 8 * st);  // the scores are done with K_j, V_j
+          if (jj == n - 1) tc_commit(qd_empty);  // Q and dO are no longer read
+        }
+        gk += n;
+      }
+      if (!ok) {
+        tc_commit(drain0);
+        drain_wait(drain0, 0, global_ns());
+      }
+    }
+  } else if (warp == kMma2) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA: products --
+      // dQ (+)= dS_j K_j (dS from TMEM) into the item's accumulator.
+      constexpr uint32_t idQ = attn::idesc(kHD, true);
+      uint32_t n_item = 0, gk = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k, ++n_item) {
+        const int w = snake_item(k, items);
+        if (w < 0) break;
+        const int n = nq - w / BH;
+        const uint32_t ab = n_item & 1u, acc = kAccColQ + ab * kHD;
+        ok = mbar_wait(acc_empty0 + 8 * ab, ((n_item >> 1) & 1u) ^ 1u, abort_flag, err);
+        for (int jj = 0; jj < n && ok; ++jj) {
+          const uint32_t gg = gk + jj;
+          const int st = gg % kKVStages, db = gg & 1;
+          ok = mbar_wait(kv_full0 + 8 * st, (gg / kKVStages) & 1u, abort_flag, err);
+          if (ok) ok = mbar_wait(ds_full0 + 8 * db, (gg >> 1) & 1u, abort_flag, err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ds = tmem + kDSCol + (uint32_t)(db * kHD), k_base = smem_u32(sK + st * kBox);
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            attn::tc_mma_ts(tmem + acc, ds + (uint32_t)(8 * kk), desc_mnmajor(k_base, kk), idQ,
+                            (jj > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(ds_empty0 + 8 * db);
+          tc_commit(kv_empty0 + 8 * st);  // the products are done with K_j
         }
         if (ok) tc_commit(acc_full0 + 8 * ab);
         gk += n;
       }
       if (!ok) {
-        tc_commit(drain);
-        drain_wait(drain, 0, global_ns());
+        tc_commit(drain0 + 8);
+        drain_wait(drain0 + 8, 0, global_ns());
       }
     }
   } else {

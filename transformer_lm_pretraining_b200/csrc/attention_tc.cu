@@ -50,7 +50,7 @@ using attn::kTile;
 
 constexpr int kKVStages = 4;
 constexpr int kRowThreads = 128;  // softmax threads per query tile
-constexpr int kThreadsAttn = 64 + 2 * kRowThreads;
+constexpr int kThreadsAttn = 64 + 2 * kRowThreads + 32;  // + the MMA warp of tile B
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 2 * kTile;         // O_t at kOCol + t * kHD
 constexpr uint32_t kPCol = kOCol + 2 * kHD;   // P_t at kPCol + t * kHD (bf16 pairs)
@@ -102,8 +102,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   const uint32_t s_empty0 = s_full0 + 16;                        // [2 tiles]
   const uint32_t p_full0 = s_full0 + 32;                         // [2 tiles]
   const uint32_t o_full0 = s_full0 + 48;                         // [2 tiles]
-  const uint32_t drain = s_full0 + 64;                           // abort path only
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 9);
+  const uint32_t drain0 = s_full0 + 64;                          // [2 tiles] abort path only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int nq = (T + kTile - 1) / kTile;
@@ -111,22 +111,22 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, 2);  // both MMA warps
     for (int s = 0; s < kKVStages; ++s) {
       mbar_init(kv_full0 + 8 * s, 1);
-      mbar_init(kv_empty0 + 8 * s, 1);
+      mbar_init(kv_empty0 + 8 * s, 2);  // both MMA warps
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full0 + 8 * t, 1);
       mbar_init(s_empty0 + 8 * t, kRowThreads);
       mbar_init(p_full0 + 8 * t, kRowThreads);
       mbar_init(o_full0 + 8 * t, 1);
+      mbar_init(drain0 + 8 * t, 1);
     }
-    mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == 1) {  // TMEM owner
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(kTmemCols));
@@ -181,69 +181,69 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == kThreadsAttn / 32 - 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA --
+      // One issuing warp per query tile (warp 1: tile A, the last warp:
+      // tile B), so that neither tile's products wait behind the other's
+      // barriers.  Both release each K/V stage and the Q tiles (the
+      // barriers count two arrivals).
+      const int t = warp == 1 ? 0 : 1;
       constexpr uint32_t idS = attn::idesc(kTile, false);
       constexpr uint32_t idO = attn::idesc(kHD, true);
       uint32_t n_item = 0, g = 0;
-      uint32_t cs[2] = {0, 0}, co[2] = {0, 0};  // S / PV products issued per tile
+      uint32_t cs = 0, co = 0;  // S / PV products issued for this tile
       bool ok = true;
-      // S_t = Q_t K (key tile in ring stage st)
-      auto issue_s = [&](int t, int st) -> bool {
-        if (!mbar_wait(s_empty0 + 8 * t, (cs[t] & 1u) ^ 1u, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t q_base = smem_u32(sQ + t * kBox), k_base = smem_u32(sK + st * kBox);
-#pragma unroll
-        for (int k = 0; k < kHD / 16; ++k)
-          tc_mma(tmem + (uint32_t)(t * kTile), desc_kmajor(q_base, k), desc_kmajor(k_base, k), idS,
-                 k > 0 ? 1u : 0u);
-        tc_commit(s_full0 + 8 * t);
-        ++cs[t];
-        return true;
-      };
-      // O_t (+)= P_t V (P_t from TMEM, value tile in ring stage st); the
-      // item's first product initialises O_t
-      auto issue_pv = [&](int t, int st, bool first) -> bool {
-        if (!mbar_wait(p_full0 + 8 * t, co[t] & 1u, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(sV + st * kBox);
-        const uint32_t p_t = tmem + kPCol + (uint32_t)(t * kHD);
-#pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)
-          attn::tc_mma_ts(tmem + kOCol + (uint32_t)(t * kHD), p_t + (uint32_t)(8 * k),
-                          desc_mnmajor(v_base, k), idO, (k > 0 || !first) ? 1u : 0u);
-        tc_commit(o_full0 + 8 * t);
-        ++co[t];
-        return true;
-      };
+      const uint32_t q_base = smem_u32(sQ + t * kBox);
+      const uint32_t p_t = tmem + kPCol + (uint32_t)(t * kHD);
+      const uint32_t o_t = tmem + kOCol + (uint32_t)(t * kHD);
+      const uint32_t s_t = tmem + (uint32_t)(t * kTile);
       FwdItem it;
       for (int k = 0; ok && fwd_item(k, B, H, nq, it); ++k, ++n_item) {
         ok = mbar_wait(q_full, n_item & 1u, abort_flag, err);
         if (!ok) break;
         tc_fence_after();
         const int nkv = it.nkv_b ? it.nkv_b : it.nkv_a;
+        const int mine = t ? it.nkv_b : it.nkv_a;  // key tiles of this query tile (0: none)
+        if (mine == 0) tc_commit(q_empty);
         for (int j = 0; j <= nkv && ok; ++j) {
-          if (j < nkv) {
-            const uint32_t gj = g + j;
-            ok = mbar_wait(kv_full0 + 8 * (gj % kKVStages), (gj / kKVStages) & 1u, abort_flag, err);
-            if (ok && j < it.nkv_a) ok = issue_s(0, gj % kKVStages);
-            if (ok && j < it.nkv_b) ok = issue_s(1, gj % kKVStages);
-            if (ok && j == nkv - 1) tc_commit(q_empty);  // the item's Q tiles are read
+          if (j < mine) {  // S_t = Q_t K_j^T
+            const uint32_t gj = g + j, st = gj % kKVStages;
+            ok = mbar_wait(kv_full0 + 8 * st, (gj / kKVStages) & 1u, abort_flag, err);
+            if (ok) ok = mbar_wait(s_empty0 + 8 * t, (cs & 1u) ^ 1u, abort_flag, err);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t k_base = smem_u32(sK + st * kBox);
+#pragma unroll
+            for (int kk = 0; kk < kHD / 16; ++kk)
+              tc_mma(s_t, desc_kmajor(q_base, kk), desc_kmajor(k_base, kk), idS, kk > 0 ? 1u : 0u);
+            tc_commit(s_full0 + 8 * t);
+            ++cs;
+            if (j == mine - 1) tc_commit(q_empty);  // this tile's Q is read
           }
-          if (ok && j >= 1) {
+          if (j >= 1) {
             const uint32_t st = (g + j - 1) % kKVStages;
-            if (j - 1 < it.nkv_a) ok = issue_pv(0, st, j == 1);
-            if (ok && j - 1 < it.nkv_b) ok = issue_pv(1, st, j == 1);
-            if (ok) tc_commit(kv_empty0 + 8 * st);  // K and V of key tile j-1 are no longer read
+            if (j - 1 < mine) {  // O_t (+)= P_t V_{j-1}, P_t from TMEM
+              ok = mbar_wait(p_full0 + 8 * t, co & 1u, abort_flag, err);
+              if (!ok) break;
+              tc_fence_after();
+              const uint32_t v_base = smem_u32(sV + st * kBox);
+#pragma unroll
+              for (int kk = 0; kk < kTile / 16; ++kk)
+                attn::tc_mma_ts(o_t, p_t + (uint32_t)(8 * kk), desc_mnmajor(v_base, kk), idO,
+                                (kk > 0 || j > 1) ? 1u : 0u);
+              tc_commit(o_full0 + 8 * t);
+              ++co;
+            }
+            tc_commit(kv_empty0 + 8 * st);  // this tile no longer reads key tile j-1
           }
         }
         g += nkv;
       }
       if (!ok) {  // let issued MMAs finish before TMEM is released
-        tc_commit(drain);
+        tc_commit(drain0 + 8 * t);
         const uint64_t t0 = global_ns();
-        while (!mbar_try_wait(drain, 0) && global_ns() - t0 < kWaitLimitNs) {
+        while (!mbar_try_wait(drain0 + 8 * t, 0) && global_ns() - t0 < kWaitLimitNs) {
         }
       }
     }

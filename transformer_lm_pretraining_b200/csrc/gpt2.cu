@@ -723,6 +723,9 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.out = a.dbig; ga.ldo = 4 * C;
       GPT2_TRY(run_gemm(h, ga));
     }
+    // the bias gradient of W_fc while du is still in L2
+    mark(h, PK_COLSUM);
+    colsum_acc(G + y.off[T_BFC] + (size_t)l * 4 * C, a.dbig, M, 4 * C, a.partials, s);
     if (h->recompute) {  // g = gelu(u), as the forward's epilogue computed it
       mark(h, PK_RECOMPUTE);
       gelu_fwd(const_cast<act_t*>(g), u, 4 * MC, s);
@@ -753,8 +756,6 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
       GPT2_TRY(run_gemm(h, ga));
     }
-    mark(h, PK_COLSUM);
-    colsum_acc(G + y.off[T_BFC] + (size_t)l * 4 * C, a.dbig, M, 4 * C, a.partials, s);
     mark(h, PK_LN_BWD);
     // dres = d x_mid; its column sum is the bias gradient of W_o
     layernorm_bwd(a.dres, a.dh, xm, a.mean2 + (size_t)l * M, a.rstd2 + (size_t)l * M,
@@ -782,6 +783,9 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     mark(h, PK_ATTN_BWD, 10.0 * B * H * (double)T * (T + 1) / 2 * (C / H));
     GPT2_CUDA(h, attention_bwd(a.dqkv, a.dsum, a.datt, qkv, att, a.lse + (size_t)l * M * H, B, T,
                                C, H, h->err, s));
+    // the bias gradient of W_qkv while dqkv is still in L2
+    mark(h, PK_COLSUM);
+    colsum_acc(G + y.off[T_BQKV] + (size_t)l * 3 * C, a.dqkv, M, 3 * C, a.partials, s);
     {  // dh = dqkv Wqkv
       GemmArgs ga = gemm_args(M, C, 3 * C);
       ga.A = a.dqkv; ga.lda = 3 * C;
@@ -799,8 +803,6 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
       GPT2_TRY(run_gemm(h, ga));
     }
-    mark(h, PK_COLSUM);
-    colsum_acc(G + y.off[T_BQKV] + (size_t)l * 3 * C, a.dqkv, M, 3 * C, a.partials, s);
     mark(h, PK_LN_BWD);
     // dres = d x_l = gradient at the output of layer l-1: bias of its W_p
     layernorm_bwd(a.dres, a.dh, x, a.mean1 + (size_t)l * M, a.rstd1 + (size_t)l * M,
