@@ -293,7 +293,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(sr[c]));
+        for (int c = 0; c < kTile; c += 2)
+          mx4[(c >> 1) & 3] = attn::fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]),
+                                          __uint_as_float(sr[c + 1]));
         const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
         const bool raise = mt > m + kRescaleLog2;  // always on the first key tile
         const float mn = raise ? mt : m;

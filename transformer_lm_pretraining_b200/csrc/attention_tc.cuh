@@ -78,6 +78,13 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// max(a, b, c) in one instruction (three-input max of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Two floats -> one 32-bit word of two bf16 (round to nearest; lo in the
 // low half, the lower K index of an MMA operand).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
