@@ -49,6 +49,17 @@ using attn::kTile;
 constexpr int kCT = attn::kComputeThreads;
 constexpr int kThreadsBwd = 64 + kCT + 32;  // + a second MMA-issuing warp (the last one)
 constexpr int kMma2 = kThreadsBwd / 32 - 1;
+// dK/dV: KV_SPLIT compute threads per key row (four warps per lane quarter
+// of TMEM with KV_SPLIT = 4), each owning 64 / KV_SPLIT of a sub-tile's
+// query columns
+#ifndef KV_SPLIT
+#define KV_SPLIT 4
+#endif
+constexpr int kKvSplit = KV_SPLIT;
+constexpr int kCTkv = 128 * kKvSplit;
+constexpr int kThreadsKV = 64 + kCTkv + 32;
+constexpr int kMma2KV = kThreadsKV / 32 - 1;
+constexpr int kColsKV = 64 / kKvSplit;  // query columns per thread and sub-tile
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAux = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -75,6 +86,25 @@ __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t* r) {
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+
+// 32 lanes x 8 consecutive 32-bit columns from registers into TMEM.
+__device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+// TMEM load / store of N (16 or 32) columns for this lane.
+template <int N>
+__device__ __forceinline__ void tc_ldn(uint32_t taddr, uint32_t* r) {
+  if constexpr (N == 32) tc_ld32(taddr, r);
+  else attn::tc_ld16(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tc_stn(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N == 16) tc_st16(taddr, r);
+  else tc_st8(taddr, r);
 }
 
 // Bounded wait for copies issued to `bar` (latest fill parity `par`).
@@ -106,7 +136,7 @@ constexpr size_t dkdv_smem_bytes() {
          kAux;
 }
 
-__global__ void __launch_bounds__(kThreadsBwd, 1)
+__global__ void __launch_bounds__(kThreadsKV, 1)
     flash_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
                              const __grid_constant__ CUtensorMap tmDO,
                              const float2* __restrict__ pairs, __nv_bfloat16* __restrict__ dqkv,
@@ -143,8 +173,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       mbar_init(kv_full0 + 8 * s, 1);
       mbar_init(kv_empty0 + 8 * s, 1);
       mbar_init(sd_full0 + 8 * s, 1);
-      mbar_init(sd_empty0 + 8 * s, kCT);
-      mbar_init(pd_full0 + 8 * s, kCT);
+      mbar_init(sd_empty0 + 8 * s, kCTkv);
+      mbar_init(pd_full0 + 8 * s, kCTkv);
       mbar_init(pd_empty0 + 8 * s, 1);
     }
     for (int s = 0; s < kQStages; ++s) {
@@ -152,7 +182,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       mbar_init(qd_empty0 + 8 * s, 2);  // the scores and the products read Q and dO
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kCT);
+    mbar_init(acc_empty, kCTkv);
     mbar_init(drain0, 1);
     mbar_init(drain0 + 8, 1);
     *abort_flag = 0;
@@ -257,7 +287,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         drain_wait(drain0, 0, global_ns());
       }
     }
-  } else if (warp == kMma2) {
+  } else if (warp == kMma2KV) {
     if (lane == 0) {
       // ------------------------------------------------ MMA: products --
       // dV += P^T dO_s, dK += dS^T Q_s of each sub-tile once its P^T and
@@ -304,9 +334,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     }
   } else {
     // -------------------------------------------------------- compute --
-    // thread = key row r, owning 32 of a sub-tile's 64 query columns.  Every
-    // wait is per warp (warps drift apart and overlap their latencies).
-    const int qw = warp & 3, half = (warp - 2) >> 2;
+    // thread = key row r, owning kColsKV of a sub-tile's 64 query columns
+    // (slot `part` of the row).  Every wait is per warp (warps drift apart
+    // and overlap their latencies).
+    const int qw = warp & 3, part = (warp - 2) >> 2;
     const int r = qw * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
     uint32_t n_item = 0, gs = 0, gt = 0;
@@ -322,24 +353,24 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         const float4* ld4 = reinterpret_cast<const float4*>(sLD + st * kPairBytes);
         for (int hs = 0; hs < 2; ++hs, ++gs) {
           const uint32_t sb = gs & 1u;
-          const int cq = kSub * hs + 32 * half;  // first query column of this thread in the tile
+          const int cq = kSub * hs + kColsKV * part;  // first query column of this thread in the tile
           ok = warp_and(mbar_wait(sd_full0 + 8 * sb, (gs >> 1) & 1u, abort_flag, err));
           if (!ok) break;
           tc_fence_after();
-          uint32_t sr[32], dp[32];
-          tc_ld32(lane_base + sb * 2 * kSub + 32 * half, sr);
-          tc_ld32(lane_base + sb * 2 * kSub + kSub + 32 * half, dp);
+          uint32_t sr[kColsKV], dp[kColsKV];
+          tc_ldn<kColsKV>(lane_base + sb * 2 * kSub + kColsKV * part, sr);
+          tc_ldn<kColsKV>(lane_base + sb * 2 * kSub + kSub + kColsKV * part, dp);
           tc_wait_ld();
           tc_fence_before();
           mbar_arrive(sd_empty0 + 8 * sb);  // the scores are read: sub-tile gs + 2 may be computed
           if (t == 0) {  // the diagonal tile: queries before the key are masked
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
+            for (int c = 0; c < kColsKV; ++c)
               if (cq + c < r) sr[c] = kNegInf;
           }
-          uint32_t pk[16], dk[16];
+          uint32_t pk[kColsKV / 2], dk[kColsKV / 2];
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
+          for (int c = 0; c < kColsKV; c += 4) {
             // (L log2e, D) of queries cq + c .. cq + c + 3 (query-tile stage st)
             const float4 a = ld4[(cq + c) / 2];
             const float4 bq = ld4[(cq + c) / 2 + 1];
@@ -360,29 +391,31 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           ok = warp_and(mbar_wait(pd_empty0 + 8 * sb, ((gs >> 1) & 1u) ^ 1u, abort_flag, err));
           if (!ok) break;
           tc_fence_after();
-          const uint32_t op = lane_base + kOpCol + sb * kSub + 16 * half;
-          tc_st16(op, pk);
-          tc_st16(op + kSub / 2, dk);
+          const uint32_t op = lane_base + kOpCol + sb * kSub + (kColsKV / 2) * part;
+          tc_stn<kColsKV / 2>(op, pk);
+          tc_stn<kColsKV / 2>(op + kSub / 2, dk);
           attn::tc_wait_st();
           tc_fence_before();
           mbar_arrive(pd_full0 + 8 * sb);
         }
       }
       if (!ok) break;
-      // the item's dV and dK
+      // the item's dV and dK: this thread's 64 / kKvSplit columns of each
       ok = warp_and(mbar_wait(acc_full, n_item & 1u, abort_flag, err));
       if (!ok) break;
       tc_fence_after();
-      uint32_t rv[32], rk[32];
-      tc_ld32(lane_base + kAccColKV + 32 * half, rv);
-      tc_ld32(lane_base + kAccColKV + kHD + 32 * half, rk);
+      constexpr int kAccCols = kHD / kKvSplit;
+      uint32_t rv[kAccCols], rk[kAccCols];
+      tc_ldn<kAccCols>(lane_base + kAccColKV + kAccCols * part, rv);
+      tc_ldn<kAccCols>(lane_base + kAccColKV + kHD + kAccCols * part, rk);
       tc_wait_ld();
       tc_fence_before();
       mbar_arrive(acc_empty);
       if (kj < T) {
-        __nv_bfloat16* row = dqkv + ((size_t)b * T + kj) * 3 * C + (size_t)h * kHD + 32 * half;
+        __nv_bfloat16* row =
+            dqkv + ((size_t)b * T + kj) * 3 * C + (size_t)h * kHD + kAccCols * part;
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
+        for (int i = 0; i < kAccCols; i += 8) {
           float a[8], d[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -728,7 +761,7 @@ cudaError_t attention_bwd_tc(act_t* dqkv, float* scratch, const act_t* datt, con
   // (L, D) pairs for dK/dV
   flash_bwd_dq_tc_kernel<<<grid, kThreadsBwd, sm_b, s>>>(tq, td, to, lse, pairs, dqkv, B, T, C, H,
                                                          sl2, scale, err);
-  flash_bwd_dkdv_tc_kernel<<<grid, kThreadsBwd, sm_a, s>>>(tq, td, pairs, dqkv, B, T, C, H, sl2,
+  flash_bwd_dkdv_tc_kernel<<<grid, kThreadsKV, sm_a, s>>>(tq, td, pairs, dqkv, B, T, C, H, sl2,
                                                            scale, err);
   note_launch(2);
   return cudaGetLastError();
