@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -444,6 +445,25 @@ def run_ours(args, wl):
         e2e_ms = max_over_ranks(e0.elapsed_time(e1))
         e2e = {"value": reps.throughput(wl.tokens_per_step * n_e2e, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": 2 * 4 * wl.B * wl.T * wl.n_micro, "d2h_bytes_per_step": 4}
+
+    # a step that produced a non-finite loss or gradient norm measured nothing
+    # (AdamW leaves the parameters alone on a non-finite norm, which would
+    # make such a step look fast): one more step, read back and checked
+    chk = dev[args.warmup]
+    if not evaluate:
+        model.zero_grad()
+    for tok, tgt in chk:
+        if evaluate:
+            model.evaluate(tok, tgt, sync_loss=False)
+        else:
+            model.forward(tok, tgt, sync_loss=False)
+            model.backward(scale)
+    chk_norm = 0.0 if evaluate else model.grad_norm_clip(1.0)
+    chk_loss = model.read_loss()
+    if not (math.isfinite(chk_loss) and math.isfinite(chk_norm)):
+        print(f"bench: non-finite step (loss {chk_loss}, gradient norm {chk_norm}); no number reported",
+              file=sys.stderr)
+        sys.exit(3)
 
     peaks = load_peaks()
     fpt = wl.flops_per_token() / (3.0 if evaluate else 1.0)  # the forward is a third

@@ -188,12 +188,13 @@ gpt2_status gpt2_adamw_step_scheduled(gpt2_t* h, double max_lr, double min_lr, l
 
 /* One whole optimizer step captured as a CUDA graph owned by the handle and
  * replayed with gpt2_step_graph_launch, in place of the ~370 separate
- * launches of the eager calls: gpt2_zero_grad; for i < n_micro,
+ * launches of the eager calls (the graph is uploaded to the device here,
+ * on the model's stream): gpt2_zero_grad; for i < n_micro,
  * gpt2_forward(tok_dev + i B T, tgt_dev + i B T, B, T) and
  * gpt2_backward(1 / n_micro); gpt2_grad_norm_clip(max_norm);
  * gpt2_adamw_step_scheduled(...).  tok_dev and tgt_dev (n_micro B T ids
  * each) are read at every replay: write the next step's tokens there before
- * launching it.  Capturing enqueues no work.  Requirements: a stream set with
+ * launching it.  Capturing runs no kernel.  Requirements: a stream set with
  * gpt2_set_stream (not the legacy default stream), profiling off, and one
  * eager step of the same B and T run before (first-use set-up of the kernels
  * is not captured).  A new capture replaces the previous graph.

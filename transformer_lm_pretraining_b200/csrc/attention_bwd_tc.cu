@@ -6,11 +6,12 @@
 //   dV = P^T dO,  dK = dS^T Q / sqrt(d),  dQ = dS K / sqrt(d)
 //
 // Two persistent kernels, one CTA per SM walking a static snake order over
-// work items (heaviest first), 10 warps each (TMA, MMA, 8 compute warps,
-// two threads per tile row).  In both, the second product of each step
-// takes its A operand (P^T and dS^T, or dS) from TMEM, where the compute
-// warps write it as packed bf16, so shared memory only feeds the tensor core
-// the operands that TMA brings in:
+// work items (heaviest first): a TMA warp, two MMA-issuing warps (scores,
+// and the products that accumulate the gradients) and the compute warps
+// (four threads per key row in dK/dV, two per query row in dQ).  In both, the second product of each
+// step takes its A operand (P^T and dS^T, or dS) from TMEM, where the
+// compute warps write it as packed bf16, so shared memory only feeds the
+// tensor core the operands that TMA brings in:
 //   dQ:    item = (batch, head, query tile i); streams the key tiles j <= i:
 //          S = Q K^T and dP = dO V^T into TMEM, dS into one of two TMEM
 //          buffers, dQ += dS K in one of two TMEM accumulators (K read
@@ -46,9 +47,6 @@ using attn::kBox;
 using attn::kHD;
 using attn::kTile;
 
-constexpr int kCT = attn::kComputeThreads;
-constexpr int kThreadsBwd = 64 + kCT + 32;  // + a second MMA-issuing warp (the last one)
-constexpr int kMma2 = kThreadsBwd / 32 - 1;
 // dK/dV: KV_SPLIT compute threads per key row (four warps per lane quarter
 // of TMEM with KV_SPLIT = 4), each owning 64 / KV_SPLIT of a sub-tile's
 // query columns
@@ -60,6 +58,17 @@ constexpr int kCTkv = 128 * kKvSplit;
 constexpr int kThreadsKV = 64 + kCTkv + 32;
 constexpr int kMma2KV = kThreadsKV / 32 - 1;
 constexpr int kColsKV = 64 / kKvSplit;  // query columns per thread and sub-tile
+// dQ: Q_SPLIT compute threads per query row, each owning 128 / Q_SPLIT of a
+// key tile's columns (measured: 2 beats 4 here, 180 vs 202 us for the
+// backward at B16 x T1024)
+#ifndef Q_SPLIT
+#define Q_SPLIT 2
+#endif
+constexpr int kQSplit = Q_SPLIT;
+constexpr int kCTq = 128 * kQSplit;
+constexpr int kThreadsQ = 64 + kCTq + 32;
+constexpr int kMma2Q = kThreadsQ / 32 - 1;
+constexpr int kColsQ = kTile / kQSplit;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAux = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -95,15 +104,18 @@ __device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t* r) {
                "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                : "memory");
 }
-// TMEM load / store of N (16 or 32) columns for this lane.
+// TMEM load (16 or 32 columns) / store (8, 16 or 32 columns) for this lane.
 template <int N>
 __device__ __forceinline__ void tc_ldn(uint32_t taddr, uint32_t* r) {
+  static_assert(N == 16 || N == 32, "TMEM load width");
   if constexpr (N == 32) tc_ld32(taddr, r);
   else attn::tc_ld16(taddr, r);
 }
 template <int N>
 __device__ __forceinline__ void tc_stn(uint32_t taddr, const uint32_t* r) {
-  if constexpr (N == 16) tc_st16(taddr, r);
+  static_assert(N == 8 || N == 16 || N == 32, "TMEM store width");
+  if constexpr (N == 32) attn::tc_st32(taddr, r);
+  else if constexpr (N == 16) tc_st16(taddr, r);
   else tc_st8(taddr, r);
 }
 
@@ -446,7 +458,7 @@ constexpr size_t dq_smem_bytes() {
   return 1024 + 3 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + kAux;
 }
 
-__global__ void __launch_bounds__(kThreadsBwd, 1)
+__global__ void __launch_bounds__(kThreadsQ, 1)
     flash_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
                            const __grid_constant__ CUtensorMap tmDO,
                            const __grid_constant__ CUtensorMap tmO, const float* __restrict__ lse,
@@ -482,18 +494,18 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
-    mbar_init(qd_empty, 1 + kCT);  // the last S/dP product, and every compute thread's D
+    mbar_init(qd_empty, 1 + kCTq);  // the last S/dP product, and every compute thread's D
     for (int s = 0; s < kKVStages; ++s) {
       mbar_init(kv_full0 + 8 * s, 1);
       mbar_init(kv_empty0 + 8 * s, 2);  // the scores read K, V; the products K
     }
     mbar_init(sd_full, 1);
-    mbar_init(sd_empty, kCT);
+    mbar_init(sd_empty, kCTq);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(ds_full0 + 8 * s, kCT);
+      mbar_init(ds_full0 + 8 * s, kCTq);
       mbar_init(ds_empty0 + 8 * s, 1);
       mbar_init(acc_full0 + 8 * s, 1);
-      mbar_init(acc_empty0 + 8 * s, kCT);
+      mbar_init(acc_empty0 + 8 * s, kCTq);
       mbar_init(drain0 + 8 * s, 1);
     }
     *abort_flag = 0;
@@ -584,7 +596,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         drain_wait(drain0, 0, global_ns());
       }
     }
-  } else if (warp == kMma2) {
+  } else if (warp == kMma2Q) {
     if (lane == 0) {
       // ------------------------------------------------ MMA: products --
       // dQ (+)= dS_j K_j (dS from TMEM) into the item's accumulator.
@@ -622,8 +634,9 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     }
   } else {
     // -------------------------------------------------------- compute --
-    // thread = query row r, owning 64 of a key tile's 128 columns
-    const int qw = warp & 3, half = (warp - 2) >> 2;
+    // thread = query row r, owning kColsQ of a key tile's 128 columns (slot
+    // `part` of the row)
+    const int qw = warp & 3, part = (warp - 2) >> 2;
     const int r = qw * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
     uint32_t n_item = 0, gk = 0;
@@ -636,7 +649,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const int qi = i * kTile + r;  // this thread's query row
       const float lse2 = qi < T ? lse[(size_t)bh * T + qi] * kLog2e : 0.f;
       // D = rowsum(dO * O) of this row from the item's dO and O tiles (rows
-      // past T are zero-filled); stored with L for the dK/dV kernel
+      // past T are zero-filled; every thread of the row forms it); stored
+      // with L for the dK/dV kernel
       ok = warp_and(mbar_wait(qd_full, n_item & 1u, abort_flag, err));
       if (!ok) break;
       float drow = 0.f;
@@ -649,7 +663,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         for (int e = 0; e < 8; ++e) drow = fmaf(a[e], o[e], drow);
       }
       mbar_arrive(qd_empty);  // this thread is done with dO and O
-      if (half == 0)
+      if (part == 0)
         pairs[(size_t)bh * Tp + qi] = qi < T ? make_float2(lse2, drow) : make_float2(INFINITY, 0.f);
       for (int jj = 0; jj < n && ok; ++jj) {
         const uint32_t gg = gk + jj;
@@ -657,22 +671,23 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         ok = warp_and(mbar_wait(sd_full, gg & 1u, abort_flag, err));
         if (!ok) break;
         tc_fence_after();
-        uint32_t sr[64], dp[64];
-        tc_ld32(lane_base + 64 * half, sr);
-        tc_ld32(lane_base + 64 * half + 32, sr + 32);
-        tc_ld32(lane_base + kTile + 64 * half, dp);
-        tc_ld32(lane_base + kTile + 64 * half + 32, dp + 32);
+        uint32_t sr[kColsQ], dp[kColsQ];
+#pragma unroll
+        for (int c = 0; c < kColsQ; c += 32) {
+          tc_ld32(lane_base + kColsQ * part + c, sr + c);
+          tc_ld32(lane_base + kTile + kColsQ * part + c, dp + c);
+        }
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(sd_empty);  // S and dP are read: the next key tile's may be computed
         if (jj == i) {  // the diagonal tile: keys after the query are masked
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (64 * half + c > r) sr[c] = kNegInf;
+          for (int c = 0; c < kColsQ; ++c)
+            if (kColsQ * part + c > r) sr[c] = kNegInf;
         }
-        uint32_t dk[32];
+        uint32_t dk[kColsQ / 2];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
+        for (int c = 0; c < kColsQ; c += 2) {
           const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
           const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -lse2));
           dk[c / 2] = attn::pack_bf16x2(p0 * (__uint_as_float(dp[c]) - drow),
@@ -682,7 +697,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         ok = warp_and(mbar_wait(ds_empty0 + 8 * db, ((gg >> 1) & 1u) ^ 1u, abort_flag, err));
         if (!ok) break;
         tc_fence_after();
-        attn::tc_st32(lane_base + kDSCol + (uint32_t)(db * kHD) + 32 * half, dk);
+        tc_stn<kColsQ / 2>(lane_base + kDSCol + (uint32_t)(db * kHD) + (kColsQ / 2) * part, dk);
         attn::tc_wait_st();
         tc_fence_before();
         mbar_arrive(ds_full0 + 8 * db);
@@ -692,15 +707,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       ok = warp_and(mbar_wait(acc_full0 + 8 * ab, (n_item >> 1) & 1u, abort_flag, err));
       if (!ok) break;
       tc_fence_after();
-      uint32_t rq[32];
-      tc_ld32(lane_base + acc + 32 * half, rq);
+      constexpr int kAccCols = kHD / kQSplit;
+      uint32_t rq[kAccCols];
+      tc_ldn<kAccCols>(lane_base + acc + kAccCols * part, rq);
       tc_wait_ld();
       tc_fence_before();
       mbar_arrive(acc_empty0 + 8 * ab);
       if (qi < T) {
-        __nv_bfloat16* row = dqkv + ((size_t)b * T + qi) * 3 * C + (size_t)h * kHD + 32 * half;
+        __nv_bfloat16* row =
+            dqkv + ((size_t)b * T + qi) * 3 * C + (size_t)h * kHD + kAccCols * part;
 #pragma unroll
-        for (int q = 0; q < 32; q += 8) {
+        for (int q = 0; q < kAccCols; q += 8) {
           float a[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(rq[q + e]) * scale;
@@ -759,7 +776,7 @@ cudaError_t attention_bwd_tc(act_t* dqkv, float* scratch, const act_t* datt, con
   float2* pairs = reinterpret_cast<float2*>(scratch);
   // dQ first: it forms D = rowsum(dO * O) of its query tiles and stores the
   // (L, D) pairs for dK/dV
-  flash_bwd_dq_tc_kernel<<<grid, kThreadsBwd, sm_b, s>>>(tq, td, to, lse, pairs, dqkv, B, T, C, H,
+  flash_bwd_dq_tc_kernel<<<grid, kThreadsQ, sm_b, s>>>(tq, td, to, lse, pairs, dqkv, B, T, C, H,
                                                          sl2, scale, err);
   flash_bwd_dkdv_tc_kernel<<<grid, kThreadsKV, sm_a, s>>>(tq, td, pairs, dqkv, B, T, C, H, sl2,
                                                            scale, err);

@@ -49,7 +49,17 @@ using attn::kBox;
 using attn::kTile;
 
 constexpr int kKVStages = 4;
-constexpr int kRowThreads = 128;  // softmax threads per query tile
+// FWD_SPLIT softmax threads per query row (each owning 128 / FWD_SPLIT of a
+// key tile's columns; with more than one, the row max and the row sum meet
+// in shared memory behind bounded mbarrier waits).  Measured at B16 x T1024
+// x H12: 70.5 us with 1, 78.5 us with 2 (the exchange per key tile costs
+// more than the shorter rows save).
+#ifndef FWD_SPLIT
+#define FWD_SPLIT 1
+#endif
+constexpr int kFwdSplit = FWD_SPLIT;
+constexpr int kRowThreads = 128 * kFwdSplit;  // softmax threads per query tile
+constexpr int kColsF = kTile / kFwdSplit;      // key columns per softmax thread
 constexpr int kThreadsAttn = 64 + 2 * kRowThreads + 32;  // + the MMA warp of tile B
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 2 * kTile;         // O_t at kOCol + t * kHD
@@ -103,7 +113,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   const uint32_t p_full0 = s_full0 + 32;                         // [2 tiles]
   const uint32_t o_full0 = s_full0 + 48;                         // [2 tiles]
   const uint32_t drain0 = s_full0 + 64;                          // [2 tiles] abort path only
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 10);
+  const uint32_t xbar0 = s_full0 + 80;   // [2 tiles][2]: row-max exchange (FWD_SPLIT > 1)
+  const uint32_t xlbar0 = s_full0 + 112; // [2 tiles]: row-sum exchange (FWD_SPLIT > 1)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int nq = (T + kTile - 1) / kTile;
@@ -122,6 +134,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       mbar_init(p_full0 + 8 * t, kRowThreads);
       mbar_init(o_full0 + 8 * t, 1);
       mbar_init(drain0 + 8 * t, 1);
+      mbar_init(xbar0 + 16 * t, kRowThreads);
+      mbar_init(xbar0 + 16 * t + 8, kRowThreads);
+      mbar_init(xlbar0 + 8 * t, kRowThreads);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -249,13 +264,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else {
     // -------------------------------------------------------- softmax --
-    const int t = (warp - 2) >> 2;  // query tile of the item: 0 = A, 1 = B
+    const int t = (warp - 2) / (4 * kFwdSplit);        // query tile of the item: 0 = A, 1 = B
+    const int part = ((warp - 2) % (4 * kFwdSplit)) >> 2;  // this thread's slot of its row
     const int qw = warp & 3;        // TMEM lane quarter
     const int r = qw * 32 + lane;   // row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    const uint32_t s_col = lane_base + (uint32_t)(t * kTile);
-    const uint32_t o_col = lane_base + kOCol + (uint32_t)(t * kHD);
-    const uint32_t p_col = lane_base + kPCol + (uint32_t)(t * kHD);
+    const uint32_t s_col = lane_base + (uint32_t)(t * kTile + kColsF * part);
+    const uint32_t o_col = lane_base + kOCol + (uint32_t)(t * kHD + (kHD / kFwdSplit) * part);
+    const uint32_t p_col = lane_base + kPCol + (uint32_t)(t * kHD + (kColsF / 2) * part);
+    __shared__ float xch[2][2][kFwdSplit][kTile];  // [tile][step parity][part][row]
+    __shared__ float xch_l[2][kFwdSplit][kTile];   // [tile][part][row]
     uint32_t cs = 0, co = 0;  // S tiles read / PV products waited for by this tile's threads
     bool ok = true;
     // wait for the next PV product of this tile (every completion is
@@ -265,45 +283,56 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       ++co;
       return r2;
     };
+    uint32_t n_items = 0;  // items this tile has finished (row-sum exchanges)
     FwdItem it;
     for (int k = 0; ok && fwd_item(k, B, H, nq, it); ++k) {
       const int nk = t ? it.nkv_b : it.nkv_a;
       if (nk == 0) continue;  // the item has no tile B
       const int qt = t ? it.qb : it.qa;
       const int qi = qt * kTile + r;  // query index in the sequence
-      float m = -INFINITY, l = 0.f;  // reference max (log2 units) and the sum against it
+      float m = -INFINITY, l = 0.f;  // reference max (log2 units) and this thread's sum against it
       for (int j = 0; j < nk && ok; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * t, cs & 1u, abort_flag, err));
         if (!ok) break;
         ++cs;
         tc_fence_after();
-        // the whole row of S in one round trip; the buffer goes straight back
-        uint32_t sr[kTile];
-        tc_ld32(s_col, sr);
-        tc_ld32(s_col + 32, sr + 32);
-        tc_ld32(s_col + 64, sr + 64);
-        tc_ld32(s_col + 96, sr + 96);
+        // this thread's part of the row of S in one round trip; the buffer
+        // goes straight back
+        uint32_t sr[kColsF];
+#pragma unroll
+        for (int c = 0; c < kColsF; c += 32) tc_ld32(s_col + c, sr + c);
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(s_empty0 + 8 * t);  // S_t is read: the next S_t may be computed
         if (j == nk - 1) {  // the diagonal tile: keys after the query are masked
 #pragma unroll
-          for (int c = 0; c < kTile; ++c)
-            if (c > r) sr[c] = kNegInf;
+          for (int c = 0; c < kColsF; ++c)
+            if (kColsF * part + c > r) sr[c] = kNegInf;
         }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < kTile; c += 2)
+        for (int c = 0; c < kColsF; c += 2)
           mx4[(c >> 1) & 3] = attn::fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]),
                                           __uint_as_float(sr[c + 1]));
-        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+        float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        if (kFwdSplit > 1) {  // the row's max over its parts (bounded barrier wait)
+          const uint32_t sb = (cs - 1) & 1u;  // the S tiles read so far, this one included
+          xch[t][sb][part][r] = mt;
+          const uint32_t xb = xbar0 + 16 * t + 8 * sb;
+          mbar_arrive(xb);
+          ok = __all_sync(0xffffffffu, mbar_wait(xb, ((cs - 1) >> 1) & 1u, abort_flag, err));
+          if (!ok) break;
+#pragma unroll
+          for (int q = 0; q < kFwdSplit; ++q) mt = fmaxf(mt, xch[t][sb][q][r]);
+        }
+        mt *= sl2;
         const bool raise = mt > m + kRescaleLog2;  // always on the first key tile
         const float mn = raise ? mt : m;
         // P in registers (bf16 pairs) and its row sum
-        uint32_t pk[kTile / 2];
+        uint32_t pk[kColsF / 2];
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kTile / 2; ++c) {
+        for (int c = 0; c < kColsF / 2; ++c) {
           const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), sl2, -mn));
           const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -mn));
           sum4[(2 * c) & 3] += p0;
@@ -315,52 +344,61 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           ok = wait_pv();
           if (!ok) break;
           tc_fence_after();
-          if (raise) {  // rescale the row of O and the sum to the new reference
+          if (raise) {  // rescale this thread's part of the row of O and the sum
             const float f = fast_exp2(m - mn);
             l *= f;
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
+            for (int hf = 0; hf < kHD / kFwdSplit; hf += 32) {
               uint32_t o[32];
-              tc_ld32(o_col + 32 * hf, o);
+              tc_ld32(o_col + hf, o);
               tc_wait_ld();
 #pragma unroll
               for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-              attn::tc_st32(o_col + 32 * hf, o);
+              attn::tc_st32(o_col + hf, o);
             }
           }
         }
         m = mn;
-        attn::tc_st32(p_col, pk);
-        attn::tc_st32(p_col + 32, pk + 32);
+#pragma unroll
+        for (int c = 0; c < kColsF / 2; c += 32) attn::tc_st32(p_col + c, pk + c);
         attn::tc_wait_st();
         tc_fence_before();
         mbar_arrive(p_full0 + 8 * t);  // P_t (and a rescaled O_t) may be consumed
         l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       }
       if (!ok) break;
-      // the item's last product, then the normalised output row
+      if (kFwdSplit > 1) {  // the row's sum over its parts, in part order
+        xch_l[t][part][r] = l;
+        mbar_arrive(xlbar0 + 8 * t);
+        ok = __all_sync(0xffffffffu, mbar_wait(xlbar0 + 8 * t, n_items & 1u, abort_flag, err));
+        ++n_items;
+        if (!ok) break;
+        l = 0.f;
+#pragma unroll
+        for (int q = 0; q < kFwdSplit; ++q) l += xch_l[t][q][r];
+      }
+      // the item's last product, then this thread's part of the normalised row
       ok = wait_pv();
       if (!ok) break;
       tc_fence_after();
-      uint32_t ra[32], rb[32];
-      tc_ld32(o_col, ra);
-      tc_ld32(o_col + 32, rb);
+      constexpr int kOut = kHD / kFwdSplit;
+      uint32_t ra[kOut];
+#pragma unroll
+      for (int c = 0; c < kOut; c += 32) tc_ld32(o_col + c, ra + c);
       tc_wait_ld();
       tc_fence_before();  // O is read before the next item's first product overwrites it
       if (qi < T) {
         const float inv = 1.f / l;
-        __nv_bfloat16* dst = att + ((size_t)it.b * T + qi) * C + (size_t)it.h * kHD;
+        __nv_bfloat16* dst =
+            att + ((size_t)it.b * T + qi) * C + (size_t)it.h * kHD + (size_t)kOut * part;
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
+        for (int i = 0; i < kOut; i += 8) {
           float v[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) v[q] = __uint_as_float(ra[i + q]) * inv;
           store8(dst + i, v);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) v[q] = __uint_as_float(rb[i + q]) * inv;
-          store8(dst + 32 + i, v);
         }
-        lse[((size_t)it.b * H + it.h) * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
+        if (part == 0) lse[((size_t)it.b * H + it.h) * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
       }
     }
   }

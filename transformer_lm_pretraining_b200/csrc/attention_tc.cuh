@@ -11,7 +11,6 @@ namespace attn {
 constexpr int kHD = 64;
 constexpr int kTile = 128;  // query / key rows per tile
 constexpr int kBox = 16384;  // 128 rows x 64 bf16, 128-byte swizzle
-constexpr int kComputeThreads = 256;  // two threads per row (warps w, w+4)
 
 // bf16 x bf16 -> fp32, M = 128, N = n, A K-major, B K- or MN-major
 __host__ __device__ constexpr uint32_t idesc(int n, bool b_mn) {

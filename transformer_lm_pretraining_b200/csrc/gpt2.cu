@@ -995,6 +995,9 @@ gpt2_status gpt2_step_graph_capture(gpt2_t* h, const int32_t* tok_dev, const int
   h->graph = g;
   h->graph_exec = ex;
   h->graph_launches = launch_count() - n0;
+  // the one-time upload of the graph to the device, here rather than in the
+  // first replay
+  GPT2_CUDA(h, cudaGraphUpload(ex, h->stream));
   return GPT2_OK;
 }
 

@@ -76,15 +76,10 @@ struct alignas(16) Pack8 {
   act_t v[8];
 };
 
-// Rows staged through shared memory by bulk copies: TEAMS teams of TPR
-// threads per block, one row per team at a time, 8 columns per thread.  One
-// thread of each team keeps D of the team's next rows in flight (one
-// cp.async.bulk per row tensor, completing on the slot's mbarrier), so the
-// bytes in flight do not depend on registers; the team reads a row from its
-// slot, and the slot is refilled once every thread of the team has passed
-// the team's named barrier (or, for one-warp rows, its __syncwarp).  Row
-// sums go through a warp shuffle and, across the team's warps, shared memory
-// behind the named barrier: no block-wide barrier in the row loop.
+// Team kernels: TEAMS teams of TPR threads per block, one row per team at a
+// time, 8 columns per thread; row sums go through a warp shuffle and, across
+// the team's warps, shared memory behind a named barrier of the team alone:
+// no block-wide barrier in the row loop.
 template <int TPR>
 constexpr int ln_teams() {
   return TPR >= 256 ? 2 : (768 / TPR > 8 ? 8 : 768 / TPR);
@@ -112,122 +107,108 @@ __device__ __forceinline__ void chan_merge(float& mean, float& m2, float n, floa
   m2 = (m2 + m2_b) + d * d * (0.5f * n);
 }
 
+// The forward: each team keeps the loads of its next kRegDepth rows in
+// flight in registers (plain 16-byte loads; measured faster than bulk-copy
+// staging for this one-input kernel when the input is in L2, as the
+// residual stream is right after the GEMM that wrote it).  The row's mean
+// and sum of squared deviations come from each thread's own 8 values
+// (two-pass, exact) combined with chan_merge over the warp and, in warp
+// order, across the team's warps.
+constexpr int kRegDepth = 4;
 template <int TPR>
 __global__ void __launch_bounds__(TPR * ln_teams<TPR>())
-    ln_fwd_staged_kernel(act_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
-                         const act_t* __restrict__ x, const float* __restrict__ g,
-                         const float* __restrict__ b, int M) {
+    ln_fwd_reg_kernel(act_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
+                      const act_t* __restrict__ x, const float* __restrict__ g,
+                      const float* __restrict__ b, int M) {
   constexpr int TEAMS = ln_teams<TPR>();
   constexpr int WPR = TPR / 32;
   constexpr int C = 8 * TPR;
-  constexpr uint32_t kRowBytes = C * sizeof(act_t);
-  extern __shared__ __align__(128) uint8_t ln_smem[];
-  act_t* ring = reinterpret_cast<act_t*>(ln_smem);  // [TEAMS][kLnStages][C]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ln_smem + (size_t)TEAMS * kLnStages * kRowBytes);
   __shared__ float red[TEAMS][2][WPR][2];
   const int team = threadIdx.x / TPR, tc = threadIdx.x % TPR;
   const int wr = tc / 32, lane = threadIdx.x & 31;
   const int c = tc * 8;
   const int stride = gridDim.x * TEAMS;
   const int row0 = blockIdx.x * TEAMS + team;
-  const uint32_t bar0 = tc::smem_u32(bars + team * kLnStages);
-  const uint32_t slot0 = tc::smem_u32(ring + (size_t)team * kLnStages * C);
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < TEAMS * kLnStages; ++i) tc::mbar_init(tc::smem_u32(bars + i), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  auto issue = [&](int k) {  // row k of this team into slot k % kLnStages
-    const int row = row0 + k * stride;
-    if (row >= M) return;
-    const uint32_t bar = bar0 + 8 * (k % kLnStages);
-    tc::mbar_expect_tx(bar, kRowBytes);
-    tc::bulk_load_1d(slot0 + (uint32_t)(k % kLnStages) * kRowBytes, x + (size_t)row * C, kRowBytes,
-                     bar);
-  };
-  if (tc == 0)
-    for (int k = 0; k < kLnStages; ++k) issue(k);
   float gg[8], bb[8];
   load8(g + c, gg);
   load8(b + c, bb);
-  for (int k = 0;; ++k) {
-    const int row = row0 + k * stride;
-    if (row >= M) break;  // uniform over the team
-    const int st = k % kLnStages;
-    ln_slot_wait(bar0 + 8 * st, (uint32_t)(k / kLnStages) & 1u);
-    float v[8];
-    load8(ring + ((size_t)team * kLnStages + st) * C + c, v);
-    float mu = 0.f;
+  Pack8 buf[kRegDepth];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) mu += v[i];
-    mu *= 0.125f;
-    float m2 = 0.f;
+  for (int i = 0; i < kRegDepth; ++i) {
+    const int row = row0 + i * stride;
+    if (row < M) buf[i] = *reinterpret_cast<const Pack8*>(x + (size_t)row * C + c);
+  }
+  for (int k = 0;; k += kRegDepth) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m2 = fmaf(v[i] - mu, v[i] - mu, m2);
-    float n = 8.f;
+    for (int i = 0; i < kRegDepth; ++i) {
+      const int row = row0 + (k + i) * stride;
+      if (row >= M) return;  // uniform over the team
+      float v[8];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {  // pairwise merges over the warp
-      const float mb = __shfl_xor_sync(0xffffffffu, mu, o);
-      const float sb = __shfl_xor_sync(0xffffffffu, m2, o);
-      chan_merge(mu, m2, n, mb, sb);
-      n *= 2.f;
-    }
-    if (WPR > 1) {  // the team's warps, merged in warp order
-      float* rr = &red[team][k & 1][0][0];
-      if (lane == 0) {
-        rr[2 * wr] = mu;
-        rr[2 * wr + 1] = m2;
+      for (int e = 0; e < 8; ++e) v[e] = to_f(buf[i].v[e]);
+      const int nrow = row + kRegDepth * stride;
+      if (nrow < M) buf[i] = *reinterpret_cast<const Pack8*>(x + (size_t)nrow * C + c);
+      float mu = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mu += v[e];
+      mu *= 0.125f;
+      float m2 = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m2 = fmaf(v[e] - mu, v[e] - mu, m2);
+      float n = 8.f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float mb = __shfl_xor_sync(0xffffffffu, mu, o);
+        const float sb = __shfl_xor_sync(0xffffffffu, m2, o);
+        chan_merge(mu, m2, n, mb, sb);
+        n *= 2.f;
       }
-      asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "n"(TPR) : "memory");
-      mu = rr[0];
-      m2 = rr[1];
-      float na = 256.f;
+      if (WPR > 1) {
+        float* rr = &red[team][(k + i) & 1][0][0];
+        if (lane == 0) {
+          rr[2 * wr] = mu;
+          rr[2 * wr + 1] = m2;
+        }
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "n"(TPR) : "memory");
+        mu = rr[0];
+        m2 = rr[1];
+        float na = 256.f;
 #pragma unroll
-      for (int w = 1; w < WPR; ++w) {
-        const float d = rr[2 * w] - mu;
-        const float nn = na + 256.f;
-        mu = fmaf(d, 256.f / nn, mu);
-        m2 = m2 + rr[2 * w + 1] + d * d * (na * 256.f / nn);
-        na = nn;
+        for (int w = 1; w < WPR; ++w) {
+          const float d = rr[2 * w] - mu;
+          const float nn = na + 256.f;
+          mu = fmaf(d, 256.f / nn, mu);
+          m2 = m2 + rr[2 * w + 1] + d * d * (na * 256.f / nn);
+          na = nn;
+        }
       }
-    } else {
-      __syncwarp();
-    }
-    if (tc == 0) issue(k + kLnStages);  // every thread of the team has read the slot
-    const float rs = rsqrtf(m2 * (1.0f / C) + kLnEps);
-    Pack8 q;
+      const float rs = rsqrtf(m2 * (1.0f / C) + kLnEps);
+      Pack8 q;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q.v[i] = from_f<act_t>(fmaf((v[i] - mu) * rs, gg[i], bb[i]));
-    *reinterpret_cast<Pack8*>(y + (size_t)row * C + c) = q;
-    if (tc == 0) {
-      mean[row] = mu;
-      rstd[row] = rs;
+      for (int e = 0; e < 8; ++e) q.v[e] = from_f<act_t>(fmaf((v[e] - mu) * rs, gg[e], bb[e]));
+      *reinterpret_cast<Pack8*>(y + (size_t)row * C + c) = q;
+      if (tc == 0) {
+        mean[row] = mu;
+        rstd[row] = rs;
+      }
     }
   }
 }
 
 template <int TPR>
-constexpr size_t ln_fwd_smem() {
-  return (size_t)ln_teams<TPR>() * kLnStages * (8 * TPR * sizeof(act_t) + 8);
-}
-
-template <int TPR>
-void ln_fwd_staged_launch(act_t* y, float* mean, float* rstd, const act_t* x, const float* g,
-                          const float* b, int M, cudaStream_t s) {
+void ln_fwd_reg_launch(act_t* y, float* mean, float* rstd, const act_t* x, const float* g,
+                       const float* b, int M, cudaStream_t s) {
   constexpr int threads = TPR * ln_teams<TPR>();
-  constexpr size_t smem = ln_fwd_smem<TPR>();
   static int grid = 0;
   if (!grid) {
-    cudaFuncSetAttribute(ln_fwd_staged_kernel<TPR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
     int per_sm = 0, sms = 0, dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_fwd_staged_kernel<TPR>, threads, smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_fwd_reg_kernel<TPR>, threads, 0);
     grid = per_sm * sms;
     if (grid < 1) grid = sms;
   }
-  ln_fwd_staged_kernel<TPR><<<grid, threads, smem, s>>>(y, mean, rstd, x, g, b, M);
+  ln_fwd_reg_kernel<TPR><<<grid, threads, 0, s>>>(y, mean, rstd, x, g, b, M);
 }
 
 // grid = nblk blocks of 8 warps; warp w of block blk handles rows
@@ -324,9 +305,14 @@ __global__ void __launch_bounds__(256, 2)
   }
 }
 
-// The backward with the same staging as ln_fwd_staged_kernel: a slot holds
-// the row of x, of dy and (when accumulating) of dres, brought by one bulk
-// copy each; mean and rstd of the next rows are loaded into registers ahead.
+// The backward stages its rows through shared memory: one thread of each
+// team keeps kLnStages of the team's next rows in flight, a slot holding the
+// row of x, of dy and (when accumulating) of dres, brought by one
+// cp.async.bulk each and completing on the slot's mbarrier, so the bytes in
+// flight do not depend on registers; a slot is refilled once every thread
+// of the team has passed the team's named barrier (or, for one-warp rows,
+// its __syncwarp).  mean and rstd of the next rows are loaded into registers
+// ahead.
 // Every thread keeps the column sums of its 8 columns (and gamma) in
 // registers across its rows.  partials[blk][0..NSUMS) as the per-warp
 // kernel (teams added in team order).
@@ -550,7 +536,7 @@ void layernorm_fwd(act_t* y, float* mean, float* rstd, const act_t* x, const flo
   switch (C) {  // widths with a team kernel
 #define GPT2_LNFT(W)                                           \
   case W:                                                    \
-    ln_fwd_staged_launch<W / 8>(y, mean, rstd, x, g, b, M, s); \
+    ln_fwd_reg_launch<W / 8>(y, mean, rstd, x, g, b, M, s); \
     note_launch();                                           \
     return;
     GPT2_LNFT(256) GPT2_LNFT(512) GPT2_LNFT(768) GPT2_LNFT(1024) GPT2_LNFT(2048)
