@@ -39,13 +39,14 @@ from transformer_lm_pretraining_b200.workloads import WORKLOADS  # noqa: E402
 PAGES_A100_TOK_S = 16384 / 0.090  # 90 ms per 16x1024 step on 1x A100 SXM 80GB (pages)
 SPEC_BF16_DENSE = 2.25e15
 
-# DRAM bytes (read + write) per GEMM launch, averaged over the launches of a
-# gpt2_124m step, from an ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum, profiles/gemm_tc_dram_traffic_gpt2_124m_step.md).
-# Valid only for the GEMM sources it was taken on: reported as null as soon
-# as their hash differs.
-GEMM_TRAFFIC = {"bytes_per_launch": 1.4355e8,
-                "sources_sha256": "541d3f8b84ef68ffb52bb344510a9954c936a91357a1f668d61ac2c930077e5b"}
+# DRAM bytes (read + write) per GEMM launch, averaged over the 147 GEMM
+# launches of a gpt2_124m step: each of the step's 15 products captured alone
+# at full size, one launch, with ncu's dram__bytes_read.sum +
+# dram__bytes_write.sum, weighted by its launches per step
+# (profiles/gemm_tc_dram_traffic_gpt2_124m_step.md).  Valid only for the GEMM
+# sources it was taken on: reported as null as soon as their hash differs.
+GEMM_TRAFFIC = {"bytes_per_launch": 1.4416e8,
+                "sources_sha256": "57fd6054277f6e84e6c918e9fac54057f2ba420f1ad420da6ad1d6cf6b09db6f"}
 GEMM_SOURCES = ("gemm_tc.cu", "gemm_epi.cuh", "tc_util.cuh")
 
 

@@ -90,30 +90,44 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float* v) {
 // its derivative (the tanh form named on the condensed GPT-2 page).
 #if GPT2_ACT_BF16
 // bf16 build: the same function through the identity 0.5 (1 + tanh(u)) =
-// 1 / (1 + exp(-2u)), evaluated with the fast exp and divide intrinsics (two
-// special-function ops per element, accurate to a few fp32 ulps even where
-// 1 + tanh(u) is tiny), which keeps the GEMM epilogues off the critical path.
-__device__ __forceinline__ float gelu_sigmoid_arg(float x) {
-  const float k2 = 1.5957691216057308f;  // 2 sqrt(2/pi)
-  return fmaxf(k2 * (x + 0.044715f * x * x * x), -80.0f);  // exp(-2u) stays finite
+// 1 / (1 + exp(-2u)) = 1 / (1 + 2^(-2 u log2 e)), with the constants folded
+// so that x (1 + 2^(x (a + b x^2)))^-1 takes three multiply-adds and two
+// special-function ops (ex2, rcp).  Where 2^(...) overflows to +inf the
+// reciprocal is 0 and the result the limit, -0.  Accurate to a few fp32
+// ulps even where 1 + tanh(u) is tiny; these epilogues are instruction-bound,
+// so the count matters.
+__device__ __forceinline__ float ex2_hw(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_hw(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ float gelu_tanh(float x) {
-  return __fdividef(x, 1.0f + __expf(-gelu_sigmoid_arg(x)));
+  constexpr float kA = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2 e
+  constexpr float kB = kA * 0.044715f;
+  return x * rcp_hw(1.0f + ex2_hw(x * fmaf(kB, x * x, kA)));
 }
 // The derivative uses the hardware tanh (tanh.approx.f32, one special-function
-// op instead of two; relative error about 2^-11, so GELU'(x) is off by at most
-// about one bf16 ulp, the precision its product is stored in).  Measured: it
-// makes the GELU-backward GEMM epilogue 17 % faster; the forward keeps the
-// more accurate form above (no gain there).
+// op; relative error about 2^-11, so GELU'(x) is off by at most about one
+// bf16 ulp, the precision its product is stored in):
+//   GELU'(x) = 0.5 (1 + t) + 0.5 x (1 - t^2) du/dx,  t = tanh(u),
+//   du/dx = sqrt(2/pi) (1 + 3 * 0.044715 x^2).
 __device__ __forceinline__ float tanh_hw(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 __device__ __forceinline__ float gelu_tanh_grad(float x) {
-  const float k = 0.7978845608028654f;  // sqrt(2/pi)
-  const float t = tanh_hw(k * (x + 0.044715f * x * x * x));
-  return 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * k * (1.0f + 3.0f * 0.044715f * x * x);
+  constexpr float k = 0.7978845608028654f;  // sqrt(2/pi)
+  constexpr float kc = k * 0.044715f;
+  const float x2 = x * x;
+  const float t = tanh_hw(x * fmaf(kc, x2, k));
+  const float hs = (0.5f * x) * fmaf(-t, t, 1.0f);
+  return fmaf(hs, fmaf(3.0f * kc, x2, k), fmaf(0.5f, t, 0.5f));
 }
 #else
 __device__ __forceinline__ float gelu_tanh(float x) {

@@ -418,7 +418,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_wait_ld();
           if (g + 2 >= ngroups) release_acc(acc);  // every TMEM read of this warp for the tile is done
 #pragma unroll
-          for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]) * ep.alpha;
+          for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+        }
+        if (ep.alpha != 1.0f) {  // uniform: the forward and most gradients take alpha = 1
+#pragma unroll
+          for (int i = 0; i < 64; ++i) v[i] *= ep.alpha;
         }
         if (HAS_BIAS && ep.bias) {
           if (nb + 64 <= ep.N) {
