@@ -297,6 +297,7 @@ def run_ours(args, wl):
 
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
+    g2.gpt2k_set_programmatic_launch(args.pdl)
     model = g2.GPT2(wl.L, wl.H, wl.C, wl.V, wl.Vp, wl.Tmax, seed=0, precision="bf16",
                     B=wl.B, T=wl.T, recompute=args.recompute)
     evaluate = args.mode == "eval"
@@ -494,6 +495,7 @@ def run_ours(args, wl):
                                    or ("replicas" if world > 1 else "single-gpu")),
                    "mode": args.mode, "recompute": args.recompute,
                    "cuda_graph": bool(use_graph),
+                   "programmatic_launch": bool(args.pdl),
                    "l2": "no explicit flush: every step streams ~10 GB of activations, logits and "
                          "optimizer state through HBM, far above the 126 MB L2"},
         "mfu": mfu,
@@ -619,6 +621,9 @@ def main():
     ap.add_argument("--graph", type=int, default=1, choices=[0, 1],
                     help="1: time the training step replayed as one captured CUDA graph; "
                          "0: the eager calls")
+    ap.add_argument("--pdl", type=int, default=1, choices=[0, 1],
+                    help="1: kernels launched with programmatic dependent launch (the "
+                         "library's default); 0: plain launches")
     ap.add_argument("--recompute", type=int, default=0, choices=[0, 1],
                     help="1: recompute GELU in the backward instead of keeping it")
     args = ap.parse_args()

@@ -67,6 +67,18 @@ int gpt2k_gemm_expiry_test(void* stream, int M, int N, int K, const void* A, con
  * concurrent launches; returns the previous setting. */
 int gpt2k_gemm_set_cta_pairs(int enable);
 
+/* Whether the library's kernels are launched with programmatic stream
+ * serialization (programmatic dependent launch): a kernel may then be
+ * launched while the kernel before it in the stream is still finishing,
+ * its CTAs taking SMs as that kernel's leave and running their set-up
+ * (barriers, TMEM allocation) there; each kernel waits
+ * (griddepcontrol.wait) for the kernels before it to complete before it
+ * touches global memory, so results do not change.  enable = 0 or 1; the
+ * default is 1.  Process-wide, applies to launches made after the call
+ * (a CUDA graph keeps the setting it was captured with); returns the
+ * previous setting. */
+int gpt2k_set_programmatic_launch(int enable);
+
 /* Causal attention forward over qkv [B*T, 3C] = [q | k | v] (head h in
  * columns h*C/H .. of each part): att [B*T, C], lse [B, H, T] (natural-log
  * log-sum-exp of the scaled scores, fp32). */

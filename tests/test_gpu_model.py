@@ -444,3 +444,54 @@ def test_captured_step_equals_eager_steps():
     assert got == want
     assert ta == tb == 4
     assert np.array_equal(pa, pb) and np.array_equal(ma, mb) and np.array_equal(va, vb)
+
+
+def test_programmatic_launch_leaves_the_step_unchanged():
+    """Kernels launched with programmatic stream serialization (each waits
+    for its predecessors before touching global memory) give the same bits
+    as plain launches: two eager steps and two graph replays of a step with
+    a sequence of 1024 (several attention tiles, split-K weight gradients)."""
+    cfg = Config(2, 2, 128, 1000, 1024, 1024)
+    B, T = 2, 1024
+    s = ZipfStream(cfg.V, 5)
+    steps = [[s.next_batch(B, T)] for _ in range(4)]
+    stream = torch.cuda.Stream()
+
+    def run(pdl):
+        prev = g2.gpt2k_set_programmatic_launch(pdl)
+        try:
+            with torch.cuda.stream(stream):
+                m = g2.GPT2(*cfg.args, seed=11, precision="bf16", B=B, T=T)
+                m.set_stream(stream)
+                losses = []
+                for k in range(2):
+                    (tok, tgt), = steps[k]
+                    t, y = tok_tensors(tok, tgt)
+                    m.zero_grad()
+                    m.forward(t, y, sync_loss=False)
+                    m.backward(1.0)
+                    m.grad_norm_clip(1.0, sync=False)
+                    m.adamw_step(g2.gpt2_lr(k, 1e-3, 1e-4, 2, 10), 0.9, 0.95, 1e-8, 0.1)
+                    losses.append(m.read_loss())
+                stok = torch.empty(B * T, dtype=torch.int32, device="cuda")
+                stgt = torch.empty(B * T, dtype=torch.int32, device="cuda")
+                m.capture_step(stok, stgt, B, T, 1, 1.0, 1e-3, 1e-4, 2, 10)
+                for k in range(2, 4):
+                    (tok, tgt), = steps[k]
+                    t, y = tok_tensors(tok, tgt)
+                    stok.copy_(t.view(-1))
+                    stgt.copy_(y.view(-1))
+                    m.launch_step()
+                    losses.append(m.read_loss())
+                state = m.get_state()
+                grads = m.get_grads()
+                m.close()
+        finally:
+            g2.gpt2k_set_programmatic_launch(prev)
+        return losses, state, grads
+
+    off, on = run(0), run(1)
+    assert off[0] == on[0]
+    for a, b in zip(off[1][:3], on[1][:3]):
+        assert np.array_equal(a, b)
+    assert np.array_equal(off[2], on[2])

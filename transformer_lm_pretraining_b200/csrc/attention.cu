@@ -23,6 +23,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // D[b, h, t] = sum_d dO[t, h*hd + d] * O[t, h*hd + d]
 __global__ void attn_rowdot_kernel(float* __restrict__ dsum, const act_t* __restrict__ dout,
                                    const act_t* __restrict__ out, int B, int T, int C, int H) {
+  pdl_start();
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (size_t)B * T * H) return;
   const int hd = C / H;
@@ -164,6 +165,7 @@ template <int HD>
 __global__ void __launch_bounds__(kWarps * 32)
     flash_fwd_kernel(__nv_bfloat16* __restrict__ att, float* __restrict__ lse,
                      const __nv_bfloat16* __restrict__ qkv, int T, int C, int H, float sl2) {
+  pdl_start();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   FwdSmem<HD>& sm = *reinterpret_cast<FwdSmem<HD>*>(smem_raw);
   const int qb = gridDim.x - 1 - blockIdx.x;  // heaviest tiles first
@@ -276,6 +278,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                           const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
                           const float* __restrict__ dsum, int T, int C, int H, float sl2,
                           float scale) {
+  pdl_start();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BwdSmem<HD>& sm = *reinterpret_cast<BwdSmem<HD>*>(smem_raw);
   const int j = blockIdx.x;
@@ -380,6 +383,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                         const __nv_bfloat16* __restrict__ dout, const float* __restrict__ lse,
                         const float* __restrict__ dsum, int T, int C, int H, float sl2,
                         float scale) {
+  pdl_start();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BwdSmem<HD>& sm = *reinterpret_cast<BwdSmem<HD>*>(smem_raw);
   const int i = gridDim.x - 1 - blockIdx.x;  // heaviest tiles first
@@ -476,7 +480,7 @@ cudaError_t fwd_launch(act_t* att, float* lse, const act_t* qkv, int B, int T, i
   }
   const float sl2 = kLog2e / sqrtf((float)HD);
   dim3 grid((T + kTile - 1) / kTile, B * H);
-  flash_fwd_kernel<HD><<<grid, kWarps * 32, smem, s>>>(att, lse, qkv, T, C, H, sl2);
+  launch_kernel(flash_fwd_kernel<HD>, grid, kWarps * 32, smem, s, att, lse, qkv, T, C, H, sl2);
   note_launch();
   return cudaGetLastError();
 }
@@ -498,9 +502,9 @@ cudaError_t bwd_launch(act_t* dqkv, float* dsum, const act_t* datt, const act_t*
   const float sl2 = kLog2e / sqrtf((float)HD);
   const float scale = 1.f / sqrtf((float)HD);
   dim3 grid((T + kTile - 1) / kTile, B * H);
-  flash_bwd_dkdv_kernel<HD><<<grid, kWarps * 32, smem, s>>>(dqkv, qkv, datt, lse, dsum, T, C, H,
+  launch_kernel(flash_bwd_dkdv_kernel<HD>, grid, kWarps * 32, smem, s, dqkv, qkv, datt, lse, dsum, T, C, H,
                                                              sl2, scale);
-  flash_bwd_dq_kernel<HD><<<grid, kWarps * 32, smem, s>>>(dqkv, qkv, datt, lse, dsum, T, C, H,
+  launch_kernel(flash_bwd_dq_kernel<HD>, grid, kWarps * 32, smem, s, dqkv, qkv, datt, lse, dsum, T, C, H,
                                                            sl2, scale);
   note_launch(2);
   return cudaGetLastError();
@@ -513,6 +517,7 @@ constexpr int kMaxT = 2048;
 // Scores of row (b, h, i) against keys 0..i into sc (shared), then softmax.
 __global__ void naive_fwd_kernel(float* __restrict__ att, float* __restrict__ lse,
                                  const float* __restrict__ qkv, int B, int T, int C, int H) {
+  pdl_start();
   extern __shared__ float sc_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x / 32) + warp;  // over B*H*T
@@ -549,6 +554,7 @@ __global__ void naive_fwd_kernel(float* __restrict__ att, float* __restrict__ ls
 __global__ void naive_bwd_dq_kernel(float* __restrict__ dqkv, const float* __restrict__ qkv,
                                     const float* __restrict__ dout, const float* __restrict__ lse,
                                     const float* __restrict__ dsum, int B, int T, int C, int H) {
+  pdl_start();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x / 32) + warp;
   if (row >= B * H * T) return;
@@ -583,6 +589,7 @@ __global__ void naive_bwd_dkdv_kernel(float* __restrict__ dqkv, const float* __r
                                       const float* __restrict__ dout,
                                       const float* __restrict__ lse,
                                       const float* __restrict__ dsum, int B, int T, int C, int H) {
+  pdl_start();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x / 32) + warp;
   if (row >= B * H * T) return;
@@ -640,8 +647,8 @@ cudaError_t attention_fwd(act_t* att, float* lse, const act_t* qkv, int B, int T
                          warps * kMaxT * 4);
     attr = true;
   }
-  naive_fwd_kernel<<<(unsigned)((rows + warps - 1) / warps), warps * 32, warps * T * sizeof(float),
-                     s>>>(att, lse, qkv, B, T, C, H);
+  launch_kernel(naive_fwd_kernel, (unsigned)((rows + warps - 1) / warps), warps * 32, warps * T * sizeof(float),
+                     s, att, lse, qkv, B, T, C, H);
   note_launch();
   return cudaGetLastError();
 #endif
@@ -665,7 +672,7 @@ cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act
   if (hd == 64) return attention_bwd_tc(dqkv, dsum, datt, qkv, att, lse, B, T, C, H, err, s);
 #endif
   const size_t n = (size_t)B * T * H;
-  attn_rowdot_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(dsum, datt, att, B, T, C, H);
+  launch_kernel(attn_rowdot_kernel, (unsigned)((n + 255) / 256), 256, 0, s, dsum, datt, att, B, T, C, H);
   note_launch();
 #if GPT2_ACT_BF16
   switch (hd) {
@@ -678,8 +685,8 @@ cudaError_t attention_bwd(act_t* dqkv, float* dsum, const act_t* datt, const act
   const int warps = 4;
   const size_t rows = (size_t)B * H * T;
   const unsigned grid = (unsigned)((rows + warps - 1) / warps);
-  naive_bwd_dq_kernel<<<grid, warps * 32, 0, s>>>(dqkv, qkv, datt, lse, dsum, B, T, C, H);
-  naive_bwd_dkdv_kernel<<<grid, warps * 32, 0, s>>>(dqkv, qkv, datt, lse, dsum, B, T, C, H);
+  launch_kernel(naive_bwd_dq_kernel, grid, warps * 32, 0, s, dqkv, qkv, datt, lse, dsum, B, T, C, H);
+  launch_kernel(naive_bwd_dkdv_kernel, grid, warps * 32, 0, s, dqkv, qkv, datt, lse, dsum, B, T, C, H);
   note_launch(2);
   return cudaGetLastError();
 #endif

@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
                              const __grid_constant__ CUtensorMap tmDO,
                              const float2* __restrict__ pairs, __nv_bfloat16* __restrict__ dqkv,
                              int B, int T, int C, int H, float sl2, float scale, int* err) {
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // set-up done; the inputs written by the previous kernels are complete from here on
 
   if (warp == 0) {
     if (lane == 0) {
@@ -464,6 +466,7 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
                            const __grid_constant__ CUtensorMap tmO, const float* __restrict__ lse,
                            float2* __restrict__ pairs, __nv_bfloat16* __restrict__ dqkv, int B,
                            int T, int C, int H, float sl2, float scale, int* err) {
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -516,6 +519,7 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // set-up done; the inputs written by the previous kernels are complete from here on
 
   if (warp == 0) {
     if (lane == 0) {
@@ -776,9 +780,9 @@ cudaError_t attention_bwd_tc(act_t* dqkv, float* scratch, const act_t* datt, con
   float2* pairs = reinterpret_cast<float2*>(scratch);
   // dQ first: it forms D = rowsum(dO * O) of its query tiles and stores the
   // (L, D) pairs for dK/dV
-  flash_bwd_dq_tc_kernel<<<grid, kThreadsQ, sm_b, s>>>(tq, td, to, lse, pairs, dqkv, B, T, C, H,
+  launch_kernel(flash_bwd_dq_tc_kernel, grid, kThreadsQ, sm_b, s, tq, td, to, lse, pairs, dqkv, B, T, C, H,
                                                          sl2, scale, err);
-  flash_bwd_dkdv_tc_kernel<<<grid, kThreadsKV, sm_a, s>>>(tq, td, pairs, dqkv, B, T, C, H, sl2,
+  launch_kernel(flash_bwd_dkdv_tc_kernel, grid, kThreadsKV, sm_a, s, tq, td, pairs, dqkv, B, T, C, H, sl2,
                                                            scale, err);
   note_launch(2);
   return cudaGetLastError();

@@ -97,6 +97,7 @@ __device__ __forceinline__ bool fwd_item(int k, int B, int H, int nq, FwdItem& i
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     flash_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, __nv_bfloat16* __restrict__ att,
                         float* __restrict__ lse, int B, int T, int C, int H, float sl2, int* err) {
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // set-up done; the inputs written by the previous kernels are complete from here on
 
   if (warp == 0) {
     if (lane == 0) {
@@ -477,7 +479,7 @@ cudaError_t attention_fwd_tc(act_t* att, float* lse, const act_t* qkv, int B, in
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = items < sms ? items : sms;
-  flash_fwd_tc_kernel<<<grid, kThreadsAttn, smem, s>>>(tm, att, lse, B, T, C, H, sl2, err);
+  launch_kernel(flash_fwd_tc_kernel, grid, kThreadsAttn, smem, s, tm, att, lse, B, T, C, H, sl2, err);
   note_launch();
   return cudaGetLastError();
 }

@@ -17,6 +17,62 @@ namespace gpt2k {
 
 constexpr int kNumSMs = 148;
 
+// Programmatic dependent launch.  Every kernel of the library starts with
+// pdl_launch_dependents() (the kernel that follows it in the stream may be
+// launched as soon as every CTA of this one has started, so its CTAs take
+// SMs as this grid's CTAs leave and run their set-up, barriers and TMEM
+// allocation, there) and calls pdl_wait() before its first access to global
+// memory (it returns once the grids this one depends on have completed and
+// their writes are visible; at once when the launch had no programmatic
+// dependency).  So the launch latency and prologue of each kernel overlap
+// the tail of the one before, and no data is read or written early.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_start() {
+  pdl_launch_dependents();
+  pdl_wait();
+}
+
+// Whether launches carry the programmatic-serialization attribute (default
+// on; gpt2k_set_programmatic_launch).
+bool pdl_enabled();
+
+// kern<<<grid, block, smem, s>>>(args...) with the programmatic-serialization
+// attribute when enabled (and a cluster of `cluster` CTAs along x when > 1).
+template <typename... P, typename... A>
+cudaError_t launch_kernel_cluster(void (*kern)(P...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t s, int cluster, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  int n = 0;
+  if (pdl_enabled()) {
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = (unsigned)cluster;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = (unsigned)n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<A&&>(args)...);
+}
+template <typename... P, typename... A>
+cudaError_t launch_kernel(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          A&&... args) {
+  return launch_kernel_cluster(kern, grid, block, smem, s, 1, static_cast<A&&>(args)...);
+}
+
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
@@ -96,11 +152,6 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float* v) {
 // reciprocal is 0 and the result the limit, -0.  Accurate to a few fp32
 // ulps even where 1 + tanh(u) is tiny; these epilogues are instruction-bound,
 // so the count matters.
-__device__ __forceinline__ float ex2_hw(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 __device__ __forceinline__ float rcp_hw(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -109,7 +160,7 @@ __device__ __forceinline__ float rcp_hw(float x) {
 __device__ __forceinline__ float gelu_tanh(float x) {
   constexpr float kA = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2 e
   constexpr float kB = kA * 0.044715f;
-  return x * rcp_hw(1.0f + ex2_hw(x * fmaf(kB, x * x, kA)));
+  return x * rcp_hw(1.0f + fast_exp2(x * fmaf(kB, x * x, kA)));
 }
 // The derivative uses the hardware tanh (tanh.approx.f32, one special-function
 // op; relative error about 2^-11, so GELU'(x) is off by at most about one

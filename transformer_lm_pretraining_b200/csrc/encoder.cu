@@ -21,6 +21,7 @@ __global__ void encoder_fwd_kernel(act_t* __restrict__ x0, int* __restrict__ tok
                                    const int* __restrict__ tok, const act_t* __restrict__ wte,
                                    const act_t* __restrict__ wpe, int M, int T, int C, int V,
                                    int* err) {
+  pdl_start();
   const int m = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (m >= M) return;
   const int lane = threadIdx.x & 31;
@@ -46,6 +47,7 @@ __global__ void encoder_fwd_kernel(act_t* __restrict__ x0, int* __restrict__ tok
 // dwpe[t, c] += sum over b (ascending) of dx0[b T + t, c]
 __global__ void wpe_bwd_kernel(float* __restrict__ dwpe, const act_t* __restrict__ dx0, int B,
                                int T, int C) {
+  pdl_start();
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (size_t)T * C) return;
   const int t = (int)(i / C), c = (int)(i % C);
@@ -55,6 +57,7 @@ __global__ void wpe_bwd_kernel(float* __restrict__ dwpe, const act_t* __restrict
 }
 
 __global__ void iota_kernel(int* keys_out, int* vals_out, const int* keys_in, int M) {
+  pdl_start();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < M) {
     keys_out[i] = keys_in[i];
@@ -65,6 +68,7 @@ __global__ void iota_kernel(int* keys_out, int* vals_out, const int* keys_in, in
 // hist[d * ntiles + tile] = number of keys in the tile whose digit is d
 __global__ void radix_hist_kernel(int* __restrict__ hist, const int* __restrict__ keys, int M,
                                   int shift, int ntiles) {
+  pdl_start();
   __shared__ int h[256];
   for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0;
   __syncthreads();
@@ -76,6 +80,7 @@ __global__ void radix_hist_kernel(int* __restrict__ hist, const int* __restrict_
 
 // In-place exclusive scan of n ints by one block of 1024 threads.
 __global__ void exclusive_scan_kernel(int* data, int n) {
+  pdl_start();
   __shared__ int part[1024];
   const int per = (n + 1023) / 1024;
   const int b = threadIdx.x * per;
@@ -104,6 +109,7 @@ __global__ void __launch_bounds__(kSortTile)
     radix_scatter_kernel(int* __restrict__ keys_out, int* __restrict__ vals_out,
                          const int* __restrict__ keys_in, const int* __restrict__ vals_in,
                          const int* __restrict__ offsets, int M, int shift, int ntiles) {
+  pdl_start();
   __shared__ int cnt[32][257];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < 32 * 257; i += blockDim.x) (&cnt[0][0])[i] = 0;
@@ -138,6 +144,7 @@ __global__ void __launch_bounds__(kSortTile)
 __global__ void chunk_partial_kernel(float* __restrict__ partial, const act_t* __restrict__ dx0,
                                      const int* __restrict__ skeys, const int* __restrict__ svals,
                                      int M, int C) {
+  pdl_start();
   __shared__ int k_s[kChunk], v_s[kChunk];
   const int base = blockIdx.x * kChunk;
   const int n = min(kChunk, M - base);
@@ -171,6 +178,7 @@ __global__ void chunk_partial_kernel(float* __restrict__ partial, const act_t* _
 // add the run's chunk partials (in chunk order) into dwte[id].
 __global__ void segment_sum_kernel(float* __restrict__ dwte, const float* __restrict__ partial,
                                    const int* __restrict__ skeys, int M, int C) {
+  pdl_start();
   const int s = blockIdx.x;
   const int key = skeys[s];
   if (s > 0 && skeys[s - 1] == key) return;
@@ -188,7 +196,7 @@ void encoder_fwd(act_t* x0, int* tok_saved, const int* tok, const act_t* wte, co
                  int B, int T, int C, int V, int* err, cudaStream_t s) {
   const int M = B * T;
   const int warps = 8;
-  encoder_fwd_kernel<<<(M + warps - 1) / warps, warps * 32, 0, s>>>(x0, tok_saved, tok, wte, wpe,
+  launch_kernel(encoder_fwd_kernel, (M + warps - 1) / warps, warps * 32, 0, s, x0, tok_saved, tok, wte, wpe,
                                                                       M, T, C, V, err);
   note_launch();
 }
@@ -215,17 +223,17 @@ void encoder_scratch_carve(EncoderScratch* es, void* base, int M, int C) {
 void encoder_bwd(float* dwte, float* dwpe, const act_t* dx0, const int* tok_saved, int B, int T,
                  int C, int Vp, const EncoderScratch& es, cudaStream_t s) {
   const int M = B * T;
-  wpe_bwd_kernel<<<(int)(((size_t)T * C + 255) / 256), 256, 0, s>>>(dwpe, dx0, B, T, C);
+  launch_kernel(wpe_bwd_kernel, (int)(((size_t)T * C + 255) / 256), 256, 0, s, dwpe, dx0, B, T, C);
   // stable sort of (token, position) by token
   const int ntiles = (M + kSortTile - 1) / kSortTile;
-  iota_kernel<<<(M + 255) / 256, 256, 0, s>>>(es.keys[0], es.vals[0], tok_saved, M);
+  launch_kernel(iota_kernel, (M + 255) / 256, 256, 0, s, es.keys[0], es.vals[0], tok_saved, M);
   int bits = 0;
   while ((1 << bits) < Vp) ++bits;
   int cur = 0;
   for (int shift = 0; shift < bits; shift += 8) {
-    radix_hist_kernel<<<ntiles, kSortTile, 0, s>>>(es.hist, es.keys[cur], M, shift, ntiles);
-    exclusive_scan_kernel<<<1, 1024, 0, s>>>(es.hist, 256 * ntiles);
-    radix_scatter_kernel<<<ntiles, kSortTile, 0, s>>>(es.keys[cur ^ 1], es.vals[cur ^ 1],
+    launch_kernel(radix_hist_kernel, ntiles, kSortTile, 0, s, es.hist, es.keys[cur], M, shift, ntiles);
+    launch_kernel(exclusive_scan_kernel, 1, 1024, 0, s, es.hist, 256 * ntiles);
+    launch_kernel(radix_scatter_kernel, ntiles, kSortTile, 0, s, es.keys[cur ^ 1], es.vals[cur ^ 1],
                                                       es.keys[cur], es.vals[cur], es.hist, M,
                                                       shift, ntiles);
     cur ^= 1;
@@ -233,8 +241,8 @@ void encoder_bwd(float* dwte, float* dwpe, const act_t* dx0, const int* tok_save
   }
   const int nchunks = (M + kChunk - 1) / kChunk;
   dim3 g1(nchunks, (C / 2 + 127) / 128);
-  chunk_partial_kernel<<<g1, 128, 0, s>>>(es.partial, dx0, es.keys[cur], es.vals[cur], M, C);
-  segment_sum_kernel<<<M, 128, 0, s>>>(dwte, es.partial, es.keys[cur], M, C);
+  launch_kernel(chunk_partial_kernel, g1, 128, 0, s, es.partial, dx0, es.keys[cur], es.vals[cur], M, C);
+  launch_kernel(segment_sum_kernel, M, 128, 0, s, dwte, es.partial, es.keys[cur], M, C);
   note_launch(4);
 }
 

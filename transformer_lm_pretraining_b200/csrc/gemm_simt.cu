@@ -16,6 +16,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const float* __restrict_
                                                         int a_mn, const float* __restrict__ B,
                                                         long ldb, int b_mn, int K, EpiParams ep,
                                                         int k_begin_stride, long split_stride) {
+  pdl_start();
   __shared__ float sA[TK][TS + 1];
   __shared__ float sB[TK][TS + 1];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -71,6 +72,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const float* __restrict_
 
 __global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, int splits, int M,
                                      int N) {
+  pdl_start();
   const size_t total = (size_t)M * N;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -111,7 +113,7 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   switch (epi) {
 #define GPT2_SIMT(E)                                                                               \
   case E:                                                                                          \
-    gemm_simt_kernel<E><<<grid, 256, 0, s>>>(a.A, a.lda, a.a_mn, a.B, a.ldb, a.b_mn, a.K, ep, kchunk, \
+    launch_kernel(gemm_simt_kernel<E>, grid, 256, 0, s, a.A, a.lda, a.a_mn, a.B, a.ldb, a.b_mn, a.K, ep, kchunk, \
                                              split_stride);                                        \
     break;
     GPT2_SIMT(EPI_STORE)
@@ -132,7 +134,7 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
     const size_t total = (size_t)a.M * a.N;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 1184) blocks = 1184;
-    splitk_reduce_kernel<<<blocks, 256, 0, s>>>(a.out32, a.ldo32, a.split_ws, splits, a.M, a.N);
+    launch_kernel(splitk_reduce_kernel, blocks, 256, 0, s, a.out32, a.ldo32, a.split_ws, splits, a.M, a.N);
     note_launch();
     e = cudaGetLastError();
   }

@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // CTA pair: rank 0 (the leader) issues the MMAs for both CTAs; each CTA
   // loads its 128 rows of A and BN / 2 rows of B and runs the epilogue of
   // its 128 rows of the tile.
+  pdl_launch_dependents();
   const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
   const bool leader = rank == 0;
   constexpr bool F32_OUT = (EPI == EPI_F32_ACC || EPI == EPI_F32_STORE);
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // set-up done; the operands of the previous kernels are complete from here on
 
   auto decode = [&](int u, int& tm, int& tn, int& kb0, int& kb1, int& sp) {
     sp = u / tiles;
@@ -653,26 +655,11 @@ static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CU
   const int units = tiles_m * tiles_n * splits;
   const int slots = num_sms() / CG;  // persistent CTAs (pairs)
   const int grid = CG * (units < slots ? units : slots);
-  if (CG == 1) {
-    kern<<<grid, kThreads, smem, s>>>(ta, tb, to, tx, ep, K, tiles_m, tiles_n, splits,
-                                      kb_per_split, n_fast, err);
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = 2;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, to, tx, ep, K, tiles_m, tiles_n, splits,
-                                       kb_per_split, n_fast, err);
-    if (e != cudaSuccess) return e;
-  }
+  // a pair is a cluster of two CTAs along x
+  const cudaError_t e = launch_kernel_cluster(kern, dim3(grid), dim3(kThreads), smem, s, CG, ta, tb,
+                                              to, tx, ep, K, tiles_m, tiles_n, splits, kb_per_split,
+                                              n_fast, err);
+  if (e != cudaSuccess) return e;
   note_launch();
   return cudaGetLastError();
 }
@@ -703,6 +690,7 @@ static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUte
 
 __global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, int splits, int M,
                                      int N) {
+  pdl_start();
   const size_t total = (size_t)M * N;
   if (ldo32 == N && (total & 3) == 0) {  // contiguous output: float4 path
     const size_t t4 = total / 4;
@@ -829,7 +817,7 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
     int blocks = (int)((total / 4 + 255) / 256);
     if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
     if (blocks < 1) blocks = 1;
-    splitk_reduce_kernel<<<blocks, 256, 0, s>>>(a.out32, a.ldo32, a.split_ws, splits, a.M, a.N);
+    launch_kernel(splitk_reduce_kernel, blocks, 256, 0, s, a.out32, a.ldo32, a.split_ws, splits, a.M, a.N);
     note_launch();
     e = cudaGetLastError();
   }

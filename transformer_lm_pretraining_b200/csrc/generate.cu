@@ -17,6 +17,7 @@ constexpr int kSampleThreads = 1024;
 __global__ void decode_embed_kernel(act_t* __restrict__ x, const int* __restrict__ tok, int ld_tok,
                                     int p, const act_t* __restrict__ wte,
                                     const act_t* __restrict__ wpe, int C, int V, int* err) {
+  pdl_start();
   const int b = blockIdx.x;
   int t = tok[(size_t)b * ld_tok + p];
   if (t < 0 || t >= V) {
@@ -41,6 +42,7 @@ __global__ void __launch_bounds__(128)
     decode_attention_kernel(act_t* __restrict__ att, const act_t* __restrict__ q,
                             const act_t* __restrict__ kv, int Ttot, int n, int C, int H,
                             float scale) {
+  pdl_start();
   extern __shared__ float sc[];  // [n] scores, then [128 / hd][hd] partial outputs
   __shared__ float red[4], qv[256];
   const int h = blockIdx.x, b = blockIdx.y, hd = C / H;
@@ -145,6 +147,7 @@ __global__ void __launch_bounds__(kSampleThreads)
     sample_kernel(int* __restrict__ tok, int ld_tok, int p_out, const act_t* __restrict__ logits,
                   long ld_logits, int V, float temperature, int top_k, uint64_t seed,
                   float* __restrict__ logits_out) {
+  pdl_start();
   __shared__ float redf[kSampleThreads / 32];
   __shared__ int redi[kSampleThreads / 32];
   __shared__ float scan[kSampleThreads];
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(kSampleThreads)
 
 void decode_embed(act_t* x, const int* tok, int ld_tok, int p, const act_t* wte, const act_t* wpe,
                   int B, int C, int V, int* err, cudaStream_t s) {
-  decode_embed_kernel<<<B, 128, 0, s>>>(x, tok, ld_tok, p, wte, wpe, C, V, err);
+  launch_kernel(decode_embed_kernel, B, 128, 0, s, x, tok, ld_tok, p, wte, wpe, C, V, err);
   note_launch();
 }
 
@@ -228,7 +231,7 @@ void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int
                       int H, cudaStream_t s) {
   const int hd = C / H;  // <= 128 (checked by the caller)
   const size_t smem = ((size_t)n + 128) * sizeof(float);
-  decode_attention_kernel<<<dim3(H, B), 128, smem, s>>>(att, q, kv, Ttot, n, C, H,
+  launch_kernel(decode_attention_kernel, dim3(H, B), 128, smem, s, att, q, kv, Ttot, n, C, H,
                                                          1.0f / sqrtf((float)hd));
   note_launch();
 }
@@ -236,7 +239,7 @@ void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int
 void sample_tokens(int* tok, int ld_tok, int p_out, const act_t* logits, long ld_logits, int B,
                    int V, float temperature, int top_k, uint64_t seed, float* logits_out,
                    cudaStream_t s) {
-  sample_kernel<<<B, kSampleThreads, 0, s>>>(tok, ld_tok, p_out, logits, ld_logits, V, temperature,
+  launch_kernel(sample_kernel, B, kSampleThreads, 0, s, tok, ld_tok, p_out, logits, ld_logits, V, temperature,
                                              top_k, seed, logits_out);
   note_launch();
 }

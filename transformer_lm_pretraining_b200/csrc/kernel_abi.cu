@@ -27,6 +27,8 @@ extern "C" {
 
 int gpt2k_gemm_set_cta_pairs(int enable) { return gemm_set_cta_pairs(enable); }
 
+int gpt2k_set_programmatic_launch(int enable) { return set_pdl(enable); }
+
 int gpt2k_gemm(void* stream, int epi, int M, int N, int K, const void* A, long lda, int a_mn,
                const void* B, long ldb, int b_mn, float alpha, void* out, long ldo, float* out32,
                long ldo32, const float* bias, const void* resid, long ldr, void* aux, long ldaux,

@@ -187,6 +187,10 @@ void grad_sumsq(double* out, const float* g, size_t n, double* partials, cudaStr
 // scalars[S_NORM] = sqrt(*sumsq), scalars[S_CLIP] as grad_norm_clip
 void clip_from_sumsq(float* scalars, const double* sumsq, float max_norm, cudaStream_t s);
 
+// Programmatic dependent launch of every kernel (default on); returns the
+// previous setting.
+int set_pdl(int enable);
+
 // Process-wide count of kernel launches made by this library.
 void note_launch(int n = 1);
 long launch_count();

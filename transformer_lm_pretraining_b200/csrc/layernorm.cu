@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(256)
     ln_fwd_kernel(act_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
                   const act_t* __restrict__ x, const float* __restrict__ g,
                   const float* __restrict__ b, int M, int C) {
+  pdl_start();
   const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   if (row >= M) return;
   const int lane = threadIdx.x & 31;
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(TPR * ln_teams<TPR>())
     ln_fwd_reg_kernel(act_t* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd,
                       const act_t* __restrict__ x, const float* __restrict__ g,
                       const float* __restrict__ b, int M) {
+  pdl_start();
   constexpr int TEAMS = ln_teams<TPR>();
   constexpr int WPR = TPR / 32;
   constexpr int C = 8 * TPR;
@@ -208,7 +210,7 @@ void ln_fwd_reg_launch(act_t* y, float* mean, float* rstd, const act_t* x, const
     grid = per_sm * sms;
     if (grid < 1) grid = sms;
   }
-  ln_fwd_reg_kernel<TPR><<<grid, threads, 0, s>>>(y, mean, rstd, x, g, b, M);
+  launch_kernel(ln_fwd_reg_kernel<TPR>, grid, threads, 0, s, y, mean, rstd, x, g, b, M);
 }
 
 // grid = nblk blocks of 8 warps; warp w of block blk handles rows
@@ -225,6 +227,7 @@ __global__ void __launch_bounds__(256, 2)
                   const act_t* __restrict__ x, const float* __restrict__ mean,
                   const float* __restrict__ rstd, const float* __restrict__ g,
                   float* __restrict__ partials, int M, int C, int accumulate) {
+  pdl_start();
   extern __shared__ float red[];  // [8 warps][NSUMS][C]
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int nw = blockDim.x / 32;
@@ -327,6 +330,7 @@ __global__ void __launch_bounds__(TPR * ln_bwd_teams<TPR>())
                          const act_t* __restrict__ x, const float* __restrict__ mean,
                          const float* __restrict__ rstd, const float* __restrict__ g,
                          float* __restrict__ partials, int M, int accumulate) {
+  pdl_start();
   constexpr int TEAMS = ln_bwd_teams<TPR>();
   constexpr int WPR = TPR / 32;
   constexpr int C = 8 * TPR;
@@ -462,7 +466,7 @@ int ln_bwd_staged_launch(act_t* dres, const act_t* dy, const act_t* x, const flo
     grid = per_sm * sms;
     if (grid < 1 || grid > kLnBlocks) grid = kLnBlocks;
   }
-  ln_bwd_staged_kernel<TPR, S><<<grid, threads, smem, s>>>(dres, dy, x, mean, rstd, g, partials,
+  launch_kernel(ln_bwd_staged_kernel<TPR, S>, grid, threads, smem, s, dres, dy, x, mean, rstd, g, partials,
                                                            M, accumulate);
   return grid;
 }
@@ -474,6 +478,7 @@ int ln_bwd_staged_launch(act_t* dres, const act_t* dy, const act_t* x, const flo
 __global__ void __launch_bounds__(1024)
     ln_bwd_reduce_kernel(float* __restrict__ dg, float* __restrict__ db, float* __restrict__ dsum3,
                          const float* __restrict__ partials, int nblk, int nsums, int C) {
+  pdl_start();
   __shared__ float red[32][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + tx;  // over nsums * C
@@ -524,7 +529,7 @@ int ln_bwd_launch(act_t* dres, const act_t* dy, const act_t* x, const float* mea
     if (grid < 1 || grid > kLnBlocks) grid = kLnBlocks;
     grid_c = C;
   }
-  ln_bwd_kernel<N, S><<<grid, 256, smem, s>>>(dres, dy, x, mean, rstd, g, partials, M, C,
+  launch_kernel(ln_bwd_kernel<N, S>, grid, 256, smem, s, dres, dy, x, mean, rstd, g, partials, M, C,
                                               accumulate);
   return grid;
 }
@@ -547,7 +552,7 @@ void layernorm_fwd(act_t* y, float* mean, float* rstd, const act_t* x, const flo
   const int grid = (M + warps - 1) / warps;
   switch ((C + 255) / 256) {
 #define GPT2_LNF(N) \
-  case N: ln_fwd_kernel<N><<<grid, warps * 32, 0, s>>>(y, mean, rstd, x, g, b, M, C); break;
+  case N: launch_kernel(ln_fwd_kernel<N>, grid, warps * 32, 0, s, y, mean, rstd, x, g, b, M, C); break;
     GPT2_LNF(1) GPT2_LNF(2) GPT2_LNF(3) GPT2_LNF(4) GPT2_LNF(5) GPT2_LNF(6) GPT2_LNF(7) GPT2_LNF(8)
 #undef GPT2_LNF
     default: break;
@@ -585,7 +590,7 @@ void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* me
     default: break;
   }
 reduce:
-  ln_bwd_reduce_kernel<<<(nsums * C + 31) / 32, 1024, 0, s>>>(dg, db, dbias_out, partials, nblk,
+  launch_kernel(ln_bwd_reduce_kernel, (nsums * C + 31) / 32, 1024, 0, s, dg, db, dbias_out, partials, nblk,
                                                                nsums, C);
   note_launch(2);
 }

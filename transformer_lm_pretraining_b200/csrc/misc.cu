@@ -41,6 +41,14 @@ Layout make_layout(int L, int H, int C, int V, int Vp, int Tmax) {
 }
 
 static std::atomic<long> g_launches{0};
+static int g_pdl = 1;
+bool pdl_enabled() { return g_pdl != 0; }
+int set_pdl(int enable) {
+  const int prev = g_pdl;
+  g_pdl = enable ? 1 : 0;
+  return prev;
+}
+
 void note_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 long launch_count() { return g_launches.load(std::memory_order_relaxed); }
 
@@ -57,6 +65,7 @@ namespace {
 __global__ void __launch_bounds__(256)
     colsum_partial_kernel(float* __restrict__ partials, const act_t* __restrict__ dy, int M, int N,
                           int rows_per_chunk) {
+  pdl_start();
   __shared__ float red[8][256];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int n = blockIdx.x * 256 + lane * 8;
@@ -103,6 +112,7 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(1024)
     colsum_reduce_kernel(float* __restrict__ db, const float* __restrict__ partials, int chunks,
                          int N) {
+  pdl_start();
   __shared__ float red[32][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int n = blockIdx.x * 32 + tx;
@@ -137,6 +147,7 @@ __global__ void __launch_bounds__(kClsThreads)
     classifier_kernel(act_t* __restrict__ logits, float* __restrict__ losses,
                       const int* __restrict__ tgt, int M, int V, int Vp, int write_grad,
                       int* err) {
+  pdl_start();
   const int row = blockIdx.x;
   act_t* z = logits + (size_t)row * Vp;
   const int vec = (Vp % 8 == 0) ? 8 : 1;
@@ -241,6 +252,7 @@ __global__ void __launch_bounds__(THREADS, 2048 / THREADS / 1 > 2 ? 2 : 2048 / T
     classifier_bulk_kernel(act_t* __restrict__ logits, float* __restrict__ losses,
                            const int* __restrict__ tgt, int M, int V, int Vp, int write_grad,
                            int* err) {
+  pdl_start();
   using namespace tc;
   extern __shared__ __align__(128) uint8_t cls_smem[];
   __shared__ float red[THREADS / 32];
@@ -368,6 +380,7 @@ __global__ void __launch_bounds__(THREADS, 2048 / THREADS / 1 > 2 ? 2 : 2048 / T
 }
 
 __global__ void mean_loss_kernel(float* out, const float* __restrict__ losses, int M) {
+  pdl_start();
   __shared__ float red[1024];
   float s = 0.f;
   for (int i = threadIdx.x; i < M; i += blockDim.x) s += losses[i];
@@ -398,6 +411,7 @@ struct InitTable {
 };
 
 __global__ void init_normal_kernel(float* __restrict__ p, InitTable tab) {
+  pdl_start();
   const InitSeg sg = tab.seg[blockIdx.y];
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < sg.count;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -411,6 +425,7 @@ __global__ void init_normal_kernel(float* __restrict__ p, InitTable tab) {
 }
 
 __global__ void fill_kernel(float* p, size_t n, float v) {
+  pdl_start();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
     p[i] = v;
@@ -418,6 +433,7 @@ __global__ void fill_kernel(float* p, size_t n, float v) {
 
 template <class TO, class TI>
 __global__ void convert_kernel(TO* __restrict__ out, const TI* __restrict__ in, size_t n) {
+  pdl_start();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
     out[i] = from_f<TO>(to_f(in[i]));
@@ -430,6 +446,7 @@ __global__ void convert_kernel(TO* __restrict__ out, const TI* __restrict__ in, 
 __global__ void __launch_bounds__(256) norm_partial_kernel(double* __restrict__ partials,
                                                            const float* __restrict__ g,
                                                            size_t n) {
+  pdl_start();
   __shared__ double red[256];
   double s = 0.0;
   const size_t n4 = n / 4;
@@ -451,6 +468,7 @@ __global__ void __launch_bounds__(256) norm_partial_kernel(double* __restrict__ 
 
 __global__ void sumsq_final_kernel(double* __restrict__ out, const double* __restrict__ partials,
                                    int nblk) {
+  pdl_start();
   if (threadIdx.x != 0) return;
   double s = 0.0;
   for (int b = 0; b < nblk; ++b) s += partials[b];
@@ -459,6 +477,7 @@ __global__ void sumsq_final_kernel(double* __restrict__ out, const double* __res
 
 __global__ void clip_from_sumsq_kernel(float* __restrict__ scalars, const double* __restrict__ sumsq,
                                        float max_norm) {
+  pdl_start();
   const float nrm = (float)sqrt(*sumsq);
   scalars[S_NORM] = nrm;
   scalars[S_CLIP] = (nrm > max_norm) ? max_norm / (nrm + 1e-6f) : 1.0f;
@@ -466,6 +485,7 @@ __global__ void clip_from_sumsq_kernel(float* __restrict__ scalars, const double
 
 __global__ void norm_final_kernel(float* __restrict__ scalars, const double* __restrict__ partials,
                                   int nblk, float max_norm) {
+  pdl_start();
   if (threadIdx.x != 0) return;
   double s = 0.0;
   for (int b = 0; b < nblk; ++b) s += partials[b];
@@ -485,6 +505,7 @@ __global__ void __launch_bounds__(256)
     adamw_kernel(float* __restrict__ p, act_t* __restrict__ pact, const float* __restrict__ g,
                  float* __restrict__ m, float* __restrict__ v, size_t base, size_t n, AdamArgs a,
                  DecayTable dt, const float* __restrict__ scalars) {
+  pdl_start();
   const float nrm = scalars[S_NORM];
   if (!isfinite(nrm)) return;  // never apply a non-finite update
   const float clip = scalars[S_CLIP];
@@ -545,6 +566,7 @@ struct Sched {
 };
 __global__ void adam_prep_kernel(float* scalars, int* step, float lr, int scheduled, Sched sc,
                                  float b1, float b2) {
+  pdl_start();
   const int t = *step + 1;
   *step = t;
   double l = lr;
@@ -563,6 +585,7 @@ __global__ void adam_prep_kernel(float* scalars, int* step, float lr, int schedu
 }
 
 __global__ void reset_clip_kernel(float* scalars) {
+  pdl_start();
   scalars[S_NORM] = 0.f;
   scalars[S_CLIP] = 1.f;
 }
@@ -591,8 +614,8 @@ void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaS
   const int rows = (M + want - 1) / want;
   const int chunks = (M + rows - 1) / rows;
   dim3 g(colgroups, chunks);
-  colsum_partial_kernel<<<g, 256, 0, s>>>(partials, dy, M, N, rows);
-  colsum_reduce_kernel<<<(N + 31) / 32, 1024, 0, s>>>(db, partials, chunks, N);
+  launch_kernel(colsum_partial_kernel, g, 256, 0, s, partials, dy, M, N, rows);
+  launch_kernel(colsum_reduce_kernel, (N + 31) / 32, 1024, 0, s, db, partials, chunks, N);
   note_launch(2);
 }
 
@@ -617,20 +640,21 @@ void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int slots = kClsCtasPerSm * sms;
     const int grid = M < slots ? M : slots;
-    kern<<<grid, kThr, smem, s>>>(logits, losses, tgt, M, V, Vp, write_grad, err);
+    launch_kernel(kern, grid, kThr, smem, s, logits, losses, tgt, M, V, Vp, write_grad, err);
   } else {
-    classifier_kernel<<<M, kClsThreads, 0, s>>>(logits, losses, tgt, M, V, Vp, write_grad, err);
+    launch_kernel(classifier_kernel, M, kClsThreads, 0, s, logits, losses, tgt, M, V, Vp, write_grad, err);
   }
   note_launch();
 }
 
 void mean_loss(float* out, const float* losses, int M, cudaStream_t s) {
-  mean_loss_kernel<<<1, 1024, 0, s>>>(out, losses, M);
+  launch_kernel(mean_loss_kernel, 1, 1024, 0, s, out, losses, M);
   note_launch();
 }
 
 namespace {
 __global__ void gelu_fwd_kernel(act_t* __restrict__ g, const act_t* __restrict__ u, size_t n) {
+  pdl_start();
   const size_t n8 = n / 8;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -648,7 +672,7 @@ __global__ void gelu_fwd_kernel(act_t* __restrict__ g, const act_t* __restrict__
 
 void gelu_fwd(act_t* g, const act_t* u, size_t n, cudaStream_t s) {
   if (!n) return;
-  gelu_fwd_kernel<<<grid_for(n / 8 + 1, 256, 8 * kNumSMs), 256, 0, s>>>(g, u, n);
+  launch_kernel(gelu_fwd_kernel, grid_for(n / 8 + 1, 256, 8 * kNumSMs), 256, 0, s, g, u, n);
   note_launch();
 }
 
@@ -656,7 +680,7 @@ void init_params(float* p, const Layout& lay, uint64_t seed, cudaStream_t s) {
   cudaMemsetAsync(p, 0, lay.total * sizeof(float), s);
   const int gains[3] = {T_LN1G, T_LN2G, T_LNFG};
   for (int t : gains)
-    fill_kernel<<<grid_for(lay.num[t], 256, 1024), 256, 0, s>>>(p + lay.off[t], lay.num[t], 1.0f);
+    launch_kernel(fill_kernel, grid_for(lay.num[t], 256, 1024), 256, 0, s, p + lay.off[t], lay.num[t], 1.0f);
   InitTable tab;
   tab.n = 0;
   const double sd = 0.02, sd_res = 0.02 / sqrt(2.0 * lay.L);
@@ -675,35 +699,35 @@ void init_params(float* p, const Layout& lay, uint64_t seed, cudaStream_t s) {
     if (sg.count > maxc) maxc = sg.count;
   }
   dim3 grid(grid_for(maxc, 256, 2048), tab.n);
-  init_normal_kernel<<<grid, 256, 0, s>>>(p, tab);
+  launch_kernel(init_normal_kernel, grid, 256, 0, s, p, tab);
   note_launch(4);
 }
 
 void f32_to_act(act_t* out, const float* in, size_t n, cudaStream_t s) {
-  convert_kernel<act_t, float><<<grid_for(n, 256, 4096), 256, 0, s>>>(out, in, n);
+  launch_kernel(convert_kernel<act_t, float>, grid_for(n, 256, 4096), 256, 0, s, out, in, n);
   note_launch();
 }
 
 void act_to_f32(float* out, const act_t* in, size_t n, cudaStream_t s) {
-  convert_kernel<float, act_t><<<grid_for(n, 256, 4096), 256, 0, s>>>(out, in, n);
+  launch_kernel(convert_kernel<float, act_t>, grid_for(n, 256, 4096), 256, 0, s, out, in, n);
   note_launch();
 }
 
 void grad_norm_clip(float* scalars, const float* g, size_t n, float max_norm, double* partials,
                     cudaStream_t s) {
-  norm_partial_kernel<<<kNormBlocks, 256, 0, s>>>(partials, g, n);
-  norm_final_kernel<<<1, 32, 0, s>>>(scalars, partials, kNormBlocks, max_norm);
+  launch_kernel(norm_partial_kernel, kNormBlocks, 256, 0, s, partials, g, n);
+  launch_kernel(norm_final_kernel, 1, 32, 0, s, scalars, partials, kNormBlocks, max_norm);
   note_launch(2);
 }
 
 void grad_sumsq(double* out, const float* g, size_t n, double* partials, cudaStream_t s) {
-  norm_partial_kernel<<<kNormBlocks, 256, 0, s>>>(partials, g, n);
-  sumsq_final_kernel<<<1, 32, 0, s>>>(out, partials, kNormBlocks);
+  launch_kernel(norm_partial_kernel, kNormBlocks, 256, 0, s, partials, g, n);
+  launch_kernel(sumsq_final_kernel, 1, 32, 0, s, out, partials, kNormBlocks);
   note_launch(2);
 }
 
 void clip_from_sumsq(float* scalars, const double* sumsq, float max_norm, cudaStream_t s) {
-  clip_from_sumsq_kernel<<<1, 1, 0, s>>>(scalars, sumsq, max_norm);
+  launch_kernel(clip_from_sumsq_kernel, 1, 1, 0, s, scalars, sumsq, max_norm);
   note_launch();
 }
 
@@ -711,12 +735,12 @@ void adam_prep(float* scalars, int* step, float lr, bool scheduled, const double
                float b2, cudaStream_t s) {
   Sched sc{0.0, 0.0, 1.0, 1.0};
   if (scheduled) sc = Sched{sched[0], sched[1], sched[2], sched[3]};
-  adam_prep_kernel<<<1, 1, 0, s>>>(scalars, step, lr, scheduled ? 1 : 0, sc, b1, b2);
+  launch_kernel(adam_prep_kernel, 1, 1, 0, s, scalars, step, lr, scheduled ? 1 : 0, sc, b1, b2);
   note_launch();
 }
 
 void reset_clip(float* scalars, cudaStream_t s) {
-  reset_clip_kernel<<<1, 1, 0, s>>>(scalars);
+  launch_kernel(reset_clip_kernel, 1, 1, 0, s, scalars);
   note_launch();
 }
 
@@ -732,7 +756,7 @@ void adamw(float* p, act_t* pact, const float* g, float* m, float* v, const Layo
     }
   if (end > lay.total) end = lay.total;
   if (begin >= end) return;
-  adamw_kernel<<<grid_for((end - begin) / 4, 256, kNumSMs * 8), 256, 0, s>>>(
+  launch_kernel(adamw_kernel, grid_for((end - begin) / 4, 256, kNumSMs * 8), 256, 0, s, 
       p, pact, g, m, v, begin, end - begin, a, dt, scalars);
   note_launch();
 }

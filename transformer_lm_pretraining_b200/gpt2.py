@@ -80,6 +80,7 @@ SIGNATURES = {
     "gpt2_profile_enable": (_i, [_vp, _i]),
     "gpt2_profile_read": (_i, [_vp, ctypes.POINTER(_d), ctypes.POINTER(_l), ctypes.POINTER(_d), _i]),
     "gpt2k_gemm_set_cta_pairs": (_i, [_i]),
+    "gpt2k_set_programmatic_launch": (_i, [_i]),
     "gpt2k_gemm": (_i, [_vp, _i, _i, _i, _i, _vp, _l, _i, _vp, _l, _i, _f, _vp, _l, _fp, _l, _fp,
                         _vp, _l, _vp, _l, _fp, _sz]),
     "gpt2k_attention_fwd": (_i, [_vp, _vp, _fp, _vp, _i, _i, _i, _i]),
@@ -399,6 +400,12 @@ def gpt2k_gemm_set_cta_pairs(enable, precision="bf16"):
     """Run wide products as 256 x 256 tiles over CTA pairs (1, the default)
     or as 128 x 256 tiles on single CTAs (0); returns the previous setting."""
     return load(precision).gpt2k_gemm_set_cta_pairs(1 if enable else 0)
+
+
+def gpt2k_set_programmatic_launch(enable, precision="bf16"):
+    """Programmatic dependent launch of the library's kernels on (1, the
+    default) or off (0); returns the previous setting."""
+    return load(precision).gpt2k_set_programmatic_launch(1 if enable else 0)
 
 
 def gpt2k_gemm(epi, M, N, K, A, lda, a_mn, B, ldb, b_mn, alpha=1.0, out=None, ldo=0, out32=None,
