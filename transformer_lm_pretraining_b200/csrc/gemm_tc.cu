@@ -764,6 +764,8 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   // split count with the lowest estimated time = whole waves of units at
   // ~8.5 TFLOP/s per SM + the partials' write/read and the output update
   // at ~6 TB/s (at least 4 k-blocks per split; partials must fit)
+  // (a two-way split into a zero accumulator adds both partials in place:
+  // no partials to write and read back)
   int splits = 1;
   int epi = a.epi;
   if (a.epi == EPI_F32_ACC && a.max_splits > 1 && a.split_ws && tiles < slots &&
@@ -774,7 +776,9 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
       if (sp > 1 && (sp > kb_total / 4 || (size_t)sp * a.M * a.N > a.split_ws_floats)) break;
       const int waves = (tiles * sp + slots - 1) / slots;
       const double t_unit = 2.0 * BM * BN * ((double)kb_total * BK / sp) / 8.5e12;
-      const double t_red = sp > 1 ? (2.0 * sp + 2.0) * out_bytes / 6.0e12 : 0.0;
+      const double t_red = sp == 1 ? 0.0
+                           : (sp == 2 && a.acc_zero) ? out_bytes / 6.0e12
+                                                     : (2.0 * sp + 2.0) * out_bytes / 6.0e12;
       const double t = waves * t_unit + t_red;
       if (t < best * 0.98) {
         best = t;
@@ -784,12 +788,13 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   }
   int kb_per_split = (kb_total + splits - 1) / splits;
   splits = (kb_total + kb_per_split - 1) / kb_per_split;  // no empty split
+  const bool in_place = splits == 2 && a.acc_zero;  // both halves reduce-add into out32
   if (!a.b_mn) e = make_tmap(&tb, a.B, false, a.K, a.N, a.ldb, 64, BN / CG);
   else e = make_tmap(&tb, a.B, false, a.N, a.K, a.ldb, 64, 64);
   if (e != cudaSuccess) return e;
   // epilogue tensor maps
   // epilogue tensor maps: one warp's 32-row slab per box
-  if (splits > 1) {
+  if (splits > 1 && !in_place) {
     epi = EPI_F32_STORE;
     e = make_tmap(&to, a.split_ws, true, a.N, a.M, a.N, 32, 32, splits, (uint64_t)a.M * a.N);
   } else if (f32_out) {
@@ -812,7 +817,7 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   else
     e = dispatch<128, 1>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
   if (e != cudaSuccess) return e;
-  if (splits > 1) {
+  if (splits > 1 && !in_place) {
     const size_t total = (size_t)a.M * a.N;
     int blocks = (int)((total / 4 + 255) / 256);
     if (blocks > 8 * num_sms()) blocks = 8 * num_sms();

@@ -83,6 +83,9 @@ struct gpt2 {
   int B = 0, T = 0;
   bool have_grad_logits = false;
   bool have_logits = false;
+  // every gradient is zero (gpt2_zero_grad since the last backward), so the
+  // first backward's two-way split weight gradients may add in place
+  bool grads_zero = false;
   Acts a{};
   std::string last_error;
   // events recorded after each layer's backward (and the last one after the
@@ -664,6 +667,7 @@ gpt2_status gpt2_zero_grad(gpt2_t* h) {
   gpt2_status st = ensure_state(h);
   if (st) return st;
   GPT2_CUDA(h, cudaMemsetAsync(h->grads, 0, h->lay.total * sizeof(float), h->stream));
+  h->grads_zero = true;
   return GPT2_OK;
 }
 
@@ -671,6 +675,8 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
   if (!h) return GPT2_ERR_ARG;
   if (!h->have_grad_logits)
     return fail(h, GPT2_ERR_STATE, "backward needs a preceding forward with targets");
+  const int acc_zero = h->grads_zero ? 1 : 0;
+  h->grads_zero = false;
   const Layout& y = h->lay;
   Acts& a = h->a;
   const int B = h->B, T = h->T, M = B * T, C = y.C, L = y.L, H = y.H;
@@ -697,6 +703,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     ga.epi = EPI_F32_ACC; ga.alpha = loss_scale;
     ga.out32 = G + y.off[T_WTE]; ga.ldo32 = C;
     ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+    ga.acc_zero = acc_zero;
     GPT2_TRY(run_gemm(h, ga));
   }
   mark(h, PK_LN_BWD);
@@ -737,6 +744,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.epi = EPI_F32_ACC;
       ga.out32 = G + y.off[T_WP] + (size_t)l * 4 * C * C; ga.ldo32 = 4 * C;
       ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+      ga.acc_zero = acc_zero;
       GPT2_TRY(run_gemm(h, ga));
     }
     {  // dh = du Wfc
@@ -754,6 +762,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.epi = EPI_F32_ACC;
       ga.out32 = G + y.off[T_WFC] + (size_t)l * 4 * C * C; ga.ldo32 = C;
       ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+      ga.acc_zero = acc_zero;
       GPT2_TRY(run_gemm(h, ga));
     }
     mark(h, PK_LN_BWD);
@@ -778,6 +787,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.epi = EPI_F32_ACC;
       ga.out32 = G + y.off[T_WO] + (size_t)l * C * C; ga.ldo32 = C;
       ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+      ga.acc_zero = acc_zero;
       GPT2_TRY(run_gemm(h, ga));
     }
     mark(h, PK_ATTN_BWD, 10.0 * B * H * (double)T * (T + 1) / 2 * (C / H));
@@ -801,6 +811,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.epi = EPI_F32_ACC;
       ga.out32 = G + y.off[T_WQKV] + (size_t)l * 3 * C * C; ga.ldo32 = C;
       ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
+      ga.acc_zero = acc_zero;
       GPT2_TRY(run_gemm(h, ga));
     }
     mark(h, PK_LN_BWD);

@@ -50,6 +50,11 @@ struct GemmArgs {
   // split-K (EPI_F32_ACC only): partial sums go to split_ws, then a
   // fixed-order reduction adds them into out32.  max_splits = 1 disables.
   float* split_ws; size_t split_ws_floats; int max_splits;
+  // EPI_F32_ACC: out32 is known to hold zeros.  A split in two may then add
+  // both partials straight into out32 (TMA reduce-add, no workspace, no
+  // reduction kernel): 0 + a + b is the same float in either order (and the
+  // reduction's 0 + (a + b)), so the result stays deterministic.
+  int acc_zero;
   // Test of the bounded waits only: n > 0 makes CTA 0's producer skip the
   // load of k-block n - 1 of its first tile, so that the MMA's wait for it
   // expires (error word ERR_TIMEOUT) and the kernel takes its abort path.
