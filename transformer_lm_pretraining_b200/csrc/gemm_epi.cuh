@@ -15,6 +15,7 @@ struct EpiParams {
   const act_t* resid; long ldr;
   act_t* aux; long ldaux;
   int expiry_test;  // GemmArgs::expiry_test
+  float* colsum;    // GemmArgs::colsum
 };
 
 // One output element (any epilogue kind).

@@ -542,6 +542,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(box + swz(lane, j)), v + 8 * j);
               },
               [&](uint32_t box_u) { tma_store_3d(&tmOut, box_u, nb, r0, 0); });
+          if (EPI == EPI_DGELU && ep.colsum) {
+            // column sums of the stored slab: lane l adds columns 2l, 2l + 1
+            // of the box's rows in order (the TMA store reads the same box;
+            // the next group's writes wait for both)
+            const uint8_t* box = wbox + (ob ^ (OUT_BOXES == 2 ? 1 : 0)) * kWarpBox;
+            const int rows = min(32, ep.M - r0);
+            const uint32_t cof = (uint32_t)(lane & 3) * 4u;
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+            for (int r = 0; r < rows; ++r) {
+              const uint32_t w = *reinterpret_cast<const uint32_t*>(box + swz(r, lane >> 2) + cof);
+              s0 += __uint_as_float(w << 16);
+              s1 += __uint_as_float(w & 0xffff0000u);
+            }
+            const int col = nb + 2 * lane;
+            if (col < ep.N)  // N even: both columns in range
+              *reinterpret_cast<float2*>(ep.colsum + (size_t)(r0 >> 5) * ep.N + col) =
+                  make_float2(s0, s1);
+          }
         }
       }
       acc ^= 1;
@@ -718,6 +737,8 @@ __global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, 
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+bool gemm_colsum_supported() { return true; }
+
 static int g_cta_pairs = 1;
 int gemm_set_cta_pairs(int enable) {
   const int prev = g_cta_pairs;
@@ -748,8 +769,9 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   else e = make_tmap(&ta, a.A, false, a.M, a.K, a.lda, 64, 64);
   if (e != cudaSuccess) return e;
 
+  if (a.colsum && (a.epi != EPI_DGELU || a.N % 2 || !aligned16(a.colsum))) return cudaErrorInvalidValue;
   EpiParams ep{a.M, a.N, a.alpha, a.out, a.ldo, a.out32, a.ldo32, a.bias, a.resid, a.ldr, a.aux, a.ldaux,
-               a.expiry_test};
+               a.expiry_test, a.colsum};
   // 256 x 256 tiles over CTA pairs for the wide products (measured: 5-11 %
   // faster where the main loop sets the pace).  The GELU and GELU-backward
   // epilogues set the pace of their products; there the pair waits for the

@@ -728,11 +728,17 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.B = W + y.off[T_WP] + (size_t)l * 4 * C * C; ga.ldb = 4 * C; ga.b_mn = 1;
       ga.epi = EPI_DGELU; ga.aux = const_cast<act_t*>(u); ga.ldaux = 4 * C;
       ga.out = a.dbig; ga.ldo = 4 * C;
+      // the bias gradient of W_fc: per-32-row column sums of du from the
+      // epilogue (into the split-K workspace, free until dWp below), or a
+      // pass over du while it is still in L2
+      const int slabs = (M + 31) / 32;
+      const bool fused = gemm_colsum_supported() && (size_t)slabs * 4 * C <= a.splitk_floats;
+      if (fused) ga.colsum = a.splitk;
       GPT2_TRY(run_gemm(h, ga));
+      mark(h, PK_COLSUM);
+      if (fused) colsum_reduce(G + y.off[T_BFC] + (size_t)l * 4 * C, a.splitk, slabs, 4 * C, s);
+      else colsum_acc(G + y.off[T_BFC] + (size_t)l * 4 * C, a.dbig, M, 4 * C, a.partials, s);
     }
-    // the bias gradient of W_fc while du is still in L2
-    mark(h, PK_COLSUM);
-    colsum_acc(G + y.off[T_BFC] + (size_t)l * 4 * C, a.dbig, M, 4 * C, a.partials, s);
     if (h->recompute) {  // g = gelu(u), as the forward's epilogue computed it
       mark(h, PK_RECOMPUTE);
       gelu_fwd(const_cast<act_t*>(g), u, 4 * MC, s);

@@ -60,7 +60,14 @@ struct GemmArgs {
   // expires (error word ERR_TIMEOUT) and the kernel takes its abort path.
   // 0 (the value of a zero-initialised GemmArgs) in every product call.
   int expiry_test;
+  // EPI_DGELU (when gemm_colsum_supported()): if set, colsum[s * N + n] =
+  // the sum of the stored (bf16) output over rows 32 s .. 32 s + 31 of
+  // column n, added in row order; [ceil(M / 32)][N] floats, N even,
+  // 16-byte aligned.  The bias gradient of the product whose output gradient
+  // this is, without a second pass over it.
+  float* colsum;
 };
+bool gemm_colsum_supported();
 
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err_flag);
 // Whether wide products run as 256 x 256 tiles over CTA pairs (default on;
@@ -103,6 +110,9 @@ void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* me
 constexpr int kColsumChunks = 192;
 // db[n] += sum_m dy[m, n] (fixed order); partials: [kColsumChunks * N] floats
 void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s);
+// db[n] += sum over c < chunks of partials[c * N + n], c ascending (the
+// second stage of colsum_acc, for partials a GEMM epilogue wrote)
+void colsum_reduce(float* db, const float* partials, int chunks, int N, cudaStream_t s);
 
 // ----------------------------------------------------------- attention --
 // qkv [B*T, 3C] = [q | k | v], head h at columns h*hd..; att [B*T, C];

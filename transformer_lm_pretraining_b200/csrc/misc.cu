@@ -619,6 +619,11 @@ void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaS
   note_launch(2);
 }
 
+void colsum_reduce(float* db, const float* partials, int chunks, int N, cudaStream_t s) {
+  launch_kernel(colsum_reduce_kernel, (N + 31) / 32, 1024, 0, s, db, partials, chunks, N);
+  note_launch();
+}
+
 void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int Vp, int write_grad,
                 int* err, cudaStream_t s) {
   if (M <= 0) return;
