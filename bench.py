@@ -45,8 +45,8 @@ SPEC_BF16_DENSE = 2.25e15
 # dram__bytes_write.sum, weighted by its launches per step
 # (profiles/gemm_tc_dram_traffic_gpt2_124m_step.md).  Valid only for the GEMM
 # sources it was taken on: reported as null as soon as their hash differs.
-GEMM_TRAFFIC = {"bytes_per_launch": 1.4416e8,
-                "sources_sha256": "57fd6054277f6e84e6c918e9fac54057f2ba420f1ad420da6ad1d6cf6b09db6f"}
+GEMM_TRAFFIC = {"bytes_per_launch": 1.4588e8,
+                "sources_sha256": "c367e68adb8b746cfb8d339e920dc8f42d18a2c541030a8c7e294295defb78e7"}
 GEMM_SOURCES = ("gemm_tc.cu", "gemm_epi.cuh", "tc_util.cuh")
 
 
@@ -78,7 +78,8 @@ class ClockSampler:
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "power.limit")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
@@ -110,7 +111,8 @@ class ClockSampler:
             if len(parts) < 9:
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                lim = float(parts[9]) if len(parts) > 9 else float("nan")
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9], lim))
             except ValueError:
                 continue
         os.unlink(self.path)
@@ -120,7 +122,8 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "power_w_max": max(r[2] for r in rows), "samples": len(loaded), "reasons": reasons}
+                "power_w_max": max(r[2] for r in rows), "power_limit_w": rows[-1][4],
+                "samples": len(loaded), "reasons": reasons}
 
 
 def make_batches(wl, n_steps, seed):
