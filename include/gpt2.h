@@ -142,7 +142,10 @@ gpt2_status gpt2_evaluate(gpt2_t* h, const int32_t* tok_dev, const int32_t* tgt_
  * receives the logits each token was drawn from.  The cache and the
  * one-position buffers are device memory the library allocates and keeps
  * until gpt2_destroy; the forward record afterwards holds the prompts (no
- * gpt2_backward).  Asynchronous.  Errors: GPT2_ERR_ARG (T_prompt < 1,
+ * gpt2_backward).  With a stream set (gpt2_set_stream) and profiling off,
+ * the decode steps after the first replay one captured CUDA graph (the step
+ * reads its position from a device counter); the results are the same as
+ * with plain launches.  Asynchronous.  Errors: GPT2_ERR_ARG (T_prompt < 1,
  * T_total <= T_prompt or > Tmax, head dim above 128), GPT2_ERR_CUDA. */
 gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok_dev, int B, int T_prompt, int T_total,
                           float temperature, int top_k, uint64_t seed, float* step_logits);

@@ -12,6 +12,8 @@ sampler applied to the GPU's own logits (the decision taken in the same
 fp32 precision) at the same SplitMix64 draw, lies in the top-k set, and
 reruns are identical.
 """
+import contextlib
+
 import numpy as np
 import pytest
 
@@ -30,18 +32,25 @@ CASES = [
 ]
 
 
-def run_generate(precision, cfg, B, Tp, Ttot, temperature=0.0, top_k=0, seed=0):
+def run_generate(precision, cfg, B, Tp, Ttot, temperature=0.0, top_k=0, seed=0, stream=False):
+    """stream=True runs the model on a stream of its own, where the decode
+    steps after the first replay one captured CUDA graph; on the default
+    stream every step is plain launches."""
     params = Oracle(cfg).init(0).astype(np.float32)
     prompt, _ = iid_batch(cfg.V, B, Tp, 11)
     tok = np.zeros((B, Ttot), np.int32)
     tok[:, :Tp] = prompt
     td = torch.tensor(tok, device="cuda")
     logits = torch.zeros((Ttot - Tp, B, cfg.V), dtype=torch.float32, device="cuda")
-    m = g2.GPT2(*cfg.args, seed=0, precision=precision, B=B, T=Tp)
-    m.set_params(params)
-    m.generate(td, Tp, temperature, top_k, seed, step_logits=logits)
-    torch.cuda.synchronize()
-    m.close()
+    st = torch.cuda.Stream() if stream else None
+    with torch.cuda.stream(st) if stream else contextlib.nullcontext():
+        m = g2.GPT2(*cfg.args, seed=0, precision=precision, B=B, T=Tp)
+        if stream:
+            m.set_stream(st)
+        m.set_params(params)
+        m.generate(td, Tp, temperature, top_k, seed, step_logits=logits)
+        torch.cuda.synchronize()
+        m.close()
     return params, td.cpu().numpy(), logits.cpu().numpy()
 
 
@@ -73,7 +82,7 @@ def test_greedy_generation_fp32_matches_oracle(name, cfg, B, Tp, Ttot):
 
 @pytest.mark.parametrize("name,cfg,B,Tp,Ttot", CASES)
 def test_greedy_generation_bf16_matches_oracle(name, cfg, B, Tp, Ttot):
-    params, tok, lg = run_generate("bf16", cfg, B, Tp, Ttot)
+    params, tok, lg = run_generate("bf16", cfg, B, Tp, Ttot, stream=True)  # graph-replayed decode
     ref = oracle_step_logits(cfg, params, tok, Tp, Ttot)
     assert np.all(np.abs(lg - ref) <= 3e-2 * (1.0 + np.abs(ref))), np.abs(lg - ref).max()
     assert np.array_equal(tok[:, Tp:].T, np.argmax(lg, axis=-1))
@@ -104,3 +113,15 @@ def test_generate_rejects_bad_arguments():
         with pytest.raises(g2.GPT2Error):
             m.generate(td, tp)
     m.close()
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_graph_replayed_decode_equals_plain_launches(precision):
+    """The decode steps replayed from one captured graph (a stream of the
+    model's own) give the same tokens and logits, bit for bit, as plain
+    launches on the default stream, sampled at temperature 0.8, top-k 40."""
+    name, cfg, B, Tp, Ttot = CASES[1]
+    _, tok_a, lg_a = run_generate(precision, cfg, B, Tp, Ttot, 0.8, 40, 7, stream=False)
+    _, tok_b, lg_b = run_generate(precision, cfg, B, Tp, Ttot, 0.8, 40, 7, stream=True)
+    assert np.array_equal(tok_a, tok_b)
+    assert np.array_equal(lg_a, lg_b)

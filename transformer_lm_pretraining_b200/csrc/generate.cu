@@ -12,13 +12,19 @@ namespace {
 
 constexpr int kSampleThreads = 1024;
 
+// The position a kernel works at: p, plus *p_dev when p_dev is given (the
+// position counter of a decode step replayed from a CUDA graph).
+__device__ __forceinline__ int at_pos(int p, const int* p_dev) { return p_dev ? p + *p_dev : p; }
+
 // x[b] = wte[tok[b * ld_tok + p]] + wpe[p]; ids outside [0, V) read as 0 and
 // set ERR_TOKEN.
 __global__ void decode_embed_kernel(act_t* __restrict__ x, const int* __restrict__ tok, int ld_tok,
-                                    int p, const act_t* __restrict__ wte,
-                                    const act_t* __restrict__ wpe, int C, int V, int* err) {
+                                    int p0, const int* __restrict__ p_dev,
+                                    const act_t* __restrict__ wte, const act_t* __restrict__ wpe,
+                                    int C, int V, int* err) {
   pdl_start();
   const int b = blockIdx.x;
+  const int p = at_pos(p0, p_dev);
   int t = tok[(size_t)b * ld_tok + p];
   if (t < 0 || t >= V) {
     if (threadIdx.x == 0) atomicOr(err, ERR_TOKEN);
@@ -40,9 +46,10 @@ __global__ void decode_embed_kernel(act_t* __restrict__ x, const int* __restrict
 // kv rows: [b][Ttot][2C] = [k | v].
 __global__ void __launch_bounds__(128)
     decode_attention_kernel(act_t* __restrict__ att, const act_t* __restrict__ q,
-                            const act_t* __restrict__ kv, int Ttot, int n, int C, int H,
-                            float scale) {
+                            const act_t* __restrict__ kv, int Ttot, int n0,
+                            const int* __restrict__ p_dev, int C, int H, float scale) {
   pdl_start();
+  const int n = at_pos(n0, p_dev);
   extern __shared__ float sc[];  // [n] scores, then [128 / hd][hd] partial outputs
   __shared__ float red[4], qv[256];
   const int h = blockIdx.x, b = blockIdx.y, hd = C / H;
@@ -144,10 +151,12 @@ __device__ __forceinline__ int block_min_i(int v, int* red) {
 // and the run where the cumulative mass first exceeds u * total is walked.
 // logits_out (may be null) receives the row as fp32.
 __global__ void __launch_bounds__(kSampleThreads)
-    sample_kernel(int* __restrict__ tok, int ld_tok, int p_out, const act_t* __restrict__ logits,
-                  long ld_logits, int V, float temperature, int top_k, uint64_t seed,
-                  float* __restrict__ logits_out) {
+    sample_kernel(int* __restrict__ tok, int ld_tok, int p_out0, const int* __restrict__ p_dev,
+                  const act_t* __restrict__ logits, long ld_logits, int V, float temperature,
+                  int top_k, uint64_t seed, float* __restrict__ logits_out, int out_p0) {
   pdl_start();
+  const int p_out = at_pos(p_out0, p_dev);
+  if (logits_out) logits_out += (size_t)(p_out - out_p0) * gridDim.x * V;
   __shared__ float redf[kSampleThreads / 32];
   __shared__ int redi[kSampleThreads / 32];
   __shared__ float scan[kSampleThreads];
@@ -219,28 +228,53 @@ __global__ void __launch_bounds__(kSampleThreads)
   if (tid == 0) tok[(size_t)b * ld_tok + p_out] = chosen;
 }
 
+// cache[b][p] = kvnew[b] (2C values per row; cache rows [b][Ttot][2C])
+__global__ void kv_append_kernel(act_t* __restrict__ cache, const act_t* __restrict__ kvnew,
+                                 const int* __restrict__ p_dev, int p0, int Ttot, int C2) {
+  pdl_start();
+  const int b = blockIdx.x, p = at_pos(p0, p_dev);
+  for (int c = threadIdx.x; c < C2; c += blockDim.x)
+    cache[((size_t)b * Ttot + p) * C2 + c] = kvnew[(size_t)b * C2 + c];
+}
+
+__global__ void pos_advance_kernel(int* p_dev) {
+  pdl_start();
+  if (threadIdx.x == 0) *p_dev += 1;
+}
+
 }  // namespace
 
-void decode_embed(act_t* x, const int* tok, int ld_tok, int p, const act_t* wte, const act_t* wpe,
-                  int B, int C, int V, int* err, cudaStream_t s) {
-  launch_kernel(decode_embed_kernel, B, 128, 0, s, x, tok, ld_tok, p, wte, wpe, C, V, err);
+void decode_embed(act_t* x, const int* tok, int ld_tok, int p, const int* p_dev, const act_t* wte,
+                  const act_t* wpe, int B, int C, int V, int* err, cudaStream_t s) {
+  launch_kernel(decode_embed_kernel, B, 128, 0, s, x, tok, ld_tok, p, p_dev, wte, wpe, C, V, err);
   note_launch();
 }
 
-void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int n, int B, int C,
-                      int H, cudaStream_t s) {
+void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int n,
+                      const int* p_dev, int B, int C, int H, cudaStream_t s) {
   const int hd = C / H;  // <= 128 (checked by the caller)
-  const size_t smem = ((size_t)n + 128) * sizeof(float);
-  launch_kernel(decode_attention_kernel, dim3(H, B), 128, smem, s, att, q, kv, Ttot, n, C, H,
-                                                         1.0f / sqrtf((float)hd));
+  const size_t smem = ((size_t)(p_dev ? Ttot : n) + 128) * sizeof(float);
+  launch_kernel(decode_attention_kernel, dim3(H, B), 128, smem, s, att, q, kv, Ttot, n, p_dev, C, H,
+                1.0f / sqrtf((float)hd));
   note_launch();
 }
 
-void sample_tokens(int* tok, int ld_tok, int p_out, const act_t* logits, long ld_logits, int B,
-                   int V, float temperature, int top_k, uint64_t seed, float* logits_out,
-                   cudaStream_t s) {
-  launch_kernel(sample_kernel, B, kSampleThreads, 0, s, tok, ld_tok, p_out, logits, ld_logits, V, temperature,
-                                             top_k, seed, logits_out);
+void sample_tokens(int* tok, int ld_tok, int p_out, const int* p_dev, const act_t* logits,
+                   long ld_logits, int B, int V, float temperature, int top_k, uint64_t seed,
+                   float* logits_out, int out_p0, cudaStream_t s) {
+  launch_kernel(sample_kernel, B, kSampleThreads, 0, s, tok, ld_tok, p_out, p_dev, logits,
+                ld_logits, V, temperature, top_k, seed, logits_out, out_p0);
+  note_launch();
+}
+
+void kv_append(act_t* cache, const act_t* kvnew, int p, const int* p_dev, int Ttot, int B, int C,
+               cudaStream_t s) {
+  launch_kernel(kv_append_kernel, B, 128, 0, s, cache, kvnew, p_dev, p, Ttot, 2 * C);
+  note_launch();
+}
+
+void pos_advance(int* p_dev, cudaStream_t s) {
+  launch_kernel(pos_advance_kernel, 1, 32, 0, s, p_dev);
   note_launch();
 }
 

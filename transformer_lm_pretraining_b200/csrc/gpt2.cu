@@ -513,9 +513,10 @@ namespace {
 // Generation buffers: the key/value cache [L][B][Ttot][2C] and the
 // one-position activations of a decode step.
 struct GenBufs {
-  act_t *cache, *x0, *x1, *hb, *q, *att, *xm, *u, *g, *logits;
+  act_t *cache, *x0, *x1, *hb, *q, *kvnew, *att, *xm, *u, *g, *logits;
   float *mean, *rstd;
   int* prompt;
+  int* pos;  // the decode position (device counter)
 };
 
 size_t carve_gen(const Layout& y, int B, int Tp, int Ttot, void* base, GenBufs* out) {
@@ -527,6 +528,7 @@ size_t carve_gen(const Layout& y, int B, int Tp, int Ttot, void* base, GenBufs* 
   g.x1 = c.take<act_t>(B * C);
   g.hb = c.take<act_t>(B * C);
   g.q = c.take<act_t>(B * C);
+  g.kvnew = c.take<act_t>(B * 2 * C);
   g.att = c.take<act_t>(B * C);
   g.xm = c.take<act_t>(B * C);
   g.u = c.take<act_t>(B * 4 * C);
@@ -535,6 +537,7 @@ size_t carve_gen(const Layout& y, int B, int Tp, int Ttot, void* base, GenBufs* 
   g.mean = c.take<float>(B);
   g.rstd = c.take<float>(B);
   g.prompt = c.take<int>((size_t)B * Tp);
+  g.pos = c.take<int>(1);
   if (out) *out = g;
   return c.used;
 }
@@ -577,12 +580,17 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
                                      a.qkv + (size_t)l * 3 * MCp + (size_t)b * Tp * 3 * C + C,
                                      3 * C * sizeof(act_t), 2 * C * sizeof(act_t), Tp,
                                      cudaMemcpyDeviceToDevice, s));
-  const size_t Vs = (size_t)y.V;
-  sample_tokens(tok, Ttot, Tp, a.logits + (size_t)(Tp - 1) * y.Vp, (long)Tp * y.Vp, B, y.V,
-                temperature, top_k, seed, step_logits, s);
-  // decode: position p takes token p and yields token p + 1
-  for (int p = Tp; p < Ttot - 1; ++p) {
-    decode_embed(gb.x0, tok, Ttot, p, W + y.off[T_WTE], W + y.off[T_WPE], B, C, y.V, h->err, s);
+  sample_tokens(tok, Ttot, Tp, nullptr, a.logits + (size_t)(Tp - 1) * y.Vp, (long)Tp * y.Vp, B, y.V,
+                temperature, top_k, seed, step_logits, Tp, s);
+  // decode: the step at position p takes token p and yields token p + 1.
+  // It works at the device position counter gb.pos, so that the same launch
+  // sequence serves every position: the first step runs as plain launches
+  // (first use of its kernels), the rest replay it captured as a CUDA graph.
+  const int p_first = Tp;
+  GPT2_CUDA(h, cudaMemcpyAsync(gb.pos, &p_first, sizeof(int), cudaMemcpyHostToDevice, s));
+  auto step = [&]() -> gpt2_status {
+    decode_embed(gb.x0, tok, Ttot, 0, gb.pos, W + y.off[T_WTE], W + y.off[T_WPE], B, C, y.V,
+                 h->err, s);
     act_t* x = gb.x0;
     act_t* xn = gb.x1;
     for (int l = 0; l < L; ++l) {
@@ -597,15 +605,16 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
         ga.out = gb.q; ga.ldo = C;
         GPT2_TRY(run_gemm(h, ga));
       }
-      {  // [k | v] of position p straight into the cache
+      {  // [k | v] of the position, then into the cache at it
         GemmArgs ga = gemm_args(B, 2 * C, C);
         ga.A = gb.hb; ga.lda = C;
         ga.B = W + y.off[T_WQKV] + (size_t)l * 3 * C * C + (size_t)C * C; ga.ldb = C;
         ga.epi = EPI_BIAS; ga.bias = P + y.off[T_BQKV] + (size_t)l * 3 * C + C;
-        ga.out = kv + (size_t)p * 2 * C; ga.ldo = (long)Ttot * 2 * C;
+        ga.out = gb.kvnew; ga.ldo = 2 * C;
         GPT2_TRY(run_gemm(h, ga));
       }
-      decode_attention(gb.att, gb.q, kv, Ttot, p + 1, B, C, H, s);
+      kv_append(kv, gb.kvnew, 0, gb.pos, Ttot, B, C, s);
+      decode_attention(gb.att, gb.q, kv, Ttot, 1, gb.pos, B, C, H, s);  // n = position + 1
       {  // xm = x + att W_o^T + b_o
         GemmArgs ga = gemm_args(B, C, C);
         ga.A = gb.att; ga.lda = C;
@@ -638,7 +647,7 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
       std::swap(x, xn);
     }
     layernorm_fwd(gb.hb, gb.mean, gb.rstd, x, P + y.off[T_LNFG], P + y.off[T_LNFB], B, C, s);
-    {  // logits of position p
+    {  // logits of the position
       GemmArgs ga = gemm_args(B, y.Vp, C);
       ga.A = gb.hb; ga.lda = C;
       ga.B = W + y.off[T_WTE]; ga.ldb = C;
@@ -646,8 +655,41 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
       ga.out = gb.logits; ga.ldo = y.Vp;
       GPT2_TRY(run_gemm(h, ga));
     }
-    sample_tokens(tok, Ttot, p + 1, gb.logits, y.Vp, B, y.V, temperature, top_k, seed,
-                  step_logits ? step_logits + (size_t)(p + 1 - Tp) * B * Vs : nullptr, s);
+    sample_tokens(tok, Ttot, 1, gb.pos, gb.logits, y.Vp, B, y.V, temperature, top_k, seed,
+                  step_logits, Tp, s);  // token position + 1
+    pos_advance(gb.pos, s);
+    return GPT2_OK;
+  };
+  const int nsteps = Ttot - 1 - Tp;
+  if (nsteps > 0) {
+    st = step();
+    if (st) return st;
+  }
+  if (nsteps > 1) {
+    if (h->stream && !h->prof) {  // capture needs a stream of its own; profiling marks stay eager
+      GPT2_CUDA(h, cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal));
+      st = step();
+      cudaGraph_t g = nullptr;
+      const cudaError_t ec = cudaStreamEndCapture(s, &g);
+      if (st) {
+        if (g) cudaGraphDestroy(g);
+        return st;
+      }
+      if (ec != cudaSuccess) return cuda_fail(h, ec, "cudaStreamEndCapture (decode step)");
+      cudaGraphExec_t ex = nullptr;
+      const cudaError_t ei = cudaGraphInstantiate(&ex, g, 0);
+      cudaGraphDestroy(g);
+      if (ei != cudaSuccess) return cuda_fail(h, ei, "cudaGraphInstantiate (decode step)");
+      cudaError_t el = cudaSuccess;
+      for (int i = 1; i < nsteps && el == cudaSuccess; ++i) el = cudaGraphLaunch(ex, s);
+      cudaGraphExecDestroy(ex);  // freed once its launches complete
+      if (el != cudaSuccess) return cuda_fail(h, el, "cudaGraphLaunch (decode step)");
+    } else {
+      for (int i = 1; i < nsteps; ++i) {
+        st = step();
+        if (st) return st;
+      }
+    }
   }
   h->have_logits = h->have_grad_logits = false;  // the forward record now holds the prompt only
   GPT2_CUDA(h, cudaGetLastError());

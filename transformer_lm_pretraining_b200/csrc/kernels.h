@@ -149,19 +149,28 @@ void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int 
 void mean_loss(float* out, const float* losses, int M, cudaStream_t s);
 
 // ------------------------------------------------------------ generation --
+// Positions: each of these works at p, or at p + *p_dev when p_dev is given
+// (a device position counter, so that one decode step can be captured once
+// and replayed as a CUDA graph).
 // x[b] = wte[tok[b * ld_tok + p]] + wpe[p] for b < B (bad ids: ERR_TOKEN, read as 0)
-void decode_embed(act_t* x, const int* tok, int ld_tok, int p, const act_t* wte, const act_t* wpe,
-                  int B, int C, int V, int* err, cudaStream_t s);
+void decode_embed(act_t* x, const int* tok, int ld_tok, int p, const int* p_dev, const act_t* wte,
+                  const act_t* wpe, int B, int C, int V, int* err, cudaStream_t s);
 // att[b] = causal attention of the single query q[b] over the first n
 // cached positions kv[b][0..n) ([b][Ttot][2C] rows of [k | v]); C / H <= 128
-void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int n, int B, int C,
-                      int H, cudaStream_t s);
+void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int n,
+                      const int* p_dev, int B, int C, int H, cudaStream_t s);
 // tok[b * ld_tok + p_out] = the next token drawn from the V logits of row
 // b (greedy at temperature 0; else top-k tempered softmax at the SplitMix64
-// uniform of (seed, p_out * 65536 + b)); logits_out (may be null): [B][V] fp32
-void sample_tokens(int* tok, int ld_tok, int p_out, const act_t* logits, long ld_logits, int B,
-                   int V, float temperature, int top_k, uint64_t seed, float* logits_out,
-                   cudaStream_t s);
+// uniform of (seed, p_out * 65536 + b)); logits_out (may be null): rows
+// [p_out - out_p0][B][V] fp32
+void sample_tokens(int* tok, int ld_tok, int p_out, const int* p_dev, const act_t* logits,
+                   long ld_logits, int B, int V, float temperature, int top_k, uint64_t seed,
+                   float* logits_out, int out_p0, cudaStream_t s);
+// cache[b][p] = kvnew[b] (rows of 2C: [k | v]; cache [b][Ttot][2C])
+void kv_append(act_t* cache, const act_t* kvnew, int p, const int* p_dev, int Ttot, int B, int C,
+               cudaStream_t s);
+// *p_dev += 1
+void pos_advance(int* p_dev, cudaStream_t s);
 
 // g = GELU_tanh(u) elementwise (n elements, activation dtype); the same
 // function the fc GEMM's epilogue applies to the stored u.
