@@ -101,6 +101,39 @@ def test_gemm_forward(M, N, K, epi, cta_pairs):
     assert_bf16_close(got, ref)
 
 
+@pytest.mark.parametrize("M,N,K", [(16, 768, 768), (16, 3072, 768), (5, 768, 3072), (128, 200, 520),
+                                   (16, 2304, 72)])
+@pytest.mark.parametrize("epi", ["store", "bias", "bias_gelu", "bias_resid"])
+def test_gemm_small_m_split(M, N, K, epi):
+    """A single 128-row tile (one position per sequence, as in generation)
+    with a split-K workspace: K is split across the SMs, the fp32 partials
+    summed in split order and the bf16 epilogue applied after (alpha 0.5)."""
+    rng = np.random.default_rng(M * 11 + N + 3 * K)
+    x = bf16(rng.standard_normal((M, K)))
+    W = bf16(rng.standard_normal((N, K)) * 0.05)
+    b = rng.standard_normal(N).astype(np.float32) * 0.1
+    r = bf16(rng.standard_normal((M, N)))
+    ref = 0.5 * ref_linear(x, W)
+    if epi != "store":
+        ref = ref + b.astype(np.float64)
+    out = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    aux = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(8 * M * N, dtype=torch.float32, device="cuda")
+    g2.gpt2k_gemm(epi, M, N, K, dev(x), K, 0, dev(W), K, 0, 0.5, out=out, ldo=N,
+                  bias=torch.tensor(b, device="cuda") if epi != "store" else None,
+                  resid=dev(r) if epi == "bias_resid" else None, ldr=N,
+                  aux=aux if epi == "bias_gelu" else None, ldaux=N, split_ws=ws)
+    torch.cuda.synchronize()
+    assert g2.gpt2k_take_error() == 0
+    got = host(out)
+    if epi == "bias_resid":
+        ref = ref + r
+    if epi == "bias_gelu":
+        assert_bf16_close(host(aux), ref)
+        ref = ORC.gelu_tanh(bf16(host(aux)))
+    assert_bf16_close(got, ref)
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 200, 136), (1000, 768, 3072), (256, 3072, 768),
                                    (129, 512, 200)])
 @pytest.mark.parametrize("epi", ["store", "dgelu"])

@@ -701,11 +701,26 @@ static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUte
   GPT2_TC(1, 1, EPI_F32_ACC)
   GPT2_TC(1, 1, EPI_F32_STORE)
   GPT2_TC(1, 0, EPI_STORE)
+  GPT2_TC(0, 0, EPI_F32_STORE)  // split small-M products
 #undef GPT2_TC
   return cudaErrorInvalidValue;
 }
 
 }  // namespace tc
+
+// The epilogue of a split small-M product: element (m, n) gets the sum of
+// its split partials ws[s][m][n], s ascending, then the product's epilogue.
+template <int EPI>
+__global__ void splitk_epilogue_kernel(EpiParams e, const float* __restrict__ ws, int splits) {
+  pdl_start();
+  const size_t total = (size_t)e.M * e.N;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float acc = ws[i];
+    for (int k = 1; k < splits; ++k) acc += ws[(size_t)k * total + i];
+    epi_scalar<EPI>(e, (int)(i / e.N), (int)(i % e.N), acc);
+  }
+}
 
 __global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, int splits, int M,
                                      int N) {
@@ -808,6 +823,17 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
       }
     }
   }
+  // products of a single 128-row tile with a bf16 epilogue (one position
+  // per sequence in generation): a few tiles would leave most SMs idle, so K
+  // is split until the units fill the machine; the fp32 partials are summed
+  // in split order and the epilogue applied by splitk_epilogue_kernel
+  const bool small_m = !f32_out && a.M <= BM && a.epi != EPI_DGELU && !a.colsum &&
+                       a.max_splits > 1 && a.split_ws && aligned16(a.split_ws) && a.N % 4 == 0;
+  if (small_m) {
+    int sp = min(min(slots / tiles, a.max_splits), kb_total);
+    while (sp > 1 && (size_t)sp * a.M * a.N > a.split_ws_floats) --sp;
+    splits = sp > 1 ? sp : 1;
+  }
   int kb_per_split = (kb_total + splits - 1) / splits;
   splits = (kb_total + kb_per_split - 1) / kb_per_split;  // no empty split
   const bool in_place = splits == 2 && a.acc_zero;  // both halves reduce-add into out32
@@ -839,7 +865,22 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   else
     e = dispatch<128, 1>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
   if (e != cudaSuccess) return e;
-  if (splits > 1 && !in_place) {
+  if (splits > 1 && small_m) {
+    const size_t total = (size_t)a.M * a.N;
+    int blocks = (int)((total + 255) / 256);
+    if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
+    EpiParams ep1 = ep;
+    ep1.alpha = 1.f;  // the partials are already scaled
+    switch (a.epi) {
+      case EPI_STORE: launch_kernel(splitk_epilogue_kernel<EPI_STORE>, blocks, 256, 0, s, ep1, a.split_ws, splits); break;
+      case EPI_BIAS: launch_kernel(splitk_epilogue_kernel<EPI_BIAS>, blocks, 256, 0, s, ep1, a.split_ws, splits); break;
+      case EPI_BIAS_GELU: launch_kernel(splitk_epilogue_kernel<EPI_BIAS_GELU>, blocks, 256, 0, s, ep1, a.split_ws, splits); break;
+      case EPI_BIAS_RESID: launch_kernel(splitk_epilogue_kernel<EPI_BIAS_RESID>, blocks, 256, 0, s, ep1, a.split_ws, splits); break;
+      default: return cudaErrorInvalidValue;
+    }
+    note_launch();
+    e = cudaGetLastError();
+  } else if (splits > 1 && !in_place) {
     const size_t total = (size_t)a.M * a.N;
     int blocks = (int)((total / 4 + 255) / 256);
     if (blocks > 8 * num_sms()) blocks = 8 * num_sms();

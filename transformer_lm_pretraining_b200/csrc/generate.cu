@@ -40,18 +40,20 @@ __global__ void decode_embed_kernel(act_t* __restrict__ x, const int* __restrict
   }
 }
 
-// One block per (head, sequence): the query q[b, head] against the n cached
-// keys of that sequence: scores in shared memory, softmax in fp32, then the
-// value average (threads split the keys in two halves per output dimension).
+// One block of kDecodeThreads per (head, sequence): the query q[b, head]
+// against the n cached keys of that sequence: scores in shared memory,
+// softmax in fp32, then the value average (the threads split the keys into
+// kDecodeThreads / hd parts per output dimension, added in part order).
 // kv rows: [b][Ttot][2C] = [k | v].
-__global__ void __launch_bounds__(128)
+constexpr int kDecodeThreads = 256;
+__global__ void __launch_bounds__(kDecodeThreads)
     decode_attention_kernel(act_t* __restrict__ att, const act_t* __restrict__ q,
                             const act_t* __restrict__ kv, int Ttot, int n0,
                             const int* __restrict__ p_dev, int C, int H, float scale) {
   pdl_start();
   const int n = at_pos(n0, p_dev);
   extern __shared__ float sc[];  // [n] scores, then [128 / hd][hd] partial outputs
-  __shared__ float red[4], qv[256];
+  __shared__ float red[kDecodeThreads / 32], qv[256];
   const int h = blockIdx.x, b = blockIdx.y, hd = C / H;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   for (int d = tid; d < hd; d += blockDim.x) qv[d] = to_f(q[(size_t)b * C + h * hd + d]);
@@ -74,7 +76,9 @@ __global__ void __launch_bounds__(128)
   mx = warp_max(mx);
   if (lane == 0) red[w] = mx;
   __syncthreads();
-  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  mx = red[0];
+#pragma unroll
+  for (int i = 1; i < kDecodeThreads / 32; ++i) mx = fmaxf(mx, red[i]);
   __syncthreads();
   float sum = 0.f;
   for (int k = tid; k < n; k += blockDim.x) {
@@ -85,8 +89,10 @@ __global__ void __launch_bounds__(128)
   sum = warp_sum(sum);
   if (lane == 0) red[w] = sum;
   __syncthreads();
-  sum = (red[0] + red[1]) + (red[2] + red[3]);
-  // output dimension d = tid % hd, key half = tid / hd (hd <= 64 uses both halves)
+  sum = red[0];
+#pragma unroll
+  for (int i = 1; i < kDecodeThreads / 32; ++i) sum += red[i];
+  // output dimension d = tid % hd, key part = tid / hd
   float* part = sc + n;
   const int d = tid % hd, half = tid / hd, halves = blockDim.x / hd;
   if (half < halves) {
@@ -142,58 +148,86 @@ __device__ __forceinline__ int block_min_i(int v, int* red) {
 }
 
 // One block per sequence b: the next token from the row of V logits at
-// logits + b * ld_logits, written to tok[b * ld_tok + p_out].  Temperature
-// 0: the argmax (lowest index among equal maxima).  Otherwise the softmax of
-// z / temperature over the top_k largest logits (threshold found by
-// bisection over order-preserving keys; ties kept), inverted at the uniform
-// u = SplitMix64(seed, p_out * 65536 + b) (top 53 bits): each thread owns a
-// contiguous run of columns, the runs' sums are scanned in a fixed order,
-// and the run where the cumulative mass first exceeds u * total is walked.
-// logits_out (may be null) receives the row as fp32.
-__global__ void __launch_bounds__(kSampleThreads)
+// logits + b * ld_logits, written to tok[b * ld_tok + p_out].  The row is
+// staged in shared memory (coalesced); thread t owns the contiguous run of
+// columns [t c, t c + c), c = ceil(V / kSampleThreads).  Temperature 0: the
+// argmax (lowest index among equal maxima).  Otherwise the softmax of z /
+// temperature over the top_k largest logits (ties at the k-th value kept):
+// the k-th largest order-preserving key is found by a radix select, a byte at
+// a time from the top (integer counts in shared memory), then the runs' sums
+// of exp((z - max) / T) are scanned in thread order and the run where the
+// cumulative mass first exceeds u * total is walked, u = SplitMix64(seed,
+// p_out * 65536 + b) (top 53 bits).  logits_out (may be null) receives the
+// row as fp32.  Dynamic shared memory: V activations.
+__global__ void __launch_bounds__(kSampleThreads, 1)
     sample_kernel(int* __restrict__ tok, int ld_tok, int p_out0, const int* __restrict__ p_dev,
                   const act_t* __restrict__ logits, long ld_logits, int V, float temperature,
                   int top_k, uint64_t seed, float* __restrict__ logits_out, int out_p0) {
   pdl_start();
-  const int p_out = at_pos(p_out0, p_dev);
-  if (logits_out) logits_out += (size_t)(p_out - out_p0) * gridDim.x * V;
+  extern __shared__ __align__(16) uint8_t sample_smem[];
+  act_t* zs = reinterpret_cast<act_t*>(sample_smem);
   __shared__ float redf[kSampleThreads / 32];
   __shared__ int redi[kSampleThreads / 32];
   __shared__ float scan[kSampleThreads];
+  __shared__ int hist[256];
+  __shared__ uint32_t sel[2];  // the selected key prefix and the count still to take
+  const int p_out = at_pos(p_out0, p_dev);
+  if (logits_out) logits_out += (size_t)(p_out - out_p0) * gridDim.x * V;
   const int b = blockIdx.x, tid = threadIdx.x;
   const act_t* z = logits + (size_t)b * ld_logits;
-  if (logits_out)
-    for (int v = tid; v < V; v += kSampleThreads) logits_out[(size_t)b * V + v] = to_f(z[v]);
   float mx = -INFINITY;
-  for (int v = tid; v < V; v += kSampleThreads) mx = fmaxf(mx, to_f(z[v]));
-  mx = block_max_f(mx, redf);
+  for (int v = tid; v < V; v += kSampleThreads) {
+    const act_t x = z[v];
+    zs[v] = x;
+    mx = fmaxf(mx, to_f(x));
+    if (logits_out) logits_out[(size_t)b * V + v] = to_f(x);
+  }
+  mx = block_max_f(mx, redf);  // (its barrier also publishes zs)
+  const int chunk = (V + kSampleThreads - 1) / kSampleThreads;
+  const int v0 = min(V, tid * chunk), v1 = min(V, v0 + chunk);
   int chosen;
   if (temperature <= 0.f) {
     int first = INT_MAX;
-    for (int v = tid; v < V; v += kSampleThreads)
-      if (to_f(z[v]) == mx) first = min(first, v);
+    for (int v = v1 - 1; v >= v0; --v)
+      if (to_f(zs[v]) == mx) first = v;
     chosen = block_min_i(first, redi);
   } else {
-    // keep z >= the k-th largest value: the largest key t with count(key >= t) >= k
+    // keep z >= the k-th largest value: radix select of the k-th largest key
     uint32_t thr = 0;
     if (top_k > 0 && top_k < V) {
-      uint32_t lo = 0, hi = 0xFFFFFFFFu;  // count(key >= lo) >= k always
-      while (lo < hi) {
-        const uint32_t mid = lo + (uint32_t)(((uint64_t)hi - lo + 1) >> 1);
-        int cnt = 0;
-        for (int v = tid; v < V; v += kSampleThreads) cnt += ord_key(to_f(z[v])) >= mid;
-        const float tot = block_sum_f((float)cnt, redf);
-        if (tot >= (float)top_k) lo = mid;
-        else hi = mid - 1;
+      if (tid == 0) {
+        sel[0] = 0u;
+        sel[1] = (uint32_t)top_k;
       }
-      thr = lo;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        if (tid < 256) hist[tid] = 0;
+        __syncthreads();
+        const uint32_t prefix = sel[0];
+        const uint32_t hi_mask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+        for (int v = v0; v < v1; ++v) {
+          const uint32_t key = ord_key(to_f(zs[v]));
+          if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (tid == 0) {  // the bin holding the k-th largest, from the top
+          uint32_t need = sel[1];
+          int bin = 255;
+          for (; bin > 0; --bin) {
+            const uint32_t c = (uint32_t)hist[bin];
+            if (c >= need) break;
+            need -= c;
+          }
+          sel[0] = prefix | ((uint32_t)bin << shift);
+          sel[1] = need;
+        }
+        __syncthreads();
+      }
+      thr = sel[0];
     }
     const float inv_t = 1.0f / temperature;
-    const int chunk = (V + kSampleThreads - 1) / kSampleThreads;
-    const int v0 = min(V, tid * chunk), v1 = min(V, v0 + chunk);
     float s = 0.f;
     for (int v = v0; v < v1; ++v) {
-      const float zv = to_f(z[v]);
+      const float zv = to_f(zs[v]);
       if (ord_key(zv) >= thr) s += __expf((zv - mx) * inv_t);
     }
     // exclusive scan of the runs' sums in thread order
@@ -216,7 +250,7 @@ __global__ void __launch_bounds__(kSampleThreads)
     int found = INT_MAX, last = -1;
     float cum = scan[tid];
     for (int v = v0; v < v1; ++v) {
-      const float zv = to_f(z[v]);
+      const float zv = to_f(zs[v]);
       if (ord_key(zv) < thr) continue;
       cum += __expf((zv - mx) * inv_t);
       last = v;
@@ -253,8 +287,9 @@ void decode_embed(act_t* x, const int* tok, int ld_tok, int p, const int* p_dev,
 void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int n,
                       const int* p_dev, int B, int C, int H, cudaStream_t s) {
   const int hd = C / H;  // <= 128 (checked by the caller)
-  const size_t smem = ((size_t)(p_dev ? Ttot : n) + 128) * sizeof(float);
-  launch_kernel(decode_attention_kernel, dim3(H, B), 128, smem, s, att, q, kv, Ttot, n, p_dev, C, H,
+  const size_t smem = ((size_t)(p_dev ? Ttot : n) + kDecodeThreads) * sizeof(float);
+  launch_kernel(decode_attention_kernel, dim3(H, B), kDecodeThreads, smem, s, att, q, kv, Ttot, n,
+                p_dev, C, H,
                 1.0f / sqrtf((float)hd));
   note_launch();
 }
@@ -262,7 +297,13 @@ void decode_attention(act_t* att, const act_t* q, const act_t* kv, int Ttot, int
 void sample_tokens(int* tok, int ld_tok, int p_out, const int* p_dev, const act_t* logits,
                    long ld_logits, int B, int V, float temperature, int top_k, uint64_t seed,
                    float* logits_out, int out_p0, cudaStream_t s) {
-  launch_kernel(sample_kernel, B, kSampleThreads, 0, s, tok, ld_tok, p_out, p_dev, logits,
+  const size_t smem = (size_t)V * sizeof(act_t);
+  static size_t smem_set = 0;
+  if (smem > 48 * 1024 && smem > smem_set) {
+    cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    smem_set = smem;
+  }
+  launch_kernel(sample_kernel, B, kSampleThreads, smem, s, tok, ld_tok, p_out, p_dev, logits,
                 ld_logits, V, temperature, top_k, seed, logits_out, out_p0);
   note_launch();
 }

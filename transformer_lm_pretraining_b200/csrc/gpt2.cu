@@ -512,9 +512,11 @@ namespace {
 
 // Generation buffers: the key/value cache [L][B][Ttot][2C] and the
 // one-position activations of a decode step.
+constexpr int kGenSplits = 16;  // K splits of a one-position product at most
 struct GenBufs {
   act_t *cache, *x0, *x1, *hb, *q, *kvnew, *att, *xm, *u, *g, *logits;
   float *mean, *rstd;
+  float* splitws;  // split-K partials of the one-position products
   int* prompt;
   int* pos;  // the decode position (device counter)
 };
@@ -536,6 +538,7 @@ size_t carve_gen(const Layout& y, int B, int Tp, int Ttot, void* base, GenBufs* 
   g.logits = c.take<act_t>((size_t)B * y.Vp);
   g.mean = c.take<float>(B);
   g.rstd = c.take<float>(B);
+  g.splitws = c.take<float>((size_t)kGenSplits * B * 4 * C);
   g.prompt = c.take<int>((size_t)B * Tp);
   g.pos = c.take<int>(1);
   if (out) *out = g;
@@ -588,6 +591,12 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
   // (first use of its kernels), the rest replay it captured as a CUDA graph.
   const int p_first = Tp;
   GPT2_CUDA(h, cudaMemcpyAsync(gb.pos, &p_first, sizeof(int), cudaMemcpyHostToDevice, s));
+  // the one-position products split K across the SMs (see gemm)
+  auto split = [&](GemmArgs& ga) {
+    ga.split_ws = gb.splitws;
+    ga.split_ws_floats = (size_t)kGenSplits * B * 4 * C;
+    ga.max_splits = kGenSplits;
+  };
   auto step = [&]() -> gpt2_status {
     decode_embed(gb.x0, tok, Ttot, 0, gb.pos, W + y.off[T_WTE], W + y.off[T_WPE], B, C, y.V,
                  h->err, s);
@@ -603,6 +612,7 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
         ga.B = W + y.off[T_WQKV] + (size_t)l * 3 * C * C; ga.ldb = C;
         ga.epi = EPI_BIAS; ga.bias = P + y.off[T_BQKV] + (size_t)l * 3 * C;
         ga.out = gb.q; ga.ldo = C;
+        split(ga);
         GPT2_TRY(run_gemm(h, ga));
       }
       {  // [k | v] of the position, then into the cache at it
@@ -611,6 +621,7 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
         ga.B = W + y.off[T_WQKV] + (size_t)l * 3 * C * C + (size_t)C * C; ga.ldb = C;
         ga.epi = EPI_BIAS; ga.bias = P + y.off[T_BQKV] + (size_t)l * 3 * C + C;
         ga.out = gb.kvnew; ga.ldo = 2 * C;
+        split(ga);
         GPT2_TRY(run_gemm(h, ga));
       }
       kv_append(kv, gb.kvnew, 0, gb.pos, Ttot, B, C, s);
@@ -622,6 +633,7 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
         ga.epi = EPI_BIAS_RESID; ga.bias = P + y.off[T_BO] + (size_t)l * C;
         ga.resid = x; ga.ldr = C;
         ga.out = gb.xm; ga.ldo = C;
+        split(ga);
         GPT2_TRY(run_gemm(h, ga));
       }
       layernorm_fwd(gb.hb, gb.mean, gb.rstd, gb.xm, P + y.off[T_LN2G] + (size_t)l * C,
@@ -633,6 +645,7 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
         ga.epi = EPI_BIAS_GELU; ga.bias = P + y.off[T_BFC] + (size_t)l * 4 * C;
         ga.aux = gb.u; ga.ldaux = 4 * C;
         ga.out = gb.g; ga.ldo = 4 * C;
+        split(ga);
         GPT2_TRY(run_gemm(h, ga));
       }
       {  // x_next = xm + g W_p^T + b_p
@@ -642,6 +655,7 @@ gpt2_status gpt2_generate(gpt2_t* h, int32_t* tok, int B, int Tp, int Ttot, floa
         ga.epi = EPI_BIAS_RESID; ga.bias = P + y.off[T_BP] + (size_t)l * C;
         ga.resid = gb.xm; ga.ldr = C;
         ga.out = xn; ga.ldo = C;
+        split(ga);
         GPT2_TRY(run_gemm(h, ga));
       }
       std::swap(x, xn);
