@@ -3,11 +3,12 @@
 // Persistent: one CTA per SM walks a static list of work items, each a pair
 // of adjacent 128-row query tiles (A = 2p, B = 2p + 1) of one (batch, head).
 // Items are ordered heaviest first and dealt to the CTAs in a snake order,
-// which balances the causal work across SMs.  10 warps:
+// which balances the causal work across SMs.  11 warps:
 //   warp 0     TMA: the item's two Q tiles, then its K/V tiles of 128 keys
 //              into a 4-stage ring (128-byte swizzle, zero fill past the
 //              sequence), running ahead into the next item;
-//   warp 1     TMEM owner and MMA issuer: S_t = Q_t K_j^T (M=128, N=128,
+//   warps 1, 10  MMA issuers of tiles A and B (warp 1 also owns TMEM):
+//              S_t = Q_t K_j^T (M=128, N=128,
 //              K=64) into one TMEM buffer per tile t, and O_t += P_t V_j
 //              (M=128, N=64, K=128) with P_t read from TMEM as the A operand
 //              and V read MN-major from its shared-memory tile; O_t
@@ -24,11 +25,18 @@
 //              TMEM and the running sum are rescaled first.  No thread waits
 //              for another thread's row.
 // T x T is never materialised.  The output row is normalised by the
-// running sum; the natural-log log-sum-exp of each row is stored for the
-// backward pass.  Every wait is bounded (error word ERR_TIMEOUT).
+// running sum and written into the softmax warp's own 32-row shared-memory
+// box, which one TMA store per warp sends out (measured: 70.7 -> 62.6 us at
+// B16 x T1024 x H12 against per-thread 16-byte stores of each row, which left
+// every lane writing to a different row); the natural-log log-sum-exp of each
+// row is stored for the backward pass.  Every wait is bounded (error word
+// ERR_TIMEOUT).
 //
 // TMEM columns: [0, 256) S_A | S_B (fp32), [256, 384) O_A | O_B (fp32),
 // [384, 512) P_A | P_B (128 keys as 64 columns of bf16 pairs).
+// Softmax threads per row: one.  Two (the row max and sum exchanged through
+// shared memory) measured 78.5 vs 70.5 us, and a split of each row into key
+// halves with their own accumulators 90.3 us.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -49,17 +57,7 @@ using attn::kBox;
 using attn::kTile;
 
 constexpr int kKVStages = 4;
-// FWD_SPLIT softmax threads per query row (each owning 128 / FWD_SPLIT of a
-// key tile's columns; with more than one, the row max and the row sum meet
-// in shared memory behind bounded mbarrier waits).  Measured at B16 x T1024
-// x H12: 70.5 us with 1, 78.5 us with 2 (the exchange per key tile costs
-// more than the shorter rows save).
-#ifndef FWD_SPLIT
-#define FWD_SPLIT 1
-#endif
-constexpr int kFwdSplit = FWD_SPLIT;
-constexpr int kRowThreads = 128 * kFwdSplit;  // softmax threads per query tile
-constexpr int kColsF = kTile / kFwdSplit;      // key columns per softmax thread
+constexpr int kRowThreads = 128;  // softmax threads per query tile (one per row)
 constexpr int kThreadsAttn = 64 + 2 * kRowThreads + 32;  // + the MMA warp of tile B
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 2 * kTile;         // O_t at kOCol + t * kHD
@@ -68,9 +66,11 @@ constexpr float kRescaleLog2 = 8.0f;  // raise the reference max past this margi
 constexpr int kAux = 1024;  // barriers
 constexpr uint32_t kNegInf = 0xff800000u;
 
+constexpr int kOutBox = 4096;  // one softmax warp's output rows: 32 x 64 bf16, 128-byte swizzle
+
 constexpr size_t attn_smem_bytes() {
-  // Q (two tiles), K ring, V ring, aux
-  return 1024 + 2 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + kAux;
+  // Q (two tiles), K ring, V ring, the eight softmax warps' output boxes, aux
+  return 1024 + 2 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + 8 * (size_t)kOutBox + kAux;
 }
 
 // Work item k of this CTA (snake order over the heaviest-first item list);
@@ -95,8 +95,9 @@ __device__ __forceinline__ bool fwd_item(int k, int B, int H, int nq, FwdItem& i
 }
 
 __global__ void __launch_bounds__(kThreadsAttn, 1)
-    flash_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, __nv_bfloat16* __restrict__ att,
-                        float* __restrict__ lse, int B, int T, int C, int H, float sl2, int* err) {
+    flash_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
+                        const __grid_constant__ CUtensorMap tmOut, float* __restrict__ lse, int B,
+                        int T, int C, int H, float sl2, int* err) {
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -104,7 +105,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   uint8_t* sQ = smem;                           // [2 tiles][kBox]
   uint8_t* sK = sQ + 2 * kBox;                  // [kKVStages][kBox]
   uint8_t* sV = sK + kKVStages * kBox;          // [kKVStages][kBox]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kKVStages * kBox);
+  uint8_t* sOut = sV + kKVStages * kBox;        // [2 tiles][4 lane quarters][kOutBox]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 8 * kOutBox);
   const uint32_t q_full = smem_u32(bars + 0);
   const uint32_t q_empty = smem_u32(bars + 1);
   const uint32_t kv_full0 = smem_u32(bars + 2);                  // [kKVStages]
@@ -114,9 +116,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   const uint32_t p_full0 = s_full0 + 32;                         // [2 tiles]
   const uint32_t o_full0 = s_full0 + 48;                         // [2 tiles]
   const uint32_t drain0 = s_full0 + 64;                          // [2 tiles] abort path only
-  const uint32_t xbar0 = s_full0 + 80;   // [2 tiles][2]: row-max exchange (FWD_SPLIT > 1)
-  const uint32_t xlbar0 = s_full0 + 112; // [2 tiles]: row-sum exchange (FWD_SPLIT > 1)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 16);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int nq = (T + kTile - 1) / kTile;
@@ -135,9 +135,6 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       mbar_init(p_full0 + 8 * t, kRowThreads);
       mbar_init(o_full0 + 8 * t, 1);
       mbar_init(drain0 + 8 * t, 1);
-      mbar_init(xbar0 + 16 * t, kRowThreads);
-      mbar_init(xbar0 + 16 * t + 8, kRowThreads);
-      mbar_init(xlbar0 + 8 * t, kRowThreads);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -266,16 +263,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else {
     // -------------------------------------------------------- softmax --
-    const int t = (warp - 2) / (4 * kFwdSplit);        // query tile of the item: 0 = A, 1 = B
-    const int part = ((warp - 2) % (4 * kFwdSplit)) >> 2;  // this thread's slot of its row
+    const int t = (warp - 2) >> 2;  // query tile of the item: 0 = A, 1 = B
     const int qw = warp & 3;        // TMEM lane quarter
     const int r = qw * 32 + lane;   // row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    const uint32_t s_col = lane_base + (uint32_t)(t * kTile + kColsF * part);
-    const uint32_t o_col = lane_base + kOCol + (uint32_t)(t * kHD + (kHD / kFwdSplit) * part);
-    const uint32_t p_col = lane_base + kPCol + (uint32_t)(t * kHD + (kColsF / 2) * part);
-    __shared__ float xch[2][2][kFwdSplit][kTile];  // [tile][step parity][part][row]
-    __shared__ float xch_l[2][kFwdSplit][kTile];   // [tile][part][row]
+    const uint32_t s_col = lane_base + (uint32_t)(t * kTile);
+    const uint32_t o_col = lane_base + kOCol + (uint32_t)(t * kHD);
+    const uint32_t p_col = lane_base + kPCol + (uint32_t)(t * kHD);
+    uint8_t* obox = sOut + (t * 4 + qw) * kOutBox;  // this warp's 32 output rows
+    if (warp == 2 && lane == 0)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmOut)) : "memory");
     uint32_t cs = 0, co = 0;  // S tiles read / PV products waited for by this tile's threads
     bool ok = true;
     // wait for the next PV product of this tile (every completion is
@@ -285,56 +282,43 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       ++co;
       return r2;
     };
-    uint32_t n_items = 0;  // items this tile has finished (row-sum exchanges)
     FwdItem it;
     for (int k = 0; ok && fwd_item(k, B, H, nq, it); ++k) {
       const int nk = t ? it.nkv_b : it.nkv_a;
       if (nk == 0) continue;  // the item has no tile B
       const int qt = t ? it.qb : it.qa;
       const int qi = qt * kTile + r;  // query index in the sequence
-      float m = -INFINITY, l = 0.f;  // reference max (log2 units) and this thread's sum against it
+      float m = -INFINITY, l = 0.f;  // reference max (log2 units) and the sum against it
       for (int j = 0; j < nk && ok; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * t, cs & 1u, abort_flag, err));
         if (!ok) break;
         ++cs;
         tc_fence_after();
-        // this thread's part of the row of S in one round trip; the buffer
-        // goes straight back
-        uint32_t sr[kColsF];
+        // the whole row of S in one round trip; the buffer goes straight back
+        uint32_t sr[kTile];
 #pragma unroll
-        for (int c = 0; c < kColsF; c += 32) tc_ld32(s_col + c, sr + c);
+        for (int c = 0; c < kTile; c += 32) tc_ld32(s_col + c, sr + c);
         tc_wait_ld();
         tc_fence_before();
         mbar_arrive(s_empty0 + 8 * t);  // S_t is read: the next S_t may be computed
         if (j == nk - 1) {  // the diagonal tile: keys after the query are masked
 #pragma unroll
-          for (int c = 0; c < kColsF; ++c)
-            if (kColsF * part + c > r) sr[c] = kNegInf;
+          for (int c = 0; c < kTile; ++c)
+            if (c > r) sr[c] = kNegInf;
         }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < kColsF; c += 2)
+        for (int c = 0; c < kTile; c += 2)
           mx4[(c >> 1) & 3] = attn::fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]),
                                           __uint_as_float(sr[c + 1]));
-        float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        if (kFwdSplit > 1) {  // the row's max over its parts (bounded barrier wait)
-          const uint32_t sb = (cs - 1) & 1u;  // the S tiles read so far, this one included
-          xch[t][sb][part][r] = mt;
-          const uint32_t xb = xbar0 + 16 * t + 8 * sb;
-          mbar_arrive(xb);
-          ok = __all_sync(0xffffffffu, mbar_wait(xb, ((cs - 1) >> 1) & 1u, abort_flag, err));
-          if (!ok) break;
-#pragma unroll
-          for (int q = 0; q < kFwdSplit; ++q) mt = fmaxf(mt, xch[t][sb][q][r]);
-        }
-        mt *= sl2;
+        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
         const bool raise = mt > m + kRescaleLog2;  // always on the first key tile
         const float mn = raise ? mt : m;
         // P in registers (bf16 pairs) and its row sum
-        uint32_t pk[kColsF / 2];
+        uint32_t pk[kTile / 2];
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kColsF / 2; ++c) {
+        for (int c = 0; c < kTile / 2; ++c) {
           const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), sl2, -mn));
           const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -mn));
           sum4[(2 * c) & 3] += p0;
@@ -346,11 +330,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           ok = wait_pv();
           if (!ok) break;
           tc_fence_after();
-          if (raise) {  // rescale this thread's part of the row of O and the sum
+          if (raise) {  // rescale the row of O and the sum to the new reference
             const float f = fast_exp2(m - mn);
             l *= f;
 #pragma unroll
-            for (int hf = 0; hf < kHD / kFwdSplit; hf += 32) {
+            for (int hf = 0; hf < kHD; hf += 32) {
               uint32_t o[32];
               tc_ld32(o_col + hf, o);
               tc_wait_ld();
@@ -361,48 +345,47 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           }
         }
         m = mn;
-#pragma unroll
-        for (int c = 0; c < kColsF / 2; c += 32) attn::tc_st32(p_col + c, pk + c);
+        attn::tc_st32(p_col, pk);
+        attn::tc_st32(p_col + 32, pk + 32);
         attn::tc_wait_st();
         tc_fence_before();
         mbar_arrive(p_full0 + 8 * t);  // P_t (and a rescaled O_t) may be consumed
         l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       }
       if (!ok) break;
-      if (kFwdSplit > 1) {  // the row's sum over its parts, in part order
-        xch_l[t][part][r] = l;
-        mbar_arrive(xlbar0 + 8 * t);
-        ok = __all_sync(0xffffffffu, mbar_wait(xlbar0 + 8 * t, n_items & 1u, abort_flag, err));
-        ++n_items;
-        if (!ok) break;
-        l = 0.f;
-#pragma unroll
-        for (int q = 0; q < kFwdSplit; ++q) l += xch_l[t][q][r];
-      }
-      // the item's last product, then this thread's part of the normalised row
+      // the item's last product, then the normalised row into this warp's
+      // box and out by one TMA store per warp (rows past T are clipped by
+      // the tensor map)
       ok = wait_pv();
       if (!ok) break;
       tc_fence_after();
-      constexpr int kOut = kHD / kFwdSplit;
-      uint32_t ra[kOut];
+      uint32_t ra[kHD];
 #pragma unroll
-      for (int c = 0; c < kOut; c += 32) tc_ld32(o_col + c, ra + c);
+      for (int c = 0; c < kHD; c += 32) tc_ld32(o_col + c, ra + c);
       tc_wait_ld();
       tc_fence_before();  // O is read before the next item's first product overwrites it
-      if (qi < T) {
-        const float inv = 1.f / l;
-        __nv_bfloat16* dst =
-            att + ((size_t)it.b * T + qi) * C + (size_t)it.h * kHD + (size_t)kOut * part;
+      const float inv = 1.f / l;
+      if (lane == 0) bulk_wait_read<0>();  // the box's previous store has read it
+      __syncwarp();
 #pragma unroll
-        for (int i = 0; i < kOut; i += 8) {
-          float v[8];
+      for (int i = 0; i < kHD / 8; ++i) {
+        uint4 w;
+        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) v[q] = __uint_as_float(ra[i + q]) * inv;
-          store8(dst + i, v);
-        }
-        if (part == 0) lse[((size_t)it.b * H + it.h) * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
+        for (int q = 0; q < 4; ++q)
+          wp[q] = attn::pack_bf16x2(__uint_as_float(ra[8 * i + 2 * q]) * inv,
+                                    __uint_as_float(ra[8 * i + 2 * q + 1]) * inv);
+        *reinterpret_cast<uint4*>(obox + swz(lane, i)) = w;
       }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(&tmOut, smem_u32(obox), it.h * kHD, qt * kTile + qw * 32, it.b);
+        bulk_commit();
+      }
+      if (qi < T) lse[((size_t)it.b * H + it.h) * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
     }
+    if (lane == 0) bulk_wait_all();  // the output stores complete before the CTA leaves
   }
 
   tc_fence_before();
@@ -418,12 +401,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 
 namespace attn {
 
-cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols) {
-  using Key = std::tuple<const void*, int, int, int>;
+cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols, int box_rows) {
+  using Key = std::tuple<const void*, int, int, int, int>;
   static std::map<Key, CUtensorMap> cache;
   static std::mutex mu;
   static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
-  const Key key{base, B, T, cols};
+  const Key key{base, B, T, cols, box_rows};
   std::lock_guard<std::mutex> g(mu);
   auto it = cache.find(key);
   if (it != cache.end()) {
@@ -440,7 +423,7 @@ cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols) {
   }
   cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)T * cols * 2};
-  cuuint32_t box[3] = {64u, 128u, 1u};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   if (enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -459,10 +442,13 @@ bool attention_fwd_tc_supported(int C, int H) {
 
 cudaError_t attention_fwd_tc(act_t* att, float* lse, const act_t* qkv, int B, int T, int C, int H,
                              int* err, cudaStream_t s) {
-  if (!attention_fwd_tc_supported(C, H) || (reinterpret_cast<uintptr_t>(qkv) & 15))
+  if (!attention_fwd_tc_supported(C, H) || (reinterpret_cast<uintptr_t>(qkv) & 15) ||
+      (reinterpret_cast<uintptr_t>(att) & 15))
     return cudaErrorInvalidValue;
-  CUtensorMap tm;
+  CUtensorMap tm, tmo;
   cudaError_t e = attn::seq_map(&tm, qkv, B, T, 3 * C);
+  if (e != cudaSuccess) return e;
+  e = attn::seq_map(&tmo, att, B, T, C, 32);  // one softmax warp's 32 output rows per box
   if (e != cudaSuccess) return e;
   constexpr size_t smem = attn_smem_bytes();
   static_assert(smem <= 232448, "shared memory budget");
@@ -479,7 +465,7 @@ cudaError_t attention_fwd_tc(act_t* att, float* lse, const act_t* qkv, int B, in
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = items < sms ? items : sms;
-  launch_kernel(flash_fwd_tc_kernel, grid, kThreadsAttn, smem, s, tm, att, lse, B, T, C, H, sl2, err);
+  launch_kernel(flash_fwd_tc_kernel, grid, kThreadsAttn, smem, s, tm, tmo, lse, B, T, C, H, sl2, err);
   note_launch();
   return cudaGetLastError();
 }

@@ -18,9 +18,10 @@ __host__ __device__ constexpr uint32_t idesc(int n, bool b_mn) {
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-// Tensor map over a [B][T][cols] bf16 array: box = 64 columns x 128 rows of
-// one sequence (rows past T read as zero).
-cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols);
+// Tensor map over a [B][T][cols] bf16 array: box = 64 columns x box_rows
+// rows of one sequence, 128-byte swizzle (rows past T read as zero and are
+// not written).
+cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols, int box_rows = 128);
 
 // 32 lanes x 16 consecutive 32-bit TMEM columns (thread i: row lane base + i).
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t* r) {
