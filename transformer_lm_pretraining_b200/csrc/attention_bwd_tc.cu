@@ -8,10 +8,13 @@
 // Two persistent kernels, one CTA per SM walking a static snake order over
 // work items (heaviest first): a TMA warp, two MMA-issuing warps (scores,
 // and the products that accumulate the gradients) and the compute warps
-// (four threads per key row in dK/dV, two per query row in dQ).  In both, the second product of each
-// step takes its A operand (P^T and dS^T, or dS) from TMEM, where the
-// compute warps write it as packed bf16, so shared memory only feeds the
-// tensor core the operands that TMA brings in:
+// (four threads per key row in dK/dV, two per query row in dQ).  In both,
+// the second product of each step takes its A operand (P^T and dS^T, or dS)
+// from TMEM, where the compute warps write it as packed bf16, so shared
+// memory only feeds the tensor core the operands that TMA brings in; each
+// compute warp writes its rows of the item's gradients into a shared-memory
+// box of its own that one TMA store sends out (measured: 194 -> 178 us for
+// both kernels at B16 x T1024 x H12, against per-thread row stores):
 //   dQ:    item = (batch, head, query tile i); streams the key tiles j <= i:
 //          S = Q K^T and dP = dO V^T into TMEM, dS into one of two TMEM
 //          buffers, dQ += dS K in one of two TMEM accumulators (K read
@@ -142,17 +145,20 @@ constexpr int kSub = 64;  // queries per sub-tile
 constexpr uint32_t kOpCol = 256;
 constexpr uint32_t kAccColKV = 384;
 constexpr int kPairBytes = kTile * 8;  // (L log2e, D) of one query tile
+constexpr int kOutBoxKV = 32 * (kHD / kKvSplit) * 2 * 2;  // a compute warp's dK and dV slots: 32 rows each
 constexpr size_t dkdv_smem_bytes() {
-  // [K, V] x 2 items, [Q, dO] x stages, (L, D) pairs x stages, aux
+  // [K, V] x 2 items, [Q, dO] x stages, (L, D) pairs x stages, the compute
+  // warps' dK / dV boxes, aux
   return 1024 + 4 * (size_t)kBox + 2 * (size_t)kQStages * kBox + (size_t)kQStages * kPairBytes +
-         kAux;
+         (kCTkv / 32) * (size_t)kOutBoxKV + kAux;
 }
 
 __global__ void __launch_bounds__(kThreadsKV, 1)
     flash_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
                              const __grid_constant__ CUtensorMap tmDO,
-                             const float2* __restrict__ pairs, __nv_bfloat16* __restrict__ dqkv,
-                             int B, int T, int C, int H, float sl2, float scale, int* err) {
+                             const __grid_constant__ CUtensorMap tmDKV,
+                             const float2* __restrict__ pairs, int B, int T, int C, int H,
+                             float sl2, float scale, int* err) {
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -161,7 +167,8 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
   uint8_t* sQ = sKV + 4 * kBox;           // [kQStages]
   uint8_t* sDO = sQ + kQStages * kBox;    // [kQStages]
   uint8_t* sLD = sDO + kQStages * kBox;   // [kQStages][128 pairs]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sLD + kQStages * kPairBytes);
+  uint8_t* sOut = sLD + kQStages * kPairBytes;  // [compute warp][dK box, dV box]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + (kCTkv / 32) * kOutBoxKV);
   const uint32_t kv_full0 = smem_u32(bars + 0);     // [2]
   const uint32_t kv_empty0 = smem_u32(bars + 2);    // [2]
   const uint32_t qd_full0 = smem_u32(bars + 4);     // [kQStages]
@@ -425,22 +432,40 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
       tc_wait_ld();
       tc_fence_before();
       mbar_arrive(acc_empty);
-      if (kj < T) {
-        __nv_bfloat16* row =
-            dqkv + ((size_t)b * T + kj) * 3 * C + (size_t)h * kHD + kAccCols * part;
+      // this warp's 32 rows x kAccCols columns of dK and of dV into its two
+      // boxes, out by one TMA store each (rows past T are clipped)
+      {
+        constexpr int kRowBytes = kAccCols * 2;
+        uint8_t* box_k = sOut + (warp - 2) * kOutBoxKV;
+        uint8_t* box_v = box_k + 32 * kRowBytes;
+        if (lane == 0) bulk_wait_read<0>();  // the boxes' previous stores have read them
+        __syncwarp();
 #pragma unroll
-        for (int i = 0; i < kAccCols; i += 8) {
-          float a[8], d[8];
+        for (int q = 0; q < kAccCols; q += 8) {
+          uint4 wk, wv;
+          uint32_t* pk4 = reinterpret_cast<uint32_t*>(&wk);
+          uint32_t* pv4 = reinterpret_cast<uint32_t*>(&wv);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            a[q] = __uint_as_float(rk[i + q]) * scale;
-            d[q] = __uint_as_float(rv[i + q]);
+          for (int e = 0; e < 4; ++e) {
+            pk4[e] = attn::pack_bf16x2(__uint_as_float(rk[q + 2 * e]) * scale,
+                                       __uint_as_float(rk[q + 2 * e + 1]) * scale);
+            pv4[e] = attn::pack_bf16x2(__uint_as_float(rv[q + 2 * e]),
+                                       __uint_as_float(rv[q + 2 * e + 1]));
           }
-          store8(row + C + i, a);
-          store8(row + 2 * C + i, d);
+          *reinterpret_cast<uint4*>(box_k + lane * kRowBytes + q * 2) = wk;
+          *reinterpret_cast<uint4*>(box_v + lane * kRowBytes + q * 2) = wv;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x0 = h * kHD + kAccCols * part, y0 = j * kTile + qw * 32;
+          tma_store_3d(&tmDKV, smem_u32(box_k), C + x0, y0, b);
+          tma_store_3d(&tmDKV, smem_u32(box_v), 2 * C + x0, y0, b);
+          bulk_commit();
         }
       }
     }
+    if (lane == 0) bulk_wait_all();  // the dK / dV stores complete before the CTA leaves
   }
 
   tc_fence_before();
@@ -455,17 +480,19 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
 constexpr int kKVStages = 4;
 constexpr uint32_t kDSCol = 256;
 constexpr uint32_t kAccColQ = 384;
+constexpr int kOutBoxQ = 32 * 32 * 2;  // a compute warp's dQ slot: 32 rows x 32 columns
 constexpr size_t dq_smem_bytes() {
-  // Q, dO, O, [K, V] x stages, aux
-  return 1024 + 3 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + kAux;
+  // Q, dO, O, [K, V] x stages, the compute warps' dQ boxes, aux
+  return 1024 + 3 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + (kCTq / 32) * (size_t)kOutBoxQ +
+         kAux;
 }
 
 __global__ void __launch_bounds__(kThreadsQ, 1)
     flash_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
                            const __grid_constant__ CUtensorMap tmDO,
                            const __grid_constant__ CUtensorMap tmO, const float* __restrict__ lse,
-                           float2* __restrict__ pairs, __nv_bfloat16* __restrict__ dqkv, int B,
-                           int T, int C, int H, float sl2, float scale, int* err) {
+                           const __grid_constant__ CUtensorMap tmDQ, float2* __restrict__ pairs,
+                           int B, int T, int C, int H, float sl2, float scale, int* err) {
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -475,7 +502,8 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
   uint8_t* sO = sDO + kBox;                // the forward's output rows (for D)
   uint8_t* sK = sO + kBox;                 // [kKVStages]
   uint8_t* sV = sK + kKVStages * kBox;     // [kKVStages]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kKVStages * kBox);
+  uint8_t* sOut = sV + kKVStages * kBox;   // [compute warp][kOutBoxQ]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + (kCTq / 32) * kOutBoxQ);
   const uint32_t qd_full = smem_u32(bars + 0);
   const uint32_t qd_empty = smem_u32(bars + 1);
   const uint32_t kv_full0 = smem_u32(bars + 2);              // [kKVStages]
@@ -717,19 +745,33 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
       tc_wait_ld();
       tc_fence_before();
       mbar_arrive(acc_empty0 + 8 * ab);
-      if (qi < T) {
-        __nv_bfloat16* row =
-            dqkv + ((size_t)b * T + qi) * 3 * C + (size_t)h * kHD + kAccCols * part;
+      // this warp's 32 rows x kAccCols columns of dQ into its box, out by
+      // one TMA store (rows past T are clipped by the tensor map)
+      {
+        static_assert(kAccCols == 32, "one 64-byte box row per thread");
+        uint8_t* box = sOut + (warp - 2) * kOutBoxQ;
+        if (lane == 0) bulk_wait_read<0>();  // the box's previous store has read it
+        __syncwarp();
 #pragma unroll
         for (int q = 0; q < kAccCols; q += 8) {
-          float a[8];
+          uint4 w;
+          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(rq[q + e]) * scale;
-          store8(row + q, a);
+          for (int e = 0; e < 4; ++e)
+            wp[e] = attn::pack_bf16x2(__uint_as_float(rq[q + 2 * e]) * scale,
+                                      __uint_as_float(rq[q + 2 * e + 1]) * scale);
+          *reinterpret_cast<uint4*>(box + lane * 64 + q * 2) = w;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmDQ, smem_u32(box), h * kHD + kAccCols * part, i * kTile + qw * 32, b);
+          bulk_commit();
         }
       }
       gk += n;
     }
+    if (lane == 0) bulk_wait_all();  // the dQ stores complete before the CTA leaves
   }
 
   tc_fence_before();
@@ -752,12 +794,18 @@ cudaError_t attention_bwd_tc(act_t* dqkv, float* scratch, const act_t* datt, con
       (reinterpret_cast<uintptr_t>(datt) & 15) || (reinterpret_cast<uintptr_t>(att) & 15) ||
       (reinterpret_cast<uintptr_t>(scratch) & 15))
     return cudaErrorInvalidValue;
-  CUtensorMap tq, td, to;
+  CUtensorMap tq, td, to, tdq, tdkv;
   cudaError_t e = attn::seq_map(&tq, qkv, B, T, 3 * C);
   if (e != cudaSuccess) return e;
   e = attn::seq_map(&td, datt, B, T, C);
   if (e != cudaSuccess) return e;
   e = attn::seq_map(&to, att, B, T, C);
+  if (e != cudaSuccess) return e;
+  // the gradients leave through per-warp boxes: 32 rows of 32 (dQ) or
+  // kColsKV (dK, dV) columns, no swizzle
+  e = attn::seq_map(&tdq, dqkv, B, T, 3 * C, 32, 32, false);
+  if (e != cudaSuccess) return e;
+  e = attn::seq_map(&tdkv, dqkv, B, T, 3 * C, 32, kHD / kKvSplit, false);
   if (e != cudaSuccess) return e;
   constexpr size_t sm_a = dkdv_smem_bytes(), sm_b = dq_smem_bytes();
   static_assert(sm_a <= 232448 && sm_b <= 232448, "shared memory budget");
@@ -780,10 +828,10 @@ cudaError_t attention_bwd_tc(act_t* dqkv, float* scratch, const act_t* datt, con
   float2* pairs = reinterpret_cast<float2*>(scratch);
   // dQ first: it forms D = rowsum(dO * O) of its query tiles and stores the
   // (L, D) pairs for dK/dV
-  launch_kernel(flash_bwd_dq_tc_kernel, grid, kThreadsQ, sm_b, s, tq, td, to, lse, pairs, dqkv, B, T, C, H,
-                                                         sl2, scale, err);
-  launch_kernel(flash_bwd_dkdv_tc_kernel, grid, kThreadsKV, sm_a, s, tq, td, pairs, dqkv, B, T, C, H, sl2,
-                                                           scale, err);
+  launch_kernel(flash_bwd_dq_tc_kernel, grid, kThreadsQ, sm_b, s, tq, td, to, lse, tdq, pairs, B, T,
+                C, H, sl2, scale, err);
+  launch_kernel(flash_bwd_dkdv_tc_kernel, grid, kThreadsKV, sm_a, s, tq, td, tdkv, pairs, B, T, C,
+                H, sl2, scale, err);
   note_launch(2);
   return cudaGetLastError();
 }

@@ -401,12 +401,13 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 
 namespace attn {
 
-cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols, int box_rows) {
-  using Key = std::tuple<const void*, int, int, int, int>;
+cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols, int box_rows,
+                    int box_cols, bool swizzle) {
+  using Key = std::tuple<const void*, int, int, int, int, int, bool>;
   static std::map<Key, CUtensorMap> cache;
   static std::mutex mu;
   static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
-  const Key key{base, B, T, cols, box_rows};
+  const Key key{base, B, T, cols, box_rows, box_cols, swizzle};
   std::lock_guard<std::mutex> g(mu);
   auto it = cache.find(key);
   if (it != cache.end()) {
@@ -423,10 +424,10 @@ cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols, i
   }
   cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)T * cols * 2};
-  cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+  cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   if (enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   if (cache.size() > 1024) cache.clear();

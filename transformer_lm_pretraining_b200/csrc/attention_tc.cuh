@@ -18,10 +18,11 @@ __host__ __device__ constexpr uint32_t idesc(int n, bool b_mn) {
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-// Tensor map over a [B][T][cols] bf16 array: box = 64 columns x box_rows
-// rows of one sequence, 128-byte swizzle (rows past T read as zero and are
-// not written).
-cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols, int box_rows = 128);
+// Tensor map over a [B][T][cols] bf16 array: box = box_cols columns x
+// box_rows rows of one sequence (rows past T read as zero and are not
+// written), 128-byte swizzle (box_cols = 64) or none.
+cudaError_t seq_map(CUtensorMap* tm, const void* base, int B, int T, int cols, int box_rows = 128,
+                    int box_cols = 64, bool swizzle = true);
 
 // 32 lanes x 16 consecutive 32-bit TMEM columns (thread i: row lane base + i).
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t* r) {
