@@ -45,8 +45,8 @@ SPEC_BF16_DENSE = 2.25e15
 # dram__bytes_write.sum, weighted by its launches per step
 # (profiles/gemm_tc_dram_traffic_gpt2_124m_step.md).  Valid only for the GEMM
 # sources it was taken on: reported as null as soon as their hash differs.
-GEMM_TRAFFIC = {"bytes_per_launch": 1.4588e8,
-                "sources_sha256": "c367e68adb8b746cfb8d339e920dc8f42d18a2c541030a8c7e294295defb78e7"}
+GEMM_TRAFFIC = {"bytes_per_launch": 1.4641e8,
+                "sources_sha256": "b331d2d038d750d6ac3d71fff203ec179955f8b9a68f6caca40a8116a1be5b5b"}
 GEMM_SOURCES = ("gemm_tc.cu", "gemm_epi.cuh", "tc_util.cuh")
 
 
@@ -212,7 +212,9 @@ def family_roofline(wl, fam, peaks, distinct_ids, recompute):
       ln_fwd      (2L + 1) M (4C + 8)
       ln_bwd      (2L + 1) M (8C + 8)
       classifier  M (4 Vpad + 8)
-      colsum      L M 2 (4C + 3C)   (bias gradients of W_fc and W_qkv)
+      colsum      L M 2 3C + L (M/32) 4C 4   (the bias gradient of W_qkv, a pass
+                  over dqkv; that of W_fc, the reduction of the per-32-row
+                  sums the GELU-backward GEMM's epilogue writes)
       recompute   L M 4C 4          (read u, write GELU(u))
       optimizer   34 bytes per parameter per step (norm: 4; AdamW: 30)
     gemm and attention are tensor-bound: their algorithmic FLOPs come from
@@ -227,7 +229,7 @@ def family_roofline(wl, fam, peaks, distinct_ids, recompute):
         "ln_fwd": nm * (2 * L + 1) * M * (4 * C + 8),
         "ln_bwd": nm * (2 * L + 1) * M * (8 * C + 8),
         "classifier": nm * M * (4 * Vp + 8),
-        "colsum": nm * L * M * 2 * (4 * C + 3 * C),
+        "colsum": nm * L * (M * 2 * 3 * C + ((M + 31) // 32) * 4 * C * 4),
         "recompute": nm * L * M * 4 * C * 4 if recompute else 0,
         "optimizer": 34 * P,
     }
