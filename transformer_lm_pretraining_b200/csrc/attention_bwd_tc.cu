@@ -19,17 +19,18 @@
 //          S = Q K^T and dP = dO V^T into TMEM, dS into one of two TMEM
 //          buffers, dQ += dS K in one of two TMEM accumulators (K read
 //          MN-major).  It runs first: it also forms D = rowsum(dO * O) of
-//          its rows from the dO and O tiles it loads, and stores, per query
-//          row, the pair (L log2(e), D) for the dK/dV kernel in a layout
-//          padded to whole 128-row tiles (rows past T get L = +inf, D = 0,
-//          which makes their P exactly 0 there).
+//          its rows from the dO and O tiles it loads, and stores, per
+//          128-row query tile, the 128 values of -L log2(e) followed by the
+//          128 values of D for the dK/dV kernel, padded to whole tiles (rows
+//          past T get -L log2(e) = -inf, D = 0, which makes their P exactly
+//          0 there).
 //   dK/dV: item = (batch, head, key tile j); streams the query tiles i >= j
 //          in 64-query halves (sub-tiles).  The tensor core computes
 //          S^T = K Q^T and dP^T = V dO^T of a sub-tile into one of two TMEM
 //          score buffers; the compute warps turn them into P^T and dS^T in
 //          one of two TMEM operand buffers; the tensor core then accumulates
 //          dV += P^T dO and dK += dS^T Q in TMEM (dO and Q read MN-major
-//          straight from their tiles).  The (L, D) pairs of each query tile
+//          straight from their tiles).  The (L, D) values of each query tile
 //          arrive by a bulk copy next to its Q and dO tiles.
 // Each compute thread loads its part of the scores from TMEM in one round
 // trip and hands the buffer straight back, so the tensor core computes the
@@ -144,7 +145,7 @@ constexpr int kQStages = 3;
 constexpr int kSub = 64;  // queries per sub-tile
 constexpr uint32_t kOpCol = 256;
 constexpr uint32_t kAccColKV = 384;
-constexpr int kPairBytes = kTile * 8;  // (L log2e, D) of one query tile
+constexpr int kPairBytes = kTile * 8;  // -L log2e [128], then D [128], of one query tile
 constexpr int kOutBoxKV = 32 * (kHD / kKvSplit) * 2 * 2;  // a compute warp's dK and dV slots: 32 rows each
 constexpr size_t dkdv_smem_bytes() {
   // [K, V] x 2 items, [Q, dO] x stages, (L, D) pairs x stages, the compute
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
   uint8_t* sKV = smem;                    // [2 items][K box, V box]
   uint8_t* sQ = sKV + 4 * kBox;           // [kQStages]
   uint8_t* sDO = sQ + kQStages * kBox;    // [kQStages]
-  uint8_t* sLD = sDO + kQStages * kBox;   // [kQStages][128 pairs]
+  uint8_t* sLD = sDO + kQStages * kBox;   // [kQStages][-L log2e x 128, D x 128]
   uint8_t* sOut = sLD + kQStages * kPairBytes;  // [compute warp][dK box, dV box]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + (kCTkv / 32) * kOutBoxKV);
   const uint32_t kv_full0 = smem_u32(bars + 0);     // [2]
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
       const int kj = j * kTile + r;  // this thread's key row
       for (int t = 0; t < n && ok; ++t, ++gt) {
         const int st = gt % kQStages;
-        const float4* ld4 = reinterpret_cast<const float4*>(sLD + st * kPairBytes);
+        const float* ldq = reinterpret_cast<const float*>(sLD + st * kPairBytes);
         for (int hs = 0; hs < 2; ++hs, ++gs) {
           const uint32_t sb = gs & 1u;
           const int cq = kSub * hs + kColsKV * part;  // first query column of this thread in the tile
@@ -392,21 +393,20 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
           uint32_t pk[kColsKV / 2], dk[kColsKV / 2];
 #pragma unroll
           for (int c = 0; c < kColsKV; c += 4) {
-            // (L log2e, D) of queries cq + c .. cq + c + 3 (query-tile stage st)
-            const float4 a = ld4[(cq + c) / 2];
-            const float4 bq = ld4[(cq + c) / 2 + 1];
-            const float lq[4] = {a.x, a.z, bq.x, bq.z};
-            const float dq[4] = {a.y, a.w, bq.y, bq.w};
-            float p[4], ds[4];
+            // -L log2e and D of queries cq + c .. cq + c + 3 (query-tile stage st)
+            const float4 nl = *reinterpret_cast<const float4*>(ldq + cq + c);
+            const float4 dd = *reinterpret_cast<const float4*>(ldq + kTile + cq + c);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              p[e] = fast_exp2(fmaf(__uint_as_float(sr[c + e]), sl2, -lq[e]));
-              ds[e] = p[e] * (__uint_as_float(dp[c + e]) - dq[e]);
+            for (int e = 0; e < 4; e += 2) {
+              float2 p = f2_fma(make_float2(__uint_as_float(sr[c + e]), __uint_as_float(sr[c + e + 1])),
+                                f2_splat(sl2), e ? make_float2(nl.z, nl.w) : make_float2(nl.x, nl.y));
+              p = make_float2(fast_exp2(p.x), fast_exp2(p.y));
+              const float2 ds = f2_mul(
+                  p, f2_sub(make_float2(__uint_as_float(dp[c + e]), __uint_as_float(dp[c + e + 1])),
+                            e ? make_float2(dd.z, dd.w) : make_float2(dd.x, dd.y)));
+              pk[(c + e) / 2] = attn::pack_bf16x2(p.x, p.y);
+              dk[(c + e) / 2] = attn::pack_bf16x2(ds.x, ds.y);
             }
-            pk[c / 2] = attn::pack_bf16x2(p[0], p[1]);
-            pk[c / 2 + 1] = attn::pack_bf16x2(p[2], p[3]);
-            dk[c / 2] = attn::pack_bf16x2(ds[0], ds[1]);
-            dk[c / 2 + 1] = attn::pack_bf16x2(ds[2], ds[3]);
           }
           // the products of sub-tile gs - 2 have read this operand buffer
           ok = warp_and(mbar_wait(pd_empty0 + 8 * sb, ((gs >> 1) & 1u) ^ 1u, abort_flag, err));
@@ -695,8 +695,11 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
         for (int e = 0; e < 8; ++e) drow = fmaf(a[e], o[e], drow);
       }
       mbar_arrive(qd_empty);  // this thread is done with dO and O
-      if (part == 0)
-        pairs[(size_t)bh * Tp + qi] = qi < T ? make_float2(lse2, drow) : make_float2(INFINITY, 0.f);
+      if (part == 0) {  // the query tile's 128 values of -L log2e, then its 128 values of D
+        float* ld = reinterpret_cast<float*>(pairs + (size_t)bh * Tp + (size_t)i * kTile);
+        ld[r] = qi < T ? -lse2 : -INFINITY;
+        ld[kTile + r] = qi < T ? drow : 0.f;
+      }
       for (int jj = 0; jj < n && ok; ++jj) {
         const uint32_t gg = gk + jj;
         const int db = gg & 1;
@@ -720,10 +723,12 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
         uint32_t dk[kColsQ / 2];
 #pragma unroll
         for (int c = 0; c < kColsQ; c += 2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sl2, -lse2));
-          dk[c / 2] = attn::pack_bf16x2(p0 * (__uint_as_float(dp[c]) - drow),
-                                        p1 * (__uint_as_float(dp[c + 1]) - drow));
+          float2 p = f2_fma(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                            f2_splat(sl2), f2_splat(-lse2));
+          p = make_float2(fast_exp2(p.x), fast_exp2(p.y));
+          const float2 ds = f2_mul(
+              p, f2_sub(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), f2_splat(drow)));
+          dk[c / 2] = attn::pack_bf16x2(ds.x, ds.y);
         }
         // the product two tiles back has read this dS buffer
         ok = warp_and(mbar_wait(ds_empty0 + 8 * db, ((gg >> 1) & 1u) ^ 1u, abort_flag, err));

@@ -142,6 +142,49 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float* v) {
   *reinterpret_cast<uint4*>(p) = u;
 }
 
+// Two fp32 lanes per instruction: sm_100's packed add, sub, mul and fma on f32x2.
+// Each lane rounds as the scalar instruction does, so a packed sequence gives
+// the same bits as the same scalar sequence, with half the instructions.
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2_splat(float x) { return make_float2(x, x); }
+// Elements i, i + 1 of a register array as a pair, and back.
+__device__ __forceinline__ float2 get2(const float* v, int i) { return make_float2(v[i], v[i + 1]); }
+__device__ __forceinline__ void set2(float* v, int i, float2 x) {
+  v[i] = x.x;
+  v[i + 1] = x.y;
+}
+
 // GPT-2's GELU: 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3), and
 // its derivative (the tanh form named on the condensed GPT-2 page).
 #if GPT2_ACT_BF16
@@ -157,28 +200,54 @@ __device__ __forceinline__ float rcp_hw(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+namespace gelu_c {
+constexpr float kA = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2 e
+constexpr float kB = kA * 0.044715f;
+constexpr float k = 0.7978845608028654f;  // sqrt(2/pi)
+constexpr float kc = k * 0.044715f;
+constexpr float d0 = -0.5f * k, d1 = -1.5f * kc;  // d = d0 + d1 x^2
+}  // namespace gelu_c
 __device__ __forceinline__ float gelu_tanh(float x) {
-  constexpr float kA = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2 e
-  constexpr float kB = kA * 0.044715f;
-  return x * rcp_hw(1.0f + fast_exp2(x * fmaf(kB, x * x, kA)));
+  using namespace gelu_c;
+  return x * rcp_hw(1.0f + fast_exp2(x * fmaf(x * x, kB, kA)));
 }
 // The derivative uses the hardware tanh (tanh.approx.f32, one special-function
 // op; relative error about 2^-11, so GELU'(x) is off by at most about one
 // bf16 ulp, the precision its product is stored in):
 //   GELU'(x) = 0.5 (1 + t) + 0.5 x (1 - t^2) du/dx,  t = tanh(u),
-//   du/dx = sqrt(2/pi) (1 + 3 * 0.044715 x^2).
+//   du/dx = sqrt(2/pi) (1 + 3 * 0.044715 x^2),
+// evaluated as 0.5 t + 0.5 + x d (t^2 - 1) with d = -du/dx / 2, so that every
+// step is one multiply or multiply-add with a constant operand.
 __device__ __forceinline__ float tanh_hw(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 __device__ __forceinline__ float gelu_tanh_grad(float x) {
-  constexpr float k = 0.7978845608028654f;  // sqrt(2/pi)
-  constexpr float kc = k * 0.044715f;
+  using namespace gelu_c;
   const float x2 = x * x;
-  const float t = tanh_hw(x * fmaf(kc, x2, k));
-  const float hs = (0.5f * x) * fmaf(-t, t, 1.0f);
-  return fmaf(hs, fmaf(3.0f * kc, x2, k), fmaf(0.5f, t, 0.5f));
+  const float t = tanh_hw(x * fmaf(x2, kc, k));
+  const float q = fmaf(t, t, -1.0f);
+  const float xd = x * fmaf(x2, d1, d0);
+  return fmaf(xd, q, fmaf(t, 0.5f, 0.5f));
+}
+
+// gelu_tanh and gelu_tanh_grad on two values (bit-identical to the scalar
+// forms).
+__device__ __forceinline__ float2 gelu_tanh2(float2 x) {
+  using namespace gelu_c;
+  const float2 a = f2_mul(x, f2_fma(f2_mul(x, x), f2_splat(kB), f2_splat(kA)));
+  const float2 d = f2_add(make_float2(fast_exp2(a.x), fast_exp2(a.y)), f2_splat(1.0f));
+  return f2_mul(x, make_float2(rcp_hw(d.x), rcp_hw(d.y)));
+}
+__device__ __forceinline__ float2 gelu_tanh_grad2(float2 x) {
+  using namespace gelu_c;
+  const float2 x2 = f2_mul(x, x);
+  const float2 a = f2_mul(x, f2_fma(x2, f2_splat(kc), f2_splat(k)));
+  const float2 t = make_float2(tanh_hw(a.x), tanh_hw(a.y));
+  const float2 q = f2_fma(t, t, f2_splat(-1.0f));
+  const float2 xd = f2_mul(x, f2_fma(x2, f2_splat(d1), f2_splat(d0)));
+  return f2_fma(xd, q, f2_fma(t, f2_splat(0.5f), f2_splat(0.5f)));
 }
 #else
 __device__ __forceinline__ float gelu_tanh(float x) {
@@ -190,6 +259,10 @@ __device__ __forceinline__ float gelu_tanh_grad(float x) {
   const float th = tanhf(k * (x + 0.044715f * x * x * x));
   const float dinner = k * (1.0f + 3.0f * 0.044715f * x * x);
   return 0.5f * (1.0f + th) + 0.5f * x * (1.0f - th * th) * dinner;
+}
+__device__ __forceinline__ float2 gelu_tanh2(float2 x) { return make_float2(gelu_tanh(x.x), gelu_tanh(x.y)); }
+__device__ __forceinline__ float2 gelu_tanh_grad2(float2 x) {
+  return make_float2(gelu_tanh_grad(x.x), gelu_tanh_grad(x.y));
 }
 #endif
 

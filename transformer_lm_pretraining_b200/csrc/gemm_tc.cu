@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ep.alpha != 1.0f) {  // uniform: the forward and most gradients take alpha = 1
 #pragma unroll
-          for (int i = 0; i < 64; ++i) v[i] *= ep.alpha;
+          for (int i = 0; i < 64; i += 2) set2(v, i, f2_mul(get2(v, i), f2_splat(ep.alpha)));
         }
         if (HAS_BIAS && ep.bias) {
           if (nb + 64 <= ep.N) {
@@ -432,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const float4 b = __ldg(b4 + j);
-              v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+              set2(v, 4 * j, f2_add(get2(v, 4 * j), make_float2(b.x, b.y)));
+              set2(v, 4 * j + 2, f2_add(get2(v, 4 * j + 2), make_float2(b.z, b.w)));
             }
           } else {
 #pragma unroll
@@ -482,13 +483,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float2 x = __bfloat1622float2(x2[i]);
-              if (EPI == EPI_BIAS_RESID) {
-                v[8 * c + 2 * i] += x.x;
-                v[8 * c + 2 * i + 1] += x.y;
-              } else {
-                v[8 * c + 2 * i] *= gelu_tanh_grad(x.x);
-                v[8 * c + 2 * i + 1] *= gelu_tanh_grad(x.y);
-              }
+              const int e = 8 * c + 2 * i;
+              if (EPI == EPI_BIAS_RESID) set2(v, e, f2_add(get2(v, e), x));
+              else set2(v, e, f2_mul(get2(v, e), gelu_tanh_grad2(x)));
             }
           }
         }
@@ -534,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 },
                 [&](uint32_t box_u) { tma_store_3d(&tmX, box_u, nb, r0, 0); });
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = gelu_tanh(v[i]);
+            for (int i = 0; i < 64; i += 2) set2(v, i, gelu_tanh2(get2(v, i)));
           }
           put_box(
               [&](uint8_t* box) {
@@ -549,17 +546,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint8_t* box = wbox + (ob ^ (OUT_BOXES == 2 ? 1 : 0)) * kWarpBox;
             const int rows = min(32, ep.M - r0);
             const uint32_t cof = (uint32_t)(lane & 3) * 4u;
-            float s0 = 0.f, s1 = 0.f;
+            float2 cs = make_float2(0.f, 0.f);
 #pragma unroll 8
             for (int r = 0; r < rows; ++r) {
               const uint32_t w = *reinterpret_cast<const uint32_t*>(box + swz(r, lane >> 2) + cof);
-              s0 += __uint_as_float(w << 16);
-              s1 += __uint_as_float(w & 0xffff0000u);
+              cs = f2_add(cs, make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)));
             }
             const int col = nb + 2 * lane;
             if (col < ep.N)  // N even: both columns in range
-              *reinterpret_cast<float2*>(ep.colsum + (size_t)(r0 >> 5) * ep.N + col) =
-                  make_float2(s0, s1);
+              *reinterpret_cast<float2*>(ep.colsum + (size_t)(r0 >> 5) * ep.N + col) = cs;
           }
         }
       }
