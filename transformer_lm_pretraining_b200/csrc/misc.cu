@@ -501,6 +501,36 @@ struct DecayTable {
   int n;
 };
 
+// One float4 of the update (elements i .. i + 3 of the flat order).
+__device__ __forceinline__ void adamw4(float4& pp, const float4 gg, float4& mm, float4& vv, float4& out,
+                                       const AdamArgs& a, float wd, float clip, float lr, float ibc1,
+                                       float ibc2) {
+  float* pe = &pp.x;
+  const float* ge = &gg.x;
+  float* me = &mm.x;
+  float* ve = &vv.x;
+  float* oe = &out.x;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float gr = ge[j] * clip;
+    me[j] = a.b1 * me[j] + (1.f - a.b1) * gr;
+    ve[j] = a.b2 * ve[j] + (1.f - a.b2) * gr * gr;
+    const float mh = me[j] * ibc1;
+    const float vh = ve[j] * ibc2;
+    pe[j] -= lr * (mh / (sqrtf(vh) + a.eps) + wd * pe[j]);
+    oe[j] = pe[j];
+  }
+}
+
+__device__ __forceinline__ float adamw_decay(size_t i, const DecayTable& dt, float wd) {
+  float r = 0.f;
+  for (int k = 0; k < dt.n; ++k)
+    if (i >= dt.begin[k] && i < dt.end[k]) r = wd;
+  return r;
+}
+
+// Each thread takes two float4 per pass (all eight loads issued before the
+// arithmetic), so more bytes are in flight per thread.
 __global__ void __launch_bounds__(256)
     adamw_kernel(float* __restrict__ p, act_t* __restrict__ pact, const float* __restrict__ g,
                  float* __restrict__ m, float* __restrict__ v, size_t base, size_t n, AdamArgs a,
@@ -509,52 +539,49 @@ __global__ void __launch_bounds__(256)
   const float nrm = scalars[S_NORM];
   if (!isfinite(nrm)) return;  // never apply a non-finite update
   const float clip = scalars[S_CLIP];
-  const float lr = scalars[S_LR], bc1 = scalars[S_BC1], bc2 = scalars[S_BC2];
+  const float lr = scalars[S_LR];
+  const float ibc1 = 1.f / scalars[S_BC1], ibc2 = 1.f / scalars[S_BC2];
   const size_t n4 = n / 4;
   p += base;
   pact += base;
   g += base;
   m += base;
   v += base;
-  for (size_t i4 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4;
-       i4 += (size_t)gridDim.x * blockDim.x) {
-    const size_t i = base + i4 * 4;  // index in the flat parameter order
-    float wd = 0.f;
-    for (int k = 0; k < dt.n; ++k)
-      if (i >= dt.begin[k] && i < dt.end[k]) wd = a.wd;
-    float4 pp = reinterpret_cast<float4*>(p)[i4];
-    const float4 gg = reinterpret_cast<const float4*>(g)[i4];
-    float4 mm = reinterpret_cast<float4*>(m)[i4];
-    float4 vv = reinterpret_cast<float4*>(v)[i4];
-    float* pe = &pp.x;
-    const float* ge = &gg.x;
-    float* me = &mm.x;
-    float* ve = &vv.x;
-    float outv[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float gr = ge[j] * clip;
-      me[j] = a.b1 * me[j] + (1.f - a.b1) * gr;
-      ve[j] = a.b2 * ve[j] + (1.f - a.b2) * gr * gr;
-      const float mh = me[j] / bc1;
-      const float vh = ve[j] / bc2;
-      pe[j] -= lr * (mh / (sqrtf(vh) + a.eps) + wd * pe[j]);
-      outv[j] = pe[j];
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i4 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4; i4 += 2 * stride) {
+    const size_t j4 = i4 + stride;
+    const bool two = j4 < n4;
+    float4 pp[2], gg[2], mm[2], vv[2], out[2];
+    pp[0] = reinterpret_cast<float4*>(p)[i4];
+    gg[0] = reinterpret_cast<const float4*>(g)[i4];
+    mm[0] = reinterpret_cast<float4*>(m)[i4];
+    vv[0] = reinterpret_cast<float4*>(v)[i4];
+    if (two) {
+      pp[1] = reinterpret_cast<float4*>(p)[j4];
+      gg[1] = reinterpret_cast<const float4*>(g)[j4];
+      mm[1] = reinterpret_cast<float4*>(m)[j4];
+      vv[1] = reinterpret_cast<float4*>(v)[j4];
     }
-    reinterpret_cast<float4*>(p)[i4] = pp;
-    reinterpret_cast<float4*>(m)[i4] = mm;
-    reinterpret_cast<float4*>(v)[i4] = vv;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (h == 1 && !two) break;
+      const size_t k4 = h ? j4 : i4;
+      adamw4(pp[h], gg[h], mm[h], vv[h], out[h], a, adamw_decay(base + k4 * 4, dt, a.wd), clip, lr,
+             ibc1, ibc2);
+      reinterpret_cast<float4*>(p)[k4] = pp[h];
+      reinterpret_cast<float4*>(m)[k4] = mm[h];
+      reinterpret_cast<float4*>(v)[k4] = vv[h];
 #if GPT2_ACT_BF16
-    __nv_bfloat162 lo = __floats2bfloat162_rn(outv[0], outv[1]);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(outv[2], outv[3]);
-    uint2 packed;
-    packed.x = *reinterpret_cast<uint32_t*>(&lo);
-    packed.y = *reinterpret_cast<uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(pact)[i4] = packed;
+      __nv_bfloat162 lo = __floats2bfloat162_rn(out[h].x, out[h].y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(out[h].z, out[h].w);
+      uint2 packed;
+      packed.x = *reinterpret_cast<uint32_t*>(&lo);
+      packed.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(pact)[k4] = packed;
 #else
-    (void)pact;
-    (void)outv;
+      (void)pact;
 #endif
+    }
   }
 }
 
