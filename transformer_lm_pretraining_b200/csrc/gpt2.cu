@@ -37,9 +37,23 @@ struct Acts {
   int* tok;
   act_t *dres, *dh, *datt, *dqkv, *dbig;
   float *dsum, *partials, *splitk;
+  // partials of the backward's parameter-gradient column reductions, one
+  // slice per reduction, so that their second stages run together at the
+  // end of the backward (deferred_floats: the arena's size)
+  float* deferred;
+  size_t deferred_floats;
   void* enc_scratch;
   size_t splitk_floats;
 };
+
+// Floats of the deferred-reduction arena: per layer two layernorm backwards
+// (kLnBlocks x 3C partials each), the W_fc bias (per-32-row slabs of 4C) and
+// the W_qkv bias (kColsumChunks x 3C), plus the final layernorm.
+size_t deferred_floats(size_t M, size_t C, size_t L) {
+  const size_t ln = (size_t)kLnBlocks * 3 * C;
+  const size_t fc = std::max((M + 31) / 32, (size_t)kColsumChunks) * 4 * C;
+  return (2 * L + 1) * ln + L * (fc + (size_t)kColsumChunks * 3 * C);
+}
 
 constexpr int kMaxSplits = 8;
 
@@ -179,6 +193,8 @@ size_t carve_work(const Layout& lay, int B, int T, int recompute, void* base, Ac
   x.dsum = c.take<float>(attention_bwd_scratch_floats(B, T, (int)H));
   const size_t part = std::max((size_t)kColsumChunks * 4 * C, (size_t)kLnBlocks * 3 * C);
   x.partials = c.take<float>(part);
+  x.deferred_floats = deferred_floats(M, C, L);
+  x.deferred = c.take<float>(x.deferred_floats);
   x.splitk_floats = (size_t)kMaxSplits * 4 * C * C;
   x.splitk = c.take<float>(x.splitk_floats);
   x.enc_scratch = c.take<char>(encoder_scratch_bytes((int)M, (int)C));
@@ -743,6 +759,31 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
   float* G = h->grads;
   EncoderScratch es;
   encoder_scratch_carve(&es, a.enc_scratch, M, C);
+  // Without per-layer gradient events (no overlapped data-parallel
+  // reduction), the second stages of the parameter-gradient column
+  // reductions (layernorm gamma and beta, the biases) wait until the end of
+  // the backward and run in one grouped launch, off the path from layer to
+  // layer; each reduction keeps its partials in a slice of its own.
+  const bool defer = h->bwd_events.empty() && a.deferred != nullptr;
+  ReduceJobs jobs;
+  jobs.n = 0;
+  ReduceJob job;
+  size_t dused = 0;
+  auto slice = [&](size_t n, float* immediate) {
+    if (!defer) return immediate;
+    float* p = a.deferred + dused;
+    dused += n;
+    return p;
+  };
+  auto queue = [&]() {
+    if (!defer) return;
+    if (!reduce_jobs_add(jobs, job)) {  // the list is full: run it first
+      reduce_jobs_run(jobs, s);
+      reduce_jobs_add(jobs, job);
+    }
+  };
+  const size_t ln_part = (size_t)kLnBlocks * 3 * C;
+  ReduceJob* dj = defer ? &job : nullptr;
 
   {  // dhf = scale * dz wte  (dz: the logits buffer)
     GemmArgs ga = gemm_args(M, C, y.Vp);
@@ -766,7 +807,8 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
   // dres = d x_L; its column sum is the bias gradient of the last W_p
   layernorm_bwd(a.dres, a.dh, a.res + (size_t)L * MC, a.meanf, a.rstdf, P + y.off[T_LNFG],
                 G + y.off[T_LNFG], G + y.off[T_LNFB], G + y.off[T_BP] + (size_t)(L - 1) * C,
-                a.partials, M, C, 0, s);
+                slice(ln_part, a.partials), M, C, 0, s, dj);
+  queue();
 
   for (int l = L - 1; l >= 0; --l) {
     const act_t* x = a.res + (size_t)l * MC;
@@ -788,12 +830,16 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       // epilogue (into the split-K workspace, free until dWp below), or a
       // pass over du while it is still in L2
       const int slabs = (M + 31) / 32;
-      const bool fused = gemm_colsum_supported() && (size_t)slabs * 4 * C <= a.splitk_floats;
-      if (fused) ga.colsum = a.splitk;
+      const bool fused =
+          gemm_colsum_supported() && (defer || (size_t)slabs * 4 * C <= a.splitk_floats);
+      float* part = slice(std::max((size_t)slabs, (size_t)kColsumChunks) * 4 * C,
+                          fused ? a.splitk : a.partials);
+      if (fused) ga.colsum = part;
       GPT2_TRY(run_gemm(h, ga));
       mark(h, PK_COLSUM);
-      if (fused) colsum_reduce(G + y.off[T_BFC] + (size_t)l * 4 * C, a.splitk, slabs, 4 * C, s);
-      else colsum_acc(G + y.off[T_BFC] + (size_t)l * 4 * C, a.dbig, M, 4 * C, a.partials, s);
+      if (fused) colsum_reduce(G + y.off[T_BFC] + (size_t)l * 4 * C, part, slabs, 4 * C, s, dj);
+      else colsum_acc(G + y.off[T_BFC] + (size_t)l * 4 * C, a.dbig, M, 4 * C, part, s, dj);
+      queue();
     }
     if (h->recompute) {  // g = gelu(u), as the forward's epilogue computed it
       mark(h, PK_RECOMPUTE);
@@ -832,7 +878,8 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     layernorm_bwd(a.dres, a.dh, xm, a.mean2 + (size_t)l * M, a.rstd2 + (size_t)l * M,
                   P + y.off[T_LN2G] + (size_t)l * C, G + y.off[T_LN2G] + (size_t)l * C,
                   G + y.off[T_LN2B] + (size_t)l * C, G + y.off[T_BO] + (size_t)l * C,
-                  a.partials, M, C, 1, s);
+                  slice(ln_part, a.partials), M, C, 1, s, dj);
+    queue();
     // ---- attention: xm = x + att Wo^T + bo
     {  // datt = dres Wo
       GemmArgs ga = gemm_args(M, C, C);
@@ -857,7 +904,9 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
                                C, H, h->err, s));
     // the bias gradient of W_qkv while dqkv is still in L2
     mark(h, PK_COLSUM);
-    colsum_acc(G + y.off[T_BQKV] + (size_t)l * 3 * C, a.dqkv, M, 3 * C, a.partials, s);
+    colsum_acc(G + y.off[T_BQKV] + (size_t)l * 3 * C, a.dqkv, M, 3 * C,
+               slice((size_t)kColsumChunks * 3 * C, a.partials), s, dj);
+    queue();
     {  // dh = dqkv Wqkv
       GemmArgs ga = gemm_args(M, C, 3 * C);
       ga.A = a.dqkv; ga.lda = 3 * C;
@@ -881,8 +930,14 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     layernorm_bwd(a.dres, a.dh, x, a.mean1 + (size_t)l * M, a.rstd1 + (size_t)l * M,
                   P + y.off[T_LN1G] + (size_t)l * C, G + y.off[T_LN1G] + (size_t)l * C,
                   G + y.off[T_LN1B] + (size_t)l * C,
-                  l > 0 ? G + y.off[T_BP] + (size_t)(l - 1) * C : nullptr, a.partials, M, C, 1, s);
+                  l > 0 ? G + y.off[T_BP] + (size_t)(l - 1) * C : nullptr,
+                  slice(ln_part, a.partials), M, C, 1, s, dj);
+    queue();
     if (!h->bwd_events.empty()) GPT2_CUDA(h, cudaEventRecord(h->bwd_events[l], s));
+  }
+  if (defer) {
+    mark(h, PK_COLSUM);
+    reduce_jobs_run(jobs, s);
   }
   mark(h, PK_ENCODER);
   encoder_bwd(G + y.off[T_WTE], G + y.off[T_WPE], a.dres, a.tok, B, T, C, y.Vp, es, s);

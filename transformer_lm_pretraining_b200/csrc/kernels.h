@@ -102,17 +102,44 @@ void layernorm_fwd(act_t* y, float* mean, float* rstd, const act_t* x, const flo
 // dres.  Per-block partials in `partials` [kLnBlocks * 3C], reduced in a
 // fixed order.
 constexpr int kLnBlocks = 592;
+// The second stage of a two-stage reduction, described instead of launched:
+// dst[j][c] += sum over rows r < nrows of partials[r * nsums * C + j * C + c]
+// for j < nsums (dst[j] null: skipped), in the fixed order of `kind`
+// (REDUCE_LN: the layernorm backward's; REDUCE_COLSUM: colsum_reduce's), so
+// that a deferred reduction gives the same bits as the immediate one.
+enum ReduceKind { REDUCE_LN = 0, REDUCE_COLSUM = 1 };
+struct ReduceJob {
+  float* dst[3];
+  const float* partials;
+  int nrows, nsums, C, kind;
+};
+constexpr int kMaxReduceJobs = 64;
+struct ReduceJobs {
+  int n;
+  int group_end[kMaxReduceJobs];  // blocks of jobs 0..k (32 columns per block)
+  ReduceJob job[kMaxReduceJobs];
+};
+// Adds a job to the list (false when the list is full).
+bool reduce_jobs_add(ReduceJobs& jobs, const ReduceJob& j);
+// Runs every job of the list in one launch and empties it.
+void reduce_jobs_run(ReduceJobs& jobs, cudaStream_t s);
+
+// With `defer` set, only the first stage runs and *defer describes the
+// second (the partials must then stay untouched until it has run).
 void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
                    const float* rstd, const float* g, float* dg, float* db, float* dbias_out,
-                   float* partials, int M, int C, int accumulate, cudaStream_t s);
+                   float* partials, int M, int C, int accumulate, cudaStream_t s,
+                   ReduceJob* defer = nullptr);
 
 // ------------------------------------------------------------ column sums --
 constexpr int kColsumChunks = 192;
 // db[n] += sum_m dy[m, n] (fixed order); partials: [kColsumChunks * N] floats
-void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s);
+void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s,
+                ReduceJob* defer = nullptr);
 // db[n] += sum over c < chunks of partials[c * N + n], c ascending (the
 // second stage of colsum_acc, for partials a GEMM epilogue wrote)
-void colsum_reduce(float* db, const float* partials, int chunks, int N, cudaStream_t s);
+void colsum_reduce(float* db, const float* partials, int chunks, int N, cudaStream_t s,
+                   ReduceJob* defer = nullptr);
 
 // ----------------------------------------------------------- attention --
 // qkv [B*T, 3C] = [q | k | v], head h at columns h*hd..; att [B*T, C];

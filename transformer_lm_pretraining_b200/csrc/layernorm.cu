@@ -8,6 +8,7 @@
 // and summed over blocks in block order: no atomics, fixed summation order.
 
 #include "kernels.h"
+#include "reduce.cuh"
 #include "tc_util.cuh"
 
 namespace gpt2k {
@@ -479,31 +480,7 @@ __global__ void __launch_bounds__(1024)
     ln_bwd_reduce_kernel(float* __restrict__ dg, float* __restrict__ db, float* __restrict__ dsum3,
                          const float* __restrict__ partials, int nblk, int nsums, int C) {
   pdl_start();
-  __shared__ float red[32][33];
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int col = blockIdx.x * 32 + tx;  // over nsums * C
-  const size_t stride = (size_t)nsums * C;
-  float s[4] = {0.f, 0.f, 0.f, 0.f};
-  if (col < nsums * C) {
-    const float* p = partials + col;
-    int b = ty;
-    for (; b + 96 < nblk; b += 128) {
-      s[0] += p[(size_t)b * stride];
-      s[1] += p[(size_t)(b + 32) * stride];
-      s[2] += p[(size_t)(b + 64) * stride];
-      s[3] += p[(size_t)(b + 96) * stride];
-    }
-    for (int k = 0; b < nblk; b += 32, ++k) s[k] += p[(size_t)b * stride];
-  }
-  red[ty][tx] = (s[0] + s[1]) + (s[2] + s[3]);
-  __syncthreads();
-  if (ty == 0 && col < nsums * C) {
-    float t = 0.f;
-    for (int k = 0; k < 32; ++k) t += red[k][tx];
-    const int j = col / C, c = col % C;
-    float* dst = j == 0 ? dg : (j == 1 ? db : dsum3);
-    dst[c] += t;
-  }
+  ln_reduce_block(dg, db, dsum3, partials, nblk, nsums, C, blockIdx.x);
 }
 
 // Launches one wave: as many blocks as are resident at once (at most
@@ -562,7 +539,8 @@ void layernorm_fwd(act_t* y, float* mean, float* rstd, const act_t* x, const flo
 
 void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* mean,
                    const float* rstd, const float* g, float* dg, float* db, float* dbias_out,
-                   float* partials, int M, int C, int accumulate, cudaStream_t s) {
+                   float* partials, int M, int C, int accumulate, cudaStream_t s,
+                   ReduceJob* defer) {
   const int nsums = dbias_out ? 3 : 2;
   int nblk = kLnBlocks;
   switch (C * 4 + nsums) {  // widths with a row-group kernel
@@ -590,6 +568,11 @@ void layernorm_bwd(act_t* dres, const act_t* dy, const act_t* x, const float* me
     default: break;
   }
 reduce:
+  if (defer) {
+    *defer = ReduceJob{{dg, db, dbias_out}, partials, nblk, nsums, C, REDUCE_LN};
+    note_launch();
+    return;
+  }
   launch_kernel(ln_bwd_reduce_kernel, (nsums * C + 31) / 32, 1024, 0, s, dg, db, dbias_out, partials, nblk,
                                                                nsums, C);
   note_launch(2);

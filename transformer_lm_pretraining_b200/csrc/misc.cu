@@ -6,6 +6,7 @@
 #include <cuda_fp16.h>
 
 #include "kernels.h"
+#include "reduce.cuh"
 #include "tc_util.cuh"
 
 namespace gpt2k {
@@ -106,26 +107,25 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// db[n] += sum over chunks of partials[chunk][n] in a fixed order: thread
-// (tx, ty) of a 32 x 32 block takes column tx of a 32-column group and
-// chunks ty, ty+32, ...; the 32 partial sums are added in ty order.
+// db[n] += sum over chunks of partials[chunk][n] in a fixed order
+// (colsum_reduce_block).
 __global__ void __launch_bounds__(1024)
     colsum_reduce_kernel(float* __restrict__ db, const float* __restrict__ partials, int chunks,
                          int N) {
   pdl_start();
-  __shared__ float red[32][33];
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int n = blockIdx.x * 32 + tx;
-  float s = 0.f;
-  if (n < N)
-    for (int c = ty; c < chunks; c += 32) s += partials[(size_t)c * N + n];
-  red[ty][tx] = s;
-  __syncthreads();
-  if (ty == 0 && n < N) {
-    float t = 0.f;
-    for (int k = 0; k < 32; ++k) t += red[k][tx];
-    db[n] += t;
-  }
+  colsum_reduce_block(db, partials, chunks, N, blockIdx.x);
+}
+
+// Every job of the list: block b belongs to the first job k with
+// b < group_end[k] and reduces that job's 32-column group b - group_end[k - 1].
+__global__ void __launch_bounds__(1024) reduce_jobs_kernel(const __grid_constant__ ReduceJobs jobs) {
+  pdl_start();
+  int k = 0;
+  while (k + 1 < jobs.n && (int)blockIdx.x >= jobs.group_end[k]) ++k;
+  const ReduceJob& j = jobs.job[k];
+  const int grp = (int)blockIdx.x - (k ? jobs.group_end[k - 1] : 0);
+  if (j.kind == REDUCE_LN) ln_reduce_block(j.dst[0], j.dst[1], j.dst[2], j.partials, j.nrows, j.nsums, j.C, grp);
+  else colsum_reduce_block(j.dst[0], j.partials, j.nrows, j.C, grp);
 }
 
 // -------------------------------------------------------- classifier --
@@ -626,7 +626,8 @@ int grid_for(size_t n, int threads, int max_blocks) {
 
 }  // namespace
 
-void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s) {
+void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s,
+                ReduceJob* defer) {
   // as many blocks as are resident at once and no more: a block past the
   // first wave would run on its own after it
   static int per_sm = 0;
@@ -642,13 +643,33 @@ void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaS
   const int chunks = (M + rows - 1) / rows;
   dim3 g(colgroups, chunks);
   launch_kernel(colsum_partial_kernel, g, 256, 0, s, partials, dy, M, N, rows);
-  launch_kernel(colsum_reduce_kernel, (N + 31) / 32, 1024, 0, s, db, partials, chunks, N);
-  note_launch(2);
+  note_launch();
+  colsum_reduce(db, partials, chunks, N, s, defer);
 }
 
-void colsum_reduce(float* db, const float* partials, int chunks, int N, cudaStream_t s) {
+void colsum_reduce(float* db, const float* partials, int chunks, int N, cudaStream_t s,
+                   ReduceJob* defer) {
+  if (defer) {
+    *defer = ReduceJob{{db, nullptr, nullptr}, partials, chunks, 1, N, REDUCE_COLSUM};
+    return;
+  }
   launch_kernel(colsum_reduce_kernel, (N + 31) / 32, 1024, 0, s, db, partials, chunks, N);
   note_launch();
+}
+
+bool reduce_jobs_add(ReduceJobs& jobs, const ReduceJob& j) {
+  if (jobs.n >= kMaxReduceJobs) return false;
+  const int groups = (j.nsums * j.C + 31) / 32;
+  jobs.group_end[jobs.n] = (jobs.n ? jobs.group_end[jobs.n - 1] : 0) + groups;
+  jobs.job[jobs.n++] = j;
+  return true;
+}
+
+void reduce_jobs_run(ReduceJobs& jobs, cudaStream_t s) {
+  if (jobs.n == 0) return;
+  launch_kernel(reduce_jobs_kernel, jobs.group_end[jobs.n - 1], 1024, 0, s, jobs);
+  note_launch();
+  jobs.n = 0;
 }
 
 void classifier(act_t* logits, float* losses, const int* tgt, int M, int V, int Vp, int write_grad,
