@@ -197,9 +197,14 @@ __device__ __forceinline__ void cluster_sync() {
                    "memory");
 }
 // Arrive on an mbarrier given by its shared::cluster address (possibly in
-// the peer CTA), releasing this thread's prior accesses at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+// the peer CTA) with relaxed semantics: the arrival orders none of this
+// thread's prior memory accesses, so it does not wait for its global stores
+// in flight (a release at cluster scope did, measured: 10-12 us on each GELU
+// product in CTA pairs).  For signals whose waiter consumes nothing that the
+// arriving thread wrote, such as "these TMEM columns are read" after
+// tcgen05.wait::ld has returned their values.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
 // Phase test acquiring at cluster scope (for barriers the peer CTA arrives on).
