@@ -8,6 +8,8 @@
 // distinct id adds its chunk partials in chunk order into dwte.  The
 // summation order therefore depends only on the token sequence.
 
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace gpt2k {
@@ -175,18 +177,36 @@ __global__ void chunk_partial_kernel(float* __restrict__ partial, const act_t* _
 }
 
 // One block per sorted position; blocks at the start of a run of equal ids
-// add the run's chunk partials (in chunk order) into dwte[id].
+// add the run's chunk partials (in chunk order) into dwte[id].  VEC: four
+// columns per thread as float4 (C % 4 == 0 and 16-byte aligned rows), so a
+// block issues its whole row at once.
+template <bool VEC>
 __global__ void segment_sum_kernel(float* __restrict__ dwte, const float* __restrict__ partial,
                                    const int* __restrict__ skeys, int M, int C) {
   pdl_start();
   const int s = blockIdx.x;
   const int key = skeys[s];
   if (s > 0 && skeys[s - 1] == key) return;
-  for (int c = threadIdx.x; c < C; c += blockDim.x) {
-    float acc = partial[(size_t)s * C + c];
-    for (int j = (s / kChunk + 1) * kChunk; j < M && skeys[j] == key; j += kChunk)
-      acc += partial[(size_t)j * C + c];
-    dwte[(size_t)key * C + c] += acc;
+  const int j0 = (s / kChunk + 1) * kChunk;  // the first position of the next chunk
+  if (VEC) {
+    const int C4 = C / 4;
+    for (int c = threadIdx.x; c < C4; c += blockDim.x) {
+      float4 acc = reinterpret_cast<const float4*>(partial + (size_t)s * C)[c];
+      for (int j = j0; j < M && skeys[j] == key; j += kChunk) {
+        const float4 p = reinterpret_cast<const float4*>(partial + (size_t)j * C)[c];
+        acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+      }
+      float4* d = reinterpret_cast<float4*>(dwte + (size_t)key * C) + c;
+      float4 o = *d;
+      o.x += acc.x; o.y += acc.y; o.z += acc.z; o.w += acc.w;
+      *d = o;
+    }
+  } else {
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+      float acc = partial[(size_t)s * C + c];
+      for (int j = j0; j < M && skeys[j] == key; j += kChunk) acc += partial[(size_t)j * C + c];
+      dwte[(size_t)key * C + c] += acc;
+    }
   }
 }
 
@@ -242,7 +262,13 @@ void encoder_bwd(float* dwte, float* dwpe, const act_t* dx0, const int* tok_save
   const int nchunks = (M + kChunk - 1) / kChunk;
   dim3 g1(nchunks, (C / 2 + 127) / 128);
   launch_kernel(chunk_partial_kernel, g1, 128, 0, s, es.partial, dx0, es.keys[cur], es.vals[cur], M, C);
-  launch_kernel(segment_sum_kernel, M, 128, 0, s, dwte, es.partial, es.keys[cur], M, C);
+  if (C % 4 == 0 && !(reinterpret_cast<uintptr_t>(dwte) & 15) &&
+      !(reinterpret_cast<uintptr_t>(es.partial) & 15)) {
+    const int threads = std::min(256, (C / 4 + 31) / 32 * 32);
+    launch_kernel(segment_sum_kernel<true>, M, threads, 0, s, dwte, es.partial, es.keys[cur], M, C);
+  } else {
+    launch_kernel(segment_sum_kernel<false>, M, 128, 0, s, dwte, es.partial, es.keys[cur], M, C);
+  }
   note_launch(4);
 }
 
