@@ -477,13 +477,13 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
 // --------------------------------------------------------------------- dQ --
 // TMEM columns: [0, 128) S, [128, 256) dP (fp32); [256, 384) two dS buffers
 // (bf16 pairs of 128 keys); [384, 512) two dQ accumulators.
-constexpr int kKVStages = 4;
+constexpr int kKVStages = 3;
 constexpr uint32_t kDSCol = 256;
 constexpr uint32_t kAccColQ = 384;
 constexpr int kOutBoxQ = 32 * 32 * 2;  // a compute warp's dQ slot: 32 rows x 32 columns
 constexpr size_t dq_smem_bytes() {
-  // Q, dO, O, [K, V] x stages, the compute warps' dQ boxes, aux
-  return 1024 + 3 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + (kCTq / 32) * (size_t)kOutBoxQ +
+  // [Q, dO, O] x 2 items, [K, V] x stages, the compute warps' dQ boxes, aux
+  return 1024 + 6 * (size_t)kBox + 2 * (size_t)kKVStages * kBox + (kCTq / 32) * (size_t)kOutBoxQ +
          kAux;
 }
 
@@ -497,25 +497,25 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sDO = sQ + kBox;
-  uint8_t* sO = sDO + kBox;                // the forward's output rows (for D)
-  uint8_t* sK = sO + kBox;                 // [kKVStages]
+  // Q, dO and O (the forward's output rows, for D) of two items: the next
+  // item's tiles arrive while the current one runs
+  uint8_t* sQ0 = smem;                     // [2 items][Q, dO, O]
+  uint8_t* sK = sQ0 + 6 * kBox;            // [kKVStages]
   uint8_t* sV = sK + kKVStages * kBox;     // [kKVStages]
   uint8_t* sOut = sV + kKVStages * kBox;   // [compute warp][kOutBoxQ]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + (kCTq / 32) * kOutBoxQ);
-  const uint32_t qd_full = smem_u32(bars + 0);
-  const uint32_t qd_empty = smem_u32(bars + 1);
-  const uint32_t kv_full0 = smem_u32(bars + 2);              // [kKVStages]
-  const uint32_t kv_empty0 = smem_u32(bars + 2 + kKVStages); // [kKVStages]
-  const uint32_t sd_full = smem_u32(bars + 2 + 2 * kKVStages);
+  const uint32_t qd_full0 = smem_u32(bars + 0);             // [2 items]
+  const uint32_t qd_empty0 = smem_u32(bars + 2);            // [2 items]
+  const uint32_t kv_full0 = smem_u32(bars + 4);              // [kKVStages]
+  const uint32_t kv_empty0 = smem_u32(bars + 4 + kKVStages); // [kKVStages]
+  const uint32_t sd_full = smem_u32(bars + 4 + 2 * kKVStages);
   const uint32_t sd_empty = sd_full + 8;
   const uint32_t ds_full0 = sd_full + 16;                    // [2]
   const uint32_t ds_empty0 = sd_full + 32;                   // [2]
   const uint32_t acc_full0 = sd_full + 48;                   // [2]
   const uint32_t acc_empty0 = sd_full + 64;                  // [2]
   const uint32_t drain0 = sd_full + 80;                      // [2] abort path only
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 + 2 * kKVStages + 12);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 + 2 * kKVStages + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int nq = (T + kTile - 1) / kTile;
@@ -524,8 +524,10 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(qd_full, 1);
-    mbar_init(qd_empty, 1 + kCTq);  // the last S/dP product, and every compute thread's D
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(qd_full0 + 8 * s, 1);
+      mbar_init(qd_empty0 + 8 * s, 1 + kCTq);  // the last S/dP product, and every compute thread's D
+    }
     for (int s = 0; s < kKVStages; ++s) {
       mbar_init(kv_full0 + 8 * s, 1);
       mbar_init(kv_empty0 + 8 * s, 2);  // the scores read K, V; the products K
@@ -563,11 +565,13 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
         if (w < 0) break;
         const int i = nq - 1 - w / BH, bh = w % BH, b = bh / H, h = bh % H;
         const int n = i + 1;  // key tiles 0 .. i
-        if (!mbar_wait(qd_empty, (n_item & 1u) ^ 1u, abort_flag, err)) break;
-        mbar_expect_tx(qd_full, 3 * kBox);
-        tma_load_3d(smem_u32(sQ), &tmQKV, qd_full, h * kHD, i * kTile, b);
-        tma_load_3d(smem_u32(sDO), &tmDO, qd_full, h * kHD, i * kTile, b);
-        tma_load_3d(smem_u32(sO), &tmO, qd_full, h * kHD, i * kTile, b);
+        const uint32_t qb = n_item & 1u, qfb = qd_full0 + 8 * qb;
+        if (!mbar_wait(qd_empty0 + 8 * qb, ((n_item >> 1) & 1u) ^ 1u, abort_flag, err)) break;
+        uint8_t* sq = sQ0 + qb * 3 * kBox;
+        mbar_expect_tx(qfb, 3 * kBox);
+        tma_load_3d(smem_u32(sq), &tmQKV, qfb, h * kHD, i * kTile, b);
+        tma_load_3d(smem_u32(sq + kBox), &tmDO, qfb, h * kHD, i * kTile, b);
+        tma_load_3d(smem_u32(sq + 2 * kBox), &tmO, qfb, h * kHD, i * kTile, b);
         for (int jj = 0; jj < n; ++jj, ++gk) {
           const int st = gk % kKVStages;
           const uint32_t par = (gk / kKVStages) & 1u;
@@ -584,7 +588,8 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
         }
       }
       const uint64_t t0 = global_ns();
-      if (n_item) drain_wait(qd_full, (n_item - 1) & 1u, t0);
+      for (uint32_t m = n_item > 2 ? n_item - 2 : 0; m < n_item; ++m)
+        drain_wait(qd_full0 + 8 * (m & 1u), (m >> 1) & 1u, t0);
       for (int s = 0; s < kKVStages; ++s)
         if (issued & (1u << s)) drain_wait(kv_full0 + 8 * s, (last_par >> s) & 1u, t0);
     }
@@ -594,14 +599,15 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
       // S = Q K_j^T and dP = dO V_j^T for every key tile j of every item;
       // the dQ products run from their own warp.
       constexpr uint32_t idS = attn::idesc(kTile, false);
-      const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO);
       uint32_t n_item = 0, gk = 0;
       bool ok = true;
       for (int k = 0; ok; ++k, ++n_item) {
         const int w = snake_item(k, items);
         if (w < 0) break;
         const int n = nq - w / BH;  // i + 1
-        ok = mbar_wait(qd_full, n_item & 1u, abort_flag, err);
+        const uint32_t qb = n_item & 1u;
+        const uint32_t q_base = smem_u32(sQ0 + qb * 3 * kBox), do_base = q_base + kBox;
+        ok = mbar_wait(qd_full0 + 8 * qb, (n_item >> 1) & 1u, abort_flag, err);
         for (int jj = 0; jj < n && ok; ++jj) {
           const uint32_t gg = gk + jj;
           const int st = gg % kKVStages;
@@ -619,7 +625,7 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
                    kk > 0 ? 1u : 0u);
           tc_commit(sd_full);
           tc_commit(kv_empty0 + 8 * st);  // the scores are done with K_j, V_j
-          if (jj == n - 1) tc_commit(qd_empty);  // Q and dO are no longer read
+          if (jj == n - 1) tc_commit(qd_empty0 + 8 * qb);  // Q and dO are no longer read
         }
         gk += n;
       }
@@ -673,18 +679,31 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
     uint32_t n_item = 0, gk = 0;
     bool ok = true;
+    // this row's L of an item, loaded one item ahead (the load's latency
+    // would otherwise sit at the start of every item)
+    auto row_lse = [&](int k) {
+      const int w = snake_item(k, items);
+      if (w < 0) return 0.f;
+      const int qi = (nq - 1 - w / BH) * kTile + r;
+      return qi < T ? lse[(size_t)(w % BH) * T + qi] : 0.f;
+    };
+    float lse_next = row_lse(0);
     for (int k = 0; ok; ++k, ++n_item) {
       const int w = snake_item(k, items);
       if (w < 0) break;
       const int i = nq - 1 - w / BH, bh = w % BH, b = bh / H, h = bh % H;
       const int n = i + 1;
       const int qi = i * kTile + r;  // this thread's query row
-      const float lse2 = qi < T ? lse[(size_t)bh * T + qi] * kLog2e : 0.f;
+      const float lse2 = lse_next * kLog2e;
+      lse_next = row_lse(k + 1);
       // D = rowsum(dO * O) of this row from the item's dO and O tiles (rows
       // past T are zero-filled; every thread of the row forms it); stored
       // with L for the dK/dV kernel
-      ok = warp_and(mbar_wait(qd_full, n_item & 1u, abort_flag, err));
+      const uint32_t qb = n_item & 1u;
+      ok = warp_and(mbar_wait(qd_full0 + 8 * qb, (n_item >> 1) & 1u, abort_flag, err));
       if (!ok) break;
+      const uint8_t* sDO = sQ0 + qb * 3 * kBox + kBox;
+      const uint8_t* sO = sDO + kBox;
       float drow = 0.f;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -694,7 +713,7 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) drow = fmaf(a[e], o[e], drow);
       }
-      mbar_arrive(qd_empty);  // this thread is done with dO and O
+      mbar_arrive(qd_empty0 + 8 * qb);  // this thread is done with dO and O
       if (part == 0) {  // the query tile's 128 values of -L log2e, then its 128 values of D
         float* ld = reinterpret_cast<float*>(pairs + (size_t)bh * Tp + (size_t)i * kTile);
         ld[r] = qi < T ? -lse2 : -INFINITY;

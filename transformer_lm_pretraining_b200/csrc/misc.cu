@@ -466,13 +466,27 @@ __global__ void __launch_bounds__(256) norm_partial_kernel(double* __restrict__ 
   if (threadIdx.x == 0) partials[blockIdx.x] = red[0];
 }
 
-__global__ void sumsq_final_kernel(double* __restrict__ out, const double* __restrict__ partials,
-                                   int nblk) {
-  pdl_start();
-  if (threadIdx.x != 0) return;
+// The sum of the nblk block partials, in a fixed order: thread t of 256 adds
+// partials t, t + 256, ..., then a fixed tree over the threads.
+__device__ __forceinline__ double partials_sum(const double* __restrict__ partials, int nblk) {
+  __shared__ double red[256];
   double s = 0.0;
-  for (int b = 0; b < nblk; ++b) s += partials[b];
-  *out = s;
+  for (int b = threadIdx.x; b < nblk; b += 256) s += partials[b];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  return red[0];
+}
+
+__global__ void __launch_bounds__(256) sumsq_final_kernel(double* __restrict__ out,
+                                                          const double* __restrict__ partials,
+                                                          int nblk) {
+  pdl_start();
+  const double s = partials_sum(partials, nblk);
+  if (threadIdx.x == 0) *out = s;
 }
 
 __global__ void clip_from_sumsq_kernel(float* __restrict__ scalars, const double* __restrict__ sumsq,
@@ -483,12 +497,12 @@ __global__ void clip_from_sumsq_kernel(float* __restrict__ scalars, const double
   scalars[S_CLIP] = (nrm > max_norm) ? max_norm / (nrm + 1e-6f) : 1.0f;
 }
 
-__global__ void norm_final_kernel(float* __restrict__ scalars, const double* __restrict__ partials,
-                                  int nblk, float max_norm) {
+__global__ void __launch_bounds__(256) norm_final_kernel(float* __restrict__ scalars,
+                                                         const double* __restrict__ partials,
+                                                         int nblk, float max_norm) {
   pdl_start();
+  const double s = partials_sum(partials, nblk);
   if (threadIdx.x != 0) return;
-  double s = 0.0;
-  for (int b = 0; b < nblk; ++b) s += partials[b];
   const float nrm = (float)sqrt(s);
   scalars[S_NORM] = nrm;
   scalars[S_CLIP] = (nrm > max_norm) ? max_norm / (nrm + 1e-6f) : 1.0f;
@@ -769,13 +783,13 @@ void act_to_f32(float* out, const act_t* in, size_t n, cudaStream_t s) {
 void grad_norm_clip(float* scalars, const float* g, size_t n, float max_norm, double* partials,
                     cudaStream_t s) {
   launch_kernel(norm_partial_kernel, kNormBlocks, 256, 0, s, partials, g, n);
-  launch_kernel(norm_final_kernel, 1, 32, 0, s, scalars, partials, kNormBlocks, max_norm);
+  launch_kernel(norm_final_kernel, 1, 256, 0, s, scalars, partials, kNormBlocks, max_norm);
   note_launch(2);
 }
 
 void grad_sumsq(double* out, const float* g, size_t n, double* partials, cudaStream_t s) {
   launch_kernel(norm_partial_kernel, kNormBlocks, 256, 0, s, partials, g, n);
-  launch_kernel(sumsq_final_kernel, 1, 32, 0, s, out, partials, kNormBlocks);
+  launch_kernel(sumsq_final_kernel, 1, 256, 0, s, out, partials, kNormBlocks);
   note_launch(2);
 }
 
