@@ -364,12 +364,64 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
     uint32_t n_item = 0, gs = 0, gt = 0;
     bool ok = true;
+    // An item's dV and dK are read out of TMEM after the next item's first
+    // sub-tile has been handed to the products warp, which by then has
+    // finished the item's last products; the next item's products wait for
+    // the read-out (one accumulator pair).
+    struct PendingKV {
+      uint32_t n_item;
+      int b, h, j;
+      bool live;
+    };
+    PendingKV pend{0, 0, 0, 0, false};
+    auto read_out = [&](const PendingKV& it) {
+      // this thread's 64 / kKvSplit columns of each
+      if (!warp_and(mbar_wait(acc_full, it.n_item & 1u, abort_flag, err))) return false;
+      tc_fence_after();
+      constexpr int kAccCols = kHD / kKvSplit;
+      uint32_t rv[kAccCols], rk[kAccCols];
+      tc_ldn<kAccCols>(lane_base + kAccColKV + kAccCols * part, rv);
+      tc_ldn<kAccCols>(lane_base + kAccColKV + kHD + kAccCols * part, rk);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(acc_empty);
+      // this warp's 32 rows x kAccCols columns of dK and of dV into its two
+      // boxes, out by one TMA store each (rows past T are clipped)
+      constexpr int kRowBytes = kAccCols * 2;
+      uint8_t* box_k = sOut + (warp - 2) * kOutBoxKV;
+      uint8_t* box_v = box_k + 32 * kRowBytes;
+      if (lane == 0) bulk_wait_read<0>();  // the boxes' previous stores have read them
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < kAccCols; q += 8) {
+        uint4 wk, wv;
+        uint32_t* pk4 = reinterpret_cast<uint32_t*>(&wk);
+        uint32_t* pv4 = reinterpret_cast<uint32_t*>(&wv);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          pk4[e] = attn::pack_bf16x2(__uint_as_float(rk[q + 2 * e]) * scale,
+                                     __uint_as_float(rk[q + 2 * e + 1]) * scale);
+          pv4[e] = attn::pack_bf16x2(__uint_as_float(rv[q + 2 * e]),
+                                     __uint_as_float(rv[q + 2 * e + 1]));
+        }
+        *reinterpret_cast<uint4*>(box_k + lane * kRowBytes + q * 2) = wk;
+        *reinterpret_cast<uint4*>(box_v + lane * kRowBytes + q * 2) = wv;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int x0 = it.h * kHD + kAccCols * part, y0 = it.j * kTile + qw * 32;
+        tma_store_3d(&tmDKV, smem_u32(box_k), C + x0, y0, it.b);
+        tma_store_3d(&tmDKV, smem_u32(box_v), 2 * C + x0, y0, it.b);
+        bulk_commit();
+      }
+      return true;
+    };
     for (int k = 0; ok; ++k, ++n_item) {
       const int w = snake_item(k, items);
       if (w < 0) break;
       const int j = w / BH, bh = w % BH, b = bh / H, h = bh % H;
       const int n = nq - j;
-      const int kj = j * kTile + r;  // this thread's key row
       for (int t = 0; t < n && ok; ++t, ++gt) {
         const int st = gt % kQStages;
         const float* ldq = reinterpret_cast<const float*>(sLD + st * kPairBytes);
@@ -418,53 +470,17 @@ __global__ void __launch_bounds__(kThreadsKV, 1)
           attn::tc_wait_st();
           tc_fence_before();
           mbar_arrive(pd_full0 + 8 * sb);
-        }
-      }
-      if (!ok) break;
-      // the item's dV and dK: this thread's 64 / kKvSplit columns of each
-      ok = warp_and(mbar_wait(acc_full, n_item & 1u, abort_flag, err));
-      if (!ok) break;
-      tc_fence_after();
-      constexpr int kAccCols = kHD / kKvSplit;
-      uint32_t rv[kAccCols], rk[kAccCols];
-      tc_ldn<kAccCols>(lane_base + kAccColKV + kAccCols * part, rv);
-      tc_ldn<kAccCols>(lane_base + kAccColKV + kHD + kAccCols * part, rk);
-      tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive(acc_empty);
-      // this warp's 32 rows x kAccCols columns of dK and of dV into its two
-      // boxes, out by one TMA store each (rows past T are clipped)
-      {
-        constexpr int kRowBytes = kAccCols * 2;
-        uint8_t* box_k = sOut + (warp - 2) * kOutBoxKV;
-        uint8_t* box_v = box_k + 32 * kRowBytes;
-        if (lane == 0) bulk_wait_read<0>();  // the boxes' previous stores have read them
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < kAccCols; q += 8) {
-          uint4 wk, wv;
-          uint32_t* pk4 = reinterpret_cast<uint32_t*>(&wk);
-          uint32_t* pv4 = reinterpret_cast<uint32_t*>(&wv);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            pk4[e] = attn::pack_bf16x2(__uint_as_float(rk[q + 2 * e]) * scale,
-                                       __uint_as_float(rk[q + 2 * e + 1]) * scale);
-            pv4[e] = attn::pack_bf16x2(__uint_as_float(rv[q + 2 * e]),
-                                       __uint_as_float(rv[q + 2 * e + 1]));
+          if (pend.live) {  // the previous item's dV and dK, after this item's first sub-tile
+            ok = read_out(pend);
+            pend.live = false;
+            if (!ok) break;
           }
-          *reinterpret_cast<uint4*>(box_k + lane * kRowBytes + q * 2) = wk;
-          *reinterpret_cast<uint4*>(box_v + lane * kRowBytes + q * 2) = wv;
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          const int x0 = h * kHD + kAccCols * part, y0 = j * kTile + qw * 32;
-          tma_store_3d(&tmDKV, smem_u32(box_k), C + x0, y0, b);
-          tma_store_3d(&tmDKV, smem_u32(box_v), 2 * C + x0, y0, b);
-          bulk_commit();
         }
       }
+      if (!ok) break;
+      pend = PendingKV{n_item, b, h, j, true};
     }
+    if (ok && pend.live) ok = read_out(pend);
     if (lane == 0) bulk_wait_all();  // the dK / dV stores complete before the CTA leaves
   }
 
@@ -688,6 +704,51 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
       return qi < T ? lse[(size_t)(w % BH) * T + qi] : 0.f;
     };
     float lse_next = row_lse(0);
+    // An item's dQ is read out of its TMEM accumulator (there are two) after
+    // the first key tile of the next item, by when its last products have
+    // finished, so the compute warps do not wait for them at the item's end.
+    struct PendingDQ {
+      uint32_t n_item;
+      int b, h, i;
+      bool live;
+    };
+    PendingDQ pend{0, 0, 0, 0, false};
+    auto read_out = [&](const PendingDQ& it) {
+      const uint32_t ab = it.n_item & 1u, acc = kAccColQ + ab * kHD;
+      if (!warp_and(mbar_wait(acc_full0 + 8 * ab, (it.n_item >> 1) & 1u, abort_flag, err)))
+        return false;
+      tc_fence_after();
+      constexpr int kAccCols = kHD / kQSplit;
+      uint32_t rq[kAccCols];
+      tc_ldn<kAccCols>(lane_base + acc + kAccCols * part, rq);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(acc_empty0 + 8 * ab);
+      // this warp's 32 rows x kAccCols columns of dQ into its box, out by
+      // one TMA store (rows past T are clipped by the tensor map)
+      static_assert(kAccCols == 32, "one 64-byte box row per thread");
+      uint8_t* box = sOut + (warp - 2) * kOutBoxQ;
+      if (lane == 0) bulk_wait_read<0>();  // the box's previous store has read it
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < kAccCols; q += 8) {
+        uint4 w;
+        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          wp[e] = attn::pack_bf16x2(__uint_as_float(rq[q + 2 * e]) * scale,
+                                    __uint_as_float(rq[q + 2 * e + 1]) * scale);
+        *reinterpret_cast<uint4*>(box + lane * 64 + q * 2) = w;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(&tmDQ, smem_u32(box), it.h * kHD + kAccCols * part, it.i * kTile + qw * 32,
+                     it.b);
+        bulk_commit();
+      }
+      return true;
+    };
     for (int k = 0; ok; ++k, ++n_item) {
       const int w = snake_item(k, items);
       if (w < 0) break;
@@ -757,44 +818,16 @@ __global__ void __launch_bounds__(kThreadsQ, 1)
         attn::tc_wait_st();
         tc_fence_before();
         mbar_arrive(ds_full0 + 8 * db);
-      }
-      if (!ok) break;
-      const uint32_t ab = n_item & 1u, acc = kAccColQ + ab * kHD;
-      ok = warp_and(mbar_wait(acc_full0 + 8 * ab, (n_item >> 1) & 1u, abort_flag, err));
-      if (!ok) break;
-      tc_fence_after();
-      constexpr int kAccCols = kHD / kQSplit;
-      uint32_t rq[kAccCols];
-      tc_ldn<kAccCols>(lane_base + acc + kAccCols * part, rq);
-      tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive(acc_empty0 + 8 * ab);
-      // this warp's 32 rows x kAccCols columns of dQ into its box, out by
-      // one TMA store (rows past T are clipped by the tensor map)
-      {
-        static_assert(kAccCols == 32, "one 64-byte box row per thread");
-        uint8_t* box = sOut + (warp - 2) * kOutBoxQ;
-        if (lane == 0) bulk_wait_read<0>();  // the box's previous store has read it
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < kAccCols; q += 8) {
-          uint4 w;
-          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            wp[e] = attn::pack_bf16x2(__uint_as_float(rq[q + 2 * e]) * scale,
-                                      __uint_as_float(rq[q + 2 * e + 1]) * scale);
-          *reinterpret_cast<uint4*>(box + lane * 64 + q * 2) = w;
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_3d(&tmDQ, smem_u32(box), h * kHD + kAccCols * part, i * kTile + qw * 32, b);
-          bulk_commit();
+        if (jj == 0 && pend.live) {  // the previous item's dQ
+          ok = read_out(pend);
+          pend.live = false;
         }
       }
+      if (!ok) break;
+      pend = PendingDQ{n_item, b, h, i, true};
       gk += n;
     }
+    if (ok && pend.live) ok = read_out(pend);
     if (lane == 0) bulk_wait_all();  // the dQ stores complete before the CTA leaves
   }
 
