@@ -55,7 +55,15 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int kThreads = 64 + kEpiThreads;
+// The GELU backward on CTA pairs sums its output's columns (the W_fc bias
+// gradient) in a warp of its own after the epilogue warps, fed box by box
+// (in a pair the epilogue sets the pace, and the sums would add a third to
+// its instructions); on single CTAs the epilogue warps sum their own boxes.
+constexpr bool sums_warp(int epi, int cg) { return epi == EPI_DGELU && cg == 2; }
+constexpr int kSumsWarps = 2;  // each sums the boxes of half the epilogue warps
+constexpr int kernel_threads(int epi, int cg) {
+  return 64 + kEpiThreads + (sums_warp(epi, cg) ? 32 * kSumsWarps : 0);
+}
 constexpr int kWarpBox = 4096;  // one warp's epilogue box: 32 rows x 128 bytes
 
 // Epilogues that read a second [M, N] input (residual or pre-activation).
@@ -91,11 +99,11 @@ constexpr uint32_t tmem_cols() {
 template <int BN, int EPI, int CG>
 constexpr size_t smem_bytes() {
   return 1024 + (size_t)ring_stages(BN, EPI, CG) * (BM * BK * 2 + (BN / CG) * BK * 2) +
-         (size_t)kEpiWarps * epi_boxes(EPI) * kWarpBox + 256;
+         (size_t)kEpiWarps * epi_boxes(EPI) * kWarpBox + 256 + (sums_warp(EPI, CG) ? 128 : 0);
 }
 
 template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI, int CG>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kernel_threads(EPI, CG), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmOut,
                    const __grid_constant__ CUtensorMap tmX, const EpiParams ep, int K,
@@ -105,6 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = tmem_cols<BN>();
   constexpr bool HAS_IN = epi_has_input(EPI);
+  constexpr bool SW = sums_warp(EPI, CG);
   static_assert(STAGES == ring_stages(BN, EPI, CG), "ring depth");
   static_assert(CG == 1 || (CG == 2 && BN == 256), "CTA pairs use 256 x 256 tiles");
   // CTA pair: rank 0 (the leader) issues the MMAs for both CTAs; each CTA
@@ -124,7 +133,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NBOX = epi_boxes(EPI);
   uint8_t* sBox = smem + STAGES * (A_BYTES + B_BYTES);  // [kEpiWarps][NBOX] boxes, 1024-aligned
   uint64_t* bars = reinterpret_cast<uint64_t*>(sBox + kEpiWarps * NBOX * kWarpBox);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4 + kEpiWarps);
+  uint32_t* tmem_slot =
+      reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4 + kEpiWarps + (SW ? 2 * kEpiWarps : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t full0 = smem_u32(bars);
@@ -132,6 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
   const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
   const uint32_t in_full0 = smem_u32(bars + 2 * STAGES + 4);  // [kEpiWarps]
+  // sums warp: an epilogue warp's output box holds a group / has been summed
+  const uint32_t cs_full0 = smem_u32(bars + 2 * STAGES + 4 + kEpiWarps);       // [kEpiWarps]
+  const uint32_t cs_empty0 = smem_u32(bars + 2 * STAGES + 4 + 2 * kEpiWarps);  // [kEpiWarps]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -150,6 +163,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(tempty0 + 8 * b, CG * kEpiWarps);  // one arrival per epilogue warp of the pair
     }
     for (int w = 0; w < kEpiWarps; ++w) mbar_init(in_full0 + 8 * w, 1);
+    if (SW)
+      for (int w = 0; w < kEpiWarps; ++w) {
+        mbar_init(cs_full0 + 8 * w, 32);
+        mbar_init(cs_empty0 + 8 * w, 32);
+      }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -333,6 +351,74 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+  } else if (SW && warp >= 2 + kEpiWarps) {
+    // -------------------------------------------------------------- sums --
+    // Sums warp sw takes the epilogue warps whose groups are sw, sw + 2 of
+    // each tile, in their order (each warp's k-th group, warp by warp).
+    // Once a warp's output box holds a group, lane l reads 16-byte chunk
+    // l % 8 (8 columns) of rows l / 8 + 4i, i = 0..7, adds them in row order,
+    // the four lanes of a chunk are added pairwise (rows r, r + 1, then
+    // r + 2), and lanes 0-7 write the group's 64 column sums into its slab of
+    // ep.colsum; then the box goes back to its warp.
+    if (ep.colsum) {
+      const int sw = warp - 2 - kEpiWarps;
+      uint32_t gcw[kEpiWarps / kSumsWarps];
+#pragma unroll
+      for (int i = 0; i < kEpiWarps / kSumsWarps; ++i) gcw[i] = 0;
+      bool ok = true;
+      const int ch = lane & 7, r0l = lane >> 3;  // this lane's chunk and first row
+      for (int u = unit0; u < units && ok; u += unit_step) {
+        int tm, tn, kb0, kb1, sp;
+        decode(u, tm, tn, kb0, kb1, sp);
+        const int m0 = tm * BM * CG + (int)rank * BM, nt0 = tn * BN;
+        const int ngroups = (min(BN, ep.N - nt0) + 63) >> 6;
+        for (int k = 0; k < 2 && ok; ++k) {
+#pragma unroll
+          for (int i = 0; i < kEpiWarps / kSumsWarps; ++i) {
+            const int w = sw * (kEpiWarps / kSumsWarps) + i;  // epilogue warp w + 2
+            const int g = (w >> 2) + 2 * k;                    // its k-th group
+            const int r0 = m0 + ((w + 2) & 3) * 32;            // and its slab
+            if (!ok || g >= ngroups || r0 >= ep.M) continue;
+            ok = __all_sync(0xffffffffu, mbar_wait(cs_full0 + 8 * w, gcw[i] & 1u, abort_flag, err));
+            if (!ok) continue;
+            const uint8_t* box = sBox + w * NBOX * kWarpBox;  // the warp's output box
+            const int rows = min(32, ep.M - r0);
+            float2 cs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                            make_float2(0.f, 0.f)};
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+              const int row = r0l + 4 * rr;
+              if (row < rows) {
+                const uint4 v = *reinterpret_cast<const uint4*>(box + swz(row, ch));
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  cs[e] = f2_add(cs[e], make_float2(__uint_as_float(wv[e] << 16),
+                                                    __uint_as_float(wv[e] & 0xffff0000u)));
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              cs[e].x += __shfl_xor_sync(0xffffffffu, cs[e].x, 8);
+              cs[e].y += __shfl_xor_sync(0xffffffffu, cs[e].y, 8);
+              cs[e].x += __shfl_xor_sync(0xffffffffu, cs[e].x, 16);
+              cs[e].y += __shfl_xor_sync(0xffffffffu, cs[e].y, 16);
+            }
+            const int col = nt0 + 64 * g + 8 * ch;
+            if (lane < 8) {
+              float* dst = ep.colsum + (size_t)(r0 >> 5) * ep.N + col;
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (col + 2 * e < ep.N)  // N even: both columns of a pair in range
+                  *reinterpret_cast<float2*>(dst + 2 * e) = cs[e];
+            }
+            __syncwarp();
+            mbar_arrive(cs_empty0 + 8 * w);
+            ++gcw[i];
+          }
+        }
+      }
+    }
   } else {
     // ---------------------------------------------------------- epilogue --
     const int q = warp & 3;          // TMEM lane quarter this warp may access
@@ -389,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t gc = 0;  // groups this warp has handed to the sums warp
     bool ok = true;
     for (int u = unit0; u < units && ok; u += unit_step) {
       int tm, tn, kb0, kb1, sp;
@@ -535,13 +622,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 64; i += 2) set2(v, i, gelu_tanh2(get2(v, i)));
           }
+          if (SW && ep.colsum) {  // the sums warp has read the box's previous group
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(cs_empty0 + 8 * (warp - 2), (gc & 1u) ^ 1u, abort_flag, err));
+            if (!ok) break;
+          }
           put_box(
               [&](uint8_t* box) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(box + swz(lane, j)), v + 8 * j);
               },
               [&](uint32_t box_u) { tma_store_3d(&tmOut, box_u, nb, r0, 0); });
-          if (EPI == EPI_DGELU && ep.colsum) {
+          if (SW && ep.colsum) {
+            mbar_arrive(cs_full0 + 8 * (warp - 2));  // the box holds this group
+            ++gc;
+          } else if (EPI == EPI_DGELU && ep.colsum) {
             // column sums of the stored slab: lane l adds columns 2l, 2l + 1
             // of the box's rows in order (the TMA store reads the same box;
             // the next group's writes wait for both)
@@ -672,7 +767,7 @@ static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CU
   const int slots = num_sms() / CG;  // persistent CTAs (pairs)
   const int grid = CG * (units < slots ? units : slots);
   // a pair is a cluster of two CTAs along x
-  const cudaError_t e = launch_kernel_cluster(kern, dim3(grid), dim3(kThreads), smem, s, CG, ta, tb,
+  const cudaError_t e = launch_kernel_cluster(kern, dim3(grid), dim3(kernel_threads(EPI, CG)), smem, s, CG, ta, tb,
                                               to, tx, ep, K, tiles_m, tiles_n, splits, kb_per_split,
                                               n_fast, err);
   if (e != cudaSuccess) return e;
@@ -686,7 +781,6 @@ static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUte
                             int epi, int splits, int kb_per_split, int n_fast, cudaStream_t s,
                             int* err) {
 #define GPT2_TC(AM, BMJ, E)                                                                      \
-  if constexpr (CG == 1 || E != EPI_DGELU)                                                       \
     if (a.a_mn == AM && a.b_mn == BMJ && epi == E)                                               \
       return launch<BN, AM, BMJ, E, CG>(ta, tb, to, tx, ep, a.K, splits, kb_per_split, n_fast, s, err);
   GPT2_TC(0, 0, EPI_STORE)
@@ -789,7 +883,7 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   // forward, at M = 16384, N = 3072, K = 768, once the accumulator release
   // became a relaxed arrival).  The GELU backward keeps single CTAs: with
   // its fused column sums it measured 85 us in pairs against 82 us.
-  const int CG = (g_cta_pairs && BN == 256 && a.M > BM && a.epi != EPI_DGELU) ? 2 : 1;
+  const int CG = (g_cta_pairs && BN == 256 && a.M > BM) ? 2 : 1;
   const int slots = num_sms() / CG;  // persistent CTAs or pairs
   const int tiles = ((a.M + BM * CG - 1) / (BM * CG)) * ((a.N + BN - 1) / BN);
   const int kb_total = (a.K + BK - 1) / BK;
