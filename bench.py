@@ -45,8 +45,8 @@ SPEC_BF16_DENSE = 2.25e15
 # dram__bytes_write.sum, weighted by its launches per step
 # (profiles/gemm_tc_dram_traffic_gpt2_124m_step.md).  Valid only for the GEMM
 # sources it was taken on: reported as null as soon as their hash differs.
-GEMM_TRAFFIC = {"bytes_per_launch": 1.4474e8,
-                "sources_sha256": "1950c819e809f7ac763b46aca09ff7d0b72601ac95a0e75d9e3340ee88d5b884"}
+GEMM_TRAFFIC = {"bytes_per_launch": 1.6110e8,
+                "sources_sha256": "cd62971bde99c52b228bceb93b3b1960d24e535520c1756bfeb342452fa0cfdb"}
 GEMM_SOURCES = ("gemm_tc.cu", "gemm_epi.cuh", "tc_util.cuh")
 
 
