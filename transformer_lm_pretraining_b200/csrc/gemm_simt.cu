@@ -83,7 +83,7 @@ __global__ void splitk_reduce_kernel(float* out32, long ldo32, const float* ws, 
   }
 }
 
-int gemm_set_cta_pairs(int) { return 0; }  // no CTA pairs in this build
+int gemm_set_cta_pairs(int) { return 0; }  // the fp32 validation library has no CTA pairs
 bool gemm_colsum_supported() { return false; }  // the column sums run as their own pass
 
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
