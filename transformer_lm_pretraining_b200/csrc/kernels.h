@@ -136,6 +136,10 @@ constexpr int kColsumChunks = 192;
 // db[n] += sum_m dy[m, n] (fixed order); partials: [kColsumChunks * N] floats
 void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s,
                 ReduceJob* defer = nullptr);
+// As colsum_acc (N % 8 == 0, 16-byte aligned rows), with a kernel small
+// enough to run beside a GEMM on another stream; partials: [kColsumChunks * N].
+void colsum_acc_lite(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s,
+                     ReduceJob* defer = nullptr);
 // db[n] += sum over c < chunks of partials[c * N + n], c ascending (the
 // second stage of colsum_acc, for partials a GEMM epilogue wrote)
 void colsum_reduce(float* db, const float* partials, int chunks, int N, cudaStream_t s,
