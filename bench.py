@@ -44,7 +44,8 @@ SPEC_BF16_DENSE = 2.25e15
 # at full size, one launch, with ncu's dram__bytes_read.sum +
 # dram__bytes_write.sum, weighted by its launches per step
 # (profiles/gemm_tc_dram_traffic_gpt2_124m_step.md).  Valid only for the GEMM
-# sources it was taken on: reported as null as soon as their hash differs.
+# sources it was taken on: reported as null as soon as their hash differs
+# (as now: the weight gradients of W_qkv and W_o share one launch since).
 GEMM_TRAFFIC = {"bytes_per_launch": 1.6110e8,
                 "sources_sha256": "cd62971bde99c52b228bceb93b3b1960d24e535520c1756bfeb342452fa0cfdb"}
 GEMM_SOURCES = ("gemm_tc.cu", "gemm_epi.cuh", "tc_util.cuh")

@@ -87,6 +87,13 @@ int gemm_set_cta_pairs(int) { return 0; }  // the fp32 validation library has no
 bool gemm_colsum_supported() { return false; }  // the column sums run as their own pass
 
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
+  if (a.M2 > 0) {  // the stacked second product: one launch after the other
+    GemmArgs first = a;
+    first.M2 = 0;
+    const cudaError_t e = gemm(first, s, err);
+    if (e != cudaSuccess) return e;
+    return gemm(gemm_second(a), s, err);
+  }
   (void)err;
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return cudaSuccess;
   EpiParams ep{a.M, a.N, a.alpha, a.out, a.ldo, a.out32, a.ldo32, a.bias, a.resid, a.ldr, a.aux, a.ldaux};

@@ -106,8 +106,11 @@ template <int BN, int STAGES, bool A_MN, bool B_MN, int EPI, int CG>
 __global__ void __launch_bounds__(kernel_threads(EPI, CG), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmOut,
-                   const __grid_constant__ CUtensorMap tmX, const EpiParams ep, int K,
-                   int tiles_m, int tiles_n, int splits, int kb_per_split, int n_fast, int* err) {
+                   const __grid_constant__ CUtensorMap tmX,
+                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                   const __grid_constant__ CUtensorMap tmOut2, const EpiParams ep, int K,
+                   int tiles_m, int tiles_n, int splits, int kb_per_split, int n_fast, int tiles_m1,
+                   int M2, int* err) {
   constexpr int A_BYTES = BM * BK * 2;
   constexpr int B_BYTES = (BN / CG) * BK * 2;  // this CTA's rows of the B tile
   constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
@@ -218,7 +221,11 @@ __global__ void __launch_bounds__(kernel_threads(EPI, CG), 1)
       for (int u = unit0; u < units && ok; u += unit_step) {
         int tm, tn, kb0, kb1, sp;
         decode(u, tm, tn, kb0, kb1, sp);
-        const int am = tm * BM * CG + (int)rank * BM;          // this CTA's rows of A
+        // row tiles from tiles_m1 on belong to the second product
+        const bool p2 = tm >= tiles_m1;
+        const CUtensorMap* mA = p2 ? &tmA2 : &tmA;
+        const CUtensorMap* mB = p2 ? &tmB2 : &tmB;
+        const int am = (p2 ? tm - tiles_m1 : tm) * BM * CG + (int)rank * BM;  // this CTA's rows of A
         const int bn0 = tn * BN + (int)rank * (BN / CG);       // and of B
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, err)) {
@@ -239,16 +246,16 @@ __global__ void __launch_bounds__(kernel_threads(EPI, CG), 1)
           if (CG == 1) {
             mbar_expect_tx(fb, STAGE_TX);
             if (!A_MN) {
-              tma_load_2d(a_dst, &tmA, fb, kb * BK, am);
+              tma_load_2d(a_dst, mA, fb, kb * BK, am);
             } else {
-              tma_load_2d(a_dst, &tmA, fb, am, kb * BK);
-              tma_load_2d(a_dst + 8192, &tmA, fb, am + 64, kb * BK);
+              tma_load_2d(a_dst, mA, fb, am, kb * BK);
+              tma_load_2d(a_dst + 8192, mA, fb, am + 64, kb * BK);
             }
             if (!B_MN) {
-              tma_load_2d(b_dst, &tmB, fb, kb * BK, bn0);
+              tma_load_2d(b_dst, mB, fb, kb * BK, bn0);
             } else {
 #pragma unroll
-              for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + 8192 * j, &tmB, fb, bn0 + 64 * j, kb * BK);
+              for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + 8192 * j, mB, fb, bn0 + 64 * j, kb * BK);
             }
           } else {
             // both CTAs' copies complete on the leader's full barrier, which
@@ -256,17 +263,17 @@ __global__ void __launch_bounds__(kernel_threads(EPI, CG), 1)
             if (leader) mbar_expect_tx(fb, CG * STAGE_TX);
             const uint32_t lfb = map_shared(fb, 0);
             if (!A_MN) {
-              tma_load_2d_pair(a_dst, &tmA, lfb, kb * BK, am);
+              tma_load_2d_pair(a_dst, mA, lfb, kb * BK, am);
             } else {
-              tma_load_2d_pair(a_dst, &tmA, lfb, am, kb * BK);
-              tma_load_2d_pair(a_dst + 8192, &tmA, lfb, am + 64, kb * BK);
+              tma_load_2d_pair(a_dst, mA, lfb, am, kb * BK);
+              tma_load_2d_pair(a_dst + 8192, mA, lfb, am + 64, kb * BK);
             }
             if (!B_MN) {
-              tma_load_2d_pair(b_dst, &tmB, lfb, kb * BK, bn0);
+              tma_load_2d_pair(b_dst, mB, lfb, kb * BK, bn0);
             } else {
 #pragma unroll
               for (int j = 0; j < BN / CG / 64; ++j)
-                tma_load_2d_pair(b_dst + 8192 * j, &tmB, lfb, bn0 + 64 * j, kb * BK);
+                tma_load_2d_pair(b_dst + 8192 * j, mB, lfb, bn0 + 64 * j, kb * BK);
             }
           }
           issued_mask |= 1u << stage;
@@ -480,7 +487,10 @@ __global__ void __launch_bounds__(kernel_threads(EPI, CG), 1)
     for (int u = unit0; u < units && ok; u += unit_step) {
       int tm, tn, kb0, kb1, sp;
       decode(u, tm, tn, kb0, kb1, sp);
-      const int m0 = tm * BM * CG + (int)rank * BM, nt0 = tn * BN;
+      const bool p2 = tm >= tiles_m1;  // a tile of the second product
+      const CUtensorMap* mOut = p2 ? &tmOut2 : &tmOut;
+      const int mlim = p2 ? M2 : ep.M;
+      const int m0 = (p2 ? tm - tiles_m1 : tm) * BM * CG + (int)rank * BM, nt0 = tn * BN;
       const int r0 = m0 + q * 32;  // first row of this warp's slab
       const int ngroups = (min(BN, ep.N - nt0) + 63) >> 6;  // 64-column groups in range
       ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, err));
@@ -491,7 +501,7 @@ __global__ void __launch_bounds__(kernel_threads(EPI, CG), 1)
 #pragma unroll 1
       for (int g = h; g < ngroups; g += 2) {
         const int nb = nt0 + 64 * g;  // first column of the group
-        const bool live = r0 < ep.M;  // rows of this slab exist
+        const bool live = r0 < mlim;  // rows of this slab exist
         if (HAS_IN && live && !pre && lane == 0) {
           // the group's input slab, ahead of the accumulator read (a shared
           // box is free once the previous store has read it)
@@ -592,8 +602,8 @@ __global__ void __launch_bounds__(kernel_threads(EPI, CG), 1)
                                     v[32 * half + 4 * j + 2], v[32 * half + 4 * j + 3]);
                 },
                 [&](uint32_t box_u) {
-                  if (EPI == EPI_F32_ACC) tma_reduce_add_3d(&tmOut, box_u, nb + 32 * half, r0, 0);
-                  else tma_store_3d(&tmOut, box_u, nb + 32 * half, r0, sp);
+                  if (EPI == EPI_F32_ACC) tma_reduce_add_3d(mOut, box_u, nb + 32 * half, r0, 0);
+                  else tma_store_3d(mOut, box_u, nb + 32 * half, r0, sp);
                 });
           }
         } else {
@@ -632,7 +642,7 @@ __global__ void __launch_bounds__(kernel_threads(EPI, CG), 1)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) store8(reinterpret_cast<act_t*>(box + swz(lane, j)), v + 8 * j);
               },
-              [&](uint32_t box_u) { tma_store_3d(&tmOut, box_u, nb, r0, 0); });
+              [&](uint32_t box_u) { tma_store_3d(mOut, box_u, nb, r0, 0); });
           if (SW && ep.colsum) {
             mbar_arrive(cs_full0 + 8 * (warp - 2));  // the box holds this group
             ++gc;
@@ -750,7 +760,8 @@ static int num_sms() {
 
 template <int BN, bool A_MN, bool B_MN, int EPI, int CG>
 static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                          const CUtensorMap& tx, const EpiParams& ep, int K, int splits,
+                          const CUtensorMap& tx, const CUtensorMap& ta2, const CUtensorMap& tb2,
+                          const CUtensorMap& to2, int M2, const EpiParams& ep, int K, int splits,
                           int kb_per_split, int n_fast, cudaStream_t s, int* err) {
   auto kern = gemm_tc_kernel<BN, ring_stages(BN, EPI, CG), A_MN, B_MN, EPI, CG>;
   constexpr size_t smem = smem_bytes<BN, EPI, CG>();
@@ -761,15 +772,16 @@ static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CU
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  const int tiles_m = (ep.M + BM * CG - 1) / (BM * CG);
+  const int tiles_m1 = (ep.M + BM * CG - 1) / (BM * CG);
+  const int tiles_m = tiles_m1 + (M2 + BM * CG - 1) / (BM * CG);
   const int tiles_n = (ep.N + BN - 1) / BN;
   const int units = tiles_m * tiles_n * splits;
   const int slots = num_sms() / CG;  // persistent CTAs (pairs)
   const int grid = CG * (units < slots ? units : slots);
   // a pair is a cluster of two CTAs along x
   const cudaError_t e = launch_kernel_cluster(kern, dim3(grid), dim3(kernel_threads(EPI, CG)), smem, s, CG, ta, tb,
-                                              to, tx, ep, K, tiles_m, tiles_n, splits, kb_per_split,
-                                              n_fast, err);
+                                              to, tx, ta2, tb2, to2, ep, K, tiles_m, tiles_n, splits,
+                                              kb_per_split, n_fast, tiles_m1, M2, err);
   if (e != cudaSuccess) return e;
   note_launch();
   return cudaGetLastError();
@@ -777,12 +789,14 @@ static cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CU
 
 template <int BN, int CG>
 static cudaError_t dispatch(const GemmArgs& a, const CUtensorMap& ta, const CUtensorMap& tb,
-                            const CUtensorMap& to, const CUtensorMap& tx, const EpiParams& ep,
-                            int epi, int splits, int kb_per_split, int n_fast, cudaStream_t s,
-                            int* err) {
+                            const CUtensorMap& to, const CUtensorMap& tx, const CUtensorMap& ta2,
+                            const CUtensorMap& tb2, const CUtensorMap& to2, int M2,
+                            const EpiParams& ep, int epi, int splits, int kb_per_split, int n_fast,
+                            cudaStream_t s, int* err) {
 #define GPT2_TC(AM, BMJ, E)                                                                      \
     if (a.a_mn == AM && a.b_mn == BMJ && epi == E)                                               \
-      return launch<BN, AM, BMJ, E, CG>(ta, tb, to, tx, ep, a.K, splits, kb_per_split, n_fast, s, err);
+      return launch<BN, AM, BMJ, E, CG>(ta, tb, to, tx, ta2, tb2, to2, M2, ep, a.K, splits,      \
+                                        kb_per_split, n_fast, s, err);
   GPT2_TC(0, 0, EPI_STORE)
   GPT2_TC(0, 0, EPI_BIAS)
   GPT2_TC(0, 0, EPI_BIAS_GELU)
@@ -852,9 +866,31 @@ int gemm_set_cta_pairs(int enable) {
   return prev;
 }
 
+// The product and the one stacked under it, one launch each.
+static cudaError_t gemm_in_turn(const GemmArgs& a, cudaStream_t s, int* err) {
+  GemmArgs first = a;
+  first.M2 = 0;
+  const cudaError_t e = gemm(first, s, err);
+  if (e != cudaSuccess) return e;
+  return gemm(gemm_second(a), s, err);
+}
+
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   using namespace tc;
+  if (a.M2 > 0 && (a.M <= 0 || a.N <= 0 || a.K <= 0)) return gemm(gemm_second(a), s, err);
   if (a.M <= 0 || a.N <= 0 || a.K <= 0) return cudaSuccess;
+  // A second product stacked under this one (same N and K, fp32 accumulate)
+  // shares the launch when both are whole 256-row pair tiles and the split
+  // plan needs no partials; otherwise the two run one after the other.
+  const bool grouped = a.M2 > 0;
+  if (grouped) {
+    const bool can = a.epi == EPI_F32_ACC && g_cta_pairs && a.N >= 256 && a.a_mn && a.b_mn &&
+                     a.M % (2 * BM) == 0 && a.M2 % (2 * BM) == 0 && aligned16(a.A2) &&
+                     aligned16(a.B2) && a.out32_2 && aligned16(a.out32_2) && a.lda2 % 8 == 0 &&
+                     a.ldb2 % 8 == 0 && a.ldo32_2 % 4 == 0;
+    if (!can) return gemm_in_turn(a, s, err);
+  }
+  const int Mt = a.M + (grouped ? a.M2 : 0);  // rows of both products
   // TMA: 16-byte aligned bases and row strides for every operand and output
   if (!aligned16(a.A) || !aligned16(a.B) || (a.lda % 8) || (a.ldb % 8)) return cudaErrorInvalidValue;
   const bool f32_out = a.epi == EPI_F32_ACC || a.epi == EPI_F32_STORE;
@@ -885,7 +921,7 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   // its fused column sums it measured 85 us in pairs against 82 us.
   const int CG = (g_cta_pairs && BN == 256 && a.M > BM) ? 2 : 1;
   const int slots = num_sms() / CG;  // persistent CTAs or pairs
-  const int tiles = ((a.M + BM * CG - 1) / (BM * CG)) * ((a.N + BN - 1) / BN);
+  const int tiles = ((Mt + BM * CG - 1) / (BM * CG)) * ((a.N + BN - 1) / BN);
   const int kb_total = (a.K + BK - 1) / BK;
 
   // split-K for the weight-gradient products with few output tiles: pick the
@@ -899,9 +935,9 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   if (a.epi == EPI_F32_ACC && a.max_splits > 1 && a.split_ws && tiles < slots &&
       aligned16(a.split_ws) && a.N % 4 == 0) {
     double best = 1e30;
-    const double out_bytes = 4.0 * a.M * a.N;
+    const double out_bytes = 4.0 * Mt * a.N;
     for (int sp = 1; sp <= a.max_splits; ++sp) {
-      if (sp > 1 && (sp > kb_total / 4 || (size_t)sp * a.M * a.N > a.split_ws_floats)) break;
+      if (sp > 1 && (sp > kb_total / 4 || (size_t)sp * Mt * a.N > a.split_ws_floats)) break;
       const int waves = (tiles * sp + slots - 1) / slots;
       const double t_unit = 2.0 * BM * BN * ((double)kb_total * BK / sp) / 8.5e12;
       const double t_red = sp == 1 ? 0.0
@@ -928,6 +964,7 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   int kb_per_split = (kb_total + splits - 1) / splits;
   splits = (kb_total + kb_per_split - 1) / kb_per_split;  // no empty split
   const bool in_place = splits == 2 && a.acc_zero;  // both halves reduce-add into out32
+  if (grouped && splits > 1 && !in_place) return gemm_in_turn(a, s, err);
   if (!a.b_mn) e = make_tmap(&tb, a.B, false, a.K, a.N, a.ldb, 64, BN / CG);
   else e = make_tmap(&tb, a.B, false, a.N, a.K, a.ldb, 64, 64);
   if (e != cudaSuccess) return e;
@@ -946,15 +983,24 @@ cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err) {
   else if (a.epi == EPI_BIAS_GELU || a.epi == EPI_DGELU)
     e = make_tmap(&tx, a.aux, false, a.N, a.M, a.ldaux, 64, 32, 1);
   if (e != cudaSuccess) return e;
+  // the second product's operands and output (both operands MN-major)
+  CUtensorMap ta2 = ta, tb2 = tb, to2 = to;
+  if (grouped) {
+    e = make_tmap(&ta2, a.A2, false, a.M2, a.K, a.lda2, 64, 64);
+    if (e == cudaSuccess) e = make_tmap(&tb2, a.B2, false, a.N, a.K, a.ldb2, 64, 64);
+    if (e == cudaSuccess) e = make_tmap(&to2, a.out32_2, true, a.N, a.M2, a.ldo32_2, 32, 32, 1);
+    if (e != cudaSuccess) return e;
+  }
+  const int M2 = grouped ? a.M2 : 0;
   // The larger operand is reused by consecutive tiles (L2 locality).
-  const double a_bytes = (double)a.M * a.K, b_bytes = (double)a.N * a.K;
+  const double a_bytes = (double)Mt * a.K, b_bytes = (double)a.N * a.K;
   const int n_fast = a_bytes > b_bytes ? 1 : 0;
   if (CG == 2)
-    e = dispatch<256, 2>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
+    e = dispatch<256, 2>(a, ta, tb, to, tx, ta2, tb2, to2, M2, ep, epi, splits, kb_per_split, n_fast, s, err);
   else if (BN == 256)
-    e = dispatch<256, 1>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
+    e = dispatch<256, 1>(a, ta, tb, to, tx, ta2, tb2, to2, M2, ep, epi, splits, kb_per_split, n_fast, s, err);
   else
-    e = dispatch<128, 1>(a, ta, tb, to, tx, ep, epi, splits, kb_per_split, n_fast, s, err);
+    e = dispatch<128, 1>(a, ta, tb, to, tx, ta2, tb2, to2, M2, ep, epi, splits, kb_per_split, n_fast, s, err);
   if (e != cudaSuccess) return e;
   if (splits > 1 && small_m) {
     const size_t total = (size_t)a.M * a.N;

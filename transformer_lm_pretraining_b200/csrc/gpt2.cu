@@ -105,11 +105,6 @@ struct gpt2 {
   // events recorded after each layer's backward (and the last one after the
   // embedding's), for callers overlapping gradient communication
   std::vector<cudaEvent_t> bwd_events;
-  // a second, low-priority stream for work that can run beside the
-  // backward's products (the W_qkv bias column sums), forked from and joined
-  // back into the handle's stream by two events
-  cudaStream_t side = nullptr;
-  cudaEvent_t side_fork = nullptr, side_join = nullptr;
   // a captured optimizer step (gpt2_step_graph_capture)
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t graph_exec = nullptr;
@@ -286,7 +281,7 @@ void mark_end(gpt2_t* h) {
 }
 
 gpt2_status run_gemm(gpt2_t* h, const GemmArgs& ga) {
-  mark(h, PK_GEMM, 2.0 * ga.M * ga.N * ga.K);
+  mark(h, PK_GEMM, 2.0 * (ga.M + ga.M2) * ga.N * ga.K);
   GPT2_CUDA(h, gemm(ga, h->stream, h->err));
   return GPT2_OK;
 }
@@ -332,9 +327,6 @@ void gpt2_destroy(gpt2_t* h) {
   if (h->gen) cudaFree(h->gen);
   if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
   if (h->graph) cudaGraphDestroy(h->graph);
-  if (h->side_fork) cudaEventDestroy(h->side_fork);
-  if (h->side_join) cudaEventDestroy(h->side_join);
-  if (h->side) cudaStreamDestroy(h->side);
   std::vector<cudaEvent_t> evs = h->ev_pool;
   for (const ProfRec& r : h->recs) {
     evs.push_back(r.a);
@@ -751,35 +743,6 @@ gpt2_status gpt2_zero_grad(gpt2_t* h) {
   return GPT2_OK;
 }
 
-}  // extern "C"
-
-namespace {
-
-// The handle's second stream and its two events (created on first use);
-// false when they cannot be made, and the work stays on the main stream.
-bool ensure_side(gpt2_t* h) {
-  if (h->side) return true;
-  int lo = 0, hi = 0;
-  if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return false;
-  cudaStream_t st = nullptr;
-  if (cudaStreamCreateWithPriority(&st, cudaStreamNonBlocking, lo) != cudaSuccess) return false;
-  cudaEvent_t a = nullptr, b = nullptr;
-  if (cudaEventCreateWithFlags(&a, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&b, cudaEventDisableTiming) != cudaSuccess) {
-    if (a) cudaEventDestroy(a);
-    cudaStreamDestroy(st);
-    return false;
-  }
-  h->side = st;
-  h->side_fork = a;
-  h->side_join = b;
-  return true;
-}
-
-}  // namespace
-
-extern "C" {
-
 gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
   if (!h) return GPT2_ERR_ARG;
   if (!h->have_grad_logits)
@@ -812,32 +775,15 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
     dused += n;
     return p;
   };
-  // With deferred reductions, the W_qkv bias column sums of each layer run on
-  // the second stream beside the products that follow the attention
-  // backward (their kernel fits next to a GEMM CTA on an SM); the main
-  // stream waits for them before dqkv is overwritten and before the
-  // reductions run.
-  const bool use_side = defer && ensure_side(h);
-  bool side_pending = false;
-  auto join_side = [&]() -> gpt2_status {
-    if (side_pending) {
-      GPT2_CUDA(h, cudaStreamWaitEvent(s, h->side_join, 0));
-      side_pending = false;
-    }
-    return GPT2_OK;
-  };
-  auto queue = [&]() -> gpt2_status {
-    if (!defer) return GPT2_OK;
+  auto queue = [&]() {
+    if (!defer) return;
     if (!reduce_jobs_add(jobs, job)) {  // the list is full: run it first
-      GPT2_TRY(join_side());  // (its column-sum partials complete)
       reduce_jobs_run(jobs, s);
       reduce_jobs_add(jobs, job);
     }
-    return GPT2_OK;
   };
   const size_t ln_part = (size_t)kLnBlocks * 3 * C;
   ReduceJob* dj = defer ? &job : nullptr;
-
 
   {  // dhf = scale * dz wte  (dz: the logits buffer)
     GemmArgs ga = gemm_args(M, C, y.Vp);
@@ -862,7 +808,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
   layernorm_bwd(a.dres, a.dh, a.res + (size_t)L * MC, a.meanf, a.rstdf, P + y.off[T_LNFG],
                 G + y.off[T_LNFG], G + y.off[T_LNFB], G + y.off[T_BP] + (size_t)(L - 1) * C,
                 slice(ln_part, a.partials), M, C, 0, s, dj);
-  GPT2_TRY(queue());
+  queue();
 
   for (int l = L - 1; l >= 0; --l) {
     const act_t* x = a.res + (size_t)l * MC;
@@ -893,7 +839,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       mark(h, PK_COLSUM);
       if (fused) colsum_reduce(G + y.off[T_BFC] + (size_t)l * 4 * C, part, slabs, 4 * C, s, dj);
       else colsum_acc(G + y.off[T_BFC] + (size_t)l * 4 * C, a.dbig, M, 4 * C, part, s, dj);
-      GPT2_TRY(queue());
+      queue();
     }
     if (h->recompute) {  // g = gelu(u), as the forward's epilogue computed it
       mark(h, PK_RECOMPUTE);
@@ -933,7 +879,7 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
                   P + y.off[T_LN2G] + (size_t)l * C, G + y.off[T_LN2G] + (size_t)l * C,
                   G + y.off[T_LN2B] + (size_t)l * C, G + y.off[T_BO] + (size_t)l * C,
                   slice(ln_part, a.partials), M, C, 1, s, dj);
-    GPT2_TRY(queue());
+    queue();
     // ---- attention: xm = x + att Wo^T + bo
     {  // datt = dres Wo
       GemmArgs ga = gemm_args(M, C, C);
@@ -943,33 +889,14 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.out = a.datt; ga.ldo = C;
       GPT2_TRY(run_gemm(h, ga));
     }
-    {  // dWo += dres^T att
-      GemmArgs ga = gemm_args(C, C, M);
-      ga.A = a.dres; ga.lda = C; ga.a_mn = 1;
-      ga.B = att; ga.ldb = C; ga.b_mn = 1;
-      ga.epi = EPI_F32_ACC;
-      ga.out32 = G + y.off[T_WO] + (size_t)l * C * C; ga.ldo32 = C;
-      ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
-      ga.acc_zero = acc_zero;
-      GPT2_TRY(run_gemm(h, ga));
-    }
-    GPT2_TRY(join_side());  // the previous layer's column sums have read dqkv
     mark(h, PK_ATTN_BWD, 10.0 * B * H * (double)T * (T + 1) / 2 * (C / H));
     GPT2_CUDA(h, attention_bwd(a.dqkv, a.dsum, a.datt, qkv, att, a.lse + (size_t)l * M * H, B, T,
                                C, H, h->err, s));
     // the bias gradient of W_qkv while dqkv is still in L2
-    float* qkv_part = slice((size_t)kColsumChunks * 3 * C, a.partials);
-    if (use_side && (3 * C) % 8 == 0) {
-      GPT2_CUDA(h, cudaEventRecord(h->side_fork, s));
-      GPT2_CUDA(h, cudaStreamWaitEvent(h->side, h->side_fork, 0));
-      colsum_acc_lite(G + y.off[T_BQKV] + (size_t)l * 3 * C, a.dqkv, M, 3 * C, qkv_part, h->side, dj);
-      GPT2_CUDA(h, cudaEventRecord(h->side_join, h->side));
-      side_pending = true;
-    } else {
-      mark(h, PK_COLSUM);
-      colsum_acc(G + y.off[T_BQKV] + (size_t)l * 3 * C, a.dqkv, M, 3 * C, qkv_part, s, dj);
-    }
-    GPT2_TRY(queue());
+    mark(h, PK_COLSUM);
+    colsum_acc(G + y.off[T_BQKV] + (size_t)l * 3 * C, a.dqkv, M, 3 * C,
+               slice((size_t)kColsumChunks * 3 * C, a.partials), s, dj);
+    queue();
     {  // dh = dqkv Wqkv
       GemmArgs ga = gemm_args(M, C, 3 * C);
       ga.A = a.dqkv; ga.lda = 3 * C;
@@ -978,12 +905,18 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
       ga.out = a.dh; ga.ldo = C;
       GPT2_TRY(run_gemm(h, ga));
     }
-    {  // dWqkv += dqkv^T h1
+    {  // dWqkv += dqkv^T h1, and in the same launch dWo += dres^T att (dres
+       // still holds the gradient at x_mid): W_qkv's units alone would leave
+       // CTA pairs idle (54 for 74 at GPT-2 124M), W_o's fill them
       GemmArgs ga = gemm_args(3 * C, C, M);
       ga.A = a.dqkv; ga.lda = 3 * C; ga.a_mn = 1;
       ga.B = h1; ga.ldb = C; ga.b_mn = 1;
       ga.epi = EPI_F32_ACC;
       ga.out32 = G + y.off[T_WQKV] + (size_t)l * 3 * C * C; ga.ldo32 = C;
+      ga.M2 = C;
+      ga.A2 = a.dres; ga.lda2 = C;
+      ga.B2 = att; ga.ldb2 = C;
+      ga.out32_2 = G + y.off[T_WO] + (size_t)l * C * C; ga.ldo32_2 = C;
       ga.split_ws = a.splitk; ga.split_ws_floats = a.splitk_floats; ga.max_splits = kMaxSplits;
       ga.acc_zero = acc_zero;
       GPT2_TRY(run_gemm(h, ga));
@@ -995,10 +928,9 @@ gpt2_status gpt2_backward(gpt2_t* h, float loss_scale) {
                   G + y.off[T_LN1B] + (size_t)l * C,
                   l > 0 ? G + y.off[T_BP] + (size_t)(l - 1) * C : nullptr,
                   slice(ln_part, a.partials), M, C, 1, s, dj);
-    GPT2_TRY(queue());
+    queue();
     if (!h->bwd_events.empty()) GPT2_CUDA(h, cudaEventRecord(h->bwd_events[l], s));
   }
-  GPT2_TRY(join_side());
   if (defer) {
     mark(h, PK_COLSUM);
     reduce_jobs_run(jobs, s);
@@ -1155,7 +1087,6 @@ gpt2_status gpt2_step_graph_capture(gpt2_t* h, const int32_t* tok_dev, const int
   if (st) return st;
   st = ensure_work(h, B, T);  // no allocation may happen while capturing
   if (st) return st;
-  ensure_side(h);  // the second stream and its events exist before the capture
   if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
   if (h->graph) cudaGraphDestroy(h->graph);
   h->graph_exec = nullptr;

@@ -66,7 +66,24 @@ struct GemmArgs {
   // 16-byte aligned.  The bias gradient of the product whose output gradient
   // this is, without a second pass over it.
   float* colsum;
+  // EPI_F32_ACC with A and B MN-major: a second product with the same N and
+  // K, out32_2 += alpha * A2^T B2 over M2 rows, launched with this one where
+  // the tiles allow (M2 = 0: none).  Its accumulator holds zeros exactly
+  // when out32's does (acc_zero).
+  int M2;
+  const act_t* A2; long lda2;
+  const act_t* B2; long ldb2;
+  float* out32_2; long ldo32_2;
 };
+// The second product of a, as a product of its own.
+inline GemmArgs gemm_second(const GemmArgs& a) {
+  GemmArgs b = a;
+  b.M = a.M2; b.M2 = 0;
+  b.A = a.A2; b.lda = a.lda2;
+  b.B = a.B2; b.ldb = a.ldb2;
+  b.out32 = a.out32_2; b.ldo32 = a.ldo32_2;
+  return b;
+}
 bool gemm_colsum_supported();
 
 cudaError_t gemm(const GemmArgs& a, cudaStream_t s, int* err_flag);
@@ -136,10 +153,6 @@ constexpr int kColsumChunks = 192;
 // db[n] += sum_m dy[m, n] (fixed order); partials: [kColsumChunks * N] floats
 void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s,
                 ReduceJob* defer = nullptr);
-// As colsum_acc (N % 8 == 0, 16-byte aligned rows), with a kernel small
-// enough to run beside a GEMM on another stream; partials: [kColsumChunks * N].
-void colsum_acc_lite(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s,
-                     ReduceJob* defer = nullptr);
 // db[n] += sum over c < chunks of partials[c * N + n], c ascending (the
 // second stage of colsum_acc, for partials a GEMM epilogue wrote)
 void colsum_reduce(float* db, const float* partials, int chunks, int N, cudaStream_t s,

@@ -107,44 +107,6 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// The same partial sums with two warps a block, no shared memory and each
-// warp writing its own partial row (partials[chunk * 2 + w][n], w's rows r0 +
-// w, r0 + w + 2, ...): small enough to share an SM with a running GEMM CTA,
-// so a second stream can run it alongside the products.
-__global__ void __launch_bounds__(64)
-    colsum_partial_lite_kernel(float* __restrict__ partials, const act_t* __restrict__ dy, int M,
-                               int N, int rows_per_chunk) {
-  pdl_start();
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int n = blockIdx.x * 256 + lane * 8;
-  const int r0 = blockIdx.y * rows_per_chunk;
-  const int r1 = min(M, r0 + rows_per_chunk);
-  if (n >= N) return;
-  float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  struct alignas(16) Row8 {
-    act_t v[8];
-  };
-  for (int r = r0 + w; r < r1; r += 16) {  // eight rows in flight
-    Row8 q[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (r + 2 * k < r1) {
-        q[k] = *reinterpret_cast<const Row8*>(dy + (size_t)(r + 2 * k) * N + n);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[k].v[i] = from_f<act_t>(0.f);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) s[i] += to_f(q[k].v[i]);
-  }
-  float* dst = partials + ((size_t)blockIdx.y * 2 + w) * N + n;
-#pragma unroll
-  for (int i = 0; i < 8; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(s[i], s[i + 1], s[i + 2], s[i + 3]);
-}
-
 // db[n] += sum over chunks of partials[chunk][n] in a fixed order
 // (colsum_reduce_block).
 __global__ void __launch_bounds__(1024)
@@ -697,17 +659,6 @@ void colsum_acc(float* db, const act_t* dy, int M, int N, float* partials, cudaS
   launch_kernel(colsum_partial_kernel, g, 256, 0, s, partials, dy, M, N, rows);
   note_launch();
   colsum_reduce(db, partials, chunks, N, s, defer);
-}
-
-void colsum_acc_lite(float* db, const act_t* dy, int M, int N, float* partials, cudaStream_t s,
-                     ReduceJob* defer) {
-  const int colgroups = (N + 255) / 256;
-  const int chunks = kColsumChunks / 2;
-  const int rows = (M + chunks - 1) / chunks;
-  const int used = (M + rows - 1) / rows;
-  launch_kernel(colsum_partial_lite_kernel, dim3(colgroups, used), 64, 0, s, partials, dy, M, N, rows);
-  note_launch();
-  colsum_reduce(db, partials, 2 * used, N, s, defer);
 }
 
 void colsum_reduce(float* db, const float* partials, int chunks, int N, cudaStream_t s,
